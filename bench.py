@@ -1,0 +1,406 @@
+"""Benchmark of the sparse+linear attention layer on B200.
+
+One step = one sla_forward of the whole layer (routing, linear state and
+aggregation, sparse flash attention, epilogue) over the seeded Wan2.1-1.3B
+shaped workload (B=1, H=12, d=128, 32760 tokens padded to 32768, k_h = 5 %,
+k_l = 10 %). Inputs are resident in HBM (Q, K, V = 302 MB, larger than the
+126 MB L2, so no flush between steps). Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the float64 CPU oracle on a bounded sample
+
+With N > 1 (torchrun) every rank runs its own replica of the layer on its GPU
+(weak scaling, no collective); rank 0 prints the line with the max time over
+ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_linear_sm_b200 import workloads as wl  # noqa: E402
+
+METRIC = "ms/layer & dense-equiv TFLOP/s, sparse+linear attn N=32K d=128 95% sparse"
+UNIT = "dense-equiv TFLOP/s"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per stage (one launch each), for the roofline
+# ---------------------------------------------------------------------------
+
+def stage_model(c: wl.LayerConfig) -> dict:
+    """Per stage: ("tensor", FLOP) or ("hbm", bytes) of algorithmic work per launch."""
+    B, H, Hkv, N, Nv, d = c.B, c.H, c.H_kv, c.N, c.N_valid, c.d
+    nb = c.nqb
+    bf = 2
+    m = {}
+    m["pool"] = ("hbm", (B * H + B * Hkv) * Nv * d * bf + (B * H + B * Hkv) * nb * d * 8)
+    m["pooled_scores"] = ("hbm", (B * H + B * Hkv) * nb * d * 8 + B * H * nb * nb * 8)
+    if c.mode == wl.MODE_THREEWAY:
+        marg = nb - c.k_h - c.k_l
+        m["classify"] = ("hbm", B * H * nb * nb * 8 + B * H * nb * nb * (1 + (2 if marg else 0))
+                         + B * H * nb * c.k_h * 4)
+        dd = (d * d + d + 127) // 128 * 128
+        m["linear_state"] = ("hbm", 2 * B * Hkv * Nv * d * bf + B * Hkv * nb * dd * bf)
+        m["linear_aggregate"] = ("tensor", 2.0 * B * H * nb * nb * dd)
+        # attended FLOP over critical blocks: QK^T and PV, 2 * 2 * b^2 * d per (row, block)
+        m["sparse_flash"] = ("tensor", 4.0 * c.block * c.block * d * B * H * nb * c.k_h)
+        m["epilogue"] = ("hbm", B * H * Nv * d * bf * 3 + B * H * nb * dd * 4)
+    else:
+        m["select_topn"] = ("hbm", B * H * nb * nb * 8 / 2 + B * Hkv * nb * (c.top_n * 4 + nb))
+        # attended (query, key) pairs, upper bound: window tokens plus selected tokens
+        # (selected blocks that overlap the window are counted twice)
+        pairs = 0.0
+        for i in range(nb):
+            for r in range(c.block):
+                t = i * c.block + r
+                pairs += min(c.window, t + 1) + c.block * min(c.top_n, i)
+        m["sparse_flash"] = ("tensor", 4.0 * d * B * H * pairs)
+    return m
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, path: str | None):
+        self.idx = gpu_index
+        self.path = path
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w") if self.path else subprocess.DEVNULL
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+            if self.path:
+                self.f.write(out)
+                self.f.close()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        load = sorted(sm)[len(sm) // 4:] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg: wl.LayerConfig, x: wl.LayerInputs, units, budget_s: float | None = None):
+    """Times the float64 oracle on whole (b, h, query block) units; returns (seconds, units done)."""
+    import oracle  # test infrastructure: only this CPU leg of the benchmark uses it
+
+    class Lazy:
+        def __init__(self, bits):
+            self.bits = bits
+
+        def __getitem__(self, k):
+            return wl.bf16_bits_to_f64(self.bits[k])
+
+    t0 = time.perf_counter()
+    L = oracle.Layer(cfg, Lazy(x.q), Lazy(x.k), Lazy(x.v), x.f64("w_p"), x.f64("w_g"))
+    done = 0
+    for (b, h, i) in units:
+        L.unit(b, h, i)
+        done += 1
+        if budget_s is not None and time.perf_counter() - t0 > budget_s:
+            break
+    return time.perf_counter() - t0, done
+
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def sample_units(cfg, n, seed=1234):
+    rng = np.random.default_rng(seed)
+    heads = rng.permutation(cfg.H)[:max(1, min(cfg.H, 2))]
+    units = []
+    for h in heads:
+        for i in rng.permutation(cfg.nqb)[:max(1, n // len(heads))]:
+            units.append((0, int(h), int(i)))
+    return units
+
+
+def units_total(cfg):
+    return cfg.B * cfg.H * cfg.nqb
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = wl.generate(cfg)
+    units = sample_units(cfg, 8)
+    per_step = []
+    for s in range(args.warmup + args.steps):
+        t, n = oracle_sample(cfg, x, units)
+        if s >= args.warmup:
+            per_step.append((t, n))
+    tsum = sum(t for t, _ in per_step)
+    nsum = sum(n for _, n in per_step)
+    frac = nsum / units_total(cfg)
+    value = frac * cfg.dense_flops() / tsum / 1e12
+    full_layer_ms = tsum / frac * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tsum / len(per_step) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "N_valid": cfg.N_valid,
+                   "d": cfg.d, "k_h": cfg.k_h, "k_l": cfg.k_l, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"{len(units)} (head, query block) units of {units_total(cfg)} per step, "
+                                   "full-layer time extrapolated by unit count"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "full_layer_ms_extrapolated": full_layer_ms,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="wan1.3b", choices=list(wl.PRESETS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--clocks-csv", default=None)
+    args = ap.parse_args()
+    cfg = wl.preset(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import block_sparse_linear_sm_b200 as sla
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    x = wl.generate(cfg)
+    dev = torch.device("cuda", local)
+
+    def up(bits):
+        return None if bits is None else torch.from_numpy(bits).view(torch.bfloat16).to(dev)
+
+    q, k, v, w_p, w_g = up(x.q), up(x.k), up(x.v), up(x.w_p), up(x.w_g)
+    out = torch.empty(cfg.B, cfg.H, cfg.N, cfg.d, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(sla.sla_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    names = sla.sla_stage_names(cfg)
+    ns = len(names)
+
+    # warm-up
+    for _ in range(args.warmup):
+        sla.sla_forward(q, k, v, w_p, w_g, cfg, out, None, ws)
+    st, detail = sla.sla_check_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {detail}")
+
+    # timed region: K steps, per-stage events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clock_path = args.clocks_csv
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local, clock_path) as clk:
+        time.sleep(0.3)
+        t0.record(stream)
+        for s in range(args.steps):
+            sla.sla_forward_timed(q, k, v, w_p, w_g, cfg, out, None, ws, evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    st, detail = sla.sla_check_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {detail}")
+    if dist is not None:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    stage_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
+                for i, n in enumerate(names)}
+
+    # end to end: pinned host inputs -> device, layer, output -> host
+    hq = torch.from_numpy(x.q).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(x.k).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(x.v).view(torch.bfloat16).pin_memory()
+    hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
+    d2h = hout.numel() * 2
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        sla.sla_forward(q, k, v, w_p, w_g, cfg, out, None, ws)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    barrier()
+
+    flops = cfg.dense_flops()
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    model = stage_model(cfg)
+    stages = {}
+    for n in names:
+        kind, work = model[n]
+        t = stage_ms[n] * 1e-3
+        if kind == "tensor":
+            ach = work / t / 1e12
+            stages[n] = {"ms": stage_ms[n], "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
+                         "frac_of_sustained": ach / peaks["bf16_sus"], "work": work}
+        else:
+            ach = work / t / 1e9
+            stages[n] = {"ms": stage_ms[n], "bound": "hbm", "achieved": ach, "unit": "GB/s",
+                         "frac": ach / peaks["hbm"], "work": work}
+    dom = max(names, key=lambda n: stage_ms[n])
+    dk = stages[dom]
+    if dk["bound"] == "tensor":
+        roof = {"kernel": dom, "bound": "tensor", "achieved": dk["achieved"], "peak": peaks["bf16_sus"],
+                "unit": "TFLOP/s", "frac": dk["achieved"] / peaks["bf16_sus"],
+                "peak_kind": f"bf16 sustained, {peaks['src']}", "traffic": None}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved"], "peak": peaks["hbm"],
+                "unit": "GB/s", "frac": dk["achieved"] / peaks["hbm"],
+                "peak_kind": f"HBM copy, {peaks['src']}", "traffic": None}
+    if "sparse_flash" in stages and dom != "sparse_flash":
+        fk = stages["sparse_flash"]
+        roof["flash"] = {"achieved": fk["achieved"], "frac": fk["achieved"] / peaks["bf16_sus"]}
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "H_kv": cfg.H_kv, "N": cfg.N,
+                   "N_valid": cfg.N_valid, "d": cfg.d, "k_h": cfg.k_h, "k_l": cfg.k_l,
+                   "has_proj": cfg.has_proj, "has_gate": cfg.has_gate,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs (Q,K,V 302 MB) larger than the 126 MB L2; no flush"},
+        "ms_per_layer": ms_step,
+        "roofline": roof,
+        "stages": stages,
+        "gpu_launches": ns * args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        units = sample_units(cfg, 8)
+        t, n = oracle_sample(cfg, x, units, budget_s=30.0)
+        cv = (n / units_total(cfg)) * flops / t / 1e12
+        line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                                "sample": f"{n} (head, query block) units of {units_total(cfg)} "
+                                          f"in {t:.1f} s; throughput scaled by unit count"}
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

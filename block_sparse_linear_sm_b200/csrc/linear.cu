@@ -1,0 +1,223 @@
+// Linear branch of the layer: per-key-block states and their aggregation over
+// each query block's marginal blocks.
+//
+// SLA analysis page (arXiv 2509.24006), comparison table and core-innovation
+// paragraph: marginal blocks go through linear attention at O(N d^2). With
+// phi = elu + 1 the branch factorises per key block j into the d x d state
+// h_j = phi(K_j)^T V_j and the normaliser z_j = sum_t phi(k_t); query block i
+// then needs S_i = sum_{j marginal} h_j and Z_i = sum_{j marginal} z_j.
+//
+// Layout: Hs[bkv][j][0 : d*d] = h_j row-major, Hs[bkv][j][d*d : d*d+d] = z_j,
+// zero up to dd (a multiple of 128), rows j in [nkb, nkb_pad) zero; bf16.
+// The aggregation is the GEMM S = M . Hs with M the 0/1 marginal mask of each
+// query head (exact in bf16), accumulated in fp32: Ss[bh][i][0 : dd].
+#include "common.cuh"
+
+namespace sla {
+
+// ---------------------------------------------------------------------------
+// state kernel: one CTA per (b, kv head, key block); D/16 warps, warp w owns
+// rows 16w..16w+15 of h_j (the phi(K) feature index).
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(D * 2) state_kernel(const __nv_bfloat16* __restrict__ k,
+                                                      const __nv_bfloat16* __restrict__ v,
+                                                      __nv_bfloat16* __restrict__ hs, int N,
+                                                      int n_valid, int nkb, int dd) {
+  constexpr int RB = D * 2;  // bytes per smem row
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  __shared__ __align__(128) unsigned char fk_s[kBlock * RB];
+  __shared__ __align__(128) unsigned char v_s[kBlock * RB];
+  const int j = blockIdx.x;
+  const int bkv = blockIdx.y;
+  __nv_bfloat16* row = hs + ((size_t)bkv * gridDim.x + j) * dd;
+  if (j >= nkb) {
+    for (int e = threadIdx.x; e < dd / 8; e += blockDim.x)
+      reinterpret_cast<uint4*>(row)[e] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  int nv = n_valid - j * kBlock;
+  nv = nv > kBlock ? kBlock : nv;
+  const __nv_bfloat16* kb = k + ((size_t)bkv * N + (size_t)j * kBlock) * D;
+  const __nv_bfloat16* vb = v + ((size_t)bkv * N + (size_t)j * kBlock) * D;
+  for (int e = threadIdx.x; e < kBlock * CH; e += blockDim.x) {
+    const int t = e / CH, ch = e % CH;
+    uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (t < nv) {
+      kk = *reinterpret_cast<const uint4*>(kb + (size_t)t * D + ch * 8);
+      vv = *reinterpret_cast<const uint4*>(vb + (size_t)t * D + ch * 8);
+      uint32_t* w = reinterpret_cast<uint32_t*>(&kk);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float2 f = unpack_bf16(w[u]);
+        w[u] = pack_bf16(phi(f.x), phi(f.y));
+      }
+    }
+    *reinterpret_cast<uint4*>(fk_s + swz(t, ch, RB)) = kk;
+    *reinterpret_cast<uint4*>(v_s + swz(t, ch, RB)) = vv;
+  }
+  __syncthreads();
+  // z_j from the same bf16-rounded features the MMA uses
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float z = 0.f;
+    for (int t = 0; t < nv; ++t) {
+      const __nv_bfloat16* p =
+          reinterpret_cast<const __nv_bfloat16*>(fk_s + swz(t, c >> 3, RB)) + (c & 7);
+      z += __bfloat162float(*p);
+    }
+    row[D * D + c] = __float2bfloat16(z);
+  }
+  for (int e = D * D + D + threadIdx.x; e < dd; e += blockDim.x) row[e] = __float2bfloat16(0.f);
+
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const uint32_t fk_base = smem_u32(fk_s), v_base = smem_u32(v_s);
+  float acc[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < kBlock / 16; ++ks) {
+    uint32_t a[4];
+    ldsm_x4_t(lds_a_km(fk_base, ks * 16, 2 * w, RB, lane), a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int n2 = 0; n2 < D / 16; ++n2) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(lds_b_kn(v_base, ks * 16, 2 * n2, RB, lane), b0, b1, b2, b3);
+      mma_bf16(acc[2 * n2], a, b0, b1);
+      mma_bf16(acc[2 * n2 + 1], a, b2, b3);
+    }
+  }
+  const int r0 = 16 * w + (lane >> 2);
+  const int cc = 2 * (lane & 3);
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    *reinterpret_cast<uint32_t*>(row + (size_t)r0 * D + n * 8 + cc) = pack_bf16(acc[n][0], acc[n][1]);
+    *reinterpret_cast<uint32_t*>(row + (size_t)(r0 + 8) * D + n * 8 + cc) =
+        pack_bf16(acc[n][2], acc[n][3]);
+  }
+}
+
+cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_hs);
+  dim3 grid(p.nkb_pad, c.B * c.H_kv);
+  if (c.d == 128)
+    state_kernel<128><<<grid, 256, 0, s>>>(a.k, a.v, hs, c.N, c.N_valid, p.nkb, p.dd);
+  else
+    state_kernel<64><<<grid, 128, 0, s>>>(a.k, a.v, hs, c.N, c.N_valid, p.nkb, p.dd);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// aggregation GEMM: Ss[bh] (nqb x dd, fp32) = M[bh] (nqb_pad x nkb_pad) . Hs[bkv]
+// 128x128 tile per CTA, K steps of 64, 3-stage cp.async pipeline, 8 warps as
+// 2 (rows) x 4 (columns), warp tile 64 x 32.
+// ---------------------------------------------------------------------------
+constexpr int kAggM = 128, kAggN = 128, kAggK = 64, kAggStages = 3;
+constexpr int kAggABytes = kAggM * kAggK * 2;  // 16 KB, rows of 128 B
+constexpr int kAggBBytes = kAggK * kAggN * 2;  // 16 KB, rows of 256 B
+constexpr int kAggSmem = kAggStages * (kAggABytes + kAggBBytes);
+
+__global__ void __launch_bounds__(256) aggregate_kernel(const __nv_bfloat16* __restrict__ mmask,
+                                                        const __nv_bfloat16* __restrict__ hs,
+                                                        float* __restrict__ ss, int H, int group,
+                                                        int nqb, int nqb_pad, int nkb_pad, int dd) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int n0 = blockIdx.x * kAggN;
+  const int m0 = blockIdx.y * kAggM;
+  const int bh = blockIdx.z;
+  const int b = bh / H, h = bh % H;
+  const int bkv = b * (H / group) + h / group;
+  const __nv_bfloat16* A = mmask + (size_t)bh * nqb_pad * nkb_pad;
+  const __nv_bfloat16* Bm = hs + (size_t)bkv * nkb_pad * dd;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int wm = w >> 2, wn = w & 3;
+  const uint32_t sbase = smem_u32(smem);
+
+  auto load_stage = [&](int st, int k0) {
+    const uint32_t a_s = sbase + st * (kAggABytes + kAggBBytes);
+    const uint32_t b_s = a_s + kAggABytes;
+    // A: 128 rows x 8 chunks
+    for (int e = tid; e < kAggM * 8; e += 256) {
+      const int r = e >> 3, ch = e & 7;
+      cp_async16(a_s + swz(r, ch, 128), A + (size_t)(m0 + r) * nkb_pad + k0 + ch * 8, 16);
+    }
+    // B: 64 rows x 16 chunks
+    for (int e = tid; e < kAggK * 16; e += 256) {
+      const int r = e >> 4, ch = e & 15;
+      cp_async16(b_s + swz(r, ch, 256), Bm + (size_t)(k0 + r) * dd + n0 + ch * 8, 16);
+    }
+  };
+
+  float acc[4][4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+
+  const int nk = nkb_pad / kAggK;
+#pragma unroll
+  for (int st = 0; st < kAggStages - 1; ++st) {
+    if (st < nk) load_stage(st, st * kAggK);
+    cp_async_commit();
+  }
+  for (int kt = 0; kt < nk; ++kt) {
+    cp_async_wait<kAggStages - 2>();
+    __syncthreads();
+    const int nxt = kt + kAggStages - 1;
+    if (nxt < nk) load_stage(nxt % kAggStages, nxt * kAggK);
+    cp_async_commit();
+    const int st = kt % kAggStages;
+    const uint32_t a_s = sbase + st * (kAggABytes + kAggBBytes);
+    const uint32_t b_s = a_s + kAggABytes;
+#pragma unroll
+    for (int ks = 0; ks < kAggK / 16; ++ks) {
+      uint32_t af[4][4];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+        ldsm_x4(lds_a(a_s, wm * 64 + mt * 16, 2 * ks, 128, lane), af[mt][0], af[mt][1], af[mt][2],
+                af[mt][3]);
+#pragma unroll
+      for (int n2 = 0; n2 < 2; ++n2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(lds_b_kn(b_s, ks * 16, (wn * 32 + n2 * 16) / 8, 256, lane), b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          mma_bf16(acc[mt][2 * n2], af[mt], b0, b1);
+          mma_bf16(acc[mt][2 * n2 + 1], af[mt], b2, b3);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+  float* C = ss + (size_t)bh * nqb * dd;
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int r = m0 + wm * 64 + mt * 16 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int col = n0 + wn * 32 + nt * 8 + 2 * (lane & 3);
+      if (r < nqb)
+        *reinterpret_cast<float2*>(C + (size_t)r * dd + col) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+      if (r + 8 < nqb)
+        *reinterpret_cast<float2*>(C + (size_t)(r + 8) * dd + col) =
+            make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+    }
+  }
+}
+
+cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  const __nv_bfloat16* mm = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_mmask);
+  const __nv_bfloat16* hs = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_hs);
+  float* ss = reinterpret_cast<float*>(a.ws + p.off_ss);
+  cudaError_t e = cudaFuncSetAttribute(aggregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kAggSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.dd / kAggN, p.nqb_pad / kAggM, c.B * c.H);
+  aggregate_kernel<<<grid, 256, kAggSmem, s>>>(mm, hs, ss, c.H, p.group, p.nqb, p.nqb_pad,
+                                               p.nkb_pad, p.dd);
+  return cudaGetLastError();
+}
+
+}  // namespace sla

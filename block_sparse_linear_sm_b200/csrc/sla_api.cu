@@ -1,0 +1,274 @@
+// C ABI of the sparse+linear attention layer: validation, workspace plan and
+// the launch sequence. See include/sla.h for the contract of each entry point.
+#include <math.h>
+#include <string.h>
+
+#include "sla_internal.h"
+
+namespace sla {
+
+static sla_status check_config(const sla_config* c) {
+  if (c == nullptr) return SLA_ERR_INVALID_ARG;
+  if (c->B < 1 || c->H < 1 || c->H_kv < 1 || c->N < 1 || c->d < 1 || c->block < 1)
+    return SLA_ERR_INVALID_ARG;
+  if (c->H % c->H_kv != 0) return SLA_ERR_INVALID_ARG;
+  if (c->N % c->block != 0) return SLA_ERR_INVALID_ARG;
+  if (c->N_valid > c->N || c->N_valid <= c->N - c->block) return SLA_ERR_INVALID_ARG;
+  if (!(c->scale >= 0.f) || !isfinite(c->scale)) return SLA_ERR_INVALID_ARG;
+  if (c->block != kBlock) return SLA_ERR_UNSUPPORTED;
+  if (c->d != 64 && c->d != 128) return SLA_ERR_UNSUPPORTED;
+  const int nb = c->N / c->block;
+  if (nb > kMaxBlocks) return SLA_ERR_UNSUPPORTED;
+  if ((int64_t)c->B * c->H * c->N * c->d > ((int64_t)1 << 40)) return SLA_ERR_UNSUPPORTED;
+  if (c->mode == SLA_MODE_THREEWAY) {
+    if (c->k_h < 0 || c->k_l < 0 || c->k_h + c->k_l > nb) return SLA_ERR_INVALID_ARG;
+    if (c->causal != 0) return SLA_ERR_UNSUPPORTED;
+    if ((c->has_proj != 0 && c->has_proj != 1) || (c->has_gate != 0 && c->has_gate != 1))
+      return SLA_ERR_INVALID_ARG;
+  } else if (c->mode == SLA_MODE_TOPN_WINDOW) {
+    if (c->top_n < 0 || c->window < 0) return SLA_ERR_INVALID_ARG;
+    if (c->causal != 1) return SLA_ERR_UNSUPPORTED;
+    if (c->has_proj != 0 || c->has_gate != 0) return SLA_ERR_UNSUPPORTED;
+    // selected blocks plus window blocks must fit the kernel's 128-entry list
+    if (c->top_n > 64 || c->top_n + (c->window + 62) / kBlock + 1 > 128) return SLA_ERR_UNSUPPORTED;
+  } else {
+    return SLA_ERR_INVALID_ARG;
+  }
+  return SLA_OK;
+}
+
+bool make_plan(const sla_config* c, Plan* p) {
+  if (check_config(c) != SLA_OK) return false;
+  memset(p, 0, sizeof(*p));
+  p->c = *c;
+  p->nqb = p->nkb = c->N / kBlock;
+  p->group = c->H / c->H_kv;
+  p->nqb_pad = (int)align_up(p->nqb, 128);
+  p->nkb_pad = (int)align_up(p->nkb, 64);
+  p->dd = (int)align_up((size_t)c->d * c->d + c->d, 128);
+  p->scale = c->scale > 0.f ? c->scale : 1.f / sqrtf((float)c->d);
+  const size_t B = c->B, H = c->H, Hkv = c->H_kv, d = c->d, nqb = p->nqb, nkb = p->nkb;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  p->off_status = take(256);
+  p->off_qbar = take(B * H * nqb * d * 8);
+  p->off_kbar = take(B * Hkv * nkb * d * 8);
+  p->off_scores = take(B * H * nqb * nkb * 8);
+  if (c->mode == SLA_MODE_THREEWAY) {
+    p->off_crit = take(B * H * nqb * (size_t)c->k_h * 4);
+    p->off_neg = off;
+    const bool marginal = p->nkb - c->k_h - c->k_l > 0;
+    if (marginal) {
+      p->off_mmask = take(B * H * (size_t)p->nqb_pad * p->nkb_pad * 2);
+      p->off_hs = take(B * Hkv * (size_t)p->nkb_pad * p->dd * 2);
+      p->off_ss = take(B * H * nqb * (size_t)p->dd * 4);
+    }
+    p->off_os = take(B * H * (size_t)c->N * d * 2);
+  } else {
+    p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
+  }
+  p->total = off;
+  return true;
+}
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static bool has_marginal(const Plan& p) { return p.nkb - p.c.k_h - p.c.k_l > 0; }
+
+// Stage list of a configuration.
+enum Stage { kPool, kScores, kClassify, kSelect, kState, kAggregate, kFlash, kEpilogue };
+
+static int stages_of(const Plan& p, Stage* out) {
+  int n = 0;
+  out[n++] = kPool;
+  out[n++] = kScores;
+  if (p.c.mode == SLA_MODE_THREEWAY) {
+    out[n++] = kClassify;
+    if (has_marginal(p)) {
+      out[n++] = kState;
+      out[n++] = kAggregate;
+    }
+    out[n++] = kFlash;
+    out[n++] = kEpilogue;
+  } else {
+    out[n++] = kSelect;
+    out[n++] = kFlash;
+  }
+  return n;
+}
+
+static const char* stage_name(Stage s) {
+  switch (s) {
+    case kPool: return "pool";
+    case kScores: return "pooled_scores";
+    case kClassify: return "classify";
+    case kSelect: return "select_topn";
+    case kState: return "linear_state";
+    case kAggregate: return "linear_aggregate";
+    case kFlash: return "sparse_flash";
+    case kEpilogue: return "epilogue";
+  }
+  return "?";
+}
+
+static cudaError_t run_stage(Stage st, const Plan& p, const Args& a, cudaStream_t s) {
+  switch (st) {
+    case kPool: return launch_pool(p, a, s);
+    case kScores: return launch_scores(p, a, s);
+    case kClassify: return launch_classify(p, a, /*write_mmask=*/has_marginal(p), s);
+    case kSelect: return launch_select(p, a, s);
+    case kState: return launch_state(p, a, s);
+    case kAggregate: return launch_aggregate(p, a, s);
+    case kFlash: return launch_flash(p, a, s);
+    case kEpilogue: return launch_epilogue(p, a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+static sla_status forward_impl(const void* q, const void* k, const void* v, const void* w_p,
+                               const void* w_g, const sla_config* cfg, void* out, int8_t* mask_out,
+                               void* ws, size_t ws_bytes, void* stream, void* const* events,
+                               int32_t n_events) {
+  Plan p;
+  sla_status st = check_config(cfg);
+  if (st != SLA_OK) return st;
+  make_plan(cfg, &p);
+  if (!q || !k || !v || !out) return SLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return SLA_ERR_INVALID_ARG;
+  const bool threeway = cfg->mode == SLA_MODE_THREEWAY;
+  if (threeway && cfg->has_proj && (!w_p || !aligned(w_p, 16))) return SLA_ERR_INVALID_ARG;
+  if (threeway && cfg->has_gate && (!w_g || !aligned(w_g, 4))) return SLA_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return SLA_ERR_WORKSPACE;
+  Stage stages[8];
+  const int ns = stages_of(p, stages);
+  if (events && n_events != ns + 1) return SLA_ERR_INVALID_ARG;
+
+  Args a;
+  memset(&a, 0, sizeof(a));
+  a.q = (const __nv_bfloat16*)q;
+  a.k = (const __nv_bfloat16*)k;
+  a.v = (const __nv_bfloat16*)v;
+  a.w_p = (const __nv_bfloat16*)w_p;
+  a.w_g = (const __nv_bfloat16*)w_g;
+  a.out = (__nv_bfloat16*)out;
+  a.mask_out = mask_out;
+  a.ws = (char*)ws;
+  a.status = (int*)((char*)ws + p.off_status);
+  a.crit = (int32_t*)((char*)ws + p.off_crit);
+  a.neg = nullptr;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(a.status, 0, 8, s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (events && cudaEventRecord((cudaEvent_t)events[0], s) != cudaSuccess) return SLA_ERR_CUDA;
+  for (int i = 0; i < ns; ++i) {
+    if (run_stage(stages[i], p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (events && cudaEventRecord((cudaEvent_t)events[i + 1], s) != cudaSuccess) return SLA_ERR_CUDA;
+  }
+  return SLA_OK;
+}
+
+}  // namespace sla
+
+using namespace sla;
+
+extern "C" {
+
+sla_status sla_validate_config(const sla_config* cfg) { return check_config(cfg); }
+
+size_t sla_workspace_bytes(const sla_config* cfg) {
+  Plan p;
+  return make_plan(cfg, &p) ? p.total : 0;
+}
+
+sla_status sla_route(const void* q, const void* k, const sla_config* cfg, int8_t* mask_out,
+                     int32_t* crit_idx, int32_t* neg_idx, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  sla_status st = check_config(cfg);
+  if (st != SLA_OK) return st;
+  make_plan(cfg, &p);
+  if (!q || !k || !aligned(q, 16) || !aligned(k, 16)) return SLA_ERR_INVALID_ARG;
+  const bool threeway = cfg->mode == SLA_MODE_THREEWAY;
+  const int n_crit = threeway ? cfg->k_h : cfg->top_n;
+  if (n_crit > 0 && (!crit_idx || !aligned(crit_idx, 4))) return SLA_ERR_INVALID_ARG;
+  if (threeway && cfg->k_l > 0 && (!neg_idx || !aligned(neg_idx, 4))) return SLA_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return SLA_ERR_WORKSPACE;
+  Args a;
+  memset(&a, 0, sizeof(a));
+  a.q = (const __nv_bfloat16*)q;
+  a.k = (const __nv_bfloat16*)k;
+  a.mask_out = mask_out;
+  a.crit = n_crit > 0 ? crit_idx : nullptr;
+  a.neg = threeway && cfg->k_l > 0 ? neg_idx : nullptr;
+  a.ws = (char*)ws;
+  a.status = (int*)((char*)ws + p.off_status);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(a.status, 0, 8, s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (launch_pool(p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (launch_scores(p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
+  cudaError_t e = threeway ? launch_classify(p, a, false, s) : launch_select(p, a, s);
+  return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+}
+
+sla_status sla_forward(const void* q, const void* k, const void* v, const void* w_p,
+                       const void* w_g, const sla_config* cfg, void* out, int8_t* mask_out,
+                       void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(q, k, v, w_p, w_g, cfg, out, mask_out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+sla_status sla_forward_timed(const void* q, const void* k, const void* v, const void* w_p,
+                             const void* w_g, const sla_config* cfg, void* out, int8_t* mask_out,
+                             void* ws, size_t ws_bytes, void* stream, void* const* events,
+                             int32_t n_events) {
+  if (!events) return SLA_ERR_INVALID_ARG;
+  return forward_impl(q, k, v, w_p, w_g, cfg, out, mask_out, ws, ws_bytes, stream, events,
+                      n_events);
+}
+
+int32_t sla_num_stages(const sla_config* cfg) {
+  Plan p;
+  if (!make_plan(cfg, &p)) return -1;
+  Stage st[8];
+  return stages_of(p, st);
+}
+
+const char* sla_stage_name(const sla_config* cfg, int32_t s) {
+  Plan p;
+  if (!make_plan(cfg, &p)) return nullptr;
+  Stage st[8];
+  const int n = stages_of(p, st);
+  return (s >= 0 && s < n) ? stage_name(st[s]) : nullptr;
+}
+
+sla_status sla_check_device_status(void* ws, void* stream, int32_t* detail) {
+  if (!ws || !aligned(ws, 256)) return SLA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SLA_ERR_CUDA;
+  int st[2] = {0, 0};
+  if (cudaMemcpy(st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return SLA_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(st)) != cudaSuccess) return SLA_ERR_CUDA;
+  if (detail) *detail = st[1];
+  if (st[0] == 0) return SLA_OK;
+  if (st[0] == SLA_ERR_DEVICE_TIMEOUT || st[0] == SLA_ERR_DEVICE_CHECK) return (sla_status)st[0];
+  return SLA_ERR_DEVICE_CHECK;
+}
+
+const char* sla_status_string(sla_status s) {
+  switch (s) {
+    case SLA_OK: return "ok";
+    case SLA_ERR_INVALID_ARG: return "invalid argument";
+    case SLA_ERR_UNSUPPORTED: return "configuration not supported by the kernels";
+    case SLA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SLA_ERR_CUDA: return "CUDA runtime or launch error";
+    case SLA_ERR_DEVICE_TIMEOUT: return "device-side bounded wait ran out";
+    case SLA_ERR_DEVICE_CHECK: return "device-side range check failed";
+  }
+  return "unknown status";
+}
+
+const char* sla_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// Internal host-side interface between the C ABI (sla_api.cu) and the kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sla.h"
+
+namespace sla {
+
+constexpr int kBlock = 64;
+constexpr int kMaxBlocks = 4096;  // nkb limit of the routing sort (N <= 262144)
+
+// Device status word: status[0] = sla_status code, status[1] = detail.
+enum DeviceDetail : int {
+  kDetailFlashIndex = 101,      // flash kernel read a block index outside [0, nkb)
+  kDetailEpilogueIndex = 102,
+  kDetailTimeout = 200,
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Derived sizes and the workspace carve-up for one configuration.
+struct Plan {
+  sla_config c;
+  int nqb, nkb, group;
+  int nqb_pad, nkb_pad;  // aggregation GEMM padding (128 rows, 64 columns)
+  int dd;                // row length of the per-block linear state: d*d + d, padded to 128
+  float scale;
+  // byte offsets into ws
+  size_t off_status, off_qbar, off_kbar, off_scores, off_crit, off_neg, off_mmask, off_hs, off_ss,
+      off_os, total;
+};
+
+bool make_plan(const sla_config* c, Plan* p);
+
+// Raw pointers of one launch.
+struct Args {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* w_p;
+  const __nv_bfloat16* w_g;
+  __nv_bfloat16* out;
+  int8_t* mask_out;
+  int32_t* crit;      // THREEWAY critical lists / TOPN selected lists
+  int32_t* neg;       // THREEWAY negligible lists (may be null)
+  char* ws;
+  int* status;
+};
+
+// kernel launchers (return the launch error)
+cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_scores(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cudaStream_t s);
+cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_epilogue(const Plan& p, const Args& a, cudaStream_t s);
+
+}  // namespace sla

@@ -1,0 +1,183 @@
+/*
+ * sla.h - C ABI of the block-routed sparse+linear attention layer (SLA / SALAD
+ * style) for NVIDIA B200 (sm_100a).
+ *
+ * One layer computes, per (batch b, query head h, query block i of 64 tokens):
+ *
+ *   1. block pooling      qbar_i = mean of the valid Q tokens of block i,
+ *                         kbar_j = mean of the valid K tokens of block j
+ *                         (SLA analysis, arXiv 2509.24006: compressed attention
+ *                          prediction by mean pooling; 2025 sparse-attention
+ *                          review, section 11 SpargeAttn, prediction algorithm)
+ *   2. pooled scores      s_ij = qbar_i . kbar_j * scale, P_hat = softmax_j(s_i.)
+ *                         (same SpargeAttn passage)
+ *   3. routing            SLA_MODE_THREEWAY: the k_h highest-scoring blocks of
+ *                         row i are critical, the k_l lowest negligible, the
+ *                         rest marginal (SLA analysis: critical / marginal /
+ *                         negligible split, TopK / BottomK; 2025 review,
+ *                         section 10 SLA).  Equal scores: lower block index
+ *                         ranks higher.
+ *                         SLA_MODE_TOPN_WINDOW: the query heads of one KV group
+ *                         sum their per-head softmax over past blocks j < i and
+ *                         keep the top_n, plus a causal window of `window`
+ *                         tokens (2025 review, section 4 MoBA; sparse attention
+ *                         survey, section 2 NSA: block 64, n = 16, w = 512).
+ *   4. sparse attention   O_s = exact softmax attention over the valid tokens of
+ *                         the critical blocks (top-n mode: selected blocks
+ *                         union window, causal); 0 when the set is empty
+ *                         (2025 review, section 2.3 NSA operator design).
+ *   5. linear attention   h_j = phi(K_j)^T V_j, z_j = sum_t phi(k_t) over valid
+ *                         tokens, phi = elu + 1; S_i = sum over marginal j of
+ *                         h_j, Z_i likewise; O_l = phi(q) S_i / (phi(q) . Z_i),
+ *                         0 when row i has no marginal block
+ *                         (SLA analysis: linear attention at O(N d^2) for the
+ *                          marginal part).
+ *   6. combine            O = O_s + g * (O_l W_p), g_t = sigmoid(q_t . w_g[h])
+ *                         (SLA analysis, Proj paragraph: O = O^s + Proj(O^l);
+ *                          SALAD summary: input-dependent gate).
+ *                         Without projection W_p = I; without gate g = 1.
+ *                         The top-n mode has no linear branch: O = O_s.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are dense, row-major, in device memory (the caller allocates and
+ *   frees all of them; the library never allocates):
+ *     q    bf16 [B, H,    N, d]
+ *     k, v bf16 [B, H_kv, N, d]
+ *     w_p  bf16 [d, d]   (row vector times matrix: O_l W_p), ignored unless has_proj
+ *     w_g  bf16 [H, d]   ignored unless has_gate
+ *     out  bf16 [B, H, N, d]
+ *   Tokens at index >= N_valid are padding: they are left out of pooling,
+ *   attention and the linear states, and their output rows are written as 0.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *   enqueues work on it and returns; nothing synchronises except
+ *   sla_check_device_status.
+ * - `ws` is caller-owned device scratch of at least sla_workspace_bytes(cfg)
+ *   bytes, 256-byte aligned. Its contents need no initialisation and are
+ *   clobbered. Calls that share one `ws` must not overlap on the GPU.
+ * - Errors: invalid arguments (bad config, NULL or misaligned pointers, short
+ *   workspace) return SLA_ERR_INVALID_ARG / SLA_ERR_UNSUPPORTED /
+ *   SLA_ERR_WORKSPACE before anything is launched. A failed launch returns
+ *   SLA_ERR_CUDA. Faults detected on the device (an index out of range, a
+ *   bounded wait that ran out) are recorded in a status word inside `ws` and
+ *   reported by sla_check_device_status; kernels never trap.
+ */
+#ifndef SLA_H
+#define SLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SLA_API __attribute__((visibility("default")))
+#else
+#define SLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLA_OK = 0,
+  SLA_ERR_INVALID_ARG = 1,    /* NULL pointer, inconsistent sizes, misalignment */
+  SLA_ERR_UNSUPPORTED = 2,    /* valid but outside what the kernels implement */
+  SLA_ERR_WORKSPACE = 3,      /* ws NULL or ws_bytes < sla_workspace_bytes(cfg) */
+  SLA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  SLA_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait ran out */
+  SLA_ERR_DEVICE_CHECK = 6    /* a device-side range check failed */
+} sla_status;
+
+typedef enum {
+  SLA_MODE_THREEWAY = 0,      /* critical / marginal / negligible (SLA, SALAD) */
+  SLA_MODE_TOPN_WINDOW = 1    /* top_n past blocks per KV group + causal window (NSA / MoBA) */
+} sla_mode;
+
+typedef struct {
+  int32_t B;        /* batch */
+  int32_t H;        /* query heads */
+  int32_t H_kv;     /* key/value heads; H % H_kv == 0, head h reads KV head h / (H / H_kv) */
+  int32_t N;        /* padded sequence length, a multiple of block */
+  int32_t N_valid;  /* valid tokens, N - block < N_valid <= N */
+  int32_t d;        /* head dimension: 64 or 128 */
+  int32_t block;    /* tokens per block: must be 64 */
+  int32_t mode;     /* sla_mode */
+  int32_t k_h;      /* THREEWAY: critical blocks per row, 0 <= k_h */
+  int32_t k_l;      /* THREEWAY: negligible blocks per row, k_h + k_l <= N / block */
+  int32_t top_n;    /* TOPN_WINDOW: selected past blocks per query block, >= 0 */
+  int32_t window;   /* TOPN_WINDOW: window tokens t-window+1 .. t, >= 0 */
+  int32_t causal;   /* must be 1 in TOPN_WINDOW and 0 in THREEWAY */
+  int32_t has_proj; /* THREEWAY: 1 = apply w_p to O_l, 0 = identity */
+  int32_t has_gate; /* THREEWAY: 1 = g = sigmoid(q . w_g[h]), 0 = g = 1 */
+  float scale;      /* softmax scale of pooled scores and attention; 0 = 1/sqrt(d) */
+} sla_config;
+
+/* Checks a configuration without touching any pointer. */
+SLA_API sla_status sla_validate_config(const sla_config* cfg);
+
+/* Bytes of device workspace that sla_route / sla_forward need for cfg
+ * (0 if cfg is invalid). */
+SLA_API size_t sla_workspace_bytes(const sla_config* cfg);
+
+/*
+ * Routing only (steps 1-3).
+ *   THREEWAY:    mask_out int8  [B, H, nqb, nkb]: 2 critical, 1 marginal, 0 negligible
+ *                crit_idx int32 [B, H, nqb, k_h]: critical blocks, ascending
+ *                neg_idx  int32 [B, H, nqb, k_l]: negligible blocks, ascending
+ *   TOPN_WINDOW: mask_out int8  [B, H_kv, nqb, nkb]: 2 selected, 0 otherwise
+ *                crit_idx int32 [B, H_kv, nqb, top_n]: selected blocks ascending,
+ *                         padded with -1 when fewer than top_n exist (i < top_n)
+ *                neg_idx  unused (may be NULL)
+ * mask_out may be NULL; crit_idx may be NULL only when k_h (top_n) is 0 and
+ * neg_idx only when k_l is 0. nqb = nkb = N / block.
+ */
+SLA_API sla_status sla_route(const void* q, const void* k, const sla_config* cfg,
+                     int8_t* mask_out, int32_t* crit_idx, int32_t* neg_idx,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The whole layer (steps 1-6): writes out [B, H, N, d] bf16.
+ * w_p may be NULL unless has_proj, w_g may be NULL unless has_gate.
+ * mask_out (nullable) receives the routing mask exactly as sla_route writes it.
+ */
+SLA_API sla_status sla_forward(const void* q, const void* k, const void* v,
+                       const void* w_p, const void* w_g, const sla_config* cfg,
+                       void* out, int8_t* mask_out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * sla_forward that also records caller-created CUDA events (cudaEvent_t,
+ * passed as void*) on `stream` around its launches: events[0] before the first
+ * launch and events[s + 1] after stage s, for s < sla_num_stages(cfg).
+ * n_events must be sla_num_stages(cfg) + 1. Used to time each kernel.
+ */
+SLA_API sla_status sla_forward_timed(const void* q, const void* k, const void* v,
+                             const void* w_p, const void* w_g, const sla_config* cfg,
+                             void* out, int8_t* mask_out,
+                             void* ws, size_t ws_bytes, void* stream,
+                             void* const* events, int32_t n_events);
+
+/* Number of stages (one kernel launch each) sla_forward enqueues for cfg, or -1. */
+SLA_API int32_t sla_num_stages(const sla_config* cfg);
+
+/* Name of stage s of cfg's pipeline (static string), or NULL. */
+SLA_API const char* sla_stage_name(const sla_config* cfg, int32_t s);
+
+/*
+ * Synchronises `stream`, reads the device status word in ws and clears it.
+ * Returns SLA_OK, SLA_ERR_DEVICE_TIMEOUT, SLA_ERR_DEVICE_CHECK or SLA_ERR_CUDA;
+ * *detail (nullable) receives a code naming the kernel and check that failed.
+ */
+SLA_API sla_status sla_check_device_status(void* ws, void* stream, int32_t* detail);
+
+/* Static description of a status code. */
+SLA_API const char* sla_status_string(sla_status s);
+
+/* Library version, e.g. "0.1.0". */
+SLA_API const char* sla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H */

@@ -1,0 +1,132 @@
+"""Host-only checks of the C-ABI library: it loads without a GPU, exports every
+function include/sla.h declares, and rejects bad arguments before launching
+anything (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_linear_sm_b200 as sla
+from block_sparse_linear_sm_b200 import workloads as wl
+
+
+def declared_functions():
+    src = open(sla.HEADER_PATH).read()
+    return sorted(set(re.findall(r"^SLA_API\s+[\w\s\*]+?\b(sla_\w+)\s*\(", src, re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("sla_route", "sla_forward", "sla_workspace_bytes", "sla_status_string",
+                 "sla_check_device_status"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = sla.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_config_struct_layout_matches_header():
+    src = open(sla.HEADER_PATH).read()
+    body = src[src.index("typedef struct {"):src.index("} sla_config;")]
+    fields = re.findall(r"^\s*(?:int32_t|float)\s+(\w+);", body, re.M)
+    assert fields == [f for f, _ in sla.sla_config._fields_]
+    assert ctypes.sizeof(sla.sla_config) == 4 * len(fields)
+
+
+@pytest.mark.parametrize("name", wl.PRESETS)
+def test_presets_are_valid(name):
+    c = wl.preset(name)
+    assert sla.sla_validate_config(c) == sla.SLA_OK
+    assert sla.sla_workspace_bytes(c) > 0
+    assert sla.sla_num_stages(c) == len(sla.sla_stage_names(c)) > 0
+
+
+BAD = [
+    (dict(block=32), sla.SLA_ERR_UNSUPPORTED),
+    (dict(d=96), sla.SLA_ERR_UNSUPPORTED),
+    (dict(N=1000, N_valid=1000), sla.SLA_ERR_INVALID_ARG),
+    (dict(N_valid=1025), sla.SLA_ERR_INVALID_ARG),
+    (dict(N_valid=960), sla.SLA_ERR_INVALID_ARG),
+    (dict(H=3, H_kv=2), sla.SLA_ERR_INVALID_ARG),
+    (dict(k_h=10, k_l=7), sla.SLA_ERR_INVALID_ARG),
+    (dict(k_h=-1), sla.SLA_ERR_INVALID_ARG),
+    (dict(causal=1), sla.SLA_ERR_UNSUPPORTED),
+    (dict(mode=1, causal=0), sla.SLA_ERR_UNSUPPORTED),
+    (dict(mode=1, causal=1, top_n=65, has_proj=0), sla.SLA_ERR_UNSUPPORTED),
+    (dict(mode=1, causal=1, top_n=4, has_proj=1), sla.SLA_ERR_UNSUPPORTED),
+    (dict(mode=7), sla.SLA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), sla.SLA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), sla.SLA_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("kw,code", BAD)
+def test_invalid_configs_are_rejected(kw, code):
+    base = dict(N=1024, N_valid=1024)
+    base.update(kw)
+    c = wl.small_config(**base)
+    assert sla.sla_validate_config(c) == code
+    assert sla.sla_workspace_bytes(c) == 0
+    assert sla.sla_num_stages(c) == -1
+
+
+def _call_forward(cfg, q=16, k=16, v=16, w_p=16, w_g=16, out=16, ws=256, ws_bytes=None):
+    c = sla.make_config(cfg)
+    if ws_bytes is None:
+        ws_bytes = sla.sla_workspace_bytes(cfg)
+    return sla.lib().sla_forward(q, k, v, w_p, w_g, ctypes.byref(c), out, None, ws, ws_bytes, None)
+
+
+def test_forward_rejects_bad_pointers_before_launch():
+    cfg = wl.small_config(N=1024, N_valid=1024, has_gate=1)
+    # fake (never dereferenced) addresses: every case fails validation on the host
+    assert _call_forward(cfg, q=None) == sla.SLA_ERR_INVALID_ARG
+    assert _call_forward(cfg, out=None) == sla.SLA_ERR_INVALID_ARG
+    assert _call_forward(cfg, q=24) == sla.SLA_ERR_INVALID_ARG          # misaligned
+    assert _call_forward(cfg, w_p=None) == sla.SLA_ERR_INVALID_ARG      # has_proj
+    assert _call_forward(cfg, w_g=None) == sla.SLA_ERR_INVALID_ARG      # has_gate
+    assert _call_forward(cfg, ws=None) == sla.SLA_ERR_WORKSPACE
+    assert _call_forward(cfg, ws=128) == sla.SLA_ERR_WORKSPACE          # misaligned
+    assert _call_forward(cfg, ws_bytes=sla.sla_workspace_bytes(cfg) - 1) == sla.SLA_ERR_WORKSPACE
+    bad = wl.small_config(N=1024, N_valid=1024, d=80)
+    assert _call_forward(bad) == sla.SLA_ERR_UNSUPPORTED
+
+
+def test_route_rejects_missing_lists():
+    cfg = wl.small_config(N=1024, N_valid=1024, k_h=3, k_l=2)
+    c = sla.make_config(cfg)
+    nb = sla.sla_workspace_bytes(cfg)
+    L = sla.lib()
+    assert L.sla_route(16, 16, ctypes.byref(c), None, None, 16, 256, nb, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_route(16, 16, ctypes.byref(c), None, 16, None, 256, nb, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_route(16, 16, ctypes.byref(c), None, 16, 16, 256, 0, None) == sla.SLA_ERR_WORKSPACE
+
+
+def test_timed_forward_checks_event_count():
+    cfg = wl.small_config(N=1024, N_valid=1024)
+    c = sla.make_config(cfg)
+    L = sla.lib()
+    evs = (ctypes.c_void_p * 2)(1, 2)
+    r = L.sla_forward_timed(16, 16, 16, 16, None, ctypes.byref(c), 16, None, 256,
+                            sla.sla_workspace_bytes(cfg), None, evs, 2)
+    assert r == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_forward_timed(16, 16, 16, 16, None, ctypes.byref(c), 16, None, 256,
+                               sla.sla_workspace_bytes(cfg), None, None, 0) == sla.SLA_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for s in range(7):
+        assert sla.status_string(s)
+    assert "unknown" in sla.status_string(99)
+    assert sla.sla_version().count(".") == 2
+
+
+def test_workspace_grows_with_the_problem():
+    a = wl.small_config(N=1024, N_valid=1024)
+    b = wl.small_config(N=2048, N_valid=2048)
+    assert sla.sla_workspace_bytes(b) > sla.sla_workspace_bytes(a)
+    assert sla.sla_workspace_bytes(a) % 256 == 0

@@ -1,0 +1,149 @@
+"""GPU parity: the C-ABI layer against the float64 oracle on seeded inputs.
+
+Small layers are compared element by element over every output; the five
+workload shapes are compared on the full routing (bit-exact except near-tie
+rows, which are counted) and on sampled query blocks of the output.
+Tolerances: max-abs 2e-2 and mean-abs 2e-3 on bf16 outputs; the linear branch
+alone within 1e-2 relative Frobenius error.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from block_sparse_linear_sm_b200 import workloads as wl  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these anyway
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from gpu_util import (MAX_ABS, MEAN_ABS, GpuRun, check_routing, full_errors,  # noqa: E402
+                      unit_errors)
+
+
+def small(**kw):
+    return wl.small_config(**kw)
+
+
+def run_and_check_full(cfg, v_shift=0.0):
+    x = wl.generate(cfg, v_shift=v_shift)
+    run = GpuRun(cfg, x)
+    L = run.layer()
+    rep = check_routing(run, L)
+    assert rep["mismatched_rows"] == 0, rep
+    ref = L.forward()
+    err = full_errors(run, ref)
+    print(cfg.name, rep, err)
+    assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err
+    return run, L, ref
+
+
+SMALL_CASES = [
+    dict(name="tiny_like", N=1024, N_valid=1024, d=64, k_h=4, k_l=4),
+    dict(name="ragged_d128", N=2048, N_valid=2001, d=128, H=4, H_kv=4, k_h=5, k_l=7, has_gate=1),
+    dict(name="gqa_d128", N=1536, N_valid=1473, d=128, H=4, H_kv=2, k_h=3, k_l=2, has_gate=1),
+    dict(name="one_valid_token_tail", N=1024, N_valid=961, d=64, k_h=2, k_l=3),
+    dict(name="no_proj", N=1024, N_valid=1000, d=128, k_h=2, k_l=2, has_proj=0),
+    dict(name="batch2", B=2, N=640, N_valid=600, d=64, H=2, H_kv=1, k_h=2, k_l=1, has_gate=1),
+]
+
+
+@pytest.mark.parametrize("kw", SMALL_CASES, ids=[c["name"] for c in SMALL_CASES])
+def test_small_layer_matches_oracle(kw):
+    run_and_check_full(small(**kw))
+
+
+def test_tiny_workload():
+    run_and_check_full(wl.preset("tiny"))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_all_critical_is_dense(d):
+    nb = 12
+    run_and_check_full(small(name="all_crit", N=nb * 64, N_valid=nb * 64 - 5, d=d, k_h=nb, k_l=0))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_all_negligible_is_zero(d):
+    nb = 8
+    cfg = small(name="all_neg", N=nb * 64, N_valid=nb * 64, d=d, k_h=0, k_l=nb, has_gate=1)
+    run = GpuRun(cfg)
+    assert np.all(run.O() == 0)
+
+
+def test_no_critical_blocks():
+    run_and_check_full(small(name="no_crit", N=1024, N_valid=1000, d=128, k_h=0, k_l=3, has_gate=1))
+
+
+def test_no_marginal_blocks():
+    run_and_check_full(small(name="no_marg", N=1024, N_valid=1024, d=128, k_h=6, k_l=10))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_linear_branch_alone_shifted_values(d):
+    """All blocks marginal, W_p = I, no gate, V + 3: O is the linear branch and O(1)."""
+    cfg = small(name="all_marg", N=2048, N_valid=2040, d=d, k_h=0, k_l=0, has_proj=0)
+    x = wl.generate(cfg, v_shift=3.0)
+    run = GpuRun(cfg, x)
+    ref = run.layer().forward()
+    got = run.O()[:, :, :cfg.N_valid]
+    want = ref["O_l"][:, :, :cfg.N_valid]
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    print("linear branch relative Frobenius error", rel)
+    assert rel <= 1e-2
+
+
+def test_mixed_layer_shifted_values_linear_branch():
+    """Mixed classes with V + 3 so that the linear branch is O(1); W_p = I, no gate."""
+    cfg = small(name="mixed_shift", N=2048, N_valid=2030, d=128, k_h=4, k_l=6, has_proj=0)
+    x = wl.generate(cfg, v_shift=3.0)
+    run = GpuRun(cfg, x)
+    ref = run.layer().forward()
+    got = run.O()[:, :, :cfg.N_valid]
+    want_l = ref["O_l"][:, :, :cfg.N_valid]
+    got_l = got - ref["O_s"][:, :, :cfg.N_valid]
+    rel = np.linalg.norm(got_l - want_l) / np.linalg.norm(want_l)
+    print("mixed: linear branch relative Frobenius error", rel)
+    assert rel <= 1e-2
+
+
+TOPN_CASES = [
+    dict(name="topn_small", H=8, H_kv=2, N=2048, N_valid=2048, d=128, top_n=4, window=200),
+    dict(name="topn_d64_ragged", H=4, H_kv=1, N=1536, N_valid=1500, d=64, top_n=3, window=64),
+    dict(name="topn_no_window", H=4, H_kv=4, N=1024, N_valid=1024, d=128, top_n=5, window=0),
+    dict(name="topn_window_only", H=2, H_kv=1, N=1024, N_valid=1024, d=128, top_n=0, window=512),
+    dict(name="topn_nsa_params", H=16, H_kv=1, N=2048, N_valid=2048, d=128, top_n=16, window=512),
+]
+
+
+@pytest.mark.parametrize("kw", TOPN_CASES, ids=[c["name"] for c in TOPN_CASES])
+def test_topn_window_matches_oracle(kw):
+    base = dict(mode=wl.MODE_TOPN_WINDOW, causal=1, has_proj=0, has_gate=0, generator="block_shift")
+    base.update(kw)
+    run_and_check_full(small(**base))
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads in the launch configuration the benchmark times
+# ---------------------------------------------------------------------------
+
+def sampled_units(cfg, n=12, seed=0):
+    rng = np.random.default_rng(seed)
+    units = {(0, 0, 0), (0, cfg.H - 1, cfg.nqb - 1)}
+    while len(units) < n:
+        units.add((0, int(rng.integers(cfg.H)), int(rng.integers(cfg.nqb))))
+    return sorted(units)
+
+
+@pytest.mark.parametrize("name", ["wan1.3b", "salad", "nsa_causal", "wan14b"])
+def test_full_size_workload(name):
+    cfg = wl.preset(name)
+    run = GpuRun(cfg)
+    L = run.layer()
+    rep = check_routing(run, L)
+    print(name, "routing", rep)
+    assert rep["mismatched_rows"] == 0, rep
+    err = unit_errors(run, L, sampled_units(cfg))
+    print(name, "sampled output error", err)
+    assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err
