@@ -162,6 +162,9 @@ def sla_forward(q, k, v, w_p, w_g, c, out, mask_out, ws, stream=None) -> None:
 def sla_forward_timed(q, k, v, w_p, w_g, c, out, mask_out, ws, events, stream=None) -> None:
     """events: torch.cuda.Event(enable_timing=True) list of length sla_num_stages(c) + 1."""
     cfg = _cfg(c)
+    for e in events:
+        if e.cuda_event == 0:  # torch creates the CUDA event on first record
+            e.record()
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     ws_bytes = ws.numel() * ws.element_size()
     _check(lib().sla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(w_p), _ptr(w_g),

@@ -1,0 +1,521 @@
+// Sparse exact attention over indexed key blocks on the 5th-generation tensor
+// cores (tcgen05, accumulators in TMEM, operands staged by TMA).
+//
+// 2025 sparse-attention review, section 2.3 (NSA operator design): load
+// fixed-size indexed KV blocks, outer loop over queries, inner loop over the
+// indexed KV blocks, filling the tensor cores. Three-way mode (SLA analysis
+// page, arXiv 2509.24006): the blocks of a query block are its critical
+// blocks. Top-n mode (2025 review section 4, MoBA; sparse attention survey
+// section 2, NSA): the KV group's selected past blocks plus the blocks the
+// causal window reaches; element (t, s) is kept when s <= t and (block(s) is
+// selected or s > t - window).
+//
+// Work unit = 128 query rows = two halves of 64 rows:
+//   - three-way mode, and top-n mode with an odd group size: query blocks
+//     2p and 2p+1 of one head; their block lists are merged and a tile that
+//     only one half needs is masked for the other half;
+//   - top-n mode with an even group size: two query heads of one KV group at
+//     the same query block (identical lists, no masking waste).
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues tcgen05.mma, warps 2-5 (one TMEM lane quarter each) run the online
+// softmax, one thread per query row.
+//
+// Per tile n (64 keys): S_n = Q K_n^T (M=128, N=64, TMEM, double-buffered);
+// the softmax warps load S_n, mask and exponentiate it, write P_n (bf16) to
+// shared memory; O += P_n V_n (M=128, N=D) accumulates in TMEM. S_{n+1} is
+// issued before PV_n so the tensor core works while the softmax runs. The
+// running max is only moved (and O rescaled) when a row's max grows by more
+// than 2^8, so P stays below 256 and O needs no per-tile rescale.
+//
+// Shared memory: Q (128 x D bf16), a ring of three 64-row K/V slots, P
+// (128 x 64 bf16), the merged block list. All operand tiles use the 128-byte
+// swizzle. Two CTAs fit on one SM (TMEM: 256 columns each).
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace sla {
+
+struct FlashTcParams {
+  const int32_t* list;  // THREEWAY: [B*H][nb][len] critical; TOPN: [B*H_kv][nb][len] selected (-1 pad)
+  __nv_bfloat16* o;     // [B*H][N][D]
+  int* status;
+  int H, group, N, n_valid, nb, len, window;
+  int pair_heads;       // 1: halves are heads (2hp, 2hp+1) of a group; 0: query blocks (2p, 2p+1)
+  int npairs;           // units per (b, h) when pairing query blocks
+  int words;            // 32-bit words of one block bitmap
+  int list_cap;         // capacity of the merged list
+  float scale_log2;
+};
+
+constexpr int kTcThreads = 192;
+constexpr int kSlots = 3;
+constexpr float kRescaleLog2 = 8.f;
+
+template <int D>
+struct TcLayout {
+  static constexpr int kQBytes = 128 * D * 2;           // 2 halves x D/64 panels x 8 KB
+  static constexpr int kSlotBytes = 64 * D * 2;         // one K or V tile
+  static constexpr int kPBytes = 128 * 64 * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kOffQ + kQBytes;
+  static constexpr int kOffP = kOffKV + kSlots * kSlotBytes;
+  static constexpr int kOffBar = kOffP + kPBytes;        // 16 mbarriers
+  static constexpr int kOffMisc = kOffBar + 16 * 8;      // tmem addr, count, abort
+  static constexpr int kOffBits = kOffMisc + 64;         // 4 bitmaps
+  static constexpr int kTmemCols = 256;                  // O: D columns, S: 2 x 64 columns
+};
+
+template <int D, bool TOPN>
+__global__ void __launch_bounds__(kTcThreads, 2)
+    flash_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, FlashTcParams prm) {
+  using L = TcLayout<D>;
+  constexpr int NP = D / 64;  // 64-column panels
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (sbase & 1023u) {  // swizzled operand tiles need 1024-byte alignment
+    if (tid == 0) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashAlign);
+    return;
+  }
+
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + L::kOffBits);  // act0, act1, sel0, sel1
+  uint32_t* mlist = words + 4 * prm.words;                            // merged list
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
+  // misc[0] = TMEM base, misc[1] = merged count, misc[2] = abort
+  auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
+  // barrier ids
+  constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 4, S_FULL = 7, S_FREE = 9, P_FULL = 11,
+                O_DONE = 12;
+
+  // ---- unit decode ----------------------------------------------------------
+  const int Hkv = prm.H / prm.group;
+  int bh_h[2], i_h[2], bkv;
+  bool valid_h[2];
+  const int32_t* lst[2];
+  {
+    const int u = blockIdx.x;
+    if (!prm.pair_heads) {
+      const int bh = u / prm.npairs, p = u % prm.npairs;
+      const int b = bh / prm.H, h = bh % prm.H;
+      bkv = b * Hkv + h / prm.group;
+      for (int hf = 0; hf < 2; ++hf) {
+        bh_h[hf] = bh;
+        i_h[hf] = 2 * p + hf;
+      }
+    } else {
+      const int hp_n = prm.group / 2;
+      const int hp = u % hp_n;
+      const int rest = u / hp_n;
+      const int i = rest % prm.nb;
+      bkv = rest / prm.nb;
+      const int b = bkv / Hkv, g = bkv % Hkv;
+      for (int hf = 0; hf < 2; ++hf) {
+        bh_h[hf] = b * prm.H + g * prm.group + 2 * hp + hf;
+        i_h[hf] = i;
+      }
+    }
+    for (int hf = 0; hf < 2; ++hf) {
+      valid_h[hf] = i_h[hf] < prm.nb;
+      lst[hf] = nullptr;
+      if (valid_h[hf] && prm.len > 0)
+        lst[hf] = TOPN ? prm.list + ((size_t)bkv * prm.nb + i_h[hf]) * prm.len
+                       : prm.list + ((size_t)bh_h[hf] * prm.nb + i_h[hf]) * prm.len;
+    }
+  }
+
+  // ---- prologue: barriers, TMEM, merged block list --------------------------
+  for (int w = tid; w < 4 * prm.words; w += kTcThreads) words[w] = 0u;
+  if (tid == 0) {
+    misc[2] = 0;
+    tc::mbar_init(bar(Q_FULL), 1);
+    for (int s = 0; s < kSlots; ++s) {
+      tc::mbar_init(bar(KV_FULL + s), 1);
+      tc::mbar_init(bar(KV_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(bar(S_FULL + b), 1);
+      tc::mbar_init(bar(S_FREE + b), 4);
+    }
+    tc::mbar_init(bar(P_FULL), 4);
+    tc::mbar_init(bar(O_DONE), 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(sbase + L::kOffMisc, L::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  __syncthreads();
+  // bitmaps of the two halves
+  for (int hf = 0; hf < 2; ++hf) {
+    if (!valid_h[hf]) continue;
+    uint32_t* act = words + hf * prm.words;
+    uint32_t* sel = words + (2 + hf) * prm.words;
+    for (int e = tid; e < prm.len; e += kTcThreads) {
+      const int j = lst[hf][e];
+      if (TOPN && j < 0) continue;  // padding of short selections
+      if (j < 0 || j >= prm.nb || (TOPN && j >= i_h[hf])) {
+        report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
+        continue;
+      }
+      atomicOr(&act[j >> 5], 1u << (j & 31));
+      if (TOPN) atomicOr(&sel[j >> 5], 1u << (j & 31));
+    }
+    if (TOPN && prm.window > 0) {
+      const int lo = i_h[hf] * kBlock - prm.window + 1;
+      const int first = lo <= 0 ? 0 : lo / kBlock;
+      for (int j = first + tid; j <= i_h[hf]; j += kTcThreads) atomicOr(&act[j >> 5], 1u << (j & 31));
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+    for (int w0 = 0; w0 < prm.words; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t a0 = w < prm.words ? words[w] : 0u, a1 = w < prm.words ? words[prm.words + w] : 0u;
+      const uint32_t s0 = w < prm.words ? words[2 * prm.words + w] : 0u;
+      const uint32_t s1 = w < prm.words ? words[3 * prm.words + w] : 0u;
+      uint32_t any = a0 | a1;
+      const int cnt = __popc(any);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = base + incl - cnt;
+      while (any) {
+        const int bit = __ffs(any) - 1;
+        any &= any - 1;
+        const uint32_t m = 1u << bit;
+        if (pos < prm.list_cap)
+          mlist[pos] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u) |
+                       ((s0 & m) ? 1u << 18 : 0u) | ((s1 & m) ? 1u << 19 : 0u);
+        ++pos;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      if (base > prm.list_cap) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
+      misc[1] = base < prm.list_cap ? base : prm.list_cap;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const int T = misc[1];
+  const uint32_t tmem = (uint32_t)misc[0];
+  volatile int* abort = misc + 2;
+  const uint32_t sQ = sbase + L::kOffQ, sKV = sbase + L::kOffKV, sP = sbase + L::kOffP;
+
+  if (warp == 0) {
+    // ======================= TMA producer =====================================
+    if (lane == 0 && T > 0) {
+      tc::prefetch_tensormap(&tmQ);
+      tc::prefetch_tensormap(&tmK);
+      tc::prefetch_tensormap(&tmV);
+      tc::mbar_expect_tx(bar(Q_FULL), L::kQBytes);
+      for (int hf = 0; hf < 2; ++hf)
+        for (int p = 0; p < NP; ++p)
+          tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmQ, bar(Q_FULL), 64 * p, i_h[hf] * kBlock,
+                          bh_h[hf]);
+      for (int s = 0; s < 2 * T; ++s) {
+        const int n = s >> 1, slot = s % kSlots;
+        if (s >= kSlots && !tc::mbar_wait(bar(KV_EMPTY + slot), ((s / kSlots) - 1) & 1, abort)) {
+          *abort = 1;
+          report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+          break;
+        }
+        const int jb = (int)(mlist[n] & 0xFFFFu);
+        tc::mbar_expect_tx(bar(KV_FULL + slot), L::kSlotBytes);
+        for (int p = 0; p < NP; ++p)
+          tc::tma_load_3d(sKV + slot * L::kSlotBytes + p * 8192, (s & 1) ? &tmV : &tmK,
+                          bar(KV_FULL + slot), 64 * p, jb * kBlock, bkv);
+      }
+      // tail: wait for the last release of every slot, so that no tcgen05.commit
+      // arrival is still in flight when the CTA exits
+      for (int s = (2 * T > kSlots ? 2 * T - kSlots : 0); s < 2 * T && !*abort; ++s)
+        if (!tc::mbar_wait(bar(KV_EMPTY + s % kSlots), (s / kSlots) & 1, abort)) {
+          *abort = 1;
+          report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+        }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================================
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
+      constexpr uint32_t kIdPV = tc::idesc_bf16(128, D, false, true);
+      const uint32_t tO = tmem, tS0 = tmem + D;
+      bool ok = tc::mbar_wait(bar(Q_FULL), 0, abort);
+      tc::fence_after_sync();
+      auto issue_s = [&](int n) -> bool {
+        const int b = n & 1;
+        if (n >= 2 && !tc::mbar_wait(bar(S_FREE + b), ((n >> 1) - 1) & 1, abort)) return false;
+        const int s = 2 * n, slot = s % kSlots;
+        if (!tc::mbar_wait(bar(KV_FULL + slot), (s / kSlots) & 1, abort)) return false;
+        tc::fence_after_sync();
+        const uint32_t kb = sKV + slot * L::kSlotBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t da = tc::sw128_desc(sQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+          const uint64_t db = tc::sw128_desc(kb + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
+          tc::mma_bf16_ss(tS0 + 64 * b, da, db, kIdS, k > 0);
+        }
+        tc::mma_commit(bar(S_FULL + b));
+        tc::mma_commit(bar(KV_EMPTY + slot));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int n = 0; n < T && ok; ++n) {
+        if (n + 1 < T && !issue_s(n + 1)) {
+          ok = false;
+          break;
+        }
+        if (!tc::mbar_wait(bar(P_FULL), n & 1, abort)) {
+          ok = false;
+          break;
+        }
+        const int s = 2 * n + 1, slot = s % kSlots;
+        if (!tc::mbar_wait(bar(KV_FULL + slot), (s / kSlots) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t vb = sKV + slot * L::kSlotBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = tc::sw128_desc(sP + kk * 32, 16, 1024);
+          const uint64_t db = tc::sw128_desc(vb + kk * 2048, 8192, 1024);
+          tc::mma_bf16_ss(tO, da, db, kIdPV, (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(bar(O_DONE));
+        tc::mma_commit(bar(KV_EMPTY + slot));
+      }
+      if (!ok) {
+        *abort = 1;
+        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+      }
+    }
+  } else {
+    // ======================= softmax warpgroup =================================
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;       // query row of the unit
+    const int hf = r >> 6;
+    const int t = i_h[hf] * kBlock + (r & 63);
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tO = tmem + lane_off, tS0 = tmem + D + lane_off;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int n = 0; n < T; ++n) {
+      const uint32_t e = mlist[n];
+      const int jb = (int)(e & 0xFFFFu);
+      const bool act = (e >> (16 + hf)) & 1u;
+      const bool sel = (e >> (18 + hf)) & 1u;
+      const int b = n & 1;
+      // every lane takes the same branch: the TMEM loads below are warp-collective
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar(S_FULL + b), (n >> 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      uint32_t x0[32], x1[32];
+      tc::tmem_ld32(tS0 + 64 * b, x0);
+      tc::tmem_ld32(tS0 + 64 * b + 32, x1);
+      tc::tmem_ld_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(S_FREE + b));
+      float x[64];
+      float m_tile = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        const int key = jb * kBlock + j;
+        bool keep = act && key < prm.n_valid;
+        if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
+        const float sv = __uint_as_float(j < 32 ? x0[j] : x1[j - 32]);
+        x[j] = keep ? sv * prm.scale_log2 : -INFINITY;
+        m_tile = fmaxf(m_tile, x[j]);
+      }
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_tile > m_ref + kRescaleLog2 || (m_ref == -INFINITY && m_tile > -INFINITY)) {
+        if (m_ref != -INFINITY) {
+          alpha = exp2f(m_ref - m_tile);
+          resc = true;
+        }
+        m_ref = m_tile;
+      }
+      float psum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int j = 0; j < 64; j += 2) {
+        const float p0 = m_ref == -INFINITY ? 0.f : exp2f(x[j] - m_ref);
+        const float p1 = m_ref == -INFINITY ? 0.f : exp2f(x[j + 1] - m_ref);
+        psum += p0 + p1;
+        pk[j >> 1] = pack_bf16(p0, p1);
+      }
+      l_sum = l_sum * alpha + psum;
+      // PV_{n-1} must be done: it reads P and accumulates into O
+      if (n > 0) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(bar(O_DONE), (n - 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tc::tmem_ld32(tO + 32 * c, ov);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+          tc::tmem_st32(tO + 32 * c, ov);
+        }
+        tc::tmem_st_wait();
+      }
+      // P row -> shared memory, 128-byte swizzled K-major tile (row r = 128 bytes)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t addr = sP + r * 128 + ((c ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[4 * c]),
+                     "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                     : "memory");
+      }
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(P_FULL));
+    }
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(O_DONE), (T - 1) & 1, abort));
+      tc::fence_after_sync();
+    }
+    if (!ok) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
+    // epilogue: O / l -> bf16 rows (padding tokens and empty rows are zero)
+    if (valid_h[hf]) {
+      const float inv = (ok && T > 0 && l_sum > 0.f && t < prm.n_valid) ? 1.f / l_sum : 0.f;
+      __nv_bfloat16* og = prm.o + ((size_t)bh_h[hf] * prm.N + t) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (ok && T > 0) {
+          tc::tmem_ld32(tO + 32 * c, ov);
+          tc::tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = 0u;
+        }
+        uint32_t pw[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          pw[j] = inv == 0.f ? 0u
+                             : pack_bf16(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(og + 32 * c);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
+      }
+    } else if (T > 0 && ok) {
+      // keep the warp-collective TMEM loads uniform across the warp
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tc::tmem_ld32(tO + 32 * c, ov);
+        tc::tmem_ld_wait();
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 3D map over [heads][rows][D] bf16: rows beyond n_rows read as zero; box 64 x 64 x 1, 128 B swizzle.
+static bool make_map(CUtensorMap* m, const void* base, int heads, int n_rows, int N, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n_rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool TOPN>
+static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
+  using L = TcLayout<D>;
+  const sla_config& c = p.c;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, c.B * c.H, c.N_valid, c.N, D) ||
+      !make_map(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) ||
+      !make_map(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
+    return cudaErrorInvalidValue;
+  FlashTcParams prm;
+  prm.list = a.crit;
+  prm.o = TOPN ? a.out : reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_os);
+  prm.status = a.status;
+  prm.H = c.H;
+  prm.group = p.group;
+  prm.N = c.N;
+  prm.n_valid = c.N_valid;
+  prm.nb = p.nkb;
+  prm.len = TOPN ? c.top_n : c.k_h;
+  prm.window = c.window;
+  prm.pair_heads = TOPN && (p.group % 2 == 0);
+  prm.npairs = (p.nqb + 1) / 2;
+  prm.words = (p.nkb + 31) / 32;
+  int per_half = prm.len;
+  if (TOPN) per_half += (c.window + 62) / kBlock + 2;
+  prm.list_cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
+  if (prm.list_cap < 1) prm.list_cap = 1;
+  prm.scale_log2 = p.scale * 1.4426950408889634f;
+  int smem = L::kOffBits + 4 * prm.words * 4 + prm.list_cap * 4;
+  // at most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns
+  if (smem < 80 * 1024) smem = 80 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int units;
+  if (prm.pair_heads)
+    units = c.B * c.H_kv * p.nqb * (p.group / 2);
+  else
+    units = c.B * c.H * prm.npairs;
+  flash_tc_kernel<D, TOPN><<<units, kTcThreads, smem, s>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s) {
+  const bool topn = p.c.mode == SLA_MODE_TOPN_WINDOW;
+  if (p.c.d == 128) return topn ? launch_tc<128, true>(p, a, s) : launch_tc<128, false>(p, a, s);
+  return topn ? launch_tc<64, true>(p, a, s) : launch_tc<64, false>(p, a, s);
+}
+
+}  // namespace sla

@@ -16,6 +16,7 @@ constexpr int kMaxBlocks = 4096;  // nkb limit of the routing sort (N <= 262144)
 enum DeviceDetail : int {
   kDetailFlashIndex = 101,      // flash kernel read a block index outside [0, nkb)
   kDetailEpilogueIndex = 102,
+  kDetailFlashAlign = 103,     // shared-memory base not 1024-byte aligned
   kDetailTimeout = 200,
 };
 

@@ -46,6 +46,9 @@ SMALL_CASES = [
     dict(name="one_valid_token_tail", N=1024, N_valid=961, d=64, k_h=2, k_l=3),
     dict(name="no_proj", N=1024, N_valid=1000, d=128, k_h=2, k_l=2, has_proj=0),
     dict(name="batch2", B=2, N=640, N_valid=600, d=64, H=2, H_kv=1, k_h=2, k_l=1, has_gate=1),
+    dict(name="odd_blocks", N=1216, N_valid=1200, d=128, k_h=3, k_l=4, has_gate=1),
+    dict(name="odd_blocks_d64", N=1216, N_valid=1216, d=64, k_h=5, k_l=0),
+    dict(name="single_block", N=64, N_valid=50, d=128, k_h=1, k_l=0),
 ]
 
 
@@ -114,6 +117,8 @@ TOPN_CASES = [
     dict(name="topn_no_window", H=4, H_kv=4, N=1024, N_valid=1024, d=128, top_n=5, window=0),
     dict(name="topn_window_only", H=2, H_kv=1, N=1024, N_valid=1024, d=128, top_n=0, window=512),
     dict(name="topn_nsa_params", H=16, H_kv=1, N=2048, N_valid=2048, d=128, top_n=16, window=512),
+    dict(name="topn_group3_odd", H=6, H_kv=2, N=1088, N_valid=1070, d=128, top_n=3, window=100),
+    dict(name="topn_group1_odd", H=2, H_kv=2, N=1088, N_valid=1088, d=64, top_n=2, window=700),
 ]
 
 
