@@ -176,6 +176,38 @@ SLA_API const char* sla_status_string(sla_status s);
 /* Library version, e.g. "0.1.0". */
 SLA_API const char* sla_version(void);
 
+/*
+ * sla_route_noalloc - routing (steps 1-3) without a caller workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory on their call path: plugin hosts that hand a
+ * library only its input and output buffers, code running under another
+ * framework's memory pool that forbids allocations from outside it, and
+ * latency-critical loops where a cudaMalloc / cudaFree (which may synchronise
+ * the device) is not acceptable. Such callers cannot size and pass `ws`.
+ *
+ * Arguments, layouts and results are those of sla_route. The scratch that
+ * sla_route keeps in `ws` (status word, pooled means, pooled scores) lives
+ * instead in one static device array of SLA_NOALLOC_SCRATCH_BYTES (64 MiB),
+ * which every GPU that loads the library holds until the process exits. The
+ * call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine.
+ *
+ * - A configuration whose routing scratch exceeds SLA_NOALLOC_SCRATCH_BYTES is
+ *   rejected with SLA_ERR_WORKSPACE before anything is launched (about 38 MB
+ *   at B1 H12 N32768 d128; the scratch grows with B * H * (N / 64)^2).
+ * - The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ * - All calls share the one array, which keeps the last call's contents (the
+ *   status word is cleared at the start of every call). Calls that overlap on
+ *   the GPU - on two streams, or from two host threads - race on it and must
+ *   be serialised by the caller.
+ */
+#define SLA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+SLA_API sla_status sla_route_noalloc(const void* q, const void* k, const sla_config* cfg,
+                                     int8_t* mask_out, int32_t* crit_idx, int32_t* neg_idx,
+                                     void* stream);
+
 #ifdef __cplusplus
 }
 #endif
