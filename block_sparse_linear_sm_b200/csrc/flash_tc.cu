@@ -20,15 +20,17 @@
 // issues tcgen05.mma, warps 2-5 (one TMEM lane quarter each) run the online
 // softmax, one thread per query row.
 //
-// Per tile n (64 keys): S_n = Q K_n^T (M=128, N=64, TMEM, double-buffered);
-// the softmax warps load S_n, mask and exponentiate it, write P_n (bf16) to
-// shared memory; O += P_n V_n (M=128, N=D) accumulates in TMEM. S_{n+1} is
-// issued before PV_n so the tensor core works while the softmax runs. The
-// running max is only moved (and O rescaled) when a row's max grows by more
-// than 2^8, so P stays below 256 and O needs no per-tile rescale.
+// Per tile n (64 keys): S_n = Q K_n^T (M=128, N=64) into one of two TMEM
+// buffers; the softmax warps load S_n, mask and exponentiate it and write P_n
+// (bf16, two per 32-bit column) back into the same TMEM buffer; O += P_n V_n
+// (M=128, N=D, A read from TMEM) accumulates in TMEM. The MMA thread issues
+// S_{n+2} into that buffer right after PV_n (tcgen05 operations of one thread
+// execute in issue order), so two score tiles are always ahead of the softmax.
+// The running max only moves (and O is rescaled) when a row's max grows by
+// more than 2^8, so P stays below 256 and O needs no per-tile rescale.
 //
-// Shared memory: Q (128 x D bf16), a ring of three 64-row K/V slots, P
-// (128 x 64 bf16), the merged block list. All operand tiles use the 128-byte
+// Shared memory: Q (128 x D bf16), a ring of four 64-row K/V slots (K and V
+// tiles alternate), the merged block list. Operand tiles use the 128-byte
 // swizzle. Two CTAs fit on one SM (TMEM: 256 columns each).
 #include "common.cuh"
 #include "tc.cuh"
@@ -48,18 +50,16 @@ struct FlashTcParams {
 };
 
 constexpr int kTcThreads = 192;
-constexpr int kSlots = 3;
+constexpr int kSlots = 4;
 constexpr float kRescaleLog2 = 8.f;
 
 template <int D>
 struct TcLayout {
   static constexpr int kQBytes = 128 * D * 2;           // 2 halves x D/64 panels x 8 KB
   static constexpr int kSlotBytes = 64 * D * 2;         // one K or V tile
-  static constexpr int kPBytes = 128 * 64 * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + kQBytes;
-  static constexpr int kOffP = kOffKV + kSlots * kSlotBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;        // 16 mbarriers
+  static constexpr int kOffBar = kOffKV + kSlots * kSlotBytes;  // 16 mbarriers
   static constexpr int kOffMisc = kOffBar + 16 * 8;      // tmem addr, count, abort
   static constexpr int kOffBits = kOffMisc + 64;         // 4 bitmaps
   static constexpr int kTmemCols = 256;                  // O: D columns, S: 2 x 64 columns
@@ -85,8 +85,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   // misc[0] = TMEM base, misc[1] = merged count, misc[2] = abort
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
   // barrier ids
-  constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 4, S_FULL = 7, S_FREE = 9, P_FULL = 11,
-                O_DONE = 12;
+  constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + kSlots, S_FULL = 1 + 2 * kSlots,
+                P_FULL = S_FULL + 2, O_DONE = P_FULL + 2;
 
   // ---- unit decode ----------------------------------------------------------
   const int Hkv = prm.H / prm.group;
@@ -135,9 +135,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(S_FULL + b), 1);
-      tc::mbar_init(bar(S_FREE + b), 4);
+      tc::mbar_init(bar(P_FULL + b), 4);
     }
-    tc::mbar_init(bar(P_FULL), 4);
     tc::mbar_init(bar(O_DONE), 1);
     tc::fence_mbar_init();
   }
@@ -206,7 +205,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int T = misc[1];
   const uint32_t tmem = (uint32_t)misc[0];
   volatile int* abort = misc + 2;
-  const uint32_t sQ = sbase + L::kOffQ, sKV = sbase + L::kOffKV, sP = sbase + L::kOffP;
+  const uint32_t sQ = sbase + L::kOffQ, sKV = sbase + L::kOffKV;
 
   if (warp == 0) {
     // ======================= TMA producer =====================================
@@ -248,9 +247,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const uint32_t tO = tmem, tS0 = tmem + D;
       bool ok = tc::mbar_wait(bar(Q_FULL), 0, abort);
       tc::fence_after_sync();
+      // S_n = Q K_n^T into TMEM buffer n & 1
       auto issue_s = [&](int n) -> bool {
-        const int b = n & 1;
-        if (n >= 2 && !tc::mbar_wait(bar(S_FREE + b), ((n >> 1) - 1) & 1, abort)) return false;
         const int s = 2 * n, slot = s % kSlots;
         if (!tc::mbar_wait(bar(KV_FULL + slot), (s / kSlots) & 1, abort)) return false;
         tc::fence_after_sync();
@@ -259,19 +257,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         for (int k = 0; k < D / 16; ++k) {
           const uint64_t da = tc::sw128_desc(sQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
           const uint64_t db = tc::sw128_desc(kb + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
-          tc::mma_bf16_ss(tS0 + 64 * b, da, db, kIdS, k > 0);
+          tc::mma_bf16_ss(tS0 + 64 * (n & 1), da, db, kIdS, k > 0);
         }
-        tc::mma_commit(bar(S_FULL + b));
+        tc::mma_commit(bar(S_FULL + (n & 1)));
         tc::mma_commit(bar(KV_EMPTY + slot));
         return true;
       };
       if (ok) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
       for (int n = 0; n < T && ok; ++n) {
-        if (n + 1 < T && !issue_s(n + 1)) {
-          ok = false;
-          break;
-        }
-        if (!tc::mbar_wait(bar(P_FULL), n & 1, abort)) {
+        const int b = n & 1;
+        // P_n sits in TMEM buffer b (written by the softmax warps)
+        if (!tc::mbar_wait(bar(P_FULL + b), (n >> 1) & 1, abort)) {
           ok = false;
           break;
         }
@@ -284,12 +281,16 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const uint32_t vb = sKV + slot * L::kSlotBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = tc::sw128_desc(sP + kk * 32, 16, 1024);
           const uint64_t db = tc::sw128_desc(vb + kk * 2048, 8192, 1024);
-          tc::mma_bf16_ss(tO, da, db, kIdPV, (n > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(tO, tS0 + 64 * b + 8 * kk, db, kIdPV, (n > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(bar(O_DONE));
         tc::mma_commit(bar(KV_EMPTY + slot));
+        // buffer b is free once PV_n has read P_n: S_{n+2} is issued behind it
+        if (n + 2 < T && !issue_s(n + 2)) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) {
         *abort = 1;
@@ -302,60 +303,86 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int r = quarter * 32 + lane;       // query row of the unit
     const int hf = r >> 6;
     const int t = i_h[hf] * kBlock + (r & 63);
+    const int t_lo = i_h[hf] * kBlock + ((quarter * 32) & 63);  // first token of this warp
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tO = tmem + lane_off, tS0 = tmem + D + lane_off;
-    float m_ref = -INFINITY, l_sum = 0.f;
+    const float sl2 = prm.scale_log2;
+    float m_ref = -INFINITY, l_sum = 0.f;    // m_ref in the scaled log2 domain
     bool ok = true;
     for (int n = 0; n < T; ++n) {
       const uint32_t e = mlist[n];
       const int jb = (int)(e & 0xFFFFu);
-      const bool act = (e >> (16 + hf)) & 1u;
+      const bool act = (e >> (16 + hf)) & 1u;   // uniform across the warp (one half per warp)
       const bool sel = (e >> (18 + hf)) & 1u;
       const int b = n & 1;
-      // every lane takes the same branch: the TMEM loads below are warp-collective
+      const uint32_t tS = tS0 + 64 * b;
+      // every lane takes the same branch: the TMEM accesses below are warp-collective
       if (!__all_sync(0xffffffffu, tc::mbar_wait(bar(S_FULL + b), (n >> 1) & 1, abort))) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      uint32_t x0[32], x1[32];
-      tc::tmem_ld32(tS0 + 64 * b, x0);
-      tc::tmem_ld32(tS0 + 64 * b + 32, x1);
-      tc::tmem_ld_wait();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(S_FREE + b));
-      float x[64];
-      float m_tile = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const int key = jb * kBlock + j;
-        bool keep = act && key < prm.n_valid;
-        if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
-        const float sv = __uint_as_float(j < 32 ? x0[j] : x1[j - 32]);
-        x[j] = keep ? sv * prm.scale_log2 : -INFINITY;
-        m_tile = fmaxf(m_tile, x[j]);
-      }
+      uint32_t pk[32];
       float alpha = 1.f;
       bool resc = false;
-      if (m_tile > m_ref + kRescaleLog2 || (m_ref == -INFINITY && m_tile > -INFINITY)) {
-        if (m_ref != -INFINITY) {
-          alpha = exp2f(m_ref - m_tile);
-          resc = true;
-        }
-        m_ref = m_tile;
-      }
-      float psum = 0.f;
-      uint32_t pk[32];
+      if (act) {
+        uint32_t x0[32], x1[32];
+        tc::tmem_ld32(tS, x0);
+        tc::tmem_ld32(tS + 32, x1);
+        tc::tmem_ld_wait();
+        float x[64];
 #pragma unroll
-      for (int j = 0; j < 64; j += 2) {
-        const float p0 = m_ref == -INFINITY ? 0.f : exp2f(x[j] - m_ref);
-        const float p1 = m_ref == -INFINITY ? 0.f : exp2f(x[j + 1] - m_ref);
-        psum += p0 + p1;
-        pk[j >> 1] = pack_bf16(p0, p1);
+        for (int j = 0; j < 32; ++j) {
+          x[j] = __uint_as_float(x0[j]);
+          x[32 + j] = __uint_as_float(x1[j]);
+        }
+        const int k0 = jb * kBlock;
+        bool need_mask = k0 + kBlock > prm.n_valid;
+        if (TOPN) need_mask = need_mask || (k0 + kBlock - 1 > t_lo) || (!sel && k0 <= t_lo + 31 - prm.window);
+        if (need_mask) {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const int key = k0 + j;
+            bool keep = key < prm.n_valid;
+            if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
+            x[j] = keep ? x[j] : -INFINITY;
+          }
+        }
+        float mx[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = x[u];
+#pragma unroll
+        for (int j = 8; j < 64; ++j) mx[j & 7] = fmaxf(mx[j & 7], x[j]);
+        const float m_raw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float m_tile = m_raw * sl2;
+        if (m_tile > m_ref + kRescaleLog2) {
+          if (m_ref != -INFINITY) {
+            alpha = tc::ex2_approx(m_ref - m_tile);
+            resc = true;
+          }
+          m_ref = m_tile;
+        }
+        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (m_ref != -INFINITY) {
+          const float neg = -m_ref;
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const float p0 = tc::ex2_approx(fmaf(x[j], sl2, neg));
+            const float p1 = tc::ex2_approx(fmaf(x[j + 1], sl2, neg));
+            sm[(j >> 1) & 7] += p0 + p1;
+            pk[j >> 1] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pk[j] = 0u;
+        }
+        l_sum = l_sum * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pk[j] = 0u;  // this half does not use the tile
       }
-      l_sum = l_sum * alpha + psum;
-      // PV_{n-1} must be done: it reads P and accumulates into O
+      // O rescale needs PV_{n-1} complete (it accumulates into O)
       if (n > 0) {
         if (!__all_sync(0xffffffffu, tc::mbar_wait(bar(O_DONE), (n - 1) & 1, abort))) {
           ok = false;
@@ -373,20 +400,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
           tc::tmem_st32(tO + 32 * c, ov);
         }
-        tc::tmem_st_wait();
       }
-      // P row -> shared memory, 128-byte swizzled K-major tile (row r = 128 bytes)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t addr = sP + r * 128 + ((c ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[4 * c]),
-                     "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                     : "memory");
-      }
-      tc::fence_async_smem();
+      // P_n (bf16 pairs) into the first 32 columns of its S buffer
+      tc::tmem_st32(tS, pk);
+      tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(P_FULL));
+      if (lane == 0) tc::mbar_arrive(bar(P_FULL + b));
     }
     if (ok && T > 0) {
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(O_DONE), (T - 1) & 1, abort));
