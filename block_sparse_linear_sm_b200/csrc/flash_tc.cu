@@ -500,7 +500,9 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   FlashTcParams prm;
   prm.list = a.crit;
-  prm.o = TOPN ? a.out : reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_os);
+  // with a linear branch the epilogue combines; otherwise this is the output
+  const bool direct = TOPN || p.nkb - c.k_h - c.k_l <= 0;
+  prm.o = direct ? a.out : reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_os);
   prm.status = a.status;
   prm.H = c.H;
   prm.group = p.group;

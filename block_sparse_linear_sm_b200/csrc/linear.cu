@@ -7,27 +7,36 @@
 // h_j = phi(K_j)^T V_j and the normaliser z_j = sum_t phi(k_t); query block i
 // then needs S_i = sum_{j marginal} h_j and Z_i = sum_{j marginal} z_j.
 //
-// Layout: Hs[bkv][j][0 : d*d] = h_j row-major, Hs[bkv][j][d*d : d*d+d] = z_j,
+// Layout: Hs[bkv][j][0 : d*d] = h_j row-major (times W_p when the layer has a
+// projection: h'_j = phi(K_j)^T V_j W_p), Hs[bkv][j][d*d : d*d+d] = z_j,
 // zero up to dd (a multiple of 128), rows j in [nkb, nkb_pad) zero; bf16.
 // The aggregation is the GEMM S = M . Hs with M the 0/1 marginal mask of each
-// query head (exact in bf16), accumulated in fp32: Ss[bh][i][0 : dd].
+// query head (exact in bf16), accumulated in fp32 and stored as S_i (bf16,
+// [bh][i][d*d]) and Z_i (fp32, [bh][i][d]).
 #include "common.cuh"
 
 namespace sla {
 
 // ---------------------------------------------------------------------------
-// state kernel: one CTA per (b, kv head, key block); D/16 warps, warp w owns
-// rows 16w..16w+15 of h_j (the phi(K) feature index).
+// state kernel: one CTA per (b, kv head, key block); D/16 warps.
+// With a projection, W_p is folded into the state: O_l W_p =
+// phi(q) sum_j phi(K_j)^T (V_j W_p) / den, so the block first forms
+// T_j = V_j W_p (warp w owns token rows 16(w%4).. of T, column half w/4), then
+// h'_j = phi(K_j)^T T_j (warp w owns rows 16w..16w+15 of h'_j).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(D * 2) state_kernel(const __nv_bfloat16* __restrict__ k,
                                                       const __nv_bfloat16* __restrict__ v,
+                                                      const __nv_bfloat16* __restrict__ w_p,
                                                       __nv_bfloat16* __restrict__ hs, int N,
                                                       int n_valid, int nkb, int dd) {
   constexpr int RB = D * 2;  // bytes per smem row
   constexpr int CH = D / 8;  // 16-byte chunks per row
-  __shared__ __align__(128) unsigned char fk_s[kBlock * RB];
-  __shared__ __align__(128) unsigned char v_s[kBlock * RB];
+  constexpr int NW = D / 16; // warps
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* fk_s = smem;                    // [64][D]  phi(K)
+  unsigned char* v_s = fk_s + kBlock * RB;       // [64][D]  V, then T = V W_p
+  unsigned char* w_s = v_s + kBlock * RB;        // [D][D]   W_p (only with a projection)
   const int j = blockIdx.x;
   const int bkv = blockIdx.y;
   __nv_bfloat16* row = hs + ((size_t)bkv * gridDim.x + j) * dd;
@@ -40,22 +49,35 @@ __global__ void __launch_bounds__(D * 2) state_kernel(const __nv_bfloat16* __res
   nv = nv > kBlock ? kBlock : nv;
   const __nv_bfloat16* kb = k + ((size_t)bkv * N + (size_t)j * kBlock) * D;
   const __nv_bfloat16* vb = v + ((size_t)bkv * N + (size_t)j * kBlock) * D;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const uint32_t fk_base = smem_u32(fk_s), v_base = smem_u32(v_s), w_base = smem_u32(w_s);
+  if (w_p) {
+    for (int e = threadIdx.x; e < D * CH; e += blockDim.x) {
+      const int r = e / CH, ch = e % CH;
+      cp_async16(w_base + swz(r, ch, RB), w_p + (size_t)r * D + ch * 8, 16);
+    }
+  }
   for (int e = threadIdx.x; e < kBlock * CH; e += blockDim.x) {
     const int t = e / CH, ch = e % CH;
-    uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    const int bytes = t < nv ? 16 : 0;
+    cp_async16(v_base + swz(t, ch, RB), vb + (bytes ? (size_t)t * D + ch * 8 : 0), bytes);
+  }
+  cp_async_commit();
+  for (int e = threadIdx.x; e < kBlock * CH; e += blockDim.x) {
+    const int t = e / CH, ch = e % CH;
+    uint4 kk = make_uint4(0, 0, 0, 0);
     if (t < nv) {
       kk = *reinterpret_cast<const uint4*>(kb + (size_t)t * D + ch * 8);
-      vv = *reinterpret_cast<const uint4*>(vb + (size_t)t * D + ch * 8);
-      uint32_t* w = reinterpret_cast<uint32_t*>(&kk);
+      uint32_t* wv = reinterpret_cast<uint32_t*>(&kk);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        float2 f = unpack_bf16(w[u]);
-        w[u] = pack_bf16(phi(f.x), phi(f.y));
+        float2 f = unpack_bf16(wv[u]);
+        wv[u] = pack_bf16(phi(f.x), phi(f.y));
       }
     }
     *reinterpret_cast<uint4*>(fk_s + swz(t, ch, RB)) = kk;
-    *reinterpret_cast<uint4*>(v_s + swz(t, ch, RB)) = vv;
   }
+  cp_async_wait<0>();
   __syncthreads();
   // z_j from the same bf16-rounded features the MMA uses
   if (threadIdx.x < D) {
@@ -70,8 +92,39 @@ __global__ void __launch_bounds__(D * 2) state_kernel(const __nv_bfloat16* __res
   }
   for (int e = D * D + D + threadIdx.x; e < dd; e += blockDim.x) row[e] = __float2bfloat16(0.f);
 
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const uint32_t fk_base = smem_u32(fk_s), v_base = smem_u32(v_s);
+  if (w_p) {
+    // T = V W_p: warp w -> token rows 16*(w % 4) .., columns [half*D/2, (half+1)*D/2)
+    constexpr int HALVES = NW / 4;  // 2 for D=128, 1 for D=64
+    constexpr int NC = D / HALVES;  // columns per warp
+    const int mt = w & 3, half = w >> 2;
+    float t_acc[NC / 8][4];
+#pragma unroll
+    for (int n = 0; n < NC / 8; ++n) t_acc[n][0] = t_acc[n][1] = t_acc[n][2] = t_acc[n][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(lds_a(v_base, mt * 16, 2 * ks, RB, lane), a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int n2 = 0; n2 < NC / 16; ++n2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(lds_b_kn(w_base, ks * 16, (half * NC) / 8 + 2 * n2, RB, lane), b0, b1, b2, b3);
+        mma_bf16(t_acc[2 * n2], a, b0, b1);
+        mma_bf16(t_acc[2 * n2 + 1], a, b2, b3);
+      }
+    }
+    __syncthreads();  // every warp has read V: T may overwrite it
+    const int r0 = mt * 16 + (lane >> 2);
+#pragma unroll
+    for (int n = 0; n < NC / 8; ++n) {
+      const int col = half * NC + n * 8 + 2 * (lane & 3);
+      *reinterpret_cast<uint32_t*>(v_s + swz(r0, col >> 3, RB) + (col & 7) * 2) =
+          pack_bf16(t_acc[n][0], t_acc[n][1]);
+      *reinterpret_cast<uint32_t*>(v_s + swz(r0 + 8, col >> 3, RB) + (col & 7) * 2) =
+          pack_bf16(t_acc[n][2], t_acc[n][3]);
+    }
+    __syncthreads();
+  }
+
   float acc[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -100,11 +153,17 @@ __global__ void __launch_bounds__(D * 2) state_kernel(const __nv_bfloat16* __res
 cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s) {
   const sla_config& c = p.c;
   __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_hs);
+  const __nv_bfloat16* wp = c.has_proj ? a.w_p : nullptr;
   dim3 grid(p.nkb_pad, c.B * c.H_kv);
-  if (c.d == 128)
-    state_kernel<128><<<grid, 256, 0, s>>>(a.k, a.v, hs, c.N, c.N_valid, p.nkb, p.dd);
-  else
-    state_kernel<64><<<grid, 128, 0, s>>>(a.k, a.v, hs, c.N, c.N_valid, p.nkb, p.dd);
+  if (c.d == 128) {
+    const int smem = 2 * kBlock * 256 + (wp ? 128 * 256 : 0);
+    cudaError_t e = cudaFuncSetAttribute(state_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    state_kernel<128><<<grid, 256, smem, s>>>(a.k, a.v, wp, hs, c.N, c.N_valid, p.nkb, p.dd);
+  } else {
+    const int smem = 2 * kBlock * 128 + (wp ? 64 * 128 : 0);
+    state_kernel<64><<<grid, 128, smem, s>>>(a.k, a.v, wp, hs, c.N, c.N_valid, p.nkb, p.dd);
+  }
   return cudaGetLastError();
 }
 
@@ -120,8 +179,10 @@ constexpr int kAggSmem = kAggStages * (kAggABytes + kAggBBytes);
 
 __global__ void __launch_bounds__(256) aggregate_kernel(const __nv_bfloat16* __restrict__ mmask,
                                                         const __nv_bfloat16* __restrict__ hs,
-                                                        float* __restrict__ ss, int H, int group,
-                                                        int nqb, int nqb_pad, int nkb_pad, int dd) {
+                                                        __nv_bfloat16* __restrict__ ss,
+                                                        float* __restrict__ zs, int H, int group,
+                                                        int nqb, int nqb_pad, int nkb_pad, int dd,
+                                                        int d) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int n0 = blockIdx.x * kAggN;
   const int m0 = blockIdx.y * kAggM;
@@ -190,18 +251,26 @@ __global__ void __launch_bounds__(256) aggregate_kernel(const __nv_bfloat16* __r
     }
   }
   cp_async_wait<0>();
-  float* C = ss + (size_t)bh * nqb * dd;
+  // columns < d*d: S_i in bf16; the next d columns: Z_i in fp32; the rest is padding
+  const int dsq = d * d;
+  __nv_bfloat16* S = ss + (size_t)bh * nqb * dsq;
+  float* Z = zs + (size_t)bh * nqb * d;
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     const int r = m0 + wm * 64 + mt * 16 + (lane >> 2);
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
       const int col = n0 + wn * 32 + nt * 8 + 2 * (lane & 3);
-      if (r < nqb)
-        *reinterpret_cast<float2*>(C + (size_t)r * dd + col) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
-      if (r + 8 < nqb)
-        *reinterpret_cast<float2*>(C + (size_t)(r + 8) * dd + col) =
-            make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int rr = r + 8 * hh;
+        if (rr >= nqb) continue;
+        const float v0 = acc[mt][nt][2 * hh], v1 = acc[mt][nt][2 * hh + 1];
+        if (col < dsq)
+          *reinterpret_cast<uint32_t*>(S + (size_t)rr * dsq + col) = pack_bf16(v0, v1);
+        else if (col < dsq + d)
+          *reinterpret_cast<float2*>(Z + (size_t)rr * d + (col - dsq)) = make_float2(v0, v1);
+      }
     }
   }
 }
@@ -210,13 +279,14 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
   const sla_config& c = p.c;
   const __nv_bfloat16* mm = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_mmask);
   const __nv_bfloat16* hs = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_hs);
-  float* ss = reinterpret_cast<float*>(a.ws + p.off_ss);
+  __nv_bfloat16* ss = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_ss);
+  float* zs = reinterpret_cast<float*>(a.ws + p.off_zs);
   cudaError_t e = cudaFuncSetAttribute(aggregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kAggSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.dd / kAggN, p.nqb_pad / kAggM, c.B * c.H);
-  aggregate_kernel<<<grid, 256, kAggSmem, s>>>(mm, hs, ss, c.H, p.group, p.nqb, p.nqb_pad,
-                                               p.nkb_pad, p.dd);
+  aggregate_kernel<<<grid, 256, kAggSmem, s>>>(mm, hs, ss, zs, c.H, p.group, p.nqb, p.nqb_pad,
+                                               p.nkb_pad, p.dd, c.d);
   return cudaGetLastError();
 }
 

@@ -126,249 +126,278 @@ cudaError_t launch_scores(const Plan& p, const Args& a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// sorting helpers: order-preserving 64-bit key of a double, bitonic sort of
-// (key, index) pairs so that higher keys come first and equal keys keep the
-// lower index first.
+// Exact top-c selection, one warp per row.
+//
+// Scores become order-preserving 64-bit keys; "j ranks before l" means
+// key_j > key_l, or equal keys and j < l (the lower block index first). The
+// top c of a row are found by an MSD radix select over 8-bit digits: each pass
+// histograms the digit of the keys that still share the selected prefix and
+// picks the bin holding the c-th key. The pass stops early once that bin is
+// taken whole; after all 8 digits, keys equal to the boundary key are taken in
+// index order.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ unsigned long long order_key(double x) {
   const long long b = __double_as_longlong(x);
   return b < 0 ? ~(unsigned long long)b : ((unsigned long long)b | 0x8000000000000000ull);
 }
 
-__device__ __forceinline__ bool ranks_before(unsigned long long ka, int ia, unsigned long long kb,
-                                             int ib) {
-  return ka > kb || (ka == kb && ia < ib);
-}
+struct TopSel {
+  unsigned long long prefix, mask;  // keys with (key & mask) > prefix are in the set
+  int need;                         // how many keys with (key & mask) == prefix are in
+  bool whole;                       // all keys with (key & mask) == prefix are in
+};
 
-// Sorts P (a power of two) pairs in shared memory; all threads of the CTA take part.
-__device__ void bitonic_sort(unsigned long long* key, uint16_t* idx, int P) {
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < P; i += blockDim.x) {
-        const int l = i ^ j;
-        if (l > i) {
-          const bool first_half = (i & k) == 0;
-          const bool i_first = ranks_before(key[i], idx[i], key[l], idx[l]);
-          if (first_half != i_first) {
-            unsigned long long tk = key[i];
-            key[i] = key[l];
-            key[l] = tk;
-            uint16_t ti = idx[i];
-            idx[i] = idx[l];
-            idx[l] = ti;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-}
-
-// Block-wide exclusive scan of one int per thread; returns the prefix, *total gets the sum.
-__device__ int block_exclusive_scan(int v, int* total, int* scratch /* >= 33 ints */) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int x = v;
+// keys[0..n) in shared memory, hist = 256 words of this warp; 1 <= c <= n.
+__device__ TopSel warp_select_top(const unsigned long long* keys, int n, int c, unsigned* hist) {
+  const int lane = threadIdx.x & 31;
+  TopSel r{0ull, 0ull, c, false};
+  for (int shift = 56; shift >= 0; shift -= 8) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) scratch[wid] = x;
-  __syncthreads();
-  if (wid == 0) {
-    const int nw = blockDim.x >> 5;
-    int w = lane < nw ? scratch[lane] : 0;
+    for (int u = 0; u < 8; ++u) hist[lane * 8 + u] = 0u;
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const unsigned long long key = keys[j];
+      if ((key & r.mask) == r.prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane l owns bins 255-8l .. 248-8l (descending)
+    unsigned cnt[8];
+    unsigned tot = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      cnt[u] = hist[255 - 8 * lane - u];
+      tot += cnt[u];
+    }
+    unsigned incl = tot;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
+      const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    if (lane < nw) scratch[lane] = w;
-    if (lane == nw - 1) scratch[32] = w;
+    const unsigned excl = incl - tot;
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)r.need);
+    const int owner = __ffs(hit) - 1;
+    int bin = 0;
+    unsigned above = 0, inbin = 0;
+    if (lane == owner) {
+      unsigned run = excl;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (run + cnt[u] >= (unsigned)r.need) {
+          bin = 255 - 8 * lane - u;
+          above = run;
+          inbin = cnt[u];
+          break;
+        }
+        run += cnt[u];
+      }
+    }
+    bin = __shfl_sync(0xffffffffu, bin, owner);
+    above = __shfl_sync(0xffffffffu, above, owner);
+    inbin = __shfl_sync(0xffffffffu, inbin, owner);
+    __syncwarp();
+    r.need -= (int)above;
+    r.prefix |= (unsigned long long)bin << shift;
+    r.mask |= 255ull << shift;
+    if (inbin == (unsigned)r.need) {
+      r.whole = true;
+      break;
+    }
   }
-  __syncthreads();
-  const int before = (wid > 0 ? scratch[wid - 1] : 0) + x - v;
-  *total = scratch[32];
-  __syncthreads();
-  return before;
+  return r;
 }
 
-// Writes the ascending list of indices j < n with cls[j] == want into out.
-__device__ void compact_ascending(const int8_t* cls, int n, int8_t want, int32_t* out,
-                                  int* scratch) {
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int lo = threadIdx.x * per;
-  const int hi = min(lo + per, n);
-  int cnt = 0;
-  for (int j = lo; j < hi; ++j) cnt += cls[j] == want;
-  int total;
-  int pos = block_exclusive_scan(cnt, &total, scratch);
-  for (int j = lo; j < hi; ++j)
-    if (cls[j] == want) out[pos++] = j;
-}
-
-// ---------------------------------------------------------------------------
-// three-way classification: one CTA per (b, h, query block i).
-// ---------------------------------------------------------------------------
-constexpr int kSortThreads = 256;
-
-__global__ void __launch_bounds__(kSortThreads) classify_kernel(
-    const double* __restrict__ scores, int8_t* __restrict__ mask_out, int32_t* __restrict__ crit,
-    int32_t* __restrict__ neg, __nv_bfloat16* __restrict__ mmask, int nb, int P, int k_h, int k_l,
-    int nkb_pad, int nqb_pad) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem);
-  uint16_t* idx = reinterpret_cast<uint16_t*>(smem + (size_t)P * 8);
-  int8_t* cls = reinterpret_cast<int8_t*>(smem + (size_t)P * 10);
-  __shared__ int scratch[33];
-  const int i = blockIdx.x;
-  const int bh = blockIdx.y;
-  if (i >= nb) {
-    // rows past the last query block of the aggregation mask are zero
-    __nv_bfloat16* mrow = mmask + ((size_t)bh * nqb_pad + i) * nkb_pad;
-    for (int j = threadIdx.x; j < nkb_pad; j += blockDim.x) mrow[j] = __float2bfloat16(0.f);
+// Marks in_set[j] (bit flags in `flags`, value `bit`) for the top c keys.
+__device__ void warp_mark_top(const unsigned long long* keys, int n, int c, unsigned* hist,
+                              uint8_t* flags, uint8_t bit) {
+  const int lane = threadIdx.x & 31;
+  if (c <= 0) return;
+  if (c >= n) {
+    for (int j = lane; j < n; j += 32) flags[j] |= bit;
+    __syncwarp();
     return;
   }
-  const double* row = scores + ((size_t)bh * nb + i) * nb;
-  for (int j = threadIdx.x; j < P; j += blockDim.x) {
-    key[j] = j < nb ? order_key(row[j]) : 0ull;
-    idx[j] = (uint16_t)(j < nb ? j : 0xFFFF);
+  const TopSel t = warp_select_top(keys, n, c, hist);
+  int taken = 0;  // equal keys taken so far, in index order
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    bool in = false, eq = false;
+    if (j < n) {
+      const unsigned long long km = keys[j] & t.mask;
+      in = km > t.prefix;
+      eq = km == t.prefix;
+    }
+    if (t.whole) {
+      in = in || eq;
+    } else {
+      const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+      const int rank = taken + __popc(eqb & ((1u << lane) - 1u));
+      in = in || (eq && rank < t.need);
+      taken += __popc(eqb);
+    }
+    if (in) flags[j] |= bit;
   }
-  __syncthreads();
-  bitonic_sort(key, idx, P);
-  for (int p = threadIdx.x; p < nb; p += blockDim.x)
-    cls[idx[p]] = p < k_h ? (int8_t)2 : (p >= nb - k_l ? (int8_t)0 : (int8_t)1);
-  __syncthreads();
-  const size_t rowoff = ((size_t)bh * nb + i) * nb;
-  if (mask_out)
-    for (int j = threadIdx.x; j < nb; j += blockDim.x) mask_out[rowoff + j] = cls[j];
-  if (mmask) {
-    __nv_bfloat16* mrow = mmask + ((size_t)bh * nqb_pad + i) * nkb_pad;
-    for (int j = threadIdx.x; j < nkb_pad; j += blockDim.x)
-      mrow[j] = __float2bfloat16(j < nb && cls[j] == 1 ? 1.f : 0.f);
-  }
-  if (crit && k_h > 0) compact_ascending(cls, nb, 2, crit + ((size_t)bh * nb + i) * k_h, scratch);
-  if (neg && k_l > 0) compact_ascending(cls, nb, 0, neg + ((size_t)bh * nb + i) * k_l, scratch);
+  __syncwarp();
 }
 
-static int pow2_at_least(int n) {
-  int P = 1;
-  while (P < n) P <<= 1;
-  return P;
+// Ascending list of the j < n with (flags[j] & bit) == want into out.
+__device__ void warp_compact(const uint8_t* flags, int n, uint8_t bit, uint8_t want, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const bool sel = j < n && ((flags[j] & bit) == want);
+    const unsigned b = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[base + __popc(b & ((1u << lane) - 1u))] = j;
+    base += __popc(b);
+  }
+}
+
+constexpr int kRouteWarps = 8;
+
+static int route_rows_per_cta(int nb) {
+  const size_t per = (size_t)nb * 8 + (size_t)nb + 1024 + 64;  // keys, flags, histogram
+  int r = (int)((96 * 1024) / per);
+  return r < 1 ? 1 : (r > kRouteWarps ? kRouteWarps : r);
+}
+
+static size_t route_smem(int nb, int rows) {
+  return (size_t)rows * ((size_t)nb * 8 + align_up((size_t)nb, 16) + 1024);
+}
+
+// ---------------------------------------------------------------------------
+// three-way classification: one warp per (b, h, query block i).
+// flags bit 1: among the top k_h (critical); bit 2: among the top nb - k_l
+// (not negligible). Class = 2 critical, 1 marginal, 0 negligible.
+// ---------------------------------------------------------------------------
+__global__ void classify_kernel(const double* __restrict__ scores, int8_t* __restrict__ mask_out,
+                                int32_t* __restrict__ crit, int32_t* __restrict__ neg,
+                                __nv_bfloat16* __restrict__ mmask, int nb, int k_h, int k_l,
+                                int nkb_pad, int nqb_pad, int rows, int n_rows) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * rows + w;  // over B*H*nqb_pad
+  if (w >= rows || row >= n_rows) return;
+  const int bh = row / nqb_pad, i = row % nqb_pad;
+  if (i >= nb) {
+    // rows past the last query block of the aggregation mask are zero
+    if (mmask) {
+      __nv_bfloat16* mrow = mmask + ((size_t)bh * nqb_pad + i) * nkb_pad;
+      for (int j = lane; j < nkb_pad; j += 32) mrow[j] = __float2bfloat16(0.f);
+    }
+    return;
+  }
+  unsigned char* base = smem + (size_t)w * ((size_t)nb * 8 + align_up((size_t)nb, 16) + 1024);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(base);
+  uint8_t* flags = base + (size_t)nb * 8;
+  unsigned* hist = reinterpret_cast<unsigned*>(base + (size_t)nb * 8 + align_up((size_t)nb, 16));
+  const double* srow = scores + ((size_t)bh * nb + i) * nb;
+  for (int j = lane; j < nb; j += 32) {
+    keys[j] = order_key(srow[j]);
+    flags[j] = 0;
+  }
+  __syncwarp();
+  warp_mark_top(keys, nb, k_h, hist, flags, 1);
+  warp_mark_top(keys, nb, nb - k_l, hist, flags, 2);
+  const size_t rowoff = ((size_t)bh * nb + i) * nb;
+  if (mask_out)
+    for (int j = lane; j < nb; j += 32) {
+      const uint8_t f = flags[j];
+      mask_out[rowoff + j] = (f & 1) ? 2 : ((f & 2) ? 1 : 0);
+    }
+  if (mmask) {
+    __nv_bfloat16* mrow = mmask + ((size_t)bh * nqb_pad + i) * nkb_pad;
+    for (int j = lane; j < nkb_pad; j += 32)
+      mrow[j] = __float2bfloat16(j < nb && flags[j] == 2 ? 1.f : 0.f);
+  }
+  if (crit && k_h > 0) warp_compact(flags, nb, 1, 1, crit + ((size_t)bh * nb + i) * k_h);
+  if (neg && k_l > 0) warp_compact(flags, nb, 2, 0, neg + ((size_t)bh * nb + i) * k_l);
 }
 
 cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cudaStream_t s) {
   const sla_config& c = p.c;
   const double* sc = reinterpret_cast<const double*>(a.ws + p.off_scores);
   __nv_bfloat16* mm = write_mmask ? reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_mmask) : nullptr;
-  const int P = pow2_at_least(p.nkb);
-  const size_t smem = (size_t)P * 10 + align_up(p.nkb, 16);
+  const int rows = route_rows_per_cta(p.nkb);
+  const size_t smem = route_smem(p.nkb, rows);
   cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  // with the aggregation mask, extra CTAs zero its padding rows nqb..nqb_pad
-  dim3 grid(write_mmask ? p.nqb_pad : p.nqb, c.B * c.H);
-  classify_kernel<<<grid, kSortThreads, smem, s>>>(sc, a.mask_out, a.crit, a.neg, mm, p.nkb, P,
-                                                   c.k_h, c.k_l, p.nkb_pad, p.nqb_pad);
+  // with the aggregation mask, rows nqb..nqb_pad (zero padding) get warps too
+  const int per_head = write_mmask ? p.nqb_pad : p.nqb;
+  const int n_rows = c.B * c.H * per_head;
+  const int grid = (n_rows + rows - 1) / rows;
+  classify_kernel<<<grid, rows * 32, smem, s>>>(sc, a.mask_out, a.crit, a.neg, mm, p.nkb, c.k_h,
+                                                c.k_l, p.nkb_pad, per_head, rows, n_rows);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// top-n selection: one CTA per (b, KV head, query block i). The group's heads
-// each take a softmax of their pooled scores over the past blocks j < i; the
-// probabilities are summed and the top min(top_n, i) kept.
+// top-n selection: one warp per (b, KV head, query block i). Each of the
+// group's heads takes a softmax of its pooled scores over the past blocks
+// j < i (float64); the probabilities are summed and the top min(top_n, i)
+// kept (same exact select as above).
 // ---------------------------------------------------------------------------
-__device__ double block_reduce(double v, bool is_max, double* red) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    double y = __shfl_xor_sync(0xffffffffu, v, o);
-    v = is_max ? fmax(v, y) : v + y;
-  }
-  if (lane == 0) red[wid] = v;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double r = red[0];
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = is_max ? fmax(r, red[w]) : r + red[w];
-    red[32] = r;
-  }
-  __syncthreads();
-  double r = red[32];
-  __syncthreads();
-  return r;
-}
-
-__global__ void __launch_bounds__(kSortThreads) select_kernel(const double* __restrict__ scores,
-                                                              int8_t* __restrict__ mask_out,
-                                                              int32_t* __restrict__ sel, int H,
-                                                              int group, int nb, int top_n,
-                                                              int pmax) {
+__global__ void select_kernel(const double* __restrict__ scores, int8_t* __restrict__ mask_out,
+                              int32_t* __restrict__ sel, int H, int group, int nb, int top_n,
+                              int rows, int n_rows) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int i = blockIdx.x;
-  const int bkv = blockIdx.y;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * rows + w;  // over B*H_kv*nb
+  if (w >= rows || row >= n_rows) return;
+  const int bkv = row / nb, i = row % nb;
   const int Hkv = H / group;
   const int b = bkv / Hkv, hk = bkv % Hkv;
-  int P = 1;
-  while (P < i) P <<= 1;
-  double* prob = reinterpret_cast<double*>(smem);
-  // prob: nb doubles; key: pmax (a power of two >= nb) keys; idx: pmax indices
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem + (size_t)nb * 8);
-  uint16_t* idx = reinterpret_cast<uint16_t*>(smem + (size_t)nb * 8 + (size_t)pmax * 8);
-  __shared__ double red[33];
-  __shared__ int chosen[64 + 1];
-  for (int j = threadIdx.x; j < i; j += blockDim.x) prob[j] = 0.0;
-  __syncthreads();
+  unsigned char* base = smem + (size_t)w * ((size_t)nb * 8 + align_up((size_t)nb, 16) + 1024);
+  double* prob = reinterpret_cast<double*>(base);  // becomes the keys
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(base);
+  uint8_t* flags = base + (size_t)nb * 8;
+  unsigned* hist = reinterpret_cast<unsigned*>(base + (size_t)nb * 8 + align_up((size_t)nb, 16));
+  for (int j = lane; j < i; j += 32) {
+    prob[j] = 0.0;
+    flags[j] = 0;
+  }
+  __syncwarp();
   for (int g = 0; g < group && i > 0; ++g) {
-    const int h = hk * group + g;
-    const double* row = scores + (((size_t)b * H + h) * nb + i) * nb;
+    const double* srow = scores + (((size_t)b * H + hk * group + g) * nb + i) * nb;
     double m = -INFINITY;
-    for (int j = threadIdx.x; j < i; j += blockDim.x) m = fmax(m, row[j]);
-    m = block_reduce(m, true, red);
+    for (int j = lane; j < i; j += 32) m = fmax(m, srow[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
     double sum = 0.0;
-    for (int j = threadIdx.x; j < i; j += blockDim.x) sum += exp(row[j] - m);
-    sum = block_reduce(sum, false, red);
+    for (int j = lane; j < i; j += 32) sum += exp(srow[j] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const double inv = 1.0 / sum;
-    for (int j = threadIdx.x; j < i; j += blockDim.x) prob[j] += exp(row[j] - m) * inv;
-    __syncthreads();
+    for (int j = lane; j < i; j += 32) prob[j] += exp(srow[j] - m) * inv;
+    __syncwarp();
   }
+  for (int j = lane; j < i; j += 32) keys[j] = order_key(prob[j]);
+  __syncwarp();
   const int n = i < top_n ? i : top_n;
-  if (i > 0) {
-    for (int j = threadIdx.x; j < P; j += blockDim.x) {
-      key[j] = j < i ? order_key(prob[j]) : 0ull;
-      idx[j] = (uint16_t)(j < i ? j : 0xFFFF);
-    }
-    __syncthreads();
-    bitonic_sort(key, idx, P);
-  }
-  // ascending order of the chosen blocks: count how many chosen indices are smaller
-  if (threadIdx.x < n) {
-    const int me = idx[threadIdx.x];
-    int r = 0;
-    for (int u = 0; u < n; ++u) r += idx[u] < me;
-    chosen[r] = me;
-  }
-  __syncthreads();
+  warp_mark_top(keys, i, n, hist, flags, 1);
   const size_t rowid = (size_t)bkv * nb + i;
-  for (int u = threadIdx.x; u < top_n; u += blockDim.x) sel[rowid * top_n + u] = u < n ? chosen[u] : -1;
-  if (mask_out) {
-    for (int j = threadIdx.x; j < nb; j += blockDim.x) mask_out[rowid * nb + j] = 0;
-    __syncthreads();
-    if (threadIdx.x < n) mask_out[rowid * nb + chosen[threadIdx.x]] = 2;
+  int32_t* lst = sel + rowid * top_n;
+  if (top_n > 0) {
+    warp_compact(flags, i, 1, 1, lst);
+    for (int u = n + lane; u < top_n; u += 32) lst[u] = -1;
   }
+  if (mask_out)
+    for (int j = lane; j < nb; j += 32) mask_out[rowid * nb + j] = (j < i && (flags[j] & 1)) ? 2 : 0;
 }
 
 cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s) {
   const sla_config& c = p.c;
   const double* sc = reinterpret_cast<const double*>(a.ws + p.off_scores);
-  // the sort arrays hold a power of two >= i < nkb elements
-  const int P = pow2_at_least(p.nkb);
-  const size_t use = (size_t)p.nkb * 8 + (size_t)P * 10 + 16;
+  const int rows = route_rows_per_cta(p.nkb);
+  const size_t smem = route_smem(p.nkb, rows);
   cudaError_t e =
-      cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)use);
+      cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nqb, c.B * c.H_kv);
-  select_kernel<<<grid, kSortThreads, use, s>>>(sc, a.mask_out, a.crit, c.H, p.group, p.nkb,
-                                                c.top_n, P);
+  const int n_rows = c.B * c.H_kv * p.nqb;
+  const int grid = (n_rows + rows - 1) / rows;
+  select_kernel<<<grid, rows * 32, smem, s>>>(sc, a.mask_out, a.crit, c.H, p.group, p.nkb,
+                                              c.top_n, rows, n_rows);
   return cudaGetLastError();
 }
 

@@ -65,9 +65,10 @@ bool make_plan(const sla_config* c, Plan* p) {
     if (marginal) {
       p->off_mmask = take(B * H * (size_t)p->nqb_pad * p->nkb_pad * 2);
       p->off_hs = take(B * Hkv * (size_t)p->nkb_pad * p->dd * 2);
-      p->off_ss = take(B * H * nqb * (size_t)p->dd * 4);
+      p->off_ss = take(B * H * nqb * d * d * 2);  // S_i (times W_p), bf16
+      p->off_zs = take(B * H * nqb * d * 4);      // Z_i, fp32
+      p->off_os = take(B * H * (size_t)c->N * d * 2);
     }
-    p->off_os = take(B * H * (size_t)c->N * d * 2);
   } else {
     p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
   }
@@ -91,9 +92,11 @@ static int stages_of(const Plan& p, Stage* out) {
     if (has_marginal(p)) {
       out[n++] = kState;
       out[n++] = kAggregate;
+      out[n++] = kFlash;
+      out[n++] = kEpilogue;
+    } else {
+      out[n++] = kFlash;  // no linear branch: the sparse branch is the output
     }
-    out[n++] = kFlash;
-    out[n++] = kEpilogue;
   } else {
     out[n++] = kSelect;
     out[n++] = kFlash;
@@ -142,7 +145,7 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
     return SLA_ERR_INVALID_ARG;
   const bool threeway = cfg->mode == SLA_MODE_THREEWAY;
   if (threeway && cfg->has_proj && (!w_p || !aligned(w_p, 16))) return SLA_ERR_INVALID_ARG;
-  if (threeway && cfg->has_gate && (!w_g || !aligned(w_g, 4))) return SLA_ERR_INVALID_ARG;
+  if (threeway && cfg->has_gate && (!w_g || !aligned(w_g, 16))) return SLA_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return SLA_ERR_WORKSPACE;
   Stage stages[8];
   const int ns = stages_of(p, stages);

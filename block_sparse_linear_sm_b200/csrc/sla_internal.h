@@ -20,7 +20,7 @@ enum DeviceDetail : int {
   kDetailTimeout = 200,
 };
 
-inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Derived sizes and the workspace carve-up for one configuration.
 struct Plan {
@@ -31,7 +31,7 @@ struct Plan {
   float scale;
   // byte offsets into ws
   size_t off_status, off_qbar, off_kbar, off_scores, off_crit, off_neg, off_mmask, off_hs, off_ss,
-      off_os, total;
+      off_zs, off_os, total;
 };
 
 bool make_plan(const sla_config* c, Plan* p);
