@@ -10,9 +10,8 @@
 // Layout: Hs[bkv][j][0 : d*d] = h_j row-major (times W_p when the layer has a
 // projection: h'_j = phi(K_j)^T V_j W_p), Hs[bkv][j][d*d : d*d+d] = z_j,
 // zero up to dd (a multiple of 128), rows j in [nkb, nkb_pad) zero; bf16.
-// The aggregation is the GEMM S = M . Hs with M the 0/1 marginal mask of each
-// query head (exact in bf16), accumulated in fp32 and stored as S_i (bf16,
-// [bh][i][d*d]) and Z_i (fp32, [bh][i][d]).
+// The aggregation over each query block's marginal blocks is a tcgen05 GEMM
+// (aggregate_tc.cu).
 #include "common.cuh"
 
 namespace sla {
@@ -164,129 +163,6 @@ cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s) {
     const int smem = 2 * kBlock * 128 + (wp ? 64 * 128 : 0);
     state_kernel<64><<<grid, 128, smem, s>>>(a.k, a.v, wp, hs, c.N, c.N_valid, p.nkb, p.dd);
   }
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// aggregation GEMM: Ss[bh] (nqb x dd, fp32) = M[bh] (nqb_pad x nkb_pad) . Hs[bkv]
-// 128x128 tile per CTA, K steps of 64, 3-stage cp.async pipeline, 8 warps as
-// 2 (rows) x 4 (columns), warp tile 64 x 32.
-// ---------------------------------------------------------------------------
-constexpr int kAggM = 128, kAggN = 128, kAggK = 64, kAggStages = 3;
-constexpr int kAggABytes = kAggM * kAggK * 2;  // 16 KB, rows of 128 B
-constexpr int kAggBBytes = kAggK * kAggN * 2;  // 16 KB, rows of 256 B
-constexpr int kAggSmem = kAggStages * (kAggABytes + kAggBBytes);
-
-__global__ void __launch_bounds__(256) aggregate_kernel(const __nv_bfloat16* __restrict__ mmask,
-                                                        const __nv_bfloat16* __restrict__ hs,
-                                                        __nv_bfloat16* __restrict__ ss,
-                                                        float* __restrict__ zs, int H, int group,
-                                                        int nqb, int nqb_pad, int nkb_pad, int dd,
-                                                        int d) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int n0 = blockIdx.x * kAggN;
-  const int m0 = blockIdx.y * kAggM;
-  const int bh = blockIdx.z;
-  const int b = bh / H, h = bh % H;
-  const int bkv = b * (H / group) + h / group;
-  const __nv_bfloat16* A = mmask + (size_t)bh * nqb_pad * nkb_pad;
-  const __nv_bfloat16* Bm = hs + (size_t)bkv * nkb_pad * dd;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int wm = w >> 2, wn = w & 3;
-  const uint32_t sbase = smem_u32(smem);
-
-  auto load_stage = [&](int st, int k0) {
-    const uint32_t a_s = sbase + st * (kAggABytes + kAggBBytes);
-    const uint32_t b_s = a_s + kAggABytes;
-    // A: 128 rows x 8 chunks
-    for (int e = tid; e < kAggM * 8; e += 256) {
-      const int r = e >> 3, ch = e & 7;
-      cp_async16(a_s + swz(r, ch, 128), A + (size_t)(m0 + r) * nkb_pad + k0 + ch * 8, 16);
-    }
-    // B: 64 rows x 16 chunks
-    for (int e = tid; e < kAggK * 16; e += 256) {
-      const int r = e >> 4, ch = e & 15;
-      cp_async16(b_s + swz(r, ch, 256), Bm + (size_t)(k0 + r) * dd + n0 + ch * 8, 16);
-    }
-  };
-
-  float acc[4][4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
-
-  const int nk = nkb_pad / kAggK;
-#pragma unroll
-  for (int st = 0; st < kAggStages - 1; ++st) {
-    if (st < nk) load_stage(st, st * kAggK);
-    cp_async_commit();
-  }
-  for (int kt = 0; kt < nk; ++kt) {
-    cp_async_wait<kAggStages - 2>();
-    __syncthreads();
-    const int nxt = kt + kAggStages - 1;
-    if (nxt < nk) load_stage(nxt % kAggStages, nxt * kAggK);
-    cp_async_commit();
-    const int st = kt % kAggStages;
-    const uint32_t a_s = sbase + st * (kAggABytes + kAggBBytes);
-    const uint32_t b_s = a_s + kAggABytes;
-#pragma unroll
-    for (int ks = 0; ks < kAggK / 16; ++ks) {
-      uint32_t af[4][4];
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-        ldsm_x4(lds_a(a_s, wm * 64 + mt * 16, 2 * ks, 128, lane), af[mt][0], af[mt][1], af[mt][2],
-                af[mt][3]);
-#pragma unroll
-      for (int n2 = 0; n2 < 2; ++n2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(lds_b_kn(b_s, ks * 16, (wn * 32 + n2 * 16) / 8, 256, lane), b0, b1, b2, b3);
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-          mma_bf16(acc[mt][2 * n2], af[mt], b0, b1);
-          mma_bf16(acc[mt][2 * n2 + 1], af[mt], b2, b3);
-        }
-      }
-    }
-  }
-  cp_async_wait<0>();
-  // columns < d*d: S_i in bf16; the next d columns: Z_i in fp32; the rest is padding
-  const int dsq = d * d;
-  __nv_bfloat16* S = ss + (size_t)bh * nqb * dsq;
-  float* Z = zs + (size_t)bh * nqb * d;
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    const int r = m0 + wm * 64 + mt * 16 + (lane >> 2);
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int col = n0 + wn * 32 + nt * 8 + 2 * (lane & 3);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int rr = r + 8 * hh;
-        if (rr >= nqb) continue;
-        const float v0 = acc[mt][nt][2 * hh], v1 = acc[mt][nt][2 * hh + 1];
-        if (col < dsq)
-          *reinterpret_cast<uint32_t*>(S + (size_t)rr * dsq + col) = pack_bf16(v0, v1);
-        else if (col < dsq + d)
-          *reinterpret_cast<float2*>(Z + (size_t)rr * d + (col - dsq)) = make_float2(v0, v1);
-      }
-    }
-  }
-}
-
-cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
-  const sla_config& c = p.c;
-  const __nv_bfloat16* mm = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_mmask);
-  const __nv_bfloat16* hs = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_hs);
-  __nv_bfloat16* ss = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_ss);
-  float* zs = reinterpret_cast<float*>(a.ws + p.off_zs);
-  cudaError_t e = cudaFuncSetAttribute(aggregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kAggSmem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(p.dd / kAggN, p.nqb_pad / kAggM, c.B * c.H);
-  aggregate_kernel<<<grid, 256, kAggSmem, s>>>(mm, hs, ss, zs, c.H, p.group, p.nqb, p.nqb_pad,
-                                               p.nkb_pad, p.dd, c.d);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
 // Internal host-side interface between the C ABI (sla_api.cu) and the kernels.
 #pragma once
+#include <cuda.h>  // CUtensorMap (type only)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -50,6 +51,12 @@ struct Args {
   char* ws;
   int* status;
 };
+
+// 3D bf16 TMA tensor map [d2][d1][d0] (d0 innermost) with byte strides s1, s2,
+// box (b0, b1, 1) and 128-byte swizzle; out-of-range elements read as zero.
+// Defined in tmap.cu; false if the driver entry point or the encode fails.
+bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1);
 
 // kernel launchers (return the launch error)
 cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s);
