@@ -1,0 +1,276 @@
+// Per-key-block linear states on the 5th-generation tensor cores.
+//
+// SLA analysis page (arXiv 2509.24006), comparison table and core-innovation
+// paragraph: marginal blocks go through linear attention at O(N d^2). With
+// phi = elu + 1 the branch factorises per key block j into the d x d state
+// h_j = phi(K_j)^T V_j and the normaliser z_j = sum_t phi(k_t). With a
+// projection, W_p is folded in: O_l W_p = phi(q) sum_j phi(K_j)^T (V_j W_p) / den,
+// so the kernel stores h'_j = phi(K_j)^T T_j with T_j = V_j W_p.
+//
+// One CTA per pair of key blocks (128 tokens) of one KV head:
+//   1. TMA: K and V (128 tokens x d) and W_p into 128-byte-swizzled tiles.
+//   2. T = V W_p on tcgen05 (M = 128 tokens, N = d, K = d) into TMEM.
+//   3. Four worker warps (one token row each): phi(K) in place (padding tokens
+//      zero), z_j by column sums, T back to shared memory as bf16 in the same
+//      N-major layout V had.
+//   4. h'_j = phi(K_j)^T T_j for both blocks (M = d, N = d, K = 64 tokens),
+//      phi(K) read M-major straight from the K tile, into TMEM.
+//   5. Workers: h'_j rows (one feature row per thread) to bf16 in HBM.
+// Layout: Hs[bkv][j][0 : d*d] = h'_j row-major, [d*d : d*d+d] = z_j, zero up to
+// dd (a multiple of 128); rows j in [nkb, nkb_pad) zero.
+// For d = 64 the state product still uses M = 128: the second feature panel
+// of K is read beyond the tensor and filled with zeros.
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace sla {
+
+constexpr int kStThreads = 192;
+
+template <int D>
+struct StLayout {
+  static constexpr int NP = D / 64;                    // 64-column panels of V, T, W_p
+  static constexpr int kKBytes = 2 * 128 * 128;        // K: two feature panels x 128 tokens
+  static constexpr int kVBytes = NP * 128 * 128;       // V, then T
+  static constexpr int kWBytes = NP * D * 128;         // W_p: N-major panels of D rows
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKBytes;
+  static constexpr int kOffW = kOffV + kVBytes;
+  static constexpr int kOffBar = kOffW + kWBytes;
+  static constexpr int kSmem = kOffBar + 128;
+};
+
+struct StateParams {
+  __nv_bfloat16* hs;
+  int* status;
+  int nkb, nkb_pad, dd, n_valid, has_proj;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kStThreads, 2)
+    state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmW, StateParams prm) {
+  using L = StLayout<D>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (sbase & 1023u) {
+    if (tid == 0) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashAlign);
+    return;
+  }
+  const int j0 = 2 * blockIdx.x, bkv = blockIdx.y;
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffBar + 64);  // tmem, abort
+  auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
+  constexpr int LOADED = 0, T_DONE_MMA = 1, PHI_READY = 2, T_READY = 3, H_DONE = 4;
+  const bool proj = prm.has_proj != 0;
+  if (tid == 0) {
+    misc[1] = 0;
+    tc::mbar_init(bar(LOADED), 1);
+    tc::mbar_init(bar(T_DONE_MMA), 1);
+    tc::mbar_init(bar(PHI_READY), 4);
+    tc::mbar_init(bar(T_READY), 4);
+    tc::mbar_init(bar(H_DONE), 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(sbase + L::kOffBar + 64, 256);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = (uint32_t)misc[0];
+  volatile int* abort = misc + 1;
+  const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sW = sbase + L::kOffW;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::mbar_expect_tx(bar(LOADED), L::kKBytes + L::kVBytes + (proj ? L::kWBytes : 0));
+      for (int p = 0; p < 2; ++p) tc::tma_load_3d(sK + p * 16384, &tmK, bar(LOADED), 64 * p, j0 * kBlock, bkv);
+      for (int p = 0; p < L::NP; ++p)
+        tc::tma_load_3d(sV + p * 16384, &tmV, bar(LOADED), 64 * p, j0 * kBlock, bkv);
+      if (proj)
+        for (int p = 0; p < L::NP; ++p) tc::tma_load_3d(sW + p * D * 128, &tmW, bar(LOADED), 64 * p, 0, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = tc::mbar_wait(bar(LOADED), 0, abort);
+      tc::fence_after_sync();
+      if (ok && proj) {
+        // T = V W_p: A = V (K-major over features), B = W_p (N-major)
+        constexpr uint32_t kId1 = tc::idesc_bf16(128, D, false, true);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t da = tc::sw128_desc(sV + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+          const uint64_t db = tc::sw128_desc(sW + k * 2048, D * 128, 1024);
+          tc::mma_bf16_ss(tmem, da, db, kId1, k > 0);
+        }
+        tc::mma_commit(bar(T_DONE_MMA));
+      }
+      if (ok) ok = tc::mbar_wait(bar(PHI_READY), 0, abort);
+      if (ok && proj) ok = tc::mbar_wait(bar(T_READY), 0, abort);
+      tc::fence_after_sync();
+      if (ok) {
+        // h'_j = phi(K_j)^T T_j: A = phi(K) M-major (features contiguous), B = T N-major
+        constexpr uint32_t kId2 = tc::idesc_bf16(128, D, true, true);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t row_off = (uint32_t)(64 * jj + 16 * kk) * 128;
+            const uint64_t da = tc::sw128_desc(sK + row_off, 16384, 1024);
+            const uint64_t db = tc::sw128_desc(sV + row_off, 16384, 1024);
+            tc::mma_bf16_ss(tmem + jj * D, da, db, kId2, kk > 0);
+          }
+        tc::mma_commit(bar(H_DONE));
+      } else {
+        *abort = 1;
+        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+      }
+    }
+  } else {
+    // ---- workers: 128 threads, thread r = token row r of the pair / feature row r
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    bool ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED), 0, abort));
+    const int tok = j0 * kBlock + r;
+    const bool valid_tok = tok < prm.n_valid;
+    if (ok) {
+      // phi(K) in place on this token's row (only the D real feature columns)
+      for (int p = 0; p < L::NP; ++p)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          unsigned char* ptr = smem + L::kOffK + p * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
+          uint4 u = *reinterpret_cast<uint4*>(ptr);
+          uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float2 f = unpack_bf16(w[x]);
+            w[x] = valid_tok ? pack_bf16(phi(f.x), phi(f.y)) : 0u;
+          }
+          *reinterpret_cast<uint4*>(ptr) = u;
+        }
+      tc::fence_async_smem();
+    }
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(bar(PHI_READY));
+    if (ok && proj) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(T_DONE_MMA), 0, abort));
+      tc::fence_after_sync();
+      if (ok) {
+        // T row r (fp32, TMEM) -> bf16 into the V tile (same N-major layout)
+#pragma unroll
+        for (int c32 = 0; c32 < D / 32; ++c32) {
+          uint32_t v[32];
+          tc::tmem_ld32(tmem + lane_off + 32 * c32, v);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = 32 * c32 + 8 * q;  // 8 columns = one 16-byte chunk
+            const int p = col >> 6, ch = (col & 63) >> 3;
+            const uint4 u = make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                                       pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                                       pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                                       pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+            *reinterpret_cast<uint4*>(smem + L::kOffV + p * 16384 + r * 128 + ((ch ^ (r & 7)) << 4)) = u;
+          }
+        }
+        tc::fence_async_smem();
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(T_READY));
+    }
+    // z_j: column sums of phi(K) over each block's 64 tokens (all rows written above)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok && r < D) {
+      const int p = r >> 6, ch = (r & 63) >> 3, e = r & 7;
+      for (int jj = 0; jj < 2; ++jj) {
+        const int j = j0 + jj;
+        if (j >= prm.nkb) continue;
+        float z = 0.f;
+        for (int t = 64 * jj; t < 64 * jj + 64; ++t) {
+          const __nv_bfloat16* ptr = reinterpret_cast<const __nv_bfloat16*>(
+              smem + L::kOffK + p * 16384 + t * 128 + ((ch ^ (t & 7)) << 4)) + e;
+          z += __bfloat162float(*ptr);
+        }
+        prm.hs[((size_t)bkv * prm.nkb_pad + j) * prm.dd + D * D + r] = __float2bfloat16(z);
+      }
+    }
+    // h'_j rows -> HBM; rows past the last key block are zero
+    ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(H_DONE), 0, abort));
+    tc::fence_after_sync();
+    for (int jj = 0; jj < 2; ++jj) {
+      const int j = j0 + jj;
+      __nv_bfloat16* row = prm.hs + ((size_t)bkv * prm.nkb_pad + j) * prm.dd;
+      if (j >= prm.nkb) {
+        for (int e = r; e < prm.dd / 8; e += 128) reinterpret_cast<uint4*>(row)[e] = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      for (int e = D * D + D + r; e < prm.dd; e += 128) row[e] = __float2bfloat16(0.f);
+      if (!ok) continue;
+#pragma unroll
+      for (int c32 = 0; c32 < D / 32; ++c32) {
+        uint32_t v[32];
+        tc::tmem_ld32(tmem + lane_off + jj * D + 32 * c32, v);
+        tc::tmem_ld_wait();
+        if (r < D) {
+          uint4* dst = reinterpret_cast<uint4*>(row + (size_t)r * D + 32 * c32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                                pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                                pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                                pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+        }
+      }
+    }
+    if (!ok) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int D>
+static cudaError_t launch_state_t(const Plan& p, const Args& a, cudaStream_t s) {
+  using L = StLayout<D>;
+  const sla_config& c = p.c;
+  CUtensorMap mk, mv, mw;
+  const uint64_t rowb = (uint64_t)D * 2, headb = (uint64_t)c.N * D * 2;
+  if (!make_tmap_3d(&mk, a.k, D, (uint64_t)c.N_valid, (uint64_t)c.B * c.H_kv, rowb, headb, 64, 128) ||
+      !make_tmap_3d(&mv, a.v, D, (uint64_t)c.N_valid, (uint64_t)c.B * c.H_kv, rowb, headb, 64, 128))
+    return cudaErrorInvalidValue;
+  const bool proj = c.has_proj && a.w_p;
+  // without a projection the W_p map is never used; encode it over K to keep it valid
+  if (!make_tmap_3d(&mw, proj ? (const void*)a.w_p : (const void*)a.k, D, D, 1, rowb, (uint64_t)D * rowb,
+                    64, D))
+    return cudaErrorInvalidValue;
+  StateParams prm;
+  prm.hs = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_hs);
+  prm.status = a.status;
+  prm.nkb = p.nkb;
+  prm.nkb_pad = p.nkb_pad;
+  prm.dd = p.dd;
+  prm.n_valid = c.N_valid;
+  prm.has_proj = proj ? 1 : 0;
+  cudaError_t e = cudaFuncSetAttribute(state_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       L::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.nkb_pad / 2, c.B * c.H_kv);
+  state_tc_kernel<D><<<grid, kStThreads, L::kSmem, s>>>(mk, mv, mw, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s) {
+  return p.c.d == 128 ? launch_state_t<128>(p, a, s) : launch_state_t<64>(p, a, s);
+}
+
+}  // namespace sla
