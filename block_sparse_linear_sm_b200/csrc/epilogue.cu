@@ -10,9 +10,10 @@
 // projection costs no separate product here. Without a gate g = 1.
 //
 // One CTA per (b, h, query block): 4 warps of 16 rows. phi(q) (bf16) and S'_i
-// (bf16) are staged in shared memory with cp.async; the product runs on
-// mma.sync with fp32 accumulation. About 49 KB of shared memory, so four CTAs
-// share an SM and keep enough loads in flight for this HBM-bound step.
+// (bf16) and O_s are staged in shared memory with cp.async (all loads in flight
+// together); the product runs on mma.sync with fp32 accumulation; O is formed
+// in the O_s tile and written with 16-byte stores. About 65 KB of shared
+// memory, three CTAs per SM.
 #include "common.cuh"
 
 namespace sla {
@@ -33,7 +34,8 @@ __global__ void __launch_bounds__(128) epilogue_kernel(EpiParams prm) {
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* fq_s = smem;                      // [64][D]  q, then phi(q)
   unsigned char* s_s = fq_s + kBlock * RB;         // [D][D]   S'_i
-  float* z_s = reinterpret_cast<float*>(s_s + D * RB);  // [D]
+  unsigned char* o_s = s_s + D * RB;               // [64][D]  O_s, then O
+  float* z_s = reinterpret_cast<float*>(o_s + kBlock * RB);  // [D]
   float* den_s = z_s + D;                               // [64]
   float* g_s = den_s + kBlock;                          // [64]
 
@@ -44,9 +46,10 @@ __global__ void __launch_bounds__(128) epilogue_kernel(EpiParams prm) {
   const __nv_bfloat16* qg = prm.q + ((size_t)bh * prm.N + (size_t)i * kBlock) * D;
   const __nv_bfloat16* sg = prm.ss + ((size_t)bh * prm.nb + i) * D * D;
   const float* zg = prm.zs + ((size_t)bh * prm.nb + i) * D;
-  const uint32_t fq_b = smem_u32(fq_s), s_b = smem_u32(s_s), z_b = smem_u32(z_s);
+  const uint32_t fq_b = smem_u32(fq_s), s_b = smem_u32(s_s), z_b = smem_u32(z_s), o_b = smem_u32(o_s);
+  const __nv_bfloat16* osg = prm.os + ((size_t)bh * prm.N + (size_t)i * kBlock) * D;
 
-  // all loads in flight at once: S'_i, the query rows (padding rows zero), Z_i
+  // all loads in flight at once: S'_i, the query rows (padding rows zero), O_s, Z_i
   for (int e = tid; e < D * CH; e += 128) {
     const int r = e / CH, ch = e % CH;
     cp_async16(s_b + swz(r, ch, RB), sg + (size_t)r * D + ch * 8, 16);
@@ -55,6 +58,10 @@ __global__ void __launch_bounds__(128) epilogue_kernel(EpiParams prm) {
     const int t = e / CH, ch = e % CH;
     const int bytes = t < nvq ? 16 : 0;
     cp_async16(fq_b + swz(t, ch, RB), qg + (bytes ? (size_t)t * D + ch * 8 : 0), bytes);
+  }
+  for (int e = tid; e < kBlock * CH; e += 128) {
+    const int t = e / CH, ch = e % CH;
+    cp_async16(o_b + swz(t, ch, RB), osg + (size_t)t * D + ch * 8, 16);
   }
   for (int e = tid; e < D / 4; e += 128) cp_async16(z_b + e * 16, zg + e * 4, 16);
   cp_async_commit();
@@ -123,18 +130,23 @@ __global__ void __launch_bounds__(128) epilogue_kernel(EpiParams prm) {
   const float d0 = den_s[row0], d1 = den_s[row0 + 8];
   const float c0 = d0 > 0.f ? g_s[row0] / d0 : 0.f, c1 = d1 > 0.f ? g_s[row0 + 8] / d1 : 0.f;
   const bool v0 = row0 < nvq, v1 = row0 + 8 < nvq;
-  const __nv_bfloat16* osg = prm.os + ((size_t)bh * prm.N + (size_t)i * kBlock) * D;
-  __nv_bfloat16* og = prm.out + ((size_t)bh * prm.N + (size_t)i * kBlock) * D;
+  // O = O_s + c * num in place in the O_s tile (each warp owns its 16 rows) ...
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) {
     const int col = n * 8 + 2 * (lane & 3);
-    const float2 s0 = unpack_bf16(*reinterpret_cast<const uint32_t*>(osg + (size_t)row0 * D + col));
-    const float2 s1 =
-        unpack_bf16(*reinterpret_cast<const uint32_t*>(osg + (size_t)(row0 + 8) * D + col));
-    const uint32_t o0 = v0 ? pack_bf16(s0.x + c0 * num[n][0], s0.y + c0 * num[n][1]) : 0u;
-    const uint32_t o1 = v1 ? pack_bf16(s1.x + c1 * num[n][2], s1.y + c1 * num[n][3]) : 0u;
-    *reinterpret_cast<uint32_t*>(og + (size_t)row0 * D + col) = o0;
-    *reinterpret_cast<uint32_t*>(og + (size_t)(row0 + 8) * D + col) = o1;
+    uint32_t* p0 = reinterpret_cast<uint32_t*>(o_s + swz(row0, col >> 3, RB) + (col & 7) * 2);
+    uint32_t* p1 = reinterpret_cast<uint32_t*>(o_s + swz(row0 + 8, col >> 3, RB) + (col & 7) * 2);
+    const float2 s0 = unpack_bf16(*p0), s1 = unpack_bf16(*p1);
+    *p0 = v0 ? pack_bf16(s0.x + c0 * num[n][0], s0.y + c0 * num[n][1]) : 0u;
+    *p1 = v1 ? pack_bf16(s1.x + c1 * num[n][2], s1.y + c1 * num[n][3]) : 0u;
+  }
+  __syncwarp();
+  // ... then 16-byte coalesced stores of the warp's rows
+  __nv_bfloat16* og = prm.out + ((size_t)bh * prm.N + (size_t)i * kBlock) * D;
+  for (int e = lane; e < 16 * CH; e += 32) {
+    const int t = 16 * w + e / CH, ch = e % CH;
+    *reinterpret_cast<uint4*>(og + (size_t)t * D + ch * 8) =
+        *reinterpret_cast<const uint4*>(o_s + swz(t, ch, RB));
   }
 }
 
@@ -152,7 +164,7 @@ static cudaError_t launch_epi_t(const Plan& p, const Args& a, cudaStream_t s) {
   prm.N = c.N;
   prm.n_valid = c.N_valid;
   prm.nb = p.nqb;
-  const int smem = kBlock * D * 2 + D * D * 2 + (D + 2 * kBlock) * 4;
+  const int smem = 2 * kBlock * D * 2 + D * D * 2 + (D + 2 * kBlock) * 4;
   cudaError_t e = cudaFuncSetAttribute(epilogue_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        smem);
   if (e != cudaSuccess) return e;

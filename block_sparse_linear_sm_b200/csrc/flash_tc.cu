@@ -30,8 +30,8 @@
 // more than 2^8, so P stays below 256 and O needs no per-tile rescale.
 //
 // Shared memory: Q (128 x D bf16), a ring of four 64-row K/V slots (K and V
-// tiles alternate), the merged block list. Operand tiles use the 128-byte
-// swizzle. Two CTAs fit on one SM (TMEM: 256 columns each).
+// tiles alternate), the merged block list. Operand tiles use the 128-byte swizzle. Two CTAs fit on one SM
+// (TMEM: 256 columns each).
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -61,7 +61,7 @@ struct TcLayout {
   static constexpr int kOffKV = kOffQ + kQBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kSlotBytes;  // 16 mbarriers
   static constexpr int kOffMisc = kOffBar + 16 * 8;      // tmem addr, count, abort
-  static constexpr int kOffBits = kOffMisc + 64;         // 4 bitmaps
+  static constexpr int kOffList = kOffMisc + 64;         // merged block list
   static constexpr int kTmemCols = 256;                  // O: D columns, S: 2 x 64 columns
 };
 
@@ -79,8 +79,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     return;
   }
 
-  uint32_t* words = reinterpret_cast<uint32_t*>(smem + L::kOffBits);  // act0, act1, sel0, sel1
-  uint32_t* mlist = words + 4 * prm.words;                            // merged list
+  // the four block bitmaps (act0, act1, sel0, sel1) only live during set-up, in
+  // the K/V ring before its first load
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + L::kOffKV);
+  uint32_t* mlist = reinterpret_cast<uint32_t*>(smem + L::kOffList);
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] = TMEM base, misc[1] = merged count, misc[2] = abort
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
@@ -496,7 +498,8 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
   prm.list_cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
   if (prm.list_cap < 1) prm.list_cap = 1;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
-  int smem = L::kOffBits + 4 * prm.words * 4 + prm.list_cap * 4;
+  int smem = L::kOffList + prm.list_cap * 4;
+  if (4 * prm.words * 4 > kSlots * L::kSlotBytes) return cudaErrorInvalidValue;  // bitmaps in the ring
   // at most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;
   cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN>,
