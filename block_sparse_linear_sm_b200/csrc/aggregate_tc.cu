@@ -7,12 +7,13 @@
 //
 //   C[i, :] = sum_j M[i, j] * Hs[j, :]     M: 0/1 marginal mask (exact in bf16)
 //
-// with C = [S_i | Z_i] row by row. C is 128 (query blocks) x 128 (state
-// columns) per CTA, K = key blocks in steps of 64; A (the mask, K-major) and
-// B (the states, N-major) are loaded by TMA into a 3-stage ring and multiplied
-// by tcgen05.mma into a TMEM accumulator. The grid runs the query-block tiles
-// of one column tile next to each other, so a tile of states is read from HBM
-// once and from L2 by the other query-block tiles.
+// with C = [S_i | Z_i] row by row. One CTA computes a 256 (query blocks) x 256
+// (state columns) tile as two M = 128 tcgen05 accumulators (all 512 TMEM
+// columns), K = key blocks in steps of 64; A (the mask, K-major) and B (the
+// states, N-major) come by TMA through a 3-stage ring. Large tiles keep the
+// operand re-reads through L2 low: every state tile is read by nqb/256 CTAs,
+// every mask tile by dd/256. The grid runs the query-block tiles of one column
+// tile next to each other so a tile of states comes from HBM once.
 //
 // Warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2-5 = epilogue
 // (S_i columns to bf16, Z_i columns to fp32, padding columns dropped).
@@ -23,8 +24,9 @@ namespace sla {
 
 constexpr int kAgStages = 3;
 constexpr int kAgThreads = 192;
-constexpr int kAgA = 128 * 64 * 2;   // mask tile: 128 rows x 64 k, one 128-byte panel
-constexpr int kAgB = 64 * 128 * 2;   // state tile: 64 k-rows x 128 columns, two panels
+constexpr int kAgBM = 256, kAgBN = 256;
+constexpr int kAgA = kAgBM * 64 * 2;  // mask tile: 256 rows x 64 k, two 128-row boxes
+constexpr int kAgB = 64 * kAgBN * 2;  // state tile: 64 k-rows x 256 columns, four panels
 constexpr int kAgStage = kAgA + kAgB;
 constexpr int kAgOffBar = kAgStages * kAgStage;
 constexpr int kAgSmem = kAgOffBar + 128;
@@ -36,7 +38,7 @@ struct AggParams {
   int H, group, nqb, nk_steps, d;
 };
 
-__global__ void __launch_bounds__(kAgThreads, 2)
+__global__ void __launch_bounds__(kAgThreads, 1)
     aggregate_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         AggParams prm) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -47,7 +49,7 @@ __global__ void __launch_bounds__(kAgThreads, 2)
     return;
   }
   const int mt = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
-  const int m0 = mt * 128, n0 = nt * 128;
+  const int m0 = mt * kAgBM, n0 = nt * kAgBN;
   const int b = bh / prm.H, h = bh % prm.H;
   const int bkv = b * (prm.H / prm.group) + h / prm.group;
   volatile int* misc = reinterpret_cast<volatile int*>(smem + kAgOffBar + 64);  // tmem, abort
@@ -63,7 +65,7 @@ __global__ void __launch_bounds__(kAgThreads, 2)
     tc::fence_mbar_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(sbase + kAgOffBar + 64, 128);
+    tc::tmem_alloc(sbase + kAgOffBar + 64, 512);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -87,8 +89,9 @@ __global__ void __launch_bounds__(kAgThreads, 2)
         const uint32_t a_s = sbase + st * kAgStage, b_s = a_s + kAgA;
         tc::mbar_expect_tx(bar(FULL + st), kAgStage);
         tc::tma_load_3d(a_s, &tmA, bar(FULL + st), k * 64, m0, bh);
-        tc::tma_load_3d(b_s, &tmB, bar(FULL + st), n0, k * 64, bkv);
-        tc::tma_load_3d(b_s + 8192, &tmB, bar(FULL + st), n0 + 64, k * 64, bkv);
+        tc::tma_load_3d(a_s + 16384, &tmA, bar(FULL + st), k * 64, m0 + 128, bh);
+        for (int p = 0; p < 4; ++p)
+          tc::tma_load_3d(b_s + p * 8192, &tmB, bar(FULL + st), n0 + 64 * p, k * 64, bkv);
       }
       // tail: every stage's last release has landed before the CTA exits
       for (int k = (K > kAgStages ? K - kAgStages : 0); k < K && !*abort; ++k)
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(kAgThreads, 2)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kId = tc::idesc_bf16(128, 128, false, true);
+      constexpr uint32_t kId = tc::idesc_bf16(128, kAgBN, false, true);
       bool ok = true;
       for (int k = 0; k < K; ++k) {
         const int st = k % kAgStages;
@@ -111,9 +114,12 @@ __global__ void __launch_bounds__(kAgThreads, 2)
         const uint32_t a_s = sbase + st * kAgStage, b_s = a_s + kAgA;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t da = tc::sw128_desc(a_s + kk * 32, 16, 1024);
           const uint64_t db = tc::sw128_desc(b_s + kk * 2048, 8192, 1024);
-          tc::mma_bf16_ss(tmem, da, db, kId, (k > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int mh = 0; mh < 2; ++mh) {
+            const uint64_t da = tc::sw128_desc(a_s + mh * 16384 + kk * 32, 16, 1024);
+            tc::mma_bf16_ss(tmem + mh * kAgBN, da, db, kId, (k > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         tc::mma_commit(bar(EMPTY + st));
       }
@@ -124,18 +130,18 @@ __global__ void __launch_bounds__(kAgThreads, 2)
       }
     }
   } else {
-    // epilogue: thread = query block (TMEM lane), 128 columns in 4 chunks
+    // epilogue: thread = query block (TMEM lane) of each 128-row half, 256 columns in 8 chunks
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int row = m0 + r;
     const bool ok = __all_sync(0xffffffffu, K > 0 && tc::mbar_wait(bar(DONE), 0, abort));
     tc::fence_after_sync();
     const int dsq = prm.d * prm.d;
-    if (ok) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+    for (int mh = 0; mh < 2 && ok; ++mh) {
+      const int row = m0 + mh * 128 + r;
+#pragma unroll 2
+      for (int c = 0; c < kAgBN / 32; ++c) {
         uint32_t v[32];
-        tc::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + 32 * c, v);
+        tc::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + mh * kAgBN + 32 * c, v);
         tc::tmem_ld_wait();
         const int col = n0 + 32 * c;
         if (row >= prm.nqb) continue;
@@ -160,7 +166,7 @@ __global__ void __launch_bounds__(kAgThreads, 2)
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 128);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -187,7 +193,7 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(aggregate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kAgSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nqb_pad / 128, p.dd / 128, c.B * c.H);
+  dim3 grid((p.nqb_pad + kAgBM - 1) / kAgBM, (p.dd + kAgBN - 1) / kAgBN, c.B * c.H);
   aggregate_tc_kernel<<<grid, kAgThreads, kAgSmem, s>>>(ma, mb, prm);
   return cudaGetLastError();
 }
