@@ -29,8 +29,9 @@
 // The running max only moves (and O is rescaled) when a row's max grows by
 // more than 2^8, so P stays below 256 and O needs no per-tile rescale.
 //
-// Shared memory: Q (128 x D bf16), a ring of four 64-row K/V slots (K and V
-// tiles alternate), the merged block list. Operand tiles use the 128-byte swizzle. Two CTAs fit on one SM
+// Shared memory: Q (128 x D bf16), a ring of three K slots (a K tile is free
+// once S = Q K^T is done) and a ring of two V slots (free after P V), each
+// refilled as soon as a slot frees, and the merged block list. Operand tiles use the 128-byte swizzle. Two CTAs fit on one SM
 // (TMEM: 256 columns each).
 #include "common.cuh"
 #include "tc.cuh"
@@ -50,7 +51,9 @@ struct FlashTcParams {
 };
 
 constexpr int kTcThreads = 192;
-constexpr int kSlots = 4;
+constexpr int kKSlots = 3;  // K tiles: freed as soon as S = Q K^T is done
+constexpr int kVSlots = 2;  // V tiles: freed after P V
+constexpr int kSlots = kKSlots + kVSlots;
 constexpr float kRescaleLog2 = 8.f;
 
 template <int D>
@@ -87,8 +90,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   // misc[0] = TMEM base, misc[1] = merged count, misc[2] = abort
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
   // barrier ids
-  constexpr int Q_FULL = 0, KV_FULL = 1, KV_EMPTY = 1 + kSlots, S_FULL = 1 + 2 * kSlots,
-                P_FULL = S_FULL + 2, O_DONE = P_FULL + 2;
+  // barrier ids: K ring, V ring (full / empty per slot), S and P per TMEM buffer
+  constexpr int Q_FULL = 0, K_FULL = 1, K_EMPTY = K_FULL + kKSlots, V_FULL = K_EMPTY + kKSlots,
+                V_EMPTY = V_FULL + kVSlots, S_FULL = V_EMPTY + kVSlots, P_FULL = S_FULL + 2,
+                O_DONE = P_FULL + 2;
+  static_assert(O_DONE < 16, "barrier area holds 16 mbarriers");
 
   // ---- unit decode ----------------------------------------------------------
   const int Hkv = prm.H / prm.group;
@@ -131,9 +137,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   if (tid == 0) {
     misc[2] = 0;
     tc::mbar_init(bar(Q_FULL), 1);
-    for (int s = 0; s < kSlots; ++s) {
-      tc::mbar_init(bar(KV_FULL + s), 1);
-      tc::mbar_init(bar(KV_EMPTY + s), 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      tc::mbar_init(bar(K_FULL + s), 1);
+      tc::mbar_init(bar(K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      tc::mbar_init(bar(V_FULL + s), 1);
+      tc::mbar_init(bar(V_EMPTY + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(bar(S_FULL + b), 1);
@@ -220,23 +230,50 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         for (int p = 0; p < NP; ++p)
           tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmQ, bar(Q_FULL), 64 * p, i_h[hf] * kBlock,
                           bh_h[hf]);
-      for (int s = 0; s < 2 * T; ++s) {
-        const int n = s >> 1, slot = s % kSlots;
-        if (s >= kSlots && !tc::mbar_wait(bar(KV_EMPTY + slot), ((s / kSlots) - 1) & 1, abort)) {
+      // K and V tiles go to separate rings; each is refilled as soon as a slot frees
+      const uint32_t sKr = sKV, sVr = sKV + kKSlots * L::kSlotBytes;
+      int nk = 0, nv = 0;
+      uint64_t t0 = tc::globaltimer();
+      uint32_t spins = 0;
+      while (nk < T || nv < T) {
+        bool progressed = false;
+        if (nk < T && (nk < kKSlots || tc::mbar_test(bar(K_EMPTY + nk % kKSlots), ((nk / kKSlots) - 1) & 1))) {
+          const int slot = nk % kKSlots, jb = (int)(mlist[nk] & 0xFFFFu);
+          tc::mbar_expect_tx(bar(K_FULL + slot), L::kSlotBytes);
+          for (int p = 0; p < NP; ++p)
+            tc::tma_load_3d(sKr + slot * L::kSlotBytes + p * 8192, &tmK, bar(K_FULL + slot), 64 * p, jb * kBlock, bkv);
+          ++nk;
+          progressed = true;
+        }
+        if (nv < T && nv < nk && (nv < kVSlots || tc::mbar_test(bar(V_EMPTY + nv % kVSlots), ((nv / kVSlots) - 1) & 1))) {
+          const int slot = nv % kVSlots, jb = (int)(mlist[nv] & 0xFFFFu);
+          tc::mbar_expect_tx(bar(V_FULL + slot), L::kSlotBytes);
+          for (int p = 0; p < NP; ++p)
+            tc::tma_load_3d(sVr + slot * L::kSlotBytes + p * 8192, &tmV, bar(V_FULL + slot), 64 * p, jb * kBlock, bkv);
+          ++nv;
+          progressed = true;
+        }
+        if (progressed) {
+          t0 = tc::globaltimer();
+          spins = 0;
+          continue;
+        }
+        __nanosleep(64);  // leave the issue slots to the softmax warp sharing this SMSP
+        if ((++spins & 63u) == 0 && (*abort || tc::globaltimer() - t0 > tc::kTimeoutNs)) {
           *abort = 1;
           report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
           break;
         }
-        const int jb = (int)(mlist[n] & 0xFFFFu);
-        tc::mbar_expect_tx(bar(KV_FULL + slot), L::kSlotBytes);
-        for (int p = 0; p < NP; ++p)
-          tc::tma_load_3d(sKV + slot * L::kSlotBytes + p * 8192, (s & 1) ? &tmV : &tmK,
-                          bar(KV_FULL + slot), 64 * p, jb * kBlock, bkv);
       }
       // tail: wait for the last release of every slot, so that no tcgen05.commit
       // arrival is still in flight when the CTA exits
-      for (int s = (2 * T > kSlots ? 2 * T - kSlots : 0); s < 2 * T && !*abort; ++s)
-        if (!tc::mbar_wait(bar(KV_EMPTY + s % kSlots), (s / kSlots) & 1, abort)) {
+      for (int n = (T > kKSlots ? T - kKSlots : 0); n < nk && !*abort; ++n)
+        if (!tc::mbar_wait(bar(K_EMPTY + n % kKSlots), (n / kKSlots) & 1, abort)) {
+          *abort = 1;
+          report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+        }
+      for (int n = (T > kVSlots ? T - kVSlots : 0); n < nv && !*abort; ++n)
+        if (!tc::mbar_wait(bar(V_EMPTY + n % kVSlots), (n / kVSlots) & 1, abort)) {
           *abort = 1;
           report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
         }
@@ -251,8 +288,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       tc::fence_after_sync();
       // S_n = Q K_n^T into TMEM buffer n & 1
       auto issue_s = [&](int n) -> bool {
-        const int s = 2 * n, slot = s % kSlots;
-        if (!tc::mbar_wait(bar(KV_FULL + slot), (s / kSlots) & 1, abort)) return false;
+        const int slot = n % kKSlots;
+        if (!tc::mbar_wait(bar(K_FULL + slot), (n / kKSlots) & 1, abort)) return false;
         tc::fence_after_sync();
         const uint32_t kb = sKV + slot * L::kSlotBytes;
 #pragma unroll
@@ -262,7 +299,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           tc::mma_bf16_ss(tS0 + 64 * (n & 1), da, db, kIdS, k > 0);
         }
         tc::mma_commit(bar(S_FULL + (n & 1)));
-        tc::mma_commit(bar(KV_EMPTY + slot));
+        tc::mma_commit(bar(K_EMPTY + slot));
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -274,20 +311,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           ok = false;
           break;
         }
-        const int s = 2 * n + 1, slot = s % kSlots;
-        if (!tc::mbar_wait(bar(KV_FULL + slot), (s / kSlots) & 1, abort)) {
+        const int slot = n % kVSlots;
+        if (!tc::mbar_wait(bar(V_FULL + slot), (n / kVSlots) & 1, abort)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t vb = sKV + slot * L::kSlotBytes;
+        const uint32_t vb = sKV + (kKSlots + slot) * L::kSlotBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t db = tc::sw128_desc(vb + kk * 2048, 8192, 1024);
           tc::mma_bf16_ts(tO, tS0 + 64 * b + 8 * kk, db, kIdPV, (n > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(bar(O_DONE));
-        tc::mma_commit(bar(KV_EMPTY + slot));
+        tc::mma_commit(bar(V_EMPTY + slot));
         // buffer b is free once PV_n has read P_n: S_{n+2} is issued behind it
         if (n + 2 < T && !issue_s(n + 2)) {
           ok = false;
@@ -365,21 +402,25 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           }
           m_ref = m_tile;
         }
-        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float psum = 0.f;
         if (m_ref != -INFINITY) {
-          const float neg = -m_ref;
+          const uint64_t sc2 = tc::f2_pack(sl2, sl2), ng2 = tc::f2_pack(-m_ref, -m_ref);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const float p0 = tc::ex2_approx(fmaf(x[j], sl2, neg));
-            const float p1 = tc::ex2_approx(fmaf(x[j + 1], sl2, neg));
-            sm[(j >> 1) & 7] += p0 + p1;
-            pk[j >> 1] = pack_bf16(p0, p1);
+          for (int j = 0; j < 32; ++j) {
+            const uint64_t y = tc::ffma2(tc::f2_pack(x[2 * j], x[2 * j + 1]), sc2, ng2);
+            const float p0 = tc::ex2_approx(tc::f2_lo(y));
+            const float p1 = tc::ex2_approx(tc::f2_hi(y));
+            acc[j & 3] = tc::fadd2(acc[j & 3], tc::f2_pack(p0, p1));
+            pk[j] = pack_bf16(p0, p1);
           }
+          const uint64_t a2 = tc::fadd2(tc::fadd2(acc[0], acc[1]), tc::fadd2(acc[2], acc[3]));
+          psum = tc::f2_lo(a2) + tc::f2_hi(a2);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) pk[j] = 0u;
         }
-        l_sum = l_sum * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+        l_sum = l_sum * alpha + psum;
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = 0u;  // this half does not use the tile
