@@ -176,14 +176,36 @@ def oracle_threads() -> int:
         return 1
 
 
-def sample_units(cfg, n, seed=1234):
+def sample_units(cfg, n, n_heads=2, seed=1234):
     rng = np.random.default_rng(seed)
-    heads = rng.permutation(cfg.H)[:max(1, min(cfg.H, 2))]
+    heads = rng.permutation(cfg.H)[:max(1, min(cfg.H, n_heads))]
     units = []
     for h in heads:
         for i in rng.permutation(cfg.nqb)[:max(1, n // len(heads))]:
             units.append((0, int(h), int(i)))
     return units
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    csrc = os.path.join(ROOT, "block_sparse_linear_sm_b200", "csrc")
+    files = {"flash_tc_kernel": ["flash_tc.cu", "tc.cuh", "common.cuh"]}.get(kernel, [])
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    for e in json.load(open(p)):
+        if e.get("kernel") == kernel and e.get("workload") == workload and \
+                e.get("source_hash") == kernel_source_hash(kernel):
+            return e["dram_bytes_per_launch"]
+    return None
 
 
 def units_total(cfg):
@@ -357,11 +379,14 @@ def main():
             stages[n] = {"ms": stage_ms[n], "bound": "hbm", "achieved": ach, "unit": "GB/s",
                          "frac": ach / peaks["hbm"], "work": work}
     dom = max(names, key=lambda n: stage_ms[n])
+    kernel_of = {"sparse_flash": "flash_tc_kernel"}
     dk = stages[dom]
     if dk["bound"] == "tensor":
         roof = {"kernel": dom, "bound": "tensor", "achieved": dk["achieved"], "peak": peaks["bf16_sus"],
                 "unit": "TFLOP/s", "frac": dk["achieved"] / peaks["bf16_sus"],
-                "peak_kind": f"bf16 sustained, {peaks['src']}", "traffic": None}
+                "peak_kind": f"bf16 sustained, {peaks['src']}",
+                "traffic": measured_traffic(kernel_of.get(dom, dom), cfg.name),
+                "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved"], "peak": peaks["hbm"],
                 "unit": "GB/s", "frac": dk["achieved"] / peaks["hbm"],
@@ -389,12 +414,14 @@ def main():
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        units = sample_units(cfg, 8)
-        t, n = oracle_sample(cfg, x, units, budget_s=30.0)
+        # about 10-30 s of float64 oracle work on the host cores
+        units = sample_units(cfg, 512, n_heads=4)
+        t, n = oracle_sample(cfg, x, units, budget_s=20.0)
         cv = (n / units_total(cfg)) * flops / t / 1e12
         line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                                "sample": f"{n} (head, query block) units of {units_total(cfg)} "
-                                          f"in {t:.1f} s; throughput scaled by unit count"}
+                                "sample": f"{n} (head, query block) units of {units_total(cfg)} from "
+                                          f"4 heads in {t:.1f} s (stops after 20 s); throughput "
+                                          f"scaled by unit count"}
     if dist is not None:
         dist.destroy_process_group()
     if rank == 0:

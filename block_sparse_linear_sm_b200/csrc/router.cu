@@ -54,15 +54,22 @@ cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// pooled scores: s[bh][i][j] = scale * qbar[bh][i] . kbar[bkv][j], float64.
-// 64x64 output tile per CTA, 256 threads with 4x4 outputs each, K chunks of 16.
-// In top-n mode only j < i is ever read, so tiles wholly above the diagonal
-// are skipped.
+// pooled scores: s[bh][i][j] = scale * qbar[bh][i] . kbar[bkv][j], float64,
+// on the FP64 tensor-core path (mma.sync m8n8k4, fp64 in and out; every product
+// and sum is an IEEE double operation). 64 x 64 output tile per CTA, four warps
+// of 32 x 32 (4 x 4 fragments of 8 x 8), K chunks of 16. In top-n mode only
+// j < i is ever read, so tiles wholly above the diagonal are skipped.
 // ---------------------------------------------------------------------------
 constexpr int kSTile = 64;
 constexpr int kSK = 16;
 
-__global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ qbar,
+__device__ __forceinline__ void dmma_8x8x4(double (&c)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(128) scores_kernel(const double* __restrict__ qbar,
                                                      const double* __restrict__ kbar,
                                                      double* __restrict__ scores, int H, int group,
                                                      int nb, int d, double scale, int lower_only) {
@@ -71,44 +78,47 @@ __global__ void __launch_bounds__(256) scores_kernel(const double* __restrict__ 
   const int bkv = b * (H / group) + h / group;
   const int i0 = blockIdx.y * kSTile, j0 = blockIdx.x * kSTile;
   if (lower_only && j0 > i0 + kSTile - 1) return;
-  __shared__ double As[kSK][kSTile + 1];
-  __shared__ double Bs[kSK][kSTile + 1];
+  // [row][k], rows padded to 20 doubles: a fragment read takes the minimum two wavefronts
+  __shared__ double As[kSTile][kSK + 4];
+  __shared__ double Bs[kSTile][kSK + 4];
   const double* A = qbar + (size_t)bh * nb * d;
   const double* Bm = kbar + (size_t)bkv * nb * d;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  double acc[4][4] = {};
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int wi = (w >> 1) * 32, wj = (w & 1) * 32;  // warp tile origin
+  double acc[4][4][2] = {};
   for (int k0 = 0; k0 < d; k0 += kSK) {
-    for (int e = threadIdx.x; e < kSTile * kSK; e += 256) {
+    for (int e = tid; e < kSTile * kSK; e += 128) {
       const int r = e / kSK, kk = e % kSK;
       const int ia = i0 + r, jb = j0 + r;
-      As[kk][r] = ia < nb ? A[(size_t)ia * d + k0 + kk] : 0.0;
-      Bs[kk][r] = jb < nb ? Bm[(size_t)jb * d + k0 + kk] : 0.0;
+      As[r][kk] = ia < nb ? A[(size_t)ia * d + k0 + kk] : 0.0;
+      Bs[r][kk] = jb < nb ? Bm[(size_t)jb * d + k0 + kk] : 0.0;
     }
     __syncthreads();
 #pragma unroll
-    for (int kk = 0; kk < kSK; ++kk) {
-      double av[4], bv[4];
+    for (int k4 = 0; k4 < kSK; k4 += 4) {
+      double af[4], bf[4];
+      // A fragment: row lane/4, column lane%4; B fragment: row (k) lane%4, column lane/4
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        av[u] = As[kk][ty + 16 * u];
-        bv[u] = Bs[kk][tx + 16 * u];
-      }
+      for (int m = 0; m < 4; ++m) af[m] = As[wi + 8 * m + (lane >> 2)][k4 + (lane & 3)];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int n = 0; n < 4; ++n) bf[n] = Bs[wj + 8 * n + (lane >> 2)][k4 + (lane & 3)];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = fma(av[u], bv[w], acc[u][w]);
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) dmma_8x8x4(acc[m][n], af[m], bf[n]);
     }
     __syncthreads();
   }
   double* S = scores + (size_t)bh * nb * nb;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = i0 + ty + 16 * u;
+  for (int m = 0; m < 4; ++m) {
+    const int i = i0 + wi + 8 * m + (lane >> 2);
     if (i >= nb) continue;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int j = j0 + tx + 16 * w;
-      if (j < nb) S[(size_t)i * nb + j] = acc[u][w] * scale;
+    for (int n = 0; n < 4; ++n) {
+      const int j = j0 + wj + 8 * n + 2 * (lane & 3);
+      if (j < nb) S[(size_t)i * nb + j] = acc[m][n][0] * scale;
+      if (j + 1 < nb) S[(size_t)i * nb + j + 1] = acc[m][n][1] * scale;
     }
   }
 }
@@ -120,7 +130,7 @@ cudaError_t launch_scores(const Plan& p, const Args& a, cudaStream_t s) {
   double* sc = reinterpret_cast<double*>(a.ws + p.off_scores);
   const int t = (p.nqb + kSTile - 1) / kSTile;
   dim3 grid(t, t, c.B * c.H);
-  scores_kernel<<<grid, 256, 0, s>>>(qbar, kbar, sc, c.H, p.group, p.nqb, c.d, (double)p.scale,
+  scores_kernel<<<grid, 128, 0, s>>>(qbar, kbar, sc, c.H, p.group, p.nqb, c.d, (double)p.scale,
                                      c.mode == SLA_MODE_TOPN_WINDOW);
   return cudaGetLastError();
 }
