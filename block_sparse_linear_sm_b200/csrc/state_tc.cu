@@ -10,12 +10,14 @@
 // One CTA per pair of key blocks (128 tokens) of one KV head:
 //   1. TMA: K and V (128 tokens x d) and W_p into 128-byte-swizzled tiles.
 //   2. T = V W_p on tcgen05 (M = 128 tokens, N = d, K = d) into TMEM.
-//   3. Four worker warps (one token row each): phi(K) in place (padding tokens
-//      zero), z_j by column sums, T back to shared memory as bf16 in the same
-//      N-major layout V had.
+//   3. Eight worker warps (two per TMEM lane quarter; thread = token row, the
+//      two warps of a quarter split the columns): phi(K) in place (padding
+//      tokens zero), T back to shared memory as bf16 in the N-major layout V
+//      had, z_j by column sums (one block per warp half).
 //   4. h'_j = phi(K_j)^T T_j for both blocks (M = d, N = d, K = 64 tokens),
 //      phi(K) read M-major straight from the K tile, into TMEM.
-//   5. Workers: h'_j rows (one feature row per thread) to bf16 in HBM.
+//   5. Workers stage h'_j (thread = feature row) as bf16 in the freed K and V
+//      tiles, 128-byte swizzled, and one thread writes them with TMA stores.
 // Layout: Hs[bkv][j][0 : d*d] = h'_j row-major, [d*d : d*d+d] = z_j, zero up to
 // dd (a multiple of 128); rows j in [nkb, nkb_pad) zero.
 // For d = 64 the state product still uses M = 128: the second feature panel
@@ -25,7 +27,7 @@
 
 namespace sla {
 
-constexpr int kStThreads = 192;
+constexpr int kStThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 workers
 
 template <int D>
 struct StLayout {
@@ -49,7 +51,8 @@ struct StateParams {
 template <int D>
 __global__ void __launch_bounds__(kStThreads, 2)
     state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                    const __grid_constant__ CUtensorMap tmW, StateParams prm) {
+                    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmH,
+                    StateParams prm) {
   using L = StLayout<D>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -62,13 +65,14 @@ __global__ void __launch_bounds__(kStThreads, 2)
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffBar + 64);  // tmem, abort
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
   constexpr int LOADED = 0, T_DONE_MMA = 1, PHI_READY = 2, T_READY = 3, H_DONE = 4;
+  constexpr int kWorkerWarps = 8;
   const bool proj = prm.has_proj != 0;
   if (tid == 0) {
     misc[1] = 0;
     tc::mbar_init(bar(LOADED), 1);
     tc::mbar_init(bar(T_DONE_MMA), 1);
-    tc::mbar_init(bar(PHI_READY), 4);
-    tc::mbar_init(bar(T_READY), 4);
+    tc::mbar_init(bar(PHI_READY), kWorkerWarps);
+    tc::mbar_init(bar(T_READY), kWorkerWarps);
     tc::mbar_init(bar(H_DONE), 1);
     tc::fence_mbar_init();
   }
@@ -129,28 +133,33 @@ __global__ void __launch_bounds__(kStThreads, 2)
       }
     }
   } else {
-    // ---- workers: 128 threads, thread r = token row r of the pair / feature row r
+    // ---- workers: warps 2-9; thread r = token row r of the pair / feature row r;
+    // hh = which half of the columns (phi, T) or which block (z, h') this warp takes
     const int quarter = warp & 3;
+    const int hh = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     bool ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED), 0, abort));
     const int tok = j0 * kBlock + r;
     const bool valid_tok = tok < prm.n_valid;
-    if (ok) {
-      // phi(K) in place on this token's row (only the D real feature columns)
-      for (int p = 0; p < L::NP; ++p)
+    if (ok && hh < L::NP) {
+      // phi(K) in place on this token's row, feature panel hh: all 8 chunks are
+      // loaded before any is written back
+      uint4 u[8];
+      uint4* row = reinterpret_cast<uint4*>(smem + L::kOffK + hh * 16384 + r * 128);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          unsigned char* ptr = smem + L::kOffK + p * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
-          uint4 u = *reinterpret_cast<uint4*>(ptr);
-          uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+      for (int c = 0; c < 8; ++c) u[c] = row[c ^ (r & 7)];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const float2 f = unpack_bf16(w[x]);
-            w[x] = valid_tok ? pack_bf16(phi(f.x), phi(f.y)) : 0u;
-          }
-          *reinterpret_cast<uint4*>(ptr) = u;
+      for (int c = 0; c < 8; ++c) {
+        uint32_t* w = reinterpret_cast<uint32_t*>(&u[c]);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const float2 f = unpack_bf16(w[x]);
+          w[x] = valid_tok ? pack_bf16(phi(f.x), phi(f.y)) : 0u;
         }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) row[c ^ (r & 7)] = u[c];
       tc::fence_async_smem();
     }
     __syncwarp();
@@ -158,23 +167,20 @@ __global__ void __launch_bounds__(kStThreads, 2)
     if (ok && proj) {
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(T_DONE_MMA), 0, abort));
       tc::fence_after_sync();
-      if (ok) {
-        // T row r (fp32, TMEM) -> bf16 into the V tile (same N-major layout)
+      if (ok && hh < L::NP) {
+        // T row r, columns 64*hh .. +63 (fp32, TMEM) -> bf16 into the V tile (N-major)
+        uint32_t v[2][32];
+        tc::tmem_ld32(tmem + lane_off + 64 * hh, v[0]);
+        tc::tmem_ld32(tmem + lane_off + 64 * hh + 32, v[1]);
+        tc::tmem_ld_wait();
+        uint4* row = reinterpret_cast<uint4*>(smem + L::kOffV + hh * 16384 + r * 128);
 #pragma unroll
-        for (int c32 = 0; c32 < D / 32; ++c32) {
-          uint32_t v[32];
-          tc::tmem_ld32(tmem + lane_off + 32 * c32, v);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = 32 * c32 + 8 * q;  // 8 columns = one 16-byte chunk
-            const int p = col >> 6, ch = (col & 63) >> 3;
-            const uint4 u = make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                                       pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                                       pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                                       pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-            *reinterpret_cast<uint4*>(smem + L::kOffV + p * 16384 + r * 128 + ((ch ^ (r & 7)) << 4)) = u;
-          }
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t* vv = v[q >> 2] + 8 * (q & 3);
+          row[q ^ (r & 7)] = make_uint4(pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
+                                        pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
+                                        pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
+                                        pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7])));
         }
         tc::fence_async_smem();
       }
@@ -182,49 +188,62 @@ __global__ void __launch_bounds__(kStThreads, 2)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(T_READY));
     }
-    // z_j: column sums of phi(K) over each block's 64 tokens (all rows written above)
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok && r < D) {
+    // z_j for block hh: column sums of phi(K) over its 64 tokens (all rows written above)
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const int j = j0 + hh;
+    if (ok && r < D && j < prm.nkb) {
       const int p = r >> 6, ch = (r & 63) >> 3, e = r & 7;
-      for (int jj = 0; jj < 2; ++jj) {
-        const int j = j0 + jj;
-        if (j >= prm.nkb) continue;
-        float z = 0.f;
-        for (int t = 64 * jj; t < 64 * jj + 64; ++t) {
-          const __nv_bfloat16* ptr = reinterpret_cast<const __nv_bfloat16*>(
-              smem + L::kOffK + p * 16384 + t * 128 + ((ch ^ (t & 7)) << 4)) + e;
-          z += __bfloat162float(*ptr);
-        }
-        prm.hs[((size_t)bkv * prm.nkb_pad + j) * prm.dd + D * D + r] = __float2bfloat16(z);
+      const __nv_bfloat16* col = reinterpret_cast<const __nv_bfloat16*>(smem + L::kOffK + p * 16384) + e;
+      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int t = 0; t < 64; ++t) {
+        const int tt = 64 * hh + t;
+        z[t & 7] += __bfloat162float(col[(tt * 128 + ((ch ^ (tt & 7)) << 4)) / 2]);
       }
+      const float zs = ((z[0] + z[1]) + (z[2] + z[3])) + ((z[4] + z[5]) + (z[6] + z[7]));
+      prm.hs[((size_t)bkv * prm.nkb_pad + j) * prm.dd + D * D + r] = __float2bfloat16(zs);
     }
-    // h'_j rows -> HBM; rows past the last key block are zero
+    __nv_bfloat16* hrow = prm.hs + ((size_t)bkv * prm.nkb_pad + j) * prm.dd;
+    if (j >= prm.nkb) {
+      // rows past the last key block are zero
+      for (int e = r; e < prm.dd / 8; e += 128) reinterpret_cast<uint4*>(hrow)[e] = make_uint4(0, 0, 0, 0);
+    } else {
+      for (int e = D * D + D + r; e < prm.dd; e += 128) hrow[e] = __float2bfloat16(0.f);
+    }
+    // every worker has read K (z) before h' overwrites the K and V tiles
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(H_DONE), 0, abort));
     tc::fence_after_sync();
-    for (int jj = 0; jj < 2; ++jj) {
-      const int j = j0 + jj;
-      __nv_bfloat16* row = prm.hs + ((size_t)bkv * prm.nkb_pad + j) * prm.dd;
-      if (j >= prm.nkb) {
-        for (int e = r; e < prm.dd / 8; e += 128) reinterpret_cast<uint4*>(row)[e] = make_uint4(0, 0, 0, 0);
-        continue;
-      }
-      for (int e = D * D + D + r; e < prm.dd; e += 128) row[e] = __float2bfloat16(0.f);
-      if (!ok) continue;
+    if (ok) {
+      // h'_hh row r (feature c1) -> bf16 staged in the K (block 0) or V (block 1)
+      // tile: two 64-column panels of 128 rows, 128-byte swizzled
+      unsigned char* stage = smem + (hh == 0 ? L::kOffK : L::kOffV);
 #pragma unroll
-      for (int c32 = 0; c32 < D / 32; ++c32) {
-        uint32_t v[32];
-        tc::tmem_ld32(tmem + lane_off + jj * D + 32 * c32, v);
+      for (int c64 = 0; c64 < D / 64; ++c64) {
+        uint32_t v[2][32];
+        tc::tmem_ld32(tmem + lane_off + hh * D + 64 * c64, v[0]);
+        tc::tmem_ld32(tmem + lane_off + hh * D + 64 * c64 + 32, v[1]);
         tc::tmem_ld_wait();
-        if (r < D) {
-          uint4* dst = reinterpret_cast<uint4*>(row + (size_t)r * D + 32 * c32);
+        uint4* row = reinterpret_cast<uint4*>(stage + c64 * 16384 + r * 128);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                                pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                                pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                                pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t* vv = v[q >> 2] + 8 * (q & 3);
+          row[q ^ (r & 7)] = make_uint4(pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
+                                        pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
+                                        pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
+                                        pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7])));
         }
       }
+      tc::fence_async_smem();
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (ok && quarter == 0 && lane == 0 && j < prm.nkb) {
+      // one thread per block: TMA stores of its D x D state (rows c1 < D)
+      const uint32_t src = sbase + (hh == 0 ? L::kOffK : L::kOffV);
+      for (int c64 = 0; c64 < D / 64; ++c64)
+        tc::tma_store_3d(&tmH, src + c64 * 16384, 64 * c64, 0, bkv * prm.nkb_pad + j);
+      tc::bulk_commit();
+      tc::bulk_wait_all();
     }
     if (!ok) {
       *abort = 1;
@@ -249,6 +268,11 @@ static cudaError_t launch_state_t(const Plan& p, const Args& a, cudaStream_t s) 
       !make_tmap_3d(&mv, a.v, D, (uint64_t)c.N_valid, (uint64_t)c.B * c.H_kv, rowb, headb, 64, 128))
     return cudaErrorInvalidValue;
   const bool proj = c.has_proj && a.w_p;
+  // h'_j as a [D rows][D columns] tile inside row j of the state array; rows c1 < D only
+  CUtensorMap mh;
+  if (!make_tmap_3d(&mh, a.ws + p.off_hs, D, D, (uint64_t)c.B * c.H_kv * p.nkb_pad, rowb, (uint64_t)p.dd * 2,
+                    64, D))
+    return cudaErrorInvalidValue;
   // without a projection the W_p map is never used; encode it over K to keep it valid
   if (!make_tmap_3d(&mw, proj ? (const void*)a.w_p : (const void*)a.k, D, D, 1, rowb, (uint64_t)D * rowb,
                     64, D))
@@ -265,7 +289,7 @@ static cudaError_t launch_state_t(const Plan& p, const Args& a, cudaStream_t s) 
                                        L::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nkb_pad / 2, c.B * c.H_kv);
-  state_tc_kernel<D><<<grid, kStThreads, L::kSmem, s>>>(mk, mv, mw, prm);
+  state_tc_kernel<D><<<grid, kStThreads, L::kSmem, s>>>(mk, mv, mw, mh, prm);
   return cudaGetLastError();
 }
 
