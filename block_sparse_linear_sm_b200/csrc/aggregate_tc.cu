@@ -16,7 +16,8 @@
 // tile next to each other so a tile of states comes from HBM once.
 //
 // Warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2-5 = epilogue
-// (S_i columns to bf16, Z_i columns to fp32, padding columns dropped).
+// (S_i columns to bf16 staged for TMA stores, Z_i columns to fp32, padding
+// columns dropped).
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -40,7 +41,7 @@ struct AggParams {
 
 __global__ void __launch_bounds__(kAgThreads, 1)
     aggregate_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        AggParams prm) {
+                        const __grid_constant__ CUtensorMap tmS, AggParams prm) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -130,7 +131,10 @@ __global__ void __launch_bounds__(kAgThreads, 1)
       }
     }
   } else {
-    // epilogue: thread = query block (TMEM lane) of each 128-row half, 256 columns in 8 chunks
+    // epilogue: thread = query block (TMEM lane) of each 128-row half. S_i columns
+    // are staged as bf16 in the freed stage ring (per half: four 64-column
+    // panels of 128 rows, 128-byte swizzled) and written by TMA stores; Z_i
+    // columns go straight to HBM as fp32.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const bool ok = __all_sync(0xffffffffu, K > 0 && tc::mbar_wait(bar(DONE), 0, abort));
@@ -138,28 +142,48 @@ __global__ void __launch_bounds__(kAgThreads, 1)
     const int dsq = prm.d * prm.d;
     for (int mh = 0; mh < 2 && ok; ++mh) {
       const int row = m0 + mh * 128 + r;
-#pragma unroll 2
-      for (int c = 0; c < kAgBN / 32; ++c) {
-        uint32_t v[32];
-        tc::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + mh * kAgBN + 32 * c, v);
+#pragma unroll 1
+      for (int c64 = 0; c64 < kAgBN / 64; ++c64) {
+        uint32_t v[2][32];
+        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + mh * kAgBN + 64 * c64;
+        tc::tmem_ld32(ta, v[0]);
+        tc::tmem_ld32(ta + 32, v[1]);
         tc::tmem_ld_wait();
-        const int col = n0 + 32 * c;
-        if (row >= prm.nqb) continue;
+        const int col = n0 + 64 * c64;
         if (col < dsq) {
-          uint32_t pw[16];
+          uint4* srow = reinterpret_cast<uint4*>(smem + mh * 65536 + c64 * 16384 + r * 128);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) pw[j] = pack_bf16(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-          uint4* dst = reinterpret_cast<uint4*>(prm.ss + ((size_t)bh * prm.nqb + row) * dsq + col);
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t* vv = v[q >> 2] + 8 * (q & 3);
+            srow[q ^ (r & 7)] = make_uint4(pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
+                                           pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
+                                           pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
+                                           pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7])));
+          }
+        } else if (row < prm.nqb) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
-        } else if (col < dsq + prm.d) {
-          float4* dst = reinterpret_cast<float4*>(prm.zs + ((size_t)bh * prm.nqb + row) * prm.d + (col - dsq));
+          for (int hf = 0; hf < 2; ++hf) {
+            const int cz = col + 32 * hf - dsq;
+            if (cz >= prm.d) continue;
+            float4* dst = reinterpret_cast<float4*>(prm.zs + ((size_t)bh * prm.nqb + row) * prm.d + cz);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(v[hf][4 * j]), __uint_as_float(v[hf][4 * j + 1]),
+                                   __uint_as_float(v[hf][4 * j + 2]), __uint_as_float(v[hf][4 * j + 3]));
+          }
         }
       }
+    }
+    tc::fence_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok && quarter == 0 && lane == 0) {
+      // rows past nqb and columns past d*d fall outside the map and are not written
+      for (int mh = 0; mh < 2; ++mh)
+        for (int c64 = 0; c64 < kAgBN / 64; ++c64)
+          if (n0 + 64 * c64 < dsq && m0 + mh * 128 < prm.nqb)
+            tc::tma_store_3d(&tmS, sbase + mh * 65536 + c64 * 16384, n0 + 64 * c64, m0 + mh * 128, bh);
+      tc::bulk_commit();
+      tc::bulk_wait_all();
     }
   }
   tc::fence_before_sync();
@@ -181,6 +205,12 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
       !make_tmap_3d(&mb, hs, (uint64_t)p.dd, (uint64_t)p.nkb_pad, (uint64_t)c.B * c.H_kv,
                     (uint64_t)p.dd * 2, (uint64_t)p.nkb_pad * p.dd * 2, 64, 64))
     return cudaErrorInvalidValue;
+  // S_i as [B*H][nqb rows][d*d columns], box 64 x 128 (stores)
+  CUtensorMap ms;
+  const uint64_t dsq = (uint64_t)c.d * c.d;
+  if (!make_tmap_3d(&ms, a.ws + p.off_ss, dsq, (uint64_t)p.nqb, (uint64_t)c.B * c.H, dsq * 2,
+                    (uint64_t)p.nqb * dsq * 2, 64, 128))
+    return cudaErrorInvalidValue;
   AggParams prm;
   prm.ss = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_ss);
   prm.zs = reinterpret_cast<float*>(a.ws + p.off_zs);
@@ -194,7 +224,7 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
                                        kAgSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((p.nqb_pad + kAgBM - 1) / kAgBM, (p.dd + kAgBN - 1) / kAgBN, c.B * c.H);
-  aggregate_tc_kernel<<<grid, kAgThreads, kAgSmem, s>>>(ma, mb, prm);
+  aggregate_tc_kernel<<<grid, kAgThreads, kAgSmem, s>>>(ma, mb, ms, prm);
   return cudaGetLastError();
 }
 
