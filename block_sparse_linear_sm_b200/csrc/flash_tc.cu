@@ -44,6 +44,8 @@ struct FlashTcParams {
   int* status;
   int H, group, N, n_valid, nb, len, window;
   int pair_heads;       // 1: halves are heads (2hp, 2hp+1) of a group; 0: query blocks (2p, 2p+1)
+  const float* zs;           // fused epilogue: Z_i [B*H][nqb][D] (fp32)
+  const __nv_bfloat16* w_g;  // fused epilogue: gate weights [H][D] or null
   int npairs;           // units per (b, h) when pairing query blocks
   int words;            // 32-bit words of one block bitmap
   int list_cap;         // capacity of the merged list
@@ -62,16 +64,22 @@ struct TcLayout {
   static constexpr int kSlotBytes = 64 * D * 2;         // one K or V tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + kQBytes;
-  static constexpr int kOffBar = kOffKV + kSlots * kSlotBytes;  // 16 mbarriers
-  static constexpr int kOffMisc = kOffBar + 16 * 8;      // tmem addr, count, abort
+  static constexpr int kOffBar = kOffKV + kSlots * kSlotBytes;  // 32 mbarriers
+  static constexpr int kOffMisc = kOffBar + 32 * 8;      // tmem addr, count, abort
   static constexpr int kOffList = kOffMisc + 64;         // merged block list
   static constexpr int kTmemCols = 256;                  // O: D columns, S: 2 x 64 columns
 };
 
-template <int D, bool TOPN>
+// FUSE (three-way layers with a linear branch): the epilogue of the layer runs
+// in the kernel's tail. S'_i (tmS) for both query blocks of the unit is loaded
+// into the freed K/V rings, phi(Q) replaces Q in place, num = phi(Q) S'_i goes
+// to the freed S columns of TMEM (one query block at a time) and
+// O = O_s + g * num / (phi(q) . Z_i) is written to the output.
+template <int D, bool TOPN, bool FUSE>
 __global__ void __launch_bounds__(kTcThreads, 2)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, FlashTcParams prm) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
+                    FlashTcParams prm) {
   using L = TcLayout<D>;
   constexpr int NP = D / 64;  // 64-column panels
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -93,8 +101,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   // barrier ids: K ring, V ring (full / empty per slot), S and P per TMEM buffer
   constexpr int Q_FULL = 0, K_FULL = 1, K_EMPTY = K_FULL + kKSlots, V_FULL = K_EMPTY + kKSlots,
                 V_EMPTY = V_FULL + kVSlots, S_FULL = V_EMPTY + kVSlots, P_FULL = S_FULL + 2,
-                O_DONE = P_FULL + 2;
-  static_assert(O_DONE < 16, "barrier area holds 16 mbarriers");
+                O_DONE = P_FULL + 2, SP_FULL = O_DONE + 1, PHI_READY = SP_FULL + 1,
+                NUM_DONE = PHI_READY + 1, NUM_READ = NUM_DONE + 2;
+  static_assert(NUM_READ < 32, "barrier area holds 32 mbarriers");
 
   // ---- unit decode ----------------------------------------------------------
   const int Hkv = prm.H / prm.group;
@@ -150,6 +159,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       tc::mbar_init(bar(P_FULL + b), 4);
     }
     tc::mbar_init(bar(O_DONE), 1);
+    tc::mbar_init(bar(SP_FULL), 1);
+    tc::mbar_init(bar(PHI_READY), 4);
+    tc::mbar_init(bar(NUM_DONE), 1);
+    tc::mbar_init(bar(NUM_DONE + 1), 1);
+    tc::mbar_init(bar(NUM_READ), 2);
     tc::fence_mbar_init();
   }
   if (warp == 1) {
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
   if (warp == 0) {
     // ======================= TMA producer =====================================
-    if (lane == 0 && T > 0) {
+    if (lane == 0 && (T > 0 || FUSE)) {
       tc::prefetch_tensormap(&tmQ);
       tc::prefetch_tensormap(&tmK);
       tc::prefetch_tensormap(&tmV);
@@ -277,10 +291,19 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           *abort = 1;
           report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
         }
+      if (FUSE && !*abort) {
+        // the rings are free: S'_i of both query blocks, D/64 panels of D rows each
+        const int nh = valid_h[1] ? 2 : 1;
+        tc::mbar_expect_tx(bar(SP_FULL), nh * D * D * 2);
+        for (int hf = 0; hf < nh; ++hf)
+          for (int p = 0; p < NP; ++p)
+            tc::tma_load_3d(sKV + hf * D * D * 2 + p * D * 128, &tmS, bar(SP_FULL), 64 * p, 0,
+                            bh_h[hf] * prm.nb + i_h[hf]);
+      }
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================================
-    if (lane == 0 && T > 0) {
+    if (lane == 0 && (T > 0 || FUSE)) {
       constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(128, D, false, true);
       const uint32_t tO = tmem, tS0 = tmem + D;
@@ -302,7 +325,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         tc::mma_commit(bar(K_EMPTY + slot));
         return true;
       };
-      if (ok) ok = issue_s(0);
+      if (ok && T > 0) ok = issue_s(0);
       if (ok && T > 1) ok = issue_s(1);
       for (int n = 0; n < T && ok; ++n) {
         const int b = n & 1;
@@ -329,6 +352,28 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         if (n + 2 < T && !issue_s(n + 2)) {
           ok = false;
           break;
+        }
+      }
+      if (FUSE && ok) {
+        // num = phi(Q) S'_i (M = 128 rows, N = D, K = D) into the S columns, one query
+        // block at a time: the second waits until the first block's rows are read
+        constexpr uint32_t kIdN = tc::idesc_bf16(128, D, false, true);
+        ok = tc::mbar_wait(bar(PHI_READY), 0, abort) && tc::mbar_wait(bar(SP_FULL), 0, abort);
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          if (!valid_h[hf]) break;
+          if (hf == 1 && !tc::mbar_wait(bar(NUM_READ), 0, abort)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t sb = sKV + hf * D * D * 2;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t da = tc::sw128_desc(sQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+            const uint64_t db = tc::sw128_desc(sb + k * 2048, D * 128, 1024);
+            tc::mma_bf16_ss(tS0, da, db, kIdN, k > 0);
+          }
+          tc::mma_commit(bar(NUM_DONE + hf));
         }
       }
       if (!ok) {
@@ -459,8 +504,94 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       *abort = 1;
       report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
     }
-    // epilogue: O / l -> bf16 rows (padding tokens and empty rows are zero)
-    if (valid_h[hf]) {
+    if (FUSE) {
+      // ---- fused epilogue of the layer (three-way mode with a linear branch) ----
+      const int h = bh_h[hf] % prm.H;
+      ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(Q_FULL), 0, abort));
+      // gate from the raw query row, then phi in place and den = phi(q) . Z_i
+      float gdot = 0.f, den = 0.f;
+      // Z_i exists only for a real query block (the second half of the last pair may not)
+      const float* zg = valid_h[hf] ? prm.zs + ((size_t)bh_h[hf] * prm.nb + i_h[hf]) * D : nullptr;
+      const __nv_bfloat16* wg = prm.w_g ? prm.w_g + (size_t)h * D : nullptr;
+      if (ok) {
+#pragma unroll 1
+        for (int pc = 0; pc < 2 * NP; ++pc) {  // half a panel (4 chunks) at a time
+          const int p = pc >> 1, cb = 4 * (pc & 1);
+          uint4 u[4];
+          uint4* qrow = reinterpret_cast<uint4*>(smem + L::kOffQ + p * 16384 + r * 128);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) u[c] = qrow[(cb + c) ^ (r & 7)];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&u[c]);
+            const int c0 = 64 * p + 8 * (cb + c);
+            const float4 z0 = zg ? *reinterpret_cast<const float4*>(zg + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 z1 = zg ? *reinterpret_cast<const float4*>(zg + c0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+            uint4 gw = make_uint4(0, 0, 0, 0);
+            if (wg) gw = *reinterpret_cast<const uint4*>(wg + c0);
+            const uint32_t* gg = reinterpret_cast<const uint32_t*>(&gw);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const float2 f = unpack_bf16(wv[x]);
+              const float2 g2 = unpack_bf16(gg[x]);
+              gdot = fmaf(f.x, g2.x, fmaf(f.y, g2.y, gdot));
+              wv[x] = pack_bf16(phi(f.x), phi(f.y));
+              const float2 ph = unpack_bf16(wv[x]);
+              den = fmaf(ph.x, zz[2 * x], fmaf(ph.y, zz[2 * x + 1], den));
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) qrow[(cb + c) ^ (r & 7)] = u[c];
+        }
+        tc::fence_async_smem();
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(PHI_READY));
+      const float g = wg ? 1.f / (1.f + __expf(-gdot)) : 1.f;
+      const float cl = den > 0.f ? g / den : 0.f;
+      if (valid_h[hf]) {
+        ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(NUM_DONE + hf), 0, abort));
+        tc::fence_after_sync();
+        const bool live = ok && t < prm.n_valid;
+        const float inv = (live && T > 0 && l_sum > 0.f) ? 1.f / l_sum : 0.f;
+        __nv_bfloat16* og = prm.o + ((size_t)bh_h[hf] * prm.N + t) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t ov[16], nv[16];
+          if (ok) {
+            if (T > 0) tc::tmem_ld16(tO + 16 * c, ov);
+            tc::tmem_ld16(tS0 + 16 * c, nv);
+            tc::tmem_ld_wait();
+          }
+          if (!ok || T == 0) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) ov[j] = 0u;
+          }
+          uint32_t pw[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            pw[j] = live ? pack_bf16(__uint_as_float(ov[2 * j]) * inv + cl * __uint_as_float(nv[2 * j]),
+                                     __uint_as_float(ov[2 * j + 1]) * inv + cl * __uint_as_float(nv[2 * j + 1]))
+                         : 0u;
+          uint4* dst = reinterpret_cast<uint4*>(og + 16 * c);
+          dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+          dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+        }
+        if (hf == 0) {
+          // this block's rows of the num columns are read: the next block may overwrite them
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(bar(NUM_READ));
+        }
+      }
+      if (!ok) {
+        *abort = 1;
+        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+      }
+    } else if (valid_h[hf]) {
+      // epilogue: O / l -> bf16 rows (padding tokens and empty rows are zero)
       const float inv = (ok && T > 0 && l_sum > 0.f && t < prm.n_valid) ? 1.f / l_sum : 0.f;
       __nv_bfloat16* og = prm.o + ((size_t)bh_h[hf] * prm.N + t) * D;
 #pragma unroll
@@ -482,14 +613,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
         for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
       }
-    } else if (T > 0 && ok) {
-      // keep the warp-collective TMEM loads uniform across the warp
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tc::tmem_ld32(tO + 32 * c, ov);
-        tc::tmem_ld_wait();
-      }
     }
   }
   tc::fence_before_sync();
@@ -509,20 +632,24 @@ static bool make_map(CUtensorMap* m, const void* base, int heads, int n_rows, in
                       (uint64_t)N * D * 2, 64, 64);
 }
 
-template <int D, bool TOPN>
+template <int D, bool TOPN, bool FUSE>
 static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
   using L = TcLayout<D>;
   const sla_config& c = p.c;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, ms;
   if (!make_map(&mq, a.q, c.B * c.H, c.N_valid, c.N, D) ||
       !make_map(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) ||
       !make_map(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
     return cudaErrorInvalidValue;
+  // S'_i as [B*H*nqb][D rows][D columns], box 64 x D (fused epilogue); otherwise unused
+  if (!make_tmap_3d(&ms, FUSE ? (const void*)(a.ws + p.off_ss) : (const void*)a.q, D, D,
+                    FUSE ? (uint64_t)c.B * c.H * p.nqb : 1, (uint64_t)D * 2, (uint64_t)D * D * 2, 64, D))
+    return cudaErrorInvalidValue;
   FlashTcParams prm;
   prm.list = a.crit;
-  // with a linear branch the epilogue combines; otherwise this is the output
-  const bool direct = TOPN || p.nkb - c.k_h - c.k_l <= 0;
-  prm.o = direct ? a.out : reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_os);
+  prm.o = a.out;  // the sparse branch is the output, or the fused epilogue writes it
+  prm.zs = FUSE ? reinterpret_cast<const float*>(a.ws + p.off_zs) : nullptr;
+  prm.w_g = FUSE && c.has_gate ? a.w_g : nullptr;
   prm.status = a.status;
   prm.H = c.H;
   prm.group = p.group;
@@ -543,7 +670,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
   if (4 * prm.words * 4 > kSlots * L::kSlotBytes) return cudaErrorInvalidValue;  // bitmaps in the ring
   // at most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN>,
+  cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN, FUSE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int units;
@@ -551,14 +678,19 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
     units = c.B * c.H_kv * p.nqb * (p.group / 2);
   else
     units = c.B * c.H * prm.npairs;
-  flash_tc_kernel<D, TOPN><<<units, kTcThreads, smem, s>>>(mq, mk, mv, prm);
+  flash_tc_kernel<D, TOPN, FUSE><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s) {
   const bool topn = p.c.mode == SLA_MODE_TOPN_WINDOW;
-  if (p.c.d == 128) return topn ? launch_tc<128, true>(p, a, s) : launch_tc<128, false>(p, a, s);
-  return topn ? launch_tc<64, true>(p, a, s) : launch_tc<64, false>(p, a, s);
+  const bool fuse = !topn && p.nkb - p.c.k_h - p.c.k_l > 0;  // the layer has a linear branch
+  if (p.c.d == 128) {
+    if (topn) return launch_tc<128, true, false>(p, a, s);
+    return fuse ? launch_tc<128, false, true>(p, a, s) : launch_tc<128, false, false>(p, a, s);
+  }
+  if (topn) return launch_tc<64, true, false>(p, a, s);
+  return fuse ? launch_tc<64, false, true>(p, a, s) : launch_tc<64, false, false>(p, a, s);
 }
 
 }  // namespace sla

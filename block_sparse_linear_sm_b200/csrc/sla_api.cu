@@ -67,7 +67,6 @@ bool make_plan(const sla_config* c, Plan* p) {
       p->off_hs = take(B * Hkv * (size_t)p->nkb_pad * p->dd * 2);
       p->off_ss = take(B * H * nqb * d * d * 2);  // S_i (times W_p), bf16
       p->off_zs = take(B * H * nqb * d * 4);      // Z_i, fp32
-      p->off_os = take(B * H * (size_t)c->N * d * 2);
     }
   } else {
     p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
@@ -81,7 +80,7 @@ static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 static bool has_marginal(const Plan& p) { return p.nkb - p.c.k_h - p.c.k_l > 0; }
 
 // Stage list of a configuration.
-enum Stage { kPool, kScores, kClassify, kSelect, kState, kAggregate, kFlash, kEpilogue };
+enum Stage { kPool, kScores, kClassify, kSelect, kState, kAggregate, kFlash };
 
 static int stages_of(const Plan& p, Stage* out) {
   int n = 0;
@@ -92,11 +91,8 @@ static int stages_of(const Plan& p, Stage* out) {
     if (has_marginal(p)) {
       out[n++] = kState;
       out[n++] = kAggregate;
-      out[n++] = kFlash;
-      out[n++] = kEpilogue;
-    } else {
-      out[n++] = kFlash;  // no linear branch: the sparse branch is the output
     }
+    out[n++] = kFlash;  // with a linear branch its tail runs the layer's epilogue
   } else {
     out[n++] = kSelect;
     out[n++] = kFlash;
@@ -113,7 +109,6 @@ static const char* stage_name(Stage s) {
     case kState: return "linear_state";
     case kAggregate: return "linear_aggregate";
     case kFlash: return "sparse_flash";
-    case kEpilogue: return "epilogue";
   }
   return "?";
 }
@@ -127,7 +122,6 @@ static cudaError_t run_stage(Stage st, const Plan& p, const Args& a, cudaStream_
     case kState: return launch_state(p, a, s);
     case kAggregate: return launch_aggregate(p, a, s);
     case kFlash: return launch_flash(p, a, s);
-    case kEpilogue: return launch_epilogue(p, a, s);
   }
   return cudaErrorInvalidValue;
 }

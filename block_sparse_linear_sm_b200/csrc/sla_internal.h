@@ -16,7 +16,6 @@ constexpr int kMaxBlocks = 4096;  // nkb limit of the routing sort (N <= 262144)
 // Device status word: status[0] = sla_status code, status[1] = detail.
 enum DeviceDetail : int {
   kDetailFlashIndex = 101,      // flash kernel read a block index outside [0, nkb)
-  kDetailEpilogueIndex = 102,
   kDetailFlashAlign = 103,     // shared-memory base not 1024-byte aligned
   kDetailTimeout = 200,
 };
@@ -32,7 +31,7 @@ struct Plan {
   float scale;
   // byte offsets into ws
   size_t off_status, off_qbar, off_kbar, off_scores, off_crit, off_neg, off_mmask, off_hs, off_ss,
-      off_zs, off_os, total;
+      off_zs, total;
 };
 
 bool make_plan(const sla_config* c, Plan* p);
@@ -66,6 +65,5 @@ cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s);
-cudaError_t launch_epilogue(const Plan& p, const Args& a, cudaStream_t s);
 
 }  // namespace sla
