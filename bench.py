@@ -57,6 +57,9 @@ def stage_model(c: wl.LayerConfig) -> dict:
     bf = 2
     m = {}
     m["pool"] = ("hbm", (B * H + B * Hkv) * Nv * d * bf + (B * H + B * Hkv) * nb * d * 8)
+    if c.mode == wl.MODE_THREEWAY and nb - c.k_h - c.k_l > 0:
+        # phi(Q) (bf16) and, with a gate, g_t (fp32) for the linear branch
+        m["pool"] = ("hbm", m["pool"][1] + B * H * Nv * d * bf + (B * H * Nv * 4 if c.has_gate else 0))
     m["pooled_scores"] = ("hbm", (B * H + B * Hkv) * nb * d * 8 + B * H * nb * nb * 8)
     if c.mode == wl.MODE_THREEWAY:
         marg = nb - c.k_h - c.k_l
@@ -67,7 +70,6 @@ def stage_model(c: wl.LayerConfig) -> dict:
         m["linear_aggregate"] = ("tensor", 2.0 * B * H * nb * nb * dd)
         # attended FLOP over critical blocks: QK^T and PV, 2 * 2 * b^2 * d per (row, block)
         m["sparse_flash"] = ("tensor", 4.0 * c.block * c.block * d * B * H * nb * c.k_h)
-        m["epilogue"] = ("hbm", B * H * Nv * d * bf * 3 + B * H * nb * dd * 4)
     else:
         m["select_topn"] = ("hbm", B * H * nb * nb * 8 / 2 + B * Hkv * nb * (c.top_n * 4 + nb))
         # attended (query, key) pairs, upper bound: window tokens plus selected tokens

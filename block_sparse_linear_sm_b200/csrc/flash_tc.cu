@@ -44,8 +44,8 @@ struct FlashTcParams {
   int* status;
   int H, group, N, n_valid, nb, len, window;
   int pair_heads;       // 1: halves are heads (2hp, 2hp+1) of a group; 0: query blocks (2p, 2p+1)
-  const float* zs;           // fused epilogue: Z_i [B*H][nqb][D] (fp32)
-  const __nv_bfloat16* w_g;  // fused epilogue: gate weights [H][D] or null
+  const float* zs;     // fused epilogue: Z_i [B*H][nqb][D] (fp32)
+  const float* gate;   // fused epilogue: g_t = sigmoid(q_t . w_g[h]) [B*H][N] (fp32) or null
   int npairs;           // units per (b, h) when pairing query blocks
   int words;            // 32-bit words of one block bitmap
   int list_cap;         // capacity of the merged list
@@ -71,15 +71,16 @@ struct TcLayout {
 };
 
 // FUSE (three-way layers with a linear branch): the epilogue of the layer runs
-// in the kernel's tail. S'_i (tmS) for both query blocks of the unit is loaded
-// into the freed K/V rings, phi(Q) replaces Q in place, num = phi(Q) S'_i goes
-// to the freed S columns of TMEM (one query block at a time) and
+// in the kernel's tail. Once the last S and PV products are done, S'_i (tmS) and
+// Z_i of both query blocks of the unit are loaded into the freed K/V rings and
+// phi(Q) (tmF, written by the pooling pass) into the Q tiles; num = phi(Q) S'_i
+// goes to the freed S columns of TMEM (one query block at a time) and
 // O = O_s + g * num / (phi(q) . Z_i) is written to the output.
 template <int D, bool TOPN, bool FUSE>
 __global__ void __launch_bounds__(kTcThreads, 2)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
-                    FlashTcParams prm) {
+                    const __grid_constant__ CUtensorMap tmF, FlashTcParams prm) {
   using L = TcLayout<D>;
   constexpr int NP = D / 64;  // 64-column panels
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -101,8 +102,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   // barrier ids: K ring, V ring (full / empty per slot), S and P per TMEM buffer
   constexpr int Q_FULL = 0, K_FULL = 1, K_EMPTY = K_FULL + kKSlots, V_FULL = K_EMPTY + kKSlots,
                 V_EMPTY = V_FULL + kVSlots, S_FULL = V_EMPTY + kVSlots, P_FULL = S_FULL + 2,
-                O_DONE = P_FULL + 2, SP_FULL = O_DONE + 1, PHI_READY = SP_FULL + 1,
-                NUM_DONE = PHI_READY + 1, NUM_READ = NUM_DONE + 2;
+                O_DONE = P_FULL + 2, SP_FULL = O_DONE + 1, NUM_DONE = SP_FULL + 1,
+                NUM_READ = NUM_DONE + 2;
   static_assert(NUM_READ < 32, "barrier area holds 32 mbarriers");
 
   // ---- unit decode ----------------------------------------------------------
@@ -160,7 +161,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
     tc::mbar_init(bar(O_DONE), 1);
     tc::mbar_init(bar(SP_FULL), 1);
-    tc::mbar_init(bar(PHI_READY), 4);
     tc::mbar_init(bar(NUM_DONE), 1);
     tc::mbar_init(bar(NUM_DONE + 1), 1);
     tc::mbar_init(bar(NUM_READ), 2);
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
   if (warp == 0) {
     // ======================= TMA producer =====================================
-    if (lane == 0 && (T > 0 || FUSE)) {
+    if (lane == 0 && T > 0) {
       tc::prefetch_tensormap(&tmQ);
       tc::prefetch_tensormap(&tmK);
       tc::prefetch_tensormap(&tmV);
@@ -291,15 +291,22 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           *abort = 1;
           report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
         }
-      if (FUSE && !*abort) {
-        // the rings are free: S'_i of both query blocks, D/64 panels of D rows each
-        const int nh = valid_h[1] ? 2 : 1;
-        tc::mbar_expect_tx(bar(SP_FULL), nh * D * D * 2);
-        for (int hf = 0; hf < nh; ++hf)
-          for (int p = 0; p < NP; ++p)
-            tc::tma_load_3d(sKV + hf * D * D * 2 + p * D * 128, &tmS, bar(SP_FULL), 64 * p, 0,
-                            bh_h[hf] * prm.nb + i_h[hf]);
+    }
+    if (FUSE && lane == 0 && !*abort) {
+      // every S and PV product has completed (the waits above): the rings take
+      // S'_i and Z_i of both query blocks, the Q tiles take phi(Q)
+      const int nh = valid_h[1] ? 2 : 1;
+      tc::mbar_expect_tx(bar(SP_FULL), nh * (D * D * 2 + D * 4) + L::kQBytes);
+      for (int hf = 0; hf < nh; ++hf) {
+        const int blk = bh_h[hf] * prm.nb + i_h[hf];
+        for (int p = 0; p < NP; ++p)
+          tc::tma_load_3d(sKV + hf * D * D * 2 + p * D * 128, &tmS, bar(SP_FULL), 64 * p, 0, blk);
+        tc::bulk_load(sKV + 2 * D * D * 2 + hf * D * 4, prm.zs + (size_t)blk * D, D * 4, bar(SP_FULL));
       }
+      for (int hf = 0; hf < 2; ++hf)
+        for (int p = 0; p < NP; ++p)
+          tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmF, bar(SP_FULL), 64 * p, i_h[hf] * kBlock,
+                          bh_h[hf]);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================================
@@ -307,7 +314,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(128, D, false, true);
       const uint32_t tO = tmem, tS0 = tmem + D;
-      bool ok = tc::mbar_wait(bar(Q_FULL), 0, abort);
+      bool ok = T == 0 || tc::mbar_wait(bar(Q_FULL), 0, abort);
       tc::fence_after_sync();
       // S_n = Q K_n^T into TMEM buffer n & 1
       auto issue_s = [&](int n) -> bool {
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         // num = phi(Q) S'_i (M = 128 rows, N = D, K = D) into the S columns, one query
         // block at a time: the second waits until the first block's rows are read
         constexpr uint32_t kIdN = tc::idesc_bf16(128, D, false, true);
-        ok = tc::mbar_wait(bar(PHI_READY), 0, abort) && tc::mbar_wait(bar(SP_FULL), 0, abort);
+        ok = tc::mbar_wait(bar(SP_FULL), 0, abort);
         for (int hf = 0; hf < 2 && ok; ++hf) {
           if (!valid_h[hf]) break;
           if (hf == 1 && !tc::mbar_wait(bar(NUM_READ), 0, abort)) {
@@ -506,50 +513,26 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
     if (FUSE) {
       // ---- fused epilogue of the layer (three-way mode with a linear branch) ----
-      const int h = bh_h[hf] % prm.H;
-      ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(Q_FULL), 0, abort));
-      // gate from the raw query row, then phi in place and den = phi(q) . Z_i
-      float gdot = 0.f, den = 0.f;
-      // Z_i exists only for a real query block (the second half of the last pair may not)
-      const float* zg = valid_h[hf] ? prm.zs + ((size_t)bh_h[hf] * prm.nb + i_h[hf]) * D : nullptr;
-      const __nv_bfloat16* wg = prm.w_g ? prm.w_g + (size_t)h * D : nullptr;
-      if (ok) {
-#pragma unroll 1
-        for (int pc = 0; pc < 2 * NP; ++pc) {  // half a panel (4 chunks) at a time
-          const int p = pc >> 1, cb = 4 * (pc & 1);
-          uint4 u[4];
-          uint4* qrow = reinterpret_cast<uint4*>(smem + L::kOffQ + p * 16384 + r * 128);
+      // den = phi(q) . Z_i from the tiles the producer loaded
+      ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL), 0, abort));
+      float den = 0.f;
+      if (ok && valid_h[hf]) {
+        const float4* z4 = reinterpret_cast<const float4*>(smem + L::kOffKV + 2 * D * D * 2 + hf * D * 4);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) u[c] = qrow[(cb + c) ^ (r & 7)];
+        for (int p = 0; p < NP; ++p) {
+          const uint4* frow = reinterpret_cast<const uint4*>(smem + L::kOffQ + p * 16384 + r * 128);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&u[c]);
-            const int c0 = 64 * p + 8 * (cb + c);
-            const float4 z0 = zg ? *reinterpret_cast<const float4*>(zg + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 z1 = zg ? *reinterpret_cast<const float4*>(zg + c0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-            uint4 gw = make_uint4(0, 0, 0, 0);
-            if (wg) gw = *reinterpret_cast<const uint4*>(wg + c0);
-            const uint32_t* gg = reinterpret_cast<const uint32_t*>(&gw);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const float2 f = unpack_bf16(wv[x]);
-              const float2 g2 = unpack_bf16(gg[x]);
-              gdot = fmaf(f.x, g2.x, fmaf(f.y, g2.y, gdot));
-              wv[x] = pack_bf16(phi(f.x), phi(f.y));
-              const float2 ph = unpack_bf16(wv[x]);
-              den = fmaf(ph.x, zz[2 * x], fmaf(ph.y, zz[2 * x + 1], den));
-            }
+          for (int c = 0; c < 8; ++c) {
+            const uint4 u = frow[c ^ (r & 7)];
+            const float4 za = z4[16 * p + 2 * c], zb = z4[16 * p + 2 * c + 1];
+            const float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z),
+                         f3 = unpack_bf16(u.w);
+            den = fmaf(f0.x, za.x, fmaf(f0.y, za.y, fmaf(f1.x, za.z, fmaf(f1.y, za.w, den))));
+            den = fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, fmaf(f3.x, zb.z, fmaf(f3.y, zb.w, den))));
           }
-#pragma unroll
-          for (int c = 0; c < 4; ++c) qrow[(cb + c) ^ (r & 7)] = u[c];
         }
-        tc::fence_async_smem();
       }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(PHI_READY));
-      const float g = wg ? 1.f / (1.f + __expf(-gdot)) : 1.f;
+      const float g = (prm.gate && valid_h[hf] && t < prm.n_valid) ? prm.gate[(size_t)bh_h[hf] * prm.N + t] : 1.f;
       const float cl = den > 0.f ? g / den : 0.f;
       if (valid_h[hf]) {
         ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(NUM_DONE + hf), 0, abort));
@@ -641,6 +624,10 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
       !make_map(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) ||
       !make_map(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
     return cudaErrorInvalidValue;
+  // phi(Q) from the pooling pass, same geometry as Q (fused epilogue); otherwise unused
+  CUtensorMap mf;
+  if (!make_map(&mf, FUSE ? (const void*)(a.ws + p.off_phiq) : (const void*)a.q, c.B * c.H, c.N_valid, c.N, D))
+    return cudaErrorInvalidValue;
   // S'_i as [B*H*nqb][D rows][D columns], box 64 x D (fused epilogue); otherwise unused
   if (!make_tmap_3d(&ms, FUSE ? (const void*)(a.ws + p.off_ss) : (const void*)a.q, D, D,
                     FUSE ? (uint64_t)c.B * c.H * p.nqb : 1, (uint64_t)D * 2, (uint64_t)D * D * 2, 64, D))
@@ -649,7 +636,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
   prm.list = a.crit;
   prm.o = a.out;  // the sparse branch is the output, or the fused epilogue writes it
   prm.zs = FUSE ? reinterpret_cast<const float*>(a.ws + p.off_zs) : nullptr;
-  prm.w_g = FUSE && c.has_gate ? a.w_g : nullptr;
+  prm.gate = FUSE && c.has_gate ? reinterpret_cast<const float*>(a.ws + p.off_gate) : nullptr;
   prm.status = a.status;
   prm.H = c.H;
   prm.group = p.group;
@@ -678,7 +665,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
     units = c.B * c.H_kv * p.nqb * (p.group / 2);
   else
     units = c.B * c.H * prm.npairs;
-  flash_tc_kernel<D, TOPN, FUSE><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, prm);
+  flash_tc_kernel<D, TOPN, FUSE><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, mf, prm);
   return cudaGetLastError();
 }
 

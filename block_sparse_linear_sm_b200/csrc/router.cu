@@ -17,11 +17,16 @@ namespace sla {
 
 // ---------------------------------------------------------------------------
 // pooling: one CTA per (head row, block); d/2 threads, two columns each.
-// Q heads first (B*H of them), then KV heads (B*H_kv).
+// Q heads first (B*H of them), then KV heads (B*H_kv). For layers with a linear
+// branch the Q pass also writes phi(Q) (bf16, the left factor of the linear
+// branch's numerator and denominator) and, with a gate, g_t = sigmoid(q_t .
+// w_g[h]) per token: Q is read here anyway, so the epilogue need not
+// transform it again.
 // ---------------------------------------------------------------------------
 __global__ void pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                             double* __restrict__ qbar, double* __restrict__ kbar, int n_qheads,
-                            int N, int n_valid, int d, int nb) {
+                            int N, int n_valid, int d, int nb, __nv_bfloat16* __restrict__ phiq,
+                            const __nv_bfloat16* __restrict__ w_g, float* __restrict__ gate, int H) {
   const int j = blockIdx.x;
   const int hrow = blockIdx.y;
   const bool is_q = hrow < n_qheads;
@@ -31,6 +36,8 @@ __global__ void pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bflo
   const int c = threadIdx.x * 2;
   int nv = n_valid - j * kBlock;
   nv = nv > kBlock ? kBlock : nv;
+  __nv_bfloat16* fq =
+      (is_q && phiq) ? phiq + ((size_t)hh * N + (size_t)j * kBlock) * d : nullptr;
   double s0 = 0.0, s1 = 0.0;
 #pragma unroll 8
   for (int t = 0; t < nv; ++t) {
@@ -38,18 +45,46 @@ __global__ void pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bflo
     float2 f = unpack_bf16(u);
     s0 += (double)f.x;
     s1 += (double)f.y;
+    if (fq) *reinterpret_cast<uint32_t*>(fq + (size_t)t * d + c) = pack_bf16(phi(f.x), phi(f.y));
   }
   // mean = sum / count (one rounding, as a division)
   out[c] = nv > 0 ? s0 / (double)nv : 0.0;
   out[c + 1] = nv > 0 ? s1 / (double)nv : 0.0;
+  if (is_q && gate) {
+    // one token per thread; the rows were just read, so they come from cache
+    const __nv_bfloat16* wg = w_g + (size_t)(hh % H) * d;
+    for (int t = threadIdx.x; t < nv; t += blockDim.x) {
+      const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int c8 = 0; c8 < d / 8; ++c8) {
+        const uint4 u = row[c8];
+        const uint4 w = *reinterpret_cast<const uint4*>(wg + c8 * 8);
+        const uint32_t* uu = reinterpret_cast<const uint32_t*>(&u);
+        const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fu = unpack_bf16(uu[e]), fw = unpack_bf16(ww[e]);
+          acc[e] = fmaf(fu.x, fw.x, fmaf(fu.y, fw.y, acc[e]));
+        }
+      }
+      const float dot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      gate[(size_t)hh * N + (size_t)j * kBlock + t] = 1.f / (1.f + __expf(-dot));
+    }
+  }
 }
 
 cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
   const sla_config& c = p.c;
   double* qbar = reinterpret_cast<double*>(a.ws + p.off_qbar);
   double* kbar = reinterpret_cast<double*>(a.ws + p.off_kbar);
+  // phi(Q) and the gate feed the linear branch of a forward pass; routing-only
+  // calls (no V) do not produce them
+  const bool lin = a.v != nullptr && c.mode == SLA_MODE_THREEWAY && p.nkb - c.k_h - c.k_l > 0;
+  __nv_bfloat16* phiq = lin ? reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_phiq) : nullptr;
+  float* gate = (lin && c.has_gate) ? reinterpret_cast<float*>(a.ws + p.off_gate) : nullptr;
   dim3 grid(p.nqb, c.B * c.H + c.B * c.H_kv);
-  pool_kernel<<<grid, c.d / 2, 0, s>>>(a.q, a.k, qbar, kbar, c.B * c.H, c.N, c.N_valid, c.d, p.nqb);
+  pool_kernel<<<grid, c.d / 2, 0, s>>>(a.q, a.k, qbar, kbar, c.B * c.H, c.N, c.N_valid, c.d,
+                                       p.nqb, phiq, gate ? a.w_g : nullptr, gate, c.H);
   return cudaGetLastError();
 }
 

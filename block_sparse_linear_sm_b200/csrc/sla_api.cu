@@ -67,6 +67,8 @@ bool make_plan(const sla_config* c, Plan* p) {
       p->off_hs = take(B * Hkv * (size_t)p->nkb_pad * p->dd * 2);
       p->off_ss = take(B * H * nqb * d * d * 2);  // S_i (times W_p), bf16
       p->off_zs = take(B * H * nqb * d * 4);      // Z_i, fp32
+      p->off_phiq = take(B * H * (size_t)c->N * d * 2);  // phi(Q), bf16
+      if (c->has_gate) p->off_gate = take(B * H * (size_t)c->N * 4);  // sigmoid(q . w_g), fp32
     }
   } else {
     p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
