@@ -310,80 +310,85 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================================
-    if (lane == 0 && (T > 0 || FUSE)) {
+    // The whole warp runs the loop (waits, descriptors); one elected lane issues.
+    if (T > 0 || FUSE) {
       constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(128, D, false, true);
+      constexpr uint32_t kAll = 0xffffffffu;
       const uint32_t tO = tmem, tS0 = tmem + D;
-      bool ok = T == 0 || tc::mbar_wait(bar(Q_FULL), 0, abort);
+      // base descriptors; a byte offset off is added as off >> 4 (start-address field)
+      const uint64_t dQ = tc::sw128_desc(sQ, 16, 1024);
+      const uint64_t dK = tc::sw128_desc(sKV, 16, 1024);
+      const uint64_t dV = tc::sw128_desc(sKV + kKSlots * L::kSlotBytes, 8192, 1024);
+      bool ok = T == 0 || __all_sync(kAll, tc::mbar_wait(bar(Q_FULL), 0, abort));
       tc::fence_after_sync();
-      // S_n = Q K_n^T into TMEM buffer n & 1
-      auto issue_s = [&](int n) -> bool {
+      // S_n = Q K_n^T into TMEM buffer n & 1 (elected lane; K_n is resident)
+      auto issue_s = [&](int n) {
         const int slot = n % kKSlots;
-        if (!tc::mbar_wait(bar(K_FULL + slot), (n / kKSlots) & 1, abort)) return false;
-        tc::fence_after_sync();
-        const uint32_t kb = sKV + slot * L::kSlotBytes;
+        const uint64_t dk = dK + (uint32_t)(slot * L::kSlotBytes >> 4);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t da = tc::sw128_desc(sQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-          const uint64_t db = tc::sw128_desc(kb + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
-          tc::mma_bf16_ss(tS0 + 64 * (n & 1), da, db, kIdS, k > 0);
-        }
+        for (int k = 0; k < D / 16; ++k)
+          tc::mma_bf16_ss(tS0 + 64 * (n & 1), dQ + (uint32_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                          dk + (uint32_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4), kIdS, k > 0);
         tc::mma_commit(bar(S_FULL + (n & 1)));
         tc::mma_commit(bar(K_EMPTY + slot));
-        return true;
       };
-      if (ok && T > 0) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
-      for (int n = 0; n < T && ok; ++n) {
-        const int b = n & 1;
-        // P_n sits in TMEM buffer b (written by the softmax warps)
-        if (!tc::mbar_wait(bar(P_FULL + b), (n >> 1) & 1, abort)) {
-          ok = false;
-          break;
-        }
-        const int slot = n % kVSlots;
-        if (!tc::mbar_wait(bar(V_FULL + slot), (n / kVSlots) & 1, abort)) {
-          ok = false;
-          break;
-        }
+      auto wait_k = [&](int n) -> bool {
+        return __all_sync(kAll, tc::mbar_wait(bar(K_FULL + n % kKSlots), (n / kKSlots) & 1, abort));
+      };
+      for (int n = 0; n < 2 && n < T && ok; ++n) {
+        ok = wait_k(n);
         tc::fence_after_sync();
-        const uint32_t vb = sKV + (kKSlots + slot) * L::kSlotBytes;
+        if (ok && tc::elect_one()) issue_s(n);
+        __syncwarp();
+      }
+      for (int n = 0; n < T && ok; ++n) {
+        const int b = n & 1, slot = n % kVSlots;
+        // operands first (usually resident long before P_n is ready), then P_n
+        ok = __all_sync(kAll, tc::mbar_wait(bar(V_FULL + slot), (n / kVSlots) & 1, abort)) &&
+             (n + 2 >= T || wait_k(n + 2)) &&
+             __all_sync(kAll, tc::mbar_wait(bar(P_FULL + b), (n >> 1) & 1, abort));
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint64_t dv = dV + (uint32_t)(slot * L::kSlotBytes >> 4);
+        if (tc::elect_one()) {
+          // O += P_n V_n, A = P_n from TMEM buffer b
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t db = tc::sw128_desc(vb + kk * 2048, 8192, 1024);
-          tc::mma_bf16_ts(tO, tS0 + 64 * b + 8 * kk, db, kIdPV, (n > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16_ts(tO, tS0 + 64 * b + 8 * kk, dv + (uint32_t)(kk * 2048 >> 4), kIdPV,
+                            (n > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_commit(bar(O_DONE));
+          tc::mma_commit(bar(V_EMPTY + slot));
+          // buffer b is free once PV_n has read P_n: S_{n+2} goes in behind it
+          // (tcgen05 operations of one thread execute in issue order)
+          if (n + 2 < T) issue_s(n + 2);
         }
-        tc::mma_commit(bar(O_DONE));
-        tc::mma_commit(bar(V_EMPTY + slot));
-        // buffer b is free once PV_n has read P_n: S_{n+2} is issued behind it
-        if (n + 2 < T && !issue_s(n + 2)) {
-          ok = false;
-          break;
-        }
+        __syncwarp();
       }
       if (FUSE && ok) {
         // num = phi(Q) S'_i (M = 128 rows, N = D, K = D) into the S columns, one query
         // block at a time: the second waits until the first block's rows are read
         constexpr uint32_t kIdN = tc::idesc_bf16(128, D, false, true);
-        ok = tc::mbar_wait(bar(SP_FULL), 0, abort);
+        const uint64_t dS = tc::sw128_desc(sKV, D * 128, 1024);
+        ok = __all_sync(kAll, tc::mbar_wait(bar(SP_FULL), 0, abort));
         for (int hf = 0; hf < 2 && ok; ++hf) {
           if (!valid_h[hf]) break;
-          if (hf == 1 && !tc::mbar_wait(bar(NUM_READ), 0, abort)) {
+          if (hf == 1 && !__all_sync(kAll, tc::mbar_wait(bar(NUM_READ), 0, abort))) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          const uint32_t sb = sKV + hf * D * D * 2;
+          if (tc::elect_one()) {
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t da = tc::sw128_desc(sQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-            const uint64_t db = tc::sw128_desc(sb + k * 2048, D * 128, 1024);
-            tc::mma_bf16_ss(tS0, da, db, kIdN, k > 0);
+            for (int k = 0; k < D / 16; ++k)
+              tc::mma_bf16_ss(tS0, dQ + (uint32_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                              dS + (uint32_t)((hf * D * D * 2 + k * 2048) >> 4), kIdN, k > 0);
+            tc::mma_commit(bar(NUM_DONE + hf));
           }
-          tc::mma_commit(bar(NUM_DONE + hf));
+          __syncwarp();
         }
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         *abort = 1;
         report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
       }
