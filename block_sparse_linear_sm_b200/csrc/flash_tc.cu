@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   // barrier ids: K ring, V ring (full / empty per slot), S and P per TMEM buffer
   constexpr int Q_FULL = 0, K_FULL = 1, K_EMPTY = K_FULL + kKSlots, V_FULL = K_EMPTY + kKSlots,
                 V_EMPTY = V_FULL + kVSlots, S_FULL = V_EMPTY + kVSlots, P_FULL = S_FULL + 2,
-                O_DONE = P_FULL + 2, SP_FULL = O_DONE + 1, NUM_DONE = SP_FULL + 1,
+                O_DONE = P_FULL + 2, SP_FULL = O_DONE + 1, SP1_FULL = SP_FULL + 1, NUM_DONE = SP1_FULL + 1,
                 NUM_READ = NUM_DONE + 2;
   static_assert(NUM_READ < 32, "barrier area holds 32 mbarriers");
 
@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
     tc::mbar_init(bar(O_DONE), 1);
     tc::mbar_init(bar(SP_FULL), 1);
+    tc::mbar_init(bar(SP1_FULL), 1);
     tc::mbar_init(bar(NUM_DONE), 1);
     tc::mbar_init(bar(NUM_DONE + 1), 1);
     tc::mbar_init(bar(NUM_READ), 2);
@@ -279,34 +280,45 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           break;
         }
       }
-      // tail: wait for the last release of every slot, so that no tcgen05.commit
-      // arrival is still in flight when the CTA exits
+      // tail: wait for the last release of every K slot (every S product done)
       for (int n = (T > kKSlots ? T - kKSlots : 0); n < nk && !*abort; ++n)
         if (!tc::mbar_wait(bar(K_EMPTY + n % kKSlots), (n / kKSlots) & 1, abort)) {
           *abort = 1;
           report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
         }
-      for (int n = (T > kVSlots ? T - kVSlots : 0); n < nv && !*abort; ++n)
+    }
+    // Fused epilogue operands. The Q tiles and the K ring are free once every S
+    // product is done: they take phi(Q), S'_i of the first query block and Z_i of
+    // both, while the last P V products still run. S'_i of the second block goes
+    // to the V ring after its last release.
+    const int nh = valid_h[1] ? 2 : 1;
+    if (FUSE && lane == 0 && !*abort) {
+      tc::mbar_expect_tx(bar(SP_FULL), L::kQBytes + D * D * 2 + nh * D * 4);
+      for (int hf = 0; hf < 2; ++hf)
+        for (int p = 0; p < NP; ++p)
+          tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmF, bar(SP_FULL), 64 * p, i_h[hf] * kBlock,
+                          bh_h[hf]);
+      const int blk0 = bh_h[0] * prm.nb + i_h[0];
+      for (int p = 0; p < NP; ++p)
+        tc::tma_load_3d(sKV + p * D * 128, &tmS, bar(SP_FULL), 64 * p, 0, blk0);
+      for (int hf = 0; hf < nh; ++hf)
+        tc::bulk_load(sKV + D * D * 2 + hf * D * 4, prm.zs + (size_t)(bh_h[hf] * prm.nb + i_h[hf]) * D,
+                      D * 4, bar(SP_FULL));
+    }
+    if (lane == 0 && T > 0) {
+      // the last release of every V slot: no tcgen05.commit arrival is still in
+      // flight when the CTA exits, and the V ring is free
+      for (int n = (T > kVSlots ? T - kVSlots : 0); n < T && !*abort; ++n)
         if (!tc::mbar_wait(bar(V_EMPTY + n % kVSlots), (n / kVSlots) & 1, abort)) {
           *abort = 1;
           report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
         }
     }
-    if (FUSE && lane == 0 && !*abort) {
-      // every S and PV product has completed (the waits above): the rings take
-      // S'_i and Z_i of both query blocks, the Q tiles take phi(Q)
-      const int nh = valid_h[1] ? 2 : 1;
-      tc::mbar_expect_tx(bar(SP_FULL), nh * (D * D * 2 + D * 4) + L::kQBytes);
-      for (int hf = 0; hf < nh; ++hf) {
-        const int blk = bh_h[hf] * prm.nb + i_h[hf];
-        for (int p = 0; p < NP; ++p)
-          tc::tma_load_3d(sKV + hf * D * D * 2 + p * D * 128, &tmS, bar(SP_FULL), 64 * p, 0, blk);
-        tc::bulk_load(sKV + 2 * D * D * 2 + hf * D * 4, prm.zs + (size_t)blk * D, D * 4, bar(SP_FULL));
-      }
-      for (int hf = 0; hf < 2; ++hf)
-        for (int p = 0; p < NP; ++p)
-          tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmF, bar(SP_FULL), 64 * p, i_h[hf] * kBlock,
-                          bh_h[hf]);
+    if (FUSE && lane == 0 && !*abort && nh == 2) {
+      tc::mbar_expect_tx(bar(SP1_FULL), D * D * 2);
+      const int blk1 = bh_h[1] * prm.nb + i_h[1];
+      for (int p = 0; p < NP; ++p)
+        tc::tma_load_3d(sKV + kKSlots * L::kSlotBytes + p * D * 128, &tmS, bar(SP1_FULL), 64 * p, 0, blk1);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================================
@@ -373,7 +385,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         ok = __all_sync(kAll, tc::mbar_wait(bar(SP_FULL), 0, abort));
         for (int hf = 0; hf < 2 && ok; ++hf) {
           if (!valid_h[hf]) break;
-          if (hf == 1 && !__all_sync(kAll, tc::mbar_wait(bar(NUM_READ), 0, abort))) {
+          if (hf == 1 && !(__all_sync(kAll, tc::mbar_wait(bar(NUM_READ), 0, abort)) &&
+                           __all_sync(kAll, tc::mbar_wait(bar(SP1_FULL), 0, abort)))) {
             ok = false;
             break;
           }
@@ -382,7 +395,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
             for (int k = 0; k < D / 16; ++k)
               tc::mma_bf16_ss(tS0, dQ + (uint32_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                              dS + (uint32_t)((hf * D * D * 2 + k * 2048) >> 4), kIdN, k > 0);
+                              dS + (uint32_t)((hf * kKSlots * L::kSlotBytes + k * 2048) >> 4), kIdN, k > 0);
             tc::mma_commit(bar(NUM_DONE + hf));
           }
           __syncwarp();
@@ -522,7 +535,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL), 0, abort));
       float den = 0.f;
       if (ok && valid_h[hf]) {
-        const float4* z4 = reinterpret_cast<const float4*>(smem + L::kOffKV + 2 * D * D * 2 + hf * D * 4);
+        const float4* z4 = reinterpret_cast<const float4*>(smem + L::kOffKV + D * D * 2 + hf * D * 4);
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
           const uint4* frow = reinterpret_cast<const uint4*>(smem + L::kOffQ + p * 16384 + r * 128);
