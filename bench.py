@@ -407,7 +407,8 @@ def main():
         if kind == "tensor":
             ach = work / t / 1e12
             stages[n] = {"ms": stage_ms[n], "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
-                         "frac_of_sustained": ach / peaks["bf16_sus"], "work": work}
+                         "frac": ach / peaks["bf16"], "frac_of_sustained": ach / peaks["bf16_sus"],
+                         "work": work}
         else:
             ach = work / t / 1e9
             stages[n] = {"ms": stage_ms[n], "bound": "hbm", "achieved": ach, "unit": "GB/s",
@@ -416,9 +417,13 @@ def main():
     kernel_of = {"sparse_flash": "flash_tc_kernel"}
     dk = stages[dom]
     if dk["bound"] == "tensor":
-        roof = {"kernel": dom, "bound": "tensor", "achieved": dk["achieved"], "peak": peaks["bf16_sus"],
-                "unit": "TFLOP/s", "frac": dk["achieved"] / peaks["bf16_sus"],
-                "peak_kind": f"bf16 sustained, {peaks['src']}",
+        # The layer's kernels run a few ms at a time at full SM clock (see "clocks"),
+        # so the burst GEMM figure is the denominator; the sustained one (taken at
+        # the power-capped clock of a seconds-long loop) is given beside it.
+        roof = {"kernel": dom, "bound": "tensor", "achieved": dk["achieved"], "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "frac": dk["achieved"] / peaks["bf16"],
+                "peak_kind": f"bf16 burst, {peaks['src']}",
+                "peak_sustained": peaks["bf16_sus"], "frac_of_sustained": dk["achieved"] / peaks["bf16_sus"],
                 "traffic": measured_traffic(kernel_of.get(dom, dom), cfg.name),
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"}
     else:
@@ -427,7 +432,7 @@ def main():
                 "peak_kind": f"HBM copy, {peaks['src']}", "traffic": None}
     if "sparse_flash" in stages and dom != "sparse_flash":
         fk = stages["sparse_flash"]
-        roof["flash"] = {"achieved": fk["achieved"], "frac": fk["achieved"] / peaks["bf16_sus"]}
+        roof["flash"] = {"achieved": fk["achieved"], "frac": fk["achieved"] / peaks["bf16"]}
 
     clocks = clk.summary()
     c2 = clk2.summary()
