@@ -212,6 +212,22 @@ def measured_traffic(kernel: str, workload: str):
     return None
 
 
+def max_over_ranks(dist, device, *vals):
+    """The max of each value over all ranks (one all-reduce); the values themselves
+    without a process group."""
+    if dist is None:
+        return [float(v) for v in vals]
+    import torch
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world, flop_per_rank, ms_per_step):
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return world * flop_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def units_total(cfg):
     return cfg.B * cfg.H * cfg.nqb
 
@@ -352,11 +368,7 @@ def main():
     st, detail = sla.sla_check_device_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st} detail {detail}")
-    ms_total = g0.elapsed_time(g1)
-    if dist is not None:
-        tt = torch.tensor([ms_total, ms_eager], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total, ms_eager = float(tt[0].item()), float(tt[1].item())
+    ms_total, ms_eager = max_over_ranks(dist, dev, g0.elapsed_time(g1), ms_eager)
     ms_step = ms_total / args.steps
     del graph
     stage_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
@@ -387,16 +399,12 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    (e2e_ms,) = max_over_ranks(dist, dev, e0.elapsed_time(e1) / args.e2e_steps)
     barrier()
 
     flops = cfg.dense_flops()
-    value = world * flops / (ms_step * 1e-3) / 1e12
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops, ms_step)
+    e2e_value = job_throughput(world, flops, e2e_ms)
 
     peaks = load_peaks()
     model = stage_model(cfg)
