@@ -23,12 +23,14 @@ static sla_status check_config(const sla_config* c) {
   if (c->mode == SLA_MODE_THREEWAY) {
     if (c->k_h < 0 || c->k_l < 0 || c->k_h + c->k_l > nb) return SLA_ERR_INVALID_ARG;
     if (c->causal != 0) return SLA_ERR_UNSUPPORTED;
-    if ((c->has_proj != 0 && c->has_proj != 1) || (c->has_gate != 0 && c->has_gate != 1))
+    if ((c->has_proj != 0 && c->has_proj != 1) || (c->has_gate != 0 && c->has_gate != 1) ||
+        (c->proj_per_head != 0 && c->proj_per_head != 1))
       return SLA_ERR_INVALID_ARG;
+    if (c->proj_per_head && (!c->has_proj || c->H_kv != c->H)) return SLA_ERR_UNSUPPORTED;
   } else if (c->mode == SLA_MODE_TOPN_WINDOW) {
     if (c->top_n < 0 || c->window < 0) return SLA_ERR_INVALID_ARG;
     if (c->causal != 1) return SLA_ERR_UNSUPPORTED;
-    if (c->has_proj != 0 || c->has_gate != 0) return SLA_ERR_UNSUPPORTED;
+    if (c->has_proj != 0 || c->has_gate != 0 || c->proj_per_head != 0) return SLA_ERR_UNSUPPORTED;
     // selected blocks plus window blocks must fit the kernel's 128-entry list
     if (c->top_n > 64 || c->top_n + (c->window + 62) / kBlock + 1 > 128) return SLA_ERR_UNSUPPORTED;
   } else {

@@ -46,6 +46,7 @@ struct StateParams {
   __nv_bfloat16* hs;
   int* status;
   int nkb, nkb_pad, dd, n_valid, has_proj;
+  int wp_heads;  // 1: one W_p for all heads; H: W_p[h] for KV head h (H_kv == H)
 };
 
 template <int D>
@@ -94,7 +95,8 @@ __global__ void __launch_bounds__(kStThreads, 2)
       for (int p = 0; p < L::NP; ++p)
         tc::tma_load_3d(sV + p * 16384, &tmV, bar(LOADED), 64 * p, j0 * kBlock, bkv);
       if (proj)
-        for (int p = 0; p < L::NP; ++p) tc::tma_load_3d(sW + p * D * 128, &tmW, bar(LOADED), 64 * p, 0, 0);
+        for (int p = 0; p < L::NP; ++p)
+          tc::tma_load_3d(sW + p * D * 128, &tmW, bar(LOADED), 64 * p, 0, bkv % prm.wp_heads);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -274,8 +276,9 @@ static cudaError_t launch_state_t(const Plan& p, const Args& a, cudaStream_t s) 
                     64, D))
     return cudaErrorInvalidValue;
   // without a projection the W_p map is never used; encode it over K to keep it valid
-  if (!make_tmap_3d(&mw, proj ? (const void*)a.w_p : (const void*)a.k, D, D, 1, rowb, (uint64_t)D * rowb,
-                    64, D))
+  const int wp_heads = proj && c.proj_per_head ? c.H : 1;
+  if (!make_tmap_3d(&mw, proj ? (const void*)a.w_p : (const void*)a.k, D, D, (uint64_t)wp_heads, rowb,
+                    (uint64_t)D * rowb, 64, D))
     return cudaErrorInvalidValue;
   StateParams prm;
   prm.hs = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_hs);
@@ -285,6 +288,7 @@ static cudaError_t launch_state_t(const Plan& p, const Args& a, cudaStream_t s) 
   prm.dd = p.dd;
   prm.n_valid = c.N_valid;
   prm.has_proj = proj ? 1 : 0;
+  prm.wp_heads = wp_heads;
   cudaError_t e = cudaFuncSetAttribute(state_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::kSmem);
   if (e != cudaSuccess) return e;

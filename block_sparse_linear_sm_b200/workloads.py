@@ -56,6 +56,7 @@ class LayerConfig:
     window: int = 0
     causal: int = 0
     has_proj: int = 1
+    proj_per_head: int = 0        # 1: one W_p per query head ([H, d, d])
     has_gate: int = 0
     scale: float = 0.0            # 0 -> 1/sqrt(d)
     generator: str = "iid"        # iid | fourier | block_shift
@@ -157,7 +158,7 @@ class LayerInputs:
     q: np.ndarray                  # [B, H, N, d]
     k: np.ndarray                  # [B, H_kv, N, d]
     v: np.ndarray                  # [B, H_kv, N, d]
-    w_p: Optional[np.ndarray]      # [d, d] or None
+    w_p: Optional[np.ndarray]      # [d, d], [H, d, d] (per-head projection) or None
     w_g: Optional[np.ndarray]      # [H, d] or None
     extra: dict = field(default_factory=dict)
 
@@ -222,7 +223,8 @@ def generate(cfg: LayerConfig, v_shift: float = 0.0) -> LayerInputs:
             else:
                 q[b, h, :Nv] = to_bf16_bits(rng.standard_normal((Nv, d), dtype=np.float32))
     wrng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(cfg.seed).spawn(4)[3]))
-    w_p = to_bf16_bits(wrng.normal(0.0, 1.0 / math.sqrt(d), size=(d, d))) if cfg.has_proj else None
+    wp_shape = (H, d, d) if cfg.proj_per_head else (d, d)
+    w_p = to_bf16_bits(wrng.normal(0.0, 1.0 / math.sqrt(d), size=wp_shape)) if cfg.has_proj else None
     w_g = to_bf16_bits(wrng.normal(0.0, 1.0 / math.sqrt(d), size=(H, d))) if cfg.has_gate else None
     return LayerInputs(cfg, q, k, v, w_p, w_g)
 

@@ -44,7 +44,8 @@
  *   frees all of them; the library never allocates):
  *     q    bf16 [B, H,    N, d]
  *     k, v bf16 [B, H_kv, N, d]
- *     w_p  bf16 [d, d]   (row vector times matrix: O_l W_p), ignored unless has_proj
+ *     w_p  bf16 [d, d]   (row vector times matrix: O_l W_p), ignored unless has_proj;
+ *          [H, d, d] with proj_per_head (head h uses w_p[h])
  *     w_g  bf16 [H, d]   ignored unless has_gate
  *     out  bf16 [B, H, N, d]
  *   Tokens at index >= N_valid are padding: they are left out of pooling,
@@ -108,6 +109,10 @@ typedef struct {
   int32_t window;   /* TOPN_WINDOW: window tokens t-window+1 .. t, >= 0 */
   int32_t causal;   /* must be 1 in TOPN_WINDOW and 0 in THREEWAY */
   int32_t has_proj; /* THREEWAY: 1 = apply w_p to O_l, 0 = identity */
+  int32_t proj_per_head; /* THREEWAY with has_proj: 0 = one w_p [d, d] shared by all heads;
+                          * 1 = one per query head, w_p [H, d, d]; needs H_kv == H (the
+                          * projection is folded into per-KV-head states), else
+                          * SLA_ERR_UNSUPPORTED */
   int32_t has_gate; /* THREEWAY: 1 = g = sigmoid(q . w_g[h]), 0 = g = 1 */
   float scale;      /* softmax scale of pooled scores and attention; 0 = 1/sqrt(d) */
 } sla_config;

@@ -222,12 +222,14 @@ class OracleCfg:
     window: int = 0
     causal: int = 0
     has_proj: int = 1
+    proj_per_head: int = 0
     has_gate: int = 0
     scale: float = 0.0
 
     @classmethod
     def of(cls, c) -> "OracleCfg":
-        return cls(**{f: getattr(c, f) for f in cls.__dataclass_fields__})
+        return cls(**{f: getattr(c, f, 0) if f == "proj_per_head" else getattr(c, f)
+                      for f in cls.__dataclass_fields__})
 
     @property
     def nb(self) -> int:
@@ -250,7 +252,10 @@ class Layer:
         c = self.c
         assert c.N % c.block == 0 and c.H % c.H_kv == 0
         self.q, self.k, self.v = q, k, v
+        # W_p: one d x d matrix shared by the heads, or one per query head ([H, d, d])
         self.w_p = w_p if c.has_proj else None
+        if self.w_p is not None:
+            assert self.w_p.shape == ((c.H, c.d, c.d) if c.proj_per_head else (c.d, c.d))
         self.w_g = w_g if c.has_gate else None
         self._kbar: Dict[Tuple[int, int], np.ndarray] = {}
         self._scores: Dict[Tuple[int, int], np.ndarray] = {}
@@ -337,7 +342,8 @@ class Layer:
             else:
                 o_l = np.zeros_like(qr)
             w_g = self.w_g[h] if self.w_g is not None else None
-            o = combine(o_s, o_l, qr, self.w_p, w_g)
+            w_p = self.w_p[h] if self.w_p is not None and c.proj_per_head else self.w_p
+            o = combine(o_s, o_l, qr, w_p, w_g)
         else:
             sel = self.selection(b, hk)[0][i] if sel_row is None else sel_row
             # candidate tokens: selected blocks plus the blocks the window can reach

@@ -59,6 +59,10 @@ BAD = [
     (dict(mode=1, causal=1, top_n=65, has_proj=0), sla.SLA_ERR_UNSUPPORTED),
     (dict(mode=1, causal=1, top_n=4, has_proj=1), sla.SLA_ERR_UNSUPPORTED),
     (dict(mode=7), sla.SLA_ERR_INVALID_ARG),
+    (dict(proj_per_head=2), sla.SLA_ERR_INVALID_ARG),
+    (dict(proj_per_head=1, has_proj=0), sla.SLA_ERR_UNSUPPORTED),
+    (dict(proj_per_head=1, H=4, H_kv=2), sla.SLA_ERR_UNSUPPORTED),
+    (dict(mode=1, causal=1, top_n=4, has_proj=0, proj_per_head=1), sla.SLA_ERR_UNSUPPORTED),
     (dict(scale=-1.0), sla.SLA_ERR_INVALID_ARG),
     (dict(scale=float("nan")), sla.SLA_ERR_INVALID_ARG),
 ]
@@ -130,3 +134,9 @@ def test_workspace_grows_with_the_problem():
     b = wl.small_config(N=2048, N_valid=2048)
     assert sla.sla_workspace_bytes(b) > sla.sla_workspace_bytes(a)
     assert sla.sla_workspace_bytes(a) % 256 == 0
+
+
+def test_per_head_projection_is_accepted_with_one_kv_head_per_query_head():
+    c = wl.small_config(N=1024, N_valid=1000, H=4, H_kv=4, proj_per_head=1)
+    assert sla.sla_validate_config(c) == sla.SLA_OK
+    assert sla.sla_workspace_bytes(c) == sla.sla_workspace_bytes(wl.small_config(N=1024, N_valid=1000, H=4, H_kv=4))

@@ -49,6 +49,10 @@ SMALL_CASES = [
     dict(name="odd_blocks", N=1216, N_valid=1200, d=128, k_h=3, k_l=4, has_gate=1),
     dict(name="odd_blocks_d64", N=1216, N_valid=1216, d=64, k_h=5, k_l=0),
     dict(name="single_block", N=64, N_valid=50, d=128, k_h=1, k_l=0),
+    dict(name="per_head_proj_d128", N=1536, N_valid=1500, d=128, H=4, H_kv=4, k_h=3, k_l=4,
+         proj_per_head=1, has_gate=1),
+    dict(name="per_head_proj_d64", N=1024, N_valid=1024, d=64, H=3, H_kv=3, k_h=2, k_l=3,
+         proj_per_head=1),
 ]
 
 
@@ -108,6 +112,23 @@ def test_mixed_layer_shifted_values_linear_branch():
     got_l = got - ref["O_s"][:, :, :cfg.N_valid]
     rel = np.linalg.norm(got_l - want_l) / np.linalg.norm(want_l)
     print("mixed: linear branch relative Frobenius error", rel)
+    assert rel <= 1e-2
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_per_head_projection_linear_term_shifted_values(d):
+    """One W_p per head, gate on, V + 3: the projected, gated linear term O - O_s is O(1)
+    and differs per head."""
+    cfg = small(name="per_head_shift", N=2048, N_valid=2030, d=d, H=4, H_kv=4, k_h=4, k_l=6,
+                proj_per_head=1, has_gate=1)
+    x = wl.generate(cfg, v_shift=3.0)
+    run = GpuRun(cfg, x)
+    ref = run.layer().forward()
+    n = cfg.N_valid
+    got_l = run.O()[:, :, :n] - ref["O_s"][:, :, :n]
+    want_l = ref["O"][:, :, :n] - ref["O_s"][:, :, :n]
+    rel = np.linalg.norm(got_l - want_l) / np.linalg.norm(want_l)
+    print("per-head projection: linear term relative Frobenius error", rel)
     assert rel <= 1e-2
 
 

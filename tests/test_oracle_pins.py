@@ -29,7 +29,7 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 class Cfg:
     def __init__(self, **kw):
         base = dict(B=1, H=2, H_kv=2, N=256, N_valid=256, d=16, block=32, mode=0, k_h=2, k_l=2,
-                    top_n=0, window=0, causal=0, has_proj=1, has_gate=0, scale=0.0)
+                    top_n=0, window=0, causal=0, has_proj=1, proj_per_head=0, has_gate=0, scale=0.0)
         base.update(kw)
         self.__dict__.update(base)
 
@@ -45,7 +45,13 @@ def rand_inputs(c, seed=0, v_shift=0.0):
     v[:, :, c.N_valid:] = 0
     w_p = rng.normal(0, 1 / math.sqrt(c.d), (c.d, c.d))
     w_g = rng.normal(0, 1 / math.sqrt(c.d), (c.H, c.d))
+    if getattr(c, "proj_per_head", 0):
+        w_p = rng.normal(0, 1 / math.sqrt(c.d), (c.H, c.d, c.d))
     return q, k, v, w_p, w_g
+
+
+def wp_of(c, w_p, h):
+    return w_p[h] if getattr(c, "proj_per_head", 0) else w_p
 
 
 def scale_of(c):
@@ -112,7 +118,7 @@ def brute_threeway(c, q, k, v, w_p, w_g):
             a = (fq @ fk.T) * marg
             den = a.sum(1)
             o_l = np.where(den[:, None] > 0, (a @ v[b, hk]) / np.where(den > 0, den, 1)[:, None], 0)
-            proj = o_l @ w_p if c.has_proj else o_l
+            proj = o_l @ wp_of(c, w_p, h) if c.has_proj else o_l
             gate = torch.sigmoid(torch.from_numpy(q[b, h] @ w_g[h])).numpy() if c.has_gate else 1.0
             o = o_s + (gate[:, None] if c.has_gate else 1.0) * proj
             o[~valid] = 0
@@ -183,7 +189,7 @@ def pin_all_marginal(c, seed=2, v_shift=0.0):
             a = fq @ fk.T                                   # quadratic form, N x N
             ol = (a @ torch.from_numpy(v[b, h // g])) / a.sum(1, keepdim=True)
             if c.has_proj:
-                ol = ol @ torch.from_numpy(w_p)
+                ol = ol @ torch.from_numpy(wp_of(c, w_p, h))
             if c.has_gate:
                 ol = torch.sigmoid(torch.from_numpy(q[b, h]) @ torch.from_numpy(w_g[h]))[:, None] * ol
             ref[b, h] = ol.numpy()
@@ -412,3 +418,30 @@ def test_planted_window_off_by_one_is_caught(monkeypatch):
             self.c.window -= 1
     monkeypatch.setattr(so.Layer, "unit", bad_unit)
     assert pin_brute_topn(Cfg(H=4, H_kv=2, mode=1, top_n=3, window=80, causal=1)) > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# projection per query head (w_p [H, d, d]; the scope table's boundary sketch
+# allows W_p shared or per head)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kw", [dict(), dict(N_valid=250, has_gate=1), dict(H=3, H_kv=3, k_h=1, k_l=3)])
+def test_per_head_projection_matches_brute_force(kw):
+    assert pin_brute_threeway(Cfg(proj_per_head=1, **kw)) < 1e-12
+
+
+def test_per_head_projection_all_marginal_closed_form():
+    assert pin_all_marginal(Cfg(proj_per_head=1, H=3, H_kv=3, has_gate=1)) < 1e-12
+
+
+def test_per_head_projection_with_equal_matrices_is_the_shared_one():
+    c = Cfg(N_valid=250)
+    q, k, v, w_p, w_g = rand_inputs(c, 11)
+    shared = oracle.forward(c, q, k, v, w_p, w_g)["O"]
+    c2 = Cfg(N_valid=250, proj_per_head=1)
+    per_head = oracle.forward(c2, q, k, v, np.stack([w_p] * c2.H), w_g)["O"]
+    assert np.array_equal(shared, per_head)
+    # distinct matrices per head change only the heads whose matrix changed
+    w3 = np.stack([w_p, 2.0 * w_p])
+    o3 = oracle.forward(c2, q, k, v, w3, w_g)["O"]
+    assert np.array_equal(o3[:, 0], shared[:, 0]) and not np.allclose(o3[:, 1], shared[:, 1])
