@@ -7,17 +7,21 @@
 //
 //   C[i, :] = sum_j M[i, j] * Hs[j, :]     M: 0/1 marginal mask (exact in bf16)
 //
-// with C = [S_i | Z_i] row by row. One CTA computes a 256 (query blocks) x 256
-// (state columns) tile as two M = 128 tcgen05 accumulators (all 512 TMEM
-// columns), K = key blocks in steps of 64; A (the mask, K-major) and B (the
-// states, N-major) come by TMA through a 3-stage ring. Large tiles keep the
-// operand re-reads through L2 low: every state tile is read by nqb/256 CTAs,
-// every mask tile by dd/256. The grid runs the query-block tiles of one column
-// tile next to each other so a tile of states comes from HBM once.
+// with C = [S_i | Z_i] row by row.
 //
-// Warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2-5 = epilogue
-// (S_i columns to bf16 staged for TMA stores, Z_i columns to fp32, padding
-// columns dropped).
+// Persistent kernel, one CTA per SM. Output tiles are 128 (query blocks) x 256
+// (state columns), K = key blocks in steps of 64. The tile order runs the
+// query-block tiles of one column tile next to each other, so a tile of states
+// comes from HBM once and from L2 for its other users. TMEM holds two
+// accumulators (2 x 256 columns): the MMA warp fills one while the epilogue
+// warps drain the other, so a tile's epilogue (TMEM to registers to a
+// 128-byte-swizzled staging buffer to TMA stores) overlaps the next tile's
+// main loop.
+//
+// Warps: 0 = TMA producer (A = mask, K-major; B = states, N-major; 3-stage
+// ring), 1 = TMEM owner and MMA issuer (whole warp, one elected lane issues),
+// 2-5 = epilogue (S_i columns to bf16 through the staging buffer, Z_i columns
+// straight to HBM as fp32, padding columns dropped).
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -25,18 +29,20 @@ namespace sla {
 
 constexpr int kAgStages = 3;
 constexpr int kAgThreads = 192;
-constexpr int kAgBM = 256, kAgBN = 256;
-constexpr int kAgA = kAgBM * 64 * 2;  // mask tile: 256 rows x 64 k, two 128-row boxes
-constexpr int kAgB = 64 * kAgBN * 2;  // state tile: 64 k-rows x 256 columns, four panels
-constexpr int kAgStage = kAgA + kAgB;
-constexpr int kAgOffBar = kAgStages * kAgStage;
-constexpr int kAgSmem = kAgOffBar + 128;
+constexpr int kAgBM = 128, kAgBN = 256;
+constexpr int kAgA = kAgBM * 64 * 2;          // mask tile: 128 rows x 64 k
+constexpr int kAgB = 64 * kAgBN * 2;          // state tile: 64 k-rows x 256 columns, four panels
+constexpr int kAgStage = kAgA + kAgB;         // 48 KB
+constexpr int kAgOffStage = kAgStages * kAgStage;
+constexpr int kAgStaging = kAgBM * kAgBN * 2;  // 64 KB: four 64-column panels of 128 rows
+constexpr int kAgOffBar = kAgOffStage + kAgStaging;
+constexpr int kAgSmem = kAgOffBar + 256;
 
 struct AggParams {
-  __nv_bfloat16* ss;  // [B*H][nqb][d*d]
-  float* zs;          // [B*H][nqb][d]
+  float* zs;  // [B*H][nqb][d]
   int* status;
   int H, group, nqb, nk_steps, d;
+  int m_tiles, n_tiles, tiles;  // tile t: m = t % m_tiles, n = (t / m_tiles) % n_tiles, bh = rest
 };
 
 __global__ void __launch_bounds__(kAgThreads, 1)
@@ -49,24 +55,25 @@ __global__ void __launch_bounds__(kAgThreads, 1)
     if (tid == 0) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashAlign);
     return;
   }
-  const int mt = blockIdx.x, nt = blockIdx.y, bh = blockIdx.z;
-  const int m0 = mt * kAgBM, n0 = nt * kAgBN;
-  const int b = bh / prm.H, h = bh % prm.H;
-  const int bkv = b * (prm.H / prm.group) + h / prm.group;
-  volatile int* misc = reinterpret_cast<volatile int*>(smem + kAgOffBar + 64);  // tmem, abort
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + kAgOffBar + 128);  // tmem, abort
   auto bar = [&](int k) -> uint32_t { return sbase + kAgOffBar + 8 * k; };
-  constexpr int FULL = 0, EMPTY = kAgStages, DONE = 2 * kAgStages;
+  // ring full / empty per stage; accumulator full / empty per TMEM buffer
+  constexpr int FULL = 0, EMPTY = kAgStages, ACC_FULL = 2 * kAgStages, ACC_EMPTY = ACC_FULL + 2;
+  static_assert(ACC_EMPTY + 2 <= 16, "barrier area holds 16 mbarriers");
   if (tid == 0) {
     misc[1] = 0;
     for (int s = 0; s < kAgStages; ++s) {
       tc::mbar_init(bar(FULL + s), 1);
       tc::mbar_init(bar(EMPTY + s), 1);
     }
-    tc::mbar_init(bar(DONE), 1);
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(bar(ACC_FULL + a), 1);
+      tc::mbar_init(bar(ACC_EMPTY + a), 4);
+    }
     tc::fence_mbar_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(sbase + kAgOffBar + 64, 512);
+    tc::tmem_alloc(sbase + kAgOffBar + 128, 512);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -75,83 +82,115 @@ __global__ void __launch_bounds__(kAgThreads, 1)
   const uint32_t tmem = (uint32_t)misc[0];
   volatile int* abort = misc + 1;
   const int K = prm.nk_steps;
+  // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int my_tiles = prm.tiles > (int)blockIdx.x ? (prm.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto tile_of = [&](int i, int& m0, int& n0, int& bh) {
+    const int t = (int)blockIdx.x + i * (int)gridDim.x;
+    m0 = (t % prm.m_tiles) * kAgBM;
+    n0 = ((t / prm.m_tiles) % prm.n_tiles) * kAgBN;
+    bh = t / (prm.m_tiles * prm.n_tiles);
+  };
 
   if (warp == 0) {
+    // ======================= TMA producer =====================================
     if (lane == 0) {
       tc::prefetch_tensormap(&tmA);
       tc::prefetch_tensormap(&tmB);
-      for (int k = 0; k < K; ++k) {
-        const int st = k % kAgStages;
-        if (k >= kAgStages && !tc::mbar_wait(bar(EMPTY + st), ((k / kAgStages) - 1) & 1, abort)) {
-          *abort = 1;
-          report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
-          break;
+      int kg = 0;  // ring use counter over all tiles
+      for (int i = 0; i < my_tiles && !*abort; ++i) {
+        int m0, n0, bh;
+        tile_of(i, m0, n0, bh);
+        const int bkv = (bh / prm.H) * (prm.H / prm.group) + (bh % prm.H) / prm.group;
+        for (int k = 0; k < K; ++k, ++kg) {
+          const int st = kg % kAgStages;
+          if (kg >= kAgStages && !tc::mbar_wait(bar(EMPTY + st), ((kg / kAgStages) - 1) & 1, abort)) {
+            *abort = 1;
+            report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+            break;
+          }
+          const uint32_t a_s = sbase + st * kAgStage, b_s = a_s + kAgA;
+          tc::mbar_expect_tx(bar(FULL + st), kAgStage);
+          tc::tma_load_3d(a_s, &tmA, bar(FULL + st), k * 64, m0, bh);
+          for (int p = 0; p < 4; ++p)
+            tc::tma_load_3d(b_s + p * 8192, &tmB, bar(FULL + st), n0 + 64 * p, k * 64, bkv);
         }
-        const uint32_t a_s = sbase + st * kAgStage, b_s = a_s + kAgA;
-        tc::mbar_expect_tx(bar(FULL + st), kAgStage);
-        tc::tma_load_3d(a_s, &tmA, bar(FULL + st), k * 64, m0, bh);
-        tc::tma_load_3d(a_s + 16384, &tmA, bar(FULL + st), k * 64, m0 + 128, bh);
-        for (int p = 0; p < 4; ++p)
-          tc::tma_load_3d(b_s + p * 8192, &tmB, bar(FULL + st), n0 + 64 * p, k * 64, bkv);
       }
       // tail: every stage's last release has landed before the CTA exits
-      for (int k = (K > kAgStages ? K - kAgStages : 0); k < K && !*abort; ++k)
-        if (!tc::mbar_wait(bar(EMPTY + k % kAgStages), (k / kAgStages) & 1, abort)) {
+      for (int u = (kg > kAgStages ? kg - kAgStages : 0); u < kg && !*abort; ++u)
+        if (!tc::mbar_wait(bar(EMPTY + u % kAgStages), (u / kAgStages) & 1, abort)) {
           *abort = 1;
           report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
         }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t kId = tc::idesc_bf16(128, kAgBN, false, true);
-      bool ok = true;
-      for (int k = 0; k < K; ++k) {
-        const int st = k % kAgStages;
-        if (!tc::mbar_wait(bar(FULL + st), (k / kAgStages) & 1, abort)) {
+    // ======================= MMA issuer =======================================
+    constexpr uint32_t kId = tc::idesc_bf16(kAgBM, kAgBN, false, true);
+    constexpr uint32_t kAll = 0xffffffffu;
+    const uint64_t dA = tc::sw128_desc(sbase, 16, 1024);
+    const uint64_t dB = tc::sw128_desc(sbase + kAgA, 8192, 1024);
+    bool ok = true;
+    int kg = 0;
+    for (int i = 0; i < my_tiles && ok; ++i) {
+      const int acc = i & 1, use = i >> 1;
+      // the epilogue has read this accumulator's previous tile
+      if (use > 0 && !__all_sync(kAll, tc::mbar_wait(bar(ACC_EMPTY + acc), (use - 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      for (int k = 0; k < K; ++k, ++kg) {
+        const int st = kg % kAgStages;
+        if (!__all_sync(kAll, tc::mbar_wait(bar(FULL + st), (kg / kAgStages) & 1, abort))) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t a_s = sbase + st * kAgStage, b_s = a_s + kAgA;
+        const uint32_t so = (uint32_t)(st * kAgStage) >> 4;
+        if (tc::elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t db = tc::sw128_desc(b_s + kk * 2048, 8192, 1024);
-#pragma unroll
-          for (int mh = 0; mh < 2; ++mh) {
-            const uint64_t da = tc::sw128_desc(a_s + mh * 16384 + kk * 32, 16, 1024);
-            tc::mma_bf16_ss(tmem + mh * kAgBN, da, db, kId, (k > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16_ss(tmem + acc * kAgBN, dA + so + (uint32_t)(kk * 32 >> 4),
+                            dB + so + (uint32_t)(kk * 2048 >> 4), kId, (k > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_commit(bar(EMPTY + st));
+          if (k == K - 1) tc::mma_commit(bar(ACC_FULL + acc));
         }
-        tc::mma_commit(bar(EMPTY + st));
-      }
-      if (ok) tc::mma_commit(bar(DONE));
-      if (!ok) {
-        *abort = 1;
-        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+        __syncwarp();
       }
     }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
   } else {
-    // epilogue: thread = query block (TMEM lane) of each 128-row half. S_i columns
-    // are staged as bf16 in the freed stage ring (per half: four 64-column
-    // panels of 128 rows, 128-byte swizzled) and written by TMA stores; Z_i
-    // columns go straight to HBM as fp32.
+    // ======================= epilogue =========================================
+    // thread = query block (TMEM lane) of the tile's 128 rows
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const bool ok = __all_sync(0xffffffffu, K > 0 && tc::mbar_wait(bar(DONE), 0, abort));
-    tc::fence_after_sync();
     const int dsq = prm.d * prm.d;
-    for (int mh = 0; mh < 2 && ok; ++mh) {
-      const int row = m0 + mh * 128 + r;
+    const uint32_t stg = sbase + kAgOffStage;
+    // Every epilogue warp runs both named barriers of every tile, also after a
+    // failed wait (it then skips the work), so no warp is left at a barrier.
+    bool ok = true;
+    for (int i = 0; i < my_tiles; ++i) {
+      int m0, n0, bh;
+      tile_of(i, m0, n0, bh);
+      const int acc = i & 1, use = i >> 1;
+      ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(ACC_FULL + acc), use & 1, abort));
+      tc::fence_after_sync();
+      // the previous tile's TMA stores have finished reading the staging buffer
+      if (r == 0) tc::bulk_wait_read_all();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int row = m0 + r;
 #pragma unroll 1
-      for (int c64 = 0; c64 < kAgBN / 64; ++c64) {
+      for (int c64 = 0; c64 < kAgBN / 64 && ok; ++c64) {
         uint32_t v[2][32];
-        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + mh * kAgBN + 64 * c64;
+        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + acc * kAgBN + 64 * c64;
         tc::tmem_ld32(ta, v[0]);
         tc::tmem_ld32(ta + 32, v[1]);
         tc::tmem_ld_wait();
         const int col = n0 + 64 * c64;
         if (col < dsq) {
-          uint4* srow = reinterpret_cast<uint4*>(smem + mh * 65536 + c64 * 16384 + r * 128);
+          uint4* srow = reinterpret_cast<uint4*>(smem + kAgOffStage + c64 * 16384 + r * 128);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint32_t* vv = v[q >> 2] + 8 * (q & 3);
@@ -173,17 +212,23 @@ __global__ void __launch_bounds__(kAgThreads, 1)
           }
         }
       }
-    }
-    tc::fence_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok && quarter == 0 && lane == 0) {
-      // rows past nqb and columns past d*d fall outside the map and are not written
-      for (int mh = 0; mh < 2; ++mh)
+      // the accumulator is read: the MMA warp may start the tile after next in it
+      tc::fence_before_sync();
+      __syncwarp();
+      if (ok && lane == 0) tc::mbar_arrive(bar(ACC_EMPTY + acc));
+      tc::fence_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (ok && r == 0 && m0 < prm.nqb) {
+        // rows past nqb and columns past d*d fall outside the map and are not written
         for (int c64 = 0; c64 < kAgBN / 64; ++c64)
-          if (n0 + 64 * c64 < dsq && m0 + mh * 128 < prm.nqb)
-            tc::tma_store_3d(&tmS, sbase + mh * 65536 + c64 * 16384, n0 + 64 * c64, m0 + mh * 128, bh);
-      tc::bulk_commit();
-      tc::bulk_wait_all();
+          if (n0 + 64 * c64 < dsq) tc::tma_store_3d(&tmS, stg + c64 * 16384, n0 + 64 * c64, m0, bh);
+        tc::bulk_commit();
+      }
+    }
+    if (r == 0) tc::bulk_wait_all();
+    if (!ok && lane == 0) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
     }
   }
   tc::fence_before_sync();
@@ -212,7 +257,6 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
                     (uint64_t)p.nqb * dsq * 2, 64, 128))
     return cudaErrorInvalidValue;
   AggParams prm;
-  prm.ss = reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_ss);
   prm.zs = reinterpret_cast<float*>(a.ws + p.off_zs);
   prm.status = a.status;
   prm.H = c.H;
@@ -220,10 +264,16 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
   prm.nqb = p.nqb;
   prm.nk_steps = p.nkb_pad / 64;
   prm.d = c.d;
+  prm.m_tiles = (p.nqb + kAgBM - 1) / kAgBM;
+  prm.n_tiles = (p.dd + kAgBN - 1) / kAgBN;
+  prm.tiles = prm.m_tiles * prm.n_tiles * c.B * c.H;
   cudaError_t e = cudaFuncSetAttribute(aggregate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kAgSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.nqb_pad + kAgBM - 1) / kAgBM, (p.dd + kAgBN - 1) / kAgBN, c.B * c.H);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = prm.tiles < sms ? prm.tiles : sms;  // one persistent CTA per SM
   aggregate_tc_kernel<<<grid, kAgThreads, kAgSmem, s>>>(ma, mb, ms, prm);
   return cudaGetLastError();
 }
