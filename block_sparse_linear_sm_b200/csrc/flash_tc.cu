@@ -166,6 +166,15 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     tc::mbar_init(bar(NUM_DONE + 1), 1);
     tc::mbar_init(bar(NUM_READ), 2);
     tc::fence_mbar_init();
+    // Q does not depend on the block lists: its load overlaps the list merge
+    tc::prefetch_tensormap(&tmQ);
+    tc::prefetch_tensormap(&tmK);
+    tc::prefetch_tensormap(&tmV);
+    tc::mbar_expect_tx(bar(Q_FULL), L::kQBytes);
+    for (int hf = 0; hf < 2; ++hf)
+      for (int p = 0; p < NP; ++p)
+        tc::tma_load_3d(sbase + L::kOffQ + p * 16384 + hf * 8192, &tmQ, bar(Q_FULL), 64 * p,
+                        i_h[hf] * kBlock, bh_h[hf]);
   }
   if (warp == 1) {
     tc::tmem_alloc(sbase + L::kOffMisc, L::kTmemCols);
@@ -236,15 +245,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
   if (warp == 0) {
     // ======================= TMA producer =====================================
+    // without critical tiles nobody consumes Q: its load must still land before
+    // the Q tiles are reused or the CTA exits
+    if (lane == 0 && T == 0 && !tc::mbar_wait(bar(Q_FULL), 0, abort)) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
     if (lane == 0 && T > 0) {
-      tc::prefetch_tensormap(&tmQ);
-      tc::prefetch_tensormap(&tmK);
-      tc::prefetch_tensormap(&tmV);
-      tc::mbar_expect_tx(bar(Q_FULL), L::kQBytes);
-      for (int hf = 0; hf < 2; ++hf)
-        for (int p = 0; p < NP; ++p)
-          tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmQ, bar(Q_FULL), 64 * p, i_h[hf] * kBlock,
-                          bh_h[hf]);
       // K and V tiles go to separate rings; each is refilled as soon as a slot frees
       const uint32_t sKr = sKV, sVr = sKV + kKSlots * L::kSlotBytes;
       int nk = 0, nv = 0;
