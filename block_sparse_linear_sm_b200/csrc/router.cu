@@ -96,7 +96,10 @@ cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
 // j < i is ever read, so tiles wholly above the diagonal are skipped.
 // ---------------------------------------------------------------------------
 constexpr int kSTile = 64;
-constexpr int kSK = 16;
+constexpr int kSK = 16;       // k columns per pipeline stage
+constexpr int kSPad = 20;     // doubles per shared-memory row: a fragment read takes two wavefronts
+constexpr int kSStages = 4;   // cp.async ring depth
+constexpr int kScoresSmem = kSStages * 2 * kSTile * kSPad * 8;
 
 __device__ __forceinline__ void dmma_8x8x4(double (&c)[2], double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
@@ -113,36 +116,52 @@ __global__ void __launch_bounds__(128) scores_kernel(const double* __restrict__ 
   const int bkv = b * (H / group) + h / group;
   const int i0 = blockIdx.y * kSTile, j0 = blockIdx.x * kSTile;
   if (lower_only && j0 > i0 + kSTile - 1) return;
-  // [row][k], rows padded to 20 doubles: a fragment read takes the minimum two wavefronts
-  __shared__ double As[kSTile][kSK + 4];
-  __shared__ double Bs[kSTile][kSK + 4];
+  // stage s: A rows [kSTile][kSPad], then B rows; k chunks arrive by cp.async
+  extern __shared__ __align__(16) double ssm[];
   const double* A = qbar + (size_t)bh * nb * d;
   const double* Bm = kbar + (size_t)bkv * nb * d;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int wi = (w >> 1) * 32, wj = (w & 1) * 32;  // warp tile origin
-  double acc[4][4][2] = {};
-  for (int k0 = 0; k0 < d; k0 += kSK) {
-    for (int e = tid; e < kSTile * kSK; e += 128) {
-      const int r = e / kSK, kk = e % kSK;
+  const int nk = d / kSK;
+  auto load = [&](int kc, int st) {
+    double* As = ssm + (size_t)st * 2 * kSTile * kSPad;
+    double* Bs = As + kSTile * kSPad;
+    // 64 rows x 8 sixteen-byte pieces per matrix; rows past nb are zero-filled
+    for (int e = tid; e < kSTile * 8; e += 128) {
+      const int r = e >> 3, pc = e & 7;
       const int ia = i0 + r, jb = j0 + r;
-      As[r][kk] = ia < nb ? A[(size_t)ia * d + k0 + kk] : 0.0;
-      Bs[r][kk] = jb < nb ? Bm[(size_t)jb * d + k0 + kk] : 0.0;
+      cp_async16(smem_u32(As + r * kSPad + 2 * pc), A + (size_t)(ia < nb ? ia : 0) * d + kc * kSK + 2 * pc,
+                 ia < nb ? 16 : 0);
+      cp_async16(smem_u32(Bs + r * kSPad + 2 * pc), Bm + (size_t)(jb < nb ? jb : 0) * d + kc * kSK + 2 * pc,
+                 jb < nb ? 16 : 0);
     }
-    __syncthreads();
+  };
+#pragma unroll
+  for (int st = 0; st < kSStages - 1; ++st) {
+    if (st < nk) load(st, st);
+    cp_async_commit();
+  }
+  double acc[4][4][2] = {};
+  for (int kc = 0; kc < nk; ++kc) {
+    cp_async_wait<kSStages - 2>();
+    __syncthreads();  // chunk kc landed for everyone; stage (kc - 1) % S is free again
+    if (kc + kSStages - 1 < nk) load(kc + kSStages - 1, (kc + kSStages - 1) % kSStages);
+    cp_async_commit();
+    const double* As = ssm + (size_t)(kc % kSStages) * 2 * kSTile * kSPad;
+    const double* Bs = As + kSTile * kSPad;
 #pragma unroll
     for (int k4 = 0; k4 < kSK; k4 += 4) {
       double af[4], bf[4];
       // A fragment: row lane/4, column lane%4; B fragment: row (k) lane%4, column lane/4
 #pragma unroll
-      for (int m = 0; m < 4; ++m) af[m] = As[wi + 8 * m + (lane >> 2)][k4 + (lane & 3)];
+      for (int m = 0; m < 4; ++m) af[m] = As[(wi + 8 * m + (lane >> 2)) * kSPad + k4 + (lane & 3)];
 #pragma unroll
-      for (int n = 0; n < 4; ++n) bf[n] = Bs[wj + 8 * n + (lane >> 2)][k4 + (lane & 3)];
+      for (int n = 0; n < 4; ++n) bf[n] = Bs[(wj + 8 * n + (lane >> 2)) * kSPad + k4 + (lane & 3)];
 #pragma unroll
       for (int m = 0; m < 4; ++m)
 #pragma unroll
         for (int n = 0; n < 4; ++n) dmma_8x8x4(acc[m][n], af[m], bf[n]);
     }
-    __syncthreads();
   }
   double* S = scores + (size_t)bh * nb * nb;
 #pragma unroll
@@ -164,9 +183,11 @@ cudaError_t launch_scores(const Plan& p, const Args& a, cudaStream_t s) {
   const double* kbar = reinterpret_cast<const double*>(a.ws + p.off_kbar);
   double* sc = reinterpret_cast<double*>(a.ws + p.off_scores);
   const int t = (p.nqb + kSTile - 1) / kSTile;
+  cudaError_t e = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoresSmem);
+  if (e != cudaSuccess) return e;
   dim3 grid(t, t, c.B * c.H);
-  scores_kernel<<<grid, 128, 0, s>>>(qbar, kbar, sc, c.H, p.group, p.nqb, c.d, (double)p.scale,
-                                     c.mode == SLA_MODE_TOPN_WINDOW);
+  scores_kernel<<<grid, 128, kScoresSmem, s>>>(qbar, kbar, sc, c.H, p.group, p.nqb, c.d, (double)p.scale,
+                                               c.mode == SLA_MODE_TOPN_WINDOW);
   return cudaGetLastError();
 }
 
