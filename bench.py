@@ -370,6 +370,25 @@ def main():
         raise RuntimeError(f"device status {st} detail {detail}")
     ms_total, ms_eager = max_over_ranks(dist, dev, g0.elapsed_time(g1), ms_eager)
     ms_step = ms_total / args.steps
+    # per-replay medians: warm (replays back to back) and cold (a 256 MB buffer,
+    # twice the L2, written right before each timed replay)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 10)
+    pairs = {"warm": [], "cold": []}
+    for kind in ("warm", "cold"):
+        for _ in range(reps):
+            if kind == "cold":
+                flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            graph.replay()
+            a1.record(stream)
+            pairs[kind].append((a0, a1))
+    torch.cuda.synchronize()
+    warm_med = statistics.median(a.elapsed_time(b) for a, b in pairs["warm"])
+    cold_med = statistics.median(a.elapsed_time(b) for a, b in pairs["cold"])
+    warm_med, cold_med = max_over_ranks(dist, dev, warm_med, cold_med)
+    del flush, pairs
     del graph
     stage_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
                 for i, n in enumerate(names)}
@@ -457,6 +476,8 @@ def main():
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs (Q,K,V 302 MB) larger than the 126 MB L2; no flush"},
         "ms_per_layer": ms_step,
+        "per_replay_ms": {"warm_median": warm_med, "cold_median": cold_med, "reps": reps,
+                          "cold": "256 MB written before each timed replay (L2 holds none of the layer's data)"},
         "ms_per_step_eager": ms_eager,
         "launch": "CUDA graph replay of one captured sla_forward call (ms_per_step_eager: direct calls)",
         "roofline": roof,

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.sla_stage_name.restype = ctypes.c_char_p
         L.sla_check_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
         L.sla_check_device_status.restype = ctypes.c_int
+        L.sla_selftest_wait_timeout.argtypes = [P, S, ctypes.c_int64, P]
+        L.sla_selftest_wait_timeout.restype = ctypes.c_int
         L.sla_status_string.argtypes = [ctypes.c_int]
         L.sla_status_string.restype = ctypes.c_char_p
         L.sla_version.argtypes = []
@@ -178,6 +180,14 @@ def sla_check_device_status(ws, stream=None) -> tuple:
     detail = ctypes.c_int32(0)
     st = lib().sla_check_device_status(_ptr(ws), _stream(stream), ctypes.byref(detail))
     return int(st), int(detail.value)
+
+
+def sla_selftest_wait_timeout(ws, limit_ns: int, stream=None) -> None:
+    """Enqueue the failure-detection self-test: a bounded wait that runs out and is
+    recorded in ws's status word (read it with sla_check_device_status)."""
+    nbytes = ws.numel() * ws.element_size() if hasattr(ws, "numel") else 256
+    _check(lib().sla_selftest_wait_timeout(_ptr(ws), nbytes, int(limit_ns), _stream(stream)),
+           "sla_selftest_wait_timeout")
 
 
 def sla_version() -> str:

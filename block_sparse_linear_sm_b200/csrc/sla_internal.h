@@ -18,6 +18,7 @@ enum DeviceDetail : int {
   kDetailFlashIndex = 101,      // flash kernel read a block index outside [0, nkb)
   kDetailFlashAlign = 103,     // shared-memory base not 1024-byte aligned
   kDetailTimeout = 200,
+  kDetailSelftest = 300,       // the failure-detection self-test's wait ran out (expected)
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

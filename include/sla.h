@@ -175,6 +175,19 @@ SLA_API const char* sla_stage_name(const sla_config* cfg, int32_t s);
  */
 SLA_API sla_status sla_check_device_status(void* ws, void* stream, int32_t* detail);
 
+/*
+ * Failure-detection self-test (the pages have no counterpart). Clears the
+ * status word at the start of `ws` (any buffer of at least 256 bytes,
+ * 256-byte aligned) and launches one small kernel that waits, through the
+ * same bounded mbarrier wait every kernel of the library uses, on a barrier
+ * that nothing completes. After `limit_ns` (1e3 .. 1e9) the wait gives up, the
+ * kernel records SLA_ERR_DEVICE_TIMEOUT with detail 300 in the status word and
+ * returns, so sla_check_device_status(ws, ...) then reports the timeout and the
+ * GPU context stays usable. Returns SLA_ERR_INVALID_ARG for a bad ws or limit,
+ * SLA_ERR_CUDA for a failed launch, else SLA_OK.
+ */
+SLA_API sla_status sla_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t limit_ns, void* stream);
+
 /* Static description of a status code. */
 SLA_API const char* sla_status_string(sla_status s);
 

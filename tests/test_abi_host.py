@@ -140,3 +140,12 @@ def test_per_head_projection_is_accepted_with_one_kv_head_per_query_head():
     c = wl.small_config(N=1024, N_valid=1000, H=4, H_kv=4, proj_per_head=1)
     assert sla.sla_validate_config(c) == sla.SLA_OK
     assert sla.sla_workspace_bytes(c) == sla.sla_workspace_bytes(wl.small_config(N=1024, N_valid=1000, H=4, H_kv=4))
+
+
+def test_selftest_rejects_bad_arguments_before_launch():
+    L = sla.lib()
+    assert L.sla_selftest_wait_timeout(None, 4096, 1_000_000, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_selftest_wait_timeout(256 + 16, 4096, 1_000_000, None) == sla.SLA_ERR_INVALID_ARG  # misaligned
+    assert L.sla_selftest_wait_timeout(256, 128, 1_000_000, None) == sla.SLA_ERR_INVALID_ARG       # too small
+    assert L.sla_selftest_wait_timeout(256, 4096, 10, None) == sla.SLA_ERR_INVALID_ARG             # limit too short
+    assert L.sla_selftest_wait_timeout(256, 4096, 5_000_000_000, None) == sla.SLA_ERR_INVALID_ARG  # too long
