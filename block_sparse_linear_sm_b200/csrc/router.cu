@@ -402,8 +402,16 @@ cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cuda
 // top-n selection: one warp per (b, KV head, query block i). Each of the
 // group's heads takes a softmax of its pooled scores over the past blocks
 // j < i (float64); the probabilities are summed and the top min(top_n, i)
-// kept (same exact select as above).
+// kept (same exact select as above). A head's score row is first copied into
+// the warp's shared buffer with 16-byte loads, all in flight together; the
+// max, the exponentials (one per element) and the sums then work from there.
 // ---------------------------------------------------------------------------
+// per warp: keys, row buffer (16-byte aligned), flags, histogram
+__host__ __device__ inline size_t select_buf_off(int nb) { return align_up((size_t)nb * 8, 16); }
+__host__ __device__ inline size_t select_warp_bytes(int nb) {
+  return 2 * select_buf_off(nb) + align_up((size_t)nb, 16) + 1024;
+}
+
 __global__ void select_kernel(const double* __restrict__ scores, int8_t* __restrict__ mask_out,
                               int32_t* __restrict__ sel, int H, int group, int nb, int top_n,
                               int rows, int n_rows) {
@@ -414,28 +422,41 @@ __global__ void select_kernel(const double* __restrict__ scores, int8_t* __restr
   const int bkv = row / nb, i = row % nb;
   const int Hkv = H / group;
   const int b = bkv / Hkv, hk = bkv % Hkv;
-  unsigned char* base = smem + (size_t)w * ((size_t)nb * 8 + align_up((size_t)nb, 16) + 1024);
+  unsigned char* base = smem + (size_t)w * select_warp_bytes(nb);
   double* prob = reinterpret_cast<double*>(base);  // becomes the keys
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(base);
-  uint8_t* flags = base + (size_t)nb * 8;
-  unsigned* hist = reinterpret_cast<unsigned*>(base + (size_t)nb * 8 + align_up((size_t)nb, 16));
+  double* buf = reinterpret_cast<double*>(base + select_buf_off(nb));
+  uint8_t* flags = base + 2 * select_buf_off(nb);
+  unsigned* hist = reinterpret_cast<unsigned*>(base + 2 * select_buf_off(nb) + align_up((size_t)nb, 16));
   for (int j = lane; j < i; j += 32) {
     prob[j] = 0.0;
     flags[j] = 0;
   }
   __syncwarp();
+  // score rows start on 16 bytes when nb is even: pairs, then the odd last one
+  const int i2 = (nb & 1) ? 0 : (i & ~1);
   for (int g = 0; g < group && i > 0; ++g) {
     const double* srow = scores + (((size_t)b * H + hk * group + g) * nb + i) * nb;
+#pragma unroll 4
+    for (int j = 2 * lane; j < i2; j += 64)
+      *reinterpret_cast<double2*>(buf + j) = *reinterpret_cast<const double2*>(srow + j);
+#pragma unroll 4
+    for (int j = i2 + lane; j < i; j += 32) buf[j] = srow[j];
+    __syncwarp();
     double m = -INFINITY;
-    for (int j = lane; j < i; j += 32) m = fmax(m, srow[j]);
+    for (int j = lane; j < i; j += 32) m = fmax(m, buf[j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
     double sum = 0.0;
-    for (int j = lane; j < i; j += 32) sum += exp(srow[j] - m);
+    for (int j = lane; j < i; j += 32) {
+      const double e = exp(buf[j] - m);
+      buf[j] = e;
+      sum += e;
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const double inv = 1.0 / sum;
-    for (int j = lane; j < i; j += 32) prob[j] += exp(srow[j] - m) * inv;
+    for (int j = lane; j < i; j += 32) prob[j] += buf[j] * inv;
     __syncwarp();
   }
   for (int j = lane; j < i; j += 32) keys[j] = order_key(prob[j]);
@@ -455,8 +476,10 @@ __global__ void select_kernel(const double* __restrict__ scores, int8_t* __restr
 cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s) {
   const sla_config& c = p.c;
   const double* sc = reinterpret_cast<const double*>(a.ws + p.off_scores);
-  const int rows = route_rows_per_cta(p.nkb);
-  const size_t smem = route_smem(p.nkb, rows);
+  const size_t per = select_warp_bytes(p.nkb);
+  int rows = (int)((96 * 1024) / per);
+  rows = rows < 1 ? 1 : (rows > kRouteWarps ? kRouteWarps : rows);
+  const size_t smem = (size_t)rows * per;
   cudaError_t e =
       cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
