@@ -31,6 +31,11 @@ What each step follows (page title, section):
   map phi = elu + 1 (the pages leave phi open).
 * Combine: SLA analysis, Proj paragraph - O = O^s + Proj(O^l); SALAD summary,
   method details - an input-dependent gate balances the two branches.
+* Options from the SLA critique page's notes on the open-source code: smooth-K
+  (K made zero-mean; here: minus the mean of the head's valid key tokens,
+  which only changes phi(K) since softmax rows and pooled rankings shift by a
+  per-row constant) and the linear branch over all tokens instead of the
+  marginal blocks only.
 """
 from __future__ import annotations
 
@@ -171,9 +176,18 @@ def softmax_attention(q_rows: np.ndarray, keys: np.ndarray, vals: np.ndarray, sc
     return out
 
 
-def linear_states(k: np.ndarray, v: np.ndarray, n_valid: int, block: int):
-    """Per key block j: h_j = phi(K_j)^T V_j (d x d) and z_j = sum_t phi(k_t), valid tokens only."""
+def key_mean(k: np.ndarray, n_valid: int) -> np.ndarray:
+    """Mean of the valid key tokens of one head (the smooth-K offset)."""
+    return k[:n_valid].mean(axis=0) if n_valid > 0 else np.zeros(k.shape[1])
+
+
+def linear_states(k: np.ndarray, v: np.ndarray, n_valid: int, block: int,
+                  k_offset: Optional[np.ndarray] = None):
+    """Per key block j: h_j = phi(K_j - m)^T V_j (d x d) and z_j = sum_t phi(k_t - m), valid
+    tokens only; m = k_offset (smooth-K) or 0."""
     n, d = k.shape
+    if k_offset is not None:
+        k = k - k_offset[None, :]
     nb = n // block
     h = np.zeros((nb, d, v.shape[1]))
     z = np.zeros((nb, d))
@@ -224,11 +238,15 @@ class OracleCfg:
     has_proj: int = 1
     proj_per_head: int = 0
     has_gate: int = 0
+    smooth_k: int = 0    # linear branch on K minus the head's mean valid key
+    linear_all: int = 0  # linear branch over every valid key block, not only the marginal ones
     scale: float = 0.0
+
+    OPTIONAL = ("proj_per_head", "smooth_k", "linear_all")
 
     @classmethod
     def of(cls, c) -> "OracleCfg":
-        return cls(**{f: getattr(c, f, 0) if f == "proj_per_head" else getattr(c, f)
+        return cls(**{f: getattr(c, f, 0) if f in cls.OPTIONAL else getattr(c, f)
                       for f in cls.__dataclass_fields__})
 
     @property
@@ -300,8 +318,9 @@ class Layer:
     def states(self, b, hk):
         key = (b, hk)
         if key not in self._states:
-            self._states[key] = linear_states(self.k[b, hk], self.v[b, hk], self.c.N_valid,
-                                              self.c.block)
+            c = self.c
+            off = key_mean(self.k[b, hk], c.N_valid) if c.smooth_k else None
+            self._states[key] = linear_states(self.k[b, hk], self.v[b, hk], c.N_valid, c.block, off)
         return self._states[key]
 
     # -- one unit -----------------------------------------------------------
@@ -335,7 +354,10 @@ class Layer:
             row = self.classes(b, h)[i] if cls_row is None else cls_row
             crit = self._tokens_of(np.nonzero(row == CRITICAL)[0])
             o_s = softmax_attention(qr, K[crit], V[crit], c.sm_scale)
-            marg = np.nonzero(row == MARGINAL)[0]
+            # the linear branch covers the marginal blocks, or every block holding a
+            # valid token with linear_all
+            marg = (np.arange(c.nb)[np.arange(c.nb) * c.block < c.N_valid] if c.linear_all
+                    else np.nonzero(row == MARGINAL)[0])
             if marg.size:
                 hs, zs = self.states(b, hk)
                 o_l = linear_attention(qr, hs[marg].sum(axis=0), zs[marg].sum(axis=0))

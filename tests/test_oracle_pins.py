@@ -29,7 +29,8 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 class Cfg:
     def __init__(self, **kw):
         base = dict(B=1, H=2, H_kv=2, N=256, N_valid=256, d=16, block=32, mode=0, k_h=2, k_l=2,
-                    top_n=0, window=0, causal=0, has_proj=1, proj_per_head=0, has_gate=0, scale=0.0)
+                    top_n=0, window=0, causal=0, has_proj=1, proj_per_head=0, has_gate=0,
+                    smooth_k=0, linear_all=0, scale=0.0)
         base.update(kw)
         self.__dict__.update(base)
 
@@ -110,11 +111,16 @@ def brute_threeway(c, q, k, v, w_p, w_g):
             crit_b = r < c.k_h
             neg_b = r >= nb - c.k_l
             marg_b = ~crit_b & ~neg_b
+            if getattr(c, "linear_all", 0):
+                marg_b = np.ones_like(crit_b)
             crit = crit_b[tok_blk][:, tok_blk] & valid[None, :]
             marg = marg_b[tok_blk][:, tok_blk] & valid[None, :]
             o_s = sdpa(q[b, h][None], k[b, hk][None], v[b, hk][None], crit[None], sc)[0]
             fq = F.elu(torch.from_numpy(q[b, h])).numpy() + 1
-            fk = F.elu(torch.from_numpy(k[b, hk])).numpy() + 1
+            kk = torch.from_numpy(k[b, hk])
+            if getattr(c, "smooth_k", 0):
+                kk = kk - kk[:c.N_valid].mean(dim=0, keepdim=True)
+            fk = F.elu(kk).numpy() + 1
             a = (fq @ fk.T) * marg
             den = a.sum(1)
             o_l = np.where(den[:, None] > 0, (a @ v[b, hk]) / np.where(den > 0, den, 1)[:, None], 0)
@@ -394,8 +400,8 @@ def test_planted_pooling_over_padding_is_caught(monkeypatch):
 def test_planted_state_over_padding_is_caught(monkeypatch):
     orig = so.linear_states
 
-    def bad_states(k, v, n_valid, block):
-        return orig(k, v, k.shape[0], block)
+    def bad_states(k, v, n_valid, block, k_offset=None):
+        return orig(k, v, k.shape[0], block, k_offset)
     assert _fails_some_pin(monkeypatch, "linear_states", bad_states, PINS)
 
 
@@ -445,3 +451,67 @@ def test_per_head_projection_with_equal_matrices_is_the_shared_one():
     w3 = np.stack([w_p, 2.0 * w_p])
     o3 = oracle.forward(c2, q, k, v, w3, w_g)["O"]
     assert np.array_equal(o3[:, 0], shared[:, 0]) and not np.allclose(o3[:, 1], shared[:, 1])
+
+
+# ---------------------------------------------------------------------------
+# options from the SLA critique page's notes on the open-source code:
+# smooth-K (zero-mean K) and the linear branch over all tokens
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kw", [dict(smooth_k=1), dict(linear_all=1), dict(smooth_k=1, linear_all=1),
+                                dict(smooth_k=1, linear_all=1, N_valid=241, H=4, H_kv=2, has_gate=1),
+                                dict(linear_all=1, k_h=0, k_l=8)])
+def test_options_match_brute_force(kw):
+    assert pin_brute_threeway(Cfg(**kw)) < 1e-12
+
+
+def test_smooth_k_changes_only_the_linear_branch():
+    """K - m shifts every pooled score and attention logit of a row by q . m, so the classes
+    and O_s are those without smooth-K; only phi(K) in the linear branch changes."""
+    c0, c1 = Cfg(N_valid=250), Cfg(N_valid=250, smooth_k=1)
+    q, k, v, w_p, w_g = rand_inputs(c0, 21)
+    k = k + 0.7  # a key mean far from zero
+    k[:, :, c0.N_valid:] = 0
+    r0 = oracle.forward(c0, q, k, v, w_p, w_g)
+    r1 = oracle.forward(c1, q, k, v, w_p, w_g)
+    L0, L1 = so.Layer(c0, q, k, v, w_p, w_g), so.Layer(c1, q, k, v, w_p, w_g)
+    for h in range(c0.H):
+        assert np.array_equal(L0.classes(0, h), L1.classes(0, h))
+    assert max_err(r0["O_s"], r1["O_s"]) < 1e-12
+    assert max_err(r0["O_l"], r1["O_l"]) > 1e-3
+
+
+def test_smooth_k_is_a_no_op_for_zero_mean_keys():
+    c0, c1 = Cfg(N_valid=250), Cfg(N_valid=250, smooth_k=1)
+    q, k, v, w_p, w_g = rand_inputs(c0, 22)
+    k[:, :, :c0.N_valid] -= k[:, :, :c0.N_valid].mean(axis=2, keepdims=True)
+    o0 = oracle.forward(c0, q, k, v, w_p, w_g)["O"]
+    o1 = oracle.forward(c1, q, k, v, w_p, w_g)["O"]
+    assert max_err(o0, o1) < 1e-12
+
+
+def test_linear_all_with_every_block_negligible_is_linear_attention():
+    """No critical block and the linear branch over all tokens: O is plain kernelised linear
+    attention over every valid token (closed form)."""
+    c = Cfg(N_valid=250, k_h=0, k_l=8, linear_all=1, has_gate=1)
+    q, k, v, w_p, w_g = rand_inputs(c, 23)
+    o = oracle.forward(c, q, k, v, w_p, w_g)["O"]
+    ref = np.zeros_like(o)
+    valid = (np.arange(c.N) < c.N_valid).astype(np.float64)
+    for h in range(c.H):
+        fq = F.elu(torch.from_numpy(q[0, h])) + 1
+        fk = (F.elu(torch.from_numpy(k[0, h])) + 1) * torch.from_numpy(valid)[:, None]
+        a = fq @ fk.T
+        ol = (a @ torch.from_numpy(v[0, h])) / a.sum(1, keepdim=True) @ torch.from_numpy(w_p)
+        g = torch.sigmoid(torch.from_numpy(q[0, h]) @ torch.from_numpy(w_g[h]))[:, None]
+        ref[0, h] = (g * ol).numpy()
+    ref[:, :, c.N_valid:] = 0
+    assert max_err(o, ref) < 1e-12
+
+
+def test_planted_smooth_k_with_the_padded_mean_is_caught(monkeypatch):
+    """A key mean taken over the padded length instead of the valid tokens fails a pin."""
+    def bad_mean(k, n_valid):
+        return k.mean(axis=0)
+    monkeypatch.setattr(so, "key_mean", bad_mean)
+    assert pin_brute_threeway(Cfg(smooth_k=1, N_valid=241)) > 1e-6
