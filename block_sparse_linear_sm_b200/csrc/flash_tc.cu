@@ -696,7 +696,8 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
 
 cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s) {
   const bool topn = p.c.mode == SLA_MODE_TOPN_WINDOW;
-  const bool fuse = !topn && p.nkb - p.c.k_h - p.c.k_l > 0;  // the layer has a linear branch
+  // the layer has a linear branch: marginal blocks, or every block with linear_all
+  const bool fuse = !topn && (p.nkb - p.c.k_h - p.c.k_l > 0 || p.c.linear_all);
   if (p.c.d == 128) {
     if (topn) return launch_tc<128, true, false>(p, a, s);
     return fuse ? launch_tc<128, false, true>(p, a, s) : launch_tc<128, false, false>(p, a, s);

@@ -79,7 +79,8 @@ cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
   double* kbar = reinterpret_cast<double*>(a.ws + p.off_kbar);
   // phi(Q) and the gate feed the linear branch of a forward pass; routing-only
   // calls (no V) do not produce them
-  const bool lin = a.v != nullptr && c.mode == SLA_MODE_THREEWAY && p.nkb - c.k_h - c.k_l > 0;
+  const bool lin =
+      a.v != nullptr && c.mode == SLA_MODE_THREEWAY && (p.nkb - c.k_h - c.k_l > 0 || c.linear_all);
   __nv_bfloat16* phiq = lin ? reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_phiq) : nullptr;
   float* gate = (lin && c.has_gate) ? reinterpret_cast<float*>(a.ws + p.off_gate) : nullptr;
   dim3 grid(p.nqb, c.B * c.H + c.B * c.H_kv);
@@ -339,7 +340,7 @@ static size_t route_smem(int nb, int rows) {
 __global__ void classify_kernel(const double* __restrict__ scores, int8_t* __restrict__ mask_out,
                                 int32_t* __restrict__ crit, int32_t* __restrict__ neg,
                                 __nv_bfloat16* __restrict__ mmask, int nb, int k_h, int k_l,
-                                int nkb_pad, int nqb_pad, int rows, int n_rows) {
+                                int nkb_pad, int nqb_pad, int rows, int n_rows, int linear_all) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = blockIdx.x * rows + w;  // over B*H*nqb_pad
@@ -374,7 +375,8 @@ __global__ void classify_kernel(const double* __restrict__ scores, int8_t* __res
   if (mmask) {
     __nv_bfloat16* mrow = mmask + ((size_t)bh * nqb_pad + i) * nkb_pad;
     for (int j = lane; j < nkb_pad; j += 32)
-      mrow[j] = __float2bfloat16(j < nb && flags[j] == 2 ? 1.f : 0.f);
+      // the aggregation mask: the marginal blocks, or every block with linear_all
+      mrow[j] = __float2bfloat16(j < nb && (linear_all || flags[j] == 2) ? 1.f : 0.f);
   }
   if (crit && k_h > 0) warp_compact(flags, nb, 1, 1, crit + ((size_t)bh * nb + i) * k_h);
   if (neg && k_l > 0) warp_compact(flags, nb, 2, 0, neg + ((size_t)bh * nb + i) * k_l);
@@ -394,7 +396,7 @@ cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cuda
   const int n_rows = c.B * c.H * per_head;
   const int grid = (n_rows + rows - 1) / rows;
   classify_kernel<<<grid, rows * 32, smem, s>>>(sc, a.mask_out, a.crit, a.neg, mm, p.nkb, c.k_h,
-                                                c.k_l, p.nkb_pad, per_head, rows, n_rows);
+                                                c.k_l, p.nkb_pad, per_head, rows, n_rows, c.linear_all);
   return cudaGetLastError();
 }
 

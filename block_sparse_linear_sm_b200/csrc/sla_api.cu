@@ -24,13 +24,16 @@ static sla_status check_config(const sla_config* c) {
     if (c->k_h < 0 || c->k_l < 0 || c->k_h + c->k_l > nb) return SLA_ERR_INVALID_ARG;
     if (c->causal != 0) return SLA_ERR_UNSUPPORTED;
     if ((c->has_proj != 0 && c->has_proj != 1) || (c->has_gate != 0 && c->has_gate != 1) ||
-        (c->proj_per_head != 0 && c->proj_per_head != 1))
+        (c->proj_per_head != 0 && c->proj_per_head != 1) || (c->smooth_k != 0 && c->smooth_k != 1) ||
+        (c->linear_all != 0 && c->linear_all != 1))
       return SLA_ERR_INVALID_ARG;
     if (c->proj_per_head && (!c->has_proj || c->H_kv != c->H)) return SLA_ERR_UNSUPPORTED;
   } else if (c->mode == SLA_MODE_TOPN_WINDOW) {
     if (c->top_n < 0 || c->window < 0) return SLA_ERR_INVALID_ARG;
     if (c->causal != 1) return SLA_ERR_UNSUPPORTED;
-    if (c->has_proj != 0 || c->has_gate != 0 || c->proj_per_head != 0) return SLA_ERR_UNSUPPORTED;
+    if (c->has_proj != 0 || c->has_gate != 0 || c->proj_per_head != 0 || c->smooth_k != 0 ||
+        c->linear_all != 0)
+      return SLA_ERR_UNSUPPORTED;
     // selected blocks plus window blocks must fit the kernel's 128-entry list
     if (c->top_n > 64 || c->top_n + (c->window + 62) / kBlock + 1 > 128) return SLA_ERR_UNSUPPORTED;
   } else {
@@ -63,7 +66,7 @@ bool make_plan(const sla_config* c, Plan* p) {
   if (c->mode == SLA_MODE_THREEWAY) {
     p->off_crit = take(B * H * nqb * (size_t)c->k_h * 4);
     p->off_neg = off;
-    const bool marginal = p->nkb - c->k_h - c->k_l > 0;
+    const bool marginal = p->nkb - c->k_h - c->k_l > 0 || c->linear_all;
     if (marginal) {
       p->off_mmask = take(B * H * (size_t)p->nqb_pad * p->nkb_pad * 2);
       p->off_hs = take(B * Hkv * (size_t)p->nkb_pad * p->dd * 2);
@@ -71,6 +74,7 @@ bool make_plan(const sla_config* c, Plan* p) {
       p->off_zs = take(B * H * nqb * d * 4);      // Z_i, fp32
       p->off_phiq = take(B * H * (size_t)c->N * d * 2);  // phi(Q), bf16
       if (c->has_gate) p->off_gate = take(B * H * (size_t)c->N * 4);  // sigmoid(q . w_g), fp32
+      if (c->smooth_k) p->off_kmean = take(B * Hkv * d * 4);            // mean valid key, fp32
     }
   } else {
     p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
@@ -81,7 +85,7 @@ bool make_plan(const sla_config* c, Plan* p) {
 
 static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
-static bool has_marginal(const Plan& p) { return p.nkb - p.c.k_h - p.c.k_l > 0; }
+static bool has_marginal(const Plan& p) { return p.nkb - p.c.k_h - p.c.k_l > 0 || p.c.linear_all; }
 
 // Stage list of a configuration.
 enum Stage { kPool, kScores, kClassify, kSelect, kState, kAggregate, kFlash };

@@ -32,7 +32,7 @@ struct Plan {
   float scale;
   // byte offsets into ws
   size_t off_status, off_qbar, off_kbar, off_scores, off_crit, off_neg, off_mmask, off_hs, off_ss,
-      off_zs, off_phiq, off_gate, total;
+      off_zs, off_phiq, off_gate, off_kmean, total;
 };
 
 bool make_plan(const sla_config* c, Plan* p);

@@ -22,6 +22,9 @@
 // dd (a multiple of 128); rows j in [nkb, nkb_pad) zero.
 // For d = 64 the state product still uses M = 128: the second feature panel
 // of K is read beyond the tensor and filled with zeros.
+// Smooth-K (the SLA critique page's note on the open-source code: zero-mean K):
+// phi is applied to k_t - m, m = mean of the head's valid key tokens, computed
+// first from the float64 block means of the pooling pass.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -47,7 +50,23 @@ struct StateParams {
   int* status;
   int nkb, nkb_pad, dd, n_valid, has_proj;
   int wp_heads;  // 1: one W_p for all heads; H: W_p[h] for KV head h (H_kv == H)
+  const float* kmean;  // smooth-K: [B*H_kv][D] mean valid key, or null
 };
+
+// m = sum_j n_j kbar_j / N_valid over the blocks of one KV head (n_j valid tokens
+// of block j), float64 sums, one thread per column.
+__global__ void kmean_kernel(const double* __restrict__ kbar, float* __restrict__ kmean, int nb, int d,
+                             int n_valid) {
+  const int bkv = blockIdx.x, c = threadIdx.x;
+  if (c >= d) return;
+  const double* kb = kbar + (size_t)bkv * nb * d + c;
+  double s = 0.0;
+  for (int j = 0; j < nb; ++j) {
+    const int nv = n_valid - j * kBlock < kBlock ? n_valid - j * kBlock : kBlock;
+    s += (double)nv * kb[(size_t)j * d];
+  }
+  kmean[(size_t)bkv * d + c] = (float)(s / (double)n_valid);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kStThreads, 2)
@@ -151,14 +170,23 @@ __global__ void __launch_bounds__(kStThreads, 2)
       uint4* row = reinterpret_cast<uint4*>(smem + L::kOffK + hh * 16384 + r * 128);
 #pragma unroll
       for (int c = 0; c < 8; ++c) u[c] = row[c ^ (r & 7)];
+      const float* km = prm.kmean ? prm.kmean + (size_t)bkv * D + 64 * hh : nullptr;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t* w = reinterpret_cast<uint32_t*>(&u[c]);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float2 f = unpack_bf16(w[x]);
-          w[x] = valid_tok ? pack_bf16(phi(f.x), phi(f.y)) : 0u;
+        float4 m0 = make_float4(0.f, 0.f, 0.f, 0.f), m1 = m0;
+        if (km) {
+          m0 = *reinterpret_cast<const float4*>(km + 8 * c);
+          m1 = *reinterpret_cast<const float4*>(km + 8 * c + 4);
         }
+        auto shifted_phi = [&](uint32_t word, float ma, float mb) -> uint32_t {
+          const float2 f = unpack_bf16(word);
+          return valid_tok ? pack_bf16(phi(f.x - ma), phi(f.y - mb)) : 0u;
+        };
+        w[0] = shifted_phi(w[0], m0.x, m0.y);
+        w[1] = shifted_phi(w[1], m0.z, m0.w);
+        w[2] = shifted_phi(w[2], m1.x, m1.y);
+        w[3] = shifted_phi(w[3], m1.z, m1.w);
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) row[c ^ (r & 7)] = u[c];
@@ -289,6 +317,13 @@ static cudaError_t launch_state_t(const Plan& p, const Args& a, cudaStream_t s) 
   prm.n_valid = c.N_valid;
   prm.has_proj = proj ? 1 : 0;
   prm.wp_heads = wp_heads;
+  prm.kmean = nullptr;
+  if (c.smooth_k) {
+    float* km = reinterpret_cast<float*>(a.ws + p.off_kmean);
+    kmean_kernel<<<c.B * c.H_kv, D, 0, s>>>(reinterpret_cast<const double*>(a.ws + p.off_kbar), km, p.nkb, D,
+                                             c.N_valid);
+    prm.kmean = km;
+  }
   cudaError_t e = cudaFuncSetAttribute(state_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::kSmem);
   if (e != cudaSuccess) return e;

@@ -58,6 +58,8 @@ class LayerConfig:
     has_proj: int = 1
     proj_per_head: int = 0        # 1: one W_p per query head ([H, d, d])
     has_gate: int = 0
+    smooth_k: int = 0             # 1: linear branch on K minus the head's mean valid key
+    linear_all: int = 0           # 1: linear branch over all valid key blocks
     scale: float = 0.0            # 0 -> 1/sqrt(d)
     generator: str = "iid"        # iid | fourier | block_shift
     grid: Optional[tuple] = None  # (t, h, w) for the Fourier generator

@@ -114,6 +114,11 @@ typedef struct {
                           * projection is folded into per-KV-head states), else
                           * SLA_ERR_UNSUPPORTED */
   int32_t has_gate; /* THREEWAY: 1 = g = sigmoid(q . w_g[h]), 0 = g = 1 */
+  int32_t smooth_k; /* THREEWAY: 1 = the linear branch uses K minus the mean of the head's
+                     * valid key tokens (smooth-K, zero-mean K); routing and the sparse
+                     * branch are unchanged by it (each row shifts by a constant) */
+  int32_t linear_all; /* THREEWAY: 1 = the linear branch runs over every valid key block
+                       * (all tokens) instead of the marginal blocks only */
   float scale;      /* softmax scale of pooled scores and attention; 0 = 1/sqrt(d) */
 } sla_config;
 

@@ -60,6 +60,10 @@ BAD = [
     (dict(mode=1, causal=1, top_n=4, has_proj=1), sla.SLA_ERR_UNSUPPORTED),
     (dict(mode=7), sla.SLA_ERR_INVALID_ARG),
     (dict(proj_per_head=2), sla.SLA_ERR_INVALID_ARG),
+    (dict(smooth_k=2), sla.SLA_ERR_INVALID_ARG),
+    (dict(linear_all=-1), sla.SLA_ERR_INVALID_ARG),
+    (dict(mode=1, causal=1, top_n=4, has_proj=0, smooth_k=1), sla.SLA_ERR_UNSUPPORTED),
+    (dict(mode=1, causal=1, top_n=4, has_proj=0, linear_all=1), sla.SLA_ERR_UNSUPPORTED),
     (dict(proj_per_head=1, has_proj=0), sla.SLA_ERR_UNSUPPORTED),
     (dict(proj_per_head=1, H=4, H_kv=2), sla.SLA_ERR_UNSUPPORTED),
     (dict(mode=1, causal=1, top_n=4, has_proj=0, proj_per_head=1), sla.SLA_ERR_UNSUPPORTED),
@@ -149,3 +153,12 @@ def test_selftest_rejects_bad_arguments_before_launch():
     assert L.sla_selftest_wait_timeout(256, 128, 1_000_000, None) == sla.SLA_ERR_INVALID_ARG       # too small
     assert L.sla_selftest_wait_timeout(256, 4096, 10, None) == sla.SLA_ERR_INVALID_ARG             # limit too short
     assert L.sla_selftest_wait_timeout(256, 4096, 5_000_000_000, None) == sla.SLA_ERR_INVALID_ARG  # too long
+
+
+def test_linear_all_keeps_the_linear_stages_without_marginal_blocks():
+    # k_h + k_l = nb leaves no marginal block; with linear_all the linear branch still runs
+    c0 = wl.small_config(N=1024, N_valid=1024, k_h=8, k_l=8)
+    c1 = wl.small_config(N=1024, N_valid=1024, k_h=8, k_l=8, linear_all=1)
+    assert "linear_state" not in sla.sla_stage_names(c0)
+    assert "linear_state" in sla.sla_stage_names(c1) and "linear_aggregate" in sla.sla_stage_names(c1)
+    assert sla.sla_workspace_bytes(c1) > sla.sla_workspace_bytes(c0)

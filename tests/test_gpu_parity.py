@@ -53,6 +53,12 @@ SMALL_CASES = [
          proj_per_head=1, has_gate=1),
     dict(name="per_head_proj_d64", N=1024, N_valid=1024, d=64, H=3, H_kv=3, k_h=2, k_l=3,
          proj_per_head=1),
+    dict(name="smooth_k", N=1536, N_valid=1500, d=128, H=4, H_kv=4, k_h=3, k_l=4, smooth_k=1,
+         has_gate=1),
+    dict(name="linear_all_d64", N=1024, N_valid=1000, d=64, k_h=3, k_l=4, linear_all=1),
+    dict(name="smooth_linear_all_gqa", N=1536, N_valid=1473, d=128, H=4, H_kv=2, k_h=3, k_l=2,
+         smooth_k=1, linear_all=1, has_gate=1),
+    dict(name="linear_all_no_crit", N=1024, N_valid=1024, d=128, k_h=0, k_l=16, linear_all=1),
 ]
 
 
@@ -130,6 +136,26 @@ def test_per_head_projection_linear_term_shifted_values(d):
     rel = np.linalg.norm(got_l - want_l) / np.linalg.norm(want_l)
     print("per-head projection: linear term relative Frobenius error", rel)
     assert rel <= 1e-2
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_smooth_k_linear_term_with_offset_keys(d):
+    """Smooth-K with keys whose mean is far from zero and V + 3 (the linear branch O(1)):
+    the linear term O - O_s against the oracle, both options on."""
+    cfg = small(name="smooth_shift", N=2048, N_valid=2030, d=d, H=2, H_kv=2, k_h=4, k_l=6,
+                smooth_k=1, linear_all=1, has_proj=0)
+    x = wl.generate(cfg, v_shift=3.0)
+    kf = wl.bf16_bits_to_f64(x.k)
+    kf[:, :, :cfg.N_valid] += 0.75
+    x.k = wl.to_bf16_bits(kf)
+    run = GpuRun(cfg, x)
+    ref = run.layer().forward()
+    n = cfg.N_valid
+    got_l = run.O()[:, :, :n] - ref["O_s"][:, :, :n]
+    want_l = ref["O"][:, :, :n] - ref["O_s"][:, :, :n]
+    rel = np.linalg.norm(got_l - want_l) / np.linalg.norm(want_l)
+    print("smooth-K: linear term relative Frobenius error", rel)
+    assert rel <= 1e-2  # (absolute output bounds assume O(1) outputs; here V + 3 makes O ~ 3)
 
 
 TOPN_CASES = [
