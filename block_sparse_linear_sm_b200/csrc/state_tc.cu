@@ -54,18 +54,29 @@ struct StateParams {
 };
 
 // m = sum_j n_j kbar_j / N_valid over the blocks of one KV head (n_j valid tokens
-// of block j), float64 sums, one thread per column.
-__global__ void kmean_kernel(const double* __restrict__ kbar, float* __restrict__ kmean, int nb, int d,
-                             int n_valid) {
-  const int bkv = blockIdx.x, c = threadIdx.x;
-  if (c >= d) return;
+// of block j), in float64. 1024 threads: column c = tid % d, part = tid / d sums
+// the blocks j = part, part + parts, ...; the parts are added in shared memory
+// in a fixed order.
+constexpr int kKmeanThreads = 1024;
+
+__global__ void __launch_bounds__(kKmeanThreads)
+    kmean_kernel(const double* __restrict__ kbar, float* __restrict__ kmean, int nb, int d, int n_valid) {
+  __shared__ double part_sum[kKmeanThreads];
+  const int bkv = blockIdx.x, c = threadIdx.x % d, part = threadIdx.x / d, parts = kKmeanThreads / d;
   const double* kb = kbar + (size_t)bkv * nb * d + c;
   double s = 0.0;
-  for (int j = 0; j < nb; ++j) {
+#pragma unroll 4
+  for (int j = part; j < nb; j += parts) {
     const int nv = n_valid - j * kBlock < kBlock ? n_valid - j * kBlock : kBlock;
     s += (double)nv * kb[(size_t)j * d];
   }
-  kmean[(size_t)bkv * d + c] = (float)(s / (double)n_valid);
+  part_sum[threadIdx.x] = s;
+  __syncthreads();
+  if (part == 0) {
+    double t = 0.0;
+    for (int q = 0; q < parts; ++q) t += part_sum[q * d + c];
+    kmean[(size_t)bkv * d + c] = (float)(t / (double)n_valid);
+  }
 }
 
 template <int D>
@@ -320,8 +331,8 @@ static cudaError_t launch_state_t(const Plan& p, const Args& a, cudaStream_t s) 
   prm.kmean = nullptr;
   if (c.smooth_k) {
     float* km = reinterpret_cast<float*>(a.ws + p.off_kmean);
-    kmean_kernel<<<c.B * c.H_kv, D, 0, s>>>(reinterpret_cast<const double*>(a.ws + p.off_kbar), km, p.nkb, D,
-                                             c.N_valid);
+    kmean_kernel<<<c.B * c.H_kv, kKmeanThreads, 0, s>>>(reinterpret_cast<const double*>(a.ws + p.off_kbar), km,
+                                                          p.nkb, D, c.N_valid);
     prm.kmean = km;
   }
   cudaError_t e = cudaFuncSetAttribute(state_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -114,6 +114,10 @@ def _preset(name: str) -> LayerConfig:
         return LayerConfig(name, 1, 64, 4, 65536, 65536, 128, mode=MODE_TOPN_WINDOW,
                            top_n=16, window=512, causal=1, has_proj=0, has_gate=0,
                            generator="block_shift", seed=1004)
+    if name == "wan1.3b_opensource":
+        # the SLA critique page's reading of the open-source code: smooth-K and the
+        # linear branch over all tokens, on the Wan2.1-1.3B layer's inputs
+        return _preset("wan1.3b").replace(name=name, smooth_k=1, linear_all=1)
     if name == "wan14b":
         k_h, k_l = _counts(0.05, 0.10, 1182)
         return LayerConfig(name, 1, 40, 40, 75648, 75600, 128, k_h=k_h, k_l=k_l,
@@ -122,7 +126,7 @@ def _preset(name: str) -> LayerConfig:
     raise KeyError(name)
 
 
-PRESETS = ("tiny", "wan1.3b", "salad", "nsa_causal", "wan14b")
+PRESETS = ("tiny", "wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource")
 
 
 def preset(name: str) -> LayerConfig:

@@ -188,7 +188,7 @@ def sampled_units(cfg, n=12, seed=0):
     return sorted(units)
 
 
-@pytest.mark.parametrize("name", ["wan1.3b", "salad", "nsa_causal", "wan14b"])
+@pytest.mark.parametrize("name", ["wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource"])
 def test_full_size_workload(name):
     cfg = wl.preset(name)
     run = GpuRun(cfg)
