@@ -31,6 +31,12 @@ What each step follows (page title, section):
   map phi = elu + 1 (the pages leave phi open).
 * Combine: SLA analysis, Proj paragraph - O = O^s + Proj(O^l); SALAD summary,
   method details - an input-dependent gate balances the two branches.
+* Token reordering: 2025 review, section 11 (SpargeAttn), the token-reorder
+  note - ordering tokens along a Hilbert curve raises the similarity of the
+  tokens that share a block. The curve is the 3-D Hilbert curve over the
+  (t, h, w) grid, computed with Skilling's axes-to-transpose method ("Programming
+  the Hilbert curve", AIP Conf. Proc. 707, 2004); tokens are ordered by their
+  key on the smallest power-of-two cube holding the grid.
 * Options from the SLA critique page's notes on the open-source code: smooth-K
   (K made zero-mean; here: minus the mean of the head's valid key tokens,
   which only changes phi(K) since softmax rows and pooled rankings shift by a
@@ -412,3 +418,73 @@ class Layer:
 def forward(cfg, q, k, v, w_p=None, w_g=None) -> Dict[str, np.ndarray]:
     """Whole-layer outputs O, O_s, O_l as float64 [B, H, N, d]."""
     return Layer(cfg, q, k, v, w_p, w_g).forward()
+
+
+# ---------------------------------------------------------------------------
+# token reordering along a Hilbert curve (SpargeAttn token-reorder note)
+# ---------------------------------------------------------------------------
+
+def hilbert_key3(x: int, y: int, z: int, bits: int) -> int:
+    """Index of grid point (x, y, z) along the 3-D Hilbert curve of side 2**bits.
+
+    Skilling's method: undo the excess work level by level (invert or exchange
+    low bits against the first axis), Gray-encode across the axes, then read
+    the transposed index out bit by bit, first axis most significant.
+    """
+    X = [int(x), int(y), int(z)]
+    top = 1 << (bits - 1)
+    q = top
+    while q > 1:
+        low = q - 1
+        for i in range(3):
+            if X[i] & q:
+                X[0] ^= low
+            else:
+                swap = (X[0] ^ X[i]) & low
+                X[0] ^= swap
+                X[i] ^= swap
+        q >>= 1
+    for i in range(1, 3):
+        X[i] ^= X[i - 1]
+    flip = 0
+    q = top
+    while q > 1:
+        if X[2] & q:
+            flip ^= q - 1
+        q >>= 1
+    for i in range(3):
+        X[i] ^= flip
+    key = 0
+    for b in range(bits - 1, -1, -1):
+        for i in range(3):
+            key = (key << 1) | ((X[i] >> b) & 1)
+    return key
+
+
+def hilbert_order(t: int, h: int, w: int) -> np.ndarray:
+    """order[n'] = raster index (t-major, then h, then w) of the n'-th token along the curve."""
+    bits = max(1, int(max(t, h, w) - 1).bit_length())
+    keys = np.array([hilbert_key3(a, b, c, bits) for a in range(t) for b in range(h) for c in range(w)],
+                    dtype=np.int64)
+    return np.argsort(keys, kind="stable").astype(np.int32)
+
+
+def permute_tokens(x: np.ndarray, order: np.ndarray, inverse: bool = False) -> np.ndarray:
+    """Gather y[..., n', :] = x[..., order[n'], :] (inverse: the scatter back); tokens past
+    len(order) stay where they are."""
+    y = x.copy()
+    n = len(order)
+    if inverse:
+        y[..., order, :] = x[..., :n, :]
+    else:
+        y[..., :n, :] = x[..., order, :]
+    return y
+
+
+def block_cos_sim(x: np.ndarray, block: int) -> float:
+    """Mean over blocks of the mean pairwise cosine similarity of a block's tokens
+    (the SpargeAttn CosSim of a block), full blocks only."""
+    n = x.shape[0] // block * block
+    xn = x[:n] / np.linalg.norm(x[:n], axis=1, keepdims=True)
+    s = xn.reshape(-1, block, x.shape[1]).sum(axis=1)
+    return float(np.mean((s * s).sum(axis=1) / block ** 2))

@@ -515,3 +515,54 @@ def test_planted_smooth_k_with_the_padded_mean_is_caught(monkeypatch):
         return k.mean(axis=0)
     monkeypatch.setattr(so, "key_mean", bad_mean)
     assert pin_brute_threeway(Cfg(smooth_k=1, N_valid=241)) > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# token reordering along a Hilbert curve (SpargeAttn token-reorder note)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_hilbert_curve_visits_every_cell_with_unit_steps(bits):
+    side = 1 << bits
+    pts = {}
+    for x in range(side):
+        for y in range(side):
+            for z in range(side):
+                pts[so.hilbert_key3(x, y, z, bits)] = (x, y, z)
+    assert sorted(pts) == list(range(side ** 3))       # a bijection onto [0, side^3)
+    assert pts[0] == (0, 0, 0)
+    steps = [np.abs(np.subtract(pts[k + 1], pts[k])).sum() for k in range(side ** 3 - 1)]
+    assert all(st == 1 for st in steps)                 # consecutive cells are grid neighbours
+
+
+def test_hilbert_order_is_a_permutation_of_a_ragged_grid():
+    order = so.hilbert_order(3, 5, 7)
+    assert sorted(order.tolist()) == list(range(105))
+    # on a power-of-two cube the order walks the curve: unit steps in (t, h, w)
+    o = so.hilbert_order(4, 4, 4)
+    coords = np.stack(np.unravel_index(o, (4, 4, 4)), axis=1)
+    assert np.all(np.abs(np.diff(coords, axis=0)).sum(axis=1) == 1)
+
+
+def test_permute_tokens_round_trip():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((2, 3, 70, 4))
+    order = so.hilbert_order(2, 5, 6)                    # 60 grid tokens, 10 padding rows
+    y = so.permute_tokens(x, order)
+    assert np.array_equal(y[:, :, 60:], x[:, :, 60:])
+    assert np.array_equal(y[:, :, 7], x[:, :, order[7]])
+    assert np.array_equal(so.permute_tokens(y, order, inverse=True), x)
+
+
+def test_hilbert_order_raises_block_similarity_of_a_smooth_field():
+    """The reorder note's claim on a smooth field over a (t, h, w) grid: tokens that share
+    a block become more alike (mean in-block cosine similarity)."""
+    rng = np.random.default_rng(7)
+    t, h, w = 6, 10, 16
+    tt, hh, ww = np.meshgrid(np.arange(t), np.arange(h), np.arange(w), indexing="ij")
+    coords = np.stack([tt.ravel(), hh.ravel(), ww.ravel()], axis=1).astype(np.float64)
+    om = rng.normal(0, 0.3, (32, 3))
+    field = np.cos(coords @ om.T + rng.uniform(0, 6.28, 32)) @ rng.standard_normal((32, 16))
+    raster = so.block_cos_sim(field, 16)
+    curve = so.block_cos_sim(field[so.hilbert_order(t, h, w)], 16)
+    assert curve > raster + 0.1
