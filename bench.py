@@ -390,6 +390,26 @@ def main():
     warm_med, cold_med = max_over_ranks(dist, dev, warm_med, cold_med)
     del flush, pairs
     del graph
+    # token reordering along the Hilbert curve of the video grid (an optional step
+    # before the layer): the gather of Q's rows, HBM-bound
+    reorder = None
+    if cfg.grid is not None:
+        order = torch.from_numpy(sla.sla_hilbert_order(*cfg.grid)).to(dev)
+        qp = torch.empty_like(q)
+        for _ in range(3):
+            sla.sla_permute_tokens(q, qp, order)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(args.steps):
+            sla.sla_permute_tokens(q, qp, order)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        (r_ms,) = max_over_ranks(dist, dev, r0.elapsed_time(r1) / args.steps)
+        moved = 2 * q.numel() * 2 + order.numel() * 4  # read and write Q, read the order
+        reorder = {"ms": r_ms, "bound": "hbm", "achieved": moved / (r_ms * 1e-3) / 1e9, "unit": "GB/s",
+                   "frac": None,
+                   "what": "Q rows gathered into Hilbert-curve order (sla_permute_tokens)"}
+        del qp, order
     stage_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
                 for i, n in enumerate(names)}
 
@@ -426,6 +446,8 @@ def main():
     e2e_value = job_throughput(world, flops, e2e_ms)
 
     peaks = load_peaks()
+    if reorder is not None:
+        reorder["frac"] = reorder["achieved"] / peaks["hbm"]
     model = stage_model(cfg)
     stages = {}
     for n in names:
@@ -481,6 +503,7 @@ def main():
         "ms_per_step_eager": ms_eager,
         "launch": "CUDA graph replay of one captured sla_forward call (ms_per_step_eager: direct calls)",
         "roofline": roof,
+        "token_reorder": reorder,
         "stages": stages,
         "gpu_launches": ns * args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,

@@ -72,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.sla_stage_name.restype = ctypes.c_char_p
         L.sla_check_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
         L.sla_check_device_status.restype = ctypes.c_int
+        L.sla_hilbert_order.argtypes = [I32, I32, I32, ctypes.POINTER(I32)]
+        L.sla_hilbert_order.restype = ctypes.c_int
+        L.sla_permute_tokens.argtypes = [P, P, P, I32, I32, I32, I32, I32, P]
+        L.sla_permute_tokens.restype = ctypes.c_int
         L.sla_selftest_wait_timeout.argtypes = [P, S, ctypes.c_int64, P]
         L.sla_selftest_wait_timeout.restype = ctypes.c_int
         L.sla_status_string.argtypes = [ctypes.c_int]
@@ -189,6 +193,24 @@ def sla_selftest_wait_timeout(ws, limit_ns: int, stream=None) -> None:
     nbytes = ws.numel() * ws.element_size() if hasattr(ws, "numel") else 256
     _check(lib().sla_selftest_wait_timeout(_ptr(ws), nbytes, int(limit_ns), _stream(stream)),
            "sla_selftest_wait_timeout")
+
+
+def sla_hilbert_order(t: int, h: int, w: int):
+    """Raster indices of the (t, h, w) grid's tokens in Hilbert-curve order (numpy int32)."""
+    import numpy as np
+    out = np.empty(t * h * w, dtype=np.int32)
+    _check(lib().sla_hilbert_order(t, h, w, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))),
+           "sla_hilbert_order")
+    return out
+
+
+def sla_permute_tokens(x, y, order, inverse: bool = False, stream=None) -> None:
+    """y[..., n, :] = x[..., order[n], :] for n < len(order) (inverse: the scatter back);
+    x, y: bf16 [..., n_tok, d] CUDA tensors, order: int32 CUDA tensor."""
+    n_tok, d = x.shape[-2], x.shape[-1]
+    rows = x.numel() // (n_tok * d)
+    _check(lib().sla_permute_tokens(_ptr(x), _ptr(y), _ptr(order), order.numel(), rows, n_tok, d,
+                                    1 if inverse else 0, _stream(stream)), "sla_permute_tokens")
 
 
 def sla_version() -> str:

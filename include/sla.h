@@ -193,6 +193,33 @@ SLA_API sla_status sla_check_device_status(void* ws, void* stream, int32_t* deta
  */
 SLA_API sla_status sla_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t limit_ns, void* stream);
 
+/*
+ * Token order along a 3-D Hilbert curve (2025 review, section 11, SpargeAttn:
+ * reordering tokens so that the tokens of a block lie close together raises
+ * their similarity). Host function: fills order[0 .. t*h*w) (host memory,
+ * caller-owned) with the raster index (t-major, then h, then w) of the n-th
+ * token along the curve; the curve is the Hilbert curve (Skilling's method)
+ * of the smallest power-of-two cube holding the grid. Deterministic; needs no
+ * GPU. SLA_ERR_INVALID_ARG for non-positive sides, more than 2^30 tokens or a
+ * NULL order.
+ */
+SLA_API sla_status sla_hilbert_order(int32_t t, int32_t h, int32_t w, int32_t* order);
+
+/*
+ * Device gather / scatter of token rows (the reorder above, or any order).
+ *   x, y    bf16 [rows, n_tok, d] device tensors, 16-byte aligned, not the same buffer
+ *   order   int32 [n_order] device array, a permutation of 0 .. n_order-1
+ *   inverse 0: y[r, n] = x[r, order[n]] for n < n_order;
+ *           1: y[r, order[n]] = x[r, n] (undoes the gather)
+ * Rows n >= n_order are copied in place. d must be a multiple of 8.
+ * SLA_ERR_INVALID_ARG on bad pointers or sizes (nothing launched). An order
+ * entry outside 0 .. n_order-1 is skipped on the device (no read or write for
+ * it; the row it would have filled keeps its old contents).
+ */
+SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* order, int32_t n_order,
+                                      int32_t rows, int32_t n_tok, int32_t d, int32_t inverse,
+                                      void* stream);
+
 /* Static description of a status code. */
 SLA_API const char* sla_status_string(sla_status s);
 

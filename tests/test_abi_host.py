@@ -5,6 +5,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 import block_sparse_linear_sm_b200 as sla
@@ -162,3 +164,23 @@ def test_linear_all_keeps_the_linear_stages_without_marginal_blocks():
     assert "linear_state" not in sla.sla_stage_names(c0)
     assert "linear_state" in sla.sla_stage_names(c1) and "linear_aggregate" in sla.sla_stage_names(c1)
     assert sla.sla_workspace_bytes(c1) > sla.sla_workspace_bytes(c0)
+
+
+@pytest.mark.parametrize("grid", [(1, 1, 1), (2, 3, 4), (4, 4, 4), (5, 7, 3), (21, 30, 52)])
+def test_hilbert_order_matches_the_oracle(grid):
+    from oracle import sla_oracle as so
+    got = sla.sla_hilbert_order(*grid)
+    assert np.array_equal(got, so.hilbert_order(*grid))
+
+
+def test_reorder_entry_points_reject_bad_arguments():
+    L = sla.lib()
+    out = (ctypes.c_int32 * 8)()
+    assert L.sla_hilbert_order(0, 2, 2, out) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_hilbert_order(2, 2, 2, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_hilbert_order(2048, 2048, 2048, out) == sla.SLA_ERR_INVALID_ARG  # > 2^30 tokens
+    # x == y, misaligned, d not a multiple of 8, n_order > n_tok
+    assert L.sla_permute_tokens(256, 256, 256, 4, 1, 4, 8, 0, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_permute_tokens(256, 512 + 4, 256, 4, 1, 4, 8, 0, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_permute_tokens(256, 512, 256, 4, 1, 4, 12, 0, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_permute_tokens(256, 512, 256, 5, 1, 4, 8, 0, None) == sla.SLA_ERR_INVALID_ARG
