@@ -31,6 +31,14 @@ What each step follows (page title, section):
   map phi = elu + 1 (the pages leave phi open).
 * Combine: SLA analysis, Proj paragraph - O = O^s + Proj(O^l); SALAD summary,
   method details - an input-dependent gate balances the two branches.
+* Key-block similarity filter: 2025 review, section 11 (SpargeAttn), prediction
+  algorithm - s_kj = CosSim(K_j) and S_hat[i, j] = -inf when s_kj < theta.
+  CosSim is read as the mean cosine similarity over all ordered pairs of the
+  block's valid tokens, self-pairs included: |sum_t k_t / |k_t||^2 / n^2 (a
+  zero token counts as the zero vector). Filtered blocks rank below every
+  other block (equal scores: lower index first) and get probability 0 in the
+  top-n softmax; a row whose candidates are all filtered has all
+  probabilities 0.
 * Token reordering: 2025 review, section 11 (SpargeAttn), the token-reorder
   note - ordering tokens along a Hilbert curve raises the similarity of the
   tokens that share a block. The curve is the 3-D Hilbert curve over the
@@ -93,10 +101,28 @@ def pooled_scores(qbar: np.ndarray, kbar: np.ndarray, scale: float) -> np.ndarra
 
 
 def softmax(s: np.ndarray) -> np.ndarray:
-    """Row softmax (max-subtracted)."""
+    """Row softmax (max-subtracted); a row of -inf only gives zeros."""
     m = s.max(axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
     e = np.exp(s - m)
-    return e / e.sum(axis=-1, keepdims=True)
+    tot = e.sum(axis=-1, keepdims=True)
+    return np.where(tot > 0, e / np.where(tot > 0, tot, 1.0), 0.0)
+
+
+def block_cos_sims(x: np.ndarray, n_valid: int, block: int) -> np.ndarray:
+    """CosSim of every block: |sum_t x_t / |x_t||^2 / n^2 over its n valid tokens (0 if none)."""
+    nb = x.shape[0] // block
+    out = np.zeros(nb)
+    for j in range(nb):
+        lo, hi = j * block, min((j + 1) * block, n_valid)
+        if hi <= lo:
+            continue
+        xs = x[lo:hi]
+        nrm = np.linalg.norm(xs, axis=1)
+        unit = xs / np.where(nrm > 0, nrm, 1.0)[:, None]
+        acc = unit.sum(axis=0)
+        out[j] = float(acc @ acc) / float((hi - lo) ** 2)
+    return out
 
 
 def block_order(score_row: np.ndarray) -> np.ndarray:
@@ -246,9 +272,11 @@ class OracleCfg:
     has_gate: int = 0
     smooth_k: int = 0    # linear branch on K minus the head's mean valid key
     linear_all: int = 0  # linear branch over every valid key block, not only the marginal ones
+    cos_filter: int = 0  # pooled scores of key blocks with CosSim < cos_theta become -inf
     scale: float = 0.0
+    cos_theta: float = 0.0
 
-    OPTIONAL = ("proj_per_head", "smooth_k", "linear_all")
+    OPTIONAL = ("proj_per_head", "smooth_k", "linear_all", "cos_filter", "cos_theta")
 
     @classmethod
     def of(cls, c) -> "OracleCfg":
@@ -299,7 +327,12 @@ class Layer:
         if key not in self._scores:
             c = self.c
             qbar = pool_blocks(self.q[b, h], c.N_valid, c.block)
-            self._scores[key] = pooled_scores(qbar, self.kbar(b, h // c.group), c.sm_scale)
+            s = pooled_scores(qbar, self.kbar(b, h // c.group), c.sm_scale)
+            if c.cos_filter:
+                # key blocks whose tokens are not alike are not represented by their mean
+                sim = block_cos_sims(self.k[b, h // c.group], c.N_valid, c.block)
+                s[:, sim < c.cos_theta] = -np.inf
+            self._scores[key] = s
         return self._scores[key]
 
     def classes(self, b, h):

@@ -30,7 +30,7 @@ class Cfg:
     def __init__(self, **kw):
         base = dict(B=1, H=2, H_kv=2, N=256, N_valid=256, d=16, block=32, mode=0, k_h=2, k_l=2,
                     top_n=0, window=0, causal=0, has_proj=1, proj_per_head=0, has_gate=0,
-                    smooth_k=0, linear_all=0, scale=0.0)
+                    smooth_k=0, linear_all=0, cos_filter=0, scale=0.0, cos_theta=0.0)
         base.update(kw)
         self.__dict__.update(base)
 
@@ -96,6 +96,23 @@ def brute_rank(s):
     return rank
 
 
+def brute_cos_filter(c, k_head):
+    """True for key blocks whose mean pairwise cosine similarity (ordered pairs of valid
+    tokens, self-pairs included; Gram matrix of the normalised tokens) is below theta."""
+    nb = c.N // c.block
+    out = np.zeros(nb, dtype=bool)
+    if not getattr(c, "cos_filter", 0):
+        return out
+    for j in range(nb):
+        xs = k_head[j * c.block:min((j + 1) * c.block, c.N_valid)]
+        if xs.shape[0] == 0:
+            continue
+        nrm = np.sqrt((xs * xs).sum(axis=1))
+        xn = np.array([x / n if n > 0 else 0 * x for x, n in zip(xs, nrm)])
+        out[j] = (xn @ xn.T).mean() < c.cos_theta
+    return out
+
+
 def brute_threeway(c, q, k, v, w_p, w_g):
     g = c.H // c.H_kv
     sc = scale_of(c)
@@ -107,6 +124,7 @@ def brute_threeway(c, q, k, v, w_p, w_g):
         for h in range(c.H):
             hk = h // g
             s = brute_pool(q[b, h], c.N_valid, c.block) @ brute_pool(k[b, hk], c.N_valid, c.block).T * sc
+            s[:, brute_cos_filter(c, k[b, hk])] = -np.inf
             r = brute_rank(s)
             crit_b = r < c.k_h
             neg_b = r >= nb - c.k_l
@@ -145,12 +163,16 @@ def brute_topn_window(c, q, k, v):
             heads = range(hk * g, (hk + 1) * g)
             kb = brute_pool(k[b, hk], c.N_valid, c.block)
             S = [brute_pool(q[b, h], c.N_valid, c.block) @ kb.T * sc for h in heads]
+            filt = brute_cos_filter(c, k[b, hk])
+            for s in S:
+                s[:, filt] = -np.inf
             sel = np.zeros((nb, nb), dtype=bool)
             for i in range(1, nb):
                 p = np.zeros(i)
                 for s in S:
-                    e = torch.softmax(torch.from_numpy(s[i, :i]), dim=0).numpy()
-                    p += e
+                    row = s[i, :i]
+                    if np.isfinite(row).any():  # a head whose candidates are all filtered adds 0
+                        p += torch.softmax(torch.from_numpy(row), dim=0).numpy()
                 r = brute_rank(p[None, :])[0]
                 sel[i, :i] = r < min(c.top_n, i)
             allow = (t[None, :] <= t[:, None]) & valid[None, :] & (
@@ -566,3 +588,69 @@ def test_hilbert_order_raises_block_similarity_of_a_smooth_field():
     raster = so.block_cos_sim(field, 16)
     curve = so.block_cos_sim(field[so.hilbert_order(t, h, w)], 16)
     assert curve > raster + 0.1
+
+
+# ---------------------------------------------------------------------------
+# SpargeAttn key-block similarity filter (S_hat[i, j] = -inf when CosSim(K_j) < theta)
+# ---------------------------------------------------------------------------
+
+def _block_keys(c, seed, spread):
+    """Keys whose blocks differ in self-similarity: block j shares a direction with weight
+    spread[j] (1 = identical tokens, 0 = independent)."""
+    rng = np.random.default_rng(seed)
+    q, k, v, w_p, w_g = rand_inputs(c, seed)
+    for j in range(c.N // c.block):
+        lo, hi = j * c.block, (j + 1) * c.block
+        base = rng.standard_normal((c.B, c.H_kv, 1, c.d))
+        k[:, :, lo:hi] = spread[j] * base + (1 - spread[j]) * k[:, :, lo:hi]
+    k[:, :, c.N_valid:] = 0
+    return q, k, v, w_p, w_g
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(N_valid=241), dict(H=4, H_kv=2, has_gate=1, linear_all=1)])
+def test_cos_filter_matches_brute_force(kw):
+    c = Cfg(cos_filter=1, cos_theta=0.3, **kw)
+    spread = np.linspace(0.0, 0.9, c.N // c.block)
+    q, k, v, w_p, w_g = _block_keys(c, 31, spread)
+    o = oracle.forward(c, q, k, v, w_p, w_g)["O"]
+    assert max_err(o, brute_threeway(c, q, k, v, w_p, w_g)) < 1e-12
+    # some blocks are filtered and some are not
+    sims = so.block_cos_sims(k[0, 0], c.N_valid, c.block)
+    assert (sims < c.cos_theta).any() and (sims >= c.cos_theta).any()
+
+
+def test_cos_filter_in_top_n_mode_matches_brute_force():
+    c = Cfg(mode=1, causal=1, H=4, H_kv=2, has_proj=0, top_n=3, window=40, k_h=0, k_l=0,
+            cos_filter=1, cos_theta=0.3)
+    spread = np.linspace(0.0, 0.9, c.N // c.block)
+    q, k, v, w_p, w_g = _block_keys(c, 32, spread)
+    o = oracle.forward(c, q, k, v, w_p, w_g)["O"]
+    assert max_err(o, brute_topn_window(c, q, k, v)) < 1e-12
+
+
+def test_cos_filter_extremes():
+    """theta below every CosSim (>= 0) filters nothing; theta above every CosSim (<= 1)
+    filters every block, and the classes then follow the block index."""
+    c0 = Cfg(N_valid=250)
+    q, k, v, w_p, w_g = rand_inputs(c0, 33)
+    ref = oracle.forward(c0, q, k, v, w_p, w_g)["O"]
+    none = oracle.forward(Cfg(N_valid=250, cos_filter=1, cos_theta=-0.5), q, k, v, w_p, w_g)["O"]
+    assert np.array_equal(ref, none)
+    c2 = Cfg(N_valid=250, cos_filter=1, cos_theta=1.5)
+    L = so.Layer(c2, q, k, v, w_p, w_g)
+    cls = L.classes(0, 0)
+    nb = c2.N // c2.block
+    assert np.all(cls[:, :c2.k_h] == so.CRITICAL) and np.all(cls[:, nb - c2.k_l:] == so.NEGLIGIBLE)
+
+
+def test_block_cos_sims_closed_forms():
+    """Identical tokens give 1; two opposite tokens give 0; orthogonal unit tokens give 1/n."""
+    x = np.zeros((8, 4))
+    x[:4] = [1.0, 2.0, 0.0, -1.0]
+    x[4] = [1.0, 0, 0, 0]
+    x[5] = [-1.0, 0, 0, 0]
+    x[6:8] = np.eye(4)[:2]
+    sims = so.block_cos_sims(x, 8, 4)
+    assert abs(sims[0] - 1.0) < 1e-15
+    # block 1: e1, -e1, e1', e2 -> sum = (1, 1, 0, 0), |sum|^2 = 2, / 16
+    assert abs(sims[1] - 2.0 / 16.0) < 1e-15
