@@ -73,6 +73,56 @@ __global__ void pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bflo
   }
 }
 
+// ---------------------------------------------------------------------------
+// key-block similarity (2025 review, section 11, SpargeAttn: s_kj = CosSim(K_j),
+// S_hat[i, j] = -inf when s_kj < theta): one warp per (KV head row, block);
+// CosSim = |sum_t k_t / |k_t||^2 / n^2 over the n valid tokens, in float64 like
+// the pooled means (a zero token counts as the zero vector). Writes 1 for the
+// blocks below theta.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void kcos_kernel(const __nv_bfloat16* __restrict__ k, uint8_t* __restrict__ kflag, int rows,
+                            int nb, int N, int n_valid, double theta) {
+  constexpr int PER = D / 32;  // columns per lane
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (wid >= rows) return;
+  const int bkv = wid / nb, j = wid % nb;
+  const __nv_bfloat16* x = k + ((size_t)bkv * N + (size_t)j * kBlock) * D + lane * PER;
+  int nv = n_valid - j * kBlock;
+  nv = nv > kBlock ? kBlock : nv;
+  double acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.0;
+  for (int t = 0; t < nv; ++t) {
+    float f[PER];
+    if (PER == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(x + (size_t)t * D);
+      const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
+      f[0] = a.x; f[1] = a.y; f[PER > 2 ? 2 : 0] = b.x; f[PER > 3 ? 3 : 0] = b.y;
+    } else {
+      const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t*>(x + (size_t)t * D));
+      f[0] = a.x; f[PER > 1 ? 1 : 0] = a.y;
+    }
+    double ss = 0.0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) ss += (double)f[e] * (double)f[e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (ss > 0.0) {
+      const double inv = 1.0 / sqrt(ss);
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] += (double)f[e] * inv;
+    }
+  }
+  double sq = 0.0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) sq += acc[e] * acc[e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if (lane == 0) kflag[wid] = nv > 0 && sq / ((double)nv * (double)nv) < theta ? 1 : 0;
+}
+
 cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
   const sla_config& c = p.c;
   double* qbar = reinterpret_cast<double*>(a.ws + p.off_qbar);
@@ -86,6 +136,16 @@ cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
   dim3 grid(p.nqb, c.B * c.H + c.B * c.H_kv);
   pool_kernel<<<grid, c.d / 2, 0, s>>>(a.q, a.k, qbar, kbar, c.B * c.H, c.N, c.N_valid, c.d,
                                        p.nqb, phiq, gate ? a.w_g : nullptr, gate, c.H);
+  if (c.cos_filter) {
+    // part of routing: the filter flags feed classify / select
+    const int rows = c.B * c.H_kv * p.nkb;
+    uint8_t* kflag = reinterpret_cast<uint8_t*>(a.ws + p.off_kflag);
+    const int blocks = (rows + 7) / 8;
+    if (c.d == 128)
+      kcos_kernel<128><<<blocks, 256, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
+    else
+      kcos_kernel<64><<<blocks, 256, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
+  }
   return cudaGetLastError();
 }
 
@@ -340,7 +400,8 @@ static size_t route_smem(int nb, int rows) {
 __global__ void classify_kernel(const double* __restrict__ scores, int8_t* __restrict__ mask_out,
                                 int32_t* __restrict__ crit, int32_t* __restrict__ neg,
                                 __nv_bfloat16* __restrict__ mmask, int nb, int k_h, int k_l,
-                                int nkb_pad, int nqb_pad, int rows, int n_rows, int linear_all) {
+                                int nkb_pad, int nqb_pad, int rows, int n_rows, int linear_all,
+                                const uint8_t* __restrict__ kflag, int H, int group) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = blockIdx.x * rows + w;  // over B*H*nqb_pad
@@ -359,8 +420,10 @@ __global__ void classify_kernel(const double* __restrict__ scores, int8_t* __res
   uint8_t* flags = base + (size_t)nb * 8;
   unsigned* hist = reinterpret_cast<unsigned*>(base + (size_t)nb * 8 + align_up((size_t)nb, 16));
   const double* srow = scores + ((size_t)bh * nb + i) * nb;
+  // filtered key blocks (cos_filter) score -inf
+  const uint8_t* kf = kflag ? kflag + ((size_t)(bh / H) * (H / group) + (bh % H) / group) * nb : nullptr;
   for (int j = lane; j < nb; j += 32) {
-    keys[j] = order_key(srow[j]);
+    keys[j] = order_key(kf && kf[j] ? -INFINITY : srow[j]);
     flags[j] = 0;
   }
   __syncwarp();
@@ -396,7 +459,10 @@ cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cuda
   const int n_rows = c.B * c.H * per_head;
   const int grid = (n_rows + rows - 1) / rows;
   classify_kernel<<<grid, rows * 32, smem, s>>>(sc, a.mask_out, a.crit, a.neg, mm, p.nkb, c.k_h,
-                                                c.k_l, p.nkb_pad, per_head, rows, n_rows, c.linear_all);
+                                                c.k_l, p.nkb_pad, per_head, rows, n_rows, c.linear_all,
+                                                c.cos_filter ? reinterpret_cast<const uint8_t*>(a.ws + p.off_kflag)
+                                                             : nullptr,
+                                                c.H, p.group);
   return cudaGetLastError();
 }
 
@@ -416,7 +482,7 @@ __host__ __device__ inline size_t select_warp_bytes(int nb) {
 
 __global__ void select_kernel(const double* __restrict__ scores, int8_t* __restrict__ mask_out,
                               int32_t* __restrict__ sel, int H, int group, int nb, int top_n,
-                              int rows, int n_rows) {
+                              int rows, int n_rows, const uint8_t* __restrict__ kflag) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = blockIdx.x * rows + w;  // over B*H_kv*nb
@@ -445,10 +511,15 @@ __global__ void select_kernel(const double* __restrict__ scores, int8_t* __restr
 #pragma unroll 4
     for (int j = i2 + lane; j < i; j += 32) buf[j] = srow[j];
     __syncwarp();
+    if (kflag)  // filtered key blocks (cos_filter) score -inf
+      for (int j = lane; j < i; j += 32)
+        if (kflag[(size_t)bkv * nb + j]) buf[j] = -INFINITY;
+    __syncwarp();
     double m = -INFINITY;
     for (int j = lane; j < i; j += 32) m = fmax(m, buf[j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (m == -INFINITY) continue;  // every candidate filtered: this head adds 0
     double sum = 0.0;
     for (int j = lane; j < i; j += 32) {
       const double e = exp(buf[j] - m);
@@ -487,8 +558,9 @@ cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int n_rows = c.B * c.H_kv * p.nqb;
   const int grid = (n_rows + rows - 1) / rows;
-  select_kernel<<<grid, rows * 32, smem, s>>>(sc, a.mask_out, a.crit, c.H, p.group, p.nkb,
-                                              c.top_n, rows, n_rows);
+  select_kernel<<<grid, rows * 32, smem, s>>>(
+      sc, a.mask_out, a.crit, c.H, p.group, p.nkb, c.top_n, rows, n_rows,
+      c.cos_filter ? reinterpret_cast<const uint8_t*>(a.ws + p.off_kflag) : nullptr);
   return cudaGetLastError();
 }
 

@@ -15,6 +15,7 @@ static sla_status check_config(const sla_config* c) {
   if (c->N % c->block != 0) return SLA_ERR_INVALID_ARG;
   if (c->N_valid > c->N || c->N_valid <= c->N - c->block) return SLA_ERR_INVALID_ARG;
   if (!(c->scale >= 0.f) || !isfinite(c->scale)) return SLA_ERR_INVALID_ARG;
+  if ((c->cos_filter != 0 && c->cos_filter != 1) || !isfinite(c->cos_theta)) return SLA_ERR_INVALID_ARG;
   if (c->block != kBlock) return SLA_ERR_UNSUPPORTED;
   if (c->d != 64 && c->d != 128) return SLA_ERR_UNSUPPORTED;
   const int nb = c->N / c->block;
@@ -63,6 +64,7 @@ bool make_plan(const sla_config* c, Plan* p) {
   p->off_qbar = take(B * H * nqb * d * 8);
   p->off_kbar = take(B * Hkv * nkb * d * 8);
   p->off_scores = take(B * H * nqb * nkb * 8);
+  if (c->cos_filter) p->off_kflag = take(B * Hkv * nkb);  // 1: the key block's pooled scores are -inf
   if (c->mode == SLA_MODE_THREEWAY) {
     p->off_crit = take(B * H * nqb * (size_t)c->k_h * 4);
     p->off_neg = off;

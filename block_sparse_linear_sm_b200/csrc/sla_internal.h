@@ -31,7 +31,7 @@ struct Plan {
   int dd;                // row length of the per-block linear state: d*d + d, padded to 128
   float scale;
   // byte offsets into ws
-  size_t off_status, off_qbar, off_kbar, off_scores, off_crit, off_neg, off_mmask, off_hs, off_ss,
+  size_t off_status, off_qbar, off_kbar, off_scores, off_kflag, off_crit, off_neg, off_mmask, off_hs, off_ss,
       off_zs, off_phiq, off_gate, off_kmean, total;
 };
 

@@ -60,7 +60,9 @@ class LayerConfig:
     has_gate: int = 0
     smooth_k: int = 0             # 1: linear branch on K minus the head's mean valid key
     linear_all: int = 0           # 1: linear branch over all valid key blocks
+    cos_filter: int = 0           # 1: key blocks with CosSim < cos_theta score -inf
     scale: float = 0.0            # 0 -> 1/sqrt(d)
+    cos_theta: float = 0.0
     generator: str = "iid"        # iid | fourier | block_shift
     grid: Optional[tuple] = None  # (t, h, w) for the Fourier generator
     seed: int = 0

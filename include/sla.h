@@ -119,7 +119,12 @@ typedef struct {
                      * branch are unchanged by it (each row shifts by a constant) */
   int32_t linear_all; /* THREEWAY: 1 = the linear branch runs over every valid key block
                        * (all tokens) instead of the marginal blocks only */
+  int32_t cos_filter; /* 1 = key blocks whose CosSim (mean cosine similarity over all
+                       * ordered pairs of their valid tokens) is below cos_theta get a
+                       * pooled score of -inf (2025 review, section 11, SpargeAttn):
+                       * they rank last and get probability 0 in the top-n softmax */
   float scale;      /* softmax scale of pooled scores and attention; 0 = 1/sqrt(d) */
+  float cos_theta;  /* CosSim threshold of cos_filter */
 } sla_config;
 
 /* Checks a configuration without touching any pointer. */

@@ -63,6 +63,8 @@ BAD = [
     (dict(mode=7), sla.SLA_ERR_INVALID_ARG),
     (dict(proj_per_head=2), sla.SLA_ERR_INVALID_ARG),
     (dict(smooth_k=2), sla.SLA_ERR_INVALID_ARG),
+    (dict(cos_filter=3), sla.SLA_ERR_INVALID_ARG),
+    (dict(cos_filter=1, cos_theta=float("nan")), sla.SLA_ERR_INVALID_ARG),
     (dict(linear_all=-1), sla.SLA_ERR_INVALID_ARG),
     (dict(mode=1, causal=1, top_n=4, has_proj=0, smooth_k=1), sla.SLA_ERR_UNSUPPORTED),
     (dict(mode=1, causal=1, top_n=4, has_proj=0, linear_all=1), sla.SLA_ERR_UNSUPPORTED),

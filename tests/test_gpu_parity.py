@@ -20,6 +20,7 @@ if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these 
 
 from gpu_util import (MAX_ABS, MEAN_ABS, GpuRun, check_routing, full_errors,  # noqa: E402
                       unit_errors)
+from oracle import sla_oracle as oracle  # noqa: E402
 
 
 def small(**kw):
@@ -156,6 +157,47 @@ def test_smooth_k_linear_term_with_offset_keys(d):
     rel = np.linalg.norm(got_l - want_l) / np.linalg.norm(want_l)
     print("smooth-K: linear term relative Frobenius error", rel)
     assert rel <= 1e-2  # (absolute output bounds assume O(1) outputs; here V + 3 makes O ~ 3)
+
+
+def _filtered_inputs(cfg, seed=41):
+    """Keys whose blocks range from unrelated tokens to one shared direction, and a
+    CosSim threshold halfway between two neighbouring block values (no block near it)."""
+    x = wl.generate(cfg)
+    rng = np.random.default_rng(seed)
+    kf = wl.bf16_bits_to_f64(x.k)
+    for j in range(cfg.nkb):
+        lo, hi = j * 64, min((j + 1) * 64, cfg.N_valid)
+        mix = 0.9 * (j % 7) / 6.0
+        base = rng.standard_normal((cfg.B, cfg.H_kv, 1, cfg.d))
+        kf[:, :, lo:hi] = mix * base + (1.0 - mix) * kf[:, :, lo:hi]
+    x.k = wl.to_bf16_bits(kf)
+    sims = np.sort(np.concatenate([oracle.block_cos_sims(wl.bf16_bits_to_f64(x.k[b, h]), cfg.N_valid, 64)
+                                   for b in range(cfg.B) for h in range(cfg.H_kv)]))
+    gaps = np.diff(sims)
+    mid = len(sims) // 2
+    g = mid + int(np.argmax(gaps[mid:mid + len(sims) // 4]))
+    return x, float((sims[g] + sims[g + 1]) / 2)
+
+
+FILTER_CASES = [
+    dict(name="filter_d128", N=1536, N_valid=1500, d=128, H=4, H_kv=4, k_h=3, k_l=4, has_gate=1),
+    dict(name="filter_d64_gqa", N=1024, N_valid=1000, d=64, H=4, H_kv=2, k_h=2, k_l=3),
+    dict(name="filter_topn", N=2048, N_valid=2048, d=128, H=8, H_kv=2, mode=wl.MODE_TOPN_WINDOW, causal=1,
+         has_proj=0, top_n=4, window=200, k_h=0, k_l=0),
+]
+
+
+@pytest.mark.parametrize("kw", FILTER_CASES, ids=[c["name"] for c in FILTER_CASES])
+def test_cos_filter_matches_oracle(kw):
+    cfg = small(cos_filter=1, **kw)
+    x, theta = _filtered_inputs(cfg)
+    cfg = cfg.replace(cos_theta=theta)
+    run = GpuRun(cfg, x)
+    L = run.layer()
+    rep = check_routing(run, L)
+    assert rep["mismatched_rows"] == 0, rep
+    err = full_errors(run, L.forward())
+    assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err
 
 
 TOPN_CASES = [
