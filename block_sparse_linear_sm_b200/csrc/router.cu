@@ -77,49 +77,69 @@ __global__ void pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bflo
 // key-block similarity (2025 review, section 11, SpargeAttn: s_kj = CosSim(K_j),
 // S_hat[i, j] = -inf when s_kj < theta): one warp per (KV head row, block);
 // CosSim = |sum_t k_t / |k_t||^2 / n^2 over the n valid tokens, in float64 like
-// the pooled means (a zero token counts as the zero vector). Writes 1 for the
-// blocks below theta.
+// the pooled means (a zero token counts as the zero vector). Each token is
+// handled by D/32 lanes holding 32 columns each, 32/(D/32) tokens at a time;
+// each lane keeps the running sum of its 32 columns of the normalised tokens.
+// Writes 1 for the blocks below theta.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void kcos_kernel(const __nv_bfloat16* __restrict__ k, uint8_t* __restrict__ kflag, int rows,
                             int nb, int N, int n_valid, double theta) {
-  constexpr int PER = D / 32;  // columns per lane
+  constexpr int LPT = D / 32;        // lanes per token
+  constexpr int TPI = 32 / LPT;      // tokens per iteration
   const int lane = threadIdx.x & 31;
   const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (wid >= rows) return;
   const int bkv = wid / nb, j = wid % nb;
-  const __nv_bfloat16* x = k + ((size_t)bkv * N + (size_t)j * kBlock) * D + lane * PER;
+  const int sub = lane % LPT, tk = lane / LPT;  // column part, token slot
   int nv = n_valid - j * kBlock;
   nv = nv > kBlock ? kBlock : nv;
-  double acc[PER];
+  const uint4* x = reinterpret_cast<const uint4*>(k + ((size_t)bkv * N + (size_t)j * kBlock) * D) + sub * 4;
+  double acc[32];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.0;
-  for (int t = 0; t < nv; ++t) {
-    float f[PER];
-    if (PER == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(x + (size_t)t * D);
-      const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
-      f[0] = a.x; f[1] = a.y; f[PER > 2 ? 2 : 0] = b.x; f[PER > 3 ? 3 : 0] = b.y;
+  for (int e = 0; e < 32; ++e) acc[e] = 0.0;
+  for (int t0 = 0; t0 < nv; t0 += TPI) {
+    const int t = t0 + tk;
+    float f[32];
+    if (t < nv) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 u = x[(size_t)t * (D / 8) + c];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 v = unpack_bf16(w[e]);
+          f[8 * c + 2 * e] = v.x;
+          f[8 * c + 2 * e + 1] = v.y;
+        }
+      }
     } else {
-      const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t*>(x + (size_t)t * D));
-      f[0] = a.x; f[PER > 1 ? 1 : 0] = a.y;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) f[e] = 0.f;
     }
     double ss = 0.0;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) ss += (double)f[e] * (double)f[e];
+    for (int e = 0; e < 32; ++e) ss = fma((double)f[e], (double)f[e], ss);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    for (int o = 1; o < LPT; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);  // the token's lanes
     if (ss > 0.0) {
       const double inv = 1.0 / sqrt(ss);
 #pragma unroll
-      for (int e = 0; e < PER; ++e) acc[e] += (double)f[e] * inv;
+      for (int e = 0; e < 32; ++e) acc[e] = fma((double)f[e], inv, acc[e]);
     }
   }
+  // add the token slots' sums (lanes with the same column part), then |sum|^2
   double sq = 0.0;
 #pragma unroll
-  for (int e = 0; e < PER; ++e) sq += acc[e] * acc[e];
+  for (int e = 0; e < 32; ++e) {
+    double v = acc[e];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    for (int o = LPT; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    sq = fma(v, v, sq);
+  }
+  // lanes 0 .. LPT-1 now hold the column parts' shares
+#pragma unroll
+  for (int o = 1; o < LPT; o <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   if (lane == 0) kflag[wid] = nv > 0 && sq / ((double)nv * (double)nv) < theta ? 1 : 0;
 }
 
@@ -140,11 +160,11 @@ cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
     // part of routing: the filter flags feed classify / select
     const int rows = c.B * c.H_kv * p.nkb;
     uint8_t* kflag = reinterpret_cast<uint8_t*>(a.ws + p.off_kflag);
-    const int blocks = (rows + 7) / 8;
+    const int blocks = (rows + 3) / 4;  // four warps (blocks) per CTA
     if (c.d == 128)
-      kcos_kernel<128><<<blocks, 256, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
+      kcos_kernel<128><<<blocks, 128, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
     else
-      kcos_kernel<64><<<blocks, 256, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
+      kcos_kernel<64><<<blocks, 128, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
   }
   return cudaGetLastError();
 }

@@ -120,6 +120,10 @@ def _preset(name: str) -> LayerConfig:
         # the SLA critique page's reading of the open-source code: smooth-K and the
         # linear branch over all tokens, on the Wan2.1-1.3B layer's inputs
         return _preset("wan1.3b").replace(name=name, smooth_k=1, linear_all=1)
+    if name == "wan1.3b_cosfilter":
+        # SpargeAttn's key-block similarity filter on the Wan2.1-1.3B layer: key blocks
+        # whose tokens are least alike (CosSim < 0.1) drop out of the critical set
+        return _preset("wan1.3b").replace(name=name, cos_filter=1, cos_theta=0.1)
     if name == "wan14b":
         k_h, k_l = _counts(0.05, 0.10, 1182)
         return LayerConfig(name, 1, 40, 40, 75648, 75600, 128, k_h=k_h, k_l=k_l,
@@ -128,7 +132,7 @@ def _preset(name: str) -> LayerConfig:
     raise KeyError(name)
 
 
-PRESETS = ("tiny", "wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource")
+PRESETS = ("tiny", "wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource", "wan1.3b_cosfilter")
 
 
 def preset(name: str) -> LayerConfig:

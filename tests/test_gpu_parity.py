@@ -230,7 +230,8 @@ def sampled_units(cfg, n=12, seed=0):
     return sorted(units)
 
 
-@pytest.mark.parametrize("name", ["wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource"])
+@pytest.mark.parametrize("name", ["wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource",
+                                  "wan1.3b_cosfilter"])
 def test_full_size_workload(name):
     cfg = wl.preset(name)
     run = GpuRun(cfg)
