@@ -1,0 +1,147 @@
+"""Pins of the float64 gradient oracle (oracle/sla_grad.py).
+
+The gradient oracle restates the layer in float64 PyTorch and lets autograd
+differentiate it. It is pinned against things other than itself:
+* its forward values equal ``sla_oracle``'s forward pass (the pinned oracle);
+* its gradients equal central finite differences of ``sla_oracle``'s forward
+  pass (routing held fixed), one random direction per input;
+* with every block critical they equal the textbook gradients of dense softmax
+  attention (dV = P^T dO, dS = P * (dP - rowsum(dO * O)), dQ = dS K s, dK = dS^T Q s);
+* with every block negligible they are zero.
+A planted mistake (a gradient that ignores the gate) fails the finite-difference pin.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sla_grad as sg
+from oracle import sla_oracle as so
+
+
+class Cfg:
+    def __init__(self, **kw):
+        base = dict(B=1, H=2, H_kv=2, N=128, N_valid=128, d=8, block=32, mode=0, k_h=1, k_l=1,
+                    top_n=0, window=0, causal=0, has_proj=1, proj_per_head=0, has_gate=1,
+                    smooth_k=0, linear_all=0, cos_filter=0, scale=0.0, cos_theta=0.0)
+        base.update(kw)
+        self.__dict__.update(base)
+
+
+def inputs(c, seed=0):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((c.B, c.H, c.N, c.d))
+    k = rng.standard_normal((c.B, c.H_kv, c.N, c.d))
+    v = rng.standard_normal((c.B, c.H_kv, c.N, c.d))
+    for x in (q, k, v):
+        x[:, :, c.N_valid:] = 0  # padding tokens are zero
+    shape_p = (c.H, c.d, c.d) if c.proj_per_head else (c.d, c.d)
+    w_p = rng.normal(0, 1 / math.sqrt(c.d), shape_p)
+    w_g = rng.normal(0, 1 / math.sqrt(c.d), (c.H, c.d))
+    d_out = rng.standard_normal((c.B, c.H, c.N, c.d))
+    return q, k, v, w_p, w_g, d_out
+
+
+def oracle_loss(c, q, k, v, w_p, w_g, d_out, classes):
+    """sum(O * d_out) from sla_oracle's own forward pass, with the classes given."""
+    layer = so.Layer(c, q, k, v, w_p, w_g)
+    total = 0.0
+    for b in range(c.B):
+        for h in range(c.H):
+            for i in range(c.N // c.block):
+                o = layer.unit(b, h, i, cls_row=classes[b, h, i])["O"]
+                total += float((o * d_out[b, h, i * c.block:(i + 1) * c.block]).sum())
+    return total
+
+
+CASES = {
+    "proj_gate": {},
+    "ragged": dict(N_valid=117),
+    "gqa": dict(H=4, H_kv=2),
+    "per_head_proj": dict(proj_per_head=1),
+    "smooth_k": dict(smooth_k=1),
+    "linear_all": dict(linear_all=1, k_l=2),
+    "plain": dict(has_proj=0, has_gate=0),
+    "all_marginal": dict(k_h=0, k_l=0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_restated_forward_matches_the_oracle(name):
+    c = Cfg(**CASES[name])
+    q, k, v, w_p, w_g, _ = inputs(c, seed=11)
+    ref = so.forward(c, q, k, v, w_p, w_g)["O"]
+    T = lambda a: torch.from_numpy(a)
+    got = sg.layer_forward_torch(c, T(q), T(k), T(v), T(w_p) if c.has_proj else None,
+                                 T(w_g) if c.has_gate else None).numpy()
+    assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def _fd_check(c, grads_fn, seed=5, eps=1e-6, rel=1e-6):
+    q, k, v, w_p, w_g, d_out = inputs(c, seed=seed)
+    classes = so.Layer(c, q, k, v, w_p, w_g).route()[0]
+    g = grads_fn(c, q, k, v, w_p, w_g, d_out, classes)
+    rng = np.random.default_rng(seed + 100)
+    names = ["q", "k", "v"] + (["w_p"] if c.has_proj else []) + (["w_g"] if c.has_gate else [])
+    worst = {}
+    for name in names:
+        args = dict(q=q, k=k, v=v, w_p=w_p, w_g=w_g)
+        delta = rng.standard_normal(args[name].shape)
+        if name in ("q", "k", "v"):
+            delta[:, :, c.N_valid:] = 0
+        plus = dict(args)
+        minus = dict(args)
+        plus[name] = args[name] + eps * delta
+        minus[name] = args[name] - eps * delta
+        fd = (oracle_loss(c, d_out=d_out, classes=classes, **plus) -
+              oracle_loss(c, d_out=d_out, classes=classes, **minus)) / (2 * eps)
+        an = float((g["d" + name] * delta).sum())
+        worst[name] = abs(fd - an) / max(1e-3, abs(fd))
+    return worst
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_gradients_match_finite_differences_of_the_oracle(name):
+    c = Cfg(**CASES[name])
+    worst = _fd_check(c, lambda c, *a: sg.layer_grads(c, *a[:6], classes=a[6]))
+    assert all(e < 1e-6 for e in worst.values()), worst
+
+
+def test_all_critical_gradients_are_dense_attention_gradients():
+    c = Cfg(k_h=4, k_l=0, has_proj=1, has_gate=1, N_valid=117)
+    q, k, v, w_p, w_g, d_out = inputs(c, seed=3)
+    g = sg.layer_grads(c, q, k, v, w_p, w_g, d_out)
+    s = 1 / math.sqrt(c.d)
+    nv = c.N_valid
+    for h in range(c.H):
+        Q, K, V, dO = q[0, h, :nv], k[0, h, :nv], v[0, h, :nv], d_out[0, h, :nv]
+        S = Q @ K.T * s
+        P = np.exp(S - S.max(axis=1, keepdims=True))
+        P /= P.sum(axis=1, keepdims=True)
+        O = P @ V
+        dV = P.T @ dO
+        dP = dO @ V.T
+        dS = P * (dP - (dO * O).sum(axis=1, keepdims=True))
+        np.testing.assert_allclose(g["dq"][0, h, :nv], dS @ K * s, atol=1e-12)
+        np.testing.assert_allclose(g["dk"][0, h, :nv], dS.T @ Q * s, atol=1e-12)
+        np.testing.assert_allclose(g["dv"][0, h, :nv], dV, atol=1e-12)
+        assert np.all(g["dq"][0, h, nv:] == 0) and np.all(g["dk"][0, h, nv:] == 0)
+    # no linear branch: the projection and the gate get no gradient
+    assert np.all(g["dw_p"] == 0) and np.all(g["dw_g"] == 0)
+
+
+def test_all_negligible_gradients_are_zero():
+    c = Cfg(k_h=0, k_l=4)
+    q, k, v, w_p, w_g, d_out = inputs(c, seed=4)
+    g = sg.layer_grads(c, q, k, v, w_p, w_g, d_out)
+    for key in ("dq", "dk", "dv", "dw_p", "dw_g"):
+        assert np.all(g[key] == 0), key
+
+
+def test_planted_gate_without_gradient_is_caught(monkeypatch):
+    c = Cfg(**CASES["proj_gate"])
+    real = torch.sigmoid
+    monkeypatch.setattr(sg.torch, "sigmoid", lambda x: real(x).detach())
+    worst = _fd_check(c, lambda c, *a: sg.layer_grads(c, *a[:6], classes=a[6]))
+    assert max(worst.values()) > 1e-3
