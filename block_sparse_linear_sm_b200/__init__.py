@@ -78,6 +78,17 @@ def lib() -> ctypes.CDLL:
         L.sla_permute_tokens.restype = ctypes.c_int
         L.sla_selftest_wait_timeout.argtypes = [P, S, ctypes.c_int64, P]
         L.sla_selftest_wait_timeout.restype = ctypes.c_int
+        L.sla_backward_workspace_bytes.argtypes = [C]
+        L.sla_backward_workspace_bytes.restype = S
+        bwd = [P, P, P, P, P, C, P, P, P, P, P, P, P, P, S, P, S, P]
+        L.sla_backward.argtypes = bwd
+        L.sla_backward.restype = ctypes.c_int
+        L.sla_backward_timed.argtypes = bwd + [ctypes.POINTER(ctypes.c_void_p), I32]
+        L.sla_backward_timed.restype = ctypes.c_int
+        L.sla_backward_num_stages.argtypes = [C]
+        L.sla_backward_num_stages.restype = I32
+        L.sla_backward_stage_name.argtypes = [C, I32]
+        L.sla_backward_stage_name.restype = ctypes.c_char_p
         L.sla_status_string.argtypes = [ctypes.c_int]
         L.sla_status_string.restype = ctypes.c_char_p
         L.sla_version.argtypes = []
@@ -178,6 +189,45 @@ def sla_forward_timed(q, k, v, w_p, w_g, c, out, mask_out, ws, events, stream=No
                                    ctypes.byref(cfg), _ptr(out), _ptr(mask_out), _ptr(ws),
                                    ws_bytes, _stream(stream), arr, len(events)),
            "sla_forward_timed")
+
+
+def sla_backward_workspace_bytes(c) -> int:
+    cfg = _cfg(c)
+    return int(lib().sla_backward_workspace_bytes(ctypes.byref(cfg)))
+
+
+def sla_backward_num_stages(c) -> int:
+    cfg = _cfg(c)
+    return int(lib().sla_backward_num_stages(ctypes.byref(cfg)))
+
+
+def sla_backward_stage_names(c) -> list:
+    cfg = _cfg(c)
+    n = lib().sla_backward_num_stages(ctypes.byref(cfg))
+    return [lib().sla_backward_stage_name(ctypes.byref(cfg), i).decode() for i in range(max(n, 0))]
+
+
+def _bwd_args(q, k, v, w_p, w_g, c, out, dout, dq, dk, dv, dw_p, dw_g, ws, bws, stream):
+    return (_ptr(q), _ptr(k), _ptr(v), _ptr(w_p), _ptr(w_g), ctypes.byref(_cfg(c)), _ptr(out), _ptr(dout),
+            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_p), _ptr(dw_g), _ptr(ws), ws.numel() * ws.element_size(),
+            _ptr(bws), bws.numel() * bws.element_size(), _stream(stream))
+
+
+def sla_backward(q, k, v, w_p, w_g, c, out, dout, dq, dk, dv, dw_p, dw_g, ws, bws, stream=None) -> None:
+    """Gradients of sum(out * dout); ws is the matching sla_forward call's workspace."""
+    _check(lib().sla_backward(*_bwd_args(q, k, v, w_p, w_g, c, out, dout, dq, dk, dv, dw_p, dw_g, ws, bws,
+                                         stream)), "sla_backward")
+
+
+def sla_backward_timed(q, k, v, w_p, w_g, c, out, dout, dq, dk, dv, dw_p, dw_g, ws, bws, events,
+                       stream=None) -> None:
+    """events: torch.cuda.Event(enable_timing=True) list of length sla_backward_num_stages(c) + 1."""
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(lib().sla_backward_timed(*_bwd_args(q, k, v, w_p, w_g, c, out, dout, dq, dk, dv, dw_p, dw_g, ws,
+                                               bws, stream), arr, len(events)), "sla_backward_timed")
 
 
 def sla_check_device_status(ws, stream=None) -> tuple:

@@ -279,3 +279,47 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
 }
 
 }  // namespace sla
+
+namespace sla {
+
+// Backward: dh'_j = sum_i M[i, j] dS'_i and dz_j = sum_i M[i, j] dZ_i over the
+// query blocks of every query head of the KV group, as the same GEMM with
+//   A = M^T [B*H_kv][nkb_pad rows][group * nqb_pad]   (0/1, exact in bf16)
+//   B = [dS'_i | dZ_i] rows [B*H_kv][group * nqb_pad][dd]
+// and the output rows (key blocks) written to dh [B*H_kv][nkb][d*d] (bf16) and
+// dz [B*H_kv][nkb][d] (fp32).
+cudaError_t launch_aggregate_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  const uint64_t bkv = (uint64_t)c.B * c.H_kv, rows_t = (uint64_t)bp.rows_t;
+  CUtensorMap ma, mb, ms;
+  if (!make_tmap_3d(&ma, a.bws + bp.off_maskt, rows_t, (uint64_t)p.nkb_pad, bkv, rows_t * 2,
+                    (uint64_t)p.nkb_pad * rows_t * 2, 64, 128) ||
+      !make_tmap_3d(&mb, a.bws + bp.off_drow, (uint64_t)p.dd, rows_t, bkv, (uint64_t)p.dd * 2, rows_t * p.dd * 2,
+                    64, 64))
+    return cudaErrorInvalidValue;
+  const uint64_t dsq = (uint64_t)c.d * c.d;
+  if (!make_tmap_3d(&ms, a.bws + bp.off_dh, dsq, (uint64_t)p.nkb, bkv, dsq * 2, (uint64_t)p.nkb * dsq * 2, 64, 128))
+    return cudaErrorInvalidValue;
+  AggParams prm;
+  prm.zs = reinterpret_cast<float*>(a.bws + bp.off_dz);
+  prm.status = a.status;
+  prm.H = c.H_kv;  // one output "head" per KV head, reading its own right-hand side
+  prm.group = 1;
+  prm.nqb = p.nkb;
+  prm.nk_steps = bp.rows_t / 64;
+  prm.d = c.d;
+  prm.m_tiles = (p.nkb + kAgBM - 1) / kAgBM;
+  prm.n_tiles = (p.dd + kAgBN - 1) / kAgBN;
+  prm.tiles = prm.m_tiles * prm.n_tiles * (int)bkv;
+  cudaError_t e = cudaFuncSetAttribute(aggregate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kAgSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = prm.tiles < sms ? prm.tiles : sms;
+  aggregate_tc_kernel<<<grid, kAgThreads, kAgSmem, s>>>(ma, mb, ms, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -1,0 +1,765 @@
+// Backward pass of the sparse branch on the 5th-generation tensor cores.
+//
+// The sparse branch is exact softmax attention of each query block over the
+// key tokens of its critical blocks (SLA analysis page, arXiv 2509.24006;
+// 2025 sparse-attention review, section 2.3, NSA operator design: indexed KV
+// blocks). Its gradient follows the FlashAttention recomputation: with the
+// row log-sum-exp the forward kept (log2 domain, lse2_t), over every critical
+// (query block i, key block j) tile
+//   P = 2^(S * scale * log2 e - lse2),  S = Q_i K_j^T
+//   dP = dO_i V_j^T,  dS = P * (dP - D_t),  D_t = dO_t . O_s,t
+//   dQ_i += scale dS K_j,  dK_j += scale dS^T Q_i,  dV_j += P^T dO_i
+// Two kernels, each with one writer per output row (no atomics):
+//   flash_dq_kernel    128 query rows (blocks 2p, 2p+1 of a head), their merged
+//                      critical key blocks streamed through a two-slot ring;
+//   flash_dkdv_kernel  128 key rows (blocks 2p, 2p+1 of a KV head), for every
+//                      query head of the group the query blocks that hold
+//                      either key block as critical, streamed through a ring.
+// The query blocks of a key block come from a bitmap per (head, key block)
+// that cols_mark_kernel fills from the critical lists.
+// Warps 0-3: one TMEM lane quarter each, thread = row; warp 4: TMA loads and
+// tcgen05.mma issue (one elected lane). Score and dP tiles are double-buffered
+// in TMEM so the next tile's products run while the current one is processed.
+// Both kernels add the linear-branch part of the gradient (fp32 scratch) and
+// write the final bf16 rows.
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace sla {
+
+// ---------------------------------------------------------------------------
+// column bitmaps: bit i of bits[bh][j] is set when query block i has j critical
+// ---------------------------------------------------------------------------
+__global__ void cols_mark_kernel(const int32_t* __restrict__ crit, uint32_t* __restrict__ bits, int64_t entries,
+                                 int nqb, int nkb, int k_h, int words, int* status) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < entries; e += stride) {
+    const int64_t row = e / k_h;  // bh * nqb + i
+    const int bh = (int)(row / nqb), i = (int)(row % nqb);
+    const int j = crit[e];
+    if (j < 0 || j >= nkb) {
+      report(status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
+      continue;
+    }
+    atomicOr(bits + ((size_t)bh * nkb + j) * words + (i >> 5), 1u << (i & 31));
+  }
+}
+
+cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(a.bws + bp.off_bits);
+  cudaError_t e = cudaMemsetAsync(bits, 0, (size_t)c.B * c.H * p.nkb * bp.words * 4, s);
+  if (e != cudaSuccess || c.k_h == 0) return e;
+  const int64_t entries = (int64_t)c.B * c.H * p.nqb * c.k_h;
+  int64_t blocks = (entries + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  cols_mark_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const int32_t*>(a.ws + p.off_crit), bits,
+                                                    entries, p.nqb, p.nkb, c.k_h, bp.words, a.status);
+  return cudaGetLastError();
+}
+
+constexpr int kBwThreads = 160;  // warps 0-3 rows, warp 4 producer / MMA
+
+// ---------------------------------------------------------------------------
+// dQ
+// ---------------------------------------------------------------------------
+template <int D>
+struct DqLayout {
+  static constexpr int NP = D / 64;
+  static constexpr int kOffQ = 0;                         // Q: 128 rows, NP panels of 16 KB
+  static constexpr int kOffO = kOffQ + NP * 16384;        // dO
+  static constexpr int kTile = NP * 8192;                 // one 64-row K or V tile
+  static constexpr int kOffRing = kOffO + NP * 16384;     // 2 slots x (K, V)
+  static constexpr int kOffDS = kOffRing + 4 * kTile;     // dS: 2 buffers x 16 KB (128 rows x 64 keys)
+  static constexpr int kOffBar = kOffDS + 2 * 16384;      // 32 mbarriers
+  static constexpr int kOffMisc = kOffBar + 32 * 8;
+  static constexpr int kOffList = kOffMisc + 64;          // merged block list
+  static constexpr int kTmemCols = 512;                   // dQ: D; S / dP: 2 x 128
+};
+
+struct DqParams {
+  const int32_t* crit;   // [B*H][nqb][k_h]
+  const float* lse;      // [B*H][N] (log2 domain)
+  const float* delta;    // [B*H][N]
+  const float* dq_acc;   // [B*H][N][D] or null
+  __nv_bfloat16* dq;     // [B*H][N][D]
+  int* status;
+  int H, group, N, n_valid, nb, k_h, npairs, words;
+  float scale, scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBwThreads, 1)
+    flash_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DqParams prm) {
+  using L = DqLayout<D>;
+  constexpr int NP = L::NP;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (sbase & 1023u) {
+    if (tid == 0) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashAlign);
+    return;
+  }
+  const int bh = blockIdx.x / prm.npairs, pr = blockIdx.x % prm.npairs;
+  const int bkv = (bh / prm.H) * (prm.H / prm.group) + (bh % prm.H) / prm.group;
+  const int i_h[2] = {2 * pr, 2 * pr + 1};
+  const bool valid_h[2] = {i_h[0] < prm.nb, i_h[1] < prm.nb};
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);  // tmem, count, abort
+  uint32_t* mlist = reinterpret_cast<uint32_t*>(smem + L::kOffList);
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + L::kOffRing);  // bitmaps live in the ring before its first load
+  auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
+  constexpr int QO_FULL = 0, LOADED = 1, SLOT_FREE = 3, SP_FULL = 5, DS_FULL = 7, DS_FREE = 9, ACC_DONE = 11;
+
+  for (int w = tid; w < 2 * prm.words; w += kBwThreads) words[w] = 0u;
+  if (tid == 0) {
+    misc[2] = 0;
+    tc::mbar_init(bar(QO_FULL), 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(bar(LOADED + b), 1);
+      tc::mbar_init(bar(SLOT_FREE + b), 1);
+      tc::mbar_init(bar(SP_FULL + b), 1);
+      tc::mbar_init(bar(DS_FULL + b), 4);
+      tc::mbar_init(bar(DS_FREE + b), 1);
+    }
+    tc::mbar_init(bar(ACC_DONE), 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 4) {
+    tc::tmem_alloc(sbase + L::kOffMisc, L::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  __syncthreads();
+  for (int hf = 0; hf < 2; ++hf) {
+    if (!valid_h[hf]) continue;
+    const int32_t* lst = prm.crit + ((size_t)bh * prm.nb + i_h[hf]) * prm.k_h;
+    for (int e = tid; e < prm.k_h; e += kBwThreads) {
+      const int j = lst[e];
+      if (j < 0 || j >= prm.nb) {
+        report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
+        continue;
+      }
+      atomicOr(&words[hf * prm.words + (j >> 5)], 1u << (j & 31));
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+    for (int w0 = 0; w0 < prm.words; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t a0 = w < prm.words ? words[w] : 0u, a1 = w < prm.words ? words[prm.words + w] : 0u;
+      uint32_t any = a0 | a1;
+      const int cnt = __popc(any);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = base + incl - cnt;
+      while (any) {
+        const int bit = __ffs(any) - 1;
+        any &= any - 1;
+        const uint32_t m = 1u << bit;
+        mlist[pos++] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) misc[1] = base;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const int T = misc[1];
+  const uint32_t tmem = (uint32_t)misc[0];
+  volatile int* abort = misc + 2;
+  const uint32_t sQ = sbase + L::kOffQ, sO = sbase + L::kOffO, sR = sbase + L::kOffRing, sDS = sbase + L::kOffDS;
+
+  if (warp == 4) {
+    // ======================= producer and MMA issuer ==========================
+    constexpr uint32_t kAll = 0xffffffffu;
+    constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
+    constexpr uint32_t kIdQ = tc::idesc_bf16(128, D, false, true);
+    bool ok = true;
+    auto load = [&](int n) {
+      const int slot = n & 1, jb = (int)(mlist[n] & 0xFFFFu);
+      const uint32_t dst = sR + slot * 2 * L::kTile;
+      tc::mbar_expect_tx(bar(LOADED + slot), 2 * L::kTile);
+      for (int p = 0; p < NP; ++p) {
+        tc::tma_load_3d(dst + p * 8192, &tmK, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
+        tc::tma_load_3d(dst + L::kTile + p * 8192, &tmV, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
+      }
+    };
+    auto issue_sp = [&](int n) {
+      // S_n = Q K_n^T and dP_n = dO V_n^T into TMEM buffer n & 1
+      const int slot = n & 1;
+      const uint32_t kt = sR + slot * 2 * L::kTile, vt = kt + L::kTile;
+      const uint32_t tS = tmem + D + 128 * (n & 1);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t qo = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), ko = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
+        tc::mma_bf16_ss(tS, tc::sw128_desc(sQ + qo, 16, 1024), tc::sw128_desc(kt + ko, 16, 1024), kIdS, k > 0);
+        tc::mma_bf16_ss(tS + 64, tc::sw128_desc(sO + qo, 16, 1024), tc::sw128_desc(vt + ko, 16, 1024), kIdS, k > 0);
+      }
+      tc::mma_commit(bar(SP_FULL + (n & 1)));
+    };
+    if (T > 0) {
+      if (lane == 0) {
+        tc::mbar_expect_tx(bar(QO_FULL), 4 * NP * 8192);
+        for (int hf = 0; hf < 2; ++hf)
+          for (int p = 0; p < NP; ++p) {
+            tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmQ, bar(QO_FULL), 64 * p, i_h[hf] * kBlock, bh);
+            tc::tma_load_3d(sO + p * 16384 + hf * 8192, &tmO, bar(QO_FULL), 64 * p, i_h[hf] * kBlock, bh);
+          }
+        for (int n = 0; n < 2 && n < T; ++n) load(n);
+      }
+      __syncwarp();
+      ok = __all_sync(kAll, tc::mbar_wait(bar(QO_FULL), 0, abort));
+      for (int n = 0; n < 2 && n < T && ok; ++n) {
+        ok = __all_sync(kAll, tc::mbar_wait(bar(LOADED + (n & 1)), 0, abort));
+        tc::fence_after_sync();
+        if (ok && tc::elect_one()) issue_sp(n);
+        __syncwarp();
+      }
+      for (int n = 0; n < T && ok; ++n) {
+        const int b = n & 1;
+        ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + b), (n >> 1) & 1, abort));
+        if (!ok) break;
+        tc::fence_after_sync();
+        if (tc::elect_one()) {
+          // dQ += dS_n K_n: A = dS (K-major), B = K_n N-major
+          const uint32_t kt = sR + b * 2 * L::kTile;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16_ss(tmem, tc::sw128_desc(sDS + b * 16384 + kk * 32, 16, 1024),
+                            tc::sw128_desc(kt + kk * 2048, 8192, 1024), kIdQ, (n > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_commit(bar(SLOT_FREE + b));
+          tc::mma_commit(bar(DS_FREE + b));
+          if (n == T - 1) tc::mma_commit(bar(ACC_DONE));
+        }
+        __syncwarp();
+        if (n + 2 < T) {
+          // the slot is free once dQ_n has read K_n: load tile n + 2 and issue its products
+          ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + b), (n >> 1) & 1, abort));
+          if (ok && lane == 0) load(n + 2);
+          __syncwarp();
+          ok = ok && __all_sync(kAll, tc::mbar_wait(bar(LOADED + b), ((n + 2) >> 1) & 1, abort));
+          tc::fence_after_sync();
+          if (ok && tc::elect_one()) issue_sp(n + 2);
+          __syncwarp();
+        }
+      }
+      // the last releases of both slots and dS buffers: no commit is in flight at exit
+      for (int n = (T > 2 ? T - 2 : 0); n < T && ok; ++n)
+        ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + (n & 1)), (n >> 1) & 1, abort)) &&
+             __all_sync(kAll, tc::mbar_wait(bar(DS_FREE + (n & 1)), (n >> 1) & 1, abort));
+      if (!ok && lane == 0) {
+        *abort = 1;
+        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+      }
+    }
+  } else {
+    // ======================= rows: dS, then the dq epilogue ===================
+    const int r = tid, hf = r >> 6;
+    const int t = i_h[hf] * kBlock + (r & 63);
+    const bool vrow = valid_h[hf] && t < prm.n_valid;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float lse2 = vrow ? prm.lse[(size_t)bh * prm.N + t] : INFINITY;
+    const float dlt = vrow ? prm.delta[(size_t)bh * prm.N + t] : 0.f;
+    const float sl2 = prm.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < T && ok; ++n) {
+      const int b = n & 1;
+      const uint32_t e = mlist[n];
+      const int jb = (int)(e & 0xFFFFu);
+      const bool act = (e >> (16 + hf)) & 1u;
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + b), (n >> 1) & 1, abort));
+      if (!ok) break;
+      tc::fence_after_sync();
+      uint32_t sv[2][32], pv[2][32];
+      tc::tmem_ld32(tmem + lane_off + D + 128 * b, sv[0]);
+      tc::tmem_ld32(tmem + lane_off + D + 128 * b + 32, sv[1]);
+      tc::tmem_ld32(tmem + lane_off + D + 128 * b + 64, pv[0]);
+      tc::tmem_ld32(tmem + lane_off + D + 128 * b + 96, pv[1]);
+      tc::tmem_ld_wait();
+      const int k0 = jb * kBlock;
+      uint32_t ds[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float g2[2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int c = 2 * j + x;
+          const float s = __uint_as_float(sv[c >> 5][c & 31]);
+          const float p = (act && k0 + c < prm.n_valid) ? tc::ex2_approx(s * sl2 - lse2) : 0.f;
+          g2[x] = p * (__uint_as_float(pv[c >> 5][c & 31]) - dlt);
+        }
+        ds[j] = pack_bf16(g2[0], g2[1]);
+      }
+      // dS buffer b was last read by dQ_{n-2}
+      if (n >= 2) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(DS_FREE + b), ((n - 2) >> 1) & 1, abort));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(smem + L::kOffDS + b * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(ds[4 * c], ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(DS_FULL + b));
+    }
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(ACC_DONE), 0, abort));
+      tc::fence_after_sync();
+    }
+    if (!ok) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
+    if (valid_h[hf]) {
+      // dq = scale dQ + the linear-branch part (padding rows 0)
+      __nv_bfloat16* dst = prm.dq + ((size_t)bh * prm.N + t) * D;
+      const float* acc = prm.dq_acc ? prm.dq_acc + ((size_t)bh * prm.N + t) * D : nullptr;
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t v[32];
+        if (ok && T > 0) {
+          tc::tmem_ld32(tmem + lane_off + 32 * ch, v);
+          tc::tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float a0 = prm.scale * __uint_as_float(v[2 * j]), a1 = prm.scale * __uint_as_float(v[2 * j + 1]);
+          if (acc) {
+            const float2 x = *reinterpret_cast<const float2*>(acc + 32 * ch + 2 * j);
+            a0 += x.x;
+            a1 += x.y;
+          }
+          w[j] = vrow && ok ? pack_bf16(a0, a1) : 0u;
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 4) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV
+// ---------------------------------------------------------------------------
+template <int D>
+struct DkvLayout {
+  static constexpr int NP = D / 64;
+  static constexpr int kOffK = 0;                              // K: 128 keys, NP panels of 16 KB
+  static constexpr int kOffV = kOffK + NP * 16384;             // V
+  static constexpr int kTile = NP * 8192;                      // one 64-row Q or dO tile
+  static constexpr int kSlot = (2 * kTile + 512 + 1023) / 1024 * 1024;  // Q_i, dO_i, lse_i, delta_i
+  static constexpr int kOffRing = kOffV + NP * 16384;
+  static constexpr int kOffPS = kOffRing + 2 * kSlot;          // 2 buffers x (P^T, dS^T), 16 KB each
+  static constexpr int kOffBar = kOffPS + 4 * 16384;
+  static constexpr int kOffMisc = kOffBar + 32 * 8;
+  static constexpr int kOffList = kOffMisc + 64;               // query blocks of one head
+  static constexpr int kTmemCols = 512;                        // dV, dK: 2 D; S^T / dP^T: 2 x 128
+};
+
+struct DkvParams {
+  const uint32_t* bits;   // [B*H][nkb][words]
+  const float* lse;       // [B*H][N] (log2 domain)
+  const float* delta;     // [B*H][N]
+  const float* dk_acc;    // [B*H_kv][N][D] or null
+  const float* dv_acc;
+  __nv_bfloat16* dk;      // [B*H_kv][N][D]
+  __nv_bfloat16* dv;
+  int* status;
+  int H, group, N, n_valid, nb, npairs, words;
+  float scale, scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBwThreads, 1)
+    flash_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      DkvParams prm) {
+  using L = DkvLayout<D>;
+  constexpr int NP = L::NP;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (sbase & 1023u) {
+    if (tid == 0) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashAlign);
+    return;
+  }
+  const int Hkv = prm.H / prm.group;
+  const int bkv = blockIdx.x / prm.npairs, pr = blockIdx.x % prm.npairs;
+  const int b = bkv / Hkv, hk = bkv % Hkv;
+  const int j_h[2] = {2 * pr, 2 * pr + 1};
+  const bool valid_j[2] = {j_h[0] < prm.nb, j_h[1] < prm.nb};
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);  // tmem, count, abort
+  uint32_t* mlist = reinterpret_cast<uint32_t*>(smem + L::kOffList);
+  auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
+  constexpr int KV_FULL = 0, LOADED = 1, SLOT_FREE = 3, SP_FULL = 5, DS_FULL = 7, PS_FREE = 9, ACC_DONE = 11;
+  const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sR = sbase + L::kOffRing, sPS = sbase + L::kOffPS;
+
+  if (tid == 0) {
+    misc[2] = 0;
+    tc::mbar_init(bar(KV_FULL), 1);
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(bar(LOADED + x), 1);
+      tc::mbar_init(bar(SLOT_FREE + x), 1);
+      tc::mbar_init(bar(SP_FULL + x), 1);
+      tc::mbar_init(bar(DS_FULL + x), 4);
+      tc::mbar_init(bar(PS_FREE + x), 1);
+    }
+    tc::mbar_init(bar(ACC_DONE), 1);
+    tc::fence_mbar_init();
+    tc::mbar_expect_tx(bar(KV_FULL), 4 * NP * 8192);
+    for (int hf = 0; hf < 2; ++hf)
+      for (int p = 0; p < NP; ++p) {
+        tc::tma_load_3d(sK + p * 16384 + hf * 8192, &tmK, bar(KV_FULL), 64 * p, j_h[hf] * kBlock, bkv);
+        tc::tma_load_3d(sV + p * 16384 + hf * 8192, &tmV, bar(KV_FULL), 64 * p, j_h[hf] * kBlock, bkv);
+      }
+  }
+  if (warp == 4) {
+    tc::tmem_alloc(sbase + L::kOffMisc, L::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = (uint32_t)misc[0];
+  volatile int* abort = misc + 2;
+  bool ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(KV_FULL), 0, abort));
+
+  const int r = tid, hf = r >> 6;
+  const int key = j_h[hf] * kBlock + (r & 63);
+  const bool vkey = valid_j[hf] && key < prm.n_valid;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const float sl2 = prm.scale_log2;
+  int m0 = 0;  // tiles of the previous heads (ring slots and TMEM buffers alternate over all tiles)
+  for (int g = 0; g < prm.group; ++g) {
+    const int bh = b * prm.H + hk * prm.group + g;
+    // merged list of the query blocks that hold j0 or j1 as critical
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t* r0 = prm.bits + ((size_t)bh * prm.nb + j_h[0]) * prm.words;
+      const uint32_t* r1 = prm.bits + ((size_t)bh * prm.nb + j_h[1]) * prm.words;
+      int base = 0;
+      for (int w0 = 0; w0 < prm.words; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t a0 = (w < prm.words && valid_j[0]) ? r0[w] : 0u;
+        const uint32_t a1 = (w < prm.words && valid_j[1]) ? r1[w] : 0u;
+        uint32_t any = a0 | a1;
+        const int cnt = __popc(any);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int pos = base + incl - cnt;
+        while (any) {
+          const int bit = __ffs(any) - 1;
+          any &= any - 1;
+          const uint32_t m = 1u << bit;
+          mlist[pos++] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u);
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) misc[1] = base;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const int T = misc[1];
+    if (warp == 4) {
+      // ===================== producer and MMA issuer ==========================
+      constexpr uint32_t kAll = 0xffffffffu;
+      constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
+      constexpr uint32_t kIdA = tc::idesc_bf16(128, D, false, true);
+      auto load = [&](int n, int m) {
+        const int slot = m & 1, i = (int)(mlist[n] & 0xFFFFu);
+        const uint32_t dst = sR + slot * L::kSlot;
+        tc::mbar_expect_tx(bar(LOADED + slot), 2 * L::kTile + 512);
+        for (int p = 0; p < NP; ++p) {
+          tc::tma_load_3d(dst + p * 8192, &tmQ, bar(LOADED + slot), 64 * p, i * kBlock, bh);
+          tc::tma_load_3d(dst + L::kTile + p * 8192, &tmO, bar(LOADED + slot), 64 * p, i * kBlock, bh);
+        }
+        tc::bulk_load(dst + 2 * L::kTile, prm.lse + (size_t)bh * prm.N + i * kBlock, 256, bar(LOADED + slot));
+        tc::bulk_load(dst + 2 * L::kTile + 256, prm.delta + (size_t)bh * prm.N + i * kBlock, 256,
+                      bar(LOADED + slot));
+      };
+      auto issue_sp = [&](int m) {
+        // S^T = K Q_i^T, dP^T = V dO_i^T (M = 128 keys, N = 64 queries)
+        const uint32_t qt = sR + (m & 1) * L::kSlot, ot = qt + L::kTile;
+        const uint32_t tS = tmem + 2 * D + 128 * (m & 1);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t ko = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), qo = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
+          tc::mma_bf16_ss(tS, tc::sw128_desc(sK + ko, 16, 1024), tc::sw128_desc(qt + qo, 16, 1024), kIdS, k > 0);
+          tc::mma_bf16_ss(tS + 64, tc::sw128_desc(sV + ko, 16, 1024), tc::sw128_desc(ot + qo, 16, 1024), kIdS, k > 0);
+        }
+        tc::mma_commit(bar(SP_FULL + (m & 1)));
+      };
+      if (ok && T > 0) {
+        if (lane == 0)
+          for (int n = 0; n < 2 && n < T; ++n) load(n, m0 + n);
+        __syncwarp();
+        for (int n = 0; n < 2 && n < T && ok; ++n) {
+          const int m = m0 + n;
+          ok = __all_sync(kAll, tc::mbar_wait(bar(LOADED + (m & 1)), (m >> 1) & 1, abort));
+          tc::fence_after_sync();
+          if (ok && tc::elect_one()) issue_sp(m);
+          __syncwarp();
+        }
+        for (int n = 0; n < T && ok; ++n) {
+          const int m = m0 + n, x = m & 1;
+          ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
+          if (!ok) break;
+          tc::fence_after_sync();
+          if (tc::elect_one()) {
+            // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T (K-major), B = dO_i / Q_i N-major
+            const uint32_t qt = sR + x * L::kSlot, ot = qt + L::kTile;
+            const uint32_t pt = sPS + x * 32768, dt = pt + 16384;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
+              tc::mma_bf16_ss(tmem, tc::sw128_desc(pt + kk * 32, 16, 1024), tc::sw128_desc(ot + kk * 2048, 8192, 1024),
+                              kIdA, acc);
+              tc::mma_bf16_ss(tmem + D, tc::sw128_desc(dt + kk * 32, 16, 1024),
+                              tc::sw128_desc(qt + kk * 2048, 8192, 1024), kIdA, acc);
+            }
+            tc::mma_commit(bar(SLOT_FREE + x));
+            tc::mma_commit(bar(PS_FREE + x));
+          }
+          __syncwarp();
+          if (n + 2 < T) {
+            ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + x), (m >> 1) & 1, abort));
+            if (ok && lane == 0) load(n + 2, m + 2);
+            __syncwarp();
+            ok = ok && __all_sync(kAll, tc::mbar_wait(bar(LOADED + x), ((m + 2) >> 1) & 1, abort));
+            tc::fence_after_sync();
+            if (ok && tc::elect_one()) issue_sp(m + 2);
+            __syncwarp();
+          }
+        }
+        // this head's last tiles have released their slot and P / dS buffer
+        for (int n = (T > 2 ? T - 2 : 0); n < T && ok; ++n) {
+          const int m = m0 + n;
+          ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + (m & 1)), (m >> 1) & 1, abort)) &&
+               __all_sync(kAll, tc::mbar_wait(bar(PS_FREE + (m & 1)), (m >> 1) & 1, abort));
+        }
+      }
+    } else if (ok) {
+      // ===================== rows: P^T and dS^T =============================
+      for (int n = 0; n < T && ok; ++n) {
+        const int m = m0 + n, x = m & 1;
+        const bool act = (mlist[n] >> (16 + hf)) & 1u;
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + x), (m >> 1) & 1, abort)) &&
+             __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED + x), (m >> 1) & 1, abort));
+        if (!ok) break;
+        tc::fence_after_sync();
+        uint32_t sv[2][32], pv[2][32];
+        const uint32_t tS = tmem + lane_off + 2 * D + 128 * x;
+        tc::tmem_ld32(tS, sv[0]);
+        tc::tmem_ld32(tS + 32, sv[1]);
+        tc::tmem_ld32(tS + 64, pv[0]);
+        tc::tmem_ld32(tS + 96, pv[1]);
+        tc::tmem_ld_wait();
+        const float* lse = reinterpret_cast<const float*>(smem + L::kOffRing + x * L::kSlot + 2 * L::kTile);
+        const float* dl = lse + 64;
+        uint32_t pw[32], dw[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float pp[2], dd[2];
+#pragma unroll
+          for (int y = 0; y < 2; ++y) {
+            const int c = 2 * j + y;
+            const float s = __uint_as_float(sv[c >> 5][c & 31]);
+            const float p = (act && vkey) ? tc::ex2_approx(s * sl2 - lse[c]) : 0.f;
+            pp[y] = p;
+            dd[y] = p * (__uint_as_float(pv[c >> 5][c & 31]) - dl[c]);
+          }
+          pw[j] = pack_bf16(pp[0], pp[1]);
+          dw[j] = pack_bf16(dd[0], dd[1]);
+        }
+        if (m >= 2) {
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(PS_FREE + x), ((m - 2) >> 1) & 1, abort));
+          if (!ok) break;
+        }
+        unsigned char* pt = smem + L::kOffPS + x * 32768;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t off = (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+          *reinterpret_cast<uint4*>(pt + off) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+          *reinterpret_cast<uint4*>(pt + 16384 + off) = make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]);
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar(DS_FULL + x));
+      }
+    }
+    m0 += T;
+  }
+  // every warp agrees on the outcome before the epilogue
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (*abort) ok = false;
+  if (warp == 4) {
+    if (ok && m0 > 0 && tc::elect_one()) tc::mma_commit(bar(ACC_DONE));
+    __syncwarp();
+  } else {
+    if (ok && m0 > 0) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(ACC_DONE), 0, abort));
+      tc::fence_after_sync();
+    }
+    if (valid_j[hf]) {
+      // dk = scale dK + linear part, dv = dV + linear part (padding keys 0)
+      const size_t row = (size_t)bkv * prm.N + key;
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* dst = (which == 0 ? prm.dv : prm.dk) + row * D;
+        const float* acc = which == 0 ? prm.dv_acc : prm.dk_acc;
+        if (acc) acc += row * D;
+        const float sc = which == 0 ? 1.f : prm.scale;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t v[32];
+          if (ok && m0 > 0) {
+            tc::tmem_ld32(tmem + lane_off + which * D + 32 * ch, v);
+            tc::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float a0 = sc * __uint_as_float(v[2 * j]), a1 = sc * __uint_as_float(v[2 * j + 1]);
+            if (acc) {
+              const float2 xx = *reinterpret_cast<const float2*>(acc + 32 * ch + 2 * j);
+              a0 += xx.x;
+              a1 += xx.y;
+            }
+            w[j] = vkey && ok ? pack_bf16(a0, a1) : 0u;
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        }
+      }
+    }
+  }
+  if (!ok && lane == 0) {
+    *abort = 1;
+    report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 4) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static bool map64(CUtensorMap* m, const void* base, int heads, int n_rows, int N, int D) {
+  return make_tmap_3d(m, base, (uint64_t)D, (uint64_t)n_rows, (uint64_t)heads, (uint64_t)D * 2,
+                      (uint64_t)N * D * 2, 64, 64);
+}
+
+template <int D>
+static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  using L = DqLayout<D>;
+  const sla_config& c = p.c;
+  CUtensorMap mq, mo, mk, mv;
+  if (!map64(&mq, a.q, c.B * c.H, c.N_valid, c.N, D) || !map64(&mo, a.dout, c.B * c.H, c.N_valid, c.N, D) ||
+      !map64(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) || !map64(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
+    return cudaErrorInvalidValue;
+  DqParams prm;
+  prm.crit = reinterpret_cast<const int32_t*>(a.ws + p.off_crit);
+  prm.lse = reinterpret_cast<const float*>(a.ws + p.off_lse);
+  prm.delta = reinterpret_cast<const float*>(a.bws + bp.off_delta);
+  prm.dq_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dqacc) : nullptr;
+  prm.dq = a.dq;
+  prm.status = a.status;
+  prm.H = c.H;
+  prm.group = p.group;
+  prm.N = c.N;
+  prm.n_valid = c.N_valid;
+  prm.nb = p.nkb;
+  prm.k_h = c.k_h;
+  prm.npairs = (p.nqb + 1) / 2;
+  prm.words = (p.nkb + 31) / 32;
+  prm.scale = p.scale;
+  prm.scale_log2 = p.scale * 1.4426950408889634f;
+  const int cap = 2 * c.k_h < p.nkb ? 2 * c.k_h : p.nkb;
+  int smem = L::kOffList + (cap > 0 ? cap : 1) * 4;
+  if (2 * prm.words * 4 > 4 * L::kTile) return cudaErrorInvalidValue;  // bitmaps in the ring
+  // one CTA per SM: each holds all 512 TMEM columns
+  if (smem < 120 * 1024) smem = 120 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  flash_dq_kernel<D><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flash_dq(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  return p.c.d == 128 ? launch_dq_t<128>(p, bp, a, s) : launch_dq_t<64>(p, bp, a, s);
+}
+
+template <int D>
+static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  using L = DkvLayout<D>;
+  const sla_config& c = p.c;
+  CUtensorMap mq, mo, mk, mv;
+  if (!map64(&mq, a.q, c.B * c.H, c.N_valid, c.N, D) || !map64(&mo, a.dout, c.B * c.H, c.N_valid, c.N, D) ||
+      !map64(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) || !map64(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
+    return cudaErrorInvalidValue;
+  DkvParams prm;
+  prm.bits = reinterpret_cast<const uint32_t*>(a.bws + bp.off_bits);
+  prm.lse = reinterpret_cast<const float*>(a.ws + p.off_lse);
+  prm.delta = reinterpret_cast<const float*>(a.bws + bp.off_delta);
+  prm.dk_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dkacc) : nullptr;
+  prm.dv_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dvacc) : nullptr;
+  prm.dk = a.dk;
+  prm.dv = a.dv;
+  prm.status = a.status;
+  prm.H = c.H;
+  prm.group = p.group;
+  prm.N = c.N;
+  prm.n_valid = c.N_valid;
+  prm.nb = p.nkb;
+  prm.npairs = (p.nkb + 1) / 2;
+  prm.words = bp.words;
+  prm.scale = p.scale;
+  prm.scale_log2 = p.scale * 1.4426950408889634f;
+  int smem = L::kOffList + p.nqb * 4;
+  if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (512 TMEM columns)
+  cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  flash_dkdv_kernel<D><<<c.B * c.H_kv * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flash_dkdv(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  return p.c.d == 128 ? launch_dkdv_t<128>(p, bp, a, s) : launch_dkdv_t<64>(p, bp, a, s);
+}
+
+}  // namespace sla

@@ -46,6 +46,7 @@ struct FlashTcParams {
   int pair_heads;       // 1: halves are heads (2hp, 2hp+1) of a group; 0: query blocks (2p, 2p+1)
   const float* zs;     // fused epilogue: Z_i [B*H][nqb][D] (fp32)
   const float* gate;   // fused epilogue: g_t = sigmoid(q_t . w_g[h]) [B*H][N] (fp32) or null
+  float* lse;           // [B*H][N] row log2-sum-exp of the scaled scores (+inf: no key), or null
   int npairs;           // units per (b, h) when pairing query blocks
   int words;            // 32-bit words of one block bitmap
   int list_cap;         // capacity of the merged list
@@ -536,6 +537,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       *abort = 1;
       report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
     }
+    // the backward pass recomputes P = 2^(s * scale * log2 e - lse) from this
+    if (prm.lse != nullptr && valid_h[hf])
+      prm.lse[(size_t)bh_h[hf] * prm.N + t] =
+          (ok && T > 0 && l_sum > 0.f && t < prm.n_valid) ? m_ref + log2f(l_sum) : INFINITY;
     if (FUSE) {
       // ---- fused epilogue of the layer (three-way mode with a linear branch) ----
       // den = phi(q) . Z_i from the tiles the producer loaded
@@ -662,6 +667,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
   prm.o = a.out;  // the sparse branch is the output, or the fused epilogue writes it
   prm.zs = FUSE ? reinterpret_cast<const float*>(a.ws + p.off_zs) : nullptr;
   prm.gate = FUSE && c.has_gate ? reinterpret_cast<const float*>(a.ws + p.off_gate) : nullptr;
+  prm.lse = !TOPN ? reinterpret_cast<float*>(a.ws + p.off_lse) : nullptr;
   prm.status = a.status;
   prm.H = c.H;
   prm.group = p.group;

@@ -68,6 +68,7 @@ bool make_plan(const sla_config* c, Plan* p) {
   if (c->mode == SLA_MODE_THREEWAY) {
     p->off_crit = take(B * H * nqb * (size_t)c->k_h * 4);
     p->off_neg = off;
+    p->off_lse = take(B * H * (size_t)c->N * 4);  // row log2-sum-exp of the sparse branch (backward)
     const bool marginal = p->nkb - c->k_h - c->k_l > 0 || c->linear_all;
     if (marginal) {
       p->off_mmask = take(B * H * (size_t)p->nqb_pad * p->nkb_pad * 2);
@@ -178,6 +179,146 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
   return SLA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// backward pass
+// ---------------------------------------------------------------------------
+static sla_status check_bwd_config(const sla_config* c) {
+  const sla_status st = check_config(c);
+  if (st != SLA_OK) return st;
+  if (c->mode != SLA_MODE_THREEWAY || c->smooth_k) return SLA_ERR_UNSUPPORTED;
+  return SLA_OK;
+}
+
+bool make_bwd_plan(const Plan& p, BwdPlan* b) {
+  memset(b, 0, sizeof(*b));
+  const sla_config& c = p.c;
+  b->lin = has_marginal(p);
+  b->rows_t = p.group * p.nqb_pad;
+  b->words = (p.nqb + 31) / 32;
+  const size_t B = c.B, H = c.H, Hkv = c.H_kv, d = c.d, N = c.N;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  b->off_status = take(256);
+  b->off_delta = take(B * H * N * 4);                       // D_t = dO_t . O_s,t
+  b->off_bits = take(B * H * p.nkb * (size_t)b->words * 4);  // query blocks of each key block
+  if (b->lin) {
+    b->off_dqacc = take(B * H * N * d * 4);    // linear-branch and gate part of dq (fp32)
+    b->off_dkacc = take(B * Hkv * N * d * 4);  // linear-branch part of dk, dv (fp32)
+    b->off_dvacc = take(B * Hkv * N * d * 4);
+    b->off_drow = take(B * Hkv * (size_t)b->rows_t * p.dd * 2);         // [dS'_i | dZ_i] rows (bf16)
+    b->off_maskt = take(B * Hkv * (size_t)p.nkb_pad * b->rows_t * 2);   // transposed aggregation mask
+    b->off_dh = take(B * Hkv * (size_t)p.nkb * d * d * 2);              // dh'_j (bf16)
+    b->off_dz = take(B * Hkv * (size_t)p.nkb * d * 4);                  // dz_j (fp32)
+  }
+  b->total = off;
+  return true;
+}
+
+enum BStage { kBZeroCols, kBDelta, kBLinear, kBMaskT, kBAggT, kBState, kBDq, kBDkdv };
+
+static int bwd_stages_of(const BwdPlan& bp, BStage* out) {
+  int n = 0;
+  out[n++] = kBZeroCols;
+  if (bp.lin) {
+    out[n++] = kBLinear;
+    out[n++] = kBMaskT;
+    out[n++] = kBAggT;
+    out[n++] = kBState;
+  } else {
+    out[n++] = kBDelta;
+  }
+  out[n++] = kBDq;
+  out[n++] = kBDkdv;
+  return n;
+}
+
+static const char* bwd_stage_name(BStage s) {
+  switch (s) {
+    case kBZeroCols: return "bwd_columns";
+    case kBDelta: return "bwd_delta";
+    case kBLinear: return "bwd_linear";
+    case kBMaskT: return "bwd_mask_transpose";
+    case kBAggT: return "bwd_aggregate_t";
+    case kBState: return "bwd_state";
+    case kBDq: return "bwd_flash_dq";
+    case kBDkdv: return "bwd_flash_dkdv";
+  }
+  return "?";
+}
+
+static cudaError_t run_bwd_stage(BStage st, const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  switch (st) {
+    case kBZeroCols: {
+      // parameter gradients are sums of atomically added partials
+      cudaError_t e = cudaSuccess;
+      if (c.has_proj)
+        e = cudaMemsetAsync(a.dw_p, 0, (size_t)(c.proj_per_head ? c.H : 1) * c.d * c.d * 4, s);
+      if (e == cudaSuccess && c.has_gate) e = cudaMemsetAsync(a.dw_g, 0, (size_t)c.H * c.d * 4, s);
+      return e == cudaSuccess ? launch_cols(p, bp, a, s) : e;
+    }
+    case kBDelta: return launch_delta(p, bp, a, s);
+    case kBLinear: return launch_lin_bwd(p, bp, a, s);
+    case kBMaskT: return launch_mask_t(p, bp, a, s);
+    case kBAggT: return launch_aggregate_t(p, bp, a, s);
+    case kBState: return launch_state_bwd(p, bp, a, s);
+    case kBDq: return launch_flash_dq(p, bp, a, s);
+    case kBDkdv: return launch_flash_dkdv(p, bp, a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+static sla_status backward_impl(const void* q, const void* k, const void* v, const void* w_p, const void* w_g,
+                                const sla_config* cfg, const void* out, const void* dout, void* dq, void* dk,
+                                void* dv, float* dw_p, float* dw_g, const void* ws, size_t ws_bytes, void* bws,
+                                size_t bws_bytes, void* stream, void* const* events, int32_t n_events) {
+  const sla_status st = check_bwd_config(cfg);
+  if (st != SLA_OK) return st;
+  Plan p;
+  BwdPlan bp;
+  make_plan(cfg, &p);
+  make_bwd_plan(p, &bp);
+  const void* bf[] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* x : bf)
+    if (!x || !aligned(x, 16)) return SLA_ERR_INVALID_ARG;
+  if (cfg->has_proj && (!w_p || !aligned(w_p, 16) || !dw_p || !aligned(dw_p, 16))) return SLA_ERR_INVALID_ARG;
+  if (cfg->has_gate && (!w_g || !aligned(w_g, 16) || !dw_g || !aligned(dw_g, 16))) return SLA_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return SLA_ERR_WORKSPACE;
+  if (!bws || !aligned(bws, 256) || bws_bytes < bp.total) return SLA_ERR_WORKSPACE;
+  BStage stages[8];
+  const int ns = bwd_stages_of(bp, stages);
+  if (events && n_events != ns + 1) return SLA_ERR_INVALID_ARG;
+  BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = (const __nv_bfloat16*)q;
+  a.k = (const __nv_bfloat16*)k;
+  a.v = (const __nv_bfloat16*)v;
+  a.w_p = (const __nv_bfloat16*)w_p;
+  a.w_g = (const __nv_bfloat16*)w_g;
+  a.out = (const __nv_bfloat16*)out;
+  a.dout = (const __nv_bfloat16*)dout;
+  a.dq = (__nv_bfloat16*)dq;
+  a.dk = (__nv_bfloat16*)dk;
+  a.dv = (__nv_bfloat16*)dv;
+  a.dw_p = dw_p;
+  a.dw_g = dw_g;
+  a.ws = (const char*)ws;
+  a.bws = (char*)bws;
+  a.status = (int*)((char*)bws + bp.off_status);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(a.status, 0, 8, s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (events && cudaEventRecord((cudaEvent_t)events[0], s) != cudaSuccess) return SLA_ERR_CUDA;
+  for (int i = 0; i < ns; ++i) {
+    if (run_bwd_stage(stages[i], p, bp, a, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (events && cudaEventRecord((cudaEvent_t)events[i + 1], s) != cudaSuccess) return SLA_ERR_CUDA;
+  }
+  return SLA_OK;
+}
+
 }  // namespace sla
 
 using namespace sla;
@@ -261,6 +402,53 @@ sla_status sla_check_device_status(void* ws, void* stream, int32_t* detail) {
   if (st[0] == 0) return SLA_OK;
   if (st[0] == SLA_ERR_DEVICE_TIMEOUT || st[0] == SLA_ERR_DEVICE_CHECK) return (sla_status)st[0];
   return SLA_ERR_DEVICE_CHECK;
+}
+
+size_t sla_backward_workspace_bytes(const sla_config* cfg) {
+  if (check_bwd_config(cfg) != SLA_OK) return 0;
+  Plan p;
+  BwdPlan bp;
+  make_plan(cfg, &p);
+  make_bwd_plan(p, &bp);
+  return bp.total;
+}
+
+sla_status sla_backward(const void* q, const void* k, const void* v, const void* w_p, const void* w_g,
+                        const sla_config* cfg, const void* out, const void* dout, void* dq, void* dk, void* dv,
+                        float* dw_p, float* dw_g, const void* ws, size_t ws_bytes, void* bws, size_t bws_bytes,
+                        void* stream) {
+  return backward_impl(q, k, v, w_p, w_g, cfg, out, dout, dq, dk, dv, dw_p, dw_g, ws, ws_bytes, bws, bws_bytes,
+                       stream, nullptr, 0);
+}
+
+sla_status sla_backward_timed(const void* q, const void* k, const void* v, const void* w_p, const void* w_g,
+                              const sla_config* cfg, const void* out, const void* dout, void* dq, void* dk,
+                              void* dv, float* dw_p, float* dw_g, const void* ws, size_t ws_bytes, void* bws,
+                              size_t bws_bytes, void* stream, void* const* events, int32_t n_events) {
+  if (!events) return SLA_ERR_INVALID_ARG;
+  return backward_impl(q, k, v, w_p, w_g, cfg, out, dout, dq, dk, dv, dw_p, dw_g, ws, ws_bytes, bws, bws_bytes,
+                       stream, events, n_events);
+}
+
+int32_t sla_backward_num_stages(const sla_config* cfg) {
+  if (check_bwd_config(cfg) != SLA_OK) return -1;
+  Plan p;
+  BwdPlan bp;
+  make_plan(cfg, &p);
+  make_bwd_plan(p, &bp);
+  BStage st[8];
+  return bwd_stages_of(bp, st);
+}
+
+const char* sla_backward_stage_name(const sla_config* cfg, int32_t s) {
+  if (check_bwd_config(cfg) != SLA_OK) return nullptr;
+  Plan p;
+  BwdPlan bp;
+  make_plan(cfg, &p);
+  make_bwd_plan(p, &bp);
+  BStage st[8];
+  const int n = bwd_stages_of(bp, st);
+  return (s >= 0 && s < n) ? bwd_stage_name(st[s]) : nullptr;
 }
 
 const char* sla_status_string(sla_status s) {

@@ -32,7 +32,7 @@ struct Plan {
   float scale;
   // byte offsets into ws
   size_t off_status, off_qbar, off_kbar, off_scores, off_kflag, off_crit, off_neg, off_mmask, off_hs, off_ss,
-      off_zs, off_phiq, off_gate, off_kmean, total;
+      off_zs, off_phiq, off_gate, off_kmean, off_lse, total;
 };
 
 bool make_plan(const sla_config* c, Plan* p);
@@ -66,5 +66,37 @@ cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// backward pass (three-way mode)
+// ---------------------------------------------------------------------------
+// Carve-up of the backward scratch (bws). nqb_pad rows per query head of a KV
+// group form the K extent of the transposed aggregation.
+struct BwdPlan {
+  bool lin;       // the layer has a linear branch
+  int rows_t;     // group * nqb_pad
+  int words;      // 32-bit words of one column bitmap (query blocks)
+  size_t off_status, off_delta, off_dqacc, off_dkacc, off_dvacc, off_drow, off_maskt, off_dh, off_dz,
+      off_bits, off_cols, off_ccnt, total;
+};
+bool make_bwd_plan(const Plan& p, BwdPlan* b);
+
+struct BwdArgs {
+  const __nv_bfloat16 *q, *k, *v, *w_p, *w_g, *out, *dout;
+  __nv_bfloat16 *dq, *dk, *dv;
+  float *dw_p, *dw_g;
+  const char* ws;  // the forward pass's workspace (read only)
+  char* bws;       // backward scratch
+  int* status;     // in bws
+};
+
+cudaError_t launch_delta(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_lin_bwd(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_mask_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_aggregate_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_state_bwd(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_flash_dq(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_flash_dkdv(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
 
 }  // namespace sla

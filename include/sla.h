@@ -225,6 +225,69 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
                                       int32_t rows, int32_t n_tok, int32_t d, int32_t inverse,
                                       void* stream);
 
+/*
+ * Backward pass of the three-way layer (fine-tuning with the layer in place:
+ * SLA analysis page, arXiv 2509.24006, and SALAD summary, both train the model
+ * with the sparse+linear layer for a few steps). The pages print no backward
+ * pass; the gradients are those of L = sum(out * dout) with the routing held
+ * fixed (the block classes are piecewise constant in the pooled scores and
+ * carry no gradient):
+ *   sparse branch   FlashAttention-style recomputation over the critical
+ *                   blocks with the row log-sum-exp sla_forward kept in ws:
+ *                   P = softmax rows, dP = dO V^T, dS = P * (dP - D_t),
+ *                   D_t = dO_t . O_s,t; dQ = scale dS K, dK = scale dS^T Q,
+ *                   dV = P^T dO (restricted to critical tiles)
+ *   linear branch   u_t = phi(q_t) S'_i / (phi(q_t) . Z_i) with S'_i = S_i W_p,
+ *                   du = g dO; dS'_i = sum_t phi(q_t)^T du_t / den_t,
+ *                   dZ_i = -sum_t phi(q_t) (du_t . u_t) / den_t,
+ *                   dh'_j = sum over rows i with j marginal of dS'_i (dz_j alike),
+ *                   dphi(K_j) = (V_j W_p) dh'_j^T + dz_j, dV_j = phi(K_j) dh'_j W_p^T,
+ *                   dW_p = sum_j V_j^T phi(K_j) dh'_j, chained through phi'
+ *   gate            dg_t = dO_t . u_t, dlogit = dg g (1 - g): dq += dlogit w_g[h],
+ *                   dw_g[h] += sum_t dlogit q_t
+ *
+ * Arguments:
+ *   q, k, v, w_p, w_g, cfg  exactly as passed to the sla_forward call that
+ *                           produced `out` (same values)
+ *   out                     bf16 [B, H, N, d]: that call's output
+ *   dout                    bf16 [B, H, N, d]: dL/dout (padding rows are ignored)
+ *   dq                      bf16 [B, H, N, d]   written (padding rows 0)
+ *   dk, dv                  bf16 [B, H_kv, N, d] written (padding rows 0)
+ *   dw_p                    fp32, shape of w_p; written; may be NULL unless has_proj
+ *   dw_g                    fp32 [H, d]; written; may be NULL unless has_gate
+ *   ws                      the workspace of that sla_forward call, unchanged
+ *                           since: the routing, the states S'_i, Z_i, phi(Q),
+ *                           the gate and the row log-sum-exp are read from it
+ *   bws                     device scratch of sla_backward_workspace_bytes(cfg)
+ *                           bytes, 256-byte aligned; its first 256 bytes hold
+ *                           this call's device status word (read it with
+ *                           sla_check_device_status(bws, ...))
+ * SLA_ERR_UNSUPPORTED for the top-n mode and for smooth_k; other errors as for
+ * sla_forward. The parameter gradients are sums of per-block partials added
+ * with floating-point atomics, so their last bits may vary from run to run;
+ * dq, dk and dv are deterministic.
+ */
+SLA_API size_t sla_backward_workspace_bytes(const sla_config* cfg);
+SLA_API sla_status sla_backward(const void* q, const void* k, const void* v,
+                                const void* w_p, const void* w_g, const sla_config* cfg,
+                                const void* out, const void* dout,
+                                void* dq, void* dk, void* dv, float* dw_p, float* dw_g,
+                                const void* ws, size_t ws_bytes, void* bws, size_t bws_bytes,
+                                void* stream);
+
+/* Number of stages (kernel launches and memsets) sla_backward enqueues for cfg, or -1;
+ * stage names as for the forward pass. */
+SLA_API int32_t sla_backward_num_stages(const sla_config* cfg);
+SLA_API const char* sla_backward_stage_name(const sla_config* cfg, int32_t s);
+
+/* sla_backward with caller-created CUDA events around its stages, as sla_forward_timed. */
+SLA_API sla_status sla_backward_timed(const void* q, const void* k, const void* v,
+                                      const void* w_p, const void* w_g, const sla_config* cfg,
+                                      const void* out, const void* dout,
+                                      void* dq, void* dk, void* dv, float* dw_p, float* dw_g,
+                                      const void* ws, size_t ws_bytes, void* bws, size_t bws_bytes,
+                                      void* stream, void* const* events, int32_t n_events);
+
 /* Static description of a status code. */
 SLA_API const char* sla_status_string(sla_status s);
 

@@ -1,0 +1,127 @@
+"""GPU parity of the backward pass (sla_backward) against the float64 gradient oracle.
+
+Each case runs sla_forward and then sla_backward through the C ABI on seeded
+bf16 inputs and a seeded bf16 dO. It compares dq, dk, dv, dW_p and dw_g element
+by element with oracle/sla_grad.py, which gets the same bf16 values and the
+GPU's own routing classes. Bar: relative Frobenius error <= 2e-2 per tensor.
+The arithmetic rounds P, dS, phi(K), the states and the outputs to bf16 (about
+4e-3 each), so a dropped term or a wrong index shows up as an O(1) error.
+The all-critical cases check the sparse branch alone, the all-marginal ones
+the linear branch, the projection and the gate alone.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import block_sparse_linear_sm_b200 as sla  # noqa: E402
+from block_sparse_linear_sm_b200 import workloads as wl  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these anyway
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from gpu_util import GpuRun, bf16_to_f64, to_dev  # noqa: E402
+from oracle import sla_grad  # noqa: E402
+
+REL = 2e-2
+
+
+def d_out_bits(c, seed):
+    rng = np.random.default_rng(seed)
+    return wl.to_bf16_bits(rng.standard_normal((c.B, c.H, c.N, c.d)))
+
+
+def run_backward(cfg, seed=3, v_shift=0.0):
+    x = wl.generate(cfg, v_shift=v_shift)
+    run = GpuRun(cfg, x, route=False)
+    c = cfg
+    dob = d_out_bits(c, seed)
+    dout = to_dev(dob)
+    dq, dk, dv = torch.empty_like(run.q), torch.empty_like(run.k), torch.empty_like(run.v)
+    dw_p = dw_g = None
+    if c.has_proj:
+        shape = (c.H, c.d, c.d) if c.proj_per_head else (c.d, c.d)
+        dw_p = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
+    if c.has_gate:
+        dw_g = torch.full((c.H, c.d), float("nan"), dtype=torch.float32, device="cuda")
+    nbytes = sla.sla_backward_workspace_bytes(c)
+    assert nbytes > 0
+    bws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    sla.sla_backward(run.q, run.k, run.v, run.w_p, run.w_g, c, run.out, dout, dq, dk, dv, dw_p, dw_g,
+                     run.ws, bws)
+    st, detail = sla.sla_check_device_status(bws)
+    assert st == 0, (st, detail)
+    classes = run.mask.cpu().numpy()
+    ref = sla_grad.layer_grads(c, x.f64("q"), x.f64("k"), x.f64("v"),
+                               x.f64("w_p") if c.has_proj else None,
+                               x.f64("w_g") if c.has_gate else None,
+                               wl.bf16_bits_to_f64(dob), classes=classes)
+    got = dict(dq=bf16_to_f64(dq), dk=bf16_to_f64(dk), dv=bf16_to_f64(dv))
+    if dw_p is not None:
+        got["dw_p"] = dw_p.double().cpu().numpy()
+    if dw_g is not None:
+        got["dw_g"] = dw_g.double().cpu().numpy()
+    errs = {}
+    for key, g in got.items():
+        r = ref[key]
+        assert np.all(np.isfinite(g)), key
+        nr = np.linalg.norm(r)
+        errs[key] = float(np.linalg.norm(g - r) / nr) if nr > 0 else float(np.abs(g).max())
+    # padding rows of the gradients are zero
+    for key in ("dq", "dk", "dv"):
+        assert np.all(got[key][:, :, c.N_valid:] == 0), key
+    return errs
+
+
+def small(**kw):
+    return wl.small_config(**kw)
+
+
+CASES = [
+    dict(name="all_crit_d64", N=768, N_valid=763, d=64, k_h=12, k_l=0),
+    dict(name="all_crit_gqa_d128", N=1024, N_valid=1024, d=128, H=4, H_kv=2, k_h=16, k_l=0),
+    dict(name="all_marg_d64", N=1024, N_valid=1000, d=64, k_h=0, k_l=0, has_gate=1),
+    dict(name="all_marg_per_head_d128", N=1024, N_valid=1024, d=128, H=2, H_kv=2, k_h=0, k_l=0,
+         proj_per_head=1, has_gate=1),
+    dict(name="mixed_d64", N=1024, N_valid=1024, d=64, k_h=4, k_l=4, has_gate=1),
+    dict(name="mixed_ragged_d128", N=2048, N_valid=2001, d=128, H=4, H_kv=4, k_h=5, k_l=7, has_gate=1),
+    dict(name="mixed_gqa_d128", N=1536, N_valid=1473, d=128, H=4, H_kv=2, k_h=3, k_l=2, has_gate=1),
+    dict(name="no_proj_d128", N=1024, N_valid=1000, d=128, k_h=2, k_l=2, has_proj=0),
+    dict(name="linear_all_d64", N=1024, N_valid=1000, d=64, k_h=3, k_l=4, linear_all=1),
+    dict(name="odd_blocks_d128", N=1216, N_valid=1200, d=128, k_h=3, k_l=4, has_gate=1),
+    dict(name="batch2_d64", B=2, N=640, N_valid=600, d=64, H=2, H_kv=1, k_h=2, k_l=1, has_gate=1),
+    dict(name="single_block_d128", N=64, N_valid=50, d=128, k_h=1, k_l=0),
+    dict(name="many_tiles_d128", N=4096, N_valid=4096, d=128, H=2, H_kv=2, k_h=16, k_l=16, has_gate=1),
+]
+
+
+@pytest.mark.parametrize("kw", CASES, ids=[c["name"] for c in CASES])
+def test_backward_matches_gradient_oracle(kw):
+    errs = run_backward(small(**kw))
+    print(kw["name"], errs)
+    assert all(e <= REL for e in errs.values()), errs
+
+
+def test_backward_linear_branch_with_shifted_values():
+    """All blocks marginal, V + 3: the linear branch's output is O(1) and dominates dV."""
+    errs = run_backward(small(name="marg_shift", N=1024, N_valid=1024, d=128, k_h=0, k_l=0, has_gate=1),
+                        v_shift=3.0)
+    assert all(e <= REL for e in errs.values()), errs
+
+
+def test_backward_all_negligible_is_zero():
+    c = small(name="all_neg", N=512, N_valid=512, d=64, k_h=0, k_l=8, has_gate=1)
+    x = wl.generate(c)
+    run = GpuRun(c, x, route=False)
+    dout = to_dev(d_out_bits(c, 5))
+    dq, dk, dv = torch.full_like(run.q, 7), torch.full_like(run.k, 7), torch.full_like(run.v, 7)
+    dw_p = torch.full((c.d, c.d), 7.0, device="cuda")
+    dw_g = torch.full((c.H, c.d), 7.0, device="cuda")
+    bws = torch.empty(sla.sla_backward_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    sla.sla_backward(run.q, run.k, run.v, run.w_p, run.w_g, c, run.out, dout, dq, dk, dv, dw_p, dw_g,
+                     run.ws, bws)
+    assert sla.sla_check_device_status(bws) == (0, 0)
+    for t in (dq, dk, dv, dw_p, dw_g):
+        assert torch.count_nonzero(t).item() == 0
