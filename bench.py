@@ -83,6 +83,99 @@ def stage_model(c: wl.LayerConfig) -> dict:
     return m
 
 
+def backward_stage_model(c: wl.LayerConfig) -> dict:
+    """Per backward stage: ("tensor", FLOP) or ("hbm", bytes) of algorithmic work per launch."""
+    B, H, Hkv, N, Nv, d = c.B, c.H, c.H_kv, c.N, c.N_valid, c.d
+    nb = c.nqb
+    bf = 2
+    pairs = c.block * c.block * B * H * nb * c.k_h  # critical (query token, key token) pairs
+    lin = nb - c.k_h - c.k_l > 0 or c.linear_all
+    dd = (d * d + d + 127) // 128 * 128
+    words = (nb + 31) // 32
+    m = {"bwd_columns": ("hbm", B * H * nb * c.k_h * 4 + 2 * B * H * nb * words * 4)}
+    if lin:
+        nqb_pad, nkb_pad = (nb + 127) // 128 * 128, (nb + 63) // 64 * 64
+        # reads phi(Q), q, O, dO, S'_i, Z_i (and g_t); writes the fp32 dq part, D_t, [dS'_i | dZ_i]
+        m["bwd_linear"] = ("hbm", 4 * B * H * Nv * d * bf + B * H * nb * (d * d * bf + d * 4)
+                           + B * H * Nv * 4 * (2 if c.has_gate else 1) + B * H * Nv * d * 4
+                           + B * H * nb * dd * bf)
+        m["bwd_mask_transpose"] = ("hbm", 2 * B * H * nqb_pad * nkb_pad * 2)
+        m["bwd_aggregate_t"] = ("tensor", 2.0 * B * H * nb * nb * dd)  # the forward aggregation, transposed
+        # reads K, V, dh'_j, dz_j; writes the fp32 dk and dv parts
+        m["bwd_state"] = ("hbm", 2 * B * Hkv * Nv * d * bf + B * Hkv * nb * (d * d * bf + d * 4)
+                          + 2 * B * Hkv * Nv * d * 4)
+    else:
+        m["bwd_delta"] = ("hbm", 2 * B * H * Nv * d * bf + B * H * N * 4)
+    # products over the critical tiles: S, dP, dQ (query-stationary) and S^T, dP^T, dV, dK
+    m["bwd_flash_dq"] = ("tensor", 6.0 * d * pairs)
+    m["bwd_flash_dkdv"] = ("tensor", 8.0 * d * pairs)
+    return m
+
+
+def stage_entries(names, stage_ms, model, peaks):
+    out = {}
+    for n in names:
+        kind, work = model[n]
+        t = stage_ms[n] * 1e-3
+        if kind == "tensor":
+            ach = work / t / 1e12
+            out[n] = {"ms": stage_ms[n], "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
+                      "frac": ach / peaks["bf16"], "frac_of_sustained": ach / peaks["bf16_sus"], "work": work}
+        else:
+            ach = work / t / 1e9
+            out[n] = {"ms": stage_ms[n], "bound": "hbm", "achieved": ach, "unit": "GB/s",
+                      "frac": ach / peaks["hbm"], "work": work}
+    return out
+
+
+def measure_backward(sla, torch, cfg, q, k, v, w_p, w_g, out, ws, steps, warmup, dist, dev, stream, peaks):
+    """sla_backward after one sla_forward (whose workspace it reads): per-stage CUDA-event times."""
+    gen = torch.Generator().manual_seed(99)
+    dout = torch.randn(tuple(out.shape), generator=gen).to(torch.bfloat16).to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dw_p = dw_g = None
+    if cfg.has_proj:
+        shape = (cfg.H, cfg.d, cfg.d) if cfg.proj_per_head else (cfg.d, cfg.d)
+        dw_p = torch.empty(shape, dtype=torch.float32, device=dev)
+    if cfg.has_gate:
+        dw_g = torch.empty((cfg.H, cfg.d), dtype=torch.float32, device=dev)
+    bws = torch.empty(sla.sla_backward_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    sla.sla_forward(q, k, v, w_p, w_g, cfg, out, None, ws)
+    names = sla.sla_backward_stage_names(cfg)
+    args = (q, k, v, w_p, w_g, cfg, out, dout, dq, dk, dv, dw_p, dw_g, ws, bws)
+    for _ in range(warmup):
+        sla.sla_backward(*args)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(steps)]
+    for e in evs:
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(steps):
+        sla.sla_backward_timed(*args, evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    st, detail = sla.sla_check_device_status(bws)
+    if st != 0:
+        raise RuntimeError(f"backward device status {st} detail {detail}")
+    (ms,) = max_over_ranks(dist, dev, t0.elapsed_time(t1) / steps)
+    stage_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(steps))
+                for i, n in enumerate(names)}
+    stages = stage_entries(names, stage_ms, backward_stage_model(cfg), peaks)
+    dom = max(names, key=lambda n: stage_ms[n])
+    dk_ = stages[dom]
+    roof = {"kernel": dom, "bound": dk_["bound"], "achieved": dk_["achieved"], "unit": dk_["unit"],
+            "peak": peaks["bf16"] if dk_["bound"] == "tensor" else peaks["hbm"], "frac": dk_["frac"],
+            "peak_kind": (f"bf16 burst, {peaks['src']}" if dk_["bound"] == "tensor"
+                          else f"HBM copy, {peaks['src']}")}
+    del bws, dq, dk, dv, dout
+    return {"ms": ms, "dense_equiv_tflops": 2.5 * cfg.dense_flops() / (ms * 1e-3) / 1e12,
+            "dense_equiv_note": "2.5 x the dense forward FLOP (the usual backward/forward ratio of attention)",
+            "what": "sla_backward: dq, dk, dv, dW_p, dw_g of sum(out * dout), routing held fixed",
+            "stages": stages, "roofline": roof, "launches_per_call": len(names) + (2 if cfg.has_proj else 1)}
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -279,8 +372,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--clocks-csv", default=None)
+    ap.add_argument("--no-backward", action="store_true", help="skip the sla_backward measurement")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads (H = H_kv; small profiler captures)")
     args = ap.parse_args()
     cfg = wl.preset(args.workload)
+    if args.heads > 0:
+        cfg = cfg.replace(name=f"{cfg.name}_h{args.heads}", H=args.heads, H_kv=args.heads)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -441,27 +539,20 @@ def main():
     (e2e_ms,) = max_over_ranks(dist, dev, e0.elapsed_time(e1) / args.e2e_steps)
     barrier()
 
+    peaks = load_peaks()
+    backward = None
+    if cfg.mode == wl.MODE_THREEWAY and not cfg.smooth_k and not args.no_backward:
+        backward = measure_backward(sla, torch, cfg, q, k, v, w_p, w_g, out, ws, args.steps, args.warmup,
+                                    dist, dev, stream, peaks)
+        barrier()
+
     flops = cfg.dense_flops()
     value = job_throughput(world, flops, ms_step)
     e2e_value = job_throughput(world, flops, e2e_ms)
 
-    peaks = load_peaks()
     if reorder is not None:
         reorder["frac"] = reorder["achieved"] / peaks["hbm"]
-    model = stage_model(cfg)
-    stages = {}
-    for n in names:
-        kind, work = model[n]
-        t = stage_ms[n] * 1e-3
-        if kind == "tensor":
-            ach = work / t / 1e12
-            stages[n] = {"ms": stage_ms[n], "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
-                         "frac": ach / peaks["bf16"], "frac_of_sustained": ach / peaks["bf16_sus"],
-                         "work": work}
-        else:
-            ach = work / t / 1e9
-            stages[n] = {"ms": stage_ms[n], "bound": "hbm", "achieved": ach, "unit": "GB/s",
-                         "frac": ach / peaks["hbm"], "work": work}
+    stages = stage_entries(names, stage_ms, stage_model(cfg), peaks)
     dom = max(names, key=lambda n: stage_ms[n])
     kernel_of = {"sparse_flash": "flash_tc_kernel"}
     dk = stages[dom]
@@ -505,6 +596,7 @@ def main():
         "roofline": roof,
         "token_reorder": reorder,
         "stages": stages,
+        "backward": backward,
         "gpu_launches": ns * args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

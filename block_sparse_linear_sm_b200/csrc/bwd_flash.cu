@@ -17,9 +17,12 @@
 //                      either key block as critical, streamed through a ring.
 // The query blocks of a key block come from a bitmap per (head, key block)
 // that cols_mark_kernel fills from the critical lists.
-// Warps 0-3: one TMEM lane quarter each, thread = row; warp 4: TMA loads and
-// tcgen05.mma issue (one elected lane). Score and dP tiles are double-buffered
-// in TMEM so the next tile's products run while the current one is processed.
+// Warps 0-3: one TMEM lane quarter each, thread = row; warp 4: tcgen05.mma
+// issue (one elected lane); warp 5: TMA loads into a four-slot ring, refilled
+// as soon as a slot frees. The score and dP tiles are double-buffered in TMEM
+// so the next tile's products run while the row warps process the current one;
+// the row warps write P and dS back into those TMEM columns as bf16 pairs and
+// the dQ / dV / dK products read them from there (A operand in TMEM).
 // Both kernels add the linear-branch part of the gradient (fp32 scratch) and
 // write the final bf16 rows.
 #include "common.cuh"
@@ -58,7 +61,36 @@ cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cuda
   return cudaGetLastError();
 }
 
-constexpr int kBwThreads = 160;  // warps 0-3 rows, warp 4 producer / MMA
+
+constexpr int kBwThreads = 192;  // warps 0-3 rows, warp 4 MMA, warp 5 TMA producer
+constexpr int kBwSlots = 4;      // ring slots
+
+// merged list of two bitmaps (warp 0, ascending): entry = index | a0 << 16 | a1 << 17 | tag << 18;
+// returns the count (in every lane)
+__device__ __forceinline__ int merge_bitmaps(const uint32_t* w0p, const uint32_t* w1p, int words, bool v0, bool v1,
+                                             uint32_t tag, uint32_t* out, int base, int lane) {
+  for (int w0 = 0; w0 < words; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t a0 = (w < words && v0) ? w0p[w] : 0u, a1 = (w < words && v1) ? w1p[w] : 0u;
+    uint32_t any = a0 | a1;
+    const int cnt = __popc(any);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = base + incl - cnt;
+    while (any) {
+      const int bit = __ffs(any) - 1;
+      any &= any - 1;
+      const uint32_t m = 1u << bit;
+      out[pos++] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u) | (tag << 18);
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return base;
+}
 
 // ---------------------------------------------------------------------------
 // dQ
@@ -69,9 +101,9 @@ struct DqLayout {
   static constexpr int kOffQ = 0;                         // Q: 128 rows, NP panels of 16 KB
   static constexpr int kOffO = kOffQ + NP * 16384;        // dO
   static constexpr int kTile = NP * 8192;                 // one 64-row K or V tile
-  static constexpr int kOffRing = kOffO + NP * 16384;     // 2 slots x (K, V)
-  static constexpr int kOffDS = kOffRing + 4 * kTile;     // dS: 2 buffers x 16 KB (128 rows x 64 keys)
-  static constexpr int kOffBar = kOffDS + 2 * 16384;      // 32 mbarriers
+  static constexpr int kSlot = 2 * kTile;                 // K_j, V_j
+  static constexpr int kOffRing = kOffO + NP * 16384;
+  static constexpr int kOffBar = kOffRing + kBwSlots * kSlot;  // 32 mbarriers
   static constexpr int kOffMisc = kOffBar + 32 * 8;
   static constexpr int kOffList = kOffMisc + 64;          // merged block list
   static constexpr int kTmemCols = 512;                   // dQ: D; S / dP: 2 x 128
@@ -93,7 +125,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     flash_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DqParams prm) {
   using L = DqLayout<D>;
-  constexpr int NP = L::NP;
+  constexpr int NP = L::NP, S = kBwSlots;
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -109,18 +141,20 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   uint32_t* mlist = reinterpret_cast<uint32_t*>(smem + L::kOffList);
   uint32_t* words = reinterpret_cast<uint32_t*>(smem + L::kOffRing);  // bitmaps live in the ring before its first load
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
-  constexpr int QO_FULL = 0, LOADED = 1, SLOT_FREE = 3, SP_FULL = 5, DS_FULL = 7, DS_FREE = 9, ACC_DONE = 11;
+  constexpr int QO_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, DS_FULL = SP_FULL + 2,
+                ACC_DONE = DS_FULL + 2;
 
   for (int w = tid; w < 2 * prm.words; w += kBwThreads) words[w] = 0u;
   if (tid == 0) {
     misc[2] = 0;
     tc::mbar_init(bar(QO_FULL), 1);
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(bar(LOADED + b), 1);
-      tc::mbar_init(bar(SLOT_FREE + b), 1);
-      tc::mbar_init(bar(SP_FULL + b), 1);
-      tc::mbar_init(bar(DS_FULL + b), 4);
-      tc::mbar_init(bar(DS_FREE + b), 1);
+    for (int x = 0; x < S; ++x) {
+      tc::mbar_init(bar(LOADED + x), 1);
+      tc::mbar_init(bar(SLOT_FREE + x), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(bar(SP_FULL + x), 1);
+      tc::mbar_init(bar(DS_FULL + x), 4);
     }
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::fence_mbar_init();
@@ -144,28 +178,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   }
   __syncthreads();
   if (warp == 0) {
-    int base = 0;
-    for (int w0 = 0; w0 < prm.words; w0 += 32) {
-      const int w = w0 + lane;
-      const uint32_t a0 = w < prm.words ? words[w] : 0u, a1 = w < prm.words ? words[prm.words + w] : 0u;
-      uint32_t any = a0 | a1;
-      const int cnt = __popc(any);
-      int incl = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int pos = base + incl - cnt;
-      while (any) {
-        const int bit = __ffs(any) - 1;
-        any &= any - 1;
-        const uint32_t m = 1u << bit;
-        mlist[pos++] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u);
-      }
-      base += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) misc[1] = base;
+    const int n = merge_bitmaps(words, words + prm.words, prm.words, true, true, 0u, mlist, 0, lane);
+    if (lane == 0) misc[1] = n;
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -173,90 +187,92 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   const int T = misc[1];
   const uint32_t tmem = (uint32_t)misc[0];
   volatile int* abort = misc + 2;
-  const uint32_t sQ = sbase + L::kOffQ, sO = sbase + L::kOffO, sR = sbase + L::kOffRing, sDS = sbase + L::kOffDS;
+  const uint32_t sQ = sbase + L::kOffQ, sO = sbase + L::kOffO, sR = sbase + L::kOffRing;
 
-  if (warp == 4) {
-    // ======================= producer and MMA issuer ==========================
+  if (warp == 5) {
+    // ======================= TMA producer =====================================
+    if (lane == 0 && T > 0) {
+      bool ok = true;
+      tc::mbar_expect_tx(bar(QO_FULL), 4 * NP * 8192);
+      for (int hf = 0; hf < 2; ++hf)
+        for (int p = 0; p < NP; ++p) {
+          tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmQ, bar(QO_FULL), 64 * p, i_h[hf] * kBlock, bh);
+          tc::tma_load_3d(sO + p * 16384 + hf * 8192, &tmO, bar(QO_FULL), 64 * p, i_h[hf] * kBlock, bh);
+        }
+      for (int m = 0; m < T && ok; ++m) {
+        const int slot = m % S;
+        if (m >= S && !(ok = tc::mbar_wait(bar(SLOT_FREE + slot), ((m / S) - 1) & 1, abort))) break;
+        const int jb = (int)(mlist[m] & 0xFFFFu);
+        const uint32_t dst = sR + slot * L::kSlot;
+        tc::mbar_expect_tx(bar(LOADED + slot), L::kSlot);
+        for (int p = 0; p < NP; ++p) {
+          tc::tma_load_3d(dst + p * 8192, &tmK, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
+          tc::tma_load_3d(dst + L::kTile + p * 8192, &tmV, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
+        }
+      }
+      // the last release of every slot: no product reads the ring and no commit is in flight at exit
+      for (int m = (T > S ? T - S : 0); m < T && ok; ++m)
+        ok = tc::mbar_wait(bar(SLOT_FREE + m % S), (m / S) & 1, abort);
+      if (!ok) {
+        *abort = 1;
+        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+      }
+    }
+  } else if (warp == 4) {
+    // ======================= MMA issuer =======================================
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t kIdQ = tc::idesc_bf16(128, D, false, true);
-    bool ok = true;
-    auto load = [&](int n) {
-      const int slot = n & 1, jb = (int)(mlist[n] & 0xFFFFu);
-      const uint32_t dst = sR + slot * 2 * L::kTile;
-      tc::mbar_expect_tx(bar(LOADED + slot), 2 * L::kTile);
-      for (int p = 0; p < NP; ++p) {
-        tc::tma_load_3d(dst + p * 8192, &tmK, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
-        tc::tma_load_3d(dst + L::kTile + p * 8192, &tmV, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
-      }
-    };
-    auto issue_sp = [&](int n) {
-      // S_n = Q K_n^T and dP_n = dO V_n^T into TMEM buffer n & 1
-      const int slot = n & 1;
-      const uint32_t kt = sR + slot * 2 * L::kTile, vt = kt + L::kTile;
-      const uint32_t tS = tmem + D + 128 * (n & 1);
+    // S_m = Q K_m^T and dP_m = dO V_m^T into TMEM buffer m & 1
+    auto issue_sp = [&](int m) {
+      const uint32_t kt = sR + (m % S) * L::kSlot, vt = kt + L::kTile;
+      const uint32_t tS = tmem + D + 128 * (m & 1);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t qo = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), ko = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
         tc::mma_bf16_ss(tS, tc::sw128_desc(sQ + qo, 16, 1024), tc::sw128_desc(kt + ko, 16, 1024), kIdS, k > 0);
         tc::mma_bf16_ss(tS + 64, tc::sw128_desc(sO + qo, 16, 1024), tc::sw128_desc(vt + ko, 16, 1024), kIdS, k > 0);
       }
-      tc::mma_commit(bar(SP_FULL + (n & 1)));
+      tc::mma_commit(bar(SP_FULL + (m & 1)));
     };
-    if (T > 0) {
-      if (lane == 0) {
-        tc::mbar_expect_tx(bar(QO_FULL), 4 * NP * 8192);
-        for (int hf = 0; hf < 2; ++hf)
-          for (int p = 0; p < NP; ++p) {
-            tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmQ, bar(QO_FULL), 64 * p, i_h[hf] * kBlock, bh);
-            tc::tma_load_3d(sO + p * 16384 + hf * 8192, &tmO, bar(QO_FULL), 64 * p, i_h[hf] * kBlock, bh);
-          }
-        for (int n = 0; n < 2 && n < T; ++n) load(n);
+    auto wait_loaded = [&](int m) -> bool {
+      return __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
+    };
+    bool ok = T == 0 || __all_sync(kAll, tc::mbar_wait(bar(QO_FULL), 0, abort));
+    for (int m = 0; m < 2 && m < T && ok; ++m) {
+      ok = wait_loaded(m);
+      tc::fence_after_sync();
+      if (ok && tc::elect_one()) issue_sp(m);
+      __syncwarp();
+    }
+    for (int m = 0; m < T && ok; ++m) {
+      const int b = m & 1;
+      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + b), (m >> 1) & 1, abort));
+      if (!ok) break;
+      tc::fence_after_sync();
+      if (tc::elect_one()) {
+        // dQ += dS_m K_m: A = dS_m from TMEM (bf16 pairs in the S columns), B = K_m N-major
+        const uint32_t kt = sR + (m % S) * L::kSlot;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16_ts(tmem, tmem + D + 128 * b + 8 * kk, tc::sw128_desc(kt + kk * 2048, 8192, 1024), kIdQ,
+                          (m > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(bar(SLOT_FREE + m % S));
+        if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
       }
       __syncwarp();
-      ok = __all_sync(kAll, tc::mbar_wait(bar(QO_FULL), 0, abort));
-      for (int n = 0; n < 2 && n < T && ok; ++n) {
-        ok = __all_sync(kAll, tc::mbar_wait(bar(LOADED + (n & 1)), 0, abort));
+      if (m + 2 < T) {
+        // buffer b is free once dQ_m has read dS_m: S_{m+2} goes in behind it
+        // (tcgen05 operations of one thread execute in issue order)
+        ok = wait_loaded(m + 2);
         tc::fence_after_sync();
-        if (ok && tc::elect_one()) issue_sp(n);
+        if (ok && tc::elect_one()) issue_sp(m + 2);
         __syncwarp();
       }
-      for (int n = 0; n < T && ok; ++n) {
-        const int b = n & 1;
-        ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + b), (n >> 1) & 1, abort));
-        if (!ok) break;
-        tc::fence_after_sync();
-        if (tc::elect_one()) {
-          // dQ += dS_n K_n: A = dS (K-major), B = K_n N-major
-          const uint32_t kt = sR + b * 2 * L::kTile;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16_ss(tmem, tc::sw128_desc(sDS + b * 16384 + kk * 32, 16, 1024),
-                            tc::sw128_desc(kt + kk * 2048, 8192, 1024), kIdQ, (n > 0 || kk > 0) ? 1u : 0u);
-          tc::mma_commit(bar(SLOT_FREE + b));
-          tc::mma_commit(bar(DS_FREE + b));
-          if (n == T - 1) tc::mma_commit(bar(ACC_DONE));
-        }
-        __syncwarp();
-        if (n + 2 < T) {
-          // the slot is free once dQ_n has read K_n: load tile n + 2 and issue its products
-          ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + b), (n >> 1) & 1, abort));
-          if (ok && lane == 0) load(n + 2);
-          __syncwarp();
-          ok = ok && __all_sync(kAll, tc::mbar_wait(bar(LOADED + b), ((n + 2) >> 1) & 1, abort));
-          tc::fence_after_sync();
-          if (ok && tc::elect_one()) issue_sp(n + 2);
-          __syncwarp();
-        }
-      }
-      // the last releases of both slots and dS buffers: no commit is in flight at exit
-      for (int n = (T > 2 ? T - 2 : 0); n < T && ok; ++n)
-        ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + (n & 1)), (n >> 1) & 1, abort)) &&
-             __all_sync(kAll, tc::mbar_wait(bar(DS_FREE + (n & 1)), (n >> 1) & 1, abort));
-      if (!ok && lane == 0) {
-        *abort = 1;
-        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
-      }
+    }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
     }
   } else {
     // ======================= rows: dS, then the dq epilogue ===================
@@ -268,21 +284,21 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const float dlt = vrow ? prm.delta[(size_t)bh * prm.N + t] : 0.f;
     const float sl2 = prm.scale_log2;
     bool ok = true;
-    for (int n = 0; n < T && ok; ++n) {
-      const int b = n & 1;
-      const uint32_t e = mlist[n];
-      const int jb = (int)(e & 0xFFFFu);
+    for (int m = 0; m < T && ok; ++m) {
+      const int b = m & 1;
+      const uint32_t e = mlist[m];
+      const int k0 = (int)(e & 0xFFFFu) * kBlock;
       const bool act = (e >> (16 + hf)) & 1u;
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + b), (n >> 1) & 1, abort));
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + b), (m >> 1) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
+      const uint32_t tS = tmem + lane_off + D + 128 * b;
       uint32_t sv[2][32], pv[2][32];
-      tc::tmem_ld32(tmem + lane_off + D + 128 * b, sv[0]);
-      tc::tmem_ld32(tmem + lane_off + D + 128 * b + 32, sv[1]);
-      tc::tmem_ld32(tmem + lane_off + D + 128 * b + 64, pv[0]);
-      tc::tmem_ld32(tmem + lane_off + D + 128 * b + 96, pv[1]);
+      tc::tmem_ld32(tS, sv[0]);
+      tc::tmem_ld32(tS + 32, sv[1]);
+      tc::tmem_ld32(tS + 64, pv[0]);
+      tc::tmem_ld32(tS + 96, pv[1]);
       tc::tmem_ld_wait();
-      const int k0 = jb * kBlock;
       uint32_t ds[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -296,16 +312,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
         ds[j] = pack_bf16(g2[0], g2[1]);
       }
-      // dS buffer b was last read by dQ_{n-2}
-      if (n >= 2) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(DS_FREE + b), ((n - 2) >> 1) & 1, abort));
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(smem + L::kOffDS + b * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(ds[4 * c], ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
-      tc::fence_async_smem();
+      tc::tmem_st32(tS, ds);
+      tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(DS_FULL + b));
@@ -368,15 +376,15 @@ struct DkvLayout {
   static constexpr int kTile = NP * 8192;                      // one 64-row Q or dO tile
   static constexpr int kSlot = (2 * kTile + 512 + 1023) / 1024 * 1024;  // Q_i, dO_i, lse_i, delta_i
   static constexpr int kOffRing = kOffV + NP * 16384;
-  static constexpr int kOffPS = kOffRing + 2 * kSlot;          // 2 buffers x (P^T, dS^T), 16 KB each
-  static constexpr int kOffBar = kOffPS + 4 * 16384;
+  static constexpr int kOffBar = kOffRing + kBwSlots * kSlot;
   static constexpr int kOffMisc = kOffBar + 32 * 8;
-  static constexpr int kOffList = kOffMisc + 64;               // query blocks of one head
+  static constexpr int kSmem = kOffMisc + 64;
   static constexpr int kTmemCols = 512;                        // dV, dK: 2 D; S^T / dP^T: 2 x 128
 };
 
 struct DkvParams {
   const uint32_t* bits;   // [B*H][nkb][words]
+  uint32_t* dlist;        // [B*H_kv*npairs][group*nqb]: merged (head, query block) list of each unit
   const float* lse;       // [B*H][N] (log2 domain)
   const float* delta;     // [B*H][N]
   const float* dk_acc;    // [B*H_kv][N][D] or null
@@ -394,7 +402,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       DkvParams prm) {
   using L = DkvLayout<D>;
-  constexpr int NP = L::NP;
+  constexpr int NP = L::NP, S = kBwSlots;
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -408,20 +416,23 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   const int j_h[2] = {2 * pr, 2 * pr + 1};
   const bool valid_j[2] = {j_h[0] < prm.nb, j_h[1] < prm.nb};
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);  // tmem, count, abort
-  uint32_t* mlist = reinterpret_cast<uint32_t*>(smem + L::kOffList);
+  uint32_t* dlist = prm.dlist + (size_t)blockIdx.x * prm.group * prm.nb;
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
-  constexpr int KV_FULL = 0, LOADED = 1, SLOT_FREE = 3, SP_FULL = 5, DS_FULL = 7, PS_FREE = 9, ACC_DONE = 11;
-  const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sR = sbase + L::kOffRing, sPS = sbase + L::kOffPS;
+  constexpr int KV_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, DS_FULL = SP_FULL + 2,
+                ACC_DONE = DS_FULL + 2;
+  const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sR = sbase + L::kOffRing;
+  auto head_of = [&](int g) { return b * prm.H + hk * prm.group + g; };
 
   if (tid == 0) {
     misc[2] = 0;
     tc::mbar_init(bar(KV_FULL), 1);
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < S; ++x) {
       tc::mbar_init(bar(LOADED + x), 1);
       tc::mbar_init(bar(SLOT_FREE + x), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
       tc::mbar_init(bar(SP_FULL + x), 1);
       tc::mbar_init(bar(DS_FULL + x), 4);
-      tc::mbar_init(bar(PS_FREE + x), 1);
     }
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::fence_mbar_init();
@@ -436,62 +447,32 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     tc::tmem_alloc(sbase + L::kOffMisc, L::kTmemCols);
     tc::tmem_relinquish();
   }
+  if (warp == 0) {
+    // every query head of the group: the query blocks that hold j0 or j1 as critical
+    int n = 0;
+    for (int g = 0; g < prm.group; ++g) {
+      const size_t row = (size_t)head_of(g) * prm.nb;
+      n = merge_bitmaps(prm.bits + (row + j_h[0]) * prm.words, prm.bits + (row + (valid_j[1] ? j_h[1] : 0)) * prm.words,
+                        prm.words, valid_j[0], valid_j[1], (uint32_t)g, dlist, n, lane);
+    }
+    if (lane == 0) misc[1] = n;
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  const int T = misc[1];
   const uint32_t tmem = (uint32_t)misc[0];
   volatile int* abort = misc + 2;
-  bool ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(KV_FULL), 0, abort));
 
-  const int r = tid, hf = r >> 6;
-  const int key = j_h[hf] * kBlock + (r & 63);
-  const bool vkey = valid_j[hf] && key < prm.n_valid;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const float sl2 = prm.scale_log2;
-  int m0 = 0;  // tiles of the previous heads (ring slots and TMEM buffers alternate over all tiles)
-  for (int g = 0; g < prm.group; ++g) {
-    const int bh = b * prm.H + hk * prm.group + g;
-    // merged list of the query blocks that hold j0 or j1 as critical
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-      const uint32_t* r0 = prm.bits + ((size_t)bh * prm.nb + j_h[0]) * prm.words;
-      const uint32_t* r1 = prm.bits + ((size_t)bh * prm.nb + j_h[1]) * prm.words;
-      int base = 0;
-      for (int w0 = 0; w0 < prm.words; w0 += 32) {
-        const int w = w0 + lane;
-        const uint32_t a0 = (w < prm.words && valid_j[0]) ? r0[w] : 0u;
-        const uint32_t a1 = (w < prm.words && valid_j[1]) ? r1[w] : 0u;
-        uint32_t any = a0 | a1;
-        const int cnt = __popc(any);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        int pos = base + incl - cnt;
-        while (any) {
-          const int bit = __ffs(any) - 1;
-          any &= any - 1;
-          const uint32_t m = 1u << bit;
-          mlist[pos++] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u);
-        }
-        base += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      if (lane == 0) misc[1] = base;
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const int T = misc[1];
-    if (warp == 4) {
-      // ===================== producer and MMA issuer ==========================
-      constexpr uint32_t kAll = 0xffffffffu;
-      constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
-      constexpr uint32_t kIdA = tc::idesc_bf16(128, D, false, true);
-      auto load = [&](int n, int m) {
-        const int slot = m & 1, i = (int)(mlist[n] & 0xFFFFu);
+  if (warp == 5) {
+    // ======================= TMA producer =====================================
+    if (lane == 0) {
+      bool ok = true;
+      for (int m = 0; m < T && ok; ++m) {
+        const int slot = m % S;
+        if (m >= S && !(ok = tc::mbar_wait(bar(SLOT_FREE + slot), ((m / S) - 1) & 1, abort))) break;
+        const uint32_t e = dlist[m];
+        const int i = (int)(e & 0xFFFFu), bh = head_of((int)(e >> 18));
         const uint32_t dst = sR + slot * L::kSlot;
         tc::mbar_expect_tx(bar(LOADED + slot), 2 * L::kTile + 512);
         for (int p = 0; p < NP; ++p) {
@@ -501,132 +482,124 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         tc::bulk_load(dst + 2 * L::kTile, prm.lse + (size_t)bh * prm.N + i * kBlock, 256, bar(LOADED + slot));
         tc::bulk_load(dst + 2 * L::kTile + 256, prm.delta + (size_t)bh * prm.N + i * kBlock, 256,
                       bar(LOADED + slot));
-      };
-      auto issue_sp = [&](int m) {
-        // S^T = K Q_i^T, dP^T = V dO_i^T (M = 128 keys, N = 64 queries)
-        const uint32_t qt = sR + (m & 1) * L::kSlot, ot = qt + L::kTile;
-        const uint32_t tS = tmem + 2 * D + 128 * (m & 1);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t ko = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), qo = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
-          tc::mma_bf16_ss(tS, tc::sw128_desc(sK + ko, 16, 1024), tc::sw128_desc(qt + qo, 16, 1024), kIdS, k > 0);
-          tc::mma_bf16_ss(tS + 64, tc::sw128_desc(sV + ko, 16, 1024), tc::sw128_desc(ot + qo, 16, 1024), kIdS, k > 0);
-        }
-        tc::mma_commit(bar(SP_FULL + (m & 1)));
-      };
-      if (ok && T > 0) {
-        if (lane == 0)
-          for (int n = 0; n < 2 && n < T; ++n) load(n, m0 + n);
-        __syncwarp();
-        for (int n = 0; n < 2 && n < T && ok; ++n) {
-          const int m = m0 + n;
-          ok = __all_sync(kAll, tc::mbar_wait(bar(LOADED + (m & 1)), (m >> 1) & 1, abort));
-          tc::fence_after_sync();
-          if (ok && tc::elect_one()) issue_sp(m);
-          __syncwarp();
-        }
-        for (int n = 0; n < T && ok; ++n) {
-          const int m = m0 + n, x = m & 1;
-          ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
-          if (!ok) break;
-          tc::fence_after_sync();
-          if (tc::elect_one()) {
-            // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T (K-major), B = dO_i / Q_i N-major
-            const uint32_t qt = sR + x * L::kSlot, ot = qt + L::kTile;
-            const uint32_t pt = sPS + x * 32768, dt = pt + 16384;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
-              tc::mma_bf16_ss(tmem, tc::sw128_desc(pt + kk * 32, 16, 1024), tc::sw128_desc(ot + kk * 2048, 8192, 1024),
-                              kIdA, acc);
-              tc::mma_bf16_ss(tmem + D, tc::sw128_desc(dt + kk * 32, 16, 1024),
-                              tc::sw128_desc(qt + kk * 2048, 8192, 1024), kIdA, acc);
-            }
-            tc::mma_commit(bar(SLOT_FREE + x));
-            tc::mma_commit(bar(PS_FREE + x));
-          }
-          __syncwarp();
-          if (n + 2 < T) {
-            ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + x), (m >> 1) & 1, abort));
-            if (ok && lane == 0) load(n + 2, m + 2);
-            __syncwarp();
-            ok = ok && __all_sync(kAll, tc::mbar_wait(bar(LOADED + x), ((m + 2) >> 1) & 1, abort));
-            tc::fence_after_sync();
-            if (ok && tc::elect_one()) issue_sp(m + 2);
-            __syncwarp();
-          }
-        }
-        // this head's last tiles have released their slot and P / dS buffer
-        for (int n = (T > 2 ? T - 2 : 0); n < T && ok; ++n) {
-          const int m = m0 + n;
-          ok = __all_sync(kAll, tc::mbar_wait(bar(SLOT_FREE + (m & 1)), (m >> 1) & 1, abort)) &&
-               __all_sync(kAll, tc::mbar_wait(bar(PS_FREE + (m & 1)), (m >> 1) & 1, abort));
-        }
       }
-    } else if (ok) {
-      // ===================== rows: P^T and dS^T =============================
-      for (int n = 0; n < T && ok; ++n) {
-        const int m = m0 + n, x = m & 1;
-        const bool act = (mlist[n] >> (16 + hf)) & 1u;
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + x), (m >> 1) & 1, abort)) &&
-             __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED + x), (m >> 1) & 1, abort));
-        if (!ok) break;
-        tc::fence_after_sync();
-        uint32_t sv[2][32], pv[2][32];
-        const uint32_t tS = tmem + lane_off + 2 * D + 128 * x;
-        tc::tmem_ld32(tS, sv[0]);
-        tc::tmem_ld32(tS + 32, sv[1]);
-        tc::tmem_ld32(tS + 64, pv[0]);
-        tc::tmem_ld32(tS + 96, pv[1]);
-        tc::tmem_ld_wait();
-        const float* lse = reinterpret_cast<const float*>(smem + L::kOffRing + x * L::kSlot + 2 * L::kTile);
-        const float* dl = lse + 64;
-        uint32_t pw[32], dw[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float pp[2], dd[2];
-#pragma unroll
-          for (int y = 0; y < 2; ++y) {
-            const int c = 2 * j + y;
-            const float s = __uint_as_float(sv[c >> 5][c & 31]);
-            const float p = (act && vkey) ? tc::ex2_approx(s * sl2 - lse[c]) : 0.f;
-            pp[y] = p;
-            dd[y] = p * (__uint_as_float(pv[c >> 5][c & 31]) - dl[c]);
-          }
-          pw[j] = pack_bf16(pp[0], pp[1]);
-          dw[j] = pack_bf16(dd[0], dd[1]);
-        }
-        if (m >= 2) {
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(PS_FREE + x), ((m - 2) >> 1) & 1, abort));
-          if (!ok) break;
-        }
-        unsigned char* pt = smem + L::kOffPS + x * 32768;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t off = (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
-          *reinterpret_cast<uint4*>(pt + off) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-          *reinterpret_cast<uint4*>(pt + 16384 + off) = make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]);
-        }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(bar(DS_FULL + x));
+      // the last release of every slot: no product reads the ring and no commit is in flight at exit
+      for (int m = (T > S ? T - S : 0); m < T && ok; ++m)
+        ok = tc::mbar_wait(bar(SLOT_FREE + m % S), (m / S) & 1, abort);
+      if (!ok) {
+        *abort = 1;
+        report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
       }
     }
-    m0 += T;
-  }
-  // every warp agrees on the outcome before the epilogue
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  if (*abort) ok = false;
-  if (warp == 4) {
-    if (ok && m0 > 0 && tc::elect_one()) tc::mma_commit(bar(ACC_DONE));
-    __syncwarp();
+  } else if (warp == 4) {
+    // ======================= MMA issuer =======================================
+    constexpr uint32_t kAll = 0xffffffffu;
+    constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
+    constexpr uint32_t kIdA = tc::idesc_bf16(128, D, false, true);
+    // S^T = K Q_i^T, dP^T = V dO_i^T (M = 128 keys, N = 64 queries) into TMEM buffer m & 1
+    auto issue_sp = [&](int m) {
+      const uint32_t qt = sR + (m % S) * L::kSlot, ot = qt + L::kTile;
+      const uint32_t tS = tmem + 2 * D + 128 * (m & 1);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t ko = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), qo = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
+        tc::mma_bf16_ss(tS, tc::sw128_desc(sK + ko, 16, 1024), tc::sw128_desc(qt + qo, 16, 1024), kIdS, k > 0);
+        tc::mma_bf16_ss(tS + 64, tc::sw128_desc(sV + ko, 16, 1024), tc::sw128_desc(ot + qo, 16, 1024), kIdS, k > 0);
+      }
+      tc::mma_commit(bar(SP_FULL + (m & 1)));
+    };
+    auto wait_loaded = [&](int m) -> bool {
+      return __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
+    };
+    bool ok = T == 0 || __all_sync(kAll, tc::mbar_wait(bar(KV_FULL), 0, abort));
+    for (int m = 0; m < 2 && m < T && ok; ++m) {
+      ok = wait_loaded(m);
+      tc::fence_after_sync();
+      if (ok && tc::elect_one()) issue_sp(m);
+      __syncwarp();
+    }
+    for (int m = 0; m < T && ok; ++m) {
+      const int x = m & 1;
+      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
+      if (!ok) break;
+      tc::fence_after_sync();
+      if (tc::elect_one()) {
+        // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T from TMEM, B = dO_i / Q_i N-major
+        const uint32_t qt = sR + (m % S) * L::kSlot, ot = qt + L::kTile;
+        const uint32_t tP = tmem + 2 * D + 128 * x;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
+          tc::mma_bf16_ts(tmem, tP + 8 * kk, tc::sw128_desc(ot + kk * 2048, 8192, 1024), kIdA, acc);
+          tc::mma_bf16_ts(tmem + D, tP + 64 + 8 * kk, tc::sw128_desc(qt + kk * 2048, 8192, 1024), kIdA, acc);
+        }
+        tc::mma_commit(bar(SLOT_FREE + m % S));
+        if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
+      }
+      __syncwarp();
+      if (m + 2 < T) {
+        ok = wait_loaded(m + 2);
+        tc::fence_after_sync();
+        if (ok && tc::elect_one()) issue_sp(m + 2);
+        __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
   } else {
-    if (ok && m0 > 0) {
+    // ======================= rows (keys): P^T and dS^T, then the epilogue =====
+    const int r = tid, hf = r >> 6;
+    const int key = j_h[hf] * kBlock + (r & 63);
+    const bool vkey = valid_j[hf] && key < prm.n_valid;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float sl2 = prm.scale_log2;
+    bool ok = true;
+    for (int m = 0; m < T && ok; ++m) {
+      const int x = m & 1, slot = m % S;
+      const bool act = vkey && ((dlist[m] >> (16 + hf)) & 1u);
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + x), (m >> 1) & 1, abort)) &&
+           __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED + slot), (m / S) & 1, abort));
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t tS = tmem + lane_off + 2 * D + 128 * x;
+      uint32_t sv[2][32], pv[2][32];
+      tc::tmem_ld32(tS, sv[0]);
+      tc::tmem_ld32(tS + 32, sv[1]);
+      tc::tmem_ld32(tS + 64, pv[0]);
+      tc::tmem_ld32(tS + 96, pv[1]);
+      tc::tmem_ld_wait();
+      const float* lse = reinterpret_cast<const float*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile);
+      const float* dl = lse + 64;
+      uint32_t pw[32], dw[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float pp[2], dd[2];
+#pragma unroll
+        for (int y = 0; y < 2; ++y) {
+          const int c = 2 * j + y;
+          const float p = act ? tc::ex2_approx(__uint_as_float(sv[c >> 5][c & 31]) * sl2 - lse[c]) : 0.f;
+          pp[y] = p;
+          dd[y] = p * (__uint_as_float(pv[c >> 5][c & 31]) - dl[c]);
+        }
+        pw[j] = pack_bf16(pp[0], pp[1]);
+        dw[j] = pack_bf16(dd[0], dd[1]);
+      }
+      tc::tmem_st32(tS, pw);
+      tc::tmem_st32(tS + 64, dw);
+      tc::tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(DS_FULL + x));
+    }
+    if (ok && T > 0) {
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(ACC_DONE), 0, abort));
       tc::fence_after_sync();
+    }
+    if (!ok) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
     }
     if (valid_j[hf]) {
       // dk = scale dK + linear part, dv = dV + linear part (padding keys 0)
@@ -639,7 +612,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t v[32];
-          if (ok && m0 > 0) {
+          if (ok && T > 0) {
             tc::tmem_ld32(tmem + lane_off + which * D + 32 * ch, v);
             tc::tmem_ld_wait();
           } else {
@@ -664,10 +637,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
     }
   }
-  if (!ok && lane == 0) {
-    *abort = 1;
-    report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
-  }
+  // without tiles nobody waited for K and V: the loads land before the CTA exits
+  if (T == 0 && tid == 0 && !tc::mbar_wait(bar(KV_FULL), 0, abort)) report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 4) {
@@ -711,9 +682,8 @@ static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& 
   prm.scale_log2 = p.scale * 1.4426950408889634f;
   const int cap = 2 * c.k_h < p.nkb ? 2 * c.k_h : p.nkb;
   int smem = L::kOffList + (cap > 0 ? cap : 1) * 4;
-  if (2 * prm.words * 4 > 4 * L::kTile) return cudaErrorInvalidValue;  // bitmaps in the ring
-  // one CTA per SM: each holds all 512 TMEM columns
-  if (smem < 120 * 1024) smem = 120 * 1024;
+  if (2 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
+  if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: it holds all 512 TMEM columns
   cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   flash_dq_kernel<D><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
@@ -734,6 +704,7 @@ static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs
     return cudaErrorInvalidValue;
   DkvParams prm;
   prm.bits = reinterpret_cast<const uint32_t*>(a.bws + bp.off_bits);
+  prm.dlist = reinterpret_cast<uint32_t*>(a.bws + bp.off_dlist);
   prm.lse = reinterpret_cast<const float*>(a.ws + p.off_lse);
   prm.delta = reinterpret_cast<const float*>(a.bws + bp.off_delta);
   prm.dk_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dkacc) : nullptr;
@@ -750,7 +721,7 @@ static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs
   prm.words = bp.words;
   prm.scale = p.scale;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
-  int smem = L::kOffList + p.nqb * 4;
+  int smem = L::kSmem;
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (512 TMEM columns)
   cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -484,7 +484,7 @@ struct StBwdParams {
   const float* dz;         // [B*H_kv][nkb][D]
   float* dk_acc;           // [B*H_kv][N][D]
   float* dv_acc;
-  float* dw_p;             // [wp_heads][D][D] or null
+  float* dwp_part;         // [B*H_kv*npairs][D][D]: this CTA's dW_p partial, or null
   int* status;
   int N, n_valid, nkb, npairs, has_proj, wp_heads;
 };
@@ -725,16 +725,21 @@ __global__ void __launch_bounds__(128, 1)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    if (ok && r < D) {
-      // dW_p row c (this CTA's 128 tokens) added into the fp32 gradient
-      float* wrow = prm.dw_p + ((size_t)(bkv % prm.wp_heads) * D + r) * D;
+    if (r < D) {
+      // dW_p row c of this CTA's 128 tokens, as a partial (reduced by dwp_reduce_kernel)
+      float4* wrow = reinterpret_cast<float4*>(prm.dwp_part + ((size_t)blockIdx.x * D + r) * D);
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t v[32];
-        tc::tmem_ld32(tmem + lane_off + D + 32 * ch, v);
-        tc::tmem_ld_wait();
+        if (ok) {
+          tc::tmem_ld32(tmem + lane_off + D + 32 * ch, v);
+          tc::tmem_ld_wait();
+        }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) atomicAdd(wrow + 32 * ch + j, __uint_as_float(v[j]));
+        for (int j = 0; j < 8; ++j)
+          wrow[8 * ch + j] = ok ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                              __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
   }
@@ -748,6 +753,31 @@ __global__ void __launch_bounds__(128, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, L::kTmemCols);
   }
+}
+
+// dW_p[w] = sum of the partials of the units whose KV head uses W_p[w] (w = bkv % wp_heads).
+// grid (D*D/4 / 128, segments, wp_heads): each thread sums one float4 column over a
+// segment of the units and adds it to the gradient.
+__global__ void dwp_reduce_kernel(const float4* __restrict__ part, float* __restrict__ dw_p, int units,
+                                  int npairs, int wp_heads, int dsq4) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x, w = blockIdx.z;
+  if (e >= dsq4) return;
+  const int seg = gridDim.y, per = (units + seg - 1) / seg;
+  const int u0 = blockIdx.y * per, u1 = min(units, u0 + per);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int u = u0; u < u1; ++u) {
+    if ((u / npairs) % wp_heads != w) continue;
+    const float4 x = part[(size_t)u * dsq4 + e];
+    acc.x += x.x;
+    acc.y += x.y;
+    acc.z += x.z;
+    acc.w += x.w;
+  }
+  float* dst = dw_p + ((size_t)w * dsq4 + e) * 4;
+  atomicAdd(dst, acc.x);
+  atomicAdd(dst + 1, acc.y);
+  atomicAdd(dst + 2, acc.z);
+  atomicAdd(dst + 3, acc.w);
 }
 
 template <int D>
@@ -769,7 +799,7 @@ static cudaError_t launch_state_bwd_t(const Plan& p, const BwdPlan& bp, const Bw
   prm.dz = reinterpret_cast<const float*>(a.bws + bp.off_dz);
   prm.dk_acc = reinterpret_cast<float*>(a.bws + bp.off_dkacc);
   prm.dv_acc = reinterpret_cast<float*>(a.bws + bp.off_dvacc);
-  prm.dw_p = proj ? a.dw_p : nullptr;
+  prm.dwp_part = proj ? reinterpret_cast<float*>(a.bws + bp.off_dwp) : nullptr;
   prm.status = a.status;
   prm.N = c.N;
   prm.n_valid = c.N_valid;
@@ -779,7 +809,12 @@ static cudaError_t launch_state_bwd_t(const Plan& p, const BwdPlan& bp, const Bw
   prm.wp_heads = wp_heads;
   cudaError_t e = cudaFuncSetAttribute(state_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
-  state_bwd_kernel<D><<<(unsigned)(bkv * prm.npairs), 128, L::kSmem, s>>>(mk, mv, mw, mh, prm);
+  const int units = (int)bkv * prm.npairs;
+  state_bwd_kernel<D><<<units, 128, L::kSmem, s>>>(mk, mv, mw, mh, prm);
+  if ((e = cudaGetLastError()) != cudaSuccess || !proj) return e;
+  dim3 grid((D * D / 4 + 127) / 128, 64, wp_heads);
+  dwp_reduce_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(prm.dwp_part), a.dw_p, units,
+                                         prm.npairs, wp_heads, D * D / 4);
   return cudaGetLastError();
 }
 

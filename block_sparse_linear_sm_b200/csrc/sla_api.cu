@@ -205,6 +205,8 @@ bool make_bwd_plan(const Plan& p, BwdPlan* b) {
   b->off_status = take(256);
   b->off_delta = take(B * H * N * 4);                       // D_t = dO_t . O_s,t
   b->off_bits = take(B * H * p.nkb * (size_t)b->words * 4);  // query blocks of each key block
+  // merged (query head, query block) list of each pair of key blocks
+  b->off_dlist = take(B * Hkv * (size_t)((p.nkb + 1) / 2) * p.group * p.nqb * 4);
   if (b->lin) {
     b->off_dqacc = take(B * H * N * d * 4);    // linear-branch and gate part of dq (fp32)
     b->off_dkacc = take(B * Hkv * N * d * 4);  // linear-branch part of dk, dv (fp32)
@@ -213,6 +215,8 @@ bool make_bwd_plan(const Plan& p, BwdPlan* b) {
     b->off_maskt = take(B * Hkv * (size_t)p.nkb_pad * b->rows_t * 2);   // transposed aggregation mask
     b->off_dh = take(B * Hkv * (size_t)p.nkb * d * d * 2);              // dh'_j (bf16)
     b->off_dz = take(B * Hkv * (size_t)p.nkb * d * 4);                  // dz_j (fp32)
+    if (c.has_proj)  // dW_p partial of each pair of key blocks (fp32)
+      b->off_dwp = take(B * Hkv * (size_t)((p.nkb + 1) / 2) * d * d * 4);
   }
   b->total = off;
   return true;
