@@ -17,8 +17,9 @@
 //                      either key block as critical, streamed through a ring.
 // The query blocks of a key block come from a bitmap per (head, key block)
 // that cols_mark_kernel fills from the critical lists.
-// Warps 0-3: one TMEM lane quarter each, thread = row; warp 4: tcgen05.mma
-// issue (one elected lane); warp 5: TMA loads into a four-slot ring, refilled
+// Warps 0-7: two warpgroups, one TMEM lane quarter per warp (thread = row),
+// the warpgroups taking the two 32-column halves of every tile; warp 8:
+// tcgen05.mma issue (one elected lane); warp 9: TMA loads into a four-slot ring, refilled
 // as soon as a slot frees. The score and dP tiles are double-buffered in TMEM
 // so the next tile's products run while the row warps process the current one;
 // the row warps write P and dS back into those TMEM columns as bf16 pairs and
@@ -62,7 +63,8 @@ cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cuda
 }
 
 
-constexpr int kBwThreads = 192;  // warps 0-3 rows, warp 4 MMA, warp 5 TMA producer
+constexpr int kBwThreads = 320;  // warps 0-7 rows (two column halves), warp 8 MMA, warp 9 TMA producer
+constexpr int kMmaWarp = 8, kProdWarp = 9, kRowWarps = 8;
 constexpr int kBwSlots = 4;      // ring slots
 
 // merged list of two bitmaps (warp 0, ascending): entry = index | a0 << 16 | a1 << 17 | tag << 18;
@@ -154,12 +156,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(bar(SP_FULL + x), 1);
-      tc::mbar_init(bar(DS_FULL + x), 4);
+      tc::mbar_init(bar(DS_FULL + x), kRowWarps);
     }
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(sbase + L::kOffMisc, L::kTmemCols);
     tc::tmem_relinquish();
   }
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   volatile int* abort = misc + 2;
   const uint32_t sQ = sbase + L::kOffQ, sO = sbase + L::kOffO, sR = sbase + L::kOffRing;
 
-  if (warp == 5) {
+  if (warp == kProdWarp) {
     // ======================= TMA producer =====================================
     if (lane == 0 && T > 0) {
       bool ok = true;
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kMmaWarp) {
     // ======================= MMA issuer =======================================
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
@@ -251,12 +253,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (!ok) break;
       tc::fence_after_sync();
       if (tc::elect_one()) {
-        // dQ += dS_m K_m: A = dS_m from TMEM (bf16 pairs in the S columns), B = K_m N-major
+        // dQ += dS_m K_m: A = dS_m from TMEM (bf16 pairs: keys 0-31 in columns 0-15 of the S
+        // buffer, keys 32-63 in columns 32-47), B = K_m N-major
         const uint32_t kt = sR + (m % S) * L::kSlot;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16_ts(tmem, tmem + D + 128 * b + 8 * kk, tc::sw128_desc(kt + kk * 2048, 8192, 1024), kIdQ,
-                          (m > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(tmem, tmem + D + 128 * b + 8 * kk + (kk >= 2 ? 16 : 0),
+                          tc::sw128_desc(kt + kk * 2048, 8192, 1024), kIdQ, (m > 0 || kk > 0) ? 1u : 0u);
         tc::mma_commit(bar(SLOT_FREE + m % S));
         if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
       }
@@ -276,10 +279,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
   } else {
     // ======================= rows: dS, then the dq epilogue ===================
-    const int r = tid, hf = r >> 6;
+    // warp = quarter (TMEM lanes) + 4 * hw (key columns 32 hw .. 32 hw + 31 of each tile)
+    const int quarter = warp & 3, hw = warp >> 2;
+    const int r = quarter * 32 + lane, hf = r >> 6;
     const int t = i_h[hf] * kBlock + (r & 63);
     const bool vrow = valid_h[hf] && t < prm.n_valid;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float lse2 = vrow ? prm.lse[(size_t)bh * prm.N + t] : INFINITY;
     const float dlt = vrow ? prm.delta[(size_t)bh * prm.N + t] : 0.f;
     const float sl2 = prm.scale_log2;
@@ -293,26 +298,25 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (!ok) break;
       tc::fence_after_sync();
       const uint32_t tS = tmem + lane_off + D + 128 * b;
-      uint32_t sv[2][32], pv[2][32];
-      tc::tmem_ld32(tS, sv[0]);
-      tc::tmem_ld32(tS + 32, sv[1]);
-      tc::tmem_ld32(tS + 64, pv[0]);
-      tc::tmem_ld32(tS + 96, pv[1]);
+      uint32_t sv[32], pv[32];
+      tc::tmem_ld32(tS + 32 * hw, sv);
+      tc::tmem_ld32(tS + 64 + 32 * hw, pv);
       tc::tmem_ld_wait();
-      uint32_t ds[32];
+      const int kc = k0 + 32 * hw;  // first key of this half
+      uint32_t ds[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < 16; ++j) {
         float g2[2];
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           const int c = 2 * j + x;
-          const float s = __uint_as_float(sv[c >> 5][c & 31]);
-          const float p = (act && k0 + c < prm.n_valid) ? tc::ex2_approx(s * sl2 - lse2) : 0.f;
-          g2[x] = p * (__uint_as_float(pv[c >> 5][c & 31]) - dlt);
+          const float p = (act && kc + c < prm.n_valid) ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse2) : 0.f;
+          g2[x] = p * (__uint_as_float(pv[c]) - dlt);
         }
         ds[j] = pack_bf16(g2[0], g2[1]);
       }
-      tc::tmem_st32(tS, ds);
+      // packed into the first 16 columns of this half (never over the other half's scores)
+      tc::tmem_st16(tS + 32 * hw, ds);
       tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       __nv_bfloat16* dst = prm.dq + ((size_t)bh * prm.N + t) * D;
       const float* acc = prm.dq_acc ? prm.dq_acc + ((size_t)bh * prm.N + t) * D : nullptr;
 #pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = hw * (D / 64); ch < (hw + 1) * (D / 64); ++ch) {  // this warpgroup's half of the columns
         uint32_t v[32];
         if (ok && T > 0) {
           tc::tmem_ld32(tmem + lane_off + 32 * ch, v);
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, L::kTmemCols);
   }
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(bar(SP_FULL + x), 1);
-      tc::mbar_init(bar(DS_FULL + x), 4);
+      tc::mbar_init(bar(DS_FULL + x), kRowWarps);
     }
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::fence_mbar_init();
@@ -443,7 +447,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         tc::tma_load_3d(sV + p * 16384 + hf * 8192, &tmV, bar(KV_FULL), 64 * p, j_h[hf] * kBlock, bkv);
       }
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(sbase + L::kOffMisc, L::kTmemCols);
     tc::tmem_relinquish();
   }
@@ -464,7 +468,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   const uint32_t tmem = (uint32_t)misc[0];
   volatile int* abort = misc + 2;
 
-  if (warp == 5) {
+  if (warp == kProdWarp) {
     // ======================= TMA producer =====================================
     if (lane == 0) {
       bool ok = true;
@@ -491,7 +495,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kMmaWarp) {
     // ======================= MMA issuer =======================================
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
@@ -524,14 +528,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (!ok) break;
       tc::fence_after_sync();
       if (tc::elect_one()) {
-        // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T from TMEM, B = dO_i / Q_i N-major
+        // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T from TMEM (bf16 pairs: queries 0-31 in
+        // columns 0-15 of the buffer half, queries 32-63 in columns 32-47), B = dO_i / Q_i N-major
         const uint32_t qt = sR + (m % S) * L::kSlot, ot = qt + L::kTile;
         const uint32_t tP = tmem + 2 * D + 128 * x;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
-          tc::mma_bf16_ts(tmem, tP + 8 * kk, tc::sw128_desc(ot + kk * 2048, 8192, 1024), kIdA, acc);
-          tc::mma_bf16_ts(tmem + D, tP + 64 + 8 * kk, tc::sw128_desc(qt + kk * 2048, 8192, 1024), kIdA, acc);
+          const uint32_t ka = 8 * kk + (kk >= 2 ? 16 : 0);
+          tc::mma_bf16_ts(tmem, tP + ka, tc::sw128_desc(ot + kk * 2048, 8192, 1024), kIdA, acc);
+          tc::mma_bf16_ts(tmem + D, tP + 64 + ka, tc::sw128_desc(qt + kk * 2048, 8192, 1024), kIdA, acc);
         }
         tc::mma_commit(bar(SLOT_FREE + m % S));
         if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
@@ -550,44 +556,48 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
   } else {
     // ======================= rows (keys): P^T and dS^T, then the epilogue =====
-    const int r = tid, hf = r >> 6;
+    // warp = quarter (TMEM lanes) + 4 * hw (query columns 32 hw .. 32 hw + 31 of each tile)
+    const int quarter = warp & 3, hw = warp >> 2;
+    const int r = quarter * 32 + lane, hf = r >> 6;
     const int key = j_h[hf] * kBlock + (r & 63);
     const bool vkey = valid_j[hf] && key < prm.n_valid;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = prm.scale_log2;
     bool ok = true;
+    uint32_t e_next = T > 0 ? dlist[0] : 0u;  // list entries are read one tile ahead
     for (int m = 0; m < T && ok; ++m) {
       const int x = m & 1, slot = m % S;
-      const bool act = vkey && ((dlist[m] >> (16 + hf)) & 1u);
+      const uint32_t e = e_next;
+      if (m + 1 < T) e_next = dlist[m + 1];
+      const bool act = vkey && ((e >> (16 + hf)) & 1u);
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + x), (m >> 1) & 1, abort)) &&
            __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED + slot), (m / S) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
       const uint32_t tS = tmem + lane_off + 2 * D + 128 * x;
-      uint32_t sv[2][32], pv[2][32];
-      tc::tmem_ld32(tS, sv[0]);
-      tc::tmem_ld32(tS + 32, sv[1]);
-      tc::tmem_ld32(tS + 64, pv[0]);
-      tc::tmem_ld32(tS + 96, pv[1]);
+      uint32_t sv[32], pv[32];
+      tc::tmem_ld32(tS + 32 * hw, sv);
+      tc::tmem_ld32(tS + 64 + 32 * hw, pv);
       tc::tmem_ld_wait();
-      const float* lse = reinterpret_cast<const float*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile);
+      const float* lse = reinterpret_cast<const float*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile) + 32 * hw;
       const float* dl = lse + 64;
-      uint32_t pw[32], dw[32];
+      uint32_t pw[16], dw[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < 16; ++j) {
         float pp[2], dd[2];
 #pragma unroll
         for (int y = 0; y < 2; ++y) {
           const int c = 2 * j + y;
-          const float p = act ? tc::ex2_approx(__uint_as_float(sv[c >> 5][c & 31]) * sl2 - lse[c]) : 0.f;
+          const float p = act ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse[c]) : 0.f;
           pp[y] = p;
-          dd[y] = p * (__uint_as_float(pv[c >> 5][c & 31]) - dl[c]);
+          dd[y] = p * (__uint_as_float(pv[c]) - dl[c]);
         }
         pw[j] = pack_bf16(pp[0], pp[1]);
         dw[j] = pack_bf16(dd[0], dd[1]);
       }
-      tc::tmem_st32(tS, pw);
-      tc::tmem_st32(tS + 64, dw);
+      // packed into the first 16 columns of this half (never over the other half's scores)
+      tc::tmem_st16(tS + 32 * hw, pw);
+      tc::tmem_st16(tS + 64 + 32 * hw, dw);
       tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
@@ -610,7 +620,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         if (acc) acc += row * D;
         const float sc = which == 0 ? 1.f : prm.scale;
 #pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = hw * (D / 64); ch < (hw + 1) * (D / 64); ++ch) {  // this warpgroup's half of the columns
           uint32_t v[32];
           if (ok && T > 0) {
             tc::tmem_ld32(tmem + lane_off + which * D + 32 * ch, v);
@@ -641,7 +651,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   if (T == 0 && tid == 0 && !tc::mbar_wait(bar(KV_FULL), 0, abort)) report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, L::kTmemCols);
   }
