@@ -129,3 +129,159 @@ def layer_grads(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, w_p: Optional[
     # an input with no path to the loss (e.g. no linear branch) has a zero gradient
     g = lambda x: None if x is None else (x.grad if x.grad is not None else torch.zeros_like(x)).detach().numpy().copy()
     return dict(dq=g(tq), dk=g(tk), dv=g(tv), dw_p=g(twp), dw_g=g(twg), O=o.detach().numpy())
+
+
+# ---------------------------------------------------------------------------
+# the same gradients block by block (full-size layers, sampled blocks)
+# ---------------------------------------------------------------------------
+
+def _dphi(x: np.ndarray) -> np.ndarray:
+    """phi'(x) for phi = elu + 1: 1 for x > 0, e^x otherwise."""
+    return np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_blocks, heads=None):
+    """Exact float64 gradients on chosen blocks, by the chain rule written out per block.
+
+    An independent statement of what ``layer_grads`` computes by autograd, for
+    layers too large for the token grid. For batch b it returns
+      dq[(h, i)]  rows of query block i of head h        (every h in ``heads``)
+      dk[(hk, j)], dv[(hk, j)]  rows of key block j of KV head hk, summed over the
+                  query heads of its group that are in ``heads``
+      dw_p        the contribution of ``heads`` to dW_p (shape of w_p), dw_g[h] rows.
+    Steps (routing fixed; phi = elu + 1; s = softmax scale):
+      sparse  per query block i over its critical tokens C_i: P = softmax(s Q_i K_C^T),
+              O_s = P V_C, dP = dO_i V_C^T, D = rowsum(dO_i * O_s), dS = P * (dP - D);
+              dq += s dS K_C, dK_C += s dS^T Q_i, dV_C += P^T dO_i
+      linear  S_i = sum_{j in M_i} phi(K_j)^T V_j, Z_i likewise, O_l = phi(q) S_i / den,
+              den = phi(q) . Z_i; u = O_l W_p, du = g dO, dO_l = du W_p^T;
+              dq += (dO_l S_i^T - (dO_l . O_l) Z_i) / den * phi'(q);
+              dS_i = sum_t phi(q_t)^T dO_l,t / den_t, dZ_i = -sum_t phi(q_t) (dO_l,t . O_l,t) / den_t;
+              dh_j = sum_{i: j in M_i} dS_i, dz_j likewise;
+              dV_j += phi(K_j) dh_j, dK_j += (V_j dh_j^T + dz_j) * phi'(K_j); dW_p += O_l^T du
+      gate    g = sigmoid(q . w_g[h]), dlogit = (dO . u) g (1 - g): dq += dlogit w_g[h],
+              dw_g[h] += sum_t dlogit q_t
+    Padding rows (index >= N_valid) contribute nothing and get zero rows.
+    """
+    c = so.OracleCfg.of(cfg)
+    assert c.mode == 0 and not c.smooth_k
+    nb, bl, nv, d, s = c.nb, c.block, c.N_valid, c.d, c.sm_scale
+    heads = list(range(c.H)) if heads is None else list(heads)
+    q_blocks, k_blocks = list(q_blocks), list(k_blocks)
+    out = dict(dq={}, dk={}, dv={}, dw_g={},
+               dw_p=None if not c.has_proj else np.zeros(np.shape(w_p)))
+    valid_kb = np.arange(nb) * bl < nv
+    rows_of = lambda i: slice(i * bl, min((i + 1) * bl, nv))
+    for h in heads:
+        hk = h // c.group
+        Q = np.asarray(q[b, h], dtype=np.float64)
+        K = np.asarray(k[b, hk], dtype=np.float64)
+        V = np.asarray(v[b, hk], dtype=np.float64)
+        dO = np.asarray(d_out[b, h], dtype=np.float64).copy()
+        dO[nv:] = 0.0
+        cls = classes[b, h]
+        wp = None
+        if c.has_proj:
+            wp = np.asarray(w_p[h] if c.proj_per_head else w_p, dtype=np.float64)
+        # ---- linear branch, every query block (dk / dv of any key block need all of them)
+        marg = (np.broadcast_to(valid_kb[None, :], cls.shape) if c.linear_all else cls == so.MARGINAL)
+        Mf = marg.astype(np.float64)
+        hs, zs = so.linear_states(K, V, nv, bl)
+        S = (Mf @ hs.reshape(nb, d * d)).reshape(nb, d, d)
+        Z = Mf @ zs
+        phq = so.phi(Q)
+        phq[nv:] = 0.0
+        den = np.zeros(c.N)
+        Ol = np.zeros((c.N, d))
+        for i in range(nb):
+            r = rows_of(i)
+            if r.start >= r.stop:
+                continue
+            den[r] = phq[r] @ Z[i]
+            num = phq[r] @ S[i]
+            Ol[r] = np.where(den[r, None] > 0, num / np.where(den[r, None] > 0, den[r, None], 1.0), 0.0)
+        u = Ol @ wp if wp is not None else Ol
+        g = so.sigmoid(Q @ np.asarray(w_g[h], dtype=np.float64)) if c.has_gate else np.ones(c.N)
+        g[nv:] = 0.0
+        du = g[:, None] * dO
+        dOl = du @ wp.T if wp is not None else du
+        if wp is not None:
+            if c.proj_per_head:
+                out["dw_p"][h] += Ol.T @ du
+            else:
+                out["dw_p"] += Ol.T @ du
+        dlogit = np.zeros(c.N)
+        if c.has_gate:
+            dlogit = (dO * u).sum(axis=1) * g * (1.0 - g)
+            dlogit[nv:] = 0.0
+            out["dw_g"][h] = dlogit @ Q
+        inv = np.where(den > 0, 1.0 / np.where(den > 0, den, 1.0), 0.0)
+        cdot = (dOl * Ol).sum(axis=1) * inv  # (dO_l . O_l) / den
+        dS = np.zeros((nb, d, d))
+        dZ = np.zeros((nb, d))
+        for i in range(nb):
+            r = rows_of(i)
+            if r.start >= r.stop:
+                continue
+            dS[i] = phq[r].T @ (dOl[r] * inv[r, None])
+            dZ[i] = -(phq[r] * cdot[r, None]).sum(axis=0)
+
+        # ---- sparse branch per query block (cached: dk / dv revisit blocks)
+        cache = {}
+
+        def sparse(i):
+            if i not in cache:
+                r = rows_of(i)
+                crit = np.nonzero(cls[i] == so.CRITICAL)[0]
+                toks = np.concatenate([np.arange(j * bl, min((j + 1) * bl, nv)) for j in crit]) \
+                    if crit.size else np.zeros(0, np.int64)
+                if toks.size == 0 or r.start >= r.stop:
+                    cache[i] = (toks, None, None)
+                else:
+                    x = Q[r] @ K[toks].T * s
+                    P = np.exp(x - x.max(axis=1, keepdims=True))
+                    P /= P.sum(axis=1, keepdims=True)
+                    Os = P @ V[toks]
+                    dP = dO[r] @ V[toks].T
+                    dSm = P * (dP - (dO[r] * Os).sum(axis=1, keepdims=True))
+                    cache[i] = (toks, P, dSm)
+            return cache[i]
+
+        for i in q_blocks:
+            r = rows_of(i)
+            g_rows = np.zeros((bl, d))
+            n = r.stop - r.start
+            if n > 0:
+                toks, P, dSm = sparse(i)
+                dq = np.zeros((n, d))
+                if P is not None:
+                    dq += s * dSm @ K[toks]
+                dphi = (dOl[r] @ S[i].T - (dOl[r] * Ol[r]).sum(axis=1, keepdims=True) * Z[i][None, :]) \
+                    * inv[r, None]
+                dq += dphi * _dphi(Q[r])
+                if c.has_gate:
+                    dq += dlogit[r, None] * np.asarray(w_g[h], dtype=np.float64)[None, :]
+                g_rows[:n] = dq
+            out["dq"][(h, i)] = g_rows
+        for j in k_blocks:
+            rk = rows_of(j)
+            nk = rk.stop - rk.start
+            dk = out["dk"].setdefault((hk, j), np.zeros((bl, d)))
+            dv = out["dv"].setdefault((hk, j), np.zeros((bl, d)))
+            if nk == 0:
+                continue
+            for i in np.nonzero(cls[:, j] == so.CRITICAL)[0]:
+                toks, P, dSm = sparse(i)
+                if P is None:
+                    continue
+                sel = (toks >= rk.start) & (toks < rk.stop)
+                r = rows_of(i)
+                dv[:nk] += P[:, sel].T @ dO[r]
+                dk[:nk] += s * dSm[:, sel].T @ Q[r]
+            dh = Mf[:, j] @ dS.reshape(nb, d * d)
+            dz = Mf[:, j] @ dZ
+            dh = dh.reshape(d, d)
+            phk = so.phi(K[rk])
+            dv[:nk] += phk @ dh
+            dk[:nk] += (V[rk] @ dh.T + dz[None, :]) * _dphi(K[rk])
+    return out

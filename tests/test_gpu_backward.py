@@ -7,7 +7,9 @@ GPU's own routing classes. Bar: relative Frobenius error <= 2e-2 per tensor.
 The arithmetic rounds P, dS, phi(K), the states and the outputs to bf16 (about
 4e-3 each), so a dropped term or a wrong index shows up as an O(1) error.
 The all-critical cases check the sparse branch alone, the all-marginal ones
-the linear branch, the projection and the gate alone.
+the linear branch, the projection and the gate alone. Full-size layers (the
+bench's shapes) are compared on sampled query and key blocks of every head, and
+on dW_p and dw_g in full, against the oracle's block-by-block statement.
 """
 import numpy as np
 import pytest
@@ -125,3 +127,53 @@ def test_backward_all_negligible_is_zero():
     assert sla.sla_check_device_status(bws) == (0, 0)
     for t in (dq, dk, dv, dw_p, dw_g):
         assert torch.count_nonzero(t).item() == 0
+
+
+# ---------------------------------------------------------------------------
+# full-size layers: sampled blocks of every head against the block-wise oracle
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["wan1.3b", "salad", "wan1.3b_cosfilter"])
+def test_full_size_backward_on_sampled_blocks(name):
+    """The bench's layer shapes (one sla_forward + sla_backward call, as bench.py times them).
+    dq on three query blocks and dk, dv on three key blocks of every head (first, middle,
+    last: the ragged tail included), dW_p and dw_g in full, against oracle block_grads."""
+    from gpu_util import LazyF64
+
+    cfg = wl.preset(name)
+    x = wl.generate(cfg)
+    run = GpuRun(cfg, x, route=False)
+    c = cfg
+    dob = d_out_bits(c, 17)
+    dout = to_dev(dob)
+    dq, dk, dv = torch.empty_like(run.q), torch.empty_like(run.k), torch.empty_like(run.v)
+    dw_p = torch.empty((c.d, c.d), dtype=torch.float32, device="cuda") if c.has_proj else None
+    dw_g = torch.empty((c.H, c.d), dtype=torch.float32, device="cuda") if c.has_gate else None
+    bws = torch.empty(sla.sla_backward_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    sla.sla_backward(run.q, run.k, run.v, run.w_p, run.w_g, c, run.out, dout, dq, dk, dv, dw_p, dw_g,
+                     run.ws, bws)
+    assert sla.sla_check_device_status(bws) == (0, 0)
+    nb = c.nqb
+    qb, kb = [0, nb // 2, nb - 1], [0, nb // 2 + 1, nb - 1]
+    classes = run.mask.cpu().numpy()
+    ref = sla_grad.block_grads(c, LazyF64(x.q), LazyF64(x.k), LazyF64(x.v),
+                               x.f64("w_p") if c.has_proj else None, x.f64("w_g") if c.has_gate else None,
+                               LazyF64(dob), classes, 0, qb, kb)
+    bl = c.block
+
+    def rel(pairs):
+        num = sum(float(np.sum((g - r) ** 2)) for g, r in pairs)
+        den = sum(float(np.sum(r ** 2)) for _, r in pairs)
+        return (num / den) ** 0.5
+
+    dq_h = lambda h, i: bf16_to_f64(dq[0, h, i * bl:(i + 1) * bl])
+    errs = {"dq": rel([(dq_h(h, i), r) for (h, i), r in ref["dq"].items()])}
+    for key, t in (("dk", dk), ("dv", dv)):
+        errs[key] = rel([(bf16_to_f64(t[0, hk, j * bl:(j + 1) * bl]), r) for (hk, j), r in ref[key].items()])
+    if c.has_proj:
+        errs["dw_p"] = rel([(dw_p.double().cpu().numpy(), ref["dw_p"])])
+    if c.has_gate:
+        g = dw_g.double().cpu().numpy()
+        errs["dw_g"] = rel([(g[h], r) for h, r in ref["dw_g"].items()])
+    print(name, errs)
+    assert all(e <= REL for e in errs.values()), errs

@@ -9,6 +9,8 @@ differentiate it. It is pinned against things other than itself:
   attention (dV = P^T dO, dS = P * (dP - rowsum(dO * O)), dQ = dS K s, dK = dS^T Q s);
 * with every block negligible they are zero.
 A planted mistake (a gradient that ignores the gate) fails the finite-difference pin.
+The block-by-block chain rule (``block_grads``, used on sampled blocks of
+full-size layers) is pinned against autograd on every block of small layers.
 """
 import math
 
@@ -145,3 +147,38 @@ def test_planted_gate_without_gradient_is_caught(monkeypatch):
     monkeypatch.setattr(sg.torch, "sigmoid", lambda x: real(x).detach())
     worst = _fd_check(c, lambda c, *a: sg.layer_grads(c, *a[:6], classes=a[6]))
     assert max(worst.values()) > 1e-3
+
+
+BLOCK_CASES = {
+    "proj_gate": dict(N=256, N_valid=250, k_h=2, k_l=2),
+    "gqa": dict(H=4, H_kv=2, N=256, k_h=2, k_l=1),
+    "per_head_proj": dict(proj_per_head=1, N=256, k_h=2, k_l=2),
+    "linear_all": dict(linear_all=1, N=256, k_h=2, k_l=3),
+    "plain": dict(has_proj=0, has_gate=0, N=256, N_valid=230, k_h=3, k_l=1),
+    "all_critical": dict(N=256, k_h=8, k_l=0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BLOCK_CASES))
+def test_block_grads_equal_autograd(name):
+    """The block-by-block chain rule (used at full size on sampled blocks) equals autograd."""
+    c = Cfg(**BLOCK_CASES[name])
+    q, k, v, w_p, w_g, d_out = inputs(c, seed=21)
+    classes = so.Layer(c, q, k, v, w_p, w_g).route()[0]
+    ref = sg.layer_grads(c, q, k, v, w_p, w_g, d_out, classes=classes)
+    nb = c.N // c.block
+    for b in range(c.B):
+        got = sg.block_grads(c, q, k, v, w_p, w_g, d_out, classes, b, range(nb), range(nb))
+        scale = lambda a: max(1e-12, float(np.abs(a).max()))
+        for (h, i), rows in got["dq"].items():
+            want = ref["dq"][b, h, i * c.block:(i + 1) * c.block]
+            assert np.abs(rows - want).max() <= 1e-10 * scale(ref["dq"]), (name, "dq", h, i)
+        for key in ("dk", "dv"):
+            for (hk, j), rows in got[key].items():
+                want = ref[key][b, hk, j * c.block:(j + 1) * c.block]
+                assert np.abs(rows - want).max() <= 1e-10 * scale(ref[key]), (name, key, hk, j)
+        if c.has_proj:
+            assert np.abs(got["dw_p"] - ref["dw_p"]).max() <= 1e-10 * scale(ref["dw_p"])
+        if c.has_gate:
+            for h, row in got["dw_g"].items():
+                assert np.abs(row - ref["dw_g"][h]).max() <= 1e-10 * scale(ref["dw_g"])
