@@ -186,3 +186,63 @@ def test_reorder_entry_points_reject_bad_arguments():
     assert L.sla_permute_tokens(256, 512 + 4, 256, 4, 1, 4, 8, 0, None) == sla.SLA_ERR_INVALID_ARG
     assert L.sla_permute_tokens(256, 512, 256, 4, 1, 4, 12, 0, None) == sla.SLA_ERR_INVALID_ARG
     assert L.sla_permute_tokens(256, 512, 256, 5, 1, 4, 8, 0, None) == sla.SLA_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------------------
+# backward entry points (host checks only: every call below fails validation)
+# ---------------------------------------------------------------------------
+
+def _call_backward(cfg, ptr=16, ws=256, bws=256, ws_bytes=None, bws_bytes=None, **over):
+    c = sla.make_config(cfg)
+    if ws_bytes is None:
+        ws_bytes = sla.sla_workspace_bytes(cfg)
+    if bws_bytes is None:
+        bws_bytes = sla.sla_backward_workspace_bytes(cfg)
+    a = dict(q=ptr, k=ptr, v=ptr, w_p=ptr, w_g=ptr, out=ptr, dout=ptr, dq=ptr, dk=ptr, dv=ptr, dw_p=ptr,
+             dw_g=ptr)
+    a.update(over)
+    return sla.lib().sla_backward(a["q"], a["k"], a["v"], a["w_p"], a["w_g"], ctypes.byref(c), a["out"],
+                                  a["dout"], a["dq"], a["dk"], a["dv"], a["dw_p"], a["dw_g"], ws, ws_bytes,
+                                  bws, bws_bytes, None)
+
+
+def test_backward_scope():
+    three = wl.small_config(N=1024, N_valid=1000, has_gate=1)
+    assert sla.sla_backward_workspace_bytes(three) > 0
+    assert sla.sla_backward_stage_names(three) == [
+        "bwd_columns", "bwd_linear", "bwd_mask_transpose", "bwd_aggregate_t", "bwd_state", "bwd_flash_dq",
+        "bwd_flash_dkdv"]
+    # no marginal block: D_t straight from the output
+    no_lin = wl.small_config(N=1024, N_valid=1024, k_h=8, k_l=8)
+    assert sla.sla_backward_stage_names(no_lin) == ["bwd_columns", "bwd_delta", "bwd_flash_dq", "bwd_flash_dkdv"]
+    for cfg in (wl.small_config(N=1024, N_valid=1024, smooth_k=1), wl.preset("nsa_causal")):
+        assert sla.sla_backward_workspace_bytes(cfg) == 0
+        assert sla.sla_backward_num_stages(cfg) == -1
+        assert _call_backward(cfg) == sla.SLA_ERR_UNSUPPORTED
+
+
+def test_backward_rejects_bad_arguments_before_launch():
+    cfg = wl.small_config(N=1024, N_valid=1000, has_gate=1)
+    for name in ("q", "k", "v", "out", "dout", "dq", "dk", "dv", "w_p", "w_g", "dw_p", "dw_g"):
+        assert _call_backward(cfg, **{name: None}) == sla.SLA_ERR_INVALID_ARG, name
+        assert _call_backward(cfg, **{name: 24}) == sla.SLA_ERR_INVALID_ARG, name  # misaligned
+    assert _call_backward(cfg, ws=None) == sla.SLA_ERR_WORKSPACE
+    assert _call_backward(cfg, ws_bytes=sla.sla_workspace_bytes(cfg) - 1) == sla.SLA_ERR_WORKSPACE
+    assert _call_backward(cfg, bws=None) == sla.SLA_ERR_WORKSPACE
+    assert _call_backward(cfg, bws=128) == sla.SLA_ERR_WORKSPACE
+    assert _call_backward(cfg, bws_bytes=sla.sla_backward_workspace_bytes(cfg) - 1) == sla.SLA_ERR_WORKSPACE
+    # without projection and gate their gradients may be NULL; a short scratch still stops the call
+    plain = wl.small_config(N=1024, N_valid=1000, has_proj=0, has_gate=0)
+    assert _call_backward(plain, w_p=None, w_g=None, dw_p=None, dw_g=None, bws_bytes=0) == sla.SLA_ERR_WORKSPACE
+    c = sla.make_config(cfg)
+    evs = (ctypes.c_void_p * 2)(1, 2)
+    r = sla.lib().sla_backward_timed(16, 16, 16, 16, 16, ctypes.byref(c), 16, 16, 16, 16, 16, 16, 16, 256,
+                                     sla.sla_workspace_bytes(cfg), 256, sla.sla_backward_workspace_bytes(cfg),
+                                     None, evs, 2)
+    assert r == sla.SLA_ERR_INVALID_ARG
+
+
+def test_backward_scratch_grows_with_the_problem():
+    small = wl.small_config(N=1024, N_valid=1024, has_gate=1)
+    big = wl.small_config(N=4096, N_valid=4096, has_gate=1)
+    assert sla.sla_backward_workspace_bytes(big) > 2 * sla.sla_backward_workspace_bytes(small)
