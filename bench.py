@@ -587,7 +587,8 @@ def main():
                    "N_valid": cfg.N_valid, "d": cfg.d, "k_h": cfg.k_h, "k_l": cfg.k_l,
                    "has_proj": cfg.has_proj, "has_gate": cfg.has_gate,
                    "parallelism": f"replicas x{world}",
-                   "l2": "inputs (Q,K,V 302 MB) larger than the 126 MB L2; no flush"},
+                   "l2": f"inputs (Q,K,V {(cfg.B * (cfg.H + 2 * cfg.H_kv) * cfg.N * cfg.d * 2) / 1e6:.0f} MB) larger "
+                         "than the 126 MB L2; no flush"},
         "ms_per_layer": ms_step,
         "per_replay_ms": {"warm_median": warm_med, "cold_median": cold_med, "reps": reps,
                           "cold": "256 MB written before each timed replay (L2 holds none of the layer's data)"},

@@ -108,7 +108,7 @@ struct DqLayout {
   static constexpr int kOffBar = kOffRing + kBwSlots * kSlot;  // 32 mbarriers
   static constexpr int kOffMisc = kOffBar + 32 * 8;
   static constexpr int kOffList = kOffMisc + 64;          // merged block list
-  static constexpr int kTmemCols = 512;                   // dQ: D; S / dP: 2 x 128
+  static constexpr int kTmemCols = 512;                   // dQ: D; S / dP: 2 x 128; dS: 2 x 32
 };
 
 struct DqParams {
@@ -143,8 +143,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   uint32_t* mlist = reinterpret_cast<uint32_t*>(smem + L::kOffList);
   uint32_t* words = reinterpret_cast<uint32_t*>(smem + L::kOffRing);  // bitmaps live in the ring before its first load
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
-  constexpr int QO_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, DS_FULL = SP_FULL + 2,
-                ACC_DONE = DS_FULL + 2;
+  // S / dP buffers: SP_FULL (products done), S_READ (row warps have loaded them);
+  // dS buffers: DS_FULL (written), DS_FREE (dQ product done)
+  constexpr int QO_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, S_READ = SP_FULL + 2,
+                DS_FULL = S_READ + 2, DS_FREE = DS_FULL + 2, ACC_DONE = DS_FREE + 2;
 
   for (int w = tid; w < 2 * prm.words; w += kBwThreads) words[w] = 0u;
   if (tid == 0) {
@@ -156,7 +158,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(bar(SP_FULL + x), 1);
+      tc::mbar_init(bar(S_READ + x), kRowWarps);
       tc::mbar_init(bar(DS_FULL + x), kRowWarps);
+      tc::mbar_init(bar(DS_FREE + x), 1);
     }
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::fence_mbar_init();
@@ -225,15 +229,19 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t kIdQ = tc::idesc_bf16(128, D, false, true);
+    // base descriptors; a byte offset off is added as off >> 4 (start-address field)
+    const uint64_t dQd = tc::sw128_desc(sQ, 16, 1024), dOd = tc::sw128_desc(sO, 16, 1024);
+    const uint64_t dRk = tc::sw128_desc(sR, 16, 1024);    // ring tiles, K-major
+    const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
     // S_m = Q K_m^T and dP_m = dO V_m^T into TMEM buffer m & 1
     auto issue_sp = [&](int m) {
-      const uint32_t kt = sR + (m % S) * L::kSlot, vt = kt + L::kTile;
+      const uint32_t so = (uint32_t)((m % S) * L::kSlot);
       const uint32_t tS = tmem + D + 128 * (m & 1);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t qo = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), ko = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
-        tc::mma_bf16_ss(tS, tc::sw128_desc(sQ + qo, 16, 1024), tc::sw128_desc(kt + ko, 16, 1024), kIdS, k > 0);
-        tc::mma_bf16_ss(tS + 64, tc::sw128_desc(sO + qo, 16, 1024), tc::sw128_desc(vt + ko, 16, 1024), kIdS, k > 0);
+        tc::mma_bf16_ss(tS, dQd + (qo >> 4), dRk + ((so + ko) >> 4), kIdS, k > 0);
+        tc::mma_bf16_ss(tS + 64, dOd + (qo >> 4), dRk + ((so + L::kTile + ko) >> 4), kIdS, k > 0);
       }
       tc::mma_commit(bar(SP_FULL + (m & 1)));
     };
@@ -249,30 +257,34 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
     for (int m = 0; m < T && ok; ++m) {
       const int b = m & 1;
-      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + b), (m >> 1) & 1, abort));
-      if (!ok) break;
-      tc::fence_after_sync();
-      if (tc::elect_one()) {
-        // dQ += dS_m K_m: A = dS_m from TMEM (bf16 pairs: keys 0-31 in columns 0-15 of the S
-        // buffer, keys 32-63 in columns 32-47), B = K_m N-major
-        const uint32_t kt = sR + (m % S) * L::kSlot;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_bf16_ts(tmem, tmem + D + 128 * b + 8 * kk + (kk >= 2 ? 16 : 0),
-                          tc::sw128_desc(kt + kk * 2048, 8192, 1024), kIdQ, (m > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_commit(bar(SLOT_FREE + m % S));
-        if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
-      }
-      __syncwarp();
-      if (m + 2 < T) {
-        // buffer b is free once dQ_m has read dS_m: S_{m+2} goes in behind it
-        // (tcgen05 operations of one thread execute in issue order)
+      // S / dP buffer b is free as soon as the row warps have loaded S_m, dP_m:
+      // the products of tile m + 2 run while they compute dS_m
+      ok = __all_sync(kAll, tc::mbar_wait(bar(S_READ + b), (m >> 1) & 1, abort));
+      if (ok && m + 2 < T) {
         ok = wait_loaded(m + 2);
         tc::fence_after_sync();
         if (ok && tc::elect_one()) issue_sp(m + 2);
         __syncwarp();
       }
+      ok = ok && __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + b), (m >> 1) & 1, abort));
+      if (!ok) break;
+      tc::fence_after_sync();
+      if (tc::elect_one()) {
+        // dQ += dS_m K_m: A = dS_m from its TMEM buffer (bf16 pairs), B = K_m N-major
+        const uint32_t so = (uint32_t)((m % S) * L::kSlot);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_bf16_ts(tmem, tmem + D + 256 + 32 * b + 8 * kk, dRn + ((so + kk * 2048) >> 4), kIdQ,
+                          (m > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_commit(bar(SLOT_FREE + m % S));
+        tc::mma_commit(bar(DS_FREE + b));
+        if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
+      }
+      __syncwarp();
     }
+    // the last two dS buffers' releases: no commit is in flight at exit
+    for (int m = (T > 2 ? T - 2 : 0); m < T && ok; ++m)
+      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FREE + (m & 1)), (m >> 1) & 1, abort));
     if (!ok && lane == 0) {
       *abort = 1;
       report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
@@ -302,6 +314,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tc::tmem_ld32(tS + 32 * hw, sv);
       tc::tmem_ld32(tS + 64 + 32 * hw, pv);
       tc::tmem_ld_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(S_READ + b));
       const int kc = k0 + 32 * hw;  // first key of this half
       uint32_t ds[16];
 #pragma unroll
@@ -315,8 +330,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         }
         ds[j] = pack_bf16(g2[0], g2[1]);
       }
-      // packed into the first 16 columns of this half (never over the other half's scores)
-      tc::tmem_st16(tS + 32 * hw, ds);
+      // dS buffer b was last read by dQ_{m-2}
+      if (m >= 2 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(DS_FREE + b), ((m - 2) >> 1) & 1, abort))))
+        break;
+      tc::fence_after_sync();
+      tc::tmem_st16(tmem + lane_off + D + 256 + 32 * b + 16 * hw, ds);
       tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
@@ -383,7 +401,7 @@ struct DkvLayout {
   static constexpr int kOffBar = kOffRing + kBwSlots * kSlot;
   static constexpr int kOffMisc = kOffBar + 32 * 8;
   static constexpr int kSmem = kOffMisc + 64;
-  static constexpr int kTmemCols = 512;                        // dV, dK: 2 D; S^T / dP^T: 2 x 128
+  static constexpr int kTmemCols = 512;  // dV, dK: 2 D; S^T / dP^T: 128; P^T / dS^T: 2 x 64 (bf16 pairs)
 };
 
 struct DkvParams {
@@ -422,8 +440,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);  // tmem, count, abort
   uint32_t* dlist = prm.dlist + (size_t)blockIdx.x * prm.group * prm.nb;
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
-  constexpr int KV_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, DS_FULL = SP_FULL + 2,
-                ACC_DONE = DS_FULL + 2;
+  // one S^T / dP^T buffer: SP_FULL (products done), S_READ (row warps have loaded them);
+  // two P^T / dS^T buffers: DS_FULL (written), PS_FREE (dV / dK products done)
+  constexpr int KV_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, S_READ = SP_FULL + 1,
+                DS_FULL = S_READ + 1, PS_FREE = DS_FULL + 2, ACC_DONE = PS_FREE + 2;
   const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sR = sbase + L::kOffRing;
   auto head_of = [&](int g) { return b * prm.H + hk * prm.group + g; };
 
@@ -434,9 +454,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tc::mbar_init(bar(LOADED + x), 1);
       tc::mbar_init(bar(SLOT_FREE + x), 1);
     }
+    tc::mbar_init(bar(SP_FULL), 1);
+    tc::mbar_init(bar(S_READ), kRowWarps);
     for (int x = 0; x < 2; ++x) {
-      tc::mbar_init(bar(SP_FULL + x), 1);
       tc::mbar_init(bar(DS_FULL + x), kRowWarps);
+      tc::mbar_init(bar(PS_FREE + x), 1);
     }
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::fence_mbar_init();
@@ -500,56 +522,66 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t kIdA = tc::idesc_bf16(128, D, false, true);
-    // S^T = K Q_i^T, dP^T = V dO_i^T (M = 128 keys, N = 64 queries) into TMEM buffer m & 1
+    // base descriptors; a byte offset off is added as off >> 4 (start-address field)
+    const uint64_t dKd = tc::sw128_desc(sK, 16, 1024), dVd = tc::sw128_desc(sV, 16, 1024);
+    const uint64_t dRk = tc::sw128_desc(sR, 16, 1024);    // ring tiles, K-major
+    const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
+    // S^T = K Q_i^T, dP^T = V dO_i^T (M = 128 keys, N = 64 queries) into the S buffer
     auto issue_sp = [&](int m) {
-      const uint32_t qt = sR + (m % S) * L::kSlot, ot = qt + L::kTile;
-      const uint32_t tS = tmem + 2 * D + 128 * (m & 1);
+      const uint32_t so = (uint32_t)((m % S) * L::kSlot);
+      const uint32_t tS = tmem + 2 * D;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ko = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), qo = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
-        tc::mma_bf16_ss(tS, tc::sw128_desc(sK + ko, 16, 1024), tc::sw128_desc(qt + qo, 16, 1024), kIdS, k > 0);
-        tc::mma_bf16_ss(tS + 64, tc::sw128_desc(sV + ko, 16, 1024), tc::sw128_desc(ot + qo, 16, 1024), kIdS, k > 0);
+        tc::mma_bf16_ss(tS, dKd + (ko >> 4), dRk + ((so + qo) >> 4), kIdS, k > 0);
+        tc::mma_bf16_ss(tS + 64, dVd + (ko >> 4), dRk + ((so + L::kTile + qo) >> 4), kIdS, k > 0);
       }
-      tc::mma_commit(bar(SP_FULL + (m & 1)));
+      tc::mma_commit(bar(SP_FULL));
     };
     auto wait_loaded = [&](int m) -> bool {
       return __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
     };
     bool ok = T == 0 || __all_sync(kAll, tc::mbar_wait(bar(KV_FULL), 0, abort));
-    for (int m = 0; m < 2 && m < T && ok; ++m) {
-      ok = wait_loaded(m);
+    if (T > 0 && ok) {
+      ok = wait_loaded(0);
       tc::fence_after_sync();
-      if (ok && tc::elect_one()) issue_sp(m);
+      if (ok && tc::elect_one()) issue_sp(0);
       __syncwarp();
     }
     for (int m = 0; m < T && ok; ++m) {
       const int x = m & 1;
-      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
+      // the S buffer is free once the row warps have loaded S^T_m, dP^T_m: the products of
+      // tile m + 1 run while they compute P^T_m and dS^T_m
+      ok = __all_sync(kAll, tc::mbar_wait(bar(S_READ), m & 1, abort));
+      if (ok && m + 1 < T) {
+        ok = wait_loaded(m + 1);
+        tc::fence_after_sync();
+        if (ok && tc::elect_one()) issue_sp(m + 1);
+        __syncwarp();
+      }
+      ok = ok && __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
       if (tc::elect_one()) {
-        // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T from TMEM (bf16 pairs: queries 0-31 in
-        // columns 0-15 of the buffer half, queries 32-63 in columns 32-47), B = dO_i / Q_i N-major
-        const uint32_t qt = sR + (m % S) * L::kSlot, ot = qt + L::kTile;
-        const uint32_t tP = tmem + 2 * D + 128 * x;
+        // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T from their TMEM buffer (bf16 pairs),
+        // B = dO_i / Q_i N-major
+        const uint32_t so = (uint32_t)((m % S) * L::kSlot);
+        const uint32_t tP = tmem + 2 * D + 128 + 64 * x;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t ka = 8 * kk + (kk >= 2 ? 16 : 0);
-          tc::mma_bf16_ts(tmem, tP + ka, tc::sw128_desc(ot + kk * 2048, 8192, 1024), kIdA, acc);
-          tc::mma_bf16_ts(tmem + D, tP + 64 + ka, tc::sw128_desc(qt + kk * 2048, 8192, 1024), kIdA, acc);
+          tc::mma_bf16_ts(tmem, tP + 8 * kk, dRn + ((so + L::kTile + kk * 2048) >> 4), kIdA, acc);
+          tc::mma_bf16_ts(tmem + D, tP + 32 + 8 * kk, dRn + ((so + kk * 2048) >> 4), kIdA, acc);
         }
         tc::mma_commit(bar(SLOT_FREE + m % S));
+        tc::mma_commit(bar(PS_FREE + x));
         if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
       }
       __syncwarp();
-      if (m + 2 < T) {
-        ok = wait_loaded(m + 2);
-        tc::fence_after_sync();
-        if (ok && tc::elect_one()) issue_sp(m + 2);
-        __syncwarp();
-      }
     }
+    // the last two P / dS buffers' releases: no commit is in flight at exit
+    for (int m = (T > 2 ? T - 2 : 0); m < T && ok; ++m)
+      ok = __all_sync(kAll, tc::mbar_wait(bar(PS_FREE + (m & 1)), (m >> 1) & 1, abort));
     if (!ok && lane == 0) {
       *abort = 1;
       report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
@@ -570,15 +602,18 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       const uint32_t e = e_next;
       if (m + 1 < T) e_next = dlist[m + 1];
       const bool act = vkey && ((e >> (16 + hf)) & 1u);
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + x), (m >> 1) & 1, abort)) &&
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL), m & 1, abort)) &&
            __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED + slot), (m / S) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
-      const uint32_t tS = tmem + lane_off + 2 * D + 128 * x;
+      const uint32_t tS = tmem + lane_off + 2 * D;
       uint32_t sv[32], pv[32];
       tc::tmem_ld32(tS + 32 * hw, sv);
       tc::tmem_ld32(tS + 64 + 32 * hw, pv);
       tc::tmem_ld_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(S_READ));
       const float* lse = reinterpret_cast<const float*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile) + 32 * hw;
       const float* dl = lse + 64;
       uint32_t pw[16], dw[16];
@@ -595,9 +630,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         pw[j] = pack_bf16(pp[0], pp[1]);
         dw[j] = pack_bf16(dd[0], dd[1]);
       }
-      // packed into the first 16 columns of this half (never over the other half's scores)
-      tc::tmem_st16(tS + 32 * hw, pw);
-      tc::tmem_st16(tS + 64 + 32 * hw, dw);
+      // P / dS buffer x was last read by the products of tile m - 2
+      if (m >= 2 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(PS_FREE + x), ((m - 2) >> 1) & 1, abort))))
+        break;
+      tc::fence_after_sync();
+      const uint32_t tP = tmem + lane_off + 2 * D + 128 + 64 * x;
+      tc::tmem_st16(tP + 16 * hw, pw);
+      tc::tmem_st16(tP + 32 + 16 * hw, dw);
       tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
