@@ -610,12 +610,21 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       uint32_t sv[32], pv[32];
       tc::tmem_ld32(tS + 32 * hw, sv);
       tc::tmem_ld32(tS + 64 + 32 * hw, pv);
+      // this half's log-sum-exp and D values (one per query column), as vectors while the
+      // TMEM loads are in flight
+      const float4* lse4 =
+          reinterpret_cast<const float4*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile) + 8 * hw;
+      float lse[32], dl[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 a = lse4[j], d4 = lse4[16 + j];
+        lse[4 * j] = a.x; lse[4 * j + 1] = a.y; lse[4 * j + 2] = a.z; lse[4 * j + 3] = a.w;
+        dl[4 * j] = d4.x; dl[4 * j + 1] = d4.y; dl[4 * j + 2] = d4.z; dl[4 * j + 3] = d4.w;
+      }
       tc::tmem_ld_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(S_READ));
-      const float* lse = reinterpret_cast<const float*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile) + 32 * hw;
-      const float* dl = lse + 64;
       uint32_t pw[16], dw[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {

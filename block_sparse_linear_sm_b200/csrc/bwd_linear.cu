@@ -680,10 +680,10 @@ __global__ void __launch_bounds__(128, 1)
       __syncwarp();
     }
   }
-  // dk = (T dh'^T + dz) * phi'(k)
+  // dk = (T dh'^T + dz) * phi'(k), phi'(k) = 1 for k > 0 and e^k = phi(k) otherwise, read off the
+  // phi(K) tile in shared memory (phi(k) >= 1 exactly when k > 0 up to the bf16 rounding of phi)
   if (ok && live) {
     float* dk_row = prm.dk_acc + ((size_t)bkv * prm.N + tok) * D;
-    const uint4* krow = reinterpret_cast<const uint4*>(prm.k + ((size_t)bkv * prm.N + tok) * D);
     const float* z = sZ + hf * D;
 #pragma unroll 1
     for (int ch = 0; ch < D / 32; ++ch) {
@@ -693,14 +693,15 @@ __global__ void __launch_bounds__(128, 1)
       float res[32];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        const uint4 kw = vtok ? krow[4 * ch + q4] : make_uint4(0, 0, 0, 0);
+        const uint4 kw = *reinterpret_cast<const uint4*>(smem + L::kOffK +
+                                                         sw_chunk((32 * ch) >> 6, r, (((32 * ch) & 63) >> 3) + q4));
         const uint32_t ks[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 kv = unpack_bf16(ks[e]);
+          const float2 fk = unpack_bf16(ks[e]);
           const int j = 8 * q4 + 2 * e, col = 32 * ch + j;
-          res[j] = vtok ? (__uint_as_float(v[j]) + z[col]) * (kv.x > 0.f ? 1.f : __expf(kv.x)) : 0.f;
-          res[j + 1] = vtok ? (__uint_as_float(v[j + 1]) + z[col + 1]) * (kv.y > 0.f ? 1.f : __expf(kv.y)) : 0.f;
+          res[j] = vtok ? (__uint_as_float(v[j]) + z[col]) * fminf(fk.x, 1.f) : 0.f;
+          res[j + 1] = vtok ? (__uint_as_float(v[j + 1]) + z[col + 1]) * fminf(fk.y, 1.f) : 0.f;
         }
       }
       float4* d4 = reinterpret_cast<float4*>(dk_row + 32 * ch);
