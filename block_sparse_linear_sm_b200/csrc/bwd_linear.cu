@@ -69,8 +69,9 @@ struct LinBwdLayout {
   static constexpr int NP = D / 64;
   static constexpr int kOffF = 0;                         // phi(Q): two feature panels (the second zero for D = 64)
   static constexpr int kOffQ = kOffF + 2 * 16384;         // q
-  static constexpr int kOffU = kOffQ + NP * 16384;        // du / den (bf16)
-  static constexpr int kOffS = kOffU + NP * 16384;        // S'_i of both blocks
+  static constexpr int kOffU = kOffQ + NP * 16384;        // dO, overwritten in place by du / den (bf16)
+  static constexpr int kOffO = kOffU + NP * 16384;        // O
+  static constexpr int kOffS = kOffO + NP * 16384;        // S'_i of both blocks
   static constexpr int kSBytes = NP * D * 128;            // one S' (D rows x D columns)
   static constexpr int kOffZ = kOffS + 2 * kSBytes;       // Z_i of both blocks (fp32)
   static constexpr int kOffC = kOffZ + 2 * D * 4;         // (du . u) / den per row
@@ -103,7 +104,8 @@ __device__ __forceinline__ uint32_t sw_chunk(int panel, int r, int cidx) {
 template <int D>
 __global__ void __launch_bounds__(128, 1)
     lin_bwd_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmQ,
-                   const __grid_constant__ CUtensorMap tmS, LinBwdParams prm) {
+                   const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmO,
+                   const __grid_constant__ CUtensorMap tmG, LinBwdParams prm) {
   using L = LinBwdLayout<D>;
   constexpr int NP = L::NP;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -160,11 +162,14 @@ __global__ void __launch_bounds__(128, 1)
   volatile int* abort = misc + 1;
 
   if (tid == 0) {
-    tc::mbar_expect_tx(bar(LOADED), 4 * NP * 8192 + nh * (L::kSBytes + D * 4));
+    tc::mbar_expect_tx(bar(LOADED), 8 * NP * 8192 + nh * (L::kSBytes + D * 4));
     for (int hf = 0; hf < 2; ++hf)
       for (int p = 0; p < NP; ++p) {
-        tc::tma_load_3d(sF + p * 16384 + hf * 8192, &tmF, bar(LOADED), 64 * p, i_h[hf] * kBlock, bh);
-        tc::tma_load_3d(sQ + p * 16384 + hf * 8192, &tmQ, bar(LOADED), 64 * p, i_h[hf] * kBlock, bh);
+        const uint32_t o = p * 16384 + hf * 8192;
+        tc::tma_load_3d(sF + o, &tmF, bar(LOADED), 64 * p, i_h[hf] * kBlock, bh);
+        tc::tma_load_3d(sQ + o, &tmQ, bar(LOADED), 64 * p, i_h[hf] * kBlock, bh);
+        tc::tma_load_3d(sU + o, &tmG, bar(LOADED), 64 * p, i_h[hf] * kBlock, bh);
+        tc::tma_load_3d(sbase + L::kOffO + o, &tmO, bar(LOADED), 64 * p, i_h[hf] * kBlock, bh);
       }
     for (int hf = 0; hf < nh; ++hf) {
       for (int p = 0; p < NP; ++p)
@@ -217,9 +222,7 @@ __global__ void __launch_bounds__(128, 1)
   tc::fence_after_sync();
   float dg = 0.f, dt = 0.f, cu = 0.f;
   if (ok) {
-    const size_t row_off = ((size_t)bh * prm.N + (valid_h[hf] ? t : 0)) * D;
-    const uint4* orow = reinterpret_cast<const uint4*>(prm.out + row_off);
-    const uint4* grow = reinterpret_cast<const uint4*>(prm.dout + row_off);
+    // O and dO rows from the tiles the loads brought in (rows past N_valid read as zero)
 #pragma unroll 1
     for (int ch = 0; ch < D / 32; ++ch) {
       uint32_t av[32];
@@ -228,8 +231,9 @@ __global__ void __launch_bounds__(128, 1)
       uint32_t ow[16], gw[16];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        const uint4 o4 = vrow ? orow[4 * ch + q4] : make_uint4(0, 0, 0, 0);
-        const uint4 g4 = vrow ? grow[4 * ch + q4] : make_uint4(0, 0, 0, 0);
+        const uint32_t off = sw_chunk((32 * ch) >> 6, r, (((32 * ch) & 63) >> 3) + q4);
+        const uint4 o4 = vrow ? *reinterpret_cast<const uint4*>(smem + L::kOffO + off) : make_uint4(0, 0, 0, 0);
+        const uint4 g4 = vrow ? *reinterpret_cast<const uint4*>(smem + L::kOffU + off) : make_uint4(0, 0, 0, 0);
         ow[4 * q4] = o4.x; ow[4 * q4 + 1] = o4.y; ow[4 * q4 + 2] = o4.z; ow[4 * q4 + 3] = o4.w;
         gw[4 * q4] = g4.x; gw[4 * q4 + 1] = g4.y; gw[4 * q4 + 2] = g4.z; gw[4 * q4 + 3] = g4.w;
       }
@@ -388,9 +392,11 @@ static cudaError_t launch_lin_bwd_t(const Plan& p, const BwdPlan& bp, const BwdA
   using L = LinBwdLayout<D>;
   const sla_config& c = p.c;
   const uint64_t rowb = (uint64_t)D * 2, headb = (uint64_t)c.N * D * 2, bh = (uint64_t)c.B * c.H;
-  CUtensorMap mf, mq, ms;
+  CUtensorMap mf, mq, ms, mo, mg;
   if (!make_tmap_3d(&mf, a.ws + p.off_phiq, D, (uint64_t)c.N_valid, bh, rowb, headb, 64, 64) ||
       !make_tmap_3d(&mq, a.q, D, (uint64_t)c.N_valid, bh, rowb, headb, 64, 64) ||
+      !make_tmap_3d(&mo, a.out, D, (uint64_t)c.N_valid, bh, rowb, headb, 64, 64) ||
+      !make_tmap_3d(&mg, a.dout, D, (uint64_t)c.N_valid, bh, rowb, headb, 64, 64) ||
       !make_tmap_3d(&ms, a.ws + p.off_ss, D, D, bh * p.nqb, rowb, (uint64_t)D * D * 2, 64, D))
     return cudaErrorInvalidValue;
   LinBwdParams prm;
@@ -414,7 +420,7 @@ static cudaError_t launch_lin_bwd_t(const Plan& p, const BwdPlan& bp, const BwdA
   prm.npairs = p.nqb_pad / 2;  // units past nqb write the zero padding rows
   cudaError_t e = cudaFuncSetAttribute(lin_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
-  lin_bwd_kernel<D><<<(unsigned)(bh * prm.npairs), 128, L::kSmem, s>>>(mf, mq, ms, prm);
+  lin_bwd_kernel<D><<<(unsigned)(bh * prm.npairs), 128, L::kSmem, s>>>(mf, mq, ms, mo, mg, prm);
   return cudaGetLastError();
 }
 
