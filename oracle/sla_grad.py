@@ -159,12 +159,14 @@ def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_bloc
               dS_i = sum_t phi(q_t)^T dO_l,t / den_t, dZ_i = -sum_t phi(q_t) (dO_l,t . O_l,t) / den_t;
               dh_j = sum_{i: j in M_i} dS_i, dz_j likewise;
               dV_j += phi(K_j) dh_j, dK_j += (V_j dh_j^T + dz_j) * phi'(K_j); dW_p += O_l^T du
+              (smooth-K: K_j - m in phi and phi', and every valid row of dK also gets
+              -1/N_valid times the sum over the head's valid tokens of that linear term)
       gate    g = sigmoid(q . w_g[h]), dlogit = (dO . u) g (1 - g): dq += dlogit w_g[h],
               dw_g[h] += sum_t dlogit q_t
     Padding rows (index >= N_valid) contribute nothing and get zero rows.
     """
     c = so.OracleCfg.of(cfg)
-    assert c.mode == 0 and not c.smooth_k
+    assert c.mode == 0
     nb, bl, nv, d, s = c.nb, c.block, c.N_valid, c.d, c.sm_scale
     heads = list(range(c.H)) if heads is None else list(heads)
     q_blocks, k_blocks = list(q_blocks), list(k_blocks)
@@ -186,7 +188,10 @@ def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_bloc
         # ---- linear branch, every query block (dk / dv of any key block need all of them)
         marg = (np.broadcast_to(valid_kb[None, :], cls.shape) if c.linear_all else cls == so.MARGINAL)
         Mf = marg.astype(np.float64)
-        hs, zs = so.linear_states(K, V, nv, bl)
+        # smooth-K: the linear branch sees K minus the mean valid key
+        koff = so.key_mean(K, nv) if c.smooth_k else np.zeros(d)
+        Kl = K - koff[None, :]
+        hs, zs = so.linear_states(K, V, nv, bl, koff if c.smooth_k else None)
         S = (Mf @ hs.reshape(nb, d * d)).reshape(nb, d, d)
         Z = Mf @ zs
         phq = so.phi(Q)
@@ -263,6 +268,18 @@ def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_bloc
                     dq += dlogit[r, None] * np.asarray(w_g[h], dtype=np.float64)[None, :]
                 g_rows[:n] = dq
             out["dq"][(h, i)] = g_rows
+        # smooth-K: dk_t = dkl_t - mean over the valid tokens of dkl (dkl = gradient through k - m)
+        kmean_grad = np.zeros(d)
+        if c.smooth_k:
+            dH = (Mf.T @ dS.reshape(nb, d * d)).reshape(nb, d, d)
+            dZk = Mf.T @ dZ
+            for j in range(nb):
+                rk = rows_of(j)
+                if rk.start >= rk.stop:
+                    continue
+                dkl = (V[rk] @ dH[j].T + dZk[j][None, :]) * _dphi(Kl[rk])
+                kmean_grad += dkl.sum(axis=0)
+            kmean_grad /= nv
         for j in k_blocks:
             rk = rows_of(j)
             nk = rk.stop - rk.start
@@ -281,7 +298,7 @@ def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_bloc
             dh = Mf[:, j] @ dS.reshape(nb, d * d)
             dz = Mf[:, j] @ dZ
             dh = dh.reshape(d, d)
-            phk = so.phi(K[rk])
+            phk = so.phi(Kl[rk])
             dv[:nk] += phk @ dh
-            dk[:nk] += (V[rk] @ dh.T + dz[None, :]) * _dphi(K[rk])
+            dk[:nk] += (V[rk] @ dh.T + dz[None, :]) * _dphi(Kl[rk]) - kmean_grad[None, :]
     return out

@@ -156,6 +156,8 @@ BLOCK_CASES = {
     "linear_all": dict(linear_all=1, N=256, k_h=2, k_l=3),
     "plain": dict(has_proj=0, has_gate=0, N=256, N_valid=230, k_h=3, k_l=1),
     "all_critical": dict(N=256, k_h=8, k_l=0),
+    "smooth_k": dict(smooth_k=1, N=256, N_valid=241, k_h=2, k_l=2),
+    "smooth_k_linear_all_gqa": dict(smooth_k=1, linear_all=1, H=4, H_kv=2, N=256, k_h=2, k_l=1),
 }
 
 
