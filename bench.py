@@ -541,7 +541,7 @@ def main():
 
     peaks = load_peaks()
     backward = None
-    if cfg.mode == wl.MODE_THREEWAY and not cfg.smooth_k and not args.no_backward:
+    if cfg.mode == wl.MODE_THREEWAY and not args.no_backward:
         backward = measure_backward(sla, torch, cfg, q, k, v, w_p, w_g, out, ws, args.steps, args.warmup,
                                     dist, dev, stream, peaks)
         barrier()

@@ -411,6 +411,7 @@ struct DkvParams {
   const float* delta;     // [B*H][N]
   const float* dk_acc;    // [B*H_kv][N][D] or null
   const float* dv_acc;
+  const float* kcol;      // smooth-K: [B*H_kv][D] = -(sum of the linear dk over valid tokens) / N_valid, or null
   __nv_bfloat16* dk;      // [B*H_kv][N][D]
   __nv_bfloat16* dv;
   int* status;
@@ -666,6 +667,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         __nv_bfloat16* dst = (which == 0 ? prm.dv : prm.dk) + row * D;
         const float* acc = which == 0 ? prm.dv_acc : prm.dk_acc;
         if (acc) acc += row * D;
+        const float* kc = (which == 1 && prm.kcol) ? prm.kcol + (size_t)bkv * D : nullptr;
         const float sc = which == 0 ? 1.f : prm.scale;
 #pragma unroll 1
         for (int ch = hw * (D / 64); ch < (hw + 1) * (D / 64); ++ch) {  // this warpgroup's half of the columns
@@ -685,6 +687,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
               const float2 xx = *reinterpret_cast<const float2*>(acc + 32 * ch + 2 * j);
               a0 += xx.x;
               a1 += xx.y;
+            }
+            if (kc) {  // smooth-K: the mean key's share of the gradient
+              a0 += kc[32 * ch + 2 * j];
+              a1 += kc[32 * ch + 2 * j + 1];
             }
             w[j] = vkey && ok ? pack_bf16(a0, a1) : 0u;
           }
@@ -767,6 +773,7 @@ static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs
   prm.delta = reinterpret_cast<const float*>(a.bws + bp.off_delta);
   prm.dk_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dkacc) : nullptr;
   prm.dv_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dvacc) : nullptr;
+  prm.kcol = bp.lin && c.smooth_k ? reinterpret_cast<const float*>(a.bws + bp.off_kcol) : nullptr;
   prm.dk = a.dk;
   prm.dv = a.dv;
   prm.status = a.status;

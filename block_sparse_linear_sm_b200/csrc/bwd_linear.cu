@@ -491,6 +491,7 @@ struct StBwdParams {
   float* dk_acc;           // [B*H_kv][N][D]
   float* dv_acc;
   float* dwp_part;         // [B*H_kv*npairs][D][D]: this CTA's dW_p partial, or null
+  const float* kmean;      // smooth-K: [B*H_kv][D] mean valid key (phi and phi' of k - m), or null
   int* status;
   int N, n_valid, nkb, npairs, has_proj, wp_heads;
 };
@@ -568,7 +569,8 @@ __global__ void __launch_bounds__(128, 1)
   const bool vtok = tok < prm.n_valid;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   if (ok) {
-    // phi(K) in place on this token's row (padding tokens zero)
+    // phi(K) (smooth-K: phi(K - m)) in place on this token's row (padding tokens zero)
+    const float* km = prm.kmean ? prm.kmean + (size_t)bkv * D : nullptr;
 #pragma unroll
     for (int p = 0; p < NP; ++p)
 #pragma unroll
@@ -576,10 +578,17 @@ __global__ void __launch_bounds__(128, 1)
         uint4* w = reinterpret_cast<uint4*>(smem + L::kOffK + sw_chunk(p, r, c));
         uint4 x = *w;
         uint32_t* xs = reinterpret_cast<uint32_t*>(&x);
+        float mv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (km) {
+          const float4 m0 = *reinterpret_cast<const float4*>(km + 64 * p + 8 * c);
+          const float4 m1 = *reinterpret_cast<const float4*>(km + 64 * p + 8 * c + 4);
+          mv[0] = m0.x; mv[1] = m0.y; mv[2] = m0.z; mv[3] = m0.w;
+          mv[4] = m1.x; mv[5] = m1.y; mv[6] = m1.z; mv[7] = m1.w;
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = unpack_bf16(xs[e]);
-          xs[e] = vtok ? pack_bf16(phi(f.x), phi(f.y)) : 0u;
+          xs[e] = vtok ? pack_bf16(phi(f.x - mv[2 * e]), phi(f.y - mv[2 * e + 1])) : 0u;
         }
         *w = x;
       }
@@ -762,6 +771,32 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// Smooth-K: column sums of the linear-branch dk (the gradient with respect to k - m) over
+// the valid tokens of each KV head, in two fixed-order passes (deterministic):
+// kcol_part_kernel grid (B*H_kv, kKcolSeg): one thread per column sums a segment of rows;
+// kcol_reduce_kernel adds the segments in order and scales by -1 / N_valid.
+constexpr int kKcolSeg = 64;
+
+__global__ void kcol_part_kernel(const float* __restrict__ dk_acc, float* __restrict__ part, int N, int n_valid,
+                                 int d) {
+  const int bkv = blockIdx.x, seg = blockIdx.y, c = threadIdx.x;
+  if (c >= d) return;
+  const int per = (n_valid + kKcolSeg - 1) / kKcolSeg;
+  const int t0 = seg * per, t1 = min(n_valid, t0 + per);
+  const float* src = dk_acc + (size_t)bkv * N * d + c;
+  float acc = 0.f;
+  for (int t = t0; t < t1; ++t) acc += src[(size_t)t * d];
+  part[((size_t)bkv * kKcolSeg + seg) * d + c] = acc;
+}
+
+__global__ void kcol_reduce_kernel(const float* __restrict__ part, float* __restrict__ kcol, int n_valid, int d) {
+  const int bkv = blockIdx.x, c = threadIdx.x;
+  if (c >= d) return;
+  float acc = 0.f;
+  for (int seg = 0; seg < kKcolSeg; ++seg) acc += part[((size_t)bkv * kKcolSeg + seg) * d + c];
+  kcol[(size_t)bkv * d + c] = -acc / (float)n_valid;
+}
+
 // dW_p[w] = sum of the partials of the units whose KV head uses W_p[w] (w = bkv % wp_heads).
 // grid (D*D/4 / 128, segments, wp_heads): each thread sums one float4 column over a
 // segment of the units and adds it to the gradient.
@@ -814,11 +849,19 @@ static cudaError_t launch_state_bwd_t(const Plan& p, const BwdPlan& bp, const Bw
   prm.npairs = (p.nkb + 1) / 2;
   prm.has_proj = proj ? 1 : 0;
   prm.wp_heads = wp_heads;
+  prm.kmean = c.smooth_k ? reinterpret_cast<const float*>(a.ws + p.off_kmean) : nullptr;
   cudaError_t e = cudaFuncSetAttribute(state_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   const int units = (int)bkv * prm.npairs;
   state_bwd_kernel<D><<<units, 128, L::kSmem, s>>>(mk, mv, mw, mh, prm);
-  if ((e = cudaGetLastError()) != cudaSuccess || !proj) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (c.smooth_k) {
+    float* part = reinterpret_cast<float*>(a.bws + bp.off_kcolp);
+    kcol_part_kernel<<<dim3((unsigned)bkv, kKcolSeg), D, 0, s>>>(prm.dk_acc, part, c.N, c.N_valid, D);
+    kcol_reduce_kernel<<<(unsigned)bkv, D, 0, s>>>(part, reinterpret_cast<float*>(a.bws + bp.off_kcol), c.N_valid, D);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (!proj) return cudaSuccess;
   dim3 grid((D * D / 4 + 127) / 128, 64, wp_heads);
   dwp_reduce_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(prm.dwp_part), a.dw_p, units,
                                          prm.npairs, wp_heads, D * D / 4);

@@ -185,7 +185,7 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
 static sla_status check_bwd_config(const sla_config* c) {
   const sla_status st = check_config(c);
   if (st != SLA_OK) return st;
-  if (c->mode != SLA_MODE_THREEWAY || c->smooth_k) return SLA_ERR_UNSUPPORTED;
+  if (c->mode != SLA_MODE_THREEWAY) return SLA_ERR_UNSUPPORTED;
   return SLA_OK;
 }
 
@@ -217,6 +217,10 @@ bool make_bwd_plan(const Plan& p, BwdPlan* b) {
     b->off_dz = take(B * Hkv * (size_t)p.nkb * d * 4);                  // dz_j (fp32)
     if (c.has_proj)  // dW_p partial of each pair of key blocks (fp32)
       b->off_dwp = take(B * Hkv * (size_t)((p.nkb + 1) / 2) * d * d * 4);
+    if (c.smooth_k) {  // column sums of the linear-branch dk: segment partials, then -sum / N_valid
+      b->off_kcolp = take(B * Hkv * 64 * d * 4);
+      b->off_kcol = take(B * Hkv * d * 4);
+    }
   }
   b->total = off;
   return true;

@@ -77,7 +77,7 @@ struct BwdPlan {
   int rows_t;     // group * nqb_pad
   int words;      // 32-bit words of one column bitmap (query blocks)
   size_t off_status, off_delta, off_dqacc, off_dkacc, off_dvacc, off_drow, off_maskt, off_dh, off_dz,
-      off_dwp, off_bits, off_dlist, total;
+      off_dwp, off_kcolp, off_kcol, off_bits, off_dlist, total;
 };
 bool make_bwd_plan(const Plan& p, BwdPlan* b);
 

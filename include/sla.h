@@ -262,10 +262,13 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
  *                           bytes, 256-byte aligned; its first 256 bytes hold
  *                           this call's device status word (read it with
  *                           sla_check_device_status(bws, ...))
- * SLA_ERR_UNSUPPORTED for the top-n mode and for smooth_k; other errors as for
- * sla_forward. The parameter gradients are sums of per-block partials added
- * with floating-point atomics, so their last bits may vary from run to run;
- * dq, dk and dv are deterministic.
+ *   smooth-K        phi and phi' of k - m (m the head's mean valid key); every valid
+ *                   row of dk also gets -1/N_valid times the head's summed
+ *                   linear-branch gradient with respect to k - m
+ * SLA_ERR_UNSUPPORTED for the top-n mode; other errors as for sla_forward. The
+ * parameter gradients are sums of per-block partials added with floating-point
+ * atomics, so their last bits may vary from run to run; dq, dk and dv are
+ * deterministic.
  */
 SLA_API size_t sla_backward_workspace_bytes(const sla_config* cfg);
 SLA_API sla_status sla_backward(const void* q, const void* k, const void* v,

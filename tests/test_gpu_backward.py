@@ -96,6 +96,10 @@ CASES = [
     dict(name="batch2_d64", B=2, N=640, N_valid=600, d=64, H=2, H_kv=1, k_h=2, k_l=1, has_gate=1),
     dict(name="single_block_d128", N=64, N_valid=50, d=128, k_h=1, k_l=0),
     dict(name="many_tiles_d128", N=4096, N_valid=4096, d=128, H=2, H_kv=2, k_h=16, k_l=16, has_gate=1),
+    dict(name="smooth_k_d128", N=1536, N_valid=1500, d=128, H=4, H_kv=4, k_h=3, k_l=4, smooth_k=1, has_gate=1),
+    dict(name="smooth_k_d64", N=1024, N_valid=1000, d=64, k_h=2, k_l=3, smooth_k=1),
+    dict(name="smooth_linear_all_gqa", N=1536, N_valid=1473, d=128, H=4, H_kv=2, k_h=3, k_l=2, smooth_k=1,
+         linear_all=1, has_gate=1),
 ]
 
 
@@ -133,7 +137,7 @@ def test_backward_all_negligible_is_zero():
 # full-size layers: sampled blocks of every head against the block-wise oracle
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("name", ["wan1.3b", "salad", "wan1.3b_cosfilter"])
+@pytest.mark.parametrize("name", ["wan1.3b", "salad", "wan1.3b_cosfilter", "wan1.3b_opensource"])
 def test_full_size_backward_on_sampled_blocks(name):
     """The bench's layer shapes (one sla_forward + sla_backward call, as bench.py times them).
     dq on three query blocks and dk, dv on three key blocks of every head (first, middle,
