@@ -62,18 +62,44 @@ def _masked_softmax_attention(q, k, v, allow, scale):
                        torch.zeros_like(q[:, :v.shape[1]]))
 
 
-def layer_forward_torch(cfg, q, k, v, w_p=None, w_g=None, classes: Optional[np.ndarray] = None):
-    """Three-way layer output O [B, H, N, d] (float64 torch, differentiable in every input).
+def _topn_allow(c, sel_rows) -> torch.Tensor:
+    """[N, N] bool, top-n mode: query t attends key s when s <= t, s is valid, and s's
+    block is selected for t's block or s > t - window."""
+    N, bl, nv = c.N, c.block, c.N_valid
+    selm = np.zeros((c.nb, c.nb), dtype=bool)
+    for i, row in enumerate(sel_rows):
+        selm[i, np.asarray(row, dtype=np.int64)] = True
+    t = np.arange(N)[:, None]
+    s = np.arange(N)[None, :]
+    in_win = (s > t - c.window) if c.window > 0 else np.zeros((N, N), dtype=bool)
+    return torch.from_numpy((s <= t) & (s < nv) & (selm[t // bl, s // bl] | in_win))
 
-    ``classes`` [B, H, nqb, nkb] fixes the routing (default: ``sla_oracle``'s own).
+
+def layer_forward_torch(cfg, q, k, v, w_p=None, w_g=None, classes=None):
+    """Layer output O [B, H, N, d] (float64 torch, differentiable in every input).
+
+    ``classes`` fixes the routing (default: ``sla_oracle``'s own): the three-way
+    classes [B, H, nqb, nkb], or in the top-n mode the selected lists
+    [B][H_kv][nqb] (the top-n mode has no linear branch: O = O_s).
     """
     c = so.OracleCfg.of(cfg)
-    assert c.mode == 0, "gradients are stated for the three-way mode"
     if classes is None:
         layer = so.Layer(cfg, q.detach().numpy(), k.detach().numpy(), v.detach().numpy(),
                          None if w_p is None else w_p.detach().numpy(),
                          None if w_g is None else w_g.detach().numpy())
         classes = layer.route()[0]
+    if c.mode != 0:
+        out = []
+        for b in range(c.B):
+            heads = []
+            for h in range(c.H):
+                hk = h // c.group
+                o = _masked_softmax_attention(q[b, h], k[b, hk], v[b, hk], _topn_allow(c, classes[b][hk]),
+                                              c.sm_scale)
+                row_ok = (torch.arange(c.N) < c.N_valid)[:, None]
+                heads.append(torch.where(row_ok, o, torch.zeros_like(o)))
+            out.append(torch.stack(heads))
+        return torch.stack(out)
     nb, bl, nv = c.nb, c.block, c.N_valid
     valid_kb = np.arange(nb) * bl < nv
     out = []
@@ -110,8 +136,9 @@ def layer_forward_torch(cfg, q, k, v, w_p=None, w_g=None, classes: Optional[np.n
 
 def layer_grads(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, w_p: Optional[np.ndarray],
                 w_g: Optional[np.ndarray], d_out: np.ndarray,
-                classes: Optional[np.ndarray] = None) -> Dict[str, Optional[np.ndarray]]:
+                classes=None) -> Dict[str, Optional[np.ndarray]]:
     """Gradients of L = sum(O * d_out) with the routing held fixed (float64 NumPy in and out).
+    ``classes``: as for ``layer_forward_torch``.
 
     Returns dq, dk, dv ([B, H(_kv), N, d]), dw_p (shape of w_p or None), dw_g
     ([H, d] or None) and O.
@@ -119,8 +146,8 @@ def layer_grads(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, w_p: Optional[
     c = so.OracleCfg.of(cfg)
     t = lambda a: None if a is None else torch.tensor(a, dtype=torch.float64, requires_grad=True)
     tq, tk, tv = t(q), t(k), t(v)
-    twp = t(w_p) if c.has_proj else None
-    twg = t(w_g) if c.has_gate else None
+    twp = t(w_p) if c.has_proj and c.mode == 0 else None
+    twg = t(w_g) if c.has_gate and c.mode == 0 else None
     if classes is None:
         classes = so.Layer(cfg, q, k, v, w_p, w_g).route()[0]
     o = layer_forward_torch(cfg, tq, tk, tv, twp, twg, classes)
@@ -166,7 +193,8 @@ def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_bloc
     Padding rows (index >= N_valid) contribute nothing and get zero rows.
     """
     c = so.OracleCfg.of(cfg)
-    assert c.mode == 0
+    if c.mode != 0:
+        return _block_grads_topn(c, q, k, v, d_out, classes, b, q_blocks, k_blocks, heads)
     nb, bl, nv, d, s = c.nb, c.block, c.N_valid, c.d, c.sm_scale
     heads = list(range(c.H)) if heads is None else list(heads)
     q_blocks, k_blocks = list(q_blocks), list(k_blocks)
@@ -301,4 +329,83 @@ def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_bloc
             phk = so.phi(Kl[rk])
             dv[:nk] += phk @ dh
             dk[:nk] += (V[rk] @ dh.T + dz[None, :]) * _dphi(Kl[rk]) - kmean_grad[None, :]
+    return out
+
+
+def _block_grads_topn(c, q, k, v, d_out, sels, b, q_blocks, k_blocks, heads=None):
+    """Top-n mode of ``block_grads`` (sparse branch only). Query block i attends the
+    tokens of its candidate blocks (selected blocks of its KV group and the blocks the
+    causal window reaches) under the element mask s <= t, s valid, (block(s) selected
+    or s > t - window); then P, dP, dS and the three products as in the three-way mode."""
+    nb, bl, nv, d, s = c.nb, c.block, c.N_valid, c.d, c.sm_scale
+    heads = list(range(c.H)) if heads is None else list(heads)
+    out = dict(dq={}, dk={}, dv={}, dw_g={}, dw_p=None)
+    rows_of = lambda i: slice(i * bl, min((i + 1) * bl, nv))
+
+    def cand_blocks(sel, i):
+        first = max(0, (i * bl - c.window + 1) // bl) if c.window > 0 else i + 1
+        return sorted(set(int(j) for j in sel) | set(range(first, i + 1)))
+
+    for h in heads:
+        hk = h // c.group
+        Q = np.asarray(q[b, h], dtype=np.float64)
+        K = np.asarray(k[b, hk], dtype=np.float64)
+        V = np.asarray(v[b, hk], dtype=np.float64)
+        dO = np.asarray(d_out[b, h], dtype=np.float64).copy()
+        dO[nv:] = 0.0
+        sel_rows = sels[b][hk]
+        cache = {}
+
+        def sparse(i):
+            if i not in cache:
+                r = rows_of(i)
+                blocks = cand_blocks(sel_rows[i], i)
+                toks = np.concatenate([np.arange(j * bl, min((j + 1) * bl, nv)) for j in blocks]) \
+                    if blocks else np.zeros(0, np.int64)
+                if toks.size == 0 or r.start >= r.stop:
+                    cache[i] = (toks, None, None)
+                else:
+                    t = np.arange(r.start, r.stop)[:, None]
+                    sj = toks[None, :]
+                    in_sel = np.isin(sj // bl, np.asarray(sel_rows[i], dtype=np.int64))
+                    in_win = (sj > t - c.window) if c.window > 0 else np.zeros_like(in_sel)
+                    allow = (sj <= t) & (in_sel | in_win)
+                    x = np.where(allow, Q[r] @ K[toks].T * s, -np.inf)
+                    m = x.max(axis=1, keepdims=True)
+                    m = np.where(np.isfinite(m), m, 0.0)
+                    P = np.where(allow, np.exp(x - m), 0.0)
+                    den = P.sum(axis=1, keepdims=True)
+                    P = np.where(den > 0, P / np.where(den > 0, den, 1.0), 0.0)
+                    Os = P @ V[toks]
+                    dP = dO[r] @ V[toks].T
+                    dSm = P * (dP - (dO[r] * Os).sum(axis=1, keepdims=True))
+                    cache[i] = (toks, P, dSm)
+            return cache[i]
+
+        for i in q_blocks:
+            r = rows_of(i)
+            g_rows = np.zeros((bl, d))
+            n = r.stop - r.start
+            if n > 0:
+                toks, P, dSm = sparse(i)
+                if P is not None:
+                    g_rows[:n] = s * dSm @ K[toks]
+            out["dq"][(h, i)] = g_rows
+        for j in k_blocks:
+            rk = rows_of(j)
+            nk = rk.stop - rk.start
+            dk = out["dk"].setdefault((hk, j), np.zeros((bl, d)))
+            dv = out["dv"].setdefault((hk, j), np.zeros((bl, d)))
+            if nk == 0:
+                continue
+            for i in range(j, nb):
+                if j not in cand_blocks(sel_rows[i], i):
+                    continue
+                toks, P, dSm = sparse(i)
+                if P is None:
+                    continue
+                selc = (toks >= rk.start) & (toks < rk.stop)
+                r = rows_of(i)
+                dv[:nk] += P[:, selc].T @ dO[r]
+                dk[:nk] += s * dSm[:, selc].T @ Q[r]
     return out

@@ -46,13 +46,16 @@ def inputs(c, seed=0):
 
 
 def oracle_loss(c, q, k, v, w_p, w_g, d_out, classes):
-    """sum(O * d_out) from sla_oracle's own forward pass, with the classes given."""
+    """sum(O * d_out) from sla_oracle's own forward pass, with the routing given."""
     layer = so.Layer(c, q, k, v, w_p, w_g)
     total = 0.0
     for b in range(c.B):
         for h in range(c.H):
             for i in range(c.N // c.block):
-                o = layer.unit(b, h, i, cls_row=classes[b, h, i])["O"]
+                if c.mode == 0:
+                    o = layer.unit(b, h, i, cls_row=classes[b, h, i])["O"]
+                else:
+                    o = layer.unit(b, h, i, sel_row=classes[b][h // (c.H // c.H_kv)][i])["O"]
                 total += float((o * d_out[b, h, i * c.block:(i + 1) * c.block]).sum())
     return total
 
@@ -66,6 +69,10 @@ CASES = {
     "linear_all": dict(linear_all=1, k_l=2),
     "plain": dict(has_proj=0, has_gate=0),
     "all_marginal": dict(k_h=0, k_l=0),
+    "topn_window_gqa": dict(mode=1, causal=1, top_n=1, window=40, k_h=0, k_l=0, has_proj=0, has_gate=0,
+                            H=4, H_kv=2),
+    "topn_ragged": dict(mode=1, causal=1, top_n=2, window=20, k_h=0, k_l=0, has_proj=0, has_gate=0,
+                        N=160, N_valid=150),
 }
 
 
@@ -85,7 +92,8 @@ def _fd_check(c, grads_fn, seed=5, eps=1e-6, rel=1e-6):
     classes = so.Layer(c, q, k, v, w_p, w_g).route()[0]
     g = grads_fn(c, q, k, v, w_p, w_g, d_out, classes)
     rng = np.random.default_rng(seed + 100)
-    names = ["q", "k", "v"] + (["w_p"] if c.has_proj else []) + (["w_g"] if c.has_gate else [])
+    names = ["q", "k", "v"] + (["w_p"] if c.has_proj and c.mode == 0 else []) + \
+        (["w_g"] if c.has_gate and c.mode == 0 else [])
     worst = {}
     for name in names:
         args = dict(q=q, k=k, v=v, w_p=w_p, w_g=w_g)
@@ -158,6 +166,8 @@ BLOCK_CASES = {
     "all_critical": dict(N=256, k_h=8, k_l=0),
     "smooth_k": dict(smooth_k=1, N=256, N_valid=241, k_h=2, k_l=2),
     "smooth_k_linear_all_gqa": dict(smooth_k=1, linear_all=1, H=4, H_kv=2, N=256, k_h=2, k_l=1),
+    "topn_window_gqa": dict(mode=1, causal=1, top_n=2, window=40, k_h=0, k_l=0, has_proj=0, has_gate=0,
+                            H=4, H_kv=2, N=256, N_valid=250),
 }
 
 
@@ -179,8 +189,8 @@ def test_block_grads_equal_autograd(name):
             for (hk, j), rows in got[key].items():
                 want = ref[key][b, hk, j * c.block:(j + 1) * c.block]
                 assert np.abs(rows - want).max() <= 1e-10 * scale(ref[key]), (name, key, hk, j)
-        if c.has_proj:
+        if c.has_proj and c.mode == 0:
             assert np.abs(got["dw_p"] - ref["dw_p"]).max() <= 1e-10 * scale(ref["dw_p"])
-        if c.has_gate:
+        if c.has_gate and c.mode == 0:
             for h, row in got["dw_g"].items():
                 assert np.abs(row - ref["dw_g"][h]).max() <= 1e-10 * scale(ref["dw_g"])
