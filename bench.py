@@ -92,6 +92,13 @@ def backward_stage_model(c: wl.LayerConfig) -> dict:
     lin = nb - c.k_h - c.k_l > 0 or c.linear_all
     dd = (d * d + d + 127) // 128 * 128
     words = (nb + 31) // 32
+    if c.mode != wl.MODE_THREEWAY:
+        # top-n mode: the attended (query, key) pairs, as counted for the forward pass
+        pairs = stage_model(c)["sparse_flash"][1] / (4.0 * d)
+        return {"bwd_columns": ("hbm", B * Hkv * nb * c.top_n * 4 + 2 * B * Hkv * nb * words * 4),
+                "bwd_delta": ("hbm", 2 * B * H * Nv * d * bf + B * H * N * 4),
+                "bwd_flash_dq": ("tensor", 6.0 * d * pairs),
+                "bwd_flash_dkdv": ("tensor", 8.0 * d * pairs)}
     m = {"bwd_columns": ("hbm", B * H * nb * c.k_h * 4 + 2 * B * H * nb * words * 4)}
     if lin:
         nqb_pad, nkb_pad = (nb + 127) // 128 * 128, (nb + 63) // 64 * 64
@@ -541,7 +548,7 @@ def main():
 
     peaks = load_peaks()
     backward = None
-    if cfg.mode == wl.MODE_THREEWAY and not args.no_backward:
+    if not args.no_backward:
         backward = measure_backward(sla, torch, cfg, q, k, v, w_p, w_g, out, ws, args.steps, args.warmup,
                                     dist, dev, stream, peaks)
         barrier()

@@ -32,48 +32,58 @@
 namespace sla {
 
 // ---------------------------------------------------------------------------
-// column bitmaps: bit i of bits[bh][j] is set when query block i has j critical
+// column bitmaps: bit i of bits[row][j] is set when query block i has key block j
+// critical (three-way: row = query head) or selected (top-n: row = KV head; the
+// selection is shared by the group, -1 entries are padding)
 // ---------------------------------------------------------------------------
 __global__ void cols_mark_kernel(const int32_t* __restrict__ crit, uint32_t* __restrict__ bits, int64_t entries,
-                                 int nqb, int nkb, int k_h, int words, int* status) {
+                                 int nqb, int nkb, int len, int words, int topn, int* status) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < entries; e += stride) {
-    const int64_t row = e / k_h;  // bh * nqb + i
-    const int bh = (int)(row / nqb), i = (int)(row % nqb);
+    const int64_t row = e / len;  // (head or KV head) * nqb + i
+    const int hr = (int)(row / nqb), i = (int)(row % nqb);
     const int j = crit[e];
-    if (j < 0 || j >= nkb) {
+    if (topn && j < 0) continue;
+    if (j < 0 || j >= nkb || (topn && j >= i)) {
       report(status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
       continue;
     }
-    atomicOr(bits + ((size_t)bh * nkb + j) * words + (i >> 5), 1u << (i & 31));
+    atomicOr(bits + ((size_t)hr * nkb + j) * words + (i >> 5), 1u << (i & 31));
   }
 }
 
 cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
   const sla_config& c = p.c;
+  const bool topn = c.mode == SLA_MODE_TOPN_WINDOW;
+  const int rows = topn ? c.H_kv : c.H, len = topn ? c.top_n : c.k_h;
   uint32_t* bits = reinterpret_cast<uint32_t*>(a.bws + bp.off_bits);
-  cudaError_t e = cudaMemsetAsync(bits, 0, (size_t)c.B * c.H * p.nkb * bp.words * 4, s);
-  if (e != cudaSuccess || c.k_h == 0) return e;
-  const int64_t entries = (int64_t)c.B * c.H * p.nqb * c.k_h;
+  cudaError_t e = cudaMemsetAsync(bits, 0, (size_t)c.B * rows * p.nkb * bp.words * 4, s);
+  if (e != cudaSuccess || len == 0) return e;
+  const int64_t entries = (int64_t)c.B * rows * p.nqb * len;
   int64_t blocks = (entries + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
   cols_mark_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const int32_t*>(a.ws + p.off_crit), bits,
-                                                    entries, p.nqb, p.nkb, c.k_h, bp.words, a.status);
+                                                    entries, p.nqb, p.nkb, len, bp.words, topn ? 1 : 0, a.status);
   return cudaGetLastError();
 }
-
 
 constexpr int kBwThreads = 320;  // warps 0-7 rows (two column halves), warp 8 MMA, warp 9 TMA producer
 constexpr int kMmaWarp = 8, kProdWarp = 9, kRowWarps = 8;
 constexpr int kBwSlots = 4;      // ring slots
 
-// merged list of two bitmaps (warp 0, ascending): entry = index | a0 << 16 | a1 << 17 | tag << 18;
-// returns the count (in every lane)
-__device__ __forceinline__ int merge_bitmaps(const uint32_t* w0p, const uint32_t* w1p, int words, bool v0, bool v1,
-                                             uint32_t tag, uint32_t* out, int base, int lane) {
+// merged list of two bitmaps (warp 0, ascending). Entry = index (bits 0-12) | a0 << 13 | a1 << 14
+// | s0 << 15 | s1 << 16 | tag << 17: a0 / a1 = the index is in bitmap a0 / a1 ("active" for
+// half 0 / 1), s0 / s1 = in bitmap s0 / s1 (top-n mode: "selected", NULL elsewhere).
+// Returns the count (in every lane).
+constexpr uint32_t kIdxMask = 0x1FFFu;
+constexpr int kActBit = 13, kSelBit = 15, kTagShift = 17;
+__device__ __forceinline__ int merge_bitmaps(const uint32_t* a0p, const uint32_t* a1p, const uint32_t* s0p,
+                                             const uint32_t* s1p, int words, bool v0, bool v1, uint32_t tag,
+                                             uint32_t* out, int base, int lane) {
   for (int w0 = 0; w0 < words; w0 += 32) {
     const int w = w0 + lane;
-    const uint32_t a0 = (w < words && v0) ? w0p[w] : 0u, a1 = (w < words && v1) ? w1p[w] : 0u;
+    const uint32_t a0 = (w < words && v0) ? a0p[w] : 0u, a1 = (w < words && v1) ? a1p[w] : 0u;
+    const uint32_t s0 = (s0p && w < words && v0) ? s0p[w] : 0u, s1 = (s1p && w < words && v1) ? s1p[w] : 0u;
     uint32_t any = a0 | a1;
     const int cnt = __popc(any);
     int incl = cnt;
@@ -87,7 +97,8 @@ __device__ __forceinline__ int merge_bitmaps(const uint32_t* w0p, const uint32_t
       const int bit = __ffs(any) - 1;
       any &= any - 1;
       const uint32_t m = 1u << bit;
-      out[pos++] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u) | (tag << 18);
+      out[pos++] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << kActBit : 0u) | ((a1 & m) ? 1u << (kActBit + 1) : 0u) |
+                   ((s0 & m) ? 1u << kSelBit : 0u) | ((s1 & m) ? 1u << (kSelBit + 1) : 0u) | (tag << kTagShift);
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
@@ -112,17 +123,18 @@ struct DqLayout {
 };
 
 struct DqParams {
-  const int32_t* crit;   // [B*H][nqb][k_h]
+  const int32_t* crit;   // three-way: [B*H][nqb][len] critical; top-n: [B*H_kv][nqb][len] selected (-1 pad)
   const float* lse;      // [B*H][N] (log2 domain)
   const float* delta;    // [B*H][N]
   const float* dq_acc;   // [B*H][N][D] or null
   __nv_bfloat16* dq;     // [B*H][N][D]
   int* status;
-  int H, group, N, n_valid, nb, k_h, npairs, words;
+  int H, group, N, n_valid, nb, len, npairs, words, window;
   float scale, scale_log2;
 };
 
-template <int D>
+// TOPN: element (t, s) is kept when s <= t and (block(s) selected or s > t - window)
+template <int D, bool TOPN>
 __global__ void __launch_bounds__(kBwThreads, 1)
     flash_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DqParams prm) {
@@ -148,7 +160,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   constexpr int QO_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, S_READ = SP_FULL + 2,
                 DS_FULL = S_READ + 2, DS_FREE = DS_FULL + 2, ACC_DONE = DS_FREE + 2;
 
-  for (int w = tid; w < 2 * prm.words; w += kBwThreads) words[w] = 0u;
+  // four bitmaps: active blocks of half 0 / 1, selected blocks of half 0 / 1 (top-n)
+  for (int w = tid; w < 4 * prm.words; w += kBwThreads) words[w] = 0u;
   if (tid == 0) {
     misc[2] = 0;
     tc::mbar_init(bar(QO_FULL), 1);
@@ -172,19 +185,29 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   __syncthreads();
   for (int hf = 0; hf < 2; ++hf) {
     if (!valid_h[hf]) continue;
-    const int32_t* lst = prm.crit + ((size_t)bh * prm.nb + i_h[hf]) * prm.k_h;
-    for (int e = tid; e < prm.k_h; e += kBwThreads) {
+    const int32_t* lst = prm.crit + ((size_t)(TOPN ? bkv : bh) * prm.nb + i_h[hf]) * prm.len;
+    uint32_t* act = words + hf * prm.words;
+    uint32_t* sel = words + (2 + hf) * prm.words;
+    for (int e = tid; e < prm.len; e += kBwThreads) {
       const int j = lst[e];
-      if (j < 0 || j >= prm.nb) {
+      if (TOPN && j < 0) continue;  // padding of short selections
+      if (j < 0 || j >= prm.nb || (TOPN && j >= i_h[hf])) {
         report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
         continue;
       }
-      atomicOr(&words[hf * prm.words + (j >> 5)], 1u << (j & 31));
+      atomicOr(&act[j >> 5], 1u << (j & 31));
+      if (TOPN) atomicOr(&sel[j >> 5], 1u << (j & 31));
+    }
+    if (TOPN && prm.window > 0) {  // the blocks the causal window reaches
+      const int lo = i_h[hf] * kBlock - prm.window + 1;
+      const int first = lo <= 0 ? 0 : lo / kBlock;
+      for (int j = first + tid; j <= i_h[hf]; j += kBwThreads) atomicOr(&act[j >> 5], 1u << (j & 31));
     }
   }
   __syncthreads();
   if (warp == 0) {
-    const int n = merge_bitmaps(words, words + prm.words, prm.words, true, true, 0u, mlist, 0, lane);
+    const int n = merge_bitmaps(words, words + prm.words, TOPN ? words + 2 * prm.words : nullptr,
+                                TOPN ? words + 3 * prm.words : nullptr, prm.words, true, true, 0u, mlist, 0, lane);
     if (lane == 0) misc[1] = n;
   }
   tc::fence_before_sync();
@@ -208,7 +231,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       for (int m = 0; m < T && ok; ++m) {
         const int slot = m % S;
         if (m >= S && !(ok = tc::mbar_wait(bar(SLOT_FREE + slot), ((m / S) - 1) & 1, abort))) break;
-        const int jb = (int)(mlist[m] & 0xFFFFu);
+        const int jb = (int)(mlist[m] & kIdxMask);
         const uint32_t dst = sR + slot * L::kSlot;
         tc::mbar_expect_tx(bar(LOADED + slot), L::kSlot);
         for (int p = 0; p < NP; ++p) {
@@ -304,8 +327,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     for (int m = 0; m < T && ok; ++m) {
       const int b = m & 1;
       const uint32_t e = mlist[m];
-      const int k0 = (int)(e & 0xFFFFu) * kBlock;
-      const bool act = (e >> (16 + hf)) & 1u;
+      const int k0 = (int)(e & kIdxMask) * kBlock;
+      const bool act = (e >> (kActBit + hf)) & 1u;
+      const bool sel = (e >> (kSelBit + hf)) & 1u;
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + b), (m >> 1) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
@@ -325,7 +349,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           const int c = 2 * j + x;
-          const float p = (act && kc + c < prm.n_valid) ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse2) : 0.f;
+          const int key = kc + c;
+          bool keep = act && key < prm.n_valid;
+          if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
+          const float p = keep ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse2) : 0.f;
           g2[x] = p * (__uint_as_float(pv[c]) - dlt);
         }
         ds[j] = pack_bf16(g2[0], g2[1]);
@@ -405,7 +432,7 @@ struct DkvLayout {
 };
 
 struct DkvParams {
-  const uint32_t* bits;   // [B*H][nkb][words]
+  const uint32_t* bits;   // three-way: [B*H][nkb][words] critical; top-n: [B*H_kv][nkb][words] selected
   uint32_t* dlist;        // [B*H_kv*npairs][group*nqb]: merged (head, query block) list of each unit
   const float* lse;       // [B*H][N] (log2 domain)
   const float* delta;     // [B*H][N]
@@ -415,11 +442,12 @@ struct DkvParams {
   __nv_bfloat16* dk;      // [B*H_kv][N][D]
   __nv_bfloat16* dv;
   int* status;
-  int H, group, N, n_valid, nb, npairs, words;
+  int H, group, N, n_valid, nb, npairs, words, window;
   float scale, scale_log2;
 };
 
-template <int D>
+// TOPN: element (query t, key s) is kept when s <= t and (block(s) selected or s > t - window)
+template <int D, bool TOPN>
 __global__ void __launch_bounds__(kBwThreads, 1)
     flash_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -475,12 +503,43 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     tc::tmem_relinquish();
   }
   if (warp == 0) {
-    // every query head of the group: the query blocks that hold j0 or j1 as critical
     int n = 0;
-    for (int g = 0; g < prm.group; ++g) {
-      const size_t row = (size_t)head_of(g) * prm.nb;
-      n = merge_bitmaps(prm.bits + (row + j_h[0]) * prm.words, prm.bits + (row + (valid_j[1] ? j_h[1] : 0)) * prm.words,
-                        prm.words, valid_j[0], valid_j[1], (uint32_t)g, dlist, n, lane);
+    if (!TOPN) {
+      // every query head of the group: the query blocks that hold j0 or j1 as critical
+      for (int g = 0; g < prm.group; ++g) {
+        const size_t row = (size_t)head_of(g) * prm.nb;
+        n = merge_bitmaps(prm.bits + (row + j_h[0]) * prm.words,
+                          prm.bits + (row + (valid_j[1] ? j_h[1] : 0)) * prm.words, nullptr, nullptr, prm.words,
+                          valid_j[0], valid_j[1], (uint32_t)g, dlist, n, lane);
+      }
+    } else {
+      // the group shares one selection: the query blocks that selected j0 / j1, plus those
+      // whose causal window reaches them (j <= i <= (64 j + 62 + window) / 64); four
+      // bitmaps (active 0 / 1, selected 0 / 1) in the ring before its first load
+      uint32_t* wb = reinterpret_cast<uint32_t*>(smem + L::kOffRing);
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t* selrow = prm.bits + ((size_t)bkv * prm.nb + (valid_j[h] ? j_h[h] : 0)) * prm.words;
+        int last = j_h[h] - 1;
+        if (prm.window > 0) {
+          last = (j_h[h] * kBlock + kBlock - 2 + prm.window) / kBlock;
+          if (last > prm.nb - 1) last = prm.nb - 1;
+        }
+        for (int w = lane; w < prm.words; w += 32) {
+          const uint32_t sv = valid_j[h] ? selrow[w] : 0u;
+          uint32_t win = 0u;
+          if (valid_j[h])
+            for (int b2 = 0; b2 < 32; ++b2) {
+              const int i = 32 * w + b2;
+              if (i >= j_h[h] && i <= last) win |= 1u << b2;
+            }
+          wb[h * prm.words + w] = sv | win;
+          wb[(2 + h) * prm.words + w] = sv;
+        }
+      }
+      __syncwarp();
+      for (int g = 0; g < prm.group; ++g)
+        n = merge_bitmaps(wb, wb + prm.words, wb + 2 * prm.words, wb + 3 * prm.words, prm.words, valid_j[0],
+                          valid_j[1], (uint32_t)g, dlist, n, lane);
     }
     if (lane == 0) misc[1] = n;
   }
@@ -499,7 +558,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         const int slot = m % S;
         if (m >= S && !(ok = tc::mbar_wait(bar(SLOT_FREE + slot), ((m / S) - 1) & 1, abort))) break;
         const uint32_t e = dlist[m];
-        const int i = (int)(e & 0xFFFFu), bh = head_of((int)(e >> 18));
+        const int i = (int)(e & kIdxMask), bh = head_of((int)(e >> kTagShift));
         const uint32_t dst = sR + slot * L::kSlot;
         tc::mbar_expect_tx(bar(LOADED + slot), 2 * L::kTile + 512);
         for (int p = 0; p < NP; ++p) {
@@ -602,7 +661,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       const int x = m & 1, slot = m % S;
       const uint32_t e = e_next;
       if (m + 1 < T) e_next = dlist[m + 1];
-      const bool act = vkey && ((e >> (16 + hf)) & 1u);
+      const bool act = vkey && ((e >> (kActBit + hf)) & 1u);
+      const bool sel = (e >> (kSelBit + hf)) & 1u;
+      const int t0 = (int)(e & kIdxMask) * kBlock + 32 * hw;  // first query token of this half
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL), m & 1, abort)) &&
            __all_sync(0xffffffffu, tc::mbar_wait(bar(LOADED + slot), (m / S) & 1, abort));
       if (!ok) break;
@@ -633,7 +694,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 #pragma unroll
         for (int y = 0; y < 2; ++y) {
           const int c = 2 * j + y;
-          const float p = act ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse[c]) : 0.f;
+          bool keep = act;
+          if (TOPN) keep = keep && key <= t0 + c && (sel || key > t0 + c - prm.window);
+          const float p = keep ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse[c]) : 0.f;
           pp[y] = p;
           dd[y] = p * (__uint_as_float(pv[c]) - dl[c]);
         }
@@ -719,7 +782,7 @@ static bool map64(CUtensorMap* m, const void* base, int heads, int n_rows, int N
                       (uint64_t)N * D * 2, 64, 64);
 }
 
-template <int D>
+template <int D, bool TOPN>
 static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
   using L = DqLayout<D>;
   const sla_config& c = p.c;
@@ -739,26 +802,31 @@ static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& 
   prm.N = c.N;
   prm.n_valid = c.N_valid;
   prm.nb = p.nkb;
-  prm.k_h = c.k_h;
+  prm.len = TOPN ? c.top_n : c.k_h;
   prm.npairs = (p.nqb + 1) / 2;
   prm.words = (p.nkb + 31) / 32;
+  prm.window = c.window;
   prm.scale = p.scale;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
-  const int cap = 2 * c.k_h < p.nkb ? 2 * c.k_h : p.nkb;
+  int per_half = prm.len;
+  if (TOPN) per_half += (c.window + 62) / kBlock + 2;  // selected blocks plus the window's reach
+  const int cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
   int smem = L::kOffList + (cap > 0 ? cap : 1) * 4;
-  if (2 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
+  if (4 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: it holds all 512 TMEM columns
-  cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D, TOPN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dq_kernel<D><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  flash_dq_kernel<D, TOPN><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_flash_dq(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
-  return p.c.d == 128 ? launch_dq_t<128>(p, bp, a, s) : launch_dq_t<64>(p, bp, a, s);
+  const bool topn = p.c.mode == SLA_MODE_TOPN_WINDOW;
+  if (p.c.d == 128) return topn ? launch_dq_t<128, true>(p, bp, a, s) : launch_dq_t<128, false>(p, bp, a, s);
+  return topn ? launch_dq_t<64, true>(p, bp, a, s) : launch_dq_t<64, false>(p, bp, a, s);
 }
 
-template <int D>
+template <int D, bool TOPN>
 static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
   using L = DkvLayout<D>;
   const sla_config& c = p.c;
@@ -784,18 +852,22 @@ static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs
   prm.nb = p.nkb;
   prm.npairs = (p.nkb + 1) / 2;
   prm.words = bp.words;
+  prm.window = c.window;
   prm.scale = p.scale;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
   int smem = L::kSmem;
+  if (TOPN && 4 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (512 TMEM columns)
-  cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D, TOPN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dkdv_kernel<D><<<c.B * c.H_kv * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  flash_dkdv_kernel<D, TOPN><<<c.B * c.H_kv * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_flash_dkdv(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
-  return p.c.d == 128 ? launch_dkdv_t<128>(p, bp, a, s) : launch_dkdv_t<64>(p, bp, a, s);
+  const bool topn = p.c.mode == SLA_MODE_TOPN_WINDOW;
+  if (p.c.d == 128) return topn ? launch_dkdv_t<128, true>(p, bp, a, s) : launch_dkdv_t<128, false>(p, bp, a, s);
+  return topn ? launch_dkdv_t<64, true>(p, bp, a, s) : launch_dkdv_t<64, false>(p, bp, a, s);
 }
 
 }  // namespace sla

@@ -667,7 +667,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
   prm.o = a.out;  // the sparse branch is the output, or the fused epilogue writes it
   prm.zs = FUSE ? reinterpret_cast<const float*>(a.ws + p.off_zs) : nullptr;
   prm.gate = FUSE && c.has_gate ? reinterpret_cast<const float*>(a.ws + p.off_gate) : nullptr;
-  prm.lse = !TOPN ? reinterpret_cast<float*>(a.ws + p.off_lse) : nullptr;
+  prm.lse = reinterpret_cast<float*>(a.ws + p.off_lse);
   prm.status = a.status;
   prm.H = c.H;
   prm.group = p.group;

@@ -81,6 +81,7 @@ bool make_plan(const sla_config* c, Plan* p) {
     }
   } else {
     p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
+    p->off_lse = take(B * H * (size_t)c->N * 4);  // row log2-sum-exp of the sparse branch (backward)
   }
   p->total = off;
   return true;
@@ -182,17 +183,12 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
 // ---------------------------------------------------------------------------
 // backward pass
 // ---------------------------------------------------------------------------
-static sla_status check_bwd_config(const sla_config* c) {
-  const sla_status st = check_config(c);
-  if (st != SLA_OK) return st;
-  if (c->mode != SLA_MODE_THREEWAY) return SLA_ERR_UNSUPPORTED;
-  return SLA_OK;
-}
+static sla_status check_bwd_config(const sla_config* c) { return check_config(c); }
 
 bool make_bwd_plan(const Plan& p, BwdPlan* b) {
   memset(b, 0, sizeof(*b));
   const sla_config& c = p.c;
-  b->lin = has_marginal(p);
+  b->lin = c.mode == SLA_MODE_THREEWAY && has_marginal(p);  // the top-n mode has no linear branch
   b->rows_t = p.group * p.nqb_pad;
   b->words = (p.nqb + 31) / 32;
   const size_t B = c.B, H = c.H, Hkv = c.H_kv, d = c.d, N = c.N;

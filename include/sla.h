@@ -226,7 +226,7 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
                                       void* stream);
 
 /*
- * Backward pass of the three-way layer (fine-tuning with the layer in place:
+ * Backward pass of the layer (fine-tuning with the layer in place:
  * SLA analysis page, arXiv 2509.24006, and SALAD summary, both train the model
  * with the sparse+linear layer for a few steps). The pages print no backward
  * pass; the gradients are those of L = sum(out * dout) with the routing held
@@ -255,6 +255,7 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
  *   dk, dv                  bf16 [B, H_kv, N, d] written (padding rows 0)
  *   dw_p                    fp32, shape of w_p; written; may be NULL unless has_proj
  *   dw_g                    fp32 [H, d]; written; may be NULL unless has_gate
+ *                           (the top-n mode has neither)
  *   ws                      the workspace of that sla_forward call, unchanged
  *                           since: the routing, the states S'_i, Z_i, phi(Q),
  *                           the gate and the row log-sum-exp are read from it
@@ -265,10 +266,12 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
  *   smooth-K        phi and phi' of k - m (m the head's mean valid key); every valid
  *                   row of dk also gets -1/N_valid times the head's summed
  *                   linear-branch gradient with respect to k - m
- * SLA_ERR_UNSUPPORTED for the top-n mode; other errors as for sla_forward. The
- * parameter gradients are sums of per-block partials added with floating-point
- * atomics, so their last bits may vary from run to run; dq, dk and dv are
- * deterministic.
+ *   top-n mode      the sparse branch only, over each query block's selected blocks and
+ *                   window with the forward's element mask (s <= t, and block(s)
+ *                   selected or s > t - window); dk, dv sum over the KV group's heads
+ * Errors as for sla_forward. The parameter gradients are sums of per-block
+ * partials added with floating-point atomics, so their last bits may vary from
+ * run to run; dq, dk and dv are deterministic.
  */
 SLA_API size_t sla_backward_workspace_bytes(const sla_config* cfg);
 SLA_API sla_status sla_backward(const void* q, const void* k, const void* v,

@@ -216,10 +216,13 @@ def test_backward_scope():
     no_lin = wl.small_config(N=1024, N_valid=1024, k_h=8, k_l=8)
     assert sla.sla_backward_stage_names(no_lin) == ["bwd_columns", "bwd_delta", "bwd_flash_dq", "bwd_flash_dkdv"]
     assert sla.sla_backward_workspace_bytes(wl.small_config(N=1024, N_valid=1024, smooth_k=1)) > 0
-    cfg = wl.preset("nsa_causal")
-    assert sla.sla_backward_workspace_bytes(cfg) == 0
-    assert sla.sla_backward_num_stages(cfg) == -1
-    assert _call_backward(cfg) == sla.SLA_ERR_UNSUPPORTED
+    # top-n mode: the sparse branch only
+    topn = wl.preset("nsa_causal")
+    assert sla.sla_backward_workspace_bytes(topn) > 0
+    assert sla.sla_backward_stage_names(topn) == ["bwd_columns", "bwd_delta", "bwd_flash_dq", "bwd_flash_dkdv"]
+    bad = wl.small_config(N=1024, N_valid=1024, d=80)
+    assert sla.sla_backward_workspace_bytes(bad) == 0 and sla.sla_backward_num_stages(bad) == -1
+    assert _call_backward(bad) == sla.SLA_ERR_UNSUPPORTED
 
 
 def test_backward_rejects_bad_arguments_before_launch():

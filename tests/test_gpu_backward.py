@@ -35,6 +35,13 @@ def d_out_bits(c, seed):
     return wl.to_bf16_bits(rng.standard_normal((c.B, c.H, c.N, c.d)))
 
 
+def topn_selection(run):
+    """The GPU's own top-n selection as lists [B][H_kv][nqb] (from its routing mask)."""
+    m = run.mask.cpu().numpy()
+    return [[[np.nonzero(m[b, hk, i] == 2)[0] for i in range(m.shape[2])] for hk in range(m.shape[1])]
+            for b in range(m.shape[0])]
+
+
 def run_backward(cfg, seed=3, v_shift=0.0):
     x = wl.generate(cfg, v_shift=v_shift)
     run = GpuRun(cfg, x, route=False)
@@ -55,7 +62,7 @@ def run_backward(cfg, seed=3, v_shift=0.0):
                      run.ws, bws)
     st, detail = sla.sla_check_device_status(bws)
     assert st == 0, (st, detail)
-    classes = run.mask.cpu().numpy()
+    classes = run.mask.cpu().numpy() if c.mode == wl.MODE_THREEWAY else topn_selection(run)
     ref = sla_grad.layer_grads(c, x.f64("q"), x.f64("k"), x.f64("v"),
                                x.f64("w_p") if c.has_proj else None,
                                x.f64("w_g") if c.has_gate else None,
@@ -100,6 +107,15 @@ CASES = [
     dict(name="smooth_k_d64", N=1024, N_valid=1000, d=64, k_h=2, k_l=3, smooth_k=1),
     dict(name="smooth_linear_all_gqa", N=1536, N_valid=1473, d=128, H=4, H_kv=2, k_h=3, k_l=2, smooth_k=1,
          linear_all=1, has_gate=1),
+    # top-n + window mode (causal, GQA, shared selections): the sparse branch only
+    dict(name="topn_gqa_d128", N=2048, N_valid=2048, d=128, H=4, H_kv=2, mode=wl.MODE_TOPN_WINDOW, causal=1,
+         top_n=4, window=256, k_h=0, k_l=0, has_proj=0),
+    dict(name="topn_odd_group_ragged_d64", N=1536, N_valid=1500, d=64, H=3, H_kv=1, mode=wl.MODE_TOPN_WINDOW,
+         causal=1, top_n=3, window=100, k_h=0, k_l=0, has_proj=0),
+    dict(name="topn_no_window_d128", N=1024, N_valid=1024, d=128, H=2, H_kv=2, mode=wl.MODE_TOPN_WINDOW,
+         causal=1, top_n=2, window=0, k_h=0, k_l=0, has_proj=0),
+    dict(name="topn_window_only_d64", N=1024, N_valid=1000, d=64, H=4, H_kv=1, mode=wl.MODE_TOPN_WINDOW,
+         causal=1, top_n=0, window=192, k_h=0, k_l=0, has_proj=0),
 ]
 
 
@@ -180,4 +196,36 @@ def test_full_size_backward_on_sampled_blocks(name):
         g = dw_g.double().cpu().numpy()
         errs["dw_g"] = rel([(g[h], r) for h, r in ref["dw_g"].items()])
     print(name, errs)
+    assert all(e <= REL for e in errs.values()), errs
+
+
+def test_full_size_topn_backward_on_sampled_blocks():
+    """The NSA-shaped top-n layer (H=64, H_kv=4, N=65536, top 16, window 512): dq on four query
+    blocks of the 16 heads of KV group 0, dk and dv on three key blocks of KV head 0 (complete:
+    they sum over exactly those heads), against oracle block_grads."""
+    from gpu_util import LazyF64
+
+    c = wl.preset("nsa_causal")
+    x = wl.generate(c)
+    run = GpuRun(c, x, route=False)
+    dob = d_out_bits(c, 19)
+    dout = to_dev(dob)
+    dq, dk, dv = torch.empty_like(run.q), torch.empty_like(run.k), torch.empty_like(run.v)
+    bws = torch.empty(sla.sla_backward_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    sla.sla_backward(run.q, run.k, run.v, None, None, c, run.out, dout, dq, dk, dv, None, None, run.ws, bws)
+    assert sla.sla_check_device_status(bws) == (0, 0)
+    nb, bl = c.nqb, c.block
+    qb, kb = [1, 17, nb // 2, nb - 1], [0, nb // 2 + 1, nb - 1]
+    ref = sla_grad.block_grads(c, LazyF64(x.q), LazyF64(x.k), LazyF64(x.v), None, None, LazyF64(dob),
+                               topn_selection(run), 0, qb, kb, heads=range(c.H // c.H_kv))
+
+    def rel(pairs):
+        num = sum(float(np.sum((g - r) ** 2)) for g, r in pairs)
+        den = sum(float(np.sum(r ** 2)) for _, r in pairs)
+        return (num / den) ** 0.5
+
+    errs = {"dq": rel([(bf16_to_f64(dq[0, h, i * bl:(i + 1) * bl]), r) for (h, i), r in ref["dq"].items()])}
+    for key, t in (("dk", dk), ("dv", dv)):
+        errs[key] = rel([(bf16_to_f64(t[0, hk, j * bl:(j + 1) * bl]), r) for (hk, j), r in ref[key].items()])
+    print("nsa_causal", errs)
     assert all(e <= REL for e in errs.values()), errs
