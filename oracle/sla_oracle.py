@@ -39,6 +39,13 @@ What each step follows (page title, section):
   other block (equal scores: lower index first) and get probability 0 in the
   top-n softmax; a row whose candidates are all filtered has all
   probabilities 0.
+* NSA's three branches (top-n mode option): sparse attention survey, section 2
+  (NSA: a compressed branch over coarse blocks of 32 tokens at stride 16, the
+  selected branch and the sliding window, in parallel); each branch is its own
+  softmax and the branches are summed with per-head gates g = sigmoid(q . w_g)
+  (one gate vector per branch; g = 1 without a gate). The compression is read
+  as the mean of each compressed block, and a query attends the compressed
+  blocks that lie entirely in its past.
 * Token reordering: 2025 review, section 11 (SpargeAttn), the token-reorder
   note - ordering tokens along a Hilbert curve raises the similarity of the
   tokens that share a block. The curve is the 3-D Hilbert curve over the
@@ -240,6 +247,18 @@ def linear_attention(q_rows: np.ndarray, s_state: np.ndarray, z_state: np.ndarra
     return (fq @ s_state) / (fq @ z_state)[:, None]
 
 
+def compress_kv(x: np.ndarray, n_valid: int, length: int, stride: int) -> np.ndarray:
+    """NSA compressed branch, token compression: compressed block c covers tokens
+    c*stride .. c*stride + length - 1 and exists while that range holds valid tokens only;
+    its key (value) is the mean of those tokens (the pages give no compression function;
+    the mean is the parameter-free reading, as for the pooled routing)."""
+    n_c = (n_valid - length) // stride + 1 if n_valid >= length else 0
+    out = np.zeros((n_c, x.shape[1]))
+    for c in range(n_c):
+        out[c] = x[c * stride:c * stride + length].mean(axis=0)
+    return out
+
+
 def combine(o_s: np.ndarray, o_l: np.ndarray, q_rows: np.ndarray,
             w_p: Optional[np.ndarray], w_g_head: Optional[np.ndarray]) -> np.ndarray:
     """O = O_s + g * (O_l W_p); W_p = I without projection, g = 1 without gate."""
@@ -275,12 +294,17 @@ class OracleCfg:
     cos_filter: int = 0  # pooled scores of key blocks with CosSim < cos_theta become -inf
     scale: float = 0.0
     cos_theta: float = 0.0
+    nsa_branches: int = 0  # top-n mode: compressed, selected and window branches, each its own softmax
+    cmp_block: int = 32    # compressed branch: tokens per compressed block ...
+    cmp_stride: int = 16   # ... and the stride between compressed blocks
 
-    OPTIONAL = ("proj_per_head", "smooth_k", "linear_all", "cos_filter", "cos_theta")
+    OPTIONAL = ("proj_per_head", "smooth_k", "linear_all", "cos_filter", "cos_theta", "nsa_branches",
+                "cmp_block", "cmp_stride")
+    DEFAULTS = {"cmp_block": 32, "cmp_stride": 16}
 
     @classmethod
     def of(cls, c) -> "OracleCfg":
-        return cls(**{f: getattr(c, f, 0) if f in cls.OPTIONAL else getattr(c, f)
+        return cls(**{f: getattr(c, f, cls.DEFAULTS.get(f, 0)) if f in cls.OPTIONAL else getattr(c, f)
                       for f in cls.__dataclass_fields__})
 
     @property
@@ -308,6 +332,7 @@ class Layer:
         self.w_p = w_p if c.has_proj else None
         if self.w_p is not None:
             assert self.w_p.shape == ((c.H, c.d, c.d) if c.proj_per_head else (c.d, c.d))
+        # w_g: [H, d] gate vectors; with NSA's branches [H, 3, d] (compressed, selected, window)
         self.w_g = w_g if c.has_gate else None
         self._kbar: Dict[Tuple[int, int], np.ndarray] = {}
         self._scores: Dict[Tuple[int, int], np.ndarray] = {}
@@ -415,12 +440,34 @@ class Layer:
             s = cand[None, :]
             in_sel = np.isin(s // c.block, np.asarray(sel, dtype=np.int64))
             in_win = (s > t - c.window) if c.window > 0 else np.zeros_like(in_sel)
-            allow = (s <= t) & (in_sel | in_win)
-            o_s = softmax_attention(qr, K[cand], V[cand], c.sm_scale, allow)
+            if not c.nsa_branches:
+                # one softmax over selected blocks and window together
+                allow = (s <= t) & (in_sel | in_win)
+                o_s = softmax_attention(qr, K[cand], V[cand], c.sm_scale, allow)
+                o = o_s
+            else:
+                # NSA's three branches, each its own softmax, combined with per-head gates
+                o_slc = softmax_attention(qr, K[cand], V[cand], c.sm_scale, (s <= t) & in_sel)
+                o_win = softmax_attention(qr, K[cand], V[cand], c.sm_scale, (s <= t) & in_win)
+                Kc, Vc = self.compressed(b, hk)
+                cidx = np.arange(Kc.shape[0])[None, :]
+                o_cmp = softmax_attention(qr, Kc, Vc, c.sm_scale,
+                                          cidx * c.cmp_stride + c.cmp_block - 1 <= t)
+                g = (sigmoid(qr @ self.w_g[h].T) if self.w_g is not None else np.ones((nv, 3)))
+                o = g[:, 0:1] * o_cmp + g[:, 1:2] * o_slc + g[:, 2:3] * o_win
+                o_s = o
             o_l = np.zeros_like(qr)
-            o = o_s
         O[:nv], O_s[:nv], O_l[:nv] = o, o_s, o_l
         return dict(O=O, O_s=O_s, O_l=O_l)
+
+    def compressed(self, b, hk):
+        """NSA compressed keys and values of KV head hk (cached)."""
+        key = ("cmp", b, hk)
+        if key not in self._states:
+            c = self.c
+            self._states[key] = (compress_kv(self.k[b, hk], c.N_valid, c.cmp_block, c.cmp_stride),
+                                 compress_kv(self.v[b, hk], c.N_valid, c.cmp_block, c.cmp_stride))
+        return self._states[key]
 
     # -- whole layer ----------------------------------------------------------
     def forward(self) -> Dict[str, np.ndarray]:

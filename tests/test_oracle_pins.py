@@ -654,3 +654,91 @@ def test_block_cos_sims_closed_forms():
     assert abs(sims[0] - 1.0) < 1e-15
     # block 1: e1, -e1, e1', e2 -> sum = (1, 1, 0, 0), |sum|^2 = 2, / 16
     assert abs(sims[1] - 2.0 / 16.0) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# NSA's three branches (top-n mode option)
+# ---------------------------------------------------------------------------
+
+def nsa_cfg(**kw):
+    base = dict(mode=1, causal=1, top_n=2, window=40, k_h=0, k_l=0, has_proj=0, has_gate=0, nsa_branches=1,
+                cmp_block=8, cmp_stride=4, N=256, N_valid=256, H=4, H_kv=2, d=16, block=32)
+    base.update(kw)
+    return Cfg(**base)
+
+
+def nsa_brute(c, q, k, v, w_g, sels):
+    """Element-mask brute force of the three branches: compressed keys through an explicit
+    pooling matrix, every branch by torch SDPA with its boolean mask."""
+    N, bl, nv = c.N, c.block, c.N_valid
+    n_c = (nv - c.cmp_block) // c.cmp_stride + 1 if nv >= c.cmp_block else 0
+    P = np.zeros((n_c, N))
+    for cc in range(n_c):
+        P[cc, cc * c.cmp_stride:cc * c.cmp_stride + c.cmp_block] = 1.0 / c.cmp_block
+    t = np.arange(N)[:, None]
+    s = np.arange(N)[None, :]
+    out = np.zeros((c.B, c.H, N, c.d))
+    for b in range(c.B):
+        for h in range(c.H):
+            hk = h // (c.H // c.H_kv)
+            selm = np.zeros((c.N // bl, c.N // bl), bool)
+            for i, row in enumerate(sels[b][hk]):
+                selm[i, np.asarray(row, dtype=np.int64)] = True
+            ok = (s <= t) & (s < nv)
+            m_slc = ok & selm[t // bl, s // bl]
+            m_win = ok & (s > t - c.window)
+            m_cmp = np.arange(n_c)[None, :] * c.cmp_stride + c.cmp_block - 1 <= t
+            Q, K, V = q[b, h], k[b, hk], v[b, hk]
+            o_slc = sdpa(Q, K, V, m_slc, scale_of(c))
+            o_win = sdpa(Q, K, V, m_win, scale_of(c))
+            o_cmp = sdpa(Q, P @ K, P @ V, m_cmp, scale_of(c)) if n_c else np.zeros_like(Q)
+            g = 1 / (1 + np.exp(-(Q @ w_g[h].T))) if c.has_gate else np.ones((N, 3))
+            o = g[:, :1] * o_cmp + g[:, 1:2] * o_slc + g[:, 2:3] * o_win
+            o[nv:] = 0
+            out[b, h] = o
+    return out
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(has_gate=1), dict(N_valid=241, has_gate=1),
+                                dict(cmp_block=32, cmp_stride=16, window=0, top_n=3),
+                                dict(top_n=0, window=64, cmp_block=16, cmp_stride=16)])
+def test_nsa_branches_match_elementwise_brute_force(kw):
+    c = nsa_cfg(**kw)
+    q, k, v, _, _ = rand_inputs(c, seed=31)
+    w_g = np.random.default_rng(32).normal(0, 0.5, (c.H, 3, c.d))
+    L = so.Layer(c, q, k, v, None, w_g)
+    sels = L.route()[0]
+    got = L.forward()["O"]
+    want = nsa_brute(c, q, k, v, w_g, sels)
+    assert np.abs(got - want).max() <= 1e-10
+
+
+def test_nsa_compressed_branch_with_unit_blocks_is_causal_attention():
+    """cmp_block = cmp_stride = 1: every token is its own compressed block, so the
+    compressed branch is dense causal attention (torch SDPA, causal mask)."""
+    c = nsa_cfg(top_n=0, window=0, cmp_block=1, cmp_stride=1, N_valid=250)
+    q, k, v, _, _ = rand_inputs(c, seed=33)
+    got = so.Layer(c, q, k, v).forward()["O"]
+    for h in range(c.H):
+        hk = h // (c.H // c.H_kv)
+        Q, K, V = (torch.from_numpy(np.ascontiguousarray(a[0, x][:c.N_valid])) for a, x in
+                   ((q, h), (k, hk), (v, hk)))
+        want = F.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=scale_of(c)).numpy()
+        assert np.abs(got[0, h, :c.N_valid] - want).max() <= 1e-12
+
+
+def test_nsa_zero_gates_halve_the_branch_sum():
+    c = nsa_cfg(has_gate=1)
+    q, k, v, _, _ = rand_inputs(c, seed=34)
+    half = so.Layer(c, q, k, v, None, np.zeros((c.H, 3, c.d))).forward()["O"]
+    c1 = nsa_cfg(has_gate=0)
+    full = so.Layer(c1, q, k, v).forward()["O"]
+    assert np.abs(half - 0.5 * full).max() <= 1e-12
+
+
+def test_compress_kv_means_and_ragged_tail():
+    x = np.arange(20.0).reshape(10, 2)
+    got = so.compress_kv(x, 9, 4, 2)  # blocks of 4 at stride 2 inside the 9 valid tokens
+    assert got.shape == (3, 2)
+    np.testing.assert_allclose(got[:, 0], [3.0, 7.0, 11.0])  # means of rows 0-3, 2-5, 4-7 (column 0 = 2 t)
+    assert so.compress_kv(x, 3, 4, 2).shape == (0, 2)
