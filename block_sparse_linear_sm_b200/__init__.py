@@ -33,7 +33,8 @@ class sla_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "H_kv", "N", "N_valid", "d", "block", "mode", "k_h", "k_l", "top_n",
                  "window", "causal", "has_proj", "proj_per_head", "has_gate", "smooth_k",
-                 "linear_all", "cos_filter")] + [("scale", ctypes.c_float), ("cos_theta", ctypes.c_float)]
+                 "linear_all", "cos_filter")] + [("scale", ctypes.c_float), ("cos_theta", ctypes.c_float)] + \
+        [(n, ctypes.c_int32) for n in ("nsa_branches", "cmp_block", "cmp_stride")]
 
 
 class SlaError(RuntimeError):

@@ -50,6 +50,11 @@ struct FlashTcParams {
   int npairs;           // units per (b, h) when pairing query blocks
   int words;            // 32-bit words of one block bitmap
   int list_cap;         // capacity of the merged list
+  // Keys: n_keys valid keys in nkt 64-key tiles. Key index c stands for token
+  // c * kstride + kspan in the causal test c * kstride + kspan <= t (1 and 0 for the
+  // token keys; NSA's compressed keys: the stride and length - 1 of a compressed block).
+  int n_keys, nkt, kstride, kspan;
+  int dense_tiles;      // top-n mode: every key tile up to the causal limit (no list)
   float scale_log2;
 };
 
@@ -190,12 +195,22 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     for (int e = tid; e < prm.len; e += kTcThreads) {
       const int j = lst[hf][e];
       if (TOPN && j < 0) continue;  // padding of short selections
-      if (j < 0 || j >= prm.nb || (TOPN && j >= i_h[hf])) {
+      if (j < 0 || j >= prm.nkt || (TOPN && j >= i_h[hf])) {
         report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
         continue;
       }
       atomicOr(&act[j >> 5], 1u << (j & 31));
       if (TOPN) atomicOr(&sel[j >> 5], 1u << (j & 31));
+    }
+    if (TOPN && prm.dense_tiles) {
+      // every key tile with a key some row of this query block may attend
+      const int last_t = i_h[hf] * kBlock + kBlock - 1 - prm.kspan;
+      int jmax = last_t < 0 ? -1 : last_t / prm.kstride / kBlock;
+      if (jmax > prm.nkt - 1) jmax = prm.nkt - 1;
+      for (int j = tid; j <= jmax; j += kTcThreads) {
+        atomicOr(&act[j >> 5], 1u << (j & 31));
+        atomicOr(&sel[j >> 5], 1u << (j & 31));
+      }
     }
     if (TOPN && prm.window > 0) {
       const int lo = i_h[hf] * kBlock - prm.window + 1;
@@ -454,14 +469,16 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           x[32 + j] = __uint_as_float(x1[j]);
         }
         const int k0 = jb * kBlock;
-        bool need_mask = k0 + kBlock > prm.n_valid;
-        if (TOPN) need_mask = need_mask || (k0 + kBlock - 1 > t_lo) || (!sel && k0 <= t_lo + 31 - prm.window);
+        bool need_mask = k0 + kBlock > prm.n_keys;
+        if (TOPN)
+          need_mask = need_mask || ((k0 + kBlock - 1) * prm.kstride + prm.kspan > t_lo) ||
+                      (!sel && k0 <= t_lo + 31 - prm.window);
         if (need_mask) {
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const int key = k0 + j;
-            bool keep = key < prm.n_valid;
-            if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
+            bool keep = key < prm.n_keys;
+            if (TOPN) keep = keep && key * prm.kstride + prm.kspan <= t && (sel || key > t - prm.window);
             x[j] = keep ? x[j] : -INFINITY;
           }
         }
@@ -645,14 +662,21 @@ static bool make_map(CUtensorMap* m, const void* base, int heads, int n_rows, in
                       (uint64_t)N * D * 2, 64, 64);
 }
 
+// branch 0: the layer's sparse branch. NSA's branches (top-n mode with nsa_branches), each
+// written to its own buffer: 1 compressed (keys: the compressed K, V; every tile up to the
+// causal limit), 2 selected (the selected blocks only), 3 window (the window only).
 template <int D, bool TOPN, bool FUSE>
-static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
+static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStream_t s) {
   using L = TcLayout<D>;
   const sla_config& c = p.c;
+  const bool cmp = branch == 1;
   CUtensorMap mq, mk, mv, ms;
+  const void* kb = cmp ? (const void*)(a.ws + p.off_kc) : (const void*)a.k;
+  const void* vb = cmp ? (const void*)(a.ws + p.off_vc) : (const void*)a.v;
+  const int key_rows = cmp ? (p.n_cmp > 0 ? p.n_cmp : 1) : c.N_valid, key_stride_rows = cmp ? p.ncmp_pad : c.N;
   if (!make_map(&mq, a.q, c.B * c.H, c.N_valid, c.N, D) ||
-      !make_map(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) ||
-      !make_map(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
+      !make_map(&mk, kb, c.B * c.H_kv, key_rows, key_stride_rows, D) ||
+      !make_map(&mv, vb, c.B * c.H_kv, key_rows, key_stride_rows, D))
     return cudaErrorInvalidValue;
   // phi(Q) from the pooling pass, same geometry as Q (fused epilogue); otherwise unused
   CUtensorMap mf;
@@ -664,24 +688,34 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   FlashTcParams prm;
   prm.list = a.crit;
-  prm.o = a.out;  // the sparse branch is the output, or the fused epilogue writes it
+  // the sparse branch is the output, or the fused epilogue writes it; NSA's branches
+  // each write their own buffer
+  prm.o = branch == 0 ? a.out
+                      : reinterpret_cast<__nv_bfloat16*>(a.ws + (branch == 1 ? p.off_oc : branch == 2 ? p.off_os
+                                                                                                   : p.off_ow));
   prm.zs = FUSE ? reinterpret_cast<const float*>(a.ws + p.off_zs) : nullptr;
   prm.gate = FUSE && c.has_gate ? reinterpret_cast<const float*>(a.ws + p.off_gate) : nullptr;
-  prm.lse = reinterpret_cast<float*>(a.ws + p.off_lse);
+  prm.lse = branch == 0 ? reinterpret_cast<float*>(a.ws + p.off_lse) : nullptr;
   prm.status = a.status;
   prm.H = c.H;
   prm.group = p.group;
   prm.N = c.N;
   prm.n_valid = c.N_valid;
   prm.nb = p.nkb;
-  prm.len = TOPN ? c.top_n : c.k_h;
-  prm.window = c.window;
+  prm.len = (branch == 1 || branch == 3) ? 0 : (TOPN ? c.top_n : c.k_h);
+  prm.window = (branch == 1 || branch == 2) ? 0 : c.window;
   prm.pair_heads = TOPN && (p.group % 2 == 0);
   prm.npairs = (p.nqb + 1) / 2;
-  prm.words = (p.nkb + 31) / 32;
+  prm.n_keys = cmp ? p.n_cmp : c.N_valid;
+  prm.nkt = cmp ? p.ncmp_pad / kBlock : p.nkb;
+  prm.kstride = cmp ? c.cmp_stride : 1;
+  prm.kspan = cmp ? c.cmp_block - 1 : 0;
+  prm.dense_tiles = cmp ? 1 : 0;
+  prm.words = (prm.nkt + 31) / 32;
   int per_half = prm.len;
-  if (TOPN) per_half += (c.window + 62) / kBlock + 2;
-  prm.list_cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
+  if (TOPN) per_half += (prm.window + 62) / kBlock + 2;
+  prm.list_cap = 2 * per_half < prm.nkt ? 2 * per_half : prm.nkt;
+  if (cmp) prm.list_cap = prm.nkt;
   if (prm.list_cap < 1) prm.list_cap = 1;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
   int smem = L::kOffList + prm.list_cap * 4;
@@ -705,11 +739,15 @@ cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s) {
   // the layer has a linear branch: marginal blocks, or every block with linear_all
   const bool fuse = !topn && (p.nkb - p.c.k_h - p.c.k_l > 0 || p.c.linear_all);
   if (p.c.d == 128) {
-    if (topn) return launch_tc<128, true, false>(p, a, s);
-    return fuse ? launch_tc<128, false, true>(p, a, s) : launch_tc<128, false, false>(p, a, s);
+    if (topn) return launch_tc<128, true, false>(p, a, 0, s);
+    return fuse ? launch_tc<128, false, true>(p, a, 0, s) : launch_tc<128, false, false>(p, a, 0, s);
   }
-  if (topn) return launch_tc<64, true, false>(p, a, s);
-  return fuse ? launch_tc<64, false, true>(p, a, s) : launch_tc<64, false, false>(p, a, s);
+  if (topn) return launch_tc<64, true, false>(p, a, 0, s);
+  return fuse ? launch_tc<64, false, true>(p, a, 0, s) : launch_tc<64, false, false>(p, a, 0, s);
+}
+
+cudaError_t launch_flash_nsa(const Plan& p, const Args& a, int branch, cudaStream_t s) {
+  return p.c.d == 128 ? launch_tc<128, true, false>(p, a, branch, s) : launch_tc<64, true, false>(p, a, branch, s);
 }
 
 }  // namespace sla

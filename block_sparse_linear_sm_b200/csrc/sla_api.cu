@@ -21,8 +21,10 @@ static sla_status check_config(const sla_config* c) {
   const int nb = c->N / c->block;
   if (nb > kMaxBlocks) return SLA_ERR_UNSUPPORTED;
   if ((int64_t)c->B * c->H * c->N * c->d > ((int64_t)1 << 40)) return SLA_ERR_UNSUPPORTED;
+  if (c->nsa_branches != 0 && c->nsa_branches != 1) return SLA_ERR_INVALID_ARG;
   if (c->mode == SLA_MODE_THREEWAY) {
     if (c->k_h < 0 || c->k_l < 0 || c->k_h + c->k_l > nb) return SLA_ERR_INVALID_ARG;
+    if (c->nsa_branches != 0) return SLA_ERR_UNSUPPORTED;
     if (c->causal != 0) return SLA_ERR_UNSUPPORTED;
     if ((c->has_proj != 0 && c->has_proj != 1) || (c->has_gate != 0 && c->has_gate != 1) ||
         (c->proj_per_head != 0 && c->proj_per_head != 1) || (c->smooth_k != 0 && c->smooth_k != 1) ||
@@ -32,9 +34,14 @@ static sla_status check_config(const sla_config* c) {
   } else if (c->mode == SLA_MODE_TOPN_WINDOW) {
     if (c->top_n < 0 || c->window < 0) return SLA_ERR_INVALID_ARG;
     if (c->causal != 1) return SLA_ERR_UNSUPPORTED;
-    if (c->has_proj != 0 || c->has_gate != 0 || c->proj_per_head != 0 || c->smooth_k != 0 ||
-        c->linear_all != 0)
+    if (c->has_proj != 0 || c->proj_per_head != 0 || c->smooth_k != 0 || c->linear_all != 0)
       return SLA_ERR_UNSUPPORTED;
+    if (c->has_gate != 0 && c->has_gate != 1) return SLA_ERR_INVALID_ARG;
+    if (c->has_gate && !c->nsa_branches) return SLA_ERR_UNSUPPORTED;  // gates belong to NSA's branches
+    if (c->nsa_branches) {
+      if (c->cmp_block < 1 || c->cmp_stride < 1) return SLA_ERR_INVALID_ARG;
+      if (c->cmp_block > 1024 || c->cmp_stride > 1024) return SLA_ERR_UNSUPPORTED;
+    }
     // selected blocks plus window blocks must fit the kernel's 128-entry list
     if (c->top_n > 64 || c->top_n + (c->window + 62) / kBlock + 1 > 128) return SLA_ERR_UNSUPPORTED;
   } else {
@@ -82,6 +89,16 @@ bool make_plan(const sla_config* c, Plan* p) {
   } else {
     p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
     p->off_lse = take(B * H * (size_t)c->N * 4);  // row log2-sum-exp of the sparse branch (backward)
+    if (c->nsa_branches) {
+      // compressed blocks that hold valid tokens only, padded to whole 64-key tiles
+      p->n_cmp = c->N_valid >= c->cmp_block ? (c->N_valid - c->cmp_block) / c->cmp_stride + 1 : 0;
+      p->ncmp_pad = (int)align_up((size_t)(p->n_cmp > 0 ? p->n_cmp : 1), 64);
+      p->off_kc = take(B * Hkv * (size_t)p->ncmp_pad * d * 2);
+      p->off_vc = take(B * Hkv * (size_t)p->ncmp_pad * d * 2);
+      p->off_oc = take(B * H * (size_t)c->N * d * 2);
+      p->off_os = take(B * H * (size_t)c->N * d * 2);
+      p->off_ow = take(B * H * (size_t)c->N * d * 2);
+    }
   }
   p->total = off;
   return true;
@@ -92,7 +109,9 @@ static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 static bool has_marginal(const Plan& p) { return p.nkb - p.c.k_h - p.c.k_l > 0 || p.c.linear_all; }
 
 // Stage list of a configuration.
-enum Stage { kPool, kScores, kClassify, kSelect, kState, kAggregate, kFlash };
+enum Stage { kPool, kScores, kClassify, kSelect, kState, kAggregate, kFlash, kCompress, kFlashCmp, kFlashSlc,
+             kFlashWin, kCombine };
+constexpr int kMaxStages = 12;
 
 static int stages_of(const Plan& p, Stage* out) {
   int n = 0;
@@ -107,7 +126,15 @@ static int stages_of(const Plan& p, Stage* out) {
     out[n++] = kFlash;  // with a linear branch its tail runs the layer's epilogue
   } else {
     out[n++] = kSelect;
-    out[n++] = kFlash;
+    if (p.c.nsa_branches) {  // NSA's three branches, then the gated sum
+      out[n++] = kCompress;
+      out[n++] = kFlashCmp;
+      out[n++] = kFlashSlc;
+      out[n++] = kFlashWin;
+      out[n++] = kCombine;
+    } else {
+      out[n++] = kFlash;
+    }
   }
   return n;
 }
@@ -121,6 +148,11 @@ static const char* stage_name(Stage s) {
     case kState: return "linear_state";
     case kAggregate: return "linear_aggregate";
     case kFlash: return "sparse_flash";
+    case kCompress: return "compress_kv";
+    case kFlashCmp: return "sparse_flash_cmp";
+    case kFlashSlc: return "sparse_flash_slc";
+    case kFlashWin: return "sparse_flash_win";
+    case kCombine: return "branch_combine";
   }
   return "?";
 }
@@ -134,6 +166,11 @@ static cudaError_t run_stage(Stage st, const Plan& p, const Args& a, cudaStream_
     case kState: return launch_state(p, a, s);
     case kAggregate: return launch_aggregate(p, a, s);
     case kFlash: return launch_flash(p, a, s);
+    case kCompress: return launch_compress(p, a, s);
+    case kFlashCmp: return launch_flash_nsa(p, a, 1, s);
+    case kFlashSlc: return launch_flash_nsa(p, a, 2, s);
+    case kFlashWin: return launch_flash_nsa(p, a, 3, s);
+    case kCombine: return launch_branch_combine(p, a, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -151,9 +188,9 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
     return SLA_ERR_INVALID_ARG;
   const bool threeway = cfg->mode == SLA_MODE_THREEWAY;
   if (threeway && cfg->has_proj && (!w_p || !aligned(w_p, 16))) return SLA_ERR_INVALID_ARG;
-  if (threeway && cfg->has_gate && (!w_g || !aligned(w_g, 16))) return SLA_ERR_INVALID_ARG;
+  if (cfg->has_gate && (!w_g || !aligned(w_g, 16))) return SLA_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return SLA_ERR_WORKSPACE;
-  Stage stages[8];
+  Stage stages[kMaxStages];
   const int ns = stages_of(p, stages);
   if (events && n_events != ns + 1) return SLA_ERR_INVALID_ARG;
 
@@ -183,7 +220,11 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
 // ---------------------------------------------------------------------------
 // backward pass
 // ---------------------------------------------------------------------------
-static sla_status check_bwd_config(const sla_config* c) { return check_config(c); }
+static sla_status check_bwd_config(const sla_config* c) {
+  const sla_status st = check_config(c);
+  if (st != SLA_OK) return st;
+  return c->nsa_branches ? SLA_ERR_UNSUPPORTED : SLA_OK;  // NSA's branches: forward only
+}
 
 bool make_bwd_plan(const Plan& p, BwdPlan* b) {
   memset(b, 0, sizeof(*b));
@@ -383,14 +424,14 @@ sla_status sla_forward_timed(const void* q, const void* k, const void* v, const 
 int32_t sla_num_stages(const sla_config* cfg) {
   Plan p;
   if (!make_plan(cfg, &p)) return -1;
-  Stage st[8];
+  Stage st[kMaxStages];
   return stages_of(p, st);
 }
 
 const char* sla_stage_name(const sla_config* cfg, int32_t s) {
   Plan p;
   if (!make_plan(cfg, &p)) return nullptr;
-  Stage st[8];
+  Stage st[kMaxStages];
   const int n = stages_of(p, st);
   return (s >= 0 && s < n) ? stage_name(st[s]) : nullptr;
 }

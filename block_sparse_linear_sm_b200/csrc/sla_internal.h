@@ -33,6 +33,10 @@ struct Plan {
   // byte offsets into ws
   size_t off_status, off_qbar, off_kbar, off_scores, off_kflag, off_crit, off_neg, off_mmask, off_hs, off_ss,
       off_zs, off_phiq, off_gate, off_kmean, off_lse, total;
+  // NSA's branches (top-n mode): compressed K, V [B*H_kv][ncmp_pad][d] and the three
+  // branch outputs [B*H][N][d] (bf16)
+  int n_cmp, ncmp_pad;
+  size_t off_kc, off_vc, off_oc, off_os, off_ow;
 };
 
 bool make_plan(const sla_config* c, Plan* p);
@@ -66,6 +70,9 @@ cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_state(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_flash_nsa(const Plan& p, const Args& a, int branch, cudaStream_t s);  // 1 cmp, 2 slc, 3 win
+cudaError_t launch_compress(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_branch_combine(const Plan& p, const Args& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // backward pass (three-way mode)

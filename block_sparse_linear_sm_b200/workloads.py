@@ -63,6 +63,9 @@ class LayerConfig:
     cos_filter: int = 0           # 1: key blocks with CosSim < cos_theta score -inf
     scale: float = 0.0            # 0 -> 1/sqrt(d)
     cos_theta: float = 0.0
+    nsa_branches: int = 0         # top-n mode: NSA's compressed, selected and window branches
+    cmp_block: int = 32           # NSA compressed blocks: tokens per block ...
+    cmp_stride: int = 16          # ... and stride
     generator: str = "iid"        # iid | fourier | block_shift
     grid: Optional[tuple] = None  # (t, h, w) for the Fourier generator
     seed: int = 0
@@ -116,6 +119,11 @@ def _preset(name: str) -> LayerConfig:
         return LayerConfig(name, 1, 64, 4, 65536, 65536, 128, mode=MODE_TOPN_WINDOW,
                            top_n=16, window=512, causal=1, has_proj=0, has_gate=0,
                            generator="block_shift", seed=1004)
+    if name == "nsa_branches":
+        # NSA's three parallel branches on the NSA-shaped layer: compressed blocks of 32
+        # tokens at stride 16, the top-16 selected blocks and the 512-token window, gated
+        return _preset("nsa_causal").replace(name=name, nsa_branches=1, cmp_block=32, cmp_stride=16,
+                                             has_gate=1)
     if name == "wan1.3b_opensource":
         # the SLA critique page's reading of the open-source code: smooth-K and the
         # linear branch over all tokens, on the Wan2.1-1.3B layer's inputs
@@ -132,7 +140,8 @@ def _preset(name: str) -> LayerConfig:
     raise KeyError(name)
 
 
-PRESETS = ("tiny", "wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource", "wan1.3b_cosfilter")
+PRESETS = ("tiny", "wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource", "wan1.3b_cosfilter",
+           "nsa_branches")
 
 
 def preset(name: str) -> LayerConfig:
@@ -237,7 +246,9 @@ def generate(cfg: LayerConfig, v_shift: float = 0.0) -> LayerInputs:
     wrng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(cfg.seed).spawn(4)[3]))
     wp_shape = (H, d, d) if cfg.proj_per_head else (d, d)
     w_p = to_bf16_bits(wrng.normal(0.0, 1.0 / math.sqrt(d), size=wp_shape)) if cfg.has_proj else None
-    w_g = to_bf16_bits(wrng.normal(0.0, 1.0 / math.sqrt(d), size=(H, d))) if cfg.has_gate else None
+    # gate vectors: one per head, or one per head and NSA branch (compressed, selected, window)
+    wg_shape = (H, 3, d) if getattr(cfg, "nsa_branches", 0) else (H, d)
+    w_g = to_bf16_bits(wrng.normal(0.0, 1.0 / math.sqrt(d), size=wg_shape)) if cfg.has_gate else None
     return LayerInputs(cfg, q, k, v, w_p, w_g)
 
 

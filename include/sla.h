@@ -46,7 +46,8 @@
  *     k, v bf16 [B, H_kv, N, d]
  *     w_p  bf16 [d, d]   (row vector times matrix: O_l W_p), ignored unless has_proj;
  *          [H, d, d] with proj_per_head (head h uses w_p[h])
- *     w_g  bf16 [H, d]   ignored unless has_gate
+ *     w_g  bf16 [H, d]   ignored unless has_gate; [H, 3, d] with nsa_branches
+ *          (gates of the compressed, selected and window branches)
  *     out  bf16 [B, H, N, d]
  *   Tokens at index >= N_valid are padding: they are left out of pooling,
  *   attention and the linear states, and their output rows are written as 0.
@@ -113,7 +114,8 @@ typedef struct {
                           * 1 = one per query head, w_p [H, d, d]; needs H_kv == H (the
                           * projection is folded into per-KV-head states), else
                           * SLA_ERR_UNSUPPORTED */
-  int32_t has_gate; /* THREEWAY: 1 = g = sigmoid(q . w_g[h]), 0 = g = 1 */
+  int32_t has_gate; /* THREEWAY: 1 = g = sigmoid(q . w_g[h]), 0 = g = 1; TOPN_WINDOW: only
+                     * with nsa_branches (the branch gates) */
   int32_t smooth_k; /* THREEWAY: 1 = the linear branch uses K minus the mean of the head's
                      * valid key tokens (smooth-K, zero-mean K); routing and the sparse
                      * branch are unchanged by it (each row shifts by a constant) */
@@ -125,6 +127,16 @@ typedef struct {
                        * they rank last and get probability 0 in the top-n softmax */
   float scale;      /* softmax scale of pooled scores and attention; 0 = 1/sqrt(d) */
   float cos_theta;  /* CosSim threshold of cos_filter */
+  int32_t nsa_branches; /* TOPN_WINDOW: 1 = NSA's three parallel branches (sparse attention
+                         * survey, section 2): compressed, selected and window, each its
+                         * own softmax, summed with gates g_b = sigmoid(q . w_g[h][b])
+                         * (w_g bf16 [H, 3, d] with has_gate, else g_b = 1); 0 = one
+                         * softmax over the selected blocks and the window together */
+  int32_t cmp_block;  /* nsa_branches: tokens per compressed block (NSA: 32); compressed
+                       * block c is the mean of tokens c*cmp_stride .. + cmp_block - 1
+                       * (all valid) and query t attends it when c*cmp_stride + cmp_block
+                       * - 1 <= t */
+  int32_t cmp_stride; /* nsa_branches: stride between compressed blocks (NSA: 16) */
 } sla_config;
 
 /* Checks a configuration without touching any pointer. */

@@ -250,3 +250,18 @@ def test_backward_scratch_grows_with_the_problem():
     small = wl.small_config(N=1024, N_valid=1024, has_gate=1)
     big = wl.small_config(N=4096, N_valid=4096, has_gate=1)
     assert sla.sla_backward_workspace_bytes(big) > 2 * sla.sla_backward_workspace_bytes(small)
+
+
+def test_nsa_branches_configuration():
+    c = wl.preset("nsa_branches")
+    assert sla.sla_validate_config(c) == sla.SLA_OK
+    assert sla.sla_stage_names(c) == ["pool", "pooled_scores", "select_topn", "compress_kv", "sparse_flash_cmp",
+                                      "sparse_flash_slc", "sparse_flash_win", "branch_combine"]
+    # the three branch outputs and the compressed keys add to the workspace
+    assert sla.sla_workspace_bytes(c) > sla.sla_workspace_bytes(wl.preset("nsa_causal"))
+    # forward only; the gates belong to NSA's branches; no branches in the three-way mode
+    assert sla.sla_backward_workspace_bytes(c) == 0
+    assert sla.sla_validate_config(wl.preset("nsa_causal").replace(has_gate=1)) == sla.SLA_ERR_UNSUPPORTED
+    assert sla.sla_validate_config(wl.preset("wan1.3b").replace(nsa_branches=1)) == sla.SLA_ERR_UNSUPPORTED
+    assert sla.sla_validate_config(c.replace(cmp_stride=0)) == sla.SLA_ERR_INVALID_ARG
+    assert sla.sla_validate_config(c.replace(nsa_branches=2)) == sla.SLA_ERR_INVALID_ARG

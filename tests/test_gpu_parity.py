@@ -63,6 +63,24 @@ SMALL_CASES = [
 ]
 
 
+NSA = dict(mode=wl.MODE_TOPN_WINDOW, causal=1, k_h=0, k_l=0, has_proj=0, nsa_branches=1)
+NSA_CASES = [
+    dict(name="nsa_gqa_gates_d128", N=2048, N_valid=2048, d=128, H=4, H_kv=2, top_n=4, window=256,
+         cmp_block=32, cmp_stride=16, has_gate=1, **NSA),
+    dict(name="nsa_odd_group_ragged_d64", N=1536, N_valid=1500, d=64, H=3, H_kv=1, top_n=3, window=100,
+         cmp_block=32, cmp_stride=16, has_gate=0, **NSA),
+    dict(name="nsa_unit_cmp_d128", N=1024, N_valid=1000, d=128, H=2, H_kv=2, top_n=2, window=64,
+         cmp_block=1, cmp_stride=1, has_gate=1, **NSA),
+    dict(name="nsa_wide_blocks_d64", N=2048, N_valid=2048, d=64, H=4, H_kv=1, top_n=2, window=0,
+         cmp_block=64, cmp_stride=48, has_gate=1, **NSA),
+]
+
+
+@pytest.mark.parametrize("kw", NSA_CASES, ids=[c["name"] for c in NSA_CASES])
+def test_nsa_branches_small_layer_matches_oracle(kw):
+    run_and_check_full(small(**kw))
+
+
 @pytest.mark.parametrize("kw", SMALL_CASES, ids=[c["name"] for c in SMALL_CASES])
 def test_small_layer_matches_oracle(kw):
     run_and_check_full(small(**kw))
@@ -231,7 +249,7 @@ def sampled_units(cfg, n=12, seed=0):
 
 
 @pytest.mark.parametrize("name", ["wan1.3b", "salad", "nsa_causal", "wan14b", "wan1.3b_opensource",
-                                  "wan1.3b_cosfilter"])
+                                  "wan1.3b_cosfilter", "nsa_branches"])
 def test_full_size_workload(name):
     cfg = wl.preset(name)
     run = GpuRun(cfg)
