@@ -80,6 +80,26 @@ def stage_model(c: wl.LayerConfig) -> dict:
                 t = i * c.block + r
                 pairs += min(c.window, t + 1) + c.block * min(c.top_n, i)
         m["sparse_flash"] = ("tensor", 4.0 * d * B * H * pairs)
+        if getattr(c, "nsa_branches", 0):
+            # NSA's branches: the selected blocks and the window each alone, and the
+            # compressed keys up to the causal limit (c * stride + length - 1 <= t)
+            slc = win = cmp_pairs = 0.0
+            n_cmp = (Nv - c.cmp_block) // c.cmp_stride + 1 if Nv >= c.cmp_block else 0
+            for i in range(nb):
+                for r in range(c.block):
+                    t = i * c.block + r
+                    slc += c.block * min(c.top_n, i)
+                    win += min(c.window, t + 1)
+                    cmp_pairs += min(n_cmp, max(0, (t - c.cmp_block + 1) // c.cmp_stride + 1))
+            kc_bytes = 2 * B * Hkv * n_cmp * d * bf
+            del m["sparse_flash"]
+            # reads K, V (each token lies in cmp_block / cmp_stride blocks), writes the compressed rows
+            m["compress_kv"] = ("hbm", 2 * B * Hkv * Nv * d * bf + kc_bytes)
+            m["sparse_flash_cmp"] = ("tensor", 4.0 * d * B * H * cmp_pairs)
+            m["sparse_flash_slc"] = ("tensor", 4.0 * d * B * H * slc)
+            m["sparse_flash_win"] = ("tensor", 4.0 * d * B * H * win)
+            # reads q and the three branch outputs, writes O
+            m["branch_combine"] = ("hbm", 5 * B * H * Nv * d * bf)
     return m
 
 
@@ -548,7 +568,7 @@ def main():
 
     peaks = load_peaks()
     backward = None
-    if not args.no_backward:
+    if not args.no_backward and not cfg.nsa_branches:  # NSA's branches: forward only
         backward = measure_backward(sla, torch, cfg, q, k, v, w_p, w_g, out, ws, args.steps, args.warmup,
                                     dist, dev, stream, peaks)
         barrier()
@@ -561,7 +581,8 @@ def main():
         reorder["frac"] = reorder["achieved"] / peaks["hbm"]
     stages = stage_entries(names, stage_ms, stage_model(cfg), peaks)
     dom = max(names, key=lambda n: stage_ms[n])
-    kernel_of = {"sparse_flash": "flash_tc_kernel"}
+    kernel_of = {"sparse_flash": "flash_tc_kernel", "sparse_flash_cmp": "flash_tc_kernel",
+                 "sparse_flash_slc": "flash_tc_kernel", "sparse_flash_win": "flash_tc_kernel"}
     dk = stages[dom]
     if dk["bound"] == "tensor":
         # The layer's kernels run a few ms at a time at full SM clock (see "clocks"),
