@@ -82,7 +82,10 @@ struct TcLayout {
 // phi(Q) (tmF, written by the pooling pass) into the Q tiles; num = phi(Q) S'_i
 // goes to the freed S columns of TMEM (one query block at a time) and
 // O = O_s + g * num / (phi(q) . Z_i) is written to the output.
-template <int D, bool TOPN, bool FUSE>
+// KMAP (NSA's compressed branch only): key c stands for token c * kstride + kspan in the causal
+// test, and the key tiles are every tile up to the causal limit (dense_tiles); compiled
+// separately so that the plain top-n kernel keeps its registers.
+template <int D, bool TOPN, bool FUSE, bool KMAP>
 __global__ void __launch_bounds__(kTcThreads, 2)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
@@ -202,7 +205,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       atomicOr(&act[j >> 5], 1u << (j & 31));
       if (TOPN) atomicOr(&sel[j >> 5], 1u << (j & 31));
     }
-    if (TOPN && prm.dense_tiles) {
+    if (TOPN && KMAP && prm.dense_tiles) {
       // every key tile with a key some row of this query block may attend
       const int last_t = i_h[hf] * kBlock + kBlock - 1 - prm.kspan;
       int jmax = last_t < 0 ? -1 : last_t / prm.kstride / kBlock;
@@ -470,15 +473,19 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
         const int k0 = jb * kBlock;
         bool need_mask = k0 + kBlock > prm.n_keys;
-        if (TOPN)
-          need_mask = need_mask || ((k0 + kBlock - 1) * prm.kstride + prm.kspan > t_lo) ||
-                      (!sel && k0 <= t_lo + 31 - prm.window);
+        if (TOPN && KMAP)  // compressed keys: every tile counts as selected, no window
+          need_mask = need_mask || (k0 + kBlock - 1) * prm.kstride + prm.kspan > t_lo;
+        else if (TOPN)
+          need_mask = need_mask || (k0 + kBlock - 1 > t_lo) || (!sel && k0 <= t_lo + 31 - prm.window);
         if (need_mask) {
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const int key = k0 + j;
             bool keep = key < prm.n_keys;
-            if (TOPN) keep = keep && key * prm.kstride + prm.kspan <= t && (sel || key > t - prm.window);
+            if (TOPN && KMAP)
+              keep = keep && key * prm.kstride + prm.kspan <= t;
+            else if (TOPN)
+              keep = keep && key <= t && (sel || key > t - prm.window);
             x[j] = keep ? x[j] : -INFINITY;
           }
         }
@@ -665,7 +672,7 @@ static bool make_map(CUtensorMap* m, const void* base, int heads, int n_rows, in
 // branch 0: the layer's sparse branch. NSA's branches (top-n mode with nsa_branches), each
 // written to its own buffer: 1 compressed (keys: the compressed K, V; every tile up to the
 // causal limit), 2 selected (the selected blocks only), 3 window (the window only).
-template <int D, bool TOPN, bool FUSE>
+template <int D, bool TOPN, bool FUSE, bool KMAP = false>
 static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStream_t s) {
   using L = TcLayout<D>;
   const sla_config& c = p.c;
@@ -722,7 +729,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
   if (4 * prm.words * 4 > kSlots * L::kSlotBytes) return cudaErrorInvalidValue;  // bitmaps in the ring
   // at most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN, FUSE>,
+  cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN, FUSE, KMAP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int units;
@@ -730,7 +737,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
     units = c.B * c.H_kv * p.nqb * (p.group / 2);
   else
     units = c.B * c.H * prm.npairs;
-  flash_tc_kernel<D, TOPN, FUSE><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, mf, prm);
+  flash_tc_kernel<D, TOPN, FUSE, KMAP><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, mf, prm);
   return cudaGetLastError();
 }
 
@@ -747,6 +754,9 @@ cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s) {
 }
 
 cudaError_t launch_flash_nsa(const Plan& p, const Args& a, int branch, cudaStream_t s) {
+  if (branch == 1)  // compressed keys: the key-to-token map and the dense tile range
+    return p.c.d == 128 ? launch_tc<128, true, false, true>(p, a, branch, s)
+                        : launch_tc<64, true, false, true>(p, a, branch, s);
   return p.c.d == 128 ? launch_tc<128, true, false>(p, a, branch, s) : launch_tc<64, true, false>(p, a, branch, s);
 }
 
