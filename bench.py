@@ -332,6 +332,24 @@ def measured_traffic(kernel: str, workload: str):
     return None
 
 
+def route_lists(sla, torch, cfg, q, k, dev):
+    """The routing's block lists of the whole layer on the host (three-way: critical lists
+    [B, H, nqb, k_h]; top-n: selected lists [B, H_kv, nqb, top_n]); None without lists."""
+    topn = cfg.mode == wl.MODE_TOPN_WINDOW
+    rows, n = (cfg.H_kv, cfg.top_n) if topn else (cfg.H, cfg.k_h)
+    if n == 0:
+        return None
+    crit = torch.empty((cfg.B, rows, cfg.nqb, n), dtype=torch.int32, device=dev)
+    neg = None if topn or cfg.k_l == 0 else torch.empty((cfg.B, cfg.H, cfg.nqb, cfg.k_l), dtype=torch.int32,
+                                                        device=dev)
+    ws = torch.empty(sla.sla_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    sla.sla_route(q, k, cfg, None, crit, neg, ws)
+    st, detail = sla.sla_check_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"routing device status {st} detail {detail}")
+    return crit.cpu().numpy()
+
+
 def max_over_ranks(dist, device, *vals):
     """The max of each value over all ranks (one all-reduce); the values themselves
     without a process group."""
@@ -400,6 +418,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--clocks-csv", default=None)
     ap.add_argument("--no-backward", action="store_true", help="skip the sla_backward measurement")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="heads: each rank runs its KV groups of one layer (LPT on the routed tiles)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads (H = H_kv; small profiler captures)")
     args = ap.parse_args()
@@ -434,6 +454,21 @@ def main():
         return None if bits is None else torch.from_numpy(bits).view(torch.bfloat16).to(dev)
 
     q, k, v, w_p, w_g = up(x.q), up(x.k), up(x.v), up(x.w_p), up(x.w_g)
+    full_cfg, shard_info = cfg, None
+    if args.shard == "heads":
+        # one layer split over the ranks by KV group: route it whole, estimate each group's
+        # work from its routed tiles, balance (LPT), and run this rank's heads
+        from block_sparse_linear_sm_b200 import sharding as sh
+        costs = sh.unit_costs(cfg, route_lists(sla, torch, cfg, q, k, dev))
+        shard = sh.HeadShard(cfg, world, rank, costs)
+        if not shard.units:
+            raise RuntimeError("more ranks than KV groups")
+        q, k, v, w_p, w_g = shard.inputs(q, k, v, w_p, w_g)
+        cfg = shard.local
+        loads = sh.plan_loads(costs, shard.plan)
+        shard_info = {"plan": shard.plan, "estimated_loads": loads,
+                      "imbalance": max(loads) / (sum(loads) / len(loads)),
+                      "what": "KV groups per rank, LPT on the tiles the routing makes the flash kernel run"}
     out = torch.empty(cfg.B, cfg.H, cfg.N, cfg.d, dtype=torch.bfloat16, device=dev)
     ws = torch.empty(sla.sla_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -539,9 +574,12 @@ def main():
                 for i, n in enumerate(names)}
 
     # end to end: pinned host inputs -> device, layer, output -> host
-    hq = torch.from_numpy(x.q).view(torch.bfloat16).pin_memory()
-    hk = torch.from_numpy(x.k).view(torch.bfloat16).pin_memory()
-    hv = torch.from_numpy(x.v).view(torch.bfloat16).pin_memory()
+    if shard_info is None:
+        hq = torch.from_numpy(x.q).view(torch.bfloat16).pin_memory()
+        hk = torch.from_numpy(x.k).view(torch.bfloat16).pin_memory()
+        hv = torch.from_numpy(x.v).view(torch.bfloat16).pin_memory()
+    else:  # this rank's heads
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = hout.numel() * 2
@@ -574,6 +612,9 @@ def main():
         barrier()
 
     flops = cfg.dense_flops()
+    if shard_info is not None:
+        # strong scaling: the ranks share one layer's work
+        flops = full_cfg.dense_flops() / world
     value = job_throughput(world, flops, ms_step)
     e2e_value = job_throughput(world, flops, e2e_ms)
 
@@ -610,11 +651,12 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "H_kv": cfg.H_kv, "N": cfg.N,
-                   "N_valid": cfg.N_valid, "d": cfg.d, "k_h": cfg.k_h, "k_l": cfg.k_l,
-                   "has_proj": cfg.has_proj, "has_gate": cfg.has_gate,
-                   "parallelism": f"replicas x{world}",
+        "scaling": "weak" if shard_info is None else "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": full_cfg.name, "B": full_cfg.B, "H": full_cfg.H, "H_kv": full_cfg.H_kv,
+                   "N": full_cfg.N, "N_valid": full_cfg.N_valid, "d": full_cfg.d, "k_h": full_cfg.k_h,
+                   "k_l": full_cfg.k_l, "has_proj": full_cfg.has_proj, "has_gate": full_cfg.has_gate,
+                   "parallelism": f"replicas x{world}" if shard_info is None else f"heads x{world}",
                    "l2": f"inputs (Q,K,V {(cfg.B * (cfg.H + 2 * cfg.H_kv) * cfg.N * cfg.d * 2) / 1e6:.0f} MB) larger "
                          "than the 126 MB L2; no flush"},
         "ms_per_layer": ms_step,
@@ -623,6 +665,7 @@ def main():
         "ms_per_step_eager": ms_eager,
         "launch": "CUDA graph replay of one captured sla_forward call (ms_per_step_eager: direct calls)",
         "roofline": roof,
+        "head_shard": shard_info,
         "token_reorder": reorder,
         "stages": stages,
         "backward": backward,
@@ -633,11 +676,11 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of float64 oracle work on the host cores
-        units = sample_units(cfg, 512, n_heads=4)
-        t, n = oracle_sample(cfg, x, units, budget_s=20.0)
-        cv = (n / units_total(cfg)) * flops / t / 1e12
+        units = sample_units(full_cfg, 512, n_heads=4)
+        t, n = oracle_sample(full_cfg, x, units, budget_s=20.0)
+        cv = (n / units_total(full_cfg)) * full_cfg.dense_flops() / t / 1e12
         line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                                "sample": f"{n} (head, query block) units of {units_total(cfg)} from "
+                                "sample": f"{n} (head, query block) units of {units_total(full_cfg)} from "
                                           f"4 heads in {t:.1f} s (stops after 20 s); throughput "
                                           f"scaled by unit count"}
     if dist is not None:

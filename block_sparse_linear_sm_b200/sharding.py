@@ -1,0 +1,148 @@
+"""Head-sharded multi-GPU layer with load balancing on the routed work.
+
+Sparse attention survey, db-SP note: when a dynamic block mask is spread over
+several GPUs, splitting the tokens (or the heads) evenly does not split the
+sparse work evenly, so the partition should balance the effective blocks each
+device executes (db-SP partitions at the head level and the block level).
+
+This module does the head level. The unit is a KV group: a KV head and the
+query heads that read it, since they share K, V and (top-n mode) the selection.
+Each unit's cost is estimated from the routing as the 64-key tiles the sparse
+flash kernel executes for it (pairs of query blocks share one merged block
+list) plus the linear branch's fixed per-head work; units go to ranks by
+longest-processing-time-first (LPT). Each rank gathers its heads into
+contiguous local tensors, runs the whole layer on them through the C ABI, and
+the outputs can be all-gathered back into head order. Nothing here computes
+any part of the layer: the layer runs in the CUDA kernels of libsla.so.
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence
+
+import numpy as np
+
+from . import workloads as wl
+
+
+def unit_costs(cfg: wl.LayerConfig, crit: Optional[np.ndarray] = None) -> np.ndarray:
+    """Estimated work per KV group, in 64 x 64 flash tiles (float64 [H_kv]).
+
+    ``crit``: the routing's block lists as host int32, three-way mode [B, H, nqb, k_h]
+    (critical blocks), top-n mode [B, H_kv, nqb, top_n] (selected, -1 padded). Without
+    routing every unit costs the same.
+    """
+    c = cfg
+    group = c.H // c.H_kv
+    if crit is None:
+        return np.ones(c.H_kv)
+    nqb = c.nqb
+    cost = np.zeros(c.H_kv)
+    if c.mode == wl.MODE_THREEWAY:
+        for b in range(c.B):
+            for h in range(c.H):
+                tiles = 0
+                for p in range(0, nqb, 2):
+                    rows = crit[b, h, p:p + 2].reshape(-1)
+                    tiles += np.unique(rows[rows >= 0]).size  # merged list of the pair
+                # the linear branch's per-head work, as tiles of the same FLOP: state and
+                # aggregation ~ 2 * nqb * nkb * d^2 against 4 * 64^2 * d per tile
+                marg = nqb - c.k_h - c.k_l > 0 or c.linear_all
+                lin = (2.0 * nqb * c.nkb * c.d * c.d) / (4.0 * 64 * 64 * c.d) if marg else 0.0
+                cost[h // group] += tiles + lin
+    else:
+        wb = (c.window + 62) // 64 + 1 if c.window > 0 else 0  # blocks the window reaches
+        for b in range(c.B):
+            for hk in range(c.H_kv):
+                tiles = 0
+                for i in range(nqb):
+                    sel = crit[b, hk, i]
+                    tiles += np.unique(sel[sel >= 0]).size + min(wb, i + 1)
+                cost[hk] += tiles * group  # every query head of the group runs the tiles
+    return cost
+
+
+def balance(costs: Sequence[float], world: int) -> List[List[int]]:
+    """LPT assignment: units by decreasing cost, each to the least-loaded rank (ties: the
+    lower unit index first, then the lower rank). Deterministic, so every rank computes
+    the same plan. Returns the ascending unit lists of the ranks."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    order = sorted(range(len(costs)), key=lambda u: (-float(costs[u]), u))
+    loads = [0.0] * world
+    plan: List[List[int]] = [[] for _ in range(world)]
+    for u in order:
+        r = min(range(world), key=lambda x: (loads[x], x))
+        plan[r].append(u)
+        loads[r] += float(costs[u])
+    return [sorted(p) for p in plan]
+
+
+def plan_loads(costs: Sequence[float], plan: List[List[int]]) -> List[float]:
+    return [float(sum(costs[u] for u in p)) for p in plan]
+
+
+def query_heads(cfg: wl.LayerConfig, units: Sequence[int]) -> List[int]:
+    """The query heads of the given KV groups, in order."""
+    group = cfg.H // cfg.H_kv
+    return [u * group + g for u in units for g in range(group)]
+
+
+def local_config(cfg: wl.LayerConfig, units: Sequence[int]) -> wl.LayerConfig:
+    """The layer restricted to the given KV groups (same sequence, routing and options)."""
+    group = cfg.H // cfg.H_kv
+    return cfg.replace(name=f"{cfg.name}_heads{len(units) * group}", H=len(units) * group, H_kv=len(units))
+
+
+def gather_heads(x, heads: Sequence[int]):
+    """Contiguous copy of heads ``heads`` (dimension 1) of a [B, H, ...] tensor."""
+    import torch
+
+    idx = torch.as_tensor(list(heads), dtype=torch.long, device=x.device)
+    return torch.index_select(x, 1, idx).contiguous()
+
+
+def all_gather_heads(local_out, cfg: wl.LayerConfig, plan: List[List[int]], rank: int, dist):
+    """Every rank's local output [B, H_local, N, d] back into the full [B, H, N, d], in head
+    order, on every rank (one all_gather of equally padded blocks)."""
+    import torch
+
+    group = cfg.H // cfg.H_kv
+    max_heads = max(len(p) for p in plan) * group
+    B, hl, N, d = local_out.shape
+    pad = torch.zeros((B, max_heads, N, d), dtype=local_out.dtype, device=local_out.device)
+    pad[:, :hl] = local_out
+    parts = [torch.empty_like(pad) for _ in plan]
+    dist.all_gather(parts, pad)
+    full = torch.empty((B, cfg.H, N, d), dtype=local_out.dtype, device=local_out.device)
+    for r, units in enumerate(plan):
+        heads = query_heads(cfg, units)
+        if heads:
+            full[:, heads] = parts[r][:, :len(heads)]
+    return full
+
+
+class HeadShard:
+    """This rank's share of a head-sharded layer: its KV groups, the local configuration,
+    and the layer run on its gathered heads through the C ABI."""
+
+    def __init__(self, cfg: wl.LayerConfig, world: int, rank: int, costs: Optional[np.ndarray] = None):
+        self.cfg = cfg
+        self.costs = unit_costs(cfg) if costs is None else np.asarray(costs, dtype=np.float64)
+        self.plan = balance(self.costs, world)
+        self.units = self.plan[rank]
+        self.heads = query_heads(cfg, self.units)
+        self.local = local_config(cfg, self.units) if self.units else None
+
+    def inputs(self, q, k, v, w_p=None, w_g=None):
+        """Local q, k, v (and per-head parameters) for this rank's heads."""
+        import torch
+
+        c = self.cfg
+        lq, lk, lv = gather_heads(q, self.heads), gather_heads(k, self.units), gather_heads(v, self.units)
+        lwp = w_p
+        if w_p is not None and c.proj_per_head:
+            lwp = torch.index_select(w_p, 0, torch.as_tensor(self.heads, device=w_p.device)).contiguous()
+        lwg = None
+        if w_g is not None:
+            lwg = torch.index_select(w_g, 0, torch.as_tensor(self.heads, device=w_g.device)).contiguous()
+        return lq, lk, lv, lwp, lwg

@@ -10,6 +10,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch.multiprocessing as mp
 
@@ -76,3 +77,85 @@ def test_reference_arm_runs_on_rank_zero_only():
                        capture_output=True, text=True, env=env, timeout=110)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+# ---------------------------------------------------------------------------
+# head-sharded layer: planning and the all-gather back into head order
+# ---------------------------------------------------------------------------
+
+def test_balance_is_deterministic_and_covers_every_unit():
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+
+    costs = [5.0, 1.0, 4.0, 4.0, 3.0, 2.0, 2.0, 1.0, 6.0, 3.0, 1.0, 1.0]
+    for world in (1, 2, 3, 5, 8, 12, 16):
+        plan = sh.balance(costs, world)
+        assert plan == sh.balance(costs, world)
+        assert sorted(u for p in plan for u in p) == list(range(len(costs)))
+        loads = sh.plan_loads(costs, plan)
+        # LPT bound: the largest load is at most the mean plus the largest single cost
+        assert max(loads) <= sum(costs) / world + max(costs) + 1e-9
+    # uneven costs: LPT beats assigning units round-robin
+    assert max(sh.plan_loads(costs, sh.balance(costs, 4))) == 9.0
+    rr = [[u for u in range(12) if u % 4 == r] for r in range(4)]
+    assert max(sh.plan_loads(costs, rr)) > 9.0
+
+
+def test_unit_costs_count_the_merged_tiles():
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+
+    c = wl.small_config(N=256, N_valid=256, H=2, H_kv=1, k_h=2, k_l=2, has_proj=1)  # 4 blocks, no marginal
+    crit = np.zeros((1, 2, 4, 2), np.int32)
+    crit[0, 0] = [[0, 1], [0, 1], [2, 3], [0, 3]]  # pairs: {0,1} -> 2 tiles, {0,2,3} -> 3
+    crit[0, 1] = [[0, 1], [2, 3], [0, 1], [0, 1]]  # {0,1,2,3} -> 4, {0,1} -> 2
+    assert sh.unit_costs(c, crit).tolist() == [2 + 3 + 4 + 2]
+    assert sh.unit_costs(c).tolist() == [1.0]
+
+
+def _shard_rank_main(rank, world, port, q):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = wl.small_config(N=128, N_valid=128, H=6, H_kv=3, d=8)
+        shard = sh.HeadShard(cfg, world, rank, costs=np.array([3.0, 1.0, 2.0]))
+        x = torch.arange(cfg.B * cfg.H * cfg.N * cfg.d, dtype=torch.float32).reshape(cfg.B, cfg.H, cfg.N, cfg.d)
+        kv = torch.arange(cfg.B * cfg.H_kv * cfg.N * cfg.d, dtype=torch.float32).reshape(
+            cfg.B, cfg.H_kv, cfg.N, cfg.d)
+        lq, lk, lv, _, _ = shard.inputs(x, kv, kv)
+        # stand-in for the layer's output: a function of each local row that remembers its head
+        local_out = lq * 2 + 1
+        full = sh.all_gather_heads(local_out, cfg, shard.plan, rank, dist)
+        ok = bool(torch.equal(full, x * 2 + 1)) and lk.shape[1] == len(shard.units)
+        dist.barrier()
+        q.put((rank, (shard.plan, ok)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_head_sharded_gather_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=100) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # costs [3, 1, 2]: rank 0 takes unit 0, rank 1 units 1 and 2; both ranks agree
+    assert res[0][0] == res[1][0] == [[0], [1, 2]]
+    assert res[0][1] and res[1][1]
