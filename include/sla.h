@@ -139,7 +139,13 @@ typedef struct {
   int32_t cmp_stride; /* nsa_branches: stride between compressed blocks (NSA: 16) */
 } sla_config;
 
-/* Checks a configuration without touching any pointer. */
+/*
+ * Checks a configuration without touching any pointer.
+ * Sizes: B, H, H_kv, N and d must be >= 1; an empty problem (any of them 0) is
+ * SLA_ERR_INVALID_ARG, not a no-op. Limits of the kernels (SLA_ERR_UNSUPPORTED
+ * beyond them): N / block <= 4096 key blocks (N <= 262144 tokens, the routing
+ * sort's row length) and B * H * N * d <= 2^40 elements.
+ */
 SLA_API sla_status sla_validate_config(const sla_config* cfg);
 
 /* Bytes of device workspace that sla_route / sla_forward need for cfg

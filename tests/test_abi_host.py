@@ -73,7 +73,21 @@ BAD = [
     (dict(mode=1, causal=1, top_n=4, has_proj=0, proj_per_head=1), sla.SLA_ERR_UNSUPPORTED),
     (dict(scale=-1.0), sla.SLA_ERR_INVALID_ARG),
     (dict(scale=float("nan")), sla.SLA_ERR_INVALID_ARG),
+    # empty problems are rejected, not treated as no-ops
+    (dict(B=0), sla.SLA_ERR_INVALID_ARG),
+    (dict(H=0, H_kv=0), sla.SLA_ERR_INVALID_ARG),
+    (dict(N=0, N_valid=0), sla.SLA_ERR_INVALID_ARG),
+    (dict(N_valid=0, N=64, k_h=1, k_l=0), sla.SLA_ERR_INVALID_ARG),
+    # one key block past the routing sort's limit of 4096
+    (dict(N=4097 * 64, N_valid=4097 * 64, k_h=4, k_l=4), sla.SLA_ERR_UNSUPPORTED),
 ]
+
+
+def test_largest_block_count_is_accepted():
+    """N = 4096 blocks of 64 (262144 tokens) is the largest supported length."""
+    c = wl.small_config(N=4096 * 64, N_valid=4096 * 64 - 5, k_h=40, k_l=400)
+    assert sla.sla_validate_config(c) == sla.SLA_OK
+    assert sla.sla_workspace_bytes(c) > 0
 
 
 @pytest.mark.parametrize("kw,code", BAD)

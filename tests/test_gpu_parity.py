@@ -260,3 +260,19 @@ def test_full_size_workload(name):
     err = unit_errors(run, L, sampled_units(cfg))
     print(name, "sampled output error", err)
     assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err
+
+
+def test_longest_supported_sequence():
+    """4096 key blocks (262144 tokens, the routing sort's row limit) with a ragged tail:
+    full routing bit-exact except near-tie rows, sampled blocks of the output."""
+    cfg = small(name="max_blocks", N=4096 * 64, N_valid=4096 * 64 - 7, d=64, H=2, H_kv=1,
+                k_h=16, k_l=64, has_gate=1)
+    run = GpuRun(cfg)
+    L = run.layer()
+    rep = check_routing(run, L)
+    print(cfg.name, "routing", rep)
+    assert rep["mismatched_rows"] == 0, rep
+    assert rep["tie_rows"] < rep["rows"] // 4, rep
+    err = unit_errors(run, L, sampled_units(cfg, n=6))
+    print(cfg.name, "sampled output error", err)
+    assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err
