@@ -37,6 +37,12 @@ METRIC = "ms/layer & dense-equiv TFLOP/s, sparse+linear attn N=32K d=128 95% spa
 UNIT = "dense-equiv TFLOP/s"
 
 
+# float64 mma.sync (m8n8k4) throughput of this machine's B200, TFLOP/s: a register-only loop of
+# independent products on all 148 SMs gave 36.7 / 37.0 / 37.1 at 8 / 16 / 32 warps per SM
+# (64 FMA per SM per clock at 1965 MHz). The peak of the pooled-scores stage.
+FP64_MMA_TFLOPS = 37.0
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -51,7 +57,8 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 
 def stage_model(c: wl.LayerConfig) -> dict:
-    """Per stage: ("tensor", FLOP) or ("hbm", bytes) of algorithmic work per launch."""
+    """Per stage: ("tensor", bf16 FLOP), ("fp64", FLOP) or ("hbm", bytes) of algorithmic work
+    per launch."""
     B, H, Hkv, N, Nv, d = c.B, c.H, c.H_kv, c.N, c.N_valid, c.d
     nb = c.nqb
     bf = 2
@@ -60,7 +67,10 @@ def stage_model(c: wl.LayerConfig) -> dict:
     if c.mode == wl.MODE_THREEWAY and nb - c.k_h - c.k_l > 0:
         # phi(Q) (bf16) and, with a gate, g_t (fp32) for the linear branch
         m["pool"] = ("hbm", m["pool"][1] + B * H * Nv * d * bf + (B * H * Nv * 4 if c.has_gate else 0))
-    m["pooled_scores"] = ("hbm", (B * H + B * Hkv) * nb * d * 8 + B * H * nb * nb * 8)
+    # float64 products q_bar . k_bar on the FP64 tensor path (mma.sync m8n8k4): every (i, j)
+    # in three-way mode, the candidates j < i in top-n mode
+    pairs = nb * nb if c.mode == wl.MODE_THREEWAY else nb * (nb - 1) // 2
+    m["pooled_scores"] = ("fp64", 2.0 * B * H * pairs * d)
     if c.mode == wl.MODE_THREEWAY:
         marg = nb - c.k_h - c.k_l
         m["classify"] = ("hbm", B * H * nb * nb * 8 + B * H * nb * nb * (1 + (2 if marg else 0))
@@ -148,6 +158,10 @@ def stage_entries(names, stage_ms, model, peaks):
             ach = work / t / 1e12
             out[n] = {"ms": stage_ms[n], "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
                       "frac": ach / peaks["bf16"], "frac_of_sustained": ach / peaks["bf16_sus"], "work": work}
+        elif kind == "fp64":
+            ach = work / t / 1e12
+            out[n] = {"ms": stage_ms[n], "bound": "fp64", "achieved": ach, "unit": "TFLOP/s",
+                      "frac": ach / FP64_MMA_TFLOPS, "peak_kind": "fp64 mma.sync, measured", "work": work}
         else:
             ach = work / t / 1e9
             out[n] = {"ms": stage_ms[n], "bound": "hbm", "achieved": ach, "unit": "GB/s",
@@ -635,6 +649,9 @@ def main():
                 "peak_sustained": peaks["bf16_sus"], "frac_of_sustained": dk["achieved"] / peaks["bf16_sus"],
                 "traffic": measured_traffic(kernel_of.get(dom, dom), cfg.name),
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"}
+    elif dk["bound"] == "fp64":
+        roof = {"kernel": dom, "bound": "fp64", "achieved": dk["achieved"], "peak": FP64_MMA_TFLOPS,
+                "unit": "TFLOP/s", "frac": dk["frac"], "peak_kind": dk["peak_kind"], "traffic": None}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved"], "peak": peaks["hbm"],
                 "unit": "GB/s", "frac": dk["achieved"] / peaks["hbm"],
