@@ -42,7 +42,9 @@ def topn_selection(run):
             for b in range(m.shape[0])]
 
 
-def run_backward(cfg, seed=3, v_shift=0.0):
+def run_backward(cfg, seed=3, v_shift=0.0, keep=None):
+    """Relative Frobenius error per gradient tensor; ``keep`` (a dict) receives the GPU's
+    gradients ("got") and the oracle's ("ref")."""
     x = wl.generate(cfg, v_shift=v_shift)
     run = GpuRun(cfg, x, route=False)
     c = cfg
@@ -81,6 +83,8 @@ def run_backward(cfg, seed=3, v_shift=0.0):
     # padding rows of the gradients are zero
     for key in ("dq", "dk", "dv"):
         assert np.all(got[key][:, :, c.N_valid:] == 0), key
+    if keep is not None:
+        keep.update(got=got, ref=ref, x=x, dout=wl.bf16_bits_to_f64(dob))
     return errs
 
 
@@ -131,6 +135,33 @@ def test_backward_linear_branch_with_shifted_values():
     errs = run_backward(small(name="marg_shift", N=1024, N_valid=1024, d=128, k_h=0, k_l=0, has_gate=1),
                         v_shift=3.0)
     assert all(e <= REL for e in errs.values()), errs
+
+
+def test_backward_smooth_k_mean_term():
+    """All blocks marginal with smooth-K. The linear branch's dk is G - colsum(G) / N_valid
+    (G: the gradient with respect to k - m), so its column sum over the valid rows is exactly
+    0. The mean term is only about 1 % of dk, below the per-tensor bar, so it is checked
+    through that column sum: the GPU's must be far below colsum(G), the value it would have
+    without the term."""
+    c = small(name="smooth_all_marg", N=1024, N_valid=1000, d=64, k_h=0, k_l=0, smooth_k=1, has_gate=1)
+    keep = {}
+    errs = run_backward(c, keep=keep)
+    assert all(e <= REL for e in errs.values()), errs
+    nv = c.N_valid
+    x = keep["x"]
+    k = x.f64("k")
+    k_c = k.copy()
+    k_c[:, :, :nv] -= k[:, :, :nv].mean(axis=2, keepdims=True)
+    # G from the oracle on the centred keys with smooth-K off (the routing is unchanged)
+    g = sla_grad.layer_grads(c.replace(smooth_k=0), x.f64("q"), k_c, x.f64("v"), x.f64("w_p"),
+                             x.f64("w_g"), keep["dout"])["dk"]
+    col_g = g[:, :, :nv].sum(axis=2)
+    col_ref = keep["ref"]["dk"][:, :, :nv].sum(axis=2)
+    col_got = keep["got"]["dk"][:, :, :nv].sum(axis=2)
+    assert np.linalg.norm(col_ref) <= 1e-9 * np.linalg.norm(col_g)
+    ratio = np.linalg.norm(col_got - col_ref) / np.linalg.norm(col_g)
+    print("smooth-K column-sum ratio", ratio)
+    assert ratio <= 0.1, ratio
 
 
 def test_backward_all_negligible_is_zero():
