@@ -24,6 +24,13 @@ N x N token grid (tiny and small shapes only):
   with smooth-K: O_l = (phi(Q) phi(K)^T . M) V / rowsum(phi(Q) phi(K)^T . M);
   a row with no such token gives 0.
 * O = O_s + g * (O_l W_p), g = sigmoid(q . w_g[h]); padding rows are 0.
+* Top-n mode: O = O_s under the element mask (selected blocks or window,
+  causal). With NSA's branches (sparse attention survey, section 2, NSA's three
+  parallel branches): O = sum_b g_b o_b over the compressed branch (attention
+  over the block means of cmp_block tokens at cmp_stride, C = A K and A V with
+  A the averaging matrix, causal at the block's last token), the selected
+  branch and the window branch, each its own softmax, g_b = sigmoid(q .
+  w_g[h][b]) or 1.
 
 ``torch.autograd`` then differentiates L = sum(O * dO). The restatement is
 pinned against ``sla_oracle`` (the same forward values) and its gradients
@@ -62,17 +69,51 @@ def _masked_softmax_attention(q, k, v, allow, scale):
                        torch.zeros_like(q[:, :v.shape[1]]))
 
 
-def _topn_allow(c, sel_rows) -> torch.Tensor:
+def _topn_allow(c, sel_rows, part: str = "union") -> torch.Tensor:
     """[N, N] bool, top-n mode: query t attends key s when s <= t, s is valid, and s's
-    block is selected for t's block or s > t - window."""
+    block is selected for t's block or s > t - window (``part`` "union"); NSA's selected
+    branch keeps only the first condition ("sel"), its window branch only the second
+    ("win")."""
     N, bl, nv = c.N, c.block, c.N_valid
     selm = np.zeros((c.nb, c.nb), dtype=bool)
     for i, row in enumerate(sel_rows):
         selm[i, np.asarray(row, dtype=np.int64)] = True
     t = np.arange(N)[:, None]
     s = np.arange(N)[None, :]
+    in_sel = selm[t // bl, s // bl]
     in_win = (s > t - c.window) if c.window > 0 else np.zeros((N, N), dtype=bool)
-    return torch.from_numpy((s <= t) & (s < nv) & (selm[t // bl, s // bl] | in_win))
+    allowed = {"union": in_sel | in_win, "sel": in_sel, "win": in_win}[part]
+    return torch.from_numpy((s <= t) & (s < nv) & allowed)
+
+
+def _compression(c):
+    """NSA's compressed branch as a linear map: the [n_c, N] matrix whose row c averages
+    tokens c*stride .. c*stride + length - 1 (compressed blocks of valid tokens only), and
+    the [N, n_c] causal mask (query t attends block c when c*stride + length - 1 <= t)."""
+    length, stride, nv = c.cmp_block, c.cmp_stride, c.N_valid
+    n_c = (nv - length) // stride + 1 if nv >= length else 0
+    m = np.zeros((n_c, c.N))
+    for j in range(n_c):
+        m[j, j * stride:j * stride + length] = 1.0 / length
+    t = np.arange(c.N)[:, None]
+    allow = np.arange(n_c)[None, :] * stride + length - 1 <= t
+    return torch.from_numpy(m), torch.from_numpy(allow)
+
+
+def _nsa_head(c, qh, kh, vh, sel_rows, w_g_head):
+    """NSA's three branches for one query head: compressed, selected and window attention,
+    each its own softmax, summed with the gates sigmoid(q . w_g[h][b]) (1 without gates)."""
+    mc, allow_c = _compression(c)
+    if mc.shape[0] > 0:
+        o_cmp = _masked_softmax_attention(qh, mc @ kh, mc @ vh, allow_c, c.sm_scale)
+    else:
+        o_cmp = torch.zeros_like(qh)
+    o_slc = _masked_softmax_attention(qh, kh, vh, _topn_allow(c, sel_rows, "sel"), c.sm_scale)
+    o_win = _masked_softmax_attention(qh, kh, vh, _topn_allow(c, sel_rows, "win"), c.sm_scale)
+    if w_g_head is not None:
+        g = torch.sigmoid(qh @ w_g_head.T)  # [N, 3]: compressed, selected, window
+        return g[:, 0:1] * o_cmp + g[:, 1:2] * o_slc + g[:, 2:3] * o_win
+    return o_cmp + o_slc + o_win
 
 
 def layer_forward_torch(cfg, q, k, v, w_p=None, w_g=None, classes=None):
@@ -80,7 +121,8 @@ def layer_forward_torch(cfg, q, k, v, w_p=None, w_g=None, classes=None):
 
     ``classes`` fixes the routing (default: ``sla_oracle``'s own): the three-way
     classes [B, H, nqb, nkb], or in the top-n mode the selected lists
-    [B][H_kv][nqb] (the top-n mode has no linear branch: O = O_s).
+    [B][H_kv][nqb] (the top-n mode has no linear branch: O = O_s, or with NSA's
+    branches the gated sum of the compressed, selected and window attentions).
     """
     c = so.OracleCfg.of(cfg)
     if classes is None:
@@ -94,8 +136,12 @@ def layer_forward_torch(cfg, q, k, v, w_p=None, w_g=None, classes=None):
             heads = []
             for h in range(c.H):
                 hk = h // c.group
-                o = _masked_softmax_attention(q[b, h], k[b, hk], v[b, hk], _topn_allow(c, classes[b][hk]),
-                                              c.sm_scale)
+                if c.nsa_branches:
+                    o = _nsa_head(c, q[b, h], k[b, hk], v[b, hk], classes[b][hk],
+                                  w_g[h] if c.has_gate and w_g is not None else None)
+                else:
+                    o = _masked_softmax_attention(q[b, h], k[b, hk], v[b, hk],
+                                                  _topn_allow(c, classes[b][hk]), c.sm_scale)
                 row_ok = (torch.arange(c.N) < c.N_valid)[:, None]
                 heads.append(torch.where(row_ok, o, torch.zeros_like(o)))
             out.append(torch.stack(heads))
@@ -141,13 +187,13 @@ def layer_grads(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, w_p: Optional[
     ``classes``: as for ``layer_forward_torch``.
 
     Returns dq, dk, dv ([B, H(_kv), N, d]), dw_p (shape of w_p or None), dw_g
-    ([H, d] or None) and O.
+    ([H, d]; [H, 3, d] with NSA's branches; or None) and O.
     """
     c = so.OracleCfg.of(cfg)
     t = lambda a: None if a is None else torch.tensor(a, dtype=torch.float64, requires_grad=True)
     tq, tk, tv = t(q), t(k), t(v)
     twp = t(w_p) if c.has_proj and c.mode == 0 else None
-    twg = t(w_g) if c.has_gate and c.mode == 0 else None
+    twg = t(w_g) if c.has_gate and (c.mode == 0 or c.nsa_branches) else None
     if classes is None:
         classes = so.Layer(cfg, q, k, v, w_p, w_g).route()[0]
     o = layer_forward_torch(cfg, tq, tk, tv, twp, twg, classes)

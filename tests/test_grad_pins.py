@@ -8,7 +8,8 @@ differentiate it. It is pinned against things other than itself:
 * with every block critical they equal the textbook gradients of dense softmax
   attention (dV = P^T dO, dS = P * (dP - rowsum(dO * O)), dQ = dS K s, dK = dS^T Q s);
 * with every block negligible they are zero.
-A planted mistake (a gradient that ignores the gate) fails the finite-difference pin.
+Planted mistakes (a gradient that ignores the gate; NSA's compressed keys taken as
+constants) fail the finite-difference pin.
 The block-by-block chain rule (``block_grads``, used on sampled blocks of
 full-size layers) is pinned against autograd on every block of small layers.
 """
@@ -40,7 +41,7 @@ def inputs(c, seed=0):
         x[:, :, c.N_valid:] = 0  # padding tokens are zero
     shape_p = (c.H, c.d, c.d) if c.proj_per_head else (c.d, c.d)
     w_p = rng.normal(0, 1 / math.sqrt(c.d), shape_p)
-    w_g = rng.normal(0, 1 / math.sqrt(c.d), (c.H, c.d))
+    w_g = rng.normal(0, 1 / math.sqrt(c.d), (c.H, 3, c.d) if getattr(c, "nsa_branches", 0) else (c.H, c.d))
     d_out = rng.standard_normal((c.B, c.H, c.N, c.d))
     return q, k, v, w_p, w_g, d_out
 
@@ -73,6 +74,12 @@ CASES = {
                             H=4, H_kv=2),
     "topn_ragged": dict(mode=1, causal=1, top_n=2, window=20, k_h=0, k_l=0, has_proj=0, has_gate=0,
                         N=160, N_valid=150),
+    # NSA's three branches: compressed blocks overlapping (length 16, stride 8), gates, GQA
+    "nsa_gates_gqa": dict(mode=1, causal=1, top_n=1, window=40, k_h=0, k_l=0, has_proj=0, has_gate=1,
+                          H=4, H_kv=2, nsa_branches=1, cmp_block=16, cmp_stride=8),
+    # ragged tail (the last compressed block ends before it), no gates, length 24 / stride 20
+    "nsa_ragged": dict(mode=1, causal=1, top_n=2, window=20, k_h=0, k_l=0, has_proj=0, has_gate=0,
+                       N=160, N_valid=150, nsa_branches=1, cmp_block=24, cmp_stride=20),
 }
 
 
@@ -93,7 +100,7 @@ def _fd_check(c, grads_fn, seed=5, eps=1e-6, rel=1e-6):
     g = grads_fn(c, q, k, v, w_p, w_g, d_out, classes)
     rng = np.random.default_rng(seed + 100)
     names = ["q", "k", "v"] + (["w_p"] if c.has_proj and c.mode == 0 else []) + \
-        (["w_g"] if c.has_gate and c.mode == 0 else [])
+        (["w_g"] if c.has_gate and (c.mode == 0 or getattr(c, "nsa_branches", 0)) else [])
     worst = {}
     for name in names:
         args = dict(q=q, k=k, v=v, w_p=w_p, w_g=w_g)
@@ -155,6 +162,23 @@ def test_planted_gate_without_gradient_is_caught(monkeypatch):
     monkeypatch.setattr(sg.torch, "sigmoid", lambda x: real(x).detach())
     worst = _fd_check(c, lambda c, *a: sg.layer_grads(c, *a[:6], classes=a[6]))
     assert max(worst.values()) > 1e-3
+
+
+def test_planted_compressed_branch_without_key_gradient_is_caught(monkeypatch):
+    """NSA: a gradient that treats the compressed keys and values as constants (no path
+    back through the block means to K and V) fails the finite-difference pin on dk / dv."""
+    c = Cfg(**CASES["nsa_gates_gqa"])
+    real = sg._masked_softmax_attention
+
+    def planted(q, k, v, allow, scale):
+        if k.shape[0] != c.N:  # the compressed branch: n_c block means instead of N tokens
+            k, v = k.detach(), v.detach()
+        return real(q, k, v, allow, scale)
+
+    monkeypatch.setattr(sg, "_masked_softmax_attention", planted)
+    worst = _fd_check(c, lambda c, *a: sg.layer_grads(c, *a[:6], classes=a[6]))
+    assert worst["k"] > 1e-3 and worst["v"] > 1e-3, worst
+    assert worst["q"] < 1e-6, worst
 
 
 BLOCK_CASES = {
