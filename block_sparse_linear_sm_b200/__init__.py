@@ -94,6 +94,10 @@ def lib() -> ctypes.CDLL:
         L.sla_status_string.restype = ctypes.c_char_p
         L.sla_version.argtypes = []
         L.sla_version.restype = ctypes.c_char_p
+        L.sla_forward_host_device_bytes.argtypes = [C, I32]
+        L.sla_forward_host_device_bytes.restype = S
+        L.sla_forward_host.argtypes = [P, P, P, P, P, C, P, I32, P, S, P, P, P]
+        L.sla_forward_host.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -190,6 +194,35 @@ def sla_forward_timed(q, k, v, w_p, w_g, c, out, mask_out, ws, events, stream=No
                                    ctypes.byref(cfg), _ptr(out), _ptr(mask_out), _ptr(ws),
                                    ws_bytes, _stream(stream), arr, len(events)),
            "sla_forward_timed")
+
+
+def _host_ptr(x) -> Optional[int]:
+    if isinstance(x, int):
+        return x
+    if x.is_cuda:
+        raise ValueError("tensor must live in host memory")
+    if not x.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return x.data_ptr()
+
+
+def sla_forward_host_device_bytes(c, n_chunks: int) -> int:
+    cfg = _cfg(c)
+    return int(lib().sla_forward_host_device_bytes(ctypes.byref(cfg), n_chunks))
+
+
+def sla_forward_host(q_host, k_host, v_host, w_p, w_g, c, out_host, n_chunks, dev, stream=None,
+                     h2d_stream=None, d2h_stream=None) -> None:
+    """The layer on host tensors (q/k/v/out in host memory, ideally pinned; w_p, w_g and the
+    arena ``dev`` of sla_forward_host_device_bytes(c, n_chunks) bytes on the device)."""
+    cfg = _cfg(c)
+    dev_bytes = dev.numel() * dev.element_size()
+    s = _stream(stream)
+    _check(lib().sla_forward_host(_host_ptr(q_host), _host_ptr(k_host), _host_ptr(v_host), _ptr(w_p),
+                                  _ptr(w_g), ctypes.byref(cfg), _host_ptr(out_host), n_chunks, _ptr(dev),
+                                  dev_bytes, s, s if h2d_stream is None else _stream(h2d_stream),
+                                  s if d2h_stream is None else _stream(d2h_stream)),
+           "sla_forward_host")
 
 
 def sla_backward_workspace_bytes(c) -> int:

@@ -204,6 +204,49 @@ SLA_API const char* sla_stage_name(const sla_config* cfg, int32_t s);
 SLA_API sla_status sla_check_device_status(void* ws, void* stream, int32_t* detail);
 
 /*
+ * The layer on HOST buffers (the pages have no counterpart: this is the call a
+ * user with activations in host memory makes). q_host, k_host and v_host are
+ * read from host memory and out_host is written there, in the layouts of
+ * sla_forward. Host memory should be page-locked: pageable memory also works,
+ * but its copies do not overlap anything.
+ *
+ * Pipelining: the layer is cut into B * n_chunks units, one batch entry and
+ * H_kv / n_chunks KV heads each, with their query heads. Every head's result
+ * is independent of the others, so a unit's output is bit-identical to the
+ * same rows of one sla_forward call. The inputs of all units are copied in on
+ * h2d_stream in order. Each unit runs sla_forward on `stream` as soon as its
+ * inputs have arrived, and its output is copied out on d2h_stream as soon as
+ * it is done. So the copies of later units overlap the kernels of earlier
+ * ones, and the two copy directions overlap each other.
+ *
+ * w_p and w_g are DEVICE pointers (resident parameters, layouts of
+ * sla_forward; NULL unless has_proj / has_gate).
+ *
+ * dev is a caller-owned device arena of sla_forward_host_device_bytes(cfg,
+ * n_chunks) bytes, 256-byte aligned. It holds a status word at offset 0,
+ * device copies of q, k, v and out, and one sla_forward workspace per unit.
+ * sla_check_device_status(dev, stream, ...) reports the first device-side
+ * error of any unit.
+ *
+ * Ordering: the call's copies start after the work queued on `stream` before
+ * the call, and `stream` waits for the last copy out before any later work.
+ * So completion of `stream` means out_host is written, and back-to-back calls
+ * on the same arena do not race. Distinct non-default streams give the
+ * overlap; passing the same stream three times is correct but serial. The
+ * call creates and releases its own CUDA events and allocates no memory.
+ *
+ * Errors: SLA_ERR_INVALID_ARG for a bad configuration, n_chunks < 1 or not
+ * dividing H_kv, or a NULL or misaligned (16 bytes) pointer;
+ * SLA_ERR_WORKSPACE for a NULL, misaligned or short arena; SLA_ERR_CUDA if
+ * a copy, event or launch fails. All checks run before the first copy.
+ */
+SLA_API size_t sla_forward_host_device_bytes(const sla_config* cfg, int32_t n_chunks);
+SLA_API sla_status sla_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                                    const void* w_p, const void* w_g, const sla_config* cfg,
+                                    void* out_host, int32_t n_chunks, void* dev, size_t dev_bytes,
+                                    void* stream, void* h2d_stream, void* d2h_stream);
+
+/*
  * Failure-detection self-test (the pages have no counterpart). Clears the
  * status word at the start of `ws` (any buffer of at least 256 bytes,
  * 256-byte aligned) and launches one small kernel that waits, through the

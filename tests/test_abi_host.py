@@ -122,6 +122,43 @@ def test_forward_rejects_bad_pointers_before_launch():
     assert _call_forward(bad) == sla.SLA_ERR_UNSUPPORTED
 
 
+def _call_forward_host(cfg, n_chunks=2, q=16, k=16, v=16, w_p=16, w_g=16, out=16, dev=256, dev_bytes=None):
+    c = sla.make_config(cfg)
+    if dev_bytes is None:
+        dev_bytes = sla.sla_forward_host_device_bytes(cfg, n_chunks)
+    return sla.lib().sla_forward_host(q, k, v, w_p, w_g, ctypes.byref(c), out, n_chunks, dev, dev_bytes,
+                                      None, None, None)
+
+
+def test_forward_host_rejects_bad_arguments_before_any_copy():
+    cfg = wl.small_config(N=1024, N_valid=1024, H=4, H_kv=2, has_gate=1)
+    # fake (never dereferenced) addresses: every case fails validation on the host
+    assert _call_forward_host(cfg, n_chunks=0) == sla.SLA_ERR_INVALID_ARG
+    assert _call_forward_host(cfg, n_chunks=3) == sla.SLA_ERR_INVALID_ARG   # does not divide H_kv
+    assert _call_forward_host(cfg, q=None) == sla.SLA_ERR_INVALID_ARG
+    assert _call_forward_host(cfg, out=None) == sla.SLA_ERR_INVALID_ARG
+    assert _call_forward_host(cfg, v=40) == sla.SLA_ERR_INVALID_ARG        # misaligned
+    assert _call_forward_host(cfg, w_p=None) == sla.SLA_ERR_INVALID_ARG    # has_proj
+    assert _call_forward_host(cfg, w_g=None) == sla.SLA_ERR_INVALID_ARG    # has_gate
+    assert _call_forward_host(cfg, dev=None) == sla.SLA_ERR_WORKSPACE
+    assert _call_forward_host(cfg, dev=128) == sla.SLA_ERR_WORKSPACE       # misaligned
+    need = sla.sla_forward_host_device_bytes(cfg, 2)
+    assert _call_forward_host(cfg, dev_bytes=need - 1) == sla.SLA_ERR_WORKSPACE
+    assert _call_forward_host(wl.small_config(N=1024, N_valid=1024, d=80)) == sla.SLA_ERR_UNSUPPORTED
+
+
+def test_forward_host_arena_holds_io_and_one_workspace_per_unit():
+    cfg = wl.small_config(B=2, N=1024, N_valid=1000, H=4, H_kv=2, has_gate=1)
+    assert sla.sla_forward_host_device_bytes(cfg, 0) == 0
+    assert sla.sla_forward_host_device_bytes(cfg, 3) == 0
+    io = (2 * cfg.B * cfg.H + 2 * cfg.B * cfg.H_kv) * cfg.N * cfg.d * 2
+    for n in (1, 2):
+        unit = cfg.replace(B=1, H=cfg.H // n, H_kv=cfg.H_kv // n)
+        ws = sla.sla_workspace_bytes(unit)
+        total = sla.sla_forward_host_device_bytes(cfg, n)
+        assert io + cfg.B * n * ws <= total <= io + cfg.B * n * ws + 256 * (6 + cfg.B * n)
+
+
 def test_route_rejects_missing_lists():
     cfg = wl.small_config(N=1024, N_valid=1024, k_h=3, k_l=2)
     c = sla.make_config(cfg)
