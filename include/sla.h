@@ -238,7 +238,9 @@ SLA_API sla_status sla_check_device_status(void* ws, void* stream, int32_t* deta
  * Errors: SLA_ERR_INVALID_ARG for a bad configuration, n_chunks < 1 or not
  * dividing H_kv, or a NULL or misaligned (16 bytes) pointer;
  * SLA_ERR_WORKSPACE for a NULL, misaligned or short arena; SLA_ERR_CUDA if
- * a copy, event or launch fails. All checks run before the first copy.
+ * a copy, event or launch fails. All checks run before the first copy. After
+ * SLA_ERR_CUDA, copies that were already queued may still run: synchronise
+ * all three streams before freeing or reusing the host buffers or the arena.
  */
 SLA_API size_t sla_forward_host_device_bytes(const sla_config* cfg, int32_t n_chunks);
 SLA_API sla_status sla_forward_host(const void* q_host, const void* k_host, const void* v_host,
