@@ -35,7 +35,7 @@ class LazyF64:
         return wl.bf16_bits_to_f64(self.bits[key])
 
 
-class GpuRun:
+class DeviceRun:
     """One sla_forward (and optionally sla_route) of a seeded layer on cuda:0."""
 
     def __init__(self, cfg: wl.LayerConfig, inputs: wl.LayerInputs | None = None, route=True):
@@ -76,7 +76,7 @@ class GpuRun:
                             x.f64("w_g"))
 
 
-def check_routing(run: GpuRun, L: oracle.Layer) -> dict:
+def check_routing(run: DeviceRun, L: oracle.Layer) -> dict:
     """Bit-exact routing except near-tie rows (counted). Returns a report."""
     c = run.cfg
     mask = run.mask.cpu().numpy()
@@ -126,7 +126,7 @@ def check_routing(run: GpuRun, L: oracle.Layer) -> dict:
     return report
 
 
-def unit_errors(run: GpuRun, L: oracle.Layer, units) -> dict:
+def unit_errors(run: DeviceRun, L: oracle.Layer, units) -> dict:
     """Max / mean abs error of O over the valid rows of the given (b, h, i) units.
 
     Rows whose routing is a near tie are scored under the GPU's own routing."""
@@ -150,7 +150,7 @@ def unit_errors(run: GpuRun, L: oracle.Layer, units) -> dict:
     return dict(max_abs=float(e.max()), mean_abs=float(e.mean()))
 
 
-def full_errors(run: GpuRun, ref: dict) -> dict:
+def full_errors(run: DeviceRun, ref: dict) -> dict:
     c = run.cfg
     O = run.O()
     assert np.all(O[:, :, c.N_valid:] == 0)

@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these anyway
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_util import GpuRun, bf16_to_f64, to_dev  # noqa: E402
+from gpu_util import DeviceRun, bf16_to_f64, to_dev  # noqa: E402
 from oracle import sla_grad  # noqa: E402
 
 REL = 2e-2
@@ -46,7 +46,7 @@ def run_backward(cfg, seed=3, v_shift=0.0, keep=None):
     """Relative Frobenius error per gradient tensor; ``keep`` (a dict) receives the GPU's
     gradients ("got") and the oracle's ("ref")."""
     x = wl.generate(cfg, v_shift=v_shift)
-    run = GpuRun(cfg, x, route=False)
+    run = DeviceRun(cfg, x, route=False)
     c = cfg
     dob = d_out_bits(c, seed)
     dout = to_dev(dob)
@@ -167,7 +167,7 @@ def test_backward_smooth_k_mean_term():
 def test_backward_all_negligible_is_zero():
     c = small(name="all_neg", N=512, N_valid=512, d=64, k_h=0, k_l=8, has_gate=1)
     x = wl.generate(c)
-    run = GpuRun(c, x, route=False)
+    run = DeviceRun(c, x, route=False)
     dout = to_dev(d_out_bits(c, 5))
     dq, dk, dv = torch.full_like(run.q, 7), torch.full_like(run.k, 7), torch.full_like(run.v, 7)
     dw_p = torch.full((c.d, c.d), 7.0, device="cuda")
@@ -193,7 +193,7 @@ def test_full_size_backward_on_sampled_blocks(name):
 
     cfg = wl.preset(name)
     x = wl.generate(cfg)
-    run = GpuRun(cfg, x, route=False)
+    run = DeviceRun(cfg, x, route=False)
     c = cfg
     dob = d_out_bits(c, 17)
     dout = to_dev(dob)
@@ -238,7 +238,7 @@ def test_full_size_topn_backward_on_sampled_blocks():
 
     c = wl.preset("nsa_causal")
     x = wl.generate(c)
-    run = GpuRun(c, x, route=False)
+    run = DeviceRun(c, x, route=False)
     dob = d_out_bits(c, 19)
     dout = to_dev(dob)
     dq, dk, dv = torch.empty_like(run.q), torch.empty_like(run.k), torch.empty_like(run.v)

@@ -14,7 +14,7 @@ import torch
 import block_sparse_linear_sm_b200 as sla
 from block_sparse_linear_sm_b200 import workloads as wl
 
-from gpu_util import GpuRun, full_errors
+from gpu_util import DeviceRun, full_errors
 
 pytestmark = pytest.mark.gpu
 
@@ -36,6 +36,6 @@ def test_context_usable_after_a_timeout():
     sla.sla_selftest_wait_timeout(ws, 1_000_000)
     assert sla.sla_check_device_status(ws)[0] == sla.SLA_ERR_DEVICE_TIMEOUT
     cfg = wl.small_config(name="after_timeout", N=1024, N_valid=1000, d=128, k_h=3, k_l=4)
-    run = GpuRun(cfg)
+    run = DeviceRun(cfg)
     err = full_errors(run, run.layer().forward())
     assert err["max_abs"] <= 2e-2 and err["mean_abs"] <= 2e-3, err

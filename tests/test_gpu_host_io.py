@@ -20,14 +20,14 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these anyway
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_util import GpuRun  # noqa: E402
+from gpu_util import DeviceRun  # noqa: E402
 
 
 def host(bits: np.ndarray):
     return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).pin_memory()
 
 
-def host_call(run: GpuRun, n_chunks: int, repeats: int = 1):
+def host_call(run: DeviceRun, n_chunks: int, repeats: int = 1):
     c = run.cfg
     hq, hk, hv = host(run.x.q), host(run.x.k), host(run.x.v)
     hout = torch.full(tuple(run.out.shape), float("nan"), dtype=torch.bfloat16).pin_memory()
@@ -60,7 +60,7 @@ CASES = [
 @pytest.mark.parametrize("kw", CASES, ids=[c["name"] for c in CASES])
 def test_host_call_equals_the_device_call(kw, per_group):
     cfg = wl.small_config(**kw)
-    run = GpuRun(cfg, route=False)
+    run = DeviceRun(cfg, route=False)
     n = cfg.H_kv if per_group else 1
     hout = host_call(run, n, repeats=2)
     assert same_bits(hout, run.out.cpu())
@@ -68,6 +68,6 @@ def test_host_call_equals_the_device_call(kw, per_group):
 
 def test_bench_shape_host_call():
     cfg = wl.preset("wan1.3b")
-    run = GpuRun(cfg, route=False)
+    run = DeviceRun(cfg, route=False)
     hout = host_call(run, cfg.H_kv)
     assert same_bits(hout, run.out.cpu())

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these anyway
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_util import (MAX_ABS, MEAN_ABS, GpuRun, check_routing, full_errors,  # noqa: E402
+from gpu_util import (MAX_ABS, MEAN_ABS, DeviceRun, check_routing, full_errors,  # noqa: E402
                       unit_errors)
 from oracle import sla_oracle as oracle  # noqa: E402
 
@@ -29,7 +29,7 @@ def small(**kw):
 
 def run_and_check_full(cfg, v_shift=0.0):
     x = wl.generate(cfg, v_shift=v_shift)
-    run = GpuRun(cfg, x)
+    run = DeviceRun(cfg, x)
     L = run.layer()
     rep = check_routing(run, L)
     assert rep["mismatched_rows"] == 0, rep
@@ -100,7 +100,7 @@ def test_all_critical_is_dense(d):
 def test_all_negligible_is_zero(d):
     nb = 8
     cfg = small(name="all_neg", N=nb * 64, N_valid=nb * 64, d=d, k_h=0, k_l=nb, has_gate=1)
-    run = GpuRun(cfg)
+    run = DeviceRun(cfg)
     assert np.all(run.O() == 0)
 
 
@@ -117,7 +117,7 @@ def test_linear_branch_alone_shifted_values(d):
     """All blocks marginal, W_p = I, no gate, V + 3: O is the linear branch and O(1)."""
     cfg = small(name="all_marg", N=2048, N_valid=2040, d=d, k_h=0, k_l=0, has_proj=0)
     x = wl.generate(cfg, v_shift=3.0)
-    run = GpuRun(cfg, x)
+    run = DeviceRun(cfg, x)
     ref = run.layer().forward()
     got = run.O()[:, :, :cfg.N_valid]
     want = ref["O_l"][:, :, :cfg.N_valid]
@@ -130,7 +130,7 @@ def test_mixed_layer_shifted_values_linear_branch():
     """Mixed classes with V + 3 so that the linear branch is O(1); W_p = I, no gate."""
     cfg = small(name="mixed_shift", N=2048, N_valid=2030, d=128, k_h=4, k_l=6, has_proj=0)
     x = wl.generate(cfg, v_shift=3.0)
-    run = GpuRun(cfg, x)
+    run = DeviceRun(cfg, x)
     ref = run.layer().forward()
     got = run.O()[:, :, :cfg.N_valid]
     want_l = ref["O_l"][:, :, :cfg.N_valid]
@@ -147,7 +147,7 @@ def test_per_head_projection_linear_term_shifted_values(d):
     cfg = small(name="per_head_shift", N=2048, N_valid=2030, d=d, H=4, H_kv=4, k_h=4, k_l=6,
                 proj_per_head=1, has_gate=1)
     x = wl.generate(cfg, v_shift=3.0)
-    run = GpuRun(cfg, x)
+    run = DeviceRun(cfg, x)
     ref = run.layer().forward()
     n = cfg.N_valid
     got_l = run.O()[:, :, :n] - ref["O_s"][:, :, :n]
@@ -167,7 +167,7 @@ def test_smooth_k_linear_term_with_offset_keys(d):
     kf = wl.bf16_bits_to_f64(x.k)
     kf[:, :, :cfg.N_valid] += 0.75
     x.k = wl.to_bf16_bits(kf)
-    run = GpuRun(cfg, x)
+    run = DeviceRun(cfg, x)
     ref = run.layer().forward()
     n = cfg.N_valid
     got_l = run.O()[:, :, :n] - ref["O_s"][:, :, :n]
@@ -210,7 +210,7 @@ def test_cos_filter_matches_oracle(kw):
     cfg = small(cos_filter=1, **kw)
     x, theta = _filtered_inputs(cfg)
     cfg = cfg.replace(cos_theta=theta)
-    run = GpuRun(cfg, x)
+    run = DeviceRun(cfg, x)
     L = run.layer()
     rep = check_routing(run, L)
     assert rep["mismatched_rows"] == 0, rep
@@ -252,7 +252,7 @@ def sampled_units(cfg, n=12, seed=0):
                                   "wan1.3b_cosfilter", "nsa_branches"])
 def test_full_size_workload(name):
     cfg = wl.preset(name)
-    run = GpuRun(cfg)
+    run = DeviceRun(cfg)
     L = run.layer()
     rep = check_routing(run, L)
     print(name, "routing", rep)
@@ -267,7 +267,7 @@ def test_longest_supported_sequence():
     full routing bit-exact except near-tie rows, sampled blocks of the output."""
     cfg = small(name="max_blocks", N=4096 * 64, N_valid=4096 * 64 - 7, d=64, H=2, H_kv=1,
                 k_h=16, k_l=64, has_gate=1)
-    run = GpuRun(cfg)
+    run = DeviceRun(cfg)
     L = run.layer()
     rep = check_routing(run, L)
     print(cfg.name, "routing", rep)

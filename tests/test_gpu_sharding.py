@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these anyway
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_util import GpuRun  # noqa: E402
+from gpu_util import DeviceRun  # noqa: E402
 
 
 CASES = [
@@ -32,7 +32,7 @@ CASES = [
 @pytest.mark.parametrize("world", [2, 3])
 def test_head_shards_reassemble_the_whole_layer(kw, world):
     cfg = wl.small_config(**kw)
-    run = GpuRun(cfg, route=True)
+    run = DeviceRun(cfg, route=True)
     crit = run.crit.cpu().numpy() if (cfg.k_h if cfg.mode == wl.MODE_THREEWAY else cfg.top_n) else None
     costs = sh.unit_costs(cfg, crit)
     full = torch.empty_like(run.out)
