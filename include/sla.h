@@ -36,12 +36,15 @@
  *                         (SLA analysis, Proj paragraph: O = O^s + Proj(O^l);
  *                          SALAD summary: input-dependent gate).
  *                         Without projection W_p = I; without gate g = 1.
- *                         The top-n mode has no linear branch: O = O_s.
+ *                         The top-n mode has no linear branch: O = O_s, or
+ *                         with nsa_branches the gated sum of NSA's compressed,
+ *                         selected and window branches (see nsa_branches).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Tensors are dense, row-major, in device memory (the caller allocates and
- *   frees all of them; the library never allocates):
+ *   frees all of them; the library never allocates). The one exception is
+ *   sla_forward_host, whose q, k, v and out are in host memory:
  *     q    bf16 [B, H,    N, d]
  *     k, v bf16 [B, H_kv, N, d]
  *     w_p  bf16 [d, d]   (row vector times matrix: O_l W_p), ignored unless has_proj;
@@ -144,7 +147,9 @@ typedef struct {
  * Sizes: B, H, H_kv, N and d must be >= 1; an empty problem (any of them 0) is
  * SLA_ERR_INVALID_ARG, not a no-op. Limits of the kernels (SLA_ERR_UNSUPPORTED
  * beyond them): N / block <= 4096 key blocks (N <= 262144 tokens, the routing
- * sort's row length) and B * H * N * d <= 2^40 elements.
+ * sort's row length) and B * H * N * d <= 2^40 elements; in TOPN_WINDOW mode
+ * top_n <= 64 and top_n + (window + 62) / 64 + 1 <= 128 (the flash kernel's
+ * block list), and cmp_block, cmp_stride <= 1024 with nsa_branches.
  */
 SLA_API sla_status sla_validate_config(const sla_config* cfg);
 
