@@ -475,8 +475,8 @@ def main():
         from block_sparse_linear_sm_b200 import sharding as sh
         costs = sh.unit_costs(cfg, route_lists(sla, torch, cfg, q, k, dev))
         shard = sh.HeadShard(cfg, world, rank, costs)
-        if not shard.units:
-            raise RuntimeError("more ranks than KV groups")
+        if any(not p for p in shard.plan):  # the same plan on every rank: all of them stop here
+            raise RuntimeError(f"{world} ranks but only {cfg.H_kv} KV groups to share")
         q, k, v, w_p, w_g = shard.inputs(q, k, v, w_p, w_g)
         cfg = shard.local
         loads = sh.plan_loads(costs, shard.plan)
