@@ -695,6 +695,9 @@ def main():
         "gpu_launches": ns * args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                # the inputs' copy rate over the whole step: the call is bound by it when the
+                # kernels and the copies out hide behind the copies in
+                "h2d_gbs_over_step": h2d / (e2e_ms * 1e-3) / 1e9,
                 "api": f"sla_forward_host (pinned host q, k, v and out; {n_chunks} units of whole KV groups "
                        "per batch entry, copies in, kernels and copies out overlapped on three streams)"},
         "clocks": clocks,
