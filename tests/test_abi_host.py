@@ -316,3 +316,21 @@ def test_nsa_branches_configuration():
     assert sla.sla_validate_config(wl.preset("wan1.3b").replace(nsa_branches=1)) == sla.SLA_ERR_UNSUPPORTED
     assert sla.sla_validate_config(c.replace(cmp_stride=0)) == sla.SLA_ERR_INVALID_ARG
     assert sla.sla_validate_config(c.replace(nsa_branches=2)) == sla.SLA_ERR_INVALID_ARG
+
+
+def test_noalloc_entry_points_reject_bad_arguments_without_a_device():
+    """sla_route_noalloc checks its arguments before it looks for a device; its status
+    reader needs a device and reports a CUDA error where there is none."""
+    c = sla.make_config(wl.preset("tiny"))
+    L = sla.lib()
+    assert L.sla_route_noalloc(None, 16, ctypes.byref(c), None, 16, 16, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_route_noalloc(16, 16, ctypes.byref(c), None, None, 16, None) == sla.SLA_ERR_INVALID_ARG
+    assert L.sla_route_noalloc(8, 16, ctypes.byref(c), None, 16, 16, None) == sla.SLA_ERR_INVALID_ARG
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:  # pragma: no cover
+        has_gpu = False
+    if not has_gpu:
+        detail = ctypes.c_int32(0)
+        assert L.sla_route_noalloc_status(None, ctypes.byref(detail)) == sla.SLA_ERR_CUDA

@@ -62,3 +62,28 @@ def test_nsa_compressed_branch_counts_causal_compressed_keys():
     assert m["sparse_flash_slc"] == ("tensor", 4.0 * c.d * c.B * c.H * slc)
     assert m["sparse_flash_win"] == ("tensor", 4.0 * c.d * c.B * c.H * win)
     assert "sparse_flash" not in m
+
+
+def test_routing_report_counts_ties_and_mismatches():
+    """bench.routing_report: a mask equal to the oracle's classes has no mismatched row;
+    one changed row that is not a near tie is counted once."""
+    c = wl.preset("tiny")
+    x = wl.generate(c)
+    L = bench.oracle_layer(c, x)
+    mask = np.stack([L.classes(0, h) for h in range(c.H)])[None]
+    rep = bench.routing_report(c, L, mask, [0, 1])
+    assert rep["rows"] == c.H * c.nqb and rep["mismatched_rows"] == 0
+    ties = L.tie_rows(0, 1)
+    i = int(np.nonzero(~ties)[0][0])
+    bad = mask.copy()
+    bad[0, 1, i] = np.roll(bad[0, 1, i], 1)
+    assert bench.routing_report(c, L, bad, [0, 1])["mismatched_rows"] == 1
+
+
+def test_oracle_sample_extrapolates_set_up_and_units():
+    c = wl.preset("tiny")
+    x = wl.generate(c)
+    r = bench.oracle_sample(c, x, [0, 1], 4)
+    assert r["heads"] == 2 and r["units"] == 8
+    want = c.B * c.H * r["setup_s_per_head"] + c.B * c.H * c.nqb * r["unit_s"]
+    assert abs(r["full_layer_s"] - want) <= 1e-12 * want

@@ -32,6 +32,13 @@ def _noalloc():
     return fn
 
 
+def _noalloc_status():
+    fn = sla.lib().sla_route_noalloc_status
+    fn.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)]
+    fn.restype = ctypes.c_int
+    return fn
+
+
 def _dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).cuda()
 
@@ -46,6 +53,10 @@ def _outputs(cfg):
 
 
 CASES = [wl.preset("tiny"), wl.preset("wan1.3b"),
+         # the key-block filter's flags also live in the static array (after the scores)
+         wl.preset("wan1.3b_cosfilter"),
+         wl.small_config(name="cosfilter_small", H=4, H_kv=2, N=1024, N_valid=1000, d=64, k_h=3, k_l=4,
+                         cos_filter=1, cos_theta=1.0 / 64),  # i.i.d. blocks: about half filtered
          wl.small_config(name="topn", mode=wl.MODE_TOPN_WINDOW, H=8, H_kv=2, N=2048, N_valid=2000,
                          d=128, top_n=4, window=200, causal=1, has_proj=0, generator="block_shift")]
 
@@ -69,6 +80,9 @@ def test_noalloc_route_matches_workspace_route(cfg):
                 got[1].data_ptr() if (cfg.k_h if threeway else cfg.top_n) else None,
                 got[2].data_ptr() if threeway and cfg.k_l else None, stream)
         assert st == sla.SLA_OK, sla.status_string(st)
+        detail = ctypes.c_int32(-1)
+        dst = _noalloc_status()(stream, ctypes.byref(detail))
+        assert dst == sla.SLA_OK and detail.value == 0, (sla.status_string(dst), detail.value)
         torch.cuda.synchronize()
         for a, b in zip(got, ref):
             assert torch.equal(a, b), f"call {call}: routing differs from sla_route"
