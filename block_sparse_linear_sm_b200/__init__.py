@@ -98,6 +98,10 @@ def lib() -> ctypes.CDLL:
         L.sla_forward_host_device_bytes.restype = S
         L.sla_forward_host.argtypes = [P, P, P, P, P, C, P, I32, P, S, P, P, P]
         L.sla_forward_host.restype = ctypes.c_int
+        L.sla_route_noalloc.argtypes = [P, P, C, P, P, P, P]
+        L.sla_route_noalloc.restype = ctypes.c_int
+        L.sla_route_noalloc_status.argtypes = [P, ctypes.POINTER(I32)]
+        L.sla_route_noalloc_status.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -262,6 +266,21 @@ def sla_backward_timed(q, k, v, w_p, w_g, c, out, dout, dq, dk, dv, dw_p, dw_g, 
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check(lib().sla_backward_timed(*_bwd_args(q, k, v, w_p, w_g, c, out, dout, dq, dk, dv, dw_p, dw_g, ws,
                                                bws, stream), arr, len(events)), "sla_backward_timed")
+
+
+def sla_route_noalloc(q, k, c, mask_out, crit_idx, neg_idx, stream=None) -> None:
+    """sla_route without a workspace: its scratch is the library's static device array."""
+    cfg = _cfg(c)
+    _check(lib().sla_route_noalloc(_ptr(q), _ptr(k), ctypes.byref(cfg), _ptr(mask_out), _ptr(crit_idx),
+                                   _ptr(neg_idx), _stream(stream)), "sla_route_noalloc")
+
+
+def sla_route_noalloc_status(stream=None) -> tuple:
+    """(status, detail) of the last sla_route_noalloc on this device, after synchronising the
+    stream; clears the status word."""
+    detail = ctypes.c_int32(0)
+    st = lib().sla_route_noalloc_status(_stream(stream), ctypes.byref(detail))
+    return int(st), int(detail.value)
 
 
 def sla_check_device_status(ws, stream=None) -> tuple:

@@ -5,6 +5,8 @@
 
 #include <mutex>
 
+#include <cuda.h>  // CUcontext (type only; the driver is reached through the runtime)
+
 #include "sla_internal.h"
 
 namespace sla {
@@ -17,21 +19,53 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // id of the context the address belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Process-unique id of the current CUDA context (0 if it cannot be read). A device
+// reset ends the primary context; the next one has another id, and the array then
+// has another device address.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = (CtxGetCurrentFn)p;
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (CtxGetIdFn)p;
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
 
 // Device address of g_route_scratch on the current device. The host-side name
-// of the array is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// of the array is only a stand-in, so the address is looked up (with that device
+// current) once per device and context, and cached.
 cudaError_t scratch_for_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
+  void* p = g_scratch_ptr[dev];
+  const unsigned long long ctx = p != nullptr ? current_context_id() : 0;
+  if (p == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
+    p = nullptr;
     e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -77,4 +111,11 @@ extern "C" SLA_API sla_status sla_route_noalloc(const void* q, const void* k, co
   if (launch_scores(p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
   const cudaError_t e = threeway ? launch_classify(p, a, false, s) : launch_select(p, a, s);
   return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+}
+
+extern "C" SLA_API sla_status sla_route_noalloc_status(void* stream, int32_t* detail) {
+  void* scratch = nullptr;
+  if (scratch_for_current_device(&scratch) != cudaSuccess) return SLA_ERR_CUDA;
+  // the status word is the first region of the routing plan (offset 0)
+  return sla_check_device_status(scratch, stream, detail);
 }

@@ -389,7 +389,10 @@ SLA_API const char* sla_version(void);
  *   rejected with SLA_ERR_WORKSPACE before anything is launched (about 38 MB
  *   at B1 H12 N32768 d128; the scratch grows with B * H * (N / 64)^2).
  * - The first call on a device looks up the array's device address with that
- *   device current; make that first call before any stream capture.
+ *   device current; make that first call before any stream capture. The
+ *   address is cached per device together with the id of the CUDA context it
+ *   belongs to; after a device reset (a new context) the next call looks it up
+ *   again.
  * - All calls share the one array, which keeps the last call's contents (the
  *   status word is cleared at the start of every call). Calls that overlap on
  *   the GPU - on two streams, or from two host threads - race on it and must
@@ -399,6 +402,18 @@ SLA_API const char* sla_version(void);
 SLA_API sla_status sla_route_noalloc(const void* q, const void* k, const sla_config* cfg,
                                      int8_t* mask_out, int32_t* crit_idx, int32_t* neg_idx,
                                      void* stream);
+
+/*
+ * Device-side status of sla_route_noalloc (it has no caller workspace to hold
+ * one). Synchronises `stream`, reads the status word at the start of the
+ * current device's static routing array, clears it and returns what
+ * sla_check_device_status returns for a workspace: SLA_OK, or
+ * SLA_ERR_DEVICE_TIMEOUT / SLA_ERR_DEVICE_CHECK with *detail (nullable) naming
+ * the kernel and check, or SLA_ERR_CUDA. Allocates nothing. Every
+ * sla_route_noalloc call clears the word when it starts, so read it after the
+ * call whose errors matter and before the next one.
+ */
+SLA_API sla_status sla_route_noalloc_status(void* stream, int32_t* detail);
 
 #ifdef __cplusplus
 }
