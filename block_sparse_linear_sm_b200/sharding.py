@@ -10,7 +10,10 @@ query heads that read it, since they share K, V and (top-n mode) the selection.
 Each unit's cost is estimated from the routing as the 64-key tiles the sparse
 flash kernel executes for it (pairs of query blocks share one merged block
 list) plus the linear branch's fixed per-head work; units go to ranks by
-longest-processing-time-first (LPT). Each rank gathers its heads into
+longest-processing-time-first (LPT). The costs need the routing of every group:
+each rank routes only every world-th group (distributed_costs) and the ranks
+share the costs with one small all_gather, so no rank routes the whole layer.
+Each rank then gathers its heads into
 contiguous local tensors, runs the whole layer on them through the C ABI, and
 the outputs can be all-gathered back into head order. Nothing here computes
 any part of the layer: the layer runs in the CUDA kernels of libsla.so.
@@ -59,6 +62,46 @@ def unit_costs(cfg: wl.LayerConfig, crit: Optional[np.ndarray] = None) -> np.nda
                     tiles += np.unique(sel[sel >= 0]).size + min(wb, i + 1)
                 cost[hk] += tiles * group  # every query head of the group runs the tiles
     return cost
+
+
+def probe_units(cfg: wl.LayerConfig, world: int, rank: int) -> List[int]:
+    """The KV groups whose routing this rank computes for the cost estimate: every
+    world-th group from this rank's index, so the ranks split the routing work evenly."""
+    return list(range(rank, cfg.H_kv, world))
+
+
+def unit_costs_of(cfg: wl.LayerConfig, units: Sequence[int], crit_local: Optional[np.ndarray]) -> np.ndarray:
+    """Costs of the given KV groups from the routing of the layer restricted to them
+    (``crit_local``: the lists of local_config(cfg, units), or None)."""
+    if not units:
+        return np.zeros(0)
+    return unit_costs(local_config(cfg, units), crit_local)
+
+
+def distributed_costs(cfg: wl.LayerConfig, world: int, rank: int, route_local, dist) -> np.ndarray:
+    """Every KV group's cost on every rank, with each rank routing only its probe groups.
+
+    ``route_local(units)`` routes the layer restricted to ``units`` (local_config) and
+    returns its host lists as unit_costs expects them (or None without lists). The costs
+    are exchanged with one all_gather of a padded float64 vector, so every rank ends with
+    the same vector and computes the same plan."""
+    import torch
+
+    mine = probe_units(cfg, world, rank)
+    local = unit_costs_of(cfg, mine, route_local(mine) if mine else None)
+    width = (cfg.H_kv + world - 1) // world
+    buf = torch.zeros(width, dtype=torch.float64)
+    buf[:len(local)] = torch.from_numpy(np.asarray(local, dtype=np.float64))
+    backend = dist.get_backend() if hasattr(dist, "get_backend") else "gloo"
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    buf = buf.to(dev)
+    parts = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(parts, buf)
+    costs = np.zeros(cfg.H_kv)
+    for r, part in enumerate(parts):
+        units = probe_units(cfg, world, r)
+        costs[units] = part.cpu().numpy()[:len(units)]
+    return costs
 
 
 def balance(costs: Sequence[float], world: int) -> List[List[int]]:

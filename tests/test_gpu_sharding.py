@@ -1,7 +1,8 @@
 """Head-sharded layer on one GPU: every rank's share run in turn and put back in head
 order equals the whole layer bit for bit (each stage works per head, or per KV group,
-so a layer restricted to some heads computes exactly their rows). The ranks run one
-after another on one device; none waits for another."""
+so a layer restricted to some heads computes exactly their rows), and matches the
+float64 oracle on sampled units of every head. The ranks run one after another on
+one device; none waits for another."""
 import numpy as np
 import pytest
 
@@ -16,7 +17,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():  # pragma: no cover - CPU runs deselect these anyway
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
-from gpu_util import DeviceRun  # noqa: E402
+from gpu_util import MAX_ABS, MEAN_ABS, DeviceRun, unit_errors  # noqa: E402
 
 
 CASES = [
@@ -48,3 +49,10 @@ def test_head_shards_reassemble_the_whole_layer(kw, world):
         assert sla.sla_check_device_status(ws) == (0, 0)
         full[:, shard.heads] = out
     assert torch.equal(full, run.out)
+    # the reassembled shards against the float64 oracle on sampled units of every head
+    L = run.layer()
+    run.out = full
+    rng = np.random.default_rng(world)
+    units = [(0, h, int(i)) for h in range(cfg.H) for i in rng.choice(cfg.nqb, 2, replace=False)]
+    err = unit_errors(run, L, units)
+    assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err

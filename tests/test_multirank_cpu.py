@@ -159,3 +159,67 @@ def test_head_sharded_gather_two_gloo_ranks():
     # costs [3, 1, 2]: rank 0 takes unit 0, rank 1 units 1 and 2; both ranks agree
     assert res[0][0] == res[1][0] == [[0], [1, 2]]
     assert res[0][1] and res[1][1]
+
+
+def _fake_routing(cfg):
+    """Deterministic critical lists [B, H, nqb, k_h] for a small layer (a stand-in for the
+    routing the GPU computes; only the cost estimate reads them)."""
+    rng = np.random.default_rng(5)
+    crit = np.zeros((cfg.B, cfg.H, cfg.nqb, cfg.k_h), np.int32)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            for i in range(cfg.nqb):
+                crit[b, h, i] = np.sort(rng.choice(cfg.nkb, cfg.k_h, replace=False))
+    return crit
+
+
+def _costs_rank_main(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = wl.small_config(N=1024, N_valid=1000, H=10, H_kv=5, k_h=3, k_l=2)
+        full = _fake_routing(cfg)
+        group = cfg.H // cfg.H_kv
+        routed = []
+
+        def route_local(units):
+            routed.extend(units)
+            heads = [u * group + g for u in units for g in range(group)]
+            return full[:, heads]
+        costs = sh.distributed_costs(cfg, world, rank, route_local, dist)
+        q.put((rank, (costs.tolist(), sorted(routed))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_distributed_costs_route_a_share_and_agree_two_gloo_ranks():
+    """Each rank routes only every second KV group; after the all_gather both ranks hold
+    the cost vector of the whole layer, equal to the single-process estimate."""
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_costs_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=100) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    cfg = wl.small_config(N=1024, N_valid=1000, H=10, H_kv=5, k_h=3, k_l=2)
+    want = sh.unit_costs(cfg, _fake_routing(cfg)).tolist()
+    assert res[0][0] == res[1][0] == want
+    assert res[0][1] == [0, 2, 4] and res[1][1] == [1, 3]
