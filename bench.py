@@ -43,6 +43,10 @@ UNIT = "dense-equiv TFLOP/s"
 FP64_MMA_TFLOPS = 37.0
 
 
+# query blocks per step of the reference arm (about 2-4 s of float64 work each)
+REF_UNITS = 48
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -64,14 +68,15 @@ def stage_model(c: wl.LayerConfig) -> dict:
     bf = 2
     m = {}
     m["pool"] = ("hbm", (B * H + B * Hkv) * Nv * d * bf + (B * H + B * Hkv) * nb * d * 8)
-    if c.mode == wl.MODE_THREEWAY and nb - c.k_h - c.k_l > 0:
-        # phi(Q) (bf16) and, with a gate, g_t (fp32) for the linear branch
-        m["pool"] = ("hbm", m["pool"][1] + B * H * Nv * d * bf + (B * H * Nv * 4 if c.has_gate else 0))
     # float64 products q_bar . k_bar on the FP64 tensor path (mma.sync m8n8k4): every (i, j)
     # in three-way mode, the candidates j < i in top-n mode
     pairs = nb * nb if c.mode == wl.MODE_THREEWAY else nb * (nb - 1) // 2
     m["pooled_scores"] = ("fp64", 2.0 * B * H * pairs * d)
     if c.mode == wl.MODE_THREEWAY:
+        # the fused router (when a tile's score rows fit in shared memory): pooled keys,
+        # then one kernel for query pooling, the float64 scores (its bound) and classify
+        m["pool_keys"] = ("hbm", B * Hkv * Nv * d * bf + B * Hkv * nb * d * 8)
+        m["route"] = ("fp64", 2.0 * B * H * nb * nb * d)
         marg = nb - c.k_h - c.k_l
         m["classify"] = ("hbm", B * H * nb * nb * 8 + B * H * nb * nb * (1 + (2 if marg else 0))
                          + B * H * nb * c.k_h * 4)
@@ -132,6 +137,8 @@ def backward_stage_model(c: wl.LayerConfig) -> dict:
     m = {"bwd_columns": ("hbm", B * H * nb * c.k_h * 4 + 2 * B * H * nb * words * 4)}
     if lin:
         nqb_pad, nkb_pad = (nb + 127) // 128 * 128, (nb + 63) // 64 * 64
+        # reads q; writes phi(Q) (bf16) and g_t (fp32)
+        m["bwd_phi_gate"] = ("hbm", 2 * B * H * Nv * d * bf + (B * H * Nv * 4 if c.has_gate else 0))
         # reads phi(Q), q, O, dO, S'_i, Z_i (and g_t); writes the fp32 dq part, D_t, [dS'_i | dZ_i]
         m["bwd_linear"] = ("hbm", 4 * B * H * Nv * d * bf + B * H * nb * (d * d * bf + d * 4)
                            + B * H * Nv * 4 * (2 if c.has_gate else 1) + B * H * Nv * d * 4
@@ -222,18 +229,61 @@ def measure_backward(sla, torch, cfg, q, k, v, w_p, w_g, out, ws, steps, warmup,
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, sampled during a region.
+
+    NVML (nvidia-ml-py) is read from a thread every 20 ms, so even a region of
+    a fraction of a second gives tens of samples; without NVML, nvidia-smi -lms 200
+    is run in the background. Nothing is set on the GPU: only queries."""
+
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index: int, path: str | None):
+    def __init__(self, gpu_index: int, path: str | None, period_s: float = 0.02):
         self.idx = gpu_index
         self.path = path
+        self.period = period_s
         self.proc = None
+        self.thread = None
+        self.samples = []   # (sm_mhz, max_mhz, power_w, reasons bitmask)
+        self.lines = []
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.idx)
 
     def __enter__(self):
+        import threading
         try:
-            self.f = open(self.path, "w") if self.path else subprocess.DEVNULL
+            nv, h = self._nvml_handle()
+            self.stop = threading.Event()
+
+            def run():
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                while not self.stop.is_set():
+                    try:
+                        self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), float(mx),
+                                             nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                             int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                    except Exception:
+                        pass
+                    self.stop.wait(self.period)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
@@ -243,7 +293,16 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        if self.thread is not None:
+            time.sleep(0.05)
+            self.stop.set()
+            self.thread.join(timeout=5)
+            if self.path:
+                with open(self.path, "w") as f:
+                    f.write("sm_mhz,max_mhz,power_w,reasons\n")
+                    for smp in self.samples:
+                        f.write(",".join(str(x) for x in smp) + "\n")
+            return
         if self.proc is not None:
             time.sleep(0.25)
             self.proc.terminate()
@@ -254,55 +313,136 @@ class ClockSampler:
                 out = ""
             self.lines = [l for l in out.splitlines() if l.strip()]
             if self.path:
-                self.f.write(out)
-                self.f.close()
+                with open(self.path, "w") as f:
+                    f.write(out)
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        sm, mx, reasons, power = [], None, set(), []
+        if self.samples:
+            for clk, m, pw, bits in self.samples:
+                sm.append(clk)
+                mx = m
+                power.append(pw)
+                reasons |= {n for n, b in self.REASONS.items() if bits & b}
+            src = f"NVML every {self.period * 1e3:.0f} ms"
+        else:
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for l in self.lines:
+                f = [x.strip() for x in l.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx = float(f[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            src = "nvidia-smi -lms 200"
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         load = sorted(sm)[len(sm) // 4:] or sm
-        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+               "samples": len(sm), "sm_mhz_min": min(sm), "source": src}
+        if power:
+            out["power_w_max"] = max(power)
+        return out
 
 
 # ---------------------------------------------------------------------------
 # CPU oracle on a bounded sample (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(cfg: wl.LayerConfig, x: wl.LayerInputs, units, budget_s: float | None = None):
-    """Times the float64 oracle on whole (b, h, query block) units; returns (seconds, units done)."""
-    import oracle  # test infrastructure: only this CPU leg of the benchmark uses it
+class _LazyBits:
+    """Float64 view of bf16 bits, converted slice by slice (full layers do not fit as float64)."""
 
-    class Lazy:
-        def __init__(self, bits):
-            self.bits = bits
+    def __init__(self, bits):
+        self.bits = bits
+        self.shape = bits.shape
 
-        def __getitem__(self, k):
-            return wl.bf16_bits_to_f64(self.bits[k])
+    def __getitem__(self, k):
+        return wl.bf16_bits_to_f64(self.bits[k])
 
+
+def oracle_layer(cfg: wl.LayerConfig, x: wl.LayerInputs):
+    import oracle  # test infrastructure: only the CPU legs of the benchmark use it
+    return oracle.Layer(cfg, _LazyBits(x.q), _LazyBits(x.k), _LazyBits(x.v), x.f64("w_p"), x.f64("w_g"))
+
+
+def oracle_sample(cfg: wl.LayerConfig, x: wl.LayerInputs, heads, units_per_head, budget_s=None,
+                  seed=1234, layer=None):
+    """Times the float64 oracle on a sample of one layer and extrapolates to the whole layer.
+
+    Per sampled head: the head's routing (pooled means, scores, classes; top-n mode: its
+    KV group's selection) and linear states are computed first and timed as the head's
+    set-up; then units_per_head (b, h, query block) units are timed one by one. The
+    full-layer time is B*H (top-n: B*H_kv) set-ups plus B*H*nqb units at the measured
+    means. Returns a dict with the extrapolated time and what was sampled."""
+    L = layer if layer is not None else oracle_layer(cfg, x)
+    rng = np.random.default_rng(seed)
+    topn = cfg.mode == wl.MODE_TOPN_WINDOW
+    group = cfg.H // cfg.H_kv
+    lin = not topn and (cfg.nkb - cfg.k_h - cfg.k_l > 0 or cfg.linear_all)
     t0 = time.perf_counter()
-    L = oracle.Layer(cfg, Lazy(x.q), Lazy(x.k), Lazy(x.v), x.f64("w_p"), x.f64("w_g"))
-    done = 0
-    for (b, h, i) in units:
-        L.unit(b, h, i)
-        done += 1
+    t_setup = t_units = 0.0
+    n_setup = n_units = 0
+    for h in heads:
+        a = time.perf_counter()
+        if topn:
+            L.selection(0, h // group)
+        else:
+            L.classes(0, h)
+            if lin:
+                L.states(0, h // group)
+        t_setup += time.perf_counter() - a
+        n_setup += 1
+        for i in rng.permutation(cfg.nqb)[:units_per_head]:
+            a = time.perf_counter()
+            L.unit(0, int(h), int(i))
+            t_units += time.perf_counter() - a
+            n_units += 1
+            if budget_s is not None and time.perf_counter() - t0 > budget_s:
+                break
         if budget_s is not None and time.perf_counter() - t0 > budget_s:
             break
-    return time.perf_counter() - t0, done
+    setups = cfg.B * (cfg.H_kv if topn else cfg.H)
+    full_s = setups * t_setup / max(n_setup, 1) + units_total(cfg) * t_units / max(n_units, 1)
+    return dict(full_layer_s=full_s, seconds=time.perf_counter() - t0, heads=n_setup, units=n_units,
+                setup_s_per_head=t_setup / max(n_setup, 1), unit_s=t_units / max(n_units, 1), layer=L)
+
+
+def routing_report(cfg, L, mask, heads):
+    """The GPU's routing (int8 class mask, [B, H or H_kv, nqb, nkb]) against the oracle's on
+    the sampled heads: rows, near-tie rows (left out of the exact comparison) and mismatched
+    rows among the others."""
+    rep = dict(rows=0, tie_rows=0, mismatched_rows=0)
+    if cfg.mode == wl.MODE_THREEWAY:
+        for h in heads:
+            cls, tie = L.classes(0, h), L.tie_rows(0, h)
+            for i in range(cfg.nqb):
+                rep["rows"] += 1
+                if tie[i]:
+                    rep["tie_rows"] += 1
+                else:
+                    rep["mismatched_rows"] += int(not np.array_equal(mask[0, h, i], cls[i]))
+    else:
+        group = cfg.H // cfg.H_kv
+        for hk in sorted({h // group for h in heads}):
+            sels, tie = L.selection(0, hk)
+            for i in range(cfg.nqb):
+                rep["rows"] += 1
+                if tie[i]:
+                    rep["tie_rows"] += 1
+                    continue
+                want = np.zeros(cfg.nkb, np.int8)
+                want[sels[i]] = 2
+                rep["mismatched_rows"] += int(not np.array_equal(mask[0, hk, i], want))
+    rep["heads"] = [int(h) for h in heads]
+    rep["rule"] = ("rows whose k-th and (k+1)-th pooled probabilities (either class boundary; top-n: "
+                   "the group sum at position top_n) are within 1e-5 relative are near ties: counted, "
+                   "not compared")
+    return rep
 
 
 def oracle_threads() -> int:
@@ -314,14 +454,9 @@ def oracle_threads() -> int:
         return 1
 
 
-def sample_units(cfg, n, n_heads=2, seed=1234):
+def sample_heads(cfg, n, seed=1234):
     rng = np.random.default_rng(seed)
-    heads = rng.permutation(cfg.H)[:max(1, min(cfg.H, n_heads))]
-    units = []
-    for h in heads:
-        for i in rng.permutation(cfg.nqb)[:max(1, n // len(heads))]:
-            units.append((0, int(h), int(i)))
-    return units
+    return sorted(int(h) for h in rng.permutation(cfg.H)[:max(1, min(cfg.H, n))])
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -384,34 +519,80 @@ def units_total(cfg):
     return cfg.B * cfg.H * cfg.nqb
 
 
+def linear_branch_cost(cfg, mask):
+    """Both ways of forming S_i, Z_i from the routing (int8 classes [B, H, nqb, nkb]):
+    the direct sum over the marginal blocks as the aggregation GEMM with the 0/1 marginal
+    mask (what runs), and the total minus the critical and negligible blocks. On the
+    tensor cores either is a dense GEMM unless whole mask tiles are zero, so the count
+    of nonzero 128 x 64 tiles (the aggregation kernel's M x K step) of each mask is the
+    cost that could differ; as a gather the complement moves every excluded state."""
+    B, H, nqb, nkb = mask.shape
+    dd = (cfg.d * cfg.d + cfg.d + 127) // 128 * 128
+    marg = mask == 1
+    excl = ~marg
+    tiles = {"marginal": 0, "excluded": 0, "total": 0}
+    for b in range(B):
+        for h in range(H):
+            for i0 in range(0, nqb, 128):
+                for j0 in range(0, nkb, 64):
+                    tiles["total"] += 1
+                    tiles["marginal"] += bool(marg[b, h, i0:i0 + 128, j0:j0 + 64].any())
+                    tiles["excluded"] += bool(excl[b, h, i0:i0 + 128, j0:j0 + 64].any())
+    direct = 2.0 * B * H * nqb * nkb * dd
+    return {"direct_gemm_flop": direct,
+            "complement_gemm_flop": direct * tiles["excluded"] / max(tiles["marginal"], 1),
+            "complement_gather_bytes": float(excl.sum()) * dd * 2,
+            "nonzero_tiles_128x64": tiles,
+            "cheaper_on_tensor_cores": "direct" if tiles["marginal"] <= tiles["excluded"] else "complement",
+            "ran": "direct",
+            "what": "S_i = sum over marginal j of h_j (GEMM with the marginal mask) against "
+                    "S_i = H_total - sum over critical and negligible j of h_j"}
+
+
+def r_heads(r, heads):
+    """The heads whose set-up the oracle sample reached."""
+    return heads[:r["heads"]]
+
+
+def config_keys(cfg, parallelism):
+    """The config object of the JSON line (the same keys in both arms)."""
+    return {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "H_kv": cfg.H_kv, "N": cfg.N, "N_valid": cfg.N_valid,
+            "d": cfg.d, "k_h": cfg.k_h, "k_l": cfg.k_l, "has_proj": cfg.has_proj, "has_gate": cfg.has_gate,
+            "parallelism": parallelism}
+
+
 def run_reference(args, cfg):
+    """The oracle arm: each step times the float64 oracle on one sampled head (its set-up and
+    REF_UNITS query blocks) and extrapolates to the whole layer like the cpu_baseline leg."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     x = wl.generate(cfg)
-    units = sample_units(cfg, 8)
     per_step = []
+    heads = sample_heads(cfg, cfg.H, seed=99)
     for s in range(args.warmup + args.steps):
-        t, n = oracle_sample(cfg, x, units)
+        h = heads[s % len(heads)]
+        r = oracle_sample(cfg, x, [h], REF_UNITS, seed=1000 + s)
+        r.pop("layer")
         if s >= args.warmup:
-            per_step.append((t, n))
-    tsum = sum(t for t, _ in per_step)
-    nsum = sum(n for _, n in per_step)
-    frac = nsum / units_total(cfg)
-    value = frac * cfg.dense_flops() / tsum / 1e12
-    full_layer_ms = tsum / frac * 1e3
+            per_step.append(r)
+    full_s = statistics.mean(r["full_layer_s"] for r in per_step)
+    value = cfg.dense_flops() / full_s / 1e12
+    sampled = sum(r["seconds"] for r in per_step)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": tsum / len(per_step) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": full_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "N_valid": cfg.N_valid,
-                   "d": cfg.d, "k_h": cfg.k_h, "k_l": cfg.k_l, "parallelism": "replicas"},
+        "config": config_keys(cfg, "replicas"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                         "sample": f"{len(units)} (head, query block) units of {units_total(cfg)} per step, "
-                                   "full-layer time extrapolated by unit count"},
+                         "sample": f"per step one head's set-up (routing, linear states) and "
+                                   f"{min(REF_UNITS, cfg.nqb)} of its {cfg.nqb} query blocks, "
+                                   f"{sampled / len(per_step):.1f} s of CPU work "
+                                   "per step; ms_per_step is the whole layer extrapolated from the "
+                                   "measured set-up and per-unit times"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "full_layer_ms_extrapolated": full_layer_ms,
+        "sampled_seconds_per_step": sampled / len(per_step),
     }
     print(json.dumps(line))
     return 0
@@ -431,9 +612,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--clocks-csv", default=None)
+    ap.add_argument("--soak-s", type=float, default=0.5,
+                    help="seconds of graph replays right before the timed replays (clock sampling)")
     ap.add_argument("--no-backward", action="store_true", help="skip the sla_backward measurement")
     ap.add_argument("--shard", default="none", choices=["none", "heads"],
                     help="heads: each rank runs its KV groups of one layer (LPT on the routed tiles)")
+    ap.add_argument("--shard-gather", action="store_true",
+                    help="with --shard heads: also time steps of the local layer plus all_gather_heads")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads (H = H_kv; small profiler captures)")
     args = ap.parse_args()
@@ -470,10 +655,19 @@ def main():
     q, k, v, w_p, w_g = up(x.q), up(x.k), up(x.v), up(x.w_p), up(x.w_g)
     full_cfg, shard_info = cfg, None
     if args.shard == "heads":
-        # one layer split over the ranks by KV group: route it whole, estimate each group's
-        # work from its routed tiles, balance (LPT), and run this rank's heads
+        # one layer split over the ranks by KV group: estimate each group's work from its
+        # routed tiles (every rank routes every world-th group; the costs are all-gathered),
+        # balance (LPT), and run this rank's heads
         from block_sparse_linear_sm_b200 import sharding as sh
-        costs = sh.unit_costs(cfg, route_lists(sla, torch, cfg, q, k, dev))
+
+        def route_local(units):
+            heads = sh.query_heads(cfg, units)
+            return route_lists(sla, torch, sh.local_config(cfg, units), sh.gather_heads(q, heads),
+                               sh.gather_heads(k, units), dev)
+        if dist is None:
+            costs = sh.unit_costs(cfg, route_lists(sla, torch, cfg, q, k, dev))
+        else:
+            costs = sh.distributed_costs(cfg, world, rank, route_local, dist)
         shard = sh.HeadShard(cfg, world, rank, costs)
         if any(not p for p in shard.plan):  # the same plan on every rank: all of them stop here
             raise RuntimeError(f"{world} ranks but only {cfg.H_kv} KV groups to share")
@@ -482,7 +676,8 @@ def main():
         loads = sh.plan_loads(costs, shard.plan)
         shard_info = {"plan": shard.plan, "estimated_loads": loads,
                       "imbalance": max(loads) / (sum(loads) / len(loads)),
-                      "what": "KV groups per rank, LPT on the tiles the routing makes the flash kernel run"}
+                      "what": "KV groups per rank, LPT on the tiles the routing makes the flash kernel run; "
+                              "each rank routed every world-th group for the estimate"}
     out = torch.empty(cfg.B, cfg.H, cfg.N, cfg.d, dtype=torch.bfloat16, device=dev)
     ws = torch.empty(sla.sla_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -502,7 +697,7 @@ def main():
     clock_path = args.clocks_csv
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local, clock_path) as clk:
+    with ClockSampler(local, None) as clk:
         time.sleep(0.3)
         t0.record(stream)
         for s in range(args.steps):
@@ -530,15 +725,28 @@ def main():
         graph.replay()
     torch.cuda.synchronize()
     barrier()
+    # A soak of replays back to back (about --soak-s seconds) runs right before the K
+    # timed replays, under the same clock sampler: the timed steps run on a GPU at its
+    # sustained clock, and the sampler sees tens of samples of that load.
+    n_soak = max(1, int(args.soak_s * 1e3 / max(ms_eager, 1e-3))) if args.soak_s > 0 else 0
+    s0 = torch.cuda.Event(enable_timing=True)
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local, None) as clk2:
-        time.sleep(0.2)
+    with ClockSampler(local, clock_path) as clk2:
+        time.sleep(0.05)
+        s0.record(stream)
+        for _ in range(n_soak):
+            graph.replay()
         g0.record(stream)
         for _ in range(args.steps):
             graph.replay()
         g1.record(stream)
         torch.cuda.synchronize()
     barrier()
+    soak = None
+    if n_soak:
+        (soak_ms,) = max_over_ranks(dist, dev, s0.elapsed_time(g0) / n_soak)
+        soak = {"replays": n_soak, "ms_per_replay": soak_ms,
+                "what": "graph replays back to back right before the timed steps (clocks sampled over both)"}
     st, detail = sla.sla_check_device_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st} detail {detail}")
@@ -586,6 +794,25 @@ def main():
         del qp, order
     stage_ms = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
                 for i, n in enumerate(names)}
+    if shard_info is not None and args.shard_gather and dist is not None:
+        # the sharded layer as a caller that needs every head on every rank runs it:
+        # the local layer, then the all_gather of the outputs back into head order
+        def shard_step():
+            sla.sla_forward(q, k, v, w_p, w_g, cfg, out, None, ws)
+            return sh.all_gather_heads(out, full_cfg, shard.plan, rank, dist)
+        for _ in range(args.warmup):
+            shard_step()
+        torch.cuda.synchronize()
+        barrier()
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for _ in range(args.steps):
+            shard_step()
+        h1.record(stream)
+        torch.cuda.synchronize()
+        (sg_ms,) = max_over_ranks(dist, dev, h0.elapsed_time(h1) / args.steps)
+        shard_info["with_gather_ms_per_step"] = sg_ms
+        shard_info["with_gather"] = "eager sla_forward on the local heads + all_gather_heads (NCCL), max over ranks"
 
     # end to end: pinned host inputs -> device, layer, output -> host
     if shard_info is None:
@@ -666,26 +893,26 @@ def main():
         fk = stages["sparse_flash"]
         roof["flash"] = {"achieved": fk["achieved"], "frac": fk["achieved"] / peaks["bf16"]}
 
-    clocks = clk.summary()
-    c2 = clk2.summary()
-    if c2.get("sm_mhz") is not None and clocks.get("sm_mhz") is not None:
-        clocks["sm_mhz_graph_replays"] = c2["sm_mhz"]
-        clocks["reasons"] = sorted(set(clocks["reasons"]) | set(c2["reasons"]))
+    # clocks of the soak and the timed graph replays (the value's region); the eager
+    # per-stage steps' own samples are kept beside them
+    clocks = clk2.summary()
+    c1 = clk.summary()
+    if c1.get("sm_mhz") is not None and clocks.get("sm_mhz") is not None:
+        clocks["sm_mhz_eager_steps"] = c1["sm_mhz"]
+        clocks["reasons"] = sorted(set(clocks["reasons"]) | set(c1["reasons"]))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak" if shard_info is None else "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": full_cfg.name, "B": full_cfg.B, "H": full_cfg.H, "H_kv": full_cfg.H_kv,
-                   "N": full_cfg.N, "N_valid": full_cfg.N_valid, "d": full_cfg.d, "k_h": full_cfg.k_h,
-                   "k_l": full_cfg.k_l, "has_proj": full_cfg.has_proj, "has_gate": full_cfg.has_gate,
-                   "parallelism": f"replicas x{world}" if shard_info is None else f"heads x{world}",
-                   "l2": f"inputs (Q,K,V {(cfg.B * (cfg.H + 2 * cfg.H_kv) * cfg.N * cfg.d * 2) / 1e6:.0f} MB) larger "
-                         "than the 126 MB L2; no flush"},
+        "config": dict(config_keys(full_cfg, "replicas" if shard_info is None else f"heads x{world}"),
+                       l2=f"inputs (Q,K,V {(cfg.B * (cfg.H + 2 * cfg.H_kv) * cfg.N * cfg.d * 2) / 1e6:.0f} MB) "
+                          "larger than the 126 MB L2; no flush"),
         "ms_per_layer": ms_step,
         "per_replay_ms": {"warm_median": warm_med, "cold_median": cold_med, "reps": reps,
                           "cold": "256 MB written before each timed replay (L2 holds none of the layer's data)"},
         "ms_per_step_eager": ms_eager,
+        "soak": soak,
         "launch": "CUDA graph replay of one captured sla_forward call (ms_per_step_eager: direct calls)",
         "roofline": roof,
         "head_shard": shard_info,
@@ -704,13 +931,28 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of float64 oracle work on the host cores
-        units = sample_units(full_cfg, 512, n_heads=4)
-        t, n = oracle_sample(full_cfg, x, units, budget_s=20.0)
-        cv = (n / units_total(full_cfg)) * full_cfg.dense_flops() / t / 1e12
+        heads = sample_heads(full_cfg, 4)
+        r = oracle_sample(full_cfg, x, heads, 128, budget_s=20.0)
+        cv = full_cfg.dense_flops() / r["full_layer_s"] / 1e12
         line["cpu_baseline"] = {"value": cv, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-                                "sample": f"{n} (head, query block) units of {units_total(full_cfg)} from "
-                                          f"4 heads in {t:.1f} s (stops after 20 s); throughput "
-                                          f"scaled by unit count"}
+                                "sample": f"{r['heads']} heads' set-up (routing, linear states) and {r['units']} "
+                                          f"of their query blocks in {r['seconds']:.1f} s (stops after 20 s); "
+                                          f"the whole layer extrapolated from the measured set-up "
+                                          f"({r['setup_s_per_head']:.2f} s per head) and per-unit "
+                                          f"({r['unit_s'] * 1e3:.1f} ms) times",
+                                "full_layer_s": r["full_layer_s"]}
+        # the GPU's routing against the oracle's on the sampled heads (near-tie rows counted)
+        rows = full_cfg.H if full_cfg.mode == wl.MODE_THREEWAY else full_cfg.H_kv
+        mask = torch.empty((full_cfg.B, rows, full_cfg.nqb, full_cfg.nkb), dtype=torch.int8, device=dev)
+        if shard_info is None:
+            sla.sla_forward(q, k, v, w_p, w_g, cfg, out, mask, ws)
+            st, detail = sla.sla_check_device_status(ws)
+            if st != 0:
+                raise RuntimeError(f"device status {st} detail {detail}")
+            m_host = mask.cpu().numpy()
+            line["routing"] = routing_report(full_cfg, r["layer"], m_host, r_heads(r, heads))
+            if full_cfg.mode == wl.MODE_THREEWAY:
+                line["linear_branch_cost"] = linear_branch_cost(full_cfg, m_host)
     if dist is not None:
         dist.destroy_process_group()
     if rank == 0:
