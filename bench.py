@@ -68,15 +68,14 @@ def stage_model(c: wl.LayerConfig) -> dict:
     bf = 2
     m = {}
     m["pool"] = ("hbm", (B * H + B * Hkv) * Nv * d * bf + (B * H + B * Hkv) * nb * d * 8)
+    if c.mode == wl.MODE_THREEWAY and (nb - c.k_h - c.k_l > 0 or c.linear_all):
+        # phi(Q) (bf16) and, with a gate, g_t (fp32) for the linear branch
+        m["pool"] = ("hbm", m["pool"][1] + B * H * Nv * d * bf + (B * H * Nv * 4 if c.has_gate else 0))
     # float64 products q_bar . k_bar on the FP64 tensor path (mma.sync m8n8k4): every (i, j)
     # in three-way mode, the candidates j < i in top-n mode
     pairs = nb * nb if c.mode == wl.MODE_THREEWAY else nb * (nb - 1) // 2
     m["pooled_scores"] = ("fp64", 2.0 * B * H * pairs * d)
     if c.mode == wl.MODE_THREEWAY:
-        # the fused router (when a tile's score rows fit in shared memory): pooled keys,
-        # then one kernel for query pooling, the float64 scores (its bound) and classify
-        m["pool_keys"] = ("hbm", B * Hkv * Nv * d * bf + B * Hkv * nb * d * 8)
-        m["route"] = ("fp64", 2.0 * B * H * nb * nb * d)
         marg = nb - c.k_h - c.k_l
         m["classify"] = ("hbm", B * H * nb * nb * 8 + B * H * nb * nb * (1 + (2 if marg else 0))
                          + B * H * nb * c.k_h * 4)
@@ -113,8 +112,6 @@ def stage_model(c: wl.LayerConfig) -> dict:
             m["sparse_flash_cmp"] = ("tensor", 4.0 * d * B * H * cmp_pairs)
             m["sparse_flash_slc"] = ("tensor", 4.0 * d * B * H * slc)
             m["sparse_flash_win"] = ("tensor", 4.0 * d * B * H * win)
-            # reads q and the three branch outputs, writes O
-            m["branch_combine"] = ("hbm", 5 * B * H * Nv * d * bf)
     return m
 
 
@@ -137,8 +134,6 @@ def backward_stage_model(c: wl.LayerConfig) -> dict:
     m = {"bwd_columns": ("hbm", B * H * nb * c.k_h * 4 + 2 * B * H * nb * words * 4)}
     if lin:
         nqb_pad, nkb_pad = (nb + 127) // 128 * 128, (nb + 63) // 64 * 64
-        # reads q; writes phi(Q) (bf16) and g_t (fp32)
-        m["bwd_phi_gate"] = ("hbm", 2 * B * H * Nv * d * bf + (B * H * Nv * 4 if c.has_gate else 0))
         # reads phi(Q), q, O, dO, S'_i, Z_i (and g_t); writes the fp32 dq part, D_t, [dS'_i | dZ_i]
         m["bwd_linear"] = ("hbm", 4 * B * H * Nv * d * bf + B * H * nb * (d * d * bf + d * 4)
                            + B * H * Nv * 4 * (2 if c.has_gate else 1) + B * H * Nv * d * 4
@@ -612,7 +607,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--clocks-csv", default=None)
-    ap.add_argument("--soak-s", type=float, default=0.5,
+    ap.add_argument("--soak-s", type=float, default=0.3,
                     help="seconds of graph replays right before the timed replays (clock sampling)")
     ap.add_argument("--no-backward", action="store_true", help="skip the sla_backward measurement")
     ap.add_argument("--shard", default="none", choices=["none", "heads"],

@@ -13,7 +13,8 @@
 // Work unit = 128 query rows = two halves of 64 rows:
 //   - three-way mode, and top-n mode with an odd group size: query blocks
 //     2p and 2p+1 of one head; their block lists are merged and a tile that
-//     only one half needs is masked for the other half;
+//     only one half needs is masked for the other half (such tiles of the two
+//     halves alternate in the tile order, so both halves' warps stay busy);
 //   - top-n mode with an even group size: two query heads of one KV group at
 //     the same query block (identical lists, no masking waste).
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
@@ -56,6 +57,11 @@ struct FlashTcParams {
   int n_keys, nkt, kstride, kspan;
   int dense_tiles;      // top-n mode: every key tile up to the causal limit (no list)
   float scale_log2;
+  // NSA's window branch (NSAC): the compressed and selected branches' outputs [B*H][N][D]
+  // and the branch gates w_g [H][3][D] (null: every gate is 1)
+  const __nv_bfloat16* oc;
+  const __nv_bfloat16* os;
+  const __nv_bfloat16* w_g3;
 };
 
 constexpr int kTcThreads = 192;
@@ -85,7 +91,11 @@ struct TcLayout {
 // KMAP (NSA's compressed branch only): key c stands for token c * kstride + kspan in the causal
 // test, and the key tiles are every tile up to the causal limit (dense_tiles); compiled
 // separately so that the plain top-n kernel keeps its registers.
-template <int D, bool TOPN, bool FUSE, bool KMAP>
+// NSAC (NSA's window branch, the last of the three): the epilogue writes the layer's
+// output O = g_c o_c + g_s o_s + g_w o_w, with this branch's o_w taken from TMEM in
+// fp32, the other two read from the buffers the earlier launches wrote, and the gates
+// g_b = sigmoid(q_t . w_g[h][b]) from the Q row still in shared memory.
+template <int D, bool TOPN, bool FUSE, bool KMAP, bool NSAC = false>
 __global__ void __launch_bounds__(kTcThreads, 2)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
@@ -100,8 +110,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     return;
   }
 
-  // the four block bitmaps (act0, act1, sel0, sel1) only live during set-up, in
-  // the K/V ring before its first load
+  // the four block bitmaps (act0, act1, sel0, sel1) and the union of the two
+  // halves' blocks in block order only live during set-up, in the K/V ring before
+  // its first load
   uint32_t* words = reinterpret_cast<uint32_t*>(smem + L::kOffKV);
   uint32_t* mlist = reinterpret_cast<uint32_t*>(smem + L::kOffList);
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
@@ -223,6 +234,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   }
   __syncthreads();
   if (warp == 0) {
+    // the merge writes the union in block order into the free ring area after the
+    // bitmaps; the reorder below moves it to mlist
+    uint32_t* ulist = words + 4 * prm.words;
     int base = 0;
     for (int w0 = 0; w0 < prm.words; w0 += 32) {
       const int w = w0 + lane;
@@ -243,15 +257,56 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         any &= any - 1;
         const uint32_t m = 1u << bit;
         if (pos < prm.list_cap)
-          mlist[pos] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u) |
+          ulist[pos] = (uint32_t)(w * 32 + bit) | ((a0 & m) ? 1u << 16 : 0u) | ((a1 & m) ? 1u << 17 : 0u) |
                        ((s0 & m) ? 1u << 18 : 0u) | ((s1 & m) ? 1u << 19 : 0u);
         ++pos;
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
+    const int tm = base < prm.list_cap ? base : prm.list_cap;
+    __syncwarp();
+    // Tile order. A tile that only one half needs keeps the other half's warps idle
+    // (they only store zero P rows), so such tiles of the two halves alternate: the
+    // two halves' softmax warps then work on consecutive tiles at the same time (both
+    // S buffers are in flight). The rest of the longer exclusive run follows, then the
+    // tiles both halves need. Online softmax does not depend on the order.
+    int n0 = 0, n1 = 0;
+    for (int e0 = 0; e0 < tm; e0 += 32) {
+      const int e = e0 + lane;
+      const uint32_t v = e < tm ? ulist[e] : 0u;
+      const bool a0 = (v >> 16) & 1u, a1 = (v >> 17) & 1u;
+      n0 += __popc(__ballot_sync(0xffffffffu, e < tm && a0 && !a1));
+      n1 += __popc(__ballot_sync(0xffffffffu, e < tm && a1 && !a0));
+    }
+    const int pairs = n0 < n1 ? n0 : n1, nex = n0 + n1;
+    int r0 = 0, r1 = 0, rs = 0;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int e0 = 0; e0 < tm; e0 += 32) {
+      const int e = e0 + lane;
+      const uint32_t v = e < tm ? ulist[e] : 0u;
+      const bool a0 = (v >> 16) & 1u, a1 = (v >> 17) & 1u;
+      const bool c0 = e < tm && a0 && !a1, c1 = e < tm && a1 && !a0, cs = e < tm && a0 && a1;
+      const uint32_t b0 = __ballot_sync(0xffffffffu, c0), b1 = __ballot_sync(0xffffffffu, c1),
+                     bs = __ballot_sync(0xffffffffu, cs);
+      int pos = -1;
+      if (c0) {
+        const int r = r0 + __popc(b0 & below);
+        pos = r < pairs ? 2 * r : pairs + r;
+      } else if (c1) {
+        const int r = r1 + __popc(b1 & below);
+        pos = r < pairs ? 2 * r + 1 : pairs + r;
+      } else if (cs) {
+        pos = nex + rs + __popc(bs & below);
+      }
+      if (pos >= 0 && pos < tm) mlist[pos] = v;
+      r0 += __popc(b0);
+      r1 += __popc(b1);
+      rs += __popc(bs);
+    }
     if (lane == 0) {
-      if (base > prm.list_cap) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
-      misc[1] = base < prm.list_cap ? base : prm.list_cap;
+      // every entry belongs to one of the three classes; anything else is a broken merge
+      if (base > prm.list_cap || nex + rs != tm) report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
+      misc[1] = nex + rs == tm ? tm : 0;
     }
   }
   tc::fence_before_sync();
@@ -627,6 +682,69 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         *abort = 1;
         report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
       }
+    } else if (NSAC && valid_h[hf]) {
+      // NSA's gated sum of the three branches; padding rows are zero
+      const bool live = ok && t < prm.n_valid;
+      const float inv = (live && T > 0 && l_sum > 0.f) ? 1.f / l_sum : 0.f;
+      float g[3] = {1.f, 1.f, 1.f};
+      if (prm.w_g3 != nullptr && live) {
+        const __nv_bfloat16* wg = prm.w_g3 + (size_t)(bh_h[hf] % prm.H) * 3 * D;
+        float dot[3] = {0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int p = 0; p < NP; ++p) {
+          const uint4* qrow = reinterpret_cast<const uint4*>(smem + L::kOffQ + p * 16384 + r * 128);
+#pragma unroll 2
+          for (int c = 0; c < 8; ++c) {
+            const uint4 u = qrow[c ^ (r & 7)];
+            const uint32_t uq[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int b = 0; b < 3; ++b) {
+              const uint4 w = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)b * D + p * 64 + c * 8));
+              const uint32_t uw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 fq = unpack_bf16(uq[e]), fw = unpack_bf16(uw[e]);
+                dot[b] = fmaf(fq.x, fw.x, fmaf(fq.y, fw.y, dot[b]));
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < 3; ++b) g[b] = 1.f / (1.f + __expf(-dot[b]));
+      }
+      const size_t rowoff = ((size_t)bh_h[hf] * prm.N + t) * D;
+      const uint4* oc4 = reinterpret_cast<const uint4*>(prm.oc + rowoff);
+      const uint4* os4 = reinterpret_cast<const uint4*>(prm.os + rowoff);
+      uint4* dst = reinterpret_cast<uint4*>(prm.o + rowoff);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (ok && T > 0) {
+          tc::tmem_ld32(tO + 32 * c, ov);
+          tc::tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = 0u;
+        }
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint4 res = make_uint4(0u, 0u, 0u, 0u);
+          if (live) {
+            const uint4 a4 = oc4[4 * c + q8], b4 = os4[4 * c + q8];
+            const uint32_t ua[4] = {a4.x, a4.y, a4.z, a4.w}, ub[4] = {b4.x, b4.y, b4.z, b4.w};
+            uint32_t pw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 fa = unpack_bf16(ua[e]), fb = unpack_bf16(ub[e]);
+              const int j = 8 * q8 + 2 * e;
+              pw[e] = pack_bf16(g[0] * fa.x + g[1] * fb.x + g[2] * (__uint_as_float(ov[j]) * inv),
+                                g[0] * fa.y + g[1] * fb.y + g[2] * (__uint_as_float(ov[j + 1]) * inv));
+            }
+            res = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+          }
+          dst[4 * c + q8] = res;
+        }
+      }
     } else if (valid_h[hf]) {
       // epilogue: O / l -> bf16 rows (padding tokens and empty rows are zero)
       const float inv = (ok && T > 0 && l_sum > 0.f && t < prm.n_valid) ? 1.f / l_sum : 0.f;
@@ -672,7 +790,7 @@ static bool make_map(CUtensorMap* m, const void* base, int heads, int n_rows, in
 // branch 0: the layer's sparse branch. NSA's branches (top-n mode with nsa_branches), each
 // written to its own buffer: 1 compressed (keys: the compressed K, V; every tile up to the
 // causal limit), 2 selected (the selected blocks only), 3 window (the window only).
-template <int D, bool TOPN, bool FUSE, bool KMAP = false>
+template <int D, bool TOPN, bool FUSE, bool KMAP = false, bool NSAC = false>
 static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStream_t s) {
   using L = TcLayout<D>;
   const sla_config& c = p.c;
@@ -697,9 +815,12 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
   prm.list = a.crit;
   // the sparse branch is the output, or the fused epilogue writes it; NSA's branches
   // each write their own buffer
-  prm.o = branch == 0 ? a.out
-                      : reinterpret_cast<__nv_bfloat16*>(a.ws + (branch == 1 ? p.off_oc : branch == 2 ? p.off_os
-                                                                                                   : p.off_ow));
+  // NSA's window branch (the last) writes the gated sum of the three into the output
+  prm.o = (branch == 0 || branch == 3) ? a.out
+                                       : reinterpret_cast<__nv_bfloat16*>(a.ws + (branch == 1 ? p.off_oc : p.off_os));
+  prm.oc = branch == 3 ? reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_oc) : nullptr;
+  prm.os = branch == 3 ? reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_os) : nullptr;
+  prm.w_g3 = branch == 3 && c.has_gate ? a.w_g : nullptr;
   prm.zs = FUSE ? reinterpret_cast<const float*>(a.ws + p.off_zs) : nullptr;
   prm.gate = FUSE && c.has_gate ? reinterpret_cast<const float*>(a.ws + p.off_gate) : nullptr;
   prm.lse = branch == 0 ? reinterpret_cast<float*>(a.ws + p.off_lse) : nullptr;
@@ -726,10 +847,11 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
   if (prm.list_cap < 1) prm.list_cap = 1;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
   int smem = L::kOffList + prm.list_cap * 4;
-  if (4 * prm.words * 4 > kSlots * L::kSlotBytes) return cudaErrorInvalidValue;  // bitmaps in the ring
+  // the set-up bitmaps and the block-order union live in the ring before its first load
+  if ((4 * prm.words + prm.list_cap) * 4 > kSlots * L::kSlotBytes) return cudaErrorInvalidValue;
   // at most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN, FUSE, KMAP>,
+  cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<D, TOPN, FUSE, KMAP, NSAC>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int units;
@@ -737,7 +859,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
     units = c.B * c.H_kv * p.nqb * (p.group / 2);
   else
     units = c.B * c.H * prm.npairs;
-  flash_tc_kernel<D, TOPN, FUSE, KMAP><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, mf, prm);
+  flash_tc_kernel<D, TOPN, FUSE, KMAP, NSAC><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, mf, prm);
   return cudaGetLastError();
 }
 
@@ -757,6 +879,9 @@ cudaError_t launch_flash_nsa(const Plan& p, const Args& a, int branch, cudaStrea
   if (branch == 1)  // compressed keys: the key-to-token map and the dense tile range
     return p.c.d == 128 ? launch_tc<128, true, false, true>(p, a, branch, s)
                         : launch_tc<64, true, false, true>(p, a, branch, s);
+  if (branch == 3)  // the window branch, with the gated sum of the three branches
+    return p.c.d == 128 ? launch_tc<128, true, false, false, true>(p, a, branch, s)
+                        : launch_tc<64, true, false, false, true>(p, a, branch, s);
   return p.c.d == 128 ? launch_tc<128, true, false>(p, a, branch, s) : launch_tc<64, true, false>(p, a, branch, s);
 }
 

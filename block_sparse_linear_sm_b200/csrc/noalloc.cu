@@ -107,10 +107,7 @@ extern "C" SLA_API sla_status sla_route_noalloc(const void* q, const void* k, co
   cudaStream_t s = (cudaStream_t)stream;
   // the array keeps the previous call's contents: the status word must start at zero
   if (cudaMemsetAsync(a.status, 0, 8, s) != cudaSuccess) return SLA_ERR_CUDA;
-  if (launch_pool(p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
-  if (launch_scores(p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
-  const cudaError_t e = threeway ? launch_classify(p, a, false, s) : launch_select(p, a, s);
-  return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+  return route_stages(p, a, s) == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
 }
 
 extern "C" SLA_API sla_status sla_route_noalloc_status(void* stream, int32_t* detail) {

@@ -8,8 +8,8 @@
 // summed with per-head gates g_b = sigmoid(q . w_g[h][b]) (g_b = 1 without gates).
 // The three attentions run in the sparse flash kernel (flash_tc.cu): the compressed
 // branch over the compressed keys, every tile up to the causal limit c * stride +
-// length - 1 <= t. This file holds the compression and the gated combine, both
-// HBM-bound, one warp per output row.
+// length - 1 <= t; the window branch's epilogue writes the gated sum. This file holds
+// the compression, HBM-bound, one warp per compressed row.
 #include "common.cuh"
 
 namespace sla {
@@ -59,60 +59,6 @@ cudaError_t launch_compress(const Plan& p, const Args& a, cudaStream_t s) {
   else
     compress_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(a.k, a.v, kc, vc, rows, c.N, p.n_cmp, p.ncmp_pad,
                                                          c.cmp_block, c.cmp_stride);
-  return cudaGetLastError();
-}
-
-// out[row] = sum_b g_b o_b[row], g_b = sigmoid(q . w_g[h][b]) or 1; padding rows 0.
-template <int D>
-__global__ void branch_combine_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ oc,
-                                      const __nv_bfloat16* __restrict__ os, const __nv_bfloat16* __restrict__ ow,
-                                      const __nv_bfloat16* __restrict__ w_g, __nv_bfloat16* __restrict__ out,
-                                      int64_t rows, int N, int n_valid, int H) {
-  constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t r = w0; r < rows; r += nw) {
-    const int t = (int)(r % N);
-    const int h = (int)((r / N) % H);
-    const size_t off = (size_t)r * D + lane * E;
-    float g[3] = {1.f, 1.f, 1.f};
-    if (w_g != nullptr) {
-      float qv[E], dot[3] = {0.f, 0.f, 0.f};
-#pragma unroll
-      for (int e = 0; e < E; ++e) qv[e] = __bfloat162float(q[off + e]);
-#pragma unroll
-      for (int b = 0; b < 3; ++b) {
-        const __nv_bfloat16* wv = w_g + ((size_t)h * 3 + b) * D + lane * E;
-#pragma unroll
-        for (int e = 0; e < E; ++e) dot[b] = fmaf(qv[e], __bfloat162float(wv[e]), dot[b]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot[b] += __shfl_xor_sync(0xffffffffu, dot[b], o);
-        g[b] = 1.f / (1.f + __expf(-dot[b]));
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float x = g[0] * __bfloat162float(oc[off + e]) + g[1] * __bfloat162float(os[off + e]) +
-                      g[2] * __bfloat162float(ow[off + e]);
-      out[off + e] = __float2bfloat16(t < n_valid ? x : 0.f);
-    }
-  }
-}
-
-cudaError_t launch_branch_combine(const Plan& p, const Args& a, cudaStream_t s) {
-  const sla_config& c = p.c;
-  const int64_t rows = (int64_t)c.B * c.H * c.N;
-  int64_t blocks = (rows + 7) / 8;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  const auto* oc = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_oc);
-  const auto* os = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_os);
-  const auto* ow = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_ow);
-  const __nv_bfloat16* wg = c.has_gate ? a.w_g : nullptr;
-  if (c.d == 128)
-    branch_combine_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(a.q, oc, os, ow, wg, a.out, rows, c.N, c.N_valid, c.H);
-  else
-    branch_combine_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(a.q, oc, os, ow, wg, a.out, rows, c.N, c.N_valid, c.H);
   return cudaGetLastError();
 }
 

@@ -156,16 +156,21 @@ cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s) {
   dim3 grid(p.nqb, c.B * c.H + c.B * c.H_kv);
   pool_kernel<<<grid, c.d / 2, 0, s>>>(a.q, a.k, qbar, kbar, c.B * c.H, c.N, c.N_valid, c.d,
                                        p.nqb, phiq, gate ? a.w_g : nullptr, gate, c.H);
-  if (c.cos_filter) {
-    // part of routing: the filter flags feed classify / select
-    const int rows = c.B * c.H_kv * p.nkb;
-    uint8_t* kflag = reinterpret_cast<uint8_t*>(a.ws + p.off_kflag);
-    const int blocks = (rows + 3) / 4;  // four warps (blocks) per CTA
-    if (c.d == 128)
-      kcos_kernel<128><<<blocks, 128, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
-    else
-      kcos_kernel<64><<<blocks, 128, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
-  }
+  cudaError_t e = cudaGetLastError();
+  // part of routing: the filter flags feed classify / select
+  if (e != cudaSuccess || !c.cos_filter) return e;
+  return launch_kcos(p, a, s);
+}
+
+cudaError_t launch_kcos(const Plan& p, const Args& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  const int rows = c.B * c.H_kv * p.nkb;
+  uint8_t* kflag = reinterpret_cast<uint8_t*>(a.ws + p.off_kflag);
+  const int blocks = (rows + 3) / 4;  // four warps (blocks) per CTA
+  if (c.d == 128)
+    kcos_kernel<128><<<blocks, 128, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
+  else
+    kcos_kernel<64><<<blocks, 128, 0, s>>>(a.k, kflag, rows, p.nkb, c.N, c.N_valid, (double)c.cos_theta);
   return cudaGetLastError();
 }
 
@@ -400,28 +405,248 @@ __device__ void warp_compact(const uint8_t* flags, int n, uint8_t bit, uint8_t w
   }
 }
 
+// ---------------------------------------------------------------------------
+// Both class boundaries of a three-way row: exact order statistics of the keys
+// (score descending, lower block index first on equal scores).
+// ---------------------------------------------------------------------------
+constexpr int kClsBins = 512;  // histogram digits (9 bits per radix level)
+
+__device__ __forceinline__ double order_key_value(unsigned long long k) {
+  const unsigned long long b = (k & 0x8000000000000000ull) ? (k & 0x7FFFFFFFFFFFFFFFull) : ~k;
+  return __longlong_as_double((long long)b);
+}
+
+// One level of the radix select over the keys of the interval [a, b] (as key - a,
+// unsigned): 512 digits of (u - a) >> shift. Returns the digit holding the r-th
+// largest of those keys (r >= 1, counting from the top) and the number of keys in
+// the interval above that digit. hist: this warp's 512 counters.
+struct Level {
+  int digit;
+  int above;   // keys of the interval in higher digits
+  int count;   // keys in the digit
+};
+
+__device__ __forceinline__ Level radix_level(const unsigned long long* keys, int n, unsigned long long a,
+                                             unsigned long long b, int shift, int r, unsigned* hist) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int u = 0; u < kClsBins / 32; ++u) hist[lane + 32 * u] = 0u;
+  __syncwarp();
+  for (int j = lane; j < n; j += 32) {
+    const unsigned long long kk = keys[j];
+    if (kk >= a && kk <= b) atomicAdd(&hist[(unsigned)((kk - a) >> shift)], 1u);
+  }
+  __syncwarp();
+  // lane l owns digits 511 - 16 l .. 496 - 16 l (descending)
+  unsigned cnt[16], tot = 0;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    cnt[u] = hist[kClsBins - 1 - 16 * lane - u];
+    tot += cnt[u];
+  }
+  unsigned incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)r);
+  const int owner = __ffs(hit) - 1;  // r <= keys in the interval: some lane reaches it
+  Level lv{0, 0, 0};
+  if (lane == owner) {
+    unsigned run = incl - tot;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      if (run + cnt[u] >= (unsigned)r) {
+        lv.digit = kClsBins - 1 - 16 * lane - u;
+        lv.above = (int)run;
+        lv.count = (int)cnt[u];
+        break;
+      }
+      run += cnt[u];
+    }
+  }
+  lv.digit = __shfl_sync(0xffffffffu, lv.digit, owner);
+  lv.above = __shfl_sync(0xffffffffu, lv.above, owner);
+  lv.count = __shfl_sync(0xffffffffu, lv.count, owner);
+  __syncwarp();
+  return lv;
+}
+
+// The c-th element (1 <= c <= n) of the order "key descending, lower index first"
+// of keys[0..n): returns its key and index. Exact: the interval holding it is
+// narrowed one 9-bit digit at a time until it is a single key value, and among
+// equal keys the (r)-th lowest index is taken.
+__device__ void select_rank(const unsigned long long* keys, int n, int c, unsigned long long kmin,
+                            unsigned long long kmax, unsigned* hist, unsigned long long* key_out, int* idx_out) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long a = kmin, b = kmax;
+  int r = c;
+  while (a != b) {
+    const unsigned long long span = b - a;
+    const int bits = 64 - __clzll((long long)span);  // span < 2^bits
+    const int shift = bits > 9 ? bits - 9 : 0;
+    const Level lv = radix_level(keys, n, a, b, shift, r, hist);
+    r -= lv.above;
+    const unsigned long long lo = a + ((unsigned long long)lv.digit << shift);
+    const unsigned long long hi_excl = shift >= 64 ? 0ull : ((unsigned long long)(lv.digit + 1) << shift);
+    const unsigned long long hi = (hi_excl == 0ull || a + hi_excl - 1 < a || a + hi_excl - 1 > b) ? b : a + hi_excl - 1;
+    a = lo;
+    b = hi;
+    if (shift == 0) break;  // one key value per digit
+  }
+  // a == b: the r-th lowest index among the keys equal to a
+  int seen = 0, idx = -1;
+  for (int j0 = 0; j0 < n && idx < 0; j0 += 32) {
+    const int j = j0 + lane;
+    const bool eq = j < n && keys[j] == a;
+    const unsigned m = __ballot_sync(0xffffffffu, eq);
+    const int cnt = __popc(m);
+    if (seen + cnt >= r) {
+      // the (r - seen)-th set bit of m
+      unsigned mm = m;
+      for (int q = 1; q < r - seen; ++q) mm &= mm - 1;
+      idx = j0 + __ffs(mm) - 1;
+    }
+    seen += cnt;
+  }
+  *key_out = a;
+  *idx_out = idx;
+}
+
+// Both class boundaries of one row in one pass. Digit 0 holds the filtered blocks
+// (-inf), digits 1..511 split [min, max] of the finite scores linearly (a monotone
+// map of the value, so the order of the digits is the order of the scores). The
+// boundary digit of each boundary is found from the histogram; the keys in it are
+// ranked exactly by comparing them with each other (lower block index first on
+// equal keys). A digit with more than 32 keys falls back to select_rank.
+struct Boundary {
+  unsigned long long key;
+  int idx;
+};
+
+__device__ void select_two(const unsigned long long* keys, int n, const int (&cnt)[2], unsigned long long kmin_f,
+                           unsigned long long kmax_f, bool any_finite, unsigned long long kmin, unsigned long long kmax,
+                           unsigned* hist, Boundary (&out)[2]) {
+  const int lane = threadIdx.x & 31;
+  const double smin = any_finite ? order_key_value(kmin_f) : 0.0, smax = any_finite ? order_key_value(kmax_f) : 0.0;
+  double fac = smax > smin ? 510.0 / (smax - smin) : 0.0;
+  if (!(fac < 1e300)) fac = 0.0;  // a subnormal range: one digit (its keys are then ranked exactly)
+  auto digit = [&](unsigned long long kk) -> int {
+    const double v = order_key_value(kk);
+    if (v == -INFINITY) return 0;
+    int d = 1 + (int)((v - smin) * fac);
+    return d > kClsBins - 1 ? kClsBins - 1 : (d < 1 ? 1 : d);
+  };
+#pragma unroll
+  for (int u = 0; u < kClsBins / 32; ++u) hist[lane + 32 * u] = 0u;
+  __syncwarp();
+  for (int j = lane; j < n; j += 32) atomicAdd(&hist[digit(keys[j])], 1u);
+  __syncwarp();
+  // lane l owns digits 511 - 16 l .. 496 - 16 l (descending)
+  unsigned c16[16], tot = 0;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    c16[u] = hist[kClsBins - 1 - 16 * lane - u];
+    tot += c16[u];
+  }
+  unsigned incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int bdig[2], need[2], bcnt[2];
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const int r = cnt[b];
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)r);
+    const int owner = __ffs(hit) - 1;
+    int dg = 0, above = 0, inb = 0;
+    if (lane == owner) {
+      unsigned run = incl - tot;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (run + c16[u] >= (unsigned)r) {
+          dg = kClsBins - 1 - 16 * lane - u;
+          above = (int)run;
+          inb = (int)c16[u];
+          break;
+        }
+        run += c16[u];
+      }
+    }
+    bdig[b] = __shfl_sync(0xffffffffu, dg, owner);
+    need[b] = r - __shfl_sync(0xffffffffu, above, owner);
+    bcnt[b] = __shfl_sync(0xffffffffu, inb, owner);
+  }
+  __syncwarp();
+  // candidates of each boundary digit, ranked among themselves
+  unsigned long long* ck = reinterpret_cast<unsigned long long*>(hist);  // 32 keys
+  int* ci = reinterpret_cast<int*>(hist + 64);                           // 32 indices
+#pragma unroll 1
+  for (int b = 0; b < 2; ++b) {
+    if (bcnt[b] > 32) {
+      select_rank(keys, n, cnt[b], kmin, kmax, hist, &out[b].key, &out[b].idx);
+      continue;
+    }
+    int base = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const bool is = j < n && digit(keys[j]) == bdig[b];
+      const unsigned m = __ballot_sync(0xffffffffu, is);
+      if (is) {
+        const int pos = base + __popc(m & ((1u << lane) - 1u));
+        ck[pos] = keys[j];
+        ci[pos] = j;
+      }
+      base += __popc(m);
+    }
+    __syncwarp();
+    const int c = bcnt[b];
+    int rank = 1 << 30;
+    unsigned long long mk = 0;
+    int mi = -1;
+    if (lane < c) {
+      mk = ck[lane];
+      mi = ci[lane];
+      rank = 0;
+      for (int t = 0; t < c; ++t) {
+        const unsigned long long ok = ck[t];
+        rank += (ok > mk || (ok == mk && ci[t] < mi)) ? 1 : 0;
+      }
+    }
+    const unsigned win = __ballot_sync(0xffffffffu, rank == need[b] - 1);
+    const int wl = win ? __ffs(win) - 1 : 0;
+    out[b].key = __shfl_sync(0xffffffffu, mk, wl);
+    out[b].idx = win ? __shfl_sync(0xffffffffu, mi, wl) : -1;
+    __syncwarp();
+  }
+}
+
 constexpr int kRouteWarps = 8;
 
+// per warp of the classify kernel: the row's keys, then the histogram / candidates
+__host__ __device__ inline size_t classify_warp_bytes(int nb) { return align_up((size_t)nb * 8, 16) + kClsBins * 4; }
+
 static int route_rows_per_cta(int nb) {
-  const size_t per = (size_t)nb * 8 + (size_t)nb + 1024 + 64;  // keys, flags, histogram
-  int r = (int)((96 * 1024) / per);
+  int r = (int)((96 * 1024) / classify_warp_bytes(nb));
   return r < 1 ? 1 : (r > kRouteWarps ? kRouteWarps : r);
 }
 
-static size_t route_smem(int nb, int rows) {
-  return (size_t)rows * ((size_t)nb * 8 + align_up((size_t)nb, 16) + 1024);
-}
+static size_t route_smem(int nb, int rows) { return (size_t)rows * classify_warp_bytes(nb); }
 
 // ---------------------------------------------------------------------------
-// three-way classification: one warp per (b, h, query block i).
-// flags bit 1: among the top k_h (critical); bit 2: among the top nb - k_l
-// (not negligible). Class = 2 critical, 1 marginal, 0 negligible.
+// three-way classification: one warp per (b, h, query block i). The k_h-th and
+// the (nb - k_l)-th block of the row's order are found exactly (select_two); a
+// block is critical when it ranks at or before the first, negligible when it ranks
+// after the second, marginal otherwise. Class = 2 critical, 1 marginal, 0 negligible.
 // ---------------------------------------------------------------------------
 __global__ void classify_kernel(const double* __restrict__ scores, int8_t* __restrict__ mask_out,
                                 int32_t* __restrict__ crit, int32_t* __restrict__ neg,
                                 __nv_bfloat16* __restrict__ mmask, int nb, int k_h, int k_l,
                                 int nkb_pad, int nqb_pad, int rows, int n_rows, int linear_all,
-                                const uint8_t* __restrict__ kflag, int H, int group) {
+                                const uint8_t* __restrict__ kflag, int H, int group, int* status) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = blockIdx.x * rows + w;  // over B*H*nqb_pad
@@ -435,34 +660,92 @@ __global__ void classify_kernel(const double* __restrict__ scores, int8_t* __res
     }
     return;
   }
-  unsigned char* base = smem + (size_t)w * ((size_t)nb * 8 + align_up((size_t)nb, 16) + 1024);
+  unsigned char* base = smem + (size_t)w * classify_warp_bytes(nb);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(base);
-  uint8_t* flags = base + (size_t)nb * 8;
-  unsigned* hist = reinterpret_cast<unsigned*>(base + (size_t)nb * 8 + align_up((size_t)nb, 16));
+  unsigned* hist = reinterpret_cast<unsigned*>(base + align_up((size_t)nb * 8, 16));
   const double* srow = scores + ((size_t)bh * nb + i) * nb;
+  // the score row lands in the key buffer with 16-byte copies, all in flight together
+  // (rows start on 16 bytes when nb is even; otherwise element by element)
+  {
+    double* dst = reinterpret_cast<double*>(keys);
+    if ((nb & 1) == 0) {
+      for (int e = lane; e < nb / 2; e += 32) cp_async16(smem_u32(dst + 2 * e), srow + 2 * e, 16);
+      cp_async_commit();
+      cp_async_wait<0>();
+    } else {
+      for (int j = lane; j < nb; j += 32) dst[j] = srow[j];
+    }
+    __syncwarp();
+  }
   // filtered key blocks (cos_filter) score -inf
   const uint8_t* kf = kflag ? kflag + ((size_t)(bh / H) * (H / group) + (bh % H) / group) * nb : nullptr;
+  unsigned long long kmin = ~0ull, kmax = 0ull, fmin = ~0ull, fmax = 0ull;
   for (int j = lane; j < nb; j += 32) {
-    keys[j] = order_key(kf && kf[j] ? -INFINITY : srow[j]);
-    flags[j] = 0;
+    const double v = kf && kf[j] ? -INFINITY : reinterpret_cast<const double*>(keys)[j];
+    const unsigned long long kk = order_key(v);
+    keys[j] = kk;
+    kmin = kk < kmin ? kk : kmin;
+    kmax = kk > kmax ? kk : kmax;
+    if (v != -INFINITY) {
+      fmin = kk < fmin ? kk : fmin;
+      fmax = kk > fmax ? kk : fmax;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o), c = __shfl_xor_sync(0xffffffffu, kmax, o);
+    kmin = a < kmin ? a : kmin;
+    kmax = c > kmax ? c : kmax;
+    a = __shfl_xor_sync(0xffffffffu, fmin, o);
+    c = __shfl_xor_sync(0xffffffffu, fmax, o);
+    fmin = a < fmin ? a : fmin;
+    fmax = c > fmax ? c : fmax;
   }
   __syncwarp();
-  warp_mark_top(keys, nb, k_h, hist, flags, 1);
-  warp_mark_top(keys, nb, nb - k_l, hist, flags, 2);
+  // the k_h-th block (last critical) and the (nb - k_l)-th (last non-negligible)
+  const bool c_some = k_h > 0, c_all = k_h >= nb;
+  const bool n_some = nb - k_l > 0, n_all = k_l == 0;
+  const int cnt2[2] = {c_some && !c_all ? k_h : 1, n_some && !n_all ? nb - k_l : 1};
+  Boundary bd[2];
+  select_two(keys, nb, cnt2, fmin, fmax, fmax >= fmin, kmin, kmax, hist, bd);
+  const unsigned long long c_key = bd[0].key, n_key = bd[1].key;
+  const int c_idx = (c_some && !c_all) ? bd[0].idx : -1, n_idx = (n_some && !n_all) ? bd[1].idx : -1;
+  if ((c_some && !c_all && c_idx < 0) || (n_some && !n_all && n_idx < 0))
+    if (lane == 0) report(status, SLA_ERR_DEVICE_CHECK, kDetailRouteSelect);
   const size_t rowoff = ((size_t)bh * nb + i) * nb;
-  if (mask_out)
-    for (int j = lane; j < nb; j += 32) {
-      const uint8_t f = flags[j];
-      mask_out[rowoff + j] = (f & 1) ? 2 : ((f & 2) ? 1 : 0);
+  int nc_w = 0, nn_w = 0;
+  int32_t* clist = crit && k_h > 0 ? crit + ((size_t)bh * nb + i) * k_h : nullptr;
+  int32_t* nlist = neg && k_l > 0 ? neg + ((size_t)bh * nb + i) * k_l : nullptr;
+  __nv_bfloat16* mrow = mmask ? mmask + ((size_t)bh * nqb_pad + i) * nkb_pad : nullptr;
+  const int jend = mrow ? nkb_pad : nb;
+  for (int j0 = 0; j0 < jend; j0 += 32) {
+    const int j = j0 + lane;
+    int cls = 0;
+    if (j < nb) {
+      const unsigned long long kk = keys[j];
+      const bool is_c = c_all || (c_some && (kk > c_key || (kk == c_key && j <= c_idx)));
+      const bool is_n = n_all || (n_some && (kk > n_key || (kk == n_key && j <= n_idx)));
+      cls = is_c ? 2 : (is_n ? 1 : 0);
+      if (mask_out) mask_out[rowoff + j] = (int8_t)cls;
     }
-  if (mmask) {
-    __nv_bfloat16* mrow = mmask + ((size_t)bh * nqb_pad + i) * nkb_pad;
-    for (int j = lane; j < nkb_pad; j += 32)
-      // the aggregation mask: the marginal blocks, or every block with linear_all
-      mrow[j] = __float2bfloat16(j < nb && (linear_all || flags[j] == 2) ? 1.f : 0.f);
+    // the aggregation mask: the marginal blocks, or every block with linear_all
+    if (mrow && j < nkb_pad) mrow[j] = __float2bfloat16(j < nb && (linear_all || cls == 1) ? 1.f : 0.f);
+    const unsigned bc = __ballot_sync(0xffffffffu, j < nb && cls == 2);
+    const unsigned bn = __ballot_sync(0xffffffffu, j < nb && cls == 0);
+    const unsigned below = (1u << lane) - 1u;
+    if (clist && j < nb && cls == 2) {
+      const int pos = nc_w + __popc(bc & below);
+      if (pos < k_h) clist[pos] = j;
+    }
+    if (nlist && j < nb && cls == 0) {
+      const int pos = nn_w + __popc(bn & below);
+      if (pos < k_l) nlist[pos] = j;
+    }
+    nc_w += __popc(bc);
+    nn_w += __popc(bn);
   }
-  if (crit && k_h > 0) warp_compact(flags, nb, 1, 1, crit + ((size_t)bh * nb + i) * k_h);
-  if (neg && k_l > 0) warp_compact(flags, nb, 2, 0, neg + ((size_t)bh * nb + i) * k_l);
+  if (lane == 0 && ((clist && nc_w != k_h) || (nlist && nn_w != k_l)))
+    report(status, SLA_ERR_DEVICE_CHECK, kDetailRouteSelect);
 }
 
 cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cudaStream_t s) {
@@ -482,7 +765,7 @@ cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cuda
                                                 c.k_l, p.nkb_pad, per_head, rows, n_rows, c.linear_all,
                                                 c.cos_filter ? reinterpret_cast<const uint8_t*>(a.ws + p.off_kflag)
                                                              : nullptr,
-                                                c.H, p.group);
+                                                c.H, p.group, a.status);
   return cudaGetLastError();
 }
 

@@ -97,7 +97,6 @@ bool make_plan(const sla_config* c, Plan* p) {
       p->off_vc = take(B * Hkv * (size_t)p->ncmp_pad * d * 2);
       p->off_oc = take(B * H * (size_t)c->N * d * 2);
       p->off_os = take(B * H * (size_t)c->N * d * 2);
-      p->off_ow = take(B * H * (size_t)c->N * d * 2);
     }
   }
   p->total = off;
@@ -110,7 +109,7 @@ static bool has_marginal(const Plan& p) { return p.nkb - p.c.k_h - p.c.k_l > 0 |
 
 // Stage list of a configuration.
 enum Stage { kPool, kScores, kClassify, kSelect, kState, kAggregate, kFlash, kCompress, kFlashCmp, kFlashSlc,
-             kFlashWin, kCombine };
+             kFlashWin };
 constexpr int kMaxStages = 12;
 
 static int stages_of(const Plan& p, Stage* out) {
@@ -126,12 +125,11 @@ static int stages_of(const Plan& p, Stage* out) {
     out[n++] = kFlash;  // with a linear branch its tail runs the layer's epilogue
   } else {
     out[n++] = kSelect;
-    if (p.c.nsa_branches) {  // NSA's three branches, then the gated sum
+    if (p.c.nsa_branches) {  // NSA's three branches; the last one sums them with their gates
       out[n++] = kCompress;
       out[n++] = kFlashCmp;
       out[n++] = kFlashSlc;
-      out[n++] = kFlashWin;
-      out[n++] = kCombine;
+      out[n++] = kFlashWin;  // its epilogue writes the gated sum of the three branches
     } else {
       out[n++] = kFlash;
     }
@@ -152,7 +150,6 @@ static const char* stage_name(Stage s) {
     case kFlashCmp: return "sparse_flash_cmp";
     case kFlashSlc: return "sparse_flash_slc";
     case kFlashWin: return "sparse_flash_win";
-    case kCombine: return "branch_combine";
   }
   return "?";
 }
@@ -170,9 +167,15 @@ static cudaError_t run_stage(Stage st, const Plan& p, const Args& a, cudaStream_
     case kFlashCmp: return launch_flash_nsa(p, a, 1, s);
     case kFlashSlc: return launch_flash_nsa(p, a, 2, s);
     case kFlashWin: return launch_flash_nsa(p, a, 3, s);
-    case kCombine: return launch_branch_combine(p, a, s);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t route_stages(const Plan& p, const Args& a, cudaStream_t s) {
+  cudaError_t e = launch_pool(p, a, s);
+  if (e == cudaSuccess) e = launch_scores(p, a, s);
+  if (e == cudaSuccess) e = p.c.mode == SLA_MODE_THREEWAY ? launch_classify(p, a, false, s) : launch_select(p, a, s);
+  return e;
 }
 
 static sla_status forward_impl(const void* q, const void* k, const void* v, const void* w_p,
@@ -334,7 +337,7 @@ static sla_status backward_impl(const void* q, const void* k, const void* v, con
   if (cfg->has_gate && (!w_g || !aligned(w_g, 16) || !dw_g || !aligned(dw_g, 16))) return SLA_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return SLA_ERR_WORKSPACE;
   if (!bws || !aligned(bws, 256) || bws_bytes < bp.total) return SLA_ERR_WORKSPACE;
-  BStage stages[8];
+  BStage stages[9];
   const int ns = bwd_stages_of(bp, stages);
   if (events && n_events != ns + 1) return SLA_ERR_INVALID_ARG;
   BwdArgs a;
@@ -400,10 +403,7 @@ sla_status sla_route(const void* q, const void* k, const sla_config* cfg, int8_t
   a.status = (int*)((char*)ws + p.off_status);
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(a.status, 0, 8, s) != cudaSuccess) return SLA_ERR_CUDA;
-  if (launch_pool(p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
-  if (launch_scores(p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
-  cudaError_t e = threeway ? launch_classify(p, a, false, s) : launch_select(p, a, s);
-  return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+  return route_stages(p, a, s) == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
 }
 
 sla_status sla_forward(const void* q, const void* k, const void* v, const void* w_p,
@@ -481,7 +481,7 @@ int32_t sla_backward_num_stages(const sla_config* cfg) {
   BwdPlan bp;
   make_plan(cfg, &p);
   make_bwd_plan(p, &bp);
-  BStage st[8];
+  BStage st[9];
   return bwd_stages_of(bp, st);
 }
 
@@ -491,7 +491,7 @@ const char* sla_backward_stage_name(const sla_config* cfg, int32_t s) {
   BwdPlan bp;
   make_plan(cfg, &p);
   make_bwd_plan(p, &bp);
-  BStage st[8];
+  BStage st[9];
   const int n = bwd_stages_of(bp, st);
   return (s >= 0 && s < n) ? bwd_stage_name(st[s]) : nullptr;
 }

@@ -16,6 +16,7 @@ constexpr int kMaxBlocks = 4096;  // nkb limit of the routing sort (N <= 262144)
 // Device status word: status[0] = sla_status code, status[1] = detail.
 enum DeviceDetail : int {
   kDetailFlashIndex = 101,      // flash kernel read a block index outside [0, nkb)
+  kDetailRouteSelect = 102,    // the exact class-boundary selection lost a block (broken invariant)
   kDetailFlashAlign = 103,     // shared-memory base not 1024-byte aligned
   kDetailTimeout = 200,
   kDetailSelftest = 300,       // the failure-detection self-test's wait ran out (expected)
@@ -36,7 +37,7 @@ struct Plan {
   // NSA's branches (top-n mode): compressed K, V [B*H_kv][ncmp_pad][d] and the three
   // branch outputs [B*H][N][d] (bf16)
   int n_cmp, ncmp_pad;
-  size_t off_kc, off_vc, off_oc, off_os, off_ow;
+  size_t off_kc, off_vc, off_oc, off_os;
 };
 
 bool make_plan(const sla_config* c, Plan* p);
@@ -64,6 +65,9 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, 
 
 // kernel launchers (return the launch error)
 cudaError_t launch_pool(const Plan& p, const Args& a, cudaStream_t s);
+cudaError_t launch_kcos(const Plan& p, const Args& a, cudaStream_t s);  // cos_filter flags
+// the routing stages alone (sla_route, sla_route_noalloc): lists and mask, no aggregation mask
+cudaError_t route_stages(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_scores(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_classify(const Plan& p, const Args& a, bool write_mmask, cudaStream_t s);
 cudaError_t launch_select(const Plan& p, const Args& a, cudaStream_t s);
@@ -72,7 +76,6 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_flash(const Plan& p, const Args& a, cudaStream_t s);
 cudaError_t launch_flash_nsa(const Plan& p, const Args& a, int branch, cudaStream_t s);  // 1 cmp, 2 slc, 3 win
 cudaError_t launch_compress(const Plan& p, const Args& a, cudaStream_t s);
-cudaError_t launch_branch_combine(const Plan& p, const Args& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // backward pass (three-way mode)

@@ -307,7 +307,7 @@ def test_nsa_branches_configuration():
     c = wl.preset("nsa_branches")
     assert sla.sla_validate_config(c) == sla.SLA_OK
     assert sla.sla_stage_names(c) == ["pool", "pooled_scores", "select_topn", "compress_kv", "sparse_flash_cmp",
-                                      "sparse_flash_slc", "sparse_flash_win", "branch_combine"]
+                                      "sparse_flash_slc", "sparse_flash_win"]
     # the three branch outputs and the compressed keys add to the workspace
     assert sla.sla_workspace_bytes(c) > sla.sla_workspace_bytes(wl.preset("nsa_causal"))
     # forward only; the gates belong to NSA's branches; no branches in the three-way mode
