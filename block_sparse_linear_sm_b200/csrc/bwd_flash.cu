@@ -26,6 +26,8 @@
 // the dQ / dV / dK products read them from there (A operand in TMEM).
 // Both kernels add the linear-branch part of the gradient (fp32 scratch) and
 // write the final bf16 rows.
+#include <cstring>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -66,6 +68,15 @@ cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cuda
                                                     entries, p.nqb, p.nkb, len, bp.words, topn ? 1 : 0, a.status);
   return cudaGetLastError();
 }
+
+// Kernel modes. kModeNsa (dQ) and kModeNsaTok / kModeNsaCmp (dK, dV) are NSA's three
+// branches (sparse attention survey, section 2: compressed, selected and window
+// attention, each its own softmax, summed with gates). Each branch b has its own row
+// log-sum-exp and D values; the gate is folded into the log-sum-exp (lse_b - log2 g_b),
+// so that the recomputed P is g_b P_b and dS = g_b P_b (dP - D_b) with D_b = dO . o_b:
+// the gradient of g_b o_b with the unscaled dO.
+constexpr int kModeThree = 0, kModeTopn = 1, kModeNsa = 2, kModeNsaTok = 2, kModeNsaCmp = 3;
+enum NsaBranch { kBrCmp = 0, kBrSel = 1, kBrWin = 2 };
 
 constexpr int kBwThreads = 320;  // warps 0-7 rows (two column halves), warp 8 MMA, warp 9 TMA producer
 constexpr int kMmaWarp = 8, kProdWarp = 9, kRowWarps = 8;
@@ -124,20 +135,33 @@ struct DqLayout {
 
 struct DqParams {
   const int32_t* crit;   // three-way: [B*H][nqb][len] critical; top-n: [B*H_kv][nqb][len] selected (-1 pad)
-  const float* lse;      // [B*H][N] (log2 domain)
-  const float* delta;    // [B*H][N]
+  const float* lse;      // [B*H][N] (log2 domain); NSA: [3][B*H][N] per branch, gate folded in
+  const float* delta;    // [B*H][N]; NSA: [3][B*H][N]
   const float* dq_acc;   // [B*H][N][D] or null
   __nv_bfloat16* dq;     // [B*H][N][D]
   int* status;
   int H, group, N, n_valid, nb, len, npairs, words, window;
   float scale, scale_log2;
+  // NSA: branch stride of lse / delta / dlogit (B*H*N), the gate logits' gradients
+  // dlogit [3][B*H][N] and gates w_g [H][3][D] (both null without gates), the compressed
+  // keys (n_cmp keys in nct 64-key tiles, key c stands for token c * kstride + kspan)
+  size_t bstride;
+  const float* dlogit;
+  const __nv_bfloat16* w_g3;
+  int n_cmp, nct, kstride, kspan;
 };
 
-// TOPN: element (t, s) is kept when s <= t and (block(s) selected or s > t - window)
-template <int D, bool TOPN>
+// TOPN: element (t, s) is kept when s <= t and (block(s) selected or s > t - window).
+// NSA: the list holds three kinds of tiles, tagged with their branch: compressed key tiles
+// (tmKc / tmVc; key c kept when c < n_cmp and c * kstride + kspan <= t), selected blocks
+// (s <= t) and window blocks (t - window < s <= t). All of them add to one dQ accumulator.
+template <int D, int MODE>
 __global__ void __launch_bounds__(kBwThreads, 1)
     flash_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, DqParams prm) {
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
+                    DqParams prm) {
+  constexpr bool TOPN = MODE != kModeThree, NSA = MODE == kModeNsa;
   using L = DqLayout<D>;
   constexpr int NP = L::NP, S = kBwSlots;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -195,7 +219,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         report(prm.status, SLA_ERR_DEVICE_CHECK, kDetailFlashIndex);
         continue;
       }
-      atomicOr(&act[j >> 5], 1u << (j & 31));
+      if (!NSA) atomicOr(&act[j >> 5], 1u << (j & 31));  // NSA: act holds the window alone
       if (TOPN) atomicOr(&sel[j >> 5], 1u << (j & 31));
     }
     if (TOPN && prm.window > 0) {  // the blocks the causal window reaches
@@ -206,8 +230,30 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   }
   __syncthreads();
   if (warp == 0) {
-    const int n = merge_bitmaps(words, words + prm.words, TOPN ? words + 2 * prm.words : nullptr,
-                                TOPN ? words + 3 * prm.words : nullptr, prm.words, true, true, 0u, mlist, 0, lane);
+    int n = 0;
+    if (NSA) {
+      // compressed key tiles up to the causal limit of either half (act bit per half),
+      // then the selected blocks, then the window blocks; the tag is the branch
+      int jmax[2];
+      for (int hf = 0; hf < 2; ++hf) {
+        const int last_t = i_h[hf] * kBlock + kBlock - 1 - prm.kspan;
+        int jm = (!valid_h[hf] || last_t < 0 || prm.n_cmp == 0) ? -1 : last_t / prm.kstride / kBlock;
+        const int jcap = (prm.n_cmp - 1) / kBlock;
+        jmax[hf] = jm > jcap ? jcap : jm;
+      }
+      const int nc = (jmax[0] > jmax[1] ? jmax[0] : jmax[1]) + 1;
+      for (int jt = lane; jt < nc; jt += 32)
+        mlist[jt] = (uint32_t)jt | (jt <= jmax[0] ? 1u << kActBit : 0u) | (jt <= jmax[1] ? 1u << (kActBit + 1) : 0u) |
+                    ((uint32_t)kBrCmp << kTagShift);
+      __syncwarp();
+      n = merge_bitmaps(words + 2 * prm.words, words + 3 * prm.words, words + 2 * prm.words,
+                        words + 3 * prm.words, prm.words, true, true, (uint32_t)kBrSel, mlist, nc, lane);
+      n = merge_bitmaps(words, words + prm.words, nullptr, nullptr, prm.words, true, true, (uint32_t)kBrWin, mlist,
+                        n, lane);
+    } else {
+      n = merge_bitmaps(words, words + prm.words, TOPN ? words + 2 * prm.words : nullptr,
+                        TOPN ? words + 3 * prm.words : nullptr, prm.words, true, true, 0u, mlist, 0, lane);
+    }
     if (lane == 0) misc[1] = n;
   }
   tc::fence_before_sync();
@@ -231,12 +277,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       for (int m = 0; m < T && ok; ++m) {
         const int slot = m % S;
         if (m >= S && !(ok = tc::mbar_wait(bar(SLOT_FREE + slot), ((m / S) - 1) & 1, abort))) break;
-        const int jb = (int)(mlist[m] & kIdxMask);
+        const uint32_t e = mlist[m];
+        const int jb = (int)(e & kIdxMask);
+        const bool cmp_tile = NSA && (e >> kTagShift) == (uint32_t)kBrCmp;
+        const CUtensorMap* mk = cmp_tile ? &tmKc : &tmK;
+        const CUtensorMap* mv = cmp_tile ? &tmVc : &tmV;
         const uint32_t dst = sR + slot * L::kSlot;
         tc::mbar_expect_tx(bar(LOADED + slot), L::kSlot);
         for (int p = 0; p < NP; ++p) {
-          tc::tma_load_3d(dst + p * 8192, &tmK, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
-          tc::tma_load_3d(dst + L::kTile + p * 8192, &tmV, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
+          tc::tma_load_3d(dst + p * 8192, mk, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
+          tc::tma_load_3d(dst + L::kTile + p * 8192, mv, bar(LOADED + slot), 64 * p, jb * kBlock, bkv);
         }
       }
       // the last release of every slot: no product reads the ring and no commit is in flight at exit
@@ -320,8 +370,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const int t = i_h[hf] * kBlock + (r & 63);
     const bool vrow = valid_h[hf] && t < prm.n_valid;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const float lse2 = vrow ? prm.lse[(size_t)bh * prm.N + t] : INFINITY;
-    const float dlt = vrow ? prm.delta[(size_t)bh * prm.N + t] : 0.f;
+    // per branch (NSA: compressed, selected, window; otherwise one)
+    float lse_b[NSA ? 3 : 1], dlt_b[NSA ? 3 : 1];
+#pragma unroll
+    for (int x = 0; x < (NSA ? 3 : 1); ++x) {
+      lse_b[x] = vrow ? prm.lse[x * prm.bstride + (size_t)bh * prm.N + t] : INFINITY;
+      dlt_b[x] = vrow ? prm.delta[x * prm.bstride + (size_t)bh * prm.N + t] : 0.f;
+    }
     const float sl2 = prm.scale_log2;
     bool ok = true;
     for (int m = 0; m < T && ok; ++m) {
@@ -330,6 +385,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       const int k0 = (int)(e & kIdxMask) * kBlock;
       const bool act = (e >> (kActBit + hf)) & 1u;
       const bool sel = (e >> (kSelBit + hf)) & 1u;
+      const int br = NSA ? (int)(e >> kTagShift) : 0;
+      const bool cmp_tile = NSA && br == kBrCmp;
+      const float lse2 = NSA ? (br == kBrCmp ? lse_b[0] : br == kBrSel ? lse_b[1] : lse_b[2]) : lse_b[0];
+      const float dlt = NSA ? (br == kBrCmp ? dlt_b[0] : br == kBrSel ? dlt_b[1] : dlt_b[2]) : dlt_b[0];
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL + b), (m >> 1) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
@@ -350,8 +409,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         for (int x = 0; x < 2; ++x) {
           const int c = 2 * j + x;
           const int key = kc + c;
-          bool keep = act && key < prm.n_valid;
-          if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
+          bool keep;
+          if (cmp_tile)
+            keep = act && key < prm.n_cmp && key * prm.kstride + prm.kspan <= t;
+          else {
+            keep = act && key < prm.n_valid;
+            if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
+          }
           const float p = keep ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse2) : 0.f;
           g2[x] = p * (__uint_as_float(pv[c]) - dlt);
         }
@@ -379,6 +443,14 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       // dq = scale dQ + the linear-branch part (padding rows 0)
       __nv_bfloat16* dst = prm.dq + ((size_t)bh * prm.N + t) * D;
       const float* acc = prm.dq_acc ? prm.dq_acc + ((size_t)bh * prm.N + t) * D : nullptr;
+      // NSA's gates: dq += sum_b dlogit_b w_g[h][b]
+      float dl[3] = {0.f, 0.f, 0.f};
+      const __nv_bfloat16* wg = nullptr;
+      if (NSA && prm.dlogit != nullptr && vrow) {
+        wg = prm.w_g3 + (size_t)(bh % prm.H) * 3 * D;
+#pragma unroll
+        for (int x = 0; x < 3; ++x) dl[x] = prm.dlogit[x * prm.bstride + (size_t)bh * prm.N + t];
+      }
 #pragma unroll 1
       for (int ch = hw * (D / 64); ch < (hw + 1) * (D / 64); ++ch) {  // this warpgroup's half of the columns
         uint32_t v[32];
@@ -397,6 +469,14 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             const float2 x = *reinterpret_cast<const float2*>(acc + 32 * ch + 2 * j);
             a0 += x.x;
             a1 += x.y;
+          }
+          if (NSA && wg != nullptr) {
+#pragma unroll
+            for (int x = 0; x < 3; ++x) {
+              const float2 wv = unpack_bf16(*reinterpret_cast<const uint32_t*>(wg + x * D + 32 * ch + 2 * j));
+              a0 = fmaf(dl[x], wv.x, a0);
+              a1 = fmaf(dl[x], wv.y, a1);
+            }
           }
           w[j] = vrow && ok ? pack_bf16(a0, a1) : 0u;
         }
@@ -433,9 +513,9 @@ struct DkvLayout {
 
 struct DkvParams {
   const uint32_t* bits;   // three-way: [B*H][nkb][words] critical; top-n: [B*H_kv][nkb][words] selected
-  uint32_t* dlist;        // [B*H_kv*npairs][group*nqb]: merged (head, query block) list of each unit
-  const float* lse;       // [B*H][N] (log2 domain)
-  const float* delta;     // [B*H][N]
+  uint32_t* dlist;        // [units][list_cap]: merged (head, query block) list of each unit
+  const float* lse;       // [B*H][N] (log2 domain); NSA: [3][B*H][N] per branch, gate folded in
+  const float* delta;     // [B*H][N]; NSA: [3][B*H][N]
   const float* dk_acc;    // [B*H_kv][N][D] or null
   const float* dv_acc;
   const float* kcol;      // smooth-K: [B*H_kv][D] = -(sum of the linear dk over valid tokens) / N_valid, or null
@@ -444,14 +524,34 @@ struct DkvParams {
   int* status;
   int H, group, N, n_valid, nb, npairs, words, window;
   float scale, scale_log2;
+  int list_cap;           // entries of one unit's list
+  int nqb;                // query blocks per head
+  size_t bstride;         // NSA: branch stride of lse / delta (B*H*N)
+  // NSA tokens: the compressed branch's key gradients dKc (scaled), dVc [B*H_kv][ncmp_pad][D]
+  // (fp32, null without compressed keys), scattered back to the tokens of each block
+  const float* dkc;
+  const float* dvc;
+  int n_cmp, ncmp_pad, kstride, kspan;
+  float inv_len;          // 1 / cmp_block
+  // NSA compressed keys: units are (KV head, pair of compressed tiles, chunk of chunk
+  // entries of its (query head, query block) list); items units per KV head; raw dV, dK
+  // partials [B*H_kv*items][2][128][D] (fp32)
+  float* part;
+  int chunk, items;
 };
 
-// TOPN: element (query t, key s) is kept when s <= t and (block(s) selected or s > t - window)
-template <int D, bool TOPN>
+
+// TOPN: element (query t, key s) is kept when s <= t and (block(s) selected or s > t - window).
+// NSA tokens (kModeNsaTok): selected and window entries are separate (each with its
+// branch's log-sum-exp and D), and the epilogue adds the compressed branch's share.
+// NSA compressed keys (kModeNsaCmp): tmK / tmV map the compressed keys; key c is kept
+// for query t when c < n_cmp and c * kstride + kspan <= t; raw fp32 partials out.
+template <int D, int MODE>
 __global__ void __launch_bounds__(kBwThreads, 1)
     flash_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       DkvParams prm) {
+  constexpr bool TOPN = MODE != kModeThree, NSAT = MODE == kModeNsaTok, NSAC = MODE == kModeNsaCmp;
   using L = DkvLayout<D>;
   constexpr int NP = L::NP, S = kBwSlots;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -462,12 +562,24 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     return;
   }
   const int Hkv = prm.H / prm.group;
-  const int bkv = blockIdx.x / prm.npairs, pr = blockIdx.x % prm.npairs;
+  // compressed keys: blockIdx = (KV head, item); the item is chunk ch of pair u
+  const CmpSplit split{prm.n_cmp, prm.kstride, prm.kspan, prm.nqb, prm.group, prm.chunk};
+  int bkv, pr, chk = 0;
+  if (NSAC) {
+    bkv = blockIdx.x / prm.items;
+    int it = blockIdx.x % prm.items, u = 0;
+    while (u < split.units() - 1 && it >= split.chunks(u)) it -= split.chunks(u++);
+    pr = u;
+    chk = it;
+  } else {
+    bkv = blockIdx.x / prm.npairs;
+    pr = blockIdx.x % prm.npairs;
+  }
   const int b = bkv / Hkv, hk = bkv % Hkv;
   const int j_h[2] = {2 * pr, 2 * pr + 1};
   const bool valid_j[2] = {j_h[0] < prm.nb, j_h[1] < prm.nb};
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);  // tmem, count, abort
-  uint32_t* dlist = prm.dlist + (size_t)blockIdx.x * prm.group * prm.nb;
+  uint32_t* dlist = prm.dlist + (size_t)blockIdx.x * prm.list_cap;
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
   // one S^T / dP^T buffer: SP_FULL (products done), S_READ (row warps have loaded them);
   // two P^T / dS^T buffers: DS_FULL (written), PS_FREE (dV / dK products done)
@@ -475,6 +587,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                 DS_FULL = S_READ + 1, PS_FREE = DS_FULL + 2, ACC_DONE = PS_FREE + 2;
   const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sR = sbase + L::kOffRing;
   auto head_of = [&](int g) { return b * prm.H + hk * prm.group + g; };
+  // list tag -> (query head of the group, branch of lse / delta)
+  auto tag_head = [&](uint32_t tag) { return head_of((int)(NSAT ? tag >> 1 : tag)); };
+  auto tag_branch = [&](uint32_t tag) { return NSAT ? (int)kBrSel + (int)(tag & 1u) : NSAC ? (int)kBrCmp : 0; };
 
   if (tid == 0) {
     misc[2] = 0;
@@ -504,7 +619,21 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   }
   if (warp == 0) {
     int n = 0;
-    if (!TOPN) {
+    if (NSAC) {
+      // chunk ch of the entries (g, i), g-major, i from the first attending block
+      const int f = split.first_block(pr), ni = prm.nqb - f;
+      const int e0 = chk * prm.chunk, total = split.entries(pr);
+      const int cnt = total - e0 < prm.chunk ? total - e0 : prm.chunk;
+      for (int x = lane; x < cnt; x += 32) {
+        const int g = (e0 + x) / ni, i = f + (e0 + x) % ni;
+        uint32_t act = 0u;
+        for (int h = 0; h < 2; ++h)  // half h is active when block i's last row reaches its first key
+          if (valid_j[h] && (long long)j_h[h] * kBlock * prm.kstride + prm.kspan <= (long long)i * kBlock + kBlock - 1)
+            act |= 1u << (kActBit + h);
+        dlist[x] = (uint32_t)i | act | ((uint32_t)g << kTagShift);
+      }
+      n = cnt > 0 ? cnt : 0;
+    } else if (!TOPN) {
       // every query head of the group: the query blocks that hold j0 or j1 as critical
       for (int g = 0; g < prm.group; ++g) {
         const size_t row = (size_t)head_of(g) * prm.nb;
@@ -532,14 +661,22 @@ __global__ void __launch_bounds__(kBwThreads, 1)
               const int i = 32 * w + b2;
               if (i >= j_h[h] && i <= last) win |= 1u << b2;
             }
-          wb[h * prm.words + w] = sv | win;
+          wb[h * prm.words + w] = NSAT ? win : (sv | win);  // NSA: the window branch alone
           wb[(2 + h) * prm.words + w] = sv;
         }
       }
       __syncwarp();
-      for (int g = 0; g < prm.group; ++g)
-        n = merge_bitmaps(wb, wb + prm.words, wb + 2 * prm.words, wb + 3 * prm.words, prm.words, valid_j[0],
-                          valid_j[1], (uint32_t)g, dlist, n, lane);
+      for (int g = 0; g < prm.group; ++g) {
+        if (NSAT) {  // selected entries (tag 2g), then window entries (tag 2g + 1)
+          n = merge_bitmaps(wb + 2 * prm.words, wb + 3 * prm.words, wb + 2 * prm.words, wb + 3 * prm.words,
+                            prm.words, valid_j[0], valid_j[1], (uint32_t)(2 * g), dlist, n, lane);
+          n = merge_bitmaps(wb, wb + prm.words, nullptr, nullptr, prm.words, valid_j[0], valid_j[1],
+                            (uint32_t)(2 * g + 1), dlist, n, lane);
+        } else {
+          n = merge_bitmaps(wb, wb + prm.words, wb + 2 * prm.words, wb + 3 * prm.words, prm.words, valid_j[0],
+                            valid_j[1], (uint32_t)g, dlist, n, lane);
+        }
+      }
     }
     if (lane == 0) misc[1] = n;
   }
@@ -558,15 +695,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         const int slot = m % S;
         if (m >= S && !(ok = tc::mbar_wait(bar(SLOT_FREE + slot), ((m / S) - 1) & 1, abort))) break;
         const uint32_t e = dlist[m];
-        const int i = (int)(e & kIdxMask), bh = head_of((int)(e >> kTagShift));
+        const int i = (int)(e & kIdxMask), bh = tag_head(e >> kTagShift);
+        const size_t boff = (size_t)tag_branch(e >> kTagShift) * prm.bstride;
         const uint32_t dst = sR + slot * L::kSlot;
         tc::mbar_expect_tx(bar(LOADED + slot), 2 * L::kTile + 512);
         for (int p = 0; p < NP; ++p) {
           tc::tma_load_3d(dst + p * 8192, &tmQ, bar(LOADED + slot), 64 * p, i * kBlock, bh);
           tc::tma_load_3d(dst + L::kTile + p * 8192, &tmO, bar(LOADED + slot), 64 * p, i * kBlock, bh);
         }
-        tc::bulk_load(dst + 2 * L::kTile, prm.lse + (size_t)bh * prm.N + i * kBlock, 256, bar(LOADED + slot));
-        tc::bulk_load(dst + 2 * L::kTile + 256, prm.delta + (size_t)bh * prm.N + i * kBlock, 256,
+        tc::bulk_load(dst + 2 * L::kTile, prm.lse + boff + (size_t)bh * prm.N + i * kBlock, 256, bar(LOADED + slot));
+        tc::bulk_load(dst + 2 * L::kTile + 256, prm.delta + boff + (size_t)bh * prm.N + i * kBlock, 256,
                       bar(LOADED + slot));
       }
       // the last release of every slot: no product reads the ring and no commit is in flight at exit
@@ -651,8 +789,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     // warp = quarter (TMEM lanes) + 4 * hw (query columns 32 hw .. 32 hw + 31 of each tile)
     const int quarter = warp & 3, hw = warp >> 2;
     const int r = quarter * 32 + lane, hf = r >> 6;
-    const int key = j_h[hf] * kBlock + (r & 63);
-    const bool vkey = valid_j[hf] && key < prm.n_valid;
+    const int key = j_h[hf] * kBlock + (r & 63);  // NSA compressed keys: the compressed key index
+    const bool vkey = valid_j[hf] && key < (NSAC ? prm.n_cmp : prm.n_valid);
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = prm.scale_log2;
     bool ok = true;
@@ -695,7 +833,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         for (int y = 0; y < 2; ++y) {
           const int c = 2 * j + y;
           bool keep = act;
-          if (TOPN) keep = keep && key <= t0 + c && (sel || key > t0 + c - prm.window);
+          if (NSAC)
+            keep = keep && key * prm.kstride + prm.kspan <= t0 + c;
+          else if (TOPN)
+            keep = keep && key <= t0 + c && (sel || key > t0 + c - prm.window);
           const float p = keep ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse[c]) : 0.f;
           pp[y] = p;
           dd[y] = p * (__uint_as_float(pv[c]) - dl[c]);
@@ -723,9 +864,38 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       *abort = 1;
       report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
     }
-    if (valid_j[hf]) {
+    if (NSAC) {
+      // raw partial sums of this chunk (every row, zero where nothing was accumulated)
+      float* prt = prm.part + (size_t)blockIdx.x * 2 * 128 * D;
+      for (int which = 0; which < 2; ++which) {
+        float* dst = prt + ((size_t)which * 128 + r) * D;
+#pragma unroll 1
+        for (int c2 = hw * (D / 64); c2 < (hw + 1) * (D / 64); ++c2) {
+          uint32_t v[32];
+          if (ok && T > 0) {
+            tc::tmem_ld32(tmem + lane_off + which * D + 32 * c2, v);
+            tc::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+          }
+          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c2);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
+                                __uint_as_float(v[4 * j + 3]));
+        }
+      }
+    } else if (valid_j[hf]) {
       // dk = scale dK + linear part, dv = dV + linear part (padding keys 0)
       const size_t row = (size_t)bkv * prm.N + key;
+      // NSA: the compressed blocks c that hold token `key` (c * kstride <= key <= c * kstride + kspan)
+      int c_lo = 0, c_hi = -1;
+      if (NSAT && prm.dkc != nullptr && vkey) {
+        c_lo = key <= prm.kspan ? 0 : (key - prm.kspan + prm.kstride - 1) / prm.kstride;
+        c_hi = key / prm.kstride;
+        if (c_hi > prm.n_cmp - 1) c_hi = prm.n_cmp - 1;
+      }
       for (int which = 0; which < 2; ++which) {
         __nv_bfloat16* dst = (which == 0 ? prm.dv : prm.dk) + row * D;
         const float* acc = which == 0 ? prm.dv_acc : prm.dk_acc;
@@ -755,6 +925,14 @@ __global__ void __launch_bounds__(kBwThreads, 1)
               a0 += kc[32 * ch + 2 * j];
               a1 += kc[32 * ch + 2 * j + 1];
             }
+            if (NSAT) {  // compressed keys and values are block means: each token gets 1 / length
+              const float* cg = which == 0 ? prm.dvc : prm.dkc;
+              for (int cc = c_lo; cc <= c_hi; ++cc) {
+                const float2 xx = *reinterpret_cast<const float2*>(cg + ((size_t)bkv * prm.ncmp_pad + cc) * D + 32 * ch + 2 * j);
+                a0 = fmaf(prm.inv_len, xx.x, a0);
+                a1 = fmaf(prm.inv_len, xx.y, a1);
+              }
+            }
             w[j] = vkey && ok ? pack_bf16(a0, a1) : 0u;
           }
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
@@ -782,17 +960,26 @@ static bool map64(CUtensorMap* m, const void* base, int heads, int n_rows, int N
                       (uint64_t)N * D * 2, 64, 64);
 }
 
-template <int D, bool TOPN>
+template <int D, int MODE>
 static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
   using L = DqLayout<D>;
+  constexpr bool TOPN = MODE != kModeThree, NSA = MODE == kModeNsa;
   const sla_config& c = p.c;
-  CUtensorMap mq, mo, mk, mv;
+  CUtensorMap mq, mo, mk, mv, mkc, mvc;
   if (!map64(&mq, a.q, c.B * c.H, c.N_valid, c.N, D) || !map64(&mo, a.dout, c.B * c.H, c.N_valid, c.N, D) ||
       !map64(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) || !map64(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
     return cudaErrorInvalidValue;
+  // NSA's compressed keys and values (rows beyond n_cmp read as zero); otherwise unused
+  const int crows = NSA && p.n_cmp > 0 ? p.n_cmp : 1;
+  if (!map64(&mkc, NSA ? (const void*)(a.ws + p.off_kc) : (const void*)a.k, c.B * c.H_kv, crows,
+             NSA ? p.ncmp_pad : c.N, D) ||
+      !map64(&mvc, NSA ? (const void*)(a.ws + p.off_vc) : (const void*)a.v, c.B * c.H_kv, crows,
+             NSA ? p.ncmp_pad : c.N, D))
+    return cudaErrorInvalidValue;
   DqParams prm;
+  memset(&prm, 0, sizeof(prm));
   prm.crit = reinterpret_cast<const int32_t*>(a.ws + p.off_crit);
-  prm.lse = reinterpret_cast<const float*>(a.ws + p.off_lse);
+  prm.lse = NSA ? reinterpret_cast<const float*>(a.bws + bp.off_lse3) : reinterpret_cast<const float*>(a.ws + p.off_lse);
   prm.delta = reinterpret_cast<const float*>(a.bws + bp.off_delta);
   prm.dq_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dqacc) : nullptr;
   prm.dq = a.dq;
@@ -808,36 +995,80 @@ static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& 
   prm.window = c.window;
   prm.scale = p.scale;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
+  prm.bstride = (size_t)c.B * c.H * c.N;
+  if (NSA) {
+    prm.dlogit = c.has_gate ? reinterpret_cast<const float*>(a.bws + bp.off_dlogit) : nullptr;
+    prm.w_g3 = c.has_gate ? a.w_g : nullptr;
+    prm.n_cmp = p.n_cmp;
+    prm.nct = p.ncmp_pad / kBlock;
+    prm.kstride = c.cmp_stride;
+    prm.kspan = c.cmp_block - 1;
+  }
   int per_half = prm.len;
   if (TOPN) per_half += (c.window + 62) / kBlock + 2;  // selected blocks plus the window's reach
-  const int cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
+  int cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
+  if (NSA) {  // compressed tiles, then the selected and the window blocks, each a union over two halves
+    const int sel = 2 * c.top_n < p.nkb ? 2 * c.top_n : p.nkb;
+    const int win = 2 * ((c.window + 62) / kBlock + 2) < p.nkb ? 2 * ((c.window + 62) / kBlock + 2) : p.nkb;
+    cap = p.ncmp_pad / kBlock + sel + win;
+  }
   int smem = L::kOffList + (cap > 0 ? cap : 1) * 4;
   if (4 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: it holds all 512 TMEM columns
-  cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D, TOPN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dq_kernel<D, TOPN><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  flash_dq_kernel<D, MODE><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, mkc, mvc, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_flash_dq(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
-  const bool topn = p.c.mode == SLA_MODE_TOPN_WINDOW;
-  if (p.c.d == 128) return topn ? launch_dq_t<128, true>(p, bp, a, s) : launch_dq_t<128, false>(p, bp, a, s);
-  return topn ? launch_dq_t<64, true>(p, bp, a, s) : launch_dq_t<64, false>(p, bp, a, s);
+  const int mode = p.c.mode == SLA_MODE_THREEWAY ? kModeThree : p.c.nsa_branches ? kModeNsa : kModeTopn;
+  if (p.c.d == 128) {
+    if (mode == kModeNsa) return launch_dq_t<128, kModeNsa>(p, bp, a, s);
+    return mode == kModeTopn ? launch_dq_t<128, kModeTopn>(p, bp, a, s) : launch_dq_t<128, kModeThree>(p, bp, a, s);
+  }
+  if (mode == kModeNsa) return launch_dq_t<64, kModeNsa>(p, bp, a, s);
+  return mode == kModeTopn ? launch_dq_t<64, kModeTopn>(p, bp, a, s) : launch_dq_t<64, kModeThree>(p, bp, a, s);
 }
 
-template <int D, bool TOPN>
+// entries of one (KV head, pair of key blocks) unit's list in the dK / dV kernel
+int dkdv_list_cap(const Plan& p) { return p.group * p.nqb * (p.c.nsa_branches ? 2 : 1); }
+
+// NSA's compressed keys: entries per item, chosen so that the items fill the GPU about
+// four times over (at least 64 entries, so that an item's fixed cost stays small)
+CmpSplit cmp_split(const Plan& p) {
+  const sla_config& c = p.c;
+  CmpSplit sp{p.n_cmp, c.cmp_stride, c.cmp_block - 1, p.nqb, p.group, 1 << 30};
+  long long total = 0;
+  for (int u = 0; u < sp.units(); ++u) total += sp.entries(u);
+  total *= (long long)c.B * c.H_kv;
+  long long ch = (total + 148 * 4 - 1) / (148 * 4);
+  if (ch < 64) ch = 64;
+  if (ch > (1 << 20)) ch = 1 << 20;
+  sp.chunk = (int)ch;
+  return sp;
+}
+
+template <int D, int MODE>
 static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
   using L = DkvLayout<D>;
+  constexpr bool TOPN = MODE != kModeThree, NSAT = MODE == kModeNsaTok, NSAC = MODE == kModeNsaCmp;
   const sla_config& c = p.c;
   CUtensorMap mq, mo, mk, mv;
+  // NSA's compressed keys: the key tiles are the compressed keys and values
+  const void* kb = NSAC ? (const void*)(a.ws + p.off_kc) : (const void*)a.k;
+  const void* vb = NSAC ? (const void*)(a.ws + p.off_vc) : (const void*)a.v;
+  const int krows = NSAC ? (p.n_cmp > 0 ? p.n_cmp : 1) : c.N_valid, kstride_rows = NSAC ? p.ncmp_pad : c.N;
   if (!map64(&mq, a.q, c.B * c.H, c.N_valid, c.N, D) || !map64(&mo, a.dout, c.B * c.H, c.N_valid, c.N, D) ||
-      !map64(&mk, a.k, c.B * c.H_kv, c.N_valid, c.N, D) || !map64(&mv, a.v, c.B * c.H_kv, c.N_valid, c.N, D))
+      !map64(&mk, kb, c.B * c.H_kv, krows, kstride_rows, D) || !map64(&mv, vb, c.B * c.H_kv, krows, kstride_rows, D))
     return cudaErrorInvalidValue;
   DkvParams prm;
+  memset(&prm, 0, sizeof(prm));
+  const bool nsa = NSAT || NSAC;
   prm.bits = reinterpret_cast<const uint32_t*>(a.bws + bp.off_bits);
-  prm.dlist = reinterpret_cast<uint32_t*>(a.bws + bp.off_dlist);
-  prm.lse = reinterpret_cast<const float*>(a.ws + p.off_lse);
+  prm.dlist = reinterpret_cast<uint32_t*>(a.bws + (NSAC ? bp.off_clist : bp.off_dlist));
+  prm.lse = nsa ? reinterpret_cast<const float*>(a.bws + bp.off_lse3) : reinterpret_cast<const float*>(a.ws + p.off_lse);
   prm.delta = reinterpret_cast<const float*>(a.bws + bp.off_delta);
   prm.dk_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dkacc) : nullptr;
   prm.dv_acc = bp.lin ? reinterpret_cast<const float*>(a.bws + bp.off_dvacc) : nullptr;
@@ -849,25 +1080,102 @@ static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs
   prm.group = p.group;
   prm.N = c.N;
   prm.n_valid = c.N_valid;
-  prm.nb = p.nkb;
-  prm.npairs = (p.nkb + 1) / 2;
+  prm.nb = NSAC ? p.ncmp_pad / kBlock : p.nkb;
+  prm.npairs = (prm.nb + 1) / 2;
   prm.words = bp.words;
   prm.window = c.window;
   prm.scale = p.scale;
   prm.scale_log2 = p.scale * 1.4426950408889634f;
+  prm.nqb = p.nqb;
+  prm.bstride = (size_t)c.B * c.H * c.N;
+  prm.list_cap = dkdv_list_cap(p);
+  if (nsa) {
+    prm.n_cmp = p.n_cmp;
+    prm.ncmp_pad = p.ncmp_pad;
+    prm.kstride = c.cmp_stride;
+    prm.kspan = c.cmp_block - 1;
+    prm.inv_len = 1.f / (float)c.cmp_block;
+    if (NSAT && p.n_cmp > 0) {
+      prm.dkc = reinterpret_cast<const float*>(a.bws + bp.off_dkc);
+      prm.dvc = reinterpret_cast<const float*>(a.bws + bp.off_dvc);
+    }
+  }
+  unsigned grid = (unsigned)(c.B * c.H_kv * prm.npairs);
+  if (NSAC) {
+    const CmpSplit sp = cmp_split(p);
+    prm.chunk = sp.chunk;
+    prm.items = bp.cmp_items;
+    prm.list_cap = sp.chunk;
+    prm.part = reinterpret_cast<float*>(a.bws + bp.off_part);
+    grid = (unsigned)(c.B * c.H_kv * bp.cmp_items);
+    if (grid == 0) return cudaSuccess;
+  }
   int smem = L::kSmem;
   if (TOPN && 4 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (512 TMEM columns)
-  cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D, TOPN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dkdv_kernel<D, TOPN><<<c.B * c.H_kv * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  flash_dkdv_kernel<D, MODE><<<grid, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_flash_dkdv(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
-  const bool topn = p.c.mode == SLA_MODE_TOPN_WINDOW;
-  if (p.c.d == 128) return topn ? launch_dkdv_t<128, true>(p, bp, a, s) : launch_dkdv_t<128, false>(p, bp, a, s);
-  return topn ? launch_dkdv_t<64, true>(p, bp, a, s) : launch_dkdv_t<64, false>(p, bp, a, s);
+  const int mode = p.c.mode == SLA_MODE_THREEWAY ? kModeThree : p.c.nsa_branches ? kModeNsaTok : kModeTopn;
+  if (p.c.d == 128) {
+    if (mode == kModeNsaTok) return launch_dkdv_t<128, kModeNsaTok>(p, bp, a, s);
+    return mode == kModeTopn ? launch_dkdv_t<128, kModeTopn>(p, bp, a, s) : launch_dkdv_t<128, kModeThree>(p, bp, a, s);
+  }
+  if (mode == kModeNsaTok) return launch_dkdv_t<64, kModeNsaTok>(p, bp, a, s);
+  return mode == kModeTopn ? launch_dkdv_t<64, kModeTopn>(p, bp, a, s) : launch_dkdv_t<64, kModeThree>(p, bp, a, s);
+}
+
+cudaError_t launch_flash_dkdv_cmp(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  return p.c.d == 128 ? launch_dkdv_t<128, kModeNsaCmp>(p, bp, a, s) : launch_dkdv_t<64, kModeNsaCmp>(p, bp, a, s);
+}
+
+// ---------------------------------------------------------------------------
+// NSA's compressed keys: dKc = scale * sum of the dK partials of a pair's chunks, dVc
+// likewise, in chunk order (deterministic); rows past n_cmp are 0
+// ---------------------------------------------------------------------------
+__global__ void cmp_reduce_kernel(const float* __restrict__ part, float* __restrict__ dkc, float* __restrict__ dvc,
+                                  CmpSplit sp, int items, int ncmp_pad, int d, int64_t total, float scale) {
+  // one thread per (KV head, compressed key row, 4 columns)
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int q4 = d / 4;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < total; x += stride) {
+    const int col = (int)(x % q4) * 4;
+    const int64_t rowg = x / q4;
+    const int row = (int)(rowg % ncmp_pad);
+    const int64_t bkv = rowg / ncmp_pad;
+    const int u = row / 128, r = row % 128;
+    float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
+    if (row < sp.n_cmp) {
+      int base = 0;
+      for (int w = 0; w < u; ++w) base += sp.chunks(w);
+      const int n = sp.chunks(u);
+      for (int it = 0; it < n; ++it) {
+        const float* pr = part + ((size_t)bkv * items + base + it) * 2 * 128 * d;
+        const float4 v4 = *reinterpret_cast<const float4*>(pr + (size_t)r * d + col);
+        const float4 k4 = *reinterpret_cast<const float4*>(pr + ((size_t)128 + r) * d + col);
+        sv.x += v4.x; sv.y += v4.y; sv.z += v4.z; sv.w += v4.w;
+        sk.x += k4.x; sk.y += k4.y; sk.z += k4.z; sk.w += k4.w;
+      }
+    }
+    const size_t o = ((size_t)bkv * ncmp_pad + row) * d + col;
+    *reinterpret_cast<float4*>(dvc + o) = sv;
+    *reinterpret_cast<float4*>(dkc + o) = make_float4(scale * sk.x, scale * sk.y, scale * sk.z, scale * sk.w);
+  }
+}
+
+cudaError_t launch_cmp_reduce(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  const int64_t total = (int64_t)c.B * c.H_kv * p.ncmp_pad * (c.d / 4);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  cmp_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+      reinterpret_cast<const float*>(a.bws + bp.off_part), reinterpret_cast<float*>(a.bws + bp.off_dkc),
+      reinterpret_cast<float*>(a.bws + bp.off_dvc), cmp_split(p), bp.cmp_items, p.ncmp_pad, c.d, total, p.scale);
+  return cudaGetLastError();
 }
 
 }  // namespace sla

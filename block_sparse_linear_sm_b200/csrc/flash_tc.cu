@@ -62,6 +62,7 @@ struct FlashTcParams {
   const __nv_bfloat16* oc;
   const __nv_bfloat16* os;
   const __nv_bfloat16* w_g3;
+  __nv_bfloat16* ow;  // NSAC: the window branch's own output o_w [B*H][N][D], kept for the backward pass
 };
 
 constexpr int kTcThreads = 192;
@@ -716,6 +717,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const uint4* oc4 = reinterpret_cast<const uint4*>(prm.oc + rowoff);
       const uint4* os4 = reinterpret_cast<const uint4*>(prm.os + rowoff);
       uint4* dst = reinterpret_cast<uint4*>(prm.o + rowoff);
+      uint4* dstw = reinterpret_cast<uint4*>(prm.ow + rowoff);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -728,21 +730,24 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          uint4 res = make_uint4(0u, 0u, 0u, 0u);
+          uint4 res = make_uint4(0u, 0u, 0u, 0u), resw = res;
           if (live) {
             const uint4 a4 = oc4[4 * c + q8], b4 = os4[4 * c + q8];
             const uint32_t ua[4] = {a4.x, a4.y, a4.z, a4.w}, ub[4] = {b4.x, b4.y, b4.z, b4.w};
-            uint32_t pw[4];
+            uint32_t pw[4], ww[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 fa = unpack_bf16(ua[e]), fb = unpack_bf16(ub[e]);
               const int j = 8 * q8 + 2 * e;
-              pw[e] = pack_bf16(g[0] * fa.x + g[1] * fb.x + g[2] * (__uint_as_float(ov[j]) * inv),
-                                g[0] * fa.y + g[1] * fb.y + g[2] * (__uint_as_float(ov[j + 1]) * inv));
+              const float w0 = __uint_as_float(ov[j]) * inv, w1 = __uint_as_float(ov[j + 1]) * inv;
+              pw[e] = pack_bf16(g[0] * fa.x + g[1] * fb.x + g[2] * w0, g[0] * fa.y + g[1] * fb.y + g[2] * w1);
+              ww[e] = pack_bf16(w0, w1);
             }
             res = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            resw = make_uint4(ww[0], ww[1], ww[2], ww[3]);
           }
           dst[4 * c + q8] = res;
+          dstw[4 * c + q8] = resw;
         }
       }
     } else if (valid_h[hf]) {
@@ -823,7 +828,10 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
   prm.w_g3 = branch == 3 && c.has_gate ? a.w_g : nullptr;
   prm.zs = FUSE ? reinterpret_cast<const float*>(a.ws + p.off_zs) : nullptr;
   prm.gate = FUSE && c.has_gate ? reinterpret_cast<const float*>(a.ws + p.off_gate) : nullptr;
-  prm.lse = branch == 0 ? reinterpret_cast<float*>(a.ws + p.off_lse) : nullptr;
+  // row log-sum-exp for the backward pass; NSA's branches keep one row each
+  // (compressed, selected, window)
+  prm.lse = reinterpret_cast<float*>(a.ws + p.off_lse) + (branch > 0 ? (size_t)(branch - 1) * c.B * c.H * c.N : 0);
+  prm.ow = branch == 3 ? reinterpret_cast<__nv_bfloat16*>(a.ws + p.off_ow) : nullptr;
   prm.status = a.status;
   prm.H = c.H;
   prm.group = p.group;

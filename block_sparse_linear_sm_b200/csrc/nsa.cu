@@ -9,7 +9,8 @@
 // The three attentions run in the sparse flash kernel (flash_tc.cu): the compressed
 // branch over the compressed keys, every tile up to the causal limit c * stride +
 // length - 1 <= t; the window branch's epilogue writes the gated sum. This file holds
-// the compression, HBM-bound, one warp per compressed row.
+// the compression, HBM-bound, one warp per compressed row, and the first step of the
+// backward pass of the three branches (nsa_prep_kernel).
 #include "common.cuh"
 
 namespace sla {
@@ -59,6 +60,124 @@ cudaError_t launch_compress(const Plan& p, const Args& a, cudaStream_t s) {
   else
     compress_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(a.k, a.v, kc, vc, rows, c.N, p.n_cmp, p.ncmp_pad,
                                                          c.cmp_block, c.cmp_stride);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Backward pass, per row t of head h (loss L = sum(O * dO), O = sum_b g_b o_b):
+//   e_b = dO_t . o_b,t; the branch's attention gradient is that of softmax attention
+//   with output gradient g_b dO_t, whose D value is g_b e_b. The flash kernels recompute
+//   P with lse_b - log2 g_b (P scaled by g_b) and take D = e_b, which gives the same dS,
+//   dK, dV and dQ; dlogit_b = e_b g_b (1 - g_b) (sigmoid gate, g_b = 1 without gates);
+//   dq_t += sum_b dlogit_b w_g[h][b] (in the dQ kernel), dw_g[h][b] += sum_t dlogit_b q_t.
+// One CTA per 256 rows of a head, a warp per row, lane = D / 32 features; the dw_g
+// partials of the CTA are summed in shared memory and added with one atomic per element.
+// Padding rows: lse = +inf, e = dlogit = 0.
+// ---------------------------------------------------------------------------
+constexpr int kPrepRows = 256, kPrepWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kPrepWarps * 32)
+    nsa_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
+                    const __nv_bfloat16* __restrict__ oc, const __nv_bfloat16* __restrict__ os,
+                    const __nv_bfloat16* __restrict__ ow, const __nv_bfloat16* __restrict__ w_g3,
+                    const float* __restrict__ lse_in, float* __restrict__ lse_out, float* __restrict__ delta,
+                    float* __restrict__ dlogit, float* __restrict__ dw_g, int H, int N, int n_valid,
+                    size_t bstride) {
+  constexpr int E = D / 32;
+  __shared__ float red[kPrepWarps][3][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunks = (N + kPrepRows - 1) / kPrepRows;
+  const int bh = blockIdx.x / chunks, t0 = (blockIdx.x % chunks) * kPrepRows;
+  const int h = bh % H;
+  float wg[3][E], acc[3][E];
+#pragma unroll
+  for (int b = 0; b < 3; ++b)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      wg[b][e] = w_g3 ? __bfloat162float(w_g3[((size_t)h * 3 + b) * D + lane * E + e]) : 0.f;
+      acc[b][e] = 0.f;
+    }
+  for (int t = t0 + warp; t < t0 + kPrepRows && t < N; t += kPrepWarps) {
+    const size_t row = (size_t)bh * N + t;
+    float ev[3] = {0.f, 0.f, 0.f}, dot[3] = {0.f, 0.f, 0.f}, qv[E];
+    const bool valid = t < n_valid;
+    if (valid) {
+      const __nv_bfloat16* src[3] = {oc + row * D, os + row * D, ow + row * D};
+      const __nv_bfloat16* g = dout + row * D + lane * E;
+      const __nv_bfloat16* qq = q + row * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float go = __bfloat162float(g[e]);
+        qv[e] = __bfloat162float(qq[e]);
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+          ev[b] = fmaf(go, __bfloat162float(src[b][lane * E + e]), ev[b]);
+          dot[b] = fmaf(qv[e], wg[b][e], dot[b]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+          ev[b] += __shfl_xor_sync(0xffffffffu, ev[b], o);
+          dot[b] += __shfl_xor_sync(0xffffffffu, dot[b], o);
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < 3; ++b) {
+      float lse = INFINITY, dl = 0.f;
+      if (valid) {
+        lse = lse_in[b * bstride + row];
+        if (w_g3) {
+          const float gb = 1.f / (1.f + __expf(-dot[b]));
+          lse -= log2f(gb);  // +inf stays +inf; gb = 0 gives +inf (P = 0)
+          dl = ev[b] * gb * (1.f - gb);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[b][e] = fmaf(dl, qv[e], acc[b][e]);
+        }
+      }
+      if (lane == 0) {
+        lse_out[b * bstride + row] = lse;
+        delta[b * bstride + row] = valid ? ev[b] : 0.f;
+        if (dlogit) dlogit[b * bstride + row] = dl;
+      }
+    }
+  }
+  if (!w_g3) return;
+#pragma unroll
+  for (int b = 0; b < 3; ++b)
+#pragma unroll
+    for (int e = 0; e < E; ++e) red[warp][b][lane * E + e] = acc[b][e];
+  __syncthreads();
+  for (int x = threadIdx.x; x < 3 * D; x += blockDim.x) {
+    const int b = x / D, col = x % D;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPrepWarps; ++w) sum += red[w][b][col];
+    atomicAdd(dw_g + ((size_t)h * 3 + b) * D + col, sum);
+  }
+}
+
+cudaError_t launch_nsa_prep(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  const sla_config& c = p.c;
+  const int chunks = (c.N + kPrepRows - 1) / kPrepRows;
+  const unsigned grid = (unsigned)(c.B * c.H * chunks);
+  const size_t bstride = (size_t)c.B * c.H * c.N;
+  const auto* oc = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_oc);
+  const auto* os = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_os);
+  const auto* ow = reinterpret_cast<const __nv_bfloat16*>(a.ws + p.off_ow);
+  const auto* lse_in = reinterpret_cast<const float*>(a.ws + p.off_lse);
+  auto* lse_out = reinterpret_cast<float*>(a.bws + bp.off_lse3);
+  auto* delta = reinterpret_cast<float*>(a.bws + bp.off_delta);
+  float* dlogit = c.has_gate ? reinterpret_cast<float*>(a.bws + bp.off_dlogit) : nullptr;
+  const __nv_bfloat16* wg = c.has_gate ? a.w_g : nullptr;
+  if (c.d == 128)
+    nsa_prep_kernel<128><<<grid, kPrepWarps * 32, 0, s>>>(a.q, a.dout, oc, os, ow, wg, lse_in, lse_out, delta, dlogit,
+                                                          a.dw_g, c.H, c.N, c.N_valid, bstride);
+  else
+    nsa_prep_kernel<64><<<grid, kPrepWarps * 32, 0, s>>>(a.q, a.dout, oc, os, ow, wg, lse_in, lse_out, delta, dlogit,
+                                                         a.dw_g, c.H, c.N, c.N_valid, bstride);
   return cudaGetLastError();
 }
 

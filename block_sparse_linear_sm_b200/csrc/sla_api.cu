@@ -88,7 +88,8 @@ bool make_plan(const sla_config* c, Plan* p) {
     }
   } else {
     p->off_crit = take(B * Hkv * nqb * (size_t)c->top_n * 4);
-    p->off_lse = take(B * H * (size_t)c->N * 4);  // row log2-sum-exp of the sparse branch (backward)
+    // row log2-sum-exp of the sparse branch (backward); NSA: one row per branch
+    p->off_lse = take((c->nsa_branches ? 3 : 1) * B * H * (size_t)c->N * 4);
     if (c->nsa_branches) {
       // compressed blocks that hold valid tokens only, padded to whole 64-key tiles
       p->n_cmp = c->N_valid >= c->cmp_block ? (c->N_valid - c->cmp_block) / c->cmp_stride + 1 : 0;
@@ -97,6 +98,7 @@ bool make_plan(const sla_config* c, Plan* p) {
       p->off_vc = take(B * Hkv * (size_t)p->ncmp_pad * d * 2);
       p->off_oc = take(B * H * (size_t)c->N * d * 2);
       p->off_os = take(B * H * (size_t)c->N * d * 2);
+      p->off_ow = take(B * H * (size_t)c->N * d * 2);  // window branch output (backward)
     }
   }
   p->total = off;
@@ -223,16 +225,13 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
 // ---------------------------------------------------------------------------
 // backward pass
 // ---------------------------------------------------------------------------
-static sla_status check_bwd_config(const sla_config* c) {
-  const sla_status st = check_config(c);
-  if (st != SLA_OK) return st;
-  return c->nsa_branches ? SLA_ERR_UNSUPPORTED : SLA_OK;  // NSA's branches: forward only
-}
+static sla_status check_bwd_config(const sla_config* c) { return check_config(c); }
 
 bool make_bwd_plan(const Plan& p, BwdPlan* b) {
   memset(b, 0, sizeof(*b));
   const sla_config& c = p.c;
   b->lin = c.mode == SLA_MODE_THREEWAY && has_marginal(p);  // the top-n mode has no linear branch
+  b->nsa = c.mode == SLA_MODE_TOPN_WINDOW && c.nsa_branches;
   b->rows_t = p.group * p.nqb_pad;
   b->words = (p.nqb + 31) / 32;
   const size_t B = c.B, H = c.H, Hkv = c.H_kv, d = c.d, N = c.N;
@@ -243,10 +242,22 @@ bool make_bwd_plan(const Plan& p, BwdPlan* b) {
     return o;
   };
   b->off_status = take(256);
-  b->off_delta = take(B * H * N * 4);                       // D_t = dO_t . O_s,t
+  b->off_delta = take((b->nsa ? 3 : 1) * B * H * N * 4);     // D_t = dO_t . O_s,t (NSA: dO_t . o_b,t)
   b->off_bits = take(B * H * p.nkb * (size_t)b->words * 4);  // query blocks of each key block
   // merged (query head, query block) list of each pair of key blocks
-  b->off_dlist = take(B * Hkv * (size_t)((p.nkb + 1) / 2) * p.group * p.nqb * 4);
+  b->off_dlist = take(B * Hkv * (size_t)((p.nkb + 1) / 2) * dkdv_list_cap(p) * 4);
+  if (b->nsa) {
+    b->off_lse3 = take(3 * B * H * N * 4);
+    if (c.has_gate) b->off_dlogit = take(3 * B * H * N * 4);
+    const CmpSplit sp = cmp_split(p);
+    b->cmp_items = sp.items();
+    if (p.n_cmp > 0) {
+      b->off_dkc = take(B * Hkv * (size_t)p.ncmp_pad * d * 4);
+      b->off_dvc = take(B * Hkv * (size_t)p.ncmp_pad * d * 4);
+      b->off_clist = take(B * Hkv * (size_t)b->cmp_items * sp.chunk * 4);
+      b->off_part = take(B * Hkv * (size_t)b->cmp_items * 2 * 128 * d * 4);
+    }
+  }
   if (b->lin) {
     b->off_dqacc = take(B * H * N * d * 4);    // linear-branch and gate part of dq (fp32)
     b->off_dkacc = take(B * Hkv * N * d * 4);  // linear-branch part of dk, dv (fp32)
@@ -266,11 +277,23 @@ bool make_bwd_plan(const Plan& p, BwdPlan* b) {
   return true;
 }
 
-enum BStage { kBZeroCols, kBDelta, kBLinear, kBMaskT, kBAggT, kBState, kBDq, kBDkdv };
+enum BStage { kBZeroCols, kBDelta, kBLinear, kBMaskT, kBAggT, kBState, kBDq, kBDkdv, kBNsaPrep, kBDkdvCmp,
+              kBCmpReduce };
 
-static int bwd_stages_of(const BwdPlan& bp, BStage* out) {
+static int bwd_stages_of(const Plan& p, const BwdPlan& bp, BStage* out) {
   int n = 0;
   out[n++] = kBZeroCols;
+  if (bp.nsa) {
+    // the compressed keys' gradients first: the token dK / dV kernel adds them
+    out[n++] = kBNsaPrep;
+    out[n++] = kBDq;
+    if (p.n_cmp > 0) {
+      out[n++] = kBDkdvCmp;
+      out[n++] = kBCmpReduce;
+    }
+    out[n++] = kBDkdv;
+    return n;
+  }
   if (bp.lin) {
     out[n++] = kBLinear;
     out[n++] = kBMaskT;
@@ -294,6 +317,9 @@ static const char* bwd_stage_name(BStage s) {
     case kBState: return "bwd_state";
     case kBDq: return "bwd_flash_dq";
     case kBDkdv: return "bwd_flash_dkdv";
+    case kBNsaPrep: return "bwd_nsa_prep";
+    case kBDkdvCmp: return "bwd_flash_dkdv_cmp";
+    case kBCmpReduce: return "bwd_cmp_reduce";
   }
   return "?";
 }
@@ -306,7 +332,8 @@ static cudaError_t run_bwd_stage(BStage st, const Plan& p, const BwdPlan& bp, co
       cudaError_t e = cudaSuccess;
       if (c.has_proj)
         e = cudaMemsetAsync(a.dw_p, 0, (size_t)(c.proj_per_head ? c.H : 1) * c.d * c.d * 4, s);
-      if (e == cudaSuccess && c.has_gate) e = cudaMemsetAsync(a.dw_g, 0, (size_t)c.H * c.d * 4, s);
+      if (e == cudaSuccess && c.has_gate)
+        e = cudaMemsetAsync(a.dw_g, 0, (size_t)c.H * (c.nsa_branches ? 3 : 1) * c.d * 4, s);
       return e == cudaSuccess ? launch_cols(p, bp, a, s) : e;
     }
     case kBDelta: return launch_delta(p, bp, a, s);
@@ -316,6 +343,9 @@ static cudaError_t run_bwd_stage(BStage st, const Plan& p, const BwdPlan& bp, co
     case kBState: return launch_state_bwd(p, bp, a, s);
     case kBDq: return launch_flash_dq(p, bp, a, s);
     case kBDkdv: return launch_flash_dkdv(p, bp, a, s);
+    case kBNsaPrep: return launch_nsa_prep(p, bp, a, s);
+    case kBDkdvCmp: return launch_flash_dkdv_cmp(p, bp, a, s);
+    case kBCmpReduce: return launch_cmp_reduce(p, bp, a, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -338,7 +368,7 @@ static sla_status backward_impl(const void* q, const void* k, const void* v, con
   if (!ws || !aligned(ws, 256) || ws_bytes < p.total) return SLA_ERR_WORKSPACE;
   if (!bws || !aligned(bws, 256) || bws_bytes < bp.total) return SLA_ERR_WORKSPACE;
   BStage stages[9];
-  const int ns = bwd_stages_of(bp, stages);
+  const int ns = bwd_stages_of(p, bp, stages);
   if (events && n_events != ns + 1) return SLA_ERR_INVALID_ARG;
   BwdArgs a;
   memset(&a, 0, sizeof(a));
@@ -482,7 +512,7 @@ int32_t sla_backward_num_stages(const sla_config* cfg) {
   make_plan(cfg, &p);
   make_bwd_plan(p, &bp);
   BStage st[9];
-  return bwd_stages_of(bp, st);
+  return bwd_stages_of(p, bp, st);
 }
 
 const char* sla_backward_stage_name(const sla_config* cfg, int32_t s) {
@@ -492,7 +522,7 @@ const char* sla_backward_stage_name(const sla_config* cfg, int32_t s) {
   make_plan(cfg, &p);
   make_bwd_plan(p, &bp);
   BStage st[9];
-  const int n = bwd_stages_of(bp, st);
+  const int n = bwd_stages_of(p, bp, st);
   return (s >= 0 && s < n) ? bwd_stage_name(st[s]) : nullptr;
 }
 

@@ -35,9 +35,10 @@ struct Plan {
   size_t off_status, off_qbar, off_kbar, off_scores, off_kflag, off_crit, off_neg, off_mmask, off_hs, off_ss,
       off_zs, off_phiq, off_gate, off_kmean, off_lse, total;
   // NSA's branches (top-n mode): compressed K, V [B*H_kv][ncmp_pad][d] and the three
-  // branch outputs [B*H][N][d] (bf16)
+  // branch outputs [B*H][N][d] (bf16); off_lse then holds three rows [3][B*H][N]
+  // (compressed, selected, window)
   int n_cmp, ncmp_pad;
-  size_t off_kc, off_vc, off_oc, off_os;
+  size_t off_kc, off_vc, off_oc, off_os, off_ow;
 };
 
 bool make_plan(const sla_config* c, Plan* p);
@@ -84,12 +85,46 @@ cudaError_t launch_compress(const Plan& p, const Args& a, cudaStream_t s);
 // group form the K extent of the transposed aggregation.
 struct BwdPlan {
   bool lin;       // the layer has a linear branch
+  bool nsa;       // NSA's three branches
   int rows_t;     // group * nqb_pad
   int words;      // 32-bit words of one column bitmap (query blocks)
+  int cmp_items;  // NSA: work items of the compressed-key dK / dV kernel per KV head
   size_t off_status, off_delta, off_dqacc, off_dkacc, off_dvacc, off_drow, off_maskt, off_dh, off_dz,
       off_dwp, off_kcolp, off_kcol, off_bits, off_dlist, total;
+  // NSA: per-branch log-sum-exp with the gate folded in [3][B*H][N], gate-logit gradients
+  // [3][B*H][N], compressed-key gradients dKc, dVc [B*H_kv][ncmp_pad][d] (fp32), the
+  // compressed-key kernel's lists and raw partials
+  size_t off_lse3, off_dlogit, off_dkc, off_dvc, off_clist, off_part;
 };
 bool make_bwd_plan(const Plan& p, BwdPlan* b);
+
+// NSA's compressed keys: the (query head, query block) entries of the pair of compressed
+// tiles u (keys 128 u .. 128 u + 127) are every query head of the group times the query
+// blocks i >= first(u), the first block with a row t = 64 i + 63 that attends key 128 u
+// (128 u * stride + span <= t); they are cut into chunks of `chunk` entries. Host and
+// device share this arithmetic.
+struct CmpSplit {
+  int n_cmp, kstride, kspan, nqb, group, chunk;
+  __host__ __device__ int first_block(int u) const {
+    const long long need = (long long)128 * u * kstride + kspan - (kBlock - 1);
+    return need <= 0 ? 0 : (int)((need + kBlock - 1) / kBlock);
+  }
+  __host__ __device__ int entries(int u) const {
+    if (128 * u >= n_cmp) return 0;
+    const int f = first_block(u);
+    return f >= nqb ? 0 : group * (nqb - f);
+  }
+  __host__ __device__ int chunks(int u) const { return (entries(u) + chunk - 1) / chunk; }
+  __host__ __device__ int units() const { return (n_cmp + 127) / 128; }
+  __host__ __device__ int items() const {
+    int n = 0;
+    for (int u = 0; u < units(); ++u) n += chunks(u);
+    return n;
+  }
+};
+
+CmpSplit cmp_split(const Plan& p);
+int dkdv_list_cap(const Plan& p);
 
 struct BwdArgs {
   const __nv_bfloat16 *q, *k, *v, *w_p, *w_g, *out, *dout;
@@ -108,5 +143,9 @@ cudaError_t launch_state_bwd(const Plan& p, const BwdPlan& bp, const BwdArgs& a,
 cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_flash_dq(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_flash_dkdv(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+// NSA's branches
+cudaError_t launch_nsa_prep(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_flash_dkdv_cmp(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_cmp_reduce(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
 
 }  // namespace sla

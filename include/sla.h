@@ -322,8 +322,8 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
  *   dq                      bf16 [B, H, N, d]   written (padding rows 0)
  *   dk, dv                  bf16 [B, H_kv, N, d] written (padding rows 0)
  *   dw_p                    fp32, shape of w_p; written; may be NULL unless has_proj
- *   dw_g                    fp32 [H, d]; written; may be NULL unless has_gate
- *                           (the top-n mode has neither)
+ *   dw_g                    fp32 [H, d] ([H, 3, d] with nsa_branches); written; may
+ *                           be NULL unless has_gate (the plain top-n mode has neither)
  *   ws                      the workspace of that sla_forward call, unchanged
  *                           since: the routing, the states S'_i, Z_i, phi(Q),
  *                           the gate and the row log-sum-exp are read from it
@@ -337,9 +337,19 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
  *   top-n mode      the sparse branch only, over each query block's selected blocks and
  *                   window with the forward's element mask (s <= t, and block(s)
  *                   selected or s > t - window); dk, dv sum over the KV group's heads
+ *   nsa_branches    O = sum_b g_b o_b over the compressed (b = 0), selected (1) and
+ *                   window (2) branches, each its own softmax (sparse attention survey,
+ *                   section 2, NSA). With e_b = dO_t . o_b,t each branch's attention
+ *                   gradient is that of softmax attention with output gradient g_b dO;
+ *                   the compressed keys and values are block means, so token s gets
+ *                   1/cmp_block of the dK and dV of every compressed block that holds
+ *                   it; with gates dlogit_b = e_b g_b (1 - g_b): dq += sum_b dlogit_b
+ *                   w_g[h][b] and dw_g[h][b] += sum_t dlogit_b q_t. The forward call
+ *                   keeps each branch's row log-sum-exp and output in ws for this.
  * Errors as for sla_forward. The parameter gradients are sums of per-block
  * partials added with floating-point atomics, so their last bits may vary from
- * run to run; dq, dk and dv are deterministic.
+ * run to run; dq, dk and dv are deterministic (NSA's compressed-key gradients are
+ * summed from per-chunk partials in a fixed order).
  */
 SLA_API size_t sla_backward_workspace_bytes(const sla_config* cfg);
 SLA_API sla_status sla_backward(const void* q, const void* k, const void* v,

@@ -271,6 +271,16 @@ def test_backward_scope():
     topn = wl.preset("nsa_causal")
     assert sla.sla_backward_workspace_bytes(topn) > 0
     assert sla.sla_backward_stage_names(topn) == ["bwd_columns", "bwd_delta", "bwd_flash_dq", "bwd_flash_dkdv"]
+    # NSA's three branches: the compressed keys' gradients come before the token dK / dV
+    nsa = wl.preset("nsa_branches")
+    assert sla.sla_backward_workspace_bytes(nsa) > 0
+    assert sla.sla_backward_stage_names(nsa) == [
+        "bwd_columns", "bwd_nsa_prep", "bwd_flash_dq", "bwd_flash_dkdv_cmp", "bwd_cmp_reduce", "bwd_flash_dkdv"]
+    # no compressed block (fewer valid tokens than one compressed block): no compressed stages
+    short = wl.small_config(name="nsa_short", N=64, N_valid=20, d=64, H=2, H_kv=1, mode=wl.MODE_TOPN_WINDOW, causal=1,
+                            top_n=2, window=16, k_h=0, k_l=0, has_proj=0, nsa_branches=1, cmp_block=32,
+                            cmp_stride=16)
+    assert sla.sla_backward_stage_names(short) == ["bwd_columns", "bwd_nsa_prep", "bwd_flash_dq", "bwd_flash_dkdv"]
     bad = wl.small_config(N=1024, N_valid=1024, d=80)
     assert sla.sla_backward_workspace_bytes(bad) == 0 and sla.sla_backward_num_stages(bad) == -1
     assert _call_backward(bad) == sla.SLA_ERR_UNSUPPORTED
@@ -310,8 +320,8 @@ def test_nsa_branches_configuration():
                                       "sparse_flash_slc", "sparse_flash_win"]
     # the three branch outputs and the compressed keys add to the workspace
     assert sla.sla_workspace_bytes(c) > sla.sla_workspace_bytes(wl.preset("nsa_causal"))
-    # forward only; the gates belong to NSA's branches; no branches in the three-way mode
-    assert sla.sla_backward_workspace_bytes(c) == 0
+    # the gates belong to NSA's branches; no branches in the three-way mode
+    assert sla.sla_backward_workspace_bytes(c) > sla.sla_backward_workspace_bytes(wl.preset("nsa_causal"))
     assert sla.sla_validate_config(wl.preset("nsa_causal").replace(has_gate=1)) == sla.SLA_ERR_UNSUPPORTED
     assert sla.sla_validate_config(wl.preset("wan1.3b").replace(nsa_branches=1)) == sla.SLA_ERR_UNSUPPORTED
     assert sla.sla_validate_config(c.replace(cmp_stride=0)) == sla.SLA_ERR_INVALID_ARG

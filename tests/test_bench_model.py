@@ -87,3 +87,34 @@ def test_oracle_sample_extrapolates_set_up_and_units():
     assert r["heads"] == 2 and r["units"] == 8
     want = c.B * c.H * r["setup_s_per_head"] + c.B * c.H * c.nqb * r["unit_s"]
     assert abs(r["full_layer_s"] - want) <= 1e-12 * want
+
+
+def test_routing_report_checks_near_tie_rows():
+    """A row with a planted tie at the critical boundary: the oracle's own classes and the
+    classes with the two tied blocks swapped are both valid resolutions (one identical, one
+    not); swapping a critical block with a negligible one is invalid."""
+    c = wl.preset("tiny")
+    x = wl.generate(c)
+    L = bench.oracle_layer(c, x)
+    h, i = 1, 3
+    s = L.scores(0, h).copy()
+    order = np.argsort(-s[i], kind="stable")
+    a, b = order[c.k_h - 1], order[c.k_h]  # last critical, first marginal
+    s[i, b] = s[i, a]  # an exact tie across the boundary
+    L._scores[(0, h)] = s
+    L._cls.pop((0, h), None)
+    assert L.tie_rows(0, h)[i]
+    mask = np.stack([L.classes(0, g) for g in range(c.H)])[None]
+    rep = bench.routing_report(c, L, mask, [h])
+    assert rep["tie_rows"] >= 1 and rep["tie_rows_identical"] == rep["tie_rows"]
+    assert rep["tie_rows_invalid"] == 0
+    swapped = mask.copy()
+    swapped[0, h, i, a], swapped[0, h, i, b] = mask[0, h, i, b], mask[0, h, i, a]
+    rep = bench.routing_report(c, L, swapped, [h])
+    assert rep["tie_rows_identical"] == rep["tie_rows"] - 1 and rep["tie_rows_invalid"] == 0
+    assert rep["mismatched_rows"] == 0
+    bad = mask.copy()
+    top, last = order[0], order[-1]
+    bad[0, h, i, top], bad[0, h, i, last] = mask[0, h, i, last], mask[0, h, i, top]
+    rep = bench.routing_report(c, L, bad, [h])
+    assert rep["tie_rows_invalid"] == 1

@@ -71,7 +71,8 @@ def run_backward(cfg, seed=3, v_shift=0.0, keep=None):
         shape = (c.H, c.d, c.d) if c.proj_per_head else (c.d, c.d)
         dw_p = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
     if c.has_gate:
-        dw_g = torch.full((c.H, c.d), float("nan"), dtype=torch.float32, device="cuda")
+        shape = (c.H, 3, c.d) if c.nsa_branches else (c.H, c.d)
+        dw_g = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
     nbytes = sla.sla_backward_workspace_bytes(c)
     assert nbytes > 0
     bws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
@@ -108,6 +109,9 @@ def small(**kw):
     return wl.small_config(**kw)
 
 
+NSA = dict(mode=wl.MODE_TOPN_WINDOW, causal=1, k_h=0, k_l=0, has_proj=0, nsa_branches=1)
+
+
 CASES = [
     dict(name="all_crit_d64", N=768, N_valid=763, d=64, k_h=12, k_l=0),
     dict(name="all_crit_gqa_d128", N=1024, N_valid=1024, d=128, H=4, H_kv=2, k_h=16, k_l=0),
@@ -136,6 +140,19 @@ CASES = [
          causal=1, top_n=2, window=0, k_h=0, k_l=0, has_proj=0),
     dict(name="topn_window_only_d64", N=1024, N_valid=1000, d=64, H=4, H_kv=1, mode=wl.MODE_TOPN_WINDOW,
          causal=1, top_n=0, window=192, k_h=0, k_l=0, has_proj=0),
+    # NSA's three branches (compressed, selected, window; gated or summed): the gradient runs
+    # back through each branch's own softmax, the gates, and the block means of the
+    # compressed keys and values to every token they average
+    dict(name="nsa_gqa_gates_d128", N=2048, N_valid=2048, d=128, H=4, H_kv=2, top_n=4, window=256,
+         cmp_block=32, cmp_stride=16, has_gate=1, **NSA),
+    dict(name="nsa_odd_group_ragged_d64", N=1536, N_valid=1500, d=64, H=3, H_kv=1, top_n=3, window=100,
+         cmp_block=32, cmp_stride=16, has_gate=0, **NSA),
+    dict(name="nsa_unit_cmp_d128", N=1024, N_valid=1000, d=128, H=2, H_kv=2, top_n=2, window=64,
+         cmp_block=1, cmp_stride=1, has_gate=1, **NSA),
+    dict(name="nsa_wide_blocks_no_window_d64", N=2048, N_valid=2048, d=64, H=4, H_kv=1, top_n=2, window=0,
+         cmp_block=64, cmp_stride=48, has_gate=1, **NSA),
+    dict(name="nsa_many_cmp_tiles_d128", N=4096, N_valid=4033, d=128, H=2, H_kv=1, top_n=3, window=128,
+         cmp_block=32, cmp_stride=16, has_gate=1, **NSA),
 ]
 
 

@@ -32,7 +32,7 @@ def run_and_check_full(cfg, v_shift=0.0):
     run = DeviceRun(cfg, x)
     L = run.layer()
     rep = check_routing(run, L)
-    assert rep["mismatched_rows"] == 0, rep
+    assert rep["mismatched_rows"] == 0 and rep["tie_rows_invalid"] == 0, rep
     ref = L.forward()
     err = full_errors(run, ref)
     print(cfg.name, rep, err)
@@ -213,7 +213,7 @@ def test_cos_filter_matches_oracle(kw):
     run = DeviceRun(cfg, x)
     L = run.layer()
     rep = check_routing(run, L)
-    assert rep["mismatched_rows"] == 0, rep
+    assert rep["mismatched_rows"] == 0 and rep["tie_rows_invalid"] == 0, rep
     err = full_errors(run, L.forward())
     assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err
 
@@ -287,7 +287,7 @@ def test_full_size_workload(name):
     rep = check_routing(run, L)
     print(name, "routing", rep)
     report_routing(name, rep)
-    assert rep["mismatched_rows"] == 0, rep
+    assert rep["mismatched_rows"] == 0 and rep["tie_rows_invalid"] == 0, rep
     units = sampled_units(cfg)
     if cfg.mode == wl.MODE_THREEWAY and cfg.k_h > 0:
         longest, umax, emax = longest_pair_units(run)
@@ -307,7 +307,7 @@ def test_longest_supported_sequence():
     L = run.layer()
     rep = check_routing(run, L)
     print(cfg.name, "routing", rep)
-    assert rep["mismatched_rows"] == 0, rep
+    assert rep["mismatched_rows"] == 0 and rep["tie_rows_invalid"] == 0, rep
     assert rep["tie_rows"] < rep["rows"] // 4, rep
     err = unit_errors(run, L, sampled_units(cfg, n=6))
     print(cfg.name, "sampled output error", err)
