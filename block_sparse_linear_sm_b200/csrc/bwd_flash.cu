@@ -401,25 +401,45 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(S_READ + b));
       const int kc = k0 + 32 * hw;  // first key of this half
+      // warp-uniform: every (row, key) of this warp's 32 x 32 sub-tile is kept, so no
+      // per-element mask (rows t_w .. t_w + 31, keys kc .. kc + 31)
+      const int t_w = i_h[hf] * kBlock + ((quarter * 32) & 63);
+      bool full;
+      if (cmp_tile)
+        full = kc + 31 < prm.n_cmp && (kc + 31) * prm.kstride + prm.kspan <= t_w;
+      else {
+        full = kc + 31 < prm.n_valid;
+        if (TOPN) full = full && kc + 31 <= t_w && (sel || kc > t_w + 31 - prm.window);
+      }
+      full = full && act;
+      // P = 2^(s * scale * log2 e - lse), dS = P (dP - D), two columns per packed op
+      const uint64_t sc2 = tc::f2_pack(sl2, sl2), nl2 = tc::f2_pack(-lse2, -lse2), dl2 = tc::f2_pack(dlt, dlt);
       uint32_t ds[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float g2[2];
+      for (int j = 0; j < 16; ++j) ds[j] = 0u;  // a half that does not use the tile
+      if (act)
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int c = 2 * j + x;
-          const int key = kc + c;
-          bool keep;
-          if (cmp_tile)
-            keep = act && key < prm.n_cmp && key * prm.kstride + prm.kspan <= t;
-          else {
-            keep = act && key < prm.n_valid;
-            if (TOPN) keep = keep && key <= t && (sel || key > t - prm.window);
+      for (int j = 0; j < 16; ++j) {
+        const uint64_t y = tc::ffma2(tc::f2_pack(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), sc2, nl2);
+        float p0 = tc::ex2_approx(tc::f2_lo(y)), p1 = tc::ex2_approx(tc::f2_hi(y));
+        if (!full) {
+          bool keep[2];
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const int key = kc + 2 * j + x;
+            if (cmp_tile)
+              keep[x] = act && key < prm.n_cmp && key * prm.kstride + prm.kspan <= t;
+            else {
+              keep[x] = act && key < prm.n_valid;
+              if (TOPN) keep[x] = keep[x] && key <= t && (sel || key > t - prm.window);
+            }
           }
-          const float p = keep ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse2) : 0.f;
-          g2[x] = p * (__uint_as_float(pv[c]) - dlt);
+          p0 = keep[0] ? p0 : 0.f;
+          p1 = keep[1] ? p1 : 0.f;
         }
-        ds[j] = pack_bf16(g2[0], g2[1]);
+        const uint64_t g = tc::fmul2(tc::f2_pack(p0, p1),
+                                     tc::fsub2(tc::f2_pack(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1])), dl2));
+        ds[j] = pack_bf16(tc::f2_lo(g), tc::f2_hi(g));
       }
       // dS buffer b was last read by dQ_{m-2}
       if (m >= 2 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(DS_FREE + b), ((m - 2) >> 1) & 1, abort))))
@@ -810,39 +830,53 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       uint32_t sv[32], pv[32];
       tc::tmem_ld32(tS + 32 * hw, sv);
       tc::tmem_ld32(tS + 64 + 32 * hw, pv);
-      // this half's log-sum-exp and D values (one per query column), as vectors while the
-      // TMEM loads are in flight
-      const float4* lse4 =
-          reinterpret_cast<const float4*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile) + 8 * hw;
-      float lse[32], dl[32];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float4 a = lse4[j], d4 = lse4[16 + j];
-        lse[4 * j] = a.x; lse[4 * j + 1] = a.y; lse[4 * j + 2] = a.z; lse[4 * j + 3] = a.w;
-        dl[4 * j] = d4.x; dl[4 * j + 1] = d4.y; dl[4 * j + 2] = d4.z; dl[4 * j + 3] = d4.w;
-      }
+      // this half's log-sum-exp and D values (one per query column), read as pairs below
+      const uint64_t* lse2 =
+          reinterpret_cast<const uint64_t*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile) + 16 * hw;
+      const uint64_t* dl2 = lse2 + 32;
       tc::tmem_ld_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar(S_READ));
+      // warp-uniform: every (key, query) of this warp's 32 x 32 sub-tile is kept (keys
+      // k_w .. k_w + 31 all valid), so no per-element mask
+      const bool act_w = valid_j[hf] && ((e >> (kActBit + hf)) & 1u);
+      const int k_w = j_h[hf] * kBlock + ((quarter * 32) & 63);
+      bool full = act_w && k_w + 31 < (NSAC ? prm.n_cmp : prm.n_valid);
+      if (NSAC)
+        full = full && (k_w + 31) * prm.kstride + prm.kspan <= t0;
+      else if (TOPN)
+        full = full && k_w + 31 <= t0 && (sel || k_w > t0 + 31 - prm.window);
+      // P^T = 2^(s * scale * log2 e - lse), dS^T = P^T (dP^T - D), two columns per packed op
+      const uint64_t sc2 = tc::f2_pack(sl2, sl2);
       uint32_t pw[16], dw[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float pp[2], dd[2];
+      for (int j = 0; j < 16; ++j) pw[j] = dw[j] = 0u;  // a half that does not use the tile
+      if (act_w)
 #pragma unroll
-        for (int y = 0; y < 2; ++y) {
-          const int c = 2 * j + y;
-          bool keep = act;
-          if (NSAC)
-            keep = keep && key * prm.kstride + prm.kspan <= t0 + c;
-          else if (TOPN)
-            keep = keep && key <= t0 + c && (sel || key > t0 + c - prm.window);
-          const float p = keep ? tc::ex2_approx(__uint_as_float(sv[c]) * sl2 - lse[c]) : 0.f;
-          pp[y] = p;
-          dd[y] = p * (__uint_as_float(pv[c]) - dl[c]);
+      for (int j = 0; j < 16; ++j) {
+        const uint64_t y = tc::fsub2(tc::fmul2(tc::f2_pack(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), sc2),
+                                     lse2[j]);
+        float p0 = tc::ex2_approx(tc::f2_lo(y)), p1 = tc::ex2_approx(tc::f2_hi(y));
+        if (!full) {
+          bool keep[2];
+#pragma unroll
+          for (int x2 = 0; x2 < 2; ++x2) {
+            const int c = 2 * j + x2;
+            keep[x2] = act;
+            if (NSAC)
+              keep[x2] = keep[x2] && key * prm.kstride + prm.kspan <= t0 + c;
+            else if (TOPN)
+              keep[x2] = keep[x2] && key <= t0 + c && (sel || key > t0 + c - prm.window);
+          }
+          p0 = keep[0] ? p0 : 0.f;
+          p1 = keep[1] ? p1 : 0.f;
         }
-        pw[j] = pack_bf16(pp[0], pp[1]);
-        dw[j] = pack_bf16(dd[0], dd[1]);
+        const uint64_t p2 = tc::f2_pack(p0, p1);
+        const uint64_t d2 = tc::fmul2(p2, tc::fsub2(tc::f2_pack(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1])),
+                                                    dl2[j]));
+        pw[j] = pack_bf16(p0, p1);
+        dw[j] = pack_bf16(tc::f2_lo(d2), tc::f2_hi(d2));
       }
       // P / dS buffer x was last read by the products of tile m - 2
       if (m >= 2 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(PS_FREE + x), ((m - 2) >> 1) & 1, abort))))
