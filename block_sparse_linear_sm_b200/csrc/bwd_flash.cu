@@ -130,7 +130,9 @@ struct DqLayout {
   static constexpr int kOffBar = kOffRing + kBwSlots * kSlot;  // 32 mbarriers
   static constexpr int kOffMisc = kOffBar + 32 * 8;
   static constexpr int kOffList = kOffMisc + 64;          // merged block list
-  static constexpr int kTmemCols = 512;                   // dQ: D; S / dP: 2 x 128; dS: 2 x 32
+  static constexpr int kTmemCols = 512;                   // dQ: D; S / dP: 2 x 128; dS: 2 x 32; Q: D / 2
+  static constexpr int kQCol = D + 320;                   // Q as the A operand of S = Q K^T (bf16 pairs)
+  static_assert(kQCol + D / 2 <= kTmemCols, "TMEM columns");
 };
 
 struct DqParams {
@@ -181,8 +183,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
   // S / dP buffers: SP_FULL (products done), S_READ (row warps have loaded them);
   // dS buffers: DS_FULL (written), DS_FREE (dQ product done)
+  // Q_TMEM: the row warps have copied Q into TMEM (the A operand of S = Q K^T)
   constexpr int QO_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, S_READ = SP_FULL + 2,
-                DS_FULL = S_READ + 2, DS_FREE = DS_FULL + 2, ACC_DONE = DS_FREE + 2;
+                DS_FULL = S_READ + 2, DS_FREE = DS_FULL + 2, ACC_DONE = DS_FREE + 2, Q_TMEM = ACC_DONE + 1;
 
   // four bitmaps: active blocks of half 0 / 1, selected blocks of half 0 / 1 (top-n)
   for (int w = tid; w < 4 * prm.words; w += kBwThreads) words[w] = 0u;
@@ -200,6 +203,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tc::mbar_init(bar(DS_FREE + x), 1);
     }
     tc::mbar_init(bar(ACC_DONE), 1);
+    tc::mbar_init(bar(Q_TMEM), kRowWarps);
     tc::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -303,17 +307,18 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
     constexpr uint32_t kIdQ = tc::idesc_bf16(128, D, false, true);
     // base descriptors; a byte offset off is added as off >> 4 (start-address field)
-    const uint64_t dQd = tc::sw128_desc(sQ, 16, 1024), dOd = tc::sw128_desc(sO, 16, 1024);
+    const uint64_t dOd = tc::sw128_desc(sO, 16, 1024);
     const uint64_t dRk = tc::sw128_desc(sR, 16, 1024);    // ring tiles, K-major
     const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
-    // S_m = Q K_m^T and dP_m = dO V_m^T into TMEM buffer m & 1
+    // S_m = Q K_m^T (A = Q in TMEM: only K is read from shared memory, full rate at N = 64)
+    // and dP_m = dO V_m^T into TMEM buffer m & 1
     auto issue_sp = [&](int m) {
       const uint32_t so = (uint32_t)((m % S) * L::kSlot);
       const uint32_t tS = tmem + D + 128 * (m & 1);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t qo = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), ko = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
-        tc::mma_bf16_ss(tS, dQd + (qo >> 4), dRk + ((so + ko) >> 4), kIdS, k > 0);
+        tc::mma_bf16_ts(tS, tmem + L::kQCol + 8 * k, dRk + ((so + ko) >> 4), kIdS, k > 0);
         tc::mma_bf16_ss(tS + 64, dOd + (qo >> 4), dRk + ((so + L::kTile + ko) >> 4), kIdS, k > 0);
       }
       tc::mma_commit(bar(SP_FULL + (m & 1)));
@@ -321,7 +326,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     auto wait_loaded = [&](int m) -> bool {
       return __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
     };
-    bool ok = T == 0 || __all_sync(kAll, tc::mbar_wait(bar(QO_FULL), 0, abort));
+    bool ok = T == 0 || (__all_sync(kAll, tc::mbar_wait(bar(QO_FULL), 0, abort)) &&
+                         __all_sync(kAll, tc::mbar_wait(bar(Q_TMEM), 0, abort)));
     for (int m = 0; m < 2 && m < T && ok; ++m) {
       ok = wait_loaded(m);
       tc::fence_after_sync();
@@ -379,6 +385,30 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
     const float sl2 = prm.scale_log2;
     bool ok = true;
+    if (T > 0) {
+      // Q row r (the TMEM lane) into columns kQCol.. as bf16 pairs, this warpgroup's half of
+      // the features: from the swizzled Q tile (16-byte chunk c of a row at c ^ (row & 7))
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(QO_FULL), 0, abort));
+      if (ok) {
+        constexpr int CH = D / 16;  // 16-byte chunks per warpgroup half: 8 (D = 128) or 4
+        uint32_t qv[CH * 4];
+#pragma unroll
+        for (int x = 0; x < CH; ++x) {
+          const int chunk = hw * CH + x;  // of the row's D / 8 chunks
+          const int p = chunk >> 3, c = chunk & 7;
+          const uint4 u = *reinterpret_cast<const uint4*>(smem + L::kOffQ + p * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+          qv[4 * x] = u.x; qv[4 * x + 1] = u.y; qv[4 * x + 2] = u.z; qv[4 * x + 3] = u.w;
+        }
+        if constexpr (CH * 4 == 32)
+          tc::tmem_st32(tmem + lane_off + L::kQCol + 32 * hw, *reinterpret_cast<const uint32_t(*)[32]>(qv));
+        else
+          tc::tmem_st16(tmem + lane_off + L::kQCol + 16 * hw, *reinterpret_cast<const uint32_t(*)[16]>(qv));
+        tc::tmem_st_wait();
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(Q_TMEM));
+    }
     for (int m = 0; m < T && ok; ++m) {
       const int b = m & 1;
       const uint32_t e = mlist[m];
