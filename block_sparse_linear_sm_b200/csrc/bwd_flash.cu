@@ -80,7 +80,6 @@ enum NsaBranch { kBrCmp = 0, kBrSel = 1, kBrWin = 2 };
 
 constexpr int kBwThreads = 320;  // warps 0-7 rows (two column halves), warp 8 MMA, warp 9 TMA producer
 constexpr int kMmaWarp = 8, kProdWarp = 9, kRowWarps = 8;
-constexpr int kBwSlots = 4;      // ring slots
 
 // merged list of two bitmaps (warp 0, ascending). Entry = index (bits 0-12) | a0 << 13 | a1 << 14
 // | s0 << 15 | s1 << 16 | tag << 17: a0 / a1 = the index is in bitmap a0 / a1 ("active" for
@@ -119,7 +118,7 @@ __device__ __forceinline__ int merge_bitmaps(const uint32_t* a0p, const uint32_t
 // ---------------------------------------------------------------------------
 // dQ
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int SL>  // SL ring slots
 struct DqLayout {
   static constexpr int NP = D / 64;
   static constexpr int kOffQ = 0;                         // Q: 128 rows, NP panels of 16 KB
@@ -127,7 +126,7 @@ struct DqLayout {
   static constexpr int kTile = NP * 8192;                 // one 64-row K or V tile
   static constexpr int kSlot = 2 * kTile;                 // K_j, V_j
   static constexpr int kOffRing = kOffO + NP * 16384;
-  static constexpr int kOffBar = kOffRing + kBwSlots * kSlot;  // 32 mbarriers
+  static constexpr int kOffBar = kOffRing + SL * kSlot;  // 32 mbarriers
   static constexpr int kOffMisc = kOffBar + 32 * 8;
   static constexpr int kOffList = kOffMisc + 64;          // merged block list
   static constexpr int kTmemCols = 512;                   // dQ: D; S / dP: 2 x 128; dS: 2 x 32; Q: D / 2
@@ -157,15 +156,15 @@ struct DqParams {
 // NSA: the list holds three kinds of tiles, tagged with their branch: compressed key tiles
 // (tmKc / tmVc; key c kept when c < n_cmp and c * kstride + kspan <= t), selected blocks
 // (s <= t) and window blocks (t - window < s <= t). All of them add to one dQ accumulator.
-template <int D, int MODE>
+template <int D, int MODE, int SL>
 __global__ void __launch_bounds__(kBwThreads, 1)
     flash_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
                     DqParams prm) {
   constexpr bool TOPN = MODE != kModeThree, NSA = MODE == kModeNsa;
-  using L = DqLayout<D>;
-  constexpr int NP = L::NP, S = kBwSlots;
+  using L = DqLayout<D, SL>;
+  constexpr int NP = L::NP, S = SL;
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -547,15 +546,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 // ---------------------------------------------------------------------------
 // dK, dV
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int SL>  // SL ring slots
 struct DkvLayout {
   static constexpr int NP = D / 64;
   static constexpr int kOffK = 0;                              // K: 128 keys, NP panels of 16 KB
   static constexpr int kOffV = kOffK + NP * 16384;             // V
   static constexpr int kTile = NP * 8192;                      // one 64-row Q or dO tile
-  static constexpr int kSlot = (2 * kTile + 512 + 1023) / 1024 * 1024;  // Q_i, dO_i, lse_i, delta_i
+  static constexpr int kSlot = 2 * kTile;                      // Q_i, dO_i
   static constexpr int kOffRing = kOffV + NP * 16384;
-  static constexpr int kOffBar = kOffRing + kBwSlots * kSlot;
+  static constexpr int kOffLD = kOffRing + SL * kSlot;         // lse_i, delta_i of each slot (512 bytes)
+  static constexpr int kOffBar = kOffLD + SL * 512;
   static constexpr int kOffMisc = kOffBar + 32 * 8;
   static constexpr int kSmem = kOffMisc + 64;
   static constexpr int kTmemCols = 512;  // dV, dK: 2 D; S^T / dP^T: 128; P^T / dS^T: 2 x 64 (bf16 pairs)
@@ -596,14 +596,14 @@ struct DkvParams {
 // branch's log-sum-exp and D), and the epilogue adds the compressed branch's share.
 // NSA compressed keys (kModeNsaCmp): tmK / tmV map the compressed keys; key c is kept
 // for query t when c < n_cmp and c * kstride + kspan <= t; raw fp32 partials out.
-template <int D, int MODE>
+template <int D, int MODE, int SL>
 __global__ void __launch_bounds__(kBwThreads, 1)
     flash_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       DkvParams prm) {
   constexpr bool TOPN = MODE != kModeThree, NSAT = MODE == kModeNsaTok, NSAC = MODE == kModeNsaCmp;
-  using L = DkvLayout<D>;
-  constexpr int NP = L::NP, S = kBwSlots;
+  using L = DkvLayout<D, SL>;
+  constexpr int NP = L::NP, S = SL;
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -753,8 +753,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           tc::tma_load_3d(dst + p * 8192, &tmQ, bar(LOADED + slot), 64 * p, i * kBlock, bh);
           tc::tma_load_3d(dst + L::kTile + p * 8192, &tmO, bar(LOADED + slot), 64 * p, i * kBlock, bh);
         }
-        tc::bulk_load(dst + 2 * L::kTile, prm.lse + boff + (size_t)bh * prm.N + i * kBlock, 256, bar(LOADED + slot));
-        tc::bulk_load(dst + 2 * L::kTile + 256, prm.delta + boff + (size_t)bh * prm.N + i * kBlock, 256,
+        const uint32_t ld = sbase + L::kOffLD + slot * 512;
+        tc::bulk_load(ld, prm.lse + boff + (size_t)bh * prm.N + i * kBlock, 256, bar(LOADED + slot));
+        tc::bulk_load(ld + 256, prm.delta + boff + (size_t)bh * prm.N + i * kBlock, 256,
                       bar(LOADED + slot));
       }
       // the last release of every slot: no product reads the ring and no commit is in flight at exit
@@ -862,7 +863,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tc::tmem_ld32(tS + 64 + 32 * hw, pv);
       // this half's log-sum-exp and D values (one per query column), read as pairs below
       const uint64_t* lse2 =
-          reinterpret_cast<const uint64_t*>(smem + L::kOffRing + slot * L::kSlot + 2 * L::kTile) + 16 * hw;
+          reinterpret_cast<const uint64_t*>(smem + L::kOffLD + slot * 512) + 16 * hw;
       const uint64_t* dl2 = lse2 + 32;
       tc::tmem_ld_wait();
       tc::fence_before_sync();
@@ -1019,14 +1020,40 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+// capacity of the dQ kernel's merged block list (at least 1)
+static int dq_list_cap(const Plan& p) {
+  const sla_config& c = p.c;
+  const bool topn = c.mode == SLA_MODE_TOPN_WINDOW;
+  int per_half = topn ? c.top_n : c.k_h;
+  if (topn) per_half += (c.window + 62) / kBlock + 2;  // selected blocks plus the window's reach
+  int cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
+  if (topn && c.nsa_branches) {  // compressed tiles, then the selected and the window blocks (two halves each)
+    const int sel = 2 * c.top_n < p.nkb ? 2 * c.top_n : p.nkb;
+    const int win = 2 * ((c.window + 62) / kBlock + 2) < p.nkb ? 2 * ((c.window + 62) / kBlock + 2) : p.nkb;
+    cap = p.ncmp_pad / kBlock + sel + win;
+  }
+  return cap > 0 ? cap : 1;
+}
+
 static bool map64(CUtensorMap* m, const void* base, int heads, int n_rows, int N, int D) {
   return make_tmap_3d(m, base, (uint64_t)D, (uint64_t)n_rows, (uint64_t)heads, (uint64_t)D * 2,
                       (uint64_t)N * D * 2, 64, 64);
 }
 
+template <int D, int MODE, int SL>
+static cudaError_t launch_dq_slots(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+
+// five ring slots where they fit in shared memory (the K / V loads then start one tile
+// earlier), else four
 template <int D, int MODE>
 static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
-  using L = DqLayout<D>;
+  return dq_list_cap(p) * 4 + DqLayout<D, 5>::kOffList <= 227 * 1024 ? launch_dq_slots<D, MODE, 5>(p, bp, a, s)
+                                                                    : launch_dq_slots<D, MODE, 4>(p, bp, a, s);
+}
+
+template <int D, int MODE, int SL>
+static cudaError_t launch_dq_slots(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  using L = DqLayout<D, SL>;
   constexpr bool TOPN = MODE != kModeThree, NSA = MODE == kModeNsa;
   const sla_config& c = p.c;
   CUtensorMap mq, mo, mk, mv, mkc, mvc;
@@ -1068,21 +1095,13 @@ static cudaError_t launch_dq_t(const Plan& p, const BwdPlan& bp, const BwdArgs& 
     prm.kstride = c.cmp_stride;
     prm.kspan = c.cmp_block - 1;
   }
-  int per_half = prm.len;
-  if (TOPN) per_half += (c.window + 62) / kBlock + 2;  // selected blocks plus the window's reach
-  int cap = 2 * per_half < p.nkb ? 2 * per_half : p.nkb;
-  if (NSA) {  // compressed tiles, then the selected and the window blocks, each a union over two halves
-    const int sel = 2 * c.top_n < p.nkb ? 2 * c.top_n : p.nkb;
-    const int win = 2 * ((c.window + 62) / kBlock + 2) < p.nkb ? 2 * ((c.window + 62) / kBlock + 2) : p.nkb;
-    cap = p.ncmp_pad / kBlock + sel + win;
-  }
-  int smem = L::kOffList + (cap > 0 ? cap : 1) * 4;
-  if (4 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
+  int smem = L::kOffList + dq_list_cap(p) * 4;
+  if (4 * prm.words * 4 > SL * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: it holds all 512 TMEM columns
-  cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D, MODE, SL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dq_kernel<D, MODE><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, mkc, mvc, prm);
+  flash_dq_kernel<D, MODE, SL><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, mkc, mvc, prm);
   return cudaGetLastError();
 }
 
@@ -1114,9 +1133,19 @@ CmpSplit cmp_split(const Plan& p) {
   return sp;
 }
 
+template <int D, int MODE, int SL>
+static cudaError_t launch_dkdv_slots(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s);
+
+// five ring slots where they fit in shared memory, else four
 template <int D, int MODE>
 static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
-  using L = DkvLayout<D>;
+  return DkvLayout<D, 5>::kSmem <= 227 * 1024 ? launch_dkdv_slots<D, MODE, 5>(p, bp, a, s)
+                                              : launch_dkdv_slots<D, MODE, 4>(p, bp, a, s);
+}
+
+template <int D, int MODE, int SL>
+static cudaError_t launch_dkdv_slots(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cudaStream_t s) {
+  using L = DkvLayout<D, SL>;
   constexpr bool TOPN = MODE != kModeThree, NSAT = MODE == kModeNsaTok, NSAC = MODE == kModeNsaCmp;
   const sla_config& c = p.c;
   CUtensorMap mq, mo, mk, mv;
@@ -1175,11 +1204,11 @@ static cudaError_t launch_dkdv_t(const Plan& p, const BwdPlan& bp, const BwdArgs
     if (grid == 0) return cudaSuccess;
   }
   int smem = L::kSmem;
-  if (TOPN && 4 * prm.words * 4 > kBwSlots * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
+  if (TOPN && 4 * prm.words * 4 > SL * L::kSlot) return cudaErrorInvalidValue;  // bitmaps in the ring
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (512 TMEM columns)
-  cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D, MODE, SL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dkdv_kernel<D, MODE><<<grid, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  flash_dkdv_kernel<D, MODE, SL><<<grid, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
   return cudaGetLastError();
 }
 
