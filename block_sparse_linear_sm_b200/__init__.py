@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.sla_route.restype = ctypes.c_int
         L.sla_forward.argtypes = [P, P, P, P, P, C, P, P, P, S, P]
         L.sla_forward.restype = ctypes.c_int
+        L.sla_forward_blocks.argtypes = [P, P, P, P, P, C, I32, I32, P, P, P, S, P]
+        L.sla_forward_blocks.restype = ctypes.c_int
         L.sla_forward_timed.argtypes = [P, P, P, P, P, C, P, P, P, S, P,
                                         ctypes.POINTER(ctypes.c_void_p), I32]
         L.sla_forward_timed.restype = ctypes.c_int
@@ -184,6 +186,15 @@ def sla_forward(q, k, v, w_p, w_g, c, out, mask_out, ws, stream=None) -> None:
     _check(lib().sla_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(w_p), _ptr(w_g), ctypes.byref(cfg),
                              _ptr(out), _ptr(mask_out), _ptr(ws), ws_bytes, _stream(stream)),
            "sla_forward")
+
+
+def sla_forward_blocks(q, k, v, w_p, w_g, c, qb_begin, qb_end, out, mask_out, ws, stream=None) -> None:
+    """sla_forward writing only the output rows of query blocks [qb_begin, qb_end)."""
+    cfg = _cfg(c)
+    ws_bytes = ws.numel() * ws.element_size()
+    _check(lib().sla_forward_blocks(_ptr(q), _ptr(k), _ptr(v), _ptr(w_p), _ptr(w_g), ctypes.byref(cfg),
+                                    int(qb_begin), int(qb_end), _ptr(out), _ptr(mask_out), _ptr(ws), ws_bytes,
+                                    _stream(stream)), "sla_forward_blocks")
 
 
 def sla_forward_timed(q, k, v, w_p, w_g, c, out, mask_out, ws, events, stream=None) -> None:

@@ -42,7 +42,8 @@ struct AggParams {
   float* zs;  // [B*H][nqb][d]
   int* status;
   int H, group, nqb, nk_steps, d;
-  int m_tiles, n_tiles, tiles;  // tile t: m = t % m_tiles, n = (t / m_tiles) % n_tiles, bh = rest
+  int m_tiles, n_tiles, tiles;  // tile t: m = m_first + t % m_tiles, n = (t / m_tiles) % n_tiles, bh = rest
+  int m_first;                  // first row tile (a call that writes a range of query blocks)
 };
 
 __global__ void __launch_bounds__(kAgThreads, 1)
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kAgThreads, 1)
   const int my_tiles = prm.tiles > (int)blockIdx.x ? (prm.tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   auto tile_of = [&](int i, int& m0, int& n0, int& bh) {
     const int t = (int)blockIdx.x + i * (int)gridDim.x;
-    m0 = (t % prm.m_tiles) * kAgBM;
+    m0 = (prm.m_first + t % prm.m_tiles) * kAgBM;
     n0 = ((t / prm.m_tiles) % prm.n_tiles) * kAgBN;
     bh = t / (prm.m_tiles * prm.n_tiles);
   };
@@ -264,7 +265,9 @@ cudaError_t launch_aggregate(const Plan& p, const Args& a, cudaStream_t s) {
   prm.nqb = p.nqb;
   prm.nk_steps = p.nkb_pad / 64;
   prm.d = c.d;
-  prm.m_tiles = (p.nqb + kAgBM - 1) / kAgBM;
+  // the row tiles that hold the call's query blocks [qb0, qb1)
+  prm.m_first = p.qb0 / kAgBM;
+  prm.m_tiles = (p.qb1 + kAgBM - 1) / kAgBM - prm.m_first;
   prm.n_tiles = (p.dd + kAgBN - 1) / kAgBN;
   prm.tiles = prm.m_tiles * prm.n_tiles * c.B * c.H;
   cudaError_t e = cudaFuncSetAttribute(aggregate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -308,6 +311,7 @@ cudaError_t launch_aggregate_t(const Plan& p, const BwdPlan& bp, const BwdArgs& 
   prm.nqb = p.nkb;
   prm.nk_steps = bp.rows_t / 64;
   prm.d = c.d;
+  prm.m_first = 0;
   prm.m_tiles = (p.nkb + kAgBM - 1) / kAgBM;
   prm.n_tiles = (p.dd + kAgBN - 1) / kAgBN;
   prm.tiles = prm.m_tiles * prm.n_tiles * (int)bkv;

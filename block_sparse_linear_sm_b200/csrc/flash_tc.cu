@@ -49,6 +49,8 @@ struct FlashTcParams {
   const float* gate;   // fused epilogue: g_t = sigmoid(q_t . w_g[h]) [B*H][N] (fp32) or null
   float* lse;           // [B*H][N] row log2-sum-exp of the scaled scores (+inf: no key), or null
   int npairs;           // units per (b, h) when pairing query blocks
+  int pair0;            // first pair of query blocks (pairing query blocks)
+  int qb_first, qb_count;  // query blocks of the units (pairing heads)
   int words;            // 32-bit words of one block bitmap
   int list_cap;         // capacity of the merged list
   // Keys: n_keys valid keys in nkt 64-key tiles. Key index c stands for token
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   {
     const int u = blockIdx.x;
     if (!prm.pair_heads) {
-      const int bh = u / prm.npairs, p = u % prm.npairs;
+      const int bh = u / prm.npairs, p = prm.pair0 + u % prm.npairs;
       const int b = bh / prm.H, h = bh % prm.H;
       bkv = b * Hkv + h / prm.group;
       for (int hf = 0; hf < 2; ++hf) {
@@ -146,8 +148,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const int hp_n = prm.group / 2;
       const int hp = u % hp_n;
       const int rest = u / hp_n;
-      const int i = rest % prm.nb;
-      bkv = rest / prm.nb;
+      const int i = prm.qb_first + rest % prm.qb_count;
+      bkv = rest / prm.qb_count;
       const int b = bkv / Hkv, g = bkv % Hkv;
       for (int hf = 0; hf < 2; ++hf) {
         bh_h[hf] = b * prm.H + g * prm.group + 2 * hp + hf;
@@ -842,7 +844,11 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
   prm.len = (branch == 1 || branch == 3) ? 0 : (TOPN ? c.top_n : c.k_h);
   prm.window = (branch == 1 || branch == 2) ? 0 : c.window;
   prm.pair_heads = TOPN && (p.group % 2 == 0);
-  prm.npairs = (p.nqb + 1) / 2;
+  // the query blocks [qb0, qb1) of the call: pairs qb0 / 2 .. (qb1 + 1) / 2 - 1
+  prm.pair0 = p.qb0 / 2;
+  prm.npairs = (p.qb1 + 1) / 2 - p.qb0 / 2;
+  prm.qb_first = p.qb0;
+  prm.qb_count = p.qb1 - p.qb0;
   prm.n_keys = cmp ? p.n_cmp : c.N_valid;
   prm.nkt = cmp ? p.ncmp_pad / kBlock : p.nkb;
   prm.kstride = cmp ? c.cmp_stride : 1;
@@ -865,7 +871,7 @@ static cudaError_t launch_tc(const Plan& p, const Args& a, int branch, cudaStrea
   if (e != cudaSuccess) return e;
   int units;
   if (prm.pair_heads)
-    units = c.B * c.H_kv * p.nqb * (p.group / 2);
+    units = c.B * c.H_kv * prm.qb_count * (p.group / 2);
   else
     units = c.B * c.H * prm.npairs;
   flash_tc_kernel<D, TOPN, FUSE, KMAP, NSAC><<<units, kTcThreads, smem, s>>>(mq, mk, mv, ms, mf, prm);

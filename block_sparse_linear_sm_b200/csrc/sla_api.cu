@@ -58,6 +58,8 @@ bool make_plan(const sla_config* c, Plan* p) {
   p->group = c->H / c->H_kv;
   p->nqb_pad = (int)align_up(p->nqb, 128);
   p->nkb_pad = (int)align_up(p->nkb, 64);
+  p->qb0 = 0;
+  p->qb1 = p->nqb;
   p->dd = (int)align_up((size_t)c->d * c->d + c->d, 128);
   p->scale = c->scale > 0.f ? c->scale : 1.f / sqrtf((float)c->d);
   const size_t B = c->B, H = c->H, Hkv = c->H_kv, d = c->d, nqb = p->nqb, nkb = p->nkb;
@@ -183,11 +185,17 @@ cudaError_t route_stages(const Plan& p, const Args& a, cudaStream_t s) {
 static sla_status forward_impl(const void* q, const void* k, const void* v, const void* w_p,
                                const void* w_g, const sla_config* cfg, void* out, int8_t* mask_out,
                                void* ws, size_t ws_bytes, void* stream, void* const* events,
-                               int32_t n_events) {
+                               int32_t n_events, int32_t qb_begin = 0, int32_t qb_end = -1) {
   Plan p;
   sla_status st = check_config(cfg);
   if (st != SLA_OK) return st;
   make_plan(cfg, &p);
+  if (qb_end < 0) qb_end = p.nqb;
+  // a range of query blocks starts on a pair of blocks (the flash kernel's 128-row units)
+  if (qb_begin < 0 || qb_begin >= qb_end || qb_end > p.nqb || (qb_begin & 1) || ((qb_end & 1) && qb_end != p.nqb))
+    return SLA_ERR_INVALID_ARG;
+  p.qb0 = qb_begin;
+  p.qb1 = qb_end;
   if (!q || !k || !v || !out) return SLA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return SLA_ERR_INVALID_ARG;
@@ -440,6 +448,12 @@ sla_status sla_forward(const void* q, const void* k, const void* v, const void* 
                        const void* w_g, const sla_config* cfg, void* out, int8_t* mask_out,
                        void* ws, size_t ws_bytes, void* stream) {
   return forward_impl(q, k, v, w_p, w_g, cfg, out, mask_out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+sla_status sla_forward_blocks(const void* q, const void* k, const void* v, const void* w_p,
+                              const void* w_g, const sla_config* cfg, int32_t qb_begin, int32_t qb_end,
+                              void* out, int8_t* mask_out, void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(q, k, v, w_p, w_g, cfg, out, mask_out, ws, ws_bytes, stream, nullptr, 0, qb_begin, qb_end);
 }
 
 sla_status sla_forward_timed(const void* q, const void* k, const void* v, const void* w_p,

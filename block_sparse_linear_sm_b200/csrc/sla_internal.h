@@ -39,6 +39,9 @@ struct Plan {
   // (compressed, selected, window)
   int n_cmp, ncmp_pad;
   size_t off_kc, off_vc, off_oc, off_os, off_ow;
+  // query blocks whose output rows this call writes: [qb0, qb1) (the whole layer by
+  // default; sla_forward_blocks narrows it, qb0 even)
+  int qb0, qb1;
 };
 
 bool make_plan(const sla_config* c, Plan* p);

@@ -189,3 +189,121 @@ class HeadShard:
         if w_g is not None:
             lwg = torch.index_select(w_g, 0, torch.as_tensor(self.heads, device=w_g.device)).contiguous()
         return lq, lk, lv, lwp, lwg
+
+
+# ---------------------------------------------------------------------------
+# block level (db-SP's second level): KV groups split into ranges of query blocks
+# ---------------------------------------------------------------------------
+
+def pair_costs(cfg: wl.LayerConfig, crit: Optional[np.ndarray] = None) -> np.ndarray:
+    """Estimated work per (KV group, pair of query blocks), in 64 x 64 flash tiles (float64
+    [H_kv, npairs]): the pair's merged block list for every head of the group (top-n mode:
+    its selected blocks and the window's blocks) plus, with a linear branch, the
+    aggregation rows of the pair. ``crit`` as for unit_costs; without it every pair costs
+    the same."""
+    c = cfg
+    group = c.H // c.H_kv
+    npairs = (c.nqb + 1) // 2
+    if crit is None:
+        return np.ones((c.H_kv, npairs))
+    cost = np.zeros((c.H_kv, npairs))
+    if c.mode == wl.MODE_THREEWAY:
+        marg = c.nqb - c.k_h - c.k_l > 0 or c.linear_all
+        # aggregation of one query block row: 2 * nkb * (d^2 + d) against 4 * 64^2 * d per tile
+        agg = (2.0 * c.nkb * c.d * c.d) / (4.0 * 64 * 64 * c.d) if marg else 0.0
+        for b in range(c.B):
+            for h in range(c.H):
+                for p in range(npairs):
+                    rows = crit[b, h, 2 * p:2 * p + 2].reshape(-1)
+                    n_rows = min(2, c.nqb - 2 * p)
+                    cost[h // group, p] += np.unique(rows[rows >= 0]).size + agg * n_rows
+    else:
+        wb = (c.window + 62) // 64 + 1 if c.window > 0 else 0
+        for b in range(c.B):
+            for hk in range(c.H_kv):
+                for i in range(c.nqb):
+                    sel = crit[b, hk, i]
+                    cost[hk, i // 2] += (np.unique(sel[sel >= 0]).size + min(wb, i + 1)) * group
+    return cost
+
+
+def fixed_costs(cfg: wl.LayerConfig, costs: np.ndarray, share: float = 0.5) -> np.ndarray:
+    """Work of a KV group that every call holding any of its query blocks repeats (routing,
+    key pooling, linear states), as ``share`` of the group's mean per-head flash work. With
+    the Wan-1.3B layer the router and the state kernels take about half the flash kernel's
+    time (0.15 + 0.11 against 0.46 ms)."""
+    group = cfg.H // cfg.H_kv
+    return np.full(cfg.H_kv, share * float(np.mean(costs.sum(axis=1))) / group * group)
+
+
+def block_plan(costs: np.ndarray, fixed: np.ndarray, world: int) -> List[List[tuple]]:
+    """Pieces (KV group, first pair, end pair) of every rank: the (group, pair) units in
+    group-major order cut into world contiguous runs of about equal work, so a rank holds
+    at most two partial groups. A run ends inside a group when the next pair would take
+    the rank past its share; every rank that holds part of a group pays the group's fixed
+    work, and the share counts the fixed work of the world - 1 cuts. Deterministic: every
+    rank computes the same plan. Returns, per rank, a list of (unit, p0, p1), p0 < p1."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    n_units, npairs = costs.shape
+    mean_fixed = float(np.mean(fixed)) if n_units else 0.0
+    target = (float(costs.sum()) + float(fixed.sum()) + (world - 1) * mean_fixed) / world
+    plan: List[List[tuple]] = [[] for _ in range(world)]
+    r, load = 0, 0.0
+    for u in range(n_units):
+        p = 0
+        while p < npairs:
+            load += float(fixed[u])  # this rank starts on (part of) group u
+            q = p
+            while q < npairs and (r == world - 1 or q == p or load + float(costs[u, q]) <= target):
+                load += float(costs[u, q])
+                q += 1
+            plan[r].append((u, p, q))
+            if r < world - 1 and (q < npairs or load >= target):  # this rank's share is used up
+                r, load = r + 1, 0.0
+            p = q
+    return plan
+
+
+def block_plan_loads(costs: np.ndarray, fixed: np.ndarray, plan: List[List[tuple]]) -> List[float]:
+    """Work of each rank under a block plan: its pairs plus the fixed work of each group it
+    touches."""
+    out = []
+    for pieces in plan:
+        units = {u for u, _, _ in pieces}
+        out.append(float(sum(costs[u, p0:p1].sum() for u, p0, p1 in pieces) + sum(fixed[u] for u in units)))
+    return out
+
+
+class BlockShard:
+    """This rank's share of a block-split layer: for every piece (KV group, pairs p0..p1)
+    it runs the layer on the group's heads through sla_forward_blocks, which writes the
+    output rows of query blocks 2 p0 .. 2 p1 - 1."""
+
+    def __init__(self, cfg: wl.LayerConfig, world: int, rank: int, costs: Optional[np.ndarray] = None,
+                 fixed: Optional[np.ndarray] = None):
+        self.cfg = cfg
+        self.costs = pair_costs(cfg) if costs is None else np.asarray(costs, dtype=np.float64)
+        self.fixed = fixed_costs(cfg, self.costs) if fixed is None else np.asarray(fixed, dtype=np.float64)
+        self.plan = block_plan(self.costs, self.fixed, world)
+        self.pieces = self.plan[rank]
+
+    def run(self, sla, q, k, v, w_p, w_g, out, ws_for, stream=None):
+        """Runs this rank's pieces; ``out`` [B, H, N, d] receives their rows (the others
+        are not written). ``ws_for(local_cfg)`` returns a workspace for that config."""
+        c = self.cfg
+        group = c.H // c.H_kv
+        for u, p0, p1 in self.pieces:
+            heads = query_heads(c, [u])
+            lc = local_config(c, [u])
+            lq, lk, lv = gather_heads(q, heads), gather_heads(k, [u]), gather_heads(v, [u])
+            lwp = w_p
+            if w_p is not None and c.proj_per_head:
+                lwp = w_p[u * group:(u + 1) * group].contiguous()
+            lwg = None if w_g is None else w_g[u * group:(u + 1) * group].contiguous()
+            lout = out[:, u * group:(u + 1) * group]
+            local = lout if lout.is_contiguous() else lout.contiguous()
+            qb0, qb1 = 2 * p0, min(2 * p1, c.nqb)
+            sla.sla_forward_blocks(lq, lk, lv, lwp, lwg, lc, qb0, qb1, local, None, ws_for(lc), stream)
+            if local is not lout:
+                lout[:, :, qb0 * 64:qb1 * 64] = local[:, :, qb0 * 64:qb1 * 64]

@@ -184,6 +184,27 @@ SLA_API sla_status sla_forward(const void* q, const void* k, const void* v,
                        void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * sla_forward restricted to the output rows of query blocks [qb_begin, qb_end) of every
+ * head of cfg: the block level of db-SP's partitioning (sparse attention survey, db-SP:
+ * work split at the head level and the block level so that devices get equal sparse
+ * work). A head whose query blocks are split over several calls (or devices) costs each
+ * of them its whole routing, key pooling and linear states (the key side of a row needs
+ * every key block), while the flash kernel and the aggregation run only for the range.
+ *   qb_begin, qb_end   0 <= qb_begin < qb_end <= N / block; qb_begin even, and qb_end even
+ *                      or N / block (the flash kernel works on pairs of query blocks);
+ *                      else SLA_ERR_INVALID_ARG
+ *   out                bf16 [B, H, N, d]: only the rows of the range are written (padding
+ *                      rows among them as 0); the others keep their contents
+ *   mask_out, ws       as sla_forward (mask_out receives the whole routing mask)
+ * The rows written are bit-identical to those of a whole-layer sla_forward. The backward
+ * pass reads a whole-layer sla_forward's workspace, not this call's.
+ */
+SLA_API sla_status sla_forward_blocks(const void* q, const void* k, const void* v,
+                                      const void* w_p, const void* w_g, const sla_config* cfg,
+                                      int32_t qb_begin, int32_t qb_end, void* out, int8_t* mask_out,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/*
  * sla_forward that also records caller-created CUDA events (cudaEvent_t,
  * passed as void*) on `stream` around its launches: events[0] before the first
  * launch and events[s + 1] after stage s, for s < sla_num_stages(cfg).

@@ -344,3 +344,15 @@ def test_noalloc_entry_points_reject_bad_arguments_without_a_device():
     if not has_gpu:
         detail = ctypes.c_int32(0)
         assert L.sla_route_noalloc_status(None, ctypes.byref(detail)) == sla.SLA_ERR_CUDA
+
+
+def test_forward_blocks_rejects_bad_ranges_before_launch():
+    """sla_forward_blocks: the query-block range starts on a pair, is not empty and stays
+    inside the layer (an odd end only at the last block); checked before any launch."""
+    c = sla.make_config(wl.small_config(N=1216, N_valid=1200, d=64))  # 19 query blocks
+    L = sla.lib()
+    ws = 256
+    nbytes = sla.sla_workspace_bytes(wl.small_config(N=1216, N_valid=1200, d=64))
+    for qb0, qb1 in ((1, 4), (0, 0), (4, 2), (0, 20), (2, 5), (-2, 4)):
+        assert L.sla_forward_blocks(16, 16, 16, 16, 16, ctypes.byref(c), qb0, qb1, 16, None, ws, nbytes,
+                                    None) == sla.SLA_ERR_INVALID_ARG, (qb0, qb1)

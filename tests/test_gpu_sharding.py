@@ -56,3 +56,47 @@ def test_head_shards_reassemble_the_whole_layer(kw, world):
     units = [(0, h, int(i)) for h in range(cfg.H) for i in rng.choice(cfg.nqb, 2, replace=False)]
     err = unit_errors(run, L, units)
     assert err["max_abs"] <= MAX_ABS and err["mean_abs"] <= MEAN_ABS, err
+
+
+BLOCK_CASES = CASES + [
+    dict(name="threeway_odd_blocks", N=1216, N_valid=1200, d=128, H=3, H_kv=3, k_h=3, k_l=4, has_gate=1),
+    dict(name="nsa_branches", N=2048, N_valid=2000, d=64, H=4, H_kv=2, mode=wl.MODE_TOPN_WINDOW, causal=1,
+         top_n=3, window=128, k_h=0, k_l=0, has_proj=0, nsa_branches=1, cmp_block=32, cmp_stride=16, has_gate=1),
+]
+
+
+@pytest.mark.parametrize("kw", BLOCK_CASES, ids=[c["name"] for c in BLOCK_CASES])
+@pytest.mark.parametrize("world", [3, 5])
+def test_block_split_reassembles_the_whole_layer(kw, world):
+    """db-SP's block level: each rank runs its pieces (KV group, range of query-block
+    pairs) through sla_forward_blocks into one output buffer; together they write every
+    row exactly as the whole-layer sla_forward does, bit for bit."""
+    cfg = wl.small_config(**kw)
+    run = DeviceRun(cfg, route=True)
+    crit = run.crit.cpu().numpy() if (cfg.k_h if cfg.mode == wl.MODE_THREEWAY else cfg.top_n) else None
+    costs = sh.pair_costs(cfg, crit)
+    full = torch.full_like(run.out, float("nan"))
+    wss = {}
+
+    def ws_for(lc):
+        if lc.name not in wss:
+            wss[lc.name] = torch.empty(sla.sla_workspace_bytes(lc), dtype=torch.uint8, device="cuda")
+        return wss[lc.name]
+
+    split_groups = 0
+    for r in range(world):
+        shard = sh.BlockShard(cfg, world, r, costs)
+        split_groups += sum(1 for u, p0, p1 in shard.pieces if p0 > 0 or p1 < costs.shape[1])
+        shard.run(sla, run.q, run.k, run.v, run.w_p, run.w_g, full, ws_for)
+        for ws in wss.values():
+            assert sla.sla_check_device_status(ws) == (0, 0)
+    assert split_groups > 0, "the plan split no group: the test would not exercise the block level"
+    assert torch.equal(full, run.out)
+
+
+def test_block_range_rejects_bad_ranges():
+    cfg = wl.small_config(N=1024, N_valid=1000, d=64, H=2, H_kv=2, k_h=2, k_l=2)
+    run = DeviceRun(cfg, route=False)
+    for qb0, qb1 in ((1, 4), (0, 0), (4, 2), (0, 17), (2, 5), (-2, 4)):
+        with pytest.raises(RuntimeError):
+            sla.sla_forward_blocks(run.q, run.k, run.v, run.w_p, run.w_g, cfg, qb0, qb1, run.out, None, run.ws)

@@ -223,3 +223,61 @@ def test_distributed_costs_route_a_share_and_agree_two_gloo_ranks():
     want = sh.unit_costs(cfg, _fake_routing(cfg)).tolist()
     assert res[0][0] == res[1][0] == want
     assert res[0][1] == [0, 2, 4] and res[1][1] == [1, 3]
+
+
+def test_block_plan_covers_every_pair_once_and_balances():
+    """db-SP's block level: the (KV group, pair) units cut into contiguous runs. Every unit
+    lands on exactly one rank, a rank's pieces are contiguous in group-major order, at most
+    two of them are partial groups, and each rank's load stays within one group's fixed
+    work plus one pair of the equal share; the plan is the same on every call."""
+    from block_sparse_linear_sm_b200 import sharding as sh
+    rng = np.random.default_rng(5)
+    for world in (1, 2, 3, 7, 12, 20):
+        costs = rng.uniform(0.5, 4.0, (6, 40))
+        costs[2] *= 4  # one heavy group
+        fixed = np.full(6, 30.0)
+        plan = sh.block_plan(costs, fixed, world)
+        assert plan == sh.block_plan(costs, fixed, world)
+        cover = np.zeros(costs.shape, dtype=int)
+        flat = []
+        for pieces in plan:
+            partial = sum(1 for u, p0, p1 in pieces if p0 > 0 or p1 < costs.shape[1])
+            assert partial <= 2
+            for u, p0, p1 in pieces:
+                assert 0 <= p0 < p1 <= costs.shape[1]
+                cover[u, p0:p1] += 1
+                flat.append((u, p0, p1))
+        assert np.all(cover == 1)
+        # contiguous in group-major order across ranks
+        order = [(u, p) for u, p0, p1 in flat for p in range(p0, p1)]
+        assert order == [(u, p) for u in range(costs.shape[0]) for p in range(costs.shape[1])]
+        loads = sh.block_plan_loads(costs, fixed, plan)
+        share = (costs.sum() + fixed.sum() + (world - 1) * fixed.mean()) / world
+        assert max(loads[:-1] or [0]) <= share + fixed.max() + costs.max() + 1e-9
+        if world > 1:
+            head = sh.plan_loads(costs.sum(1) + fixed, sh.balance(costs.sum(1) + fixed, world))
+            assert max(loads) <= max(head) + fixed.max() + costs.max() + 1e-9
+
+
+def test_pair_costs_sum_to_the_unit_costs():
+    """The per-pair work of the block level adds up to the per-group work of the head
+    level (the same merged-list tiles, the linear branch spread over the query blocks)."""
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+    from oracle import sla_oracle as oracle
+    for kw in (dict(N=1216, N_valid=1200, d=64, H=4, H_kv=2, k_h=3, k_l=4, has_gate=1),
+               dict(N=1024, N_valid=1024, d=64, H=4, H_kv=2, mode=wl.MODE_TOPN_WINDOW, causal=1, top_n=3,
+                    window=128, k_h=0, k_l=0, has_proj=0)):
+        c = wl.small_config(**kw)
+        x = wl.generate(c)
+        L = oracle.Layer(c, x.f64("q"), x.f64("k"), x.f64("v"), x.f64("w_p"), None)
+        if c.mode == wl.MODE_THREEWAY:
+            crit = np.stack([[[np.nonzero(row == 2)[0] for row in L.classes(0, h)] for h in range(c.H)]])
+        else:
+            crit = np.full((1, c.H_kv, c.nqb, c.top_n), -1)
+            for hk in range(c.H_kv):
+                for i, s in enumerate(L.selection(0, hk)[0]):
+                    crit[0, hk, i, :len(s)] = s
+        pc = sh.pair_costs(c, crit)
+        assert pc.shape == (c.H_kv, (c.nqb + 1) // 2)
+        np.testing.assert_allclose(pc.sum(axis=1), sh.unit_costs(c, crit), rtol=1e-12)
