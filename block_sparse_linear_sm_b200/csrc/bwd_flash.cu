@@ -78,8 +78,12 @@ cudaError_t launch_cols(const Plan& p, const BwdPlan& bp, const BwdArgs& a, cuda
 constexpr int kModeThree = 0, kModeTopn = 1, kModeNsa = 2, kModeNsaTok = 2, kModeNsaCmp = 3;
 enum NsaBranch { kBrCmp = 0, kBrSel = 1, kBrWin = 2 };
 
-constexpr int kBwThreads = 320;  // warps 0-7 rows (two column halves), warp 8 MMA, warp 9 TMA producer
+// warps 0-7: rows (two column halves); warp 8: TMEM owner and issuer of the S / dP
+// (S^T / dP^T) products; warp 9: TMA producer; warp 10: issuer of the dQ (dV, dK) products.
+// Two issuer warps, so that one warp's barrier waits (about 160 cycles each, measured) do
+// not leave the tensor pipe without queued work.
 constexpr int kMmaWarp = 8, kProdWarp = 9, kRowWarps = 8;
+constexpr int kDqThreads = 352, kDqWarp = 10;
 
 // merged list of two bitmaps (warp 0, ascending). Entry = index (bits 0-12) | a0 << 13 | a1 << 14
 // | s0 << 15 | s1 << 16 | tag << 17: a0 / a1 = the index is in bitmap a0 / a1 ("active" for
@@ -157,7 +161,7 @@ struct DqParams {
 // (tmKc / tmVc; key c kept when c < n_cmp and c * kstride + kspan <= t), selected blocks
 // (s <= t) and window blocks (t - window < s <= t). All of them add to one dQ accumulator.
 template <int D, int MODE, int SL>
-__global__ void __launch_bounds__(kBwThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     flash_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                 DS_FULL = S_READ + 2, DS_FREE = DS_FULL + 2, ACC_DONE = DS_FREE + 2, Q_TMEM = ACC_DONE + 1;
 
   // four bitmaps: active blocks of half 0 / 1, selected blocks of half 0 / 1 (top-n)
-  for (int w = tid; w < 4 * prm.words; w += kBwThreads) words[w] = 0u;
+  for (int w = tid; w < 4 * prm.words; w += kDqThreads) words[w] = 0u;
   if (tid == 0) {
     misc[2] = 0;
     tc::mbar_init(bar(QO_FULL), 1);
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const int32_t* lst = prm.crit + ((size_t)(TOPN ? bkv : bh) * prm.nb + i_h[hf]) * prm.len;
     uint32_t* act = words + hf * prm.words;
     uint32_t* sel = words + (2 + hf) * prm.words;
-    for (int e = tid; e < prm.len; e += kBwThreads) {
+    for (int e = tid; e < prm.len; e += kDqThreads) {
       const int j = lst[e];
       if (TOPN && j < 0) continue;  // padding of short selections
       if (j < 0 || j >= prm.nb || (TOPN && j >= i_h[hf])) {
@@ -228,7 +232,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     if (TOPN && prm.window > 0) {  // the blocks the causal window reaches
       const int lo = i_h[hf] * kBlock - prm.window + 1;
       const int first = lo <= 0 ? 0 : lo / kBlock;
-      for (int j = first + tid; j <= i_h[hf]; j += kBwThreads) atomicOr(&act[j >> 5], 1u << (j & 31));
+      for (int j = first + tid; j <= i_h[hf]; j += kDqThreads) atomicOr(&act[j >> 5], 1u << (j & 31));
     }
   }
   __syncthreads();
@@ -301,14 +305,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    // ======================= MMA issuer =======================================
+    // ======================= S / dP issuer ====================================
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
-    constexpr uint32_t kIdQ = tc::idesc_bf16(128, D, false, true);
     // base descriptors; a byte offset off is added as off >> 4 (start-address field)
     const uint64_t dOd = tc::sw128_desc(sO, 16, 1024);
     const uint64_t dRk = tc::sw128_desc(sR, 16, 1024);    // ring tiles, K-major
-    const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
     // S_m = Q K_m^T (A = Q in TMEM: only K is read from shared memory, full rate at N = 64)
     // and dP_m = dO V_m^T into TMEM buffer m & 1
     auto issue_sp = [&](int m) {
@@ -322,33 +324,36 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
       tc::mma_commit(bar(SP_FULL + (m & 1)));
     };
-    auto wait_loaded = [&](int m) -> bool {
-      return __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
-    };
     bool ok = T == 0 || (__all_sync(kAll, tc::mbar_wait(bar(QO_FULL), 0, abort)) &&
                          __all_sync(kAll, tc::mbar_wait(bar(Q_TMEM), 0, abort)));
-    for (int m = 0; m < 2 && m < T && ok; ++m) {
-      ok = wait_loaded(m);
+    for (int m = 0; m < T && ok; ++m) {
+      // S / dP buffer m & 1 is free as soon as the row warps have loaded S_{m-2}, dP_{m-2}:
+      // the products of tile m run while they compute dS_{m-2}
+      if (m >= 2) ok = __all_sync(kAll, tc::mbar_wait(bar(S_READ + (m & 1)), ((m - 2) >> 1) & 1, abort));
+      ok = ok && __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
       tc::fence_after_sync();
       if (ok && tc::elect_one()) issue_sp(m);
       __syncwarp();
     }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
+  } else if (warp == kDqWarp) {
+    // ======================= dQ issuer =========================================
+    constexpr uint32_t kAll = 0xffffffffu;
+    constexpr uint32_t kIdQ = tc::idesc_bf16(128, D, false, true);
+    const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
+    bool ok = true;
     for (int m = 0; m < T && ok; ++m) {
       const int b = m & 1;
-      // S / dP buffer b is free as soon as the row warps have loaded S_m, dP_m:
-      // the products of tile m + 2 run while they compute dS_m
-      ok = __all_sync(kAll, tc::mbar_wait(bar(S_READ + b), (m >> 1) & 1, abort));
-      if (ok && m + 2 < T) {
-        ok = wait_loaded(m + 2);
-        tc::fence_after_sync();
-        if (ok && tc::elect_one()) issue_sp(m + 2);
-        __syncwarp();
-      }
-      ok = ok && __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + b), (m >> 1) & 1, abort));
+      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + b), (m >> 1) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
       if (tc::elect_one()) {
-        // dQ += dS_m K_m: A = dS_m from its TMEM buffer (bf16 pairs), B = K_m N-major
+        // dQ += dS_m K_m: A = dS_m from its TMEM buffer (bf16 pairs), B = K_m N-major. The
+        // slot is released after this product: S_m, dP_m (its other readers) completed
+        // before the row warps could write dS_m
         const uint32_t so = (uint32_t)((m % S) * L::kSlot);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -597,7 +602,7 @@ struct DkvParams {
 // NSA compressed keys (kModeNsaCmp): tmK / tmV map the compressed keys; key c is kept
 // for query t when c < n_cmp and c * kstride + kspan <= t; raw fp32 partials out.
 template <int D, int MODE, int SL>
-__global__ void __launch_bounds__(kBwThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     flash_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       DkvParams prm) {
@@ -767,14 +772,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    // ======================= MMA issuer =======================================
+    // ======================= S^T / dP^T issuer ================================
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
-    constexpr uint32_t kIdA = tc::idesc_bf16(128, D, false, true);
     // base descriptors; a byte offset off is added as off >> 4 (start-address field)
     const uint64_t dKd = tc::sw128_desc(sK, 16, 1024), dVd = tc::sw128_desc(sV, 16, 1024);
     const uint64_t dRk = tc::sw128_desc(sR, 16, 1024);    // ring tiles, K-major
-    const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
     // S^T = K Q_i^T, dP^T = V dO_i^T (M = 128 keys, N = 64 queries) into the S buffer
     auto issue_sp = [&](int m) {
       const uint32_t so = (uint32_t)((m % S) * L::kSlot);
@@ -787,33 +790,35 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
       tc::mma_commit(bar(SP_FULL));
     };
-    auto wait_loaded = [&](int m) -> bool {
-      return __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
-    };
     bool ok = T == 0 || __all_sync(kAll, tc::mbar_wait(bar(KV_FULL), 0, abort));
-    if (T > 0 && ok) {
-      ok = wait_loaded(0);
+    for (int m = 0; m < T && ok; ++m) {
+      // the S buffer is free once the row warps have loaded S^T_{m-1}, dP^T_{m-1}: the
+      // products of tile m run while they compute P^T_{m-1} and dS^T_{m-1}
+      if (m >= 1) ok = __all_sync(kAll, tc::mbar_wait(bar(S_READ), (m - 1) & 1, abort));
+      ok = ok && __all_sync(kAll, tc::mbar_wait(bar(LOADED + m % S), (m / S) & 1, abort));
       tc::fence_after_sync();
-      if (ok && tc::elect_one()) issue_sp(0);
+      if (ok && tc::elect_one()) issue_sp(m);
       __syncwarp();
     }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
+    }
+  } else if (warp == kDqWarp) {
+    // ======================= dV / dK issuer ===================================
+    constexpr uint32_t kAll = 0xffffffffu;
+    constexpr uint32_t kIdA = tc::idesc_bf16(128, D, false, true);
+    const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
+    bool ok = true;
     for (int m = 0; m < T && ok; ++m) {
       const int x = m & 1;
-      // the S buffer is free once the row warps have loaded S^T_m, dP^T_m: the products of
-      // tile m + 1 run while they compute P^T_m and dS^T_m
-      ok = __all_sync(kAll, tc::mbar_wait(bar(S_READ), m & 1, abort));
-      if (ok && m + 1 < T) {
-        ok = wait_loaded(m + 1);
-        tc::fence_after_sync();
-        if (ok && tc::elect_one()) issue_sp(m + 1);
-        __syncwarp();
-      }
-      ok = ok && __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
+      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
       if (tc::elect_one()) {
         // dV += P^T dO_i, dK += dS^T Q_i: A = P^T / dS^T from their TMEM buffer (bf16 pairs),
-        // B = dO_i / Q_i N-major
+        // B = dO_i / Q_i N-major. The slot is released after these products: S^T_m, dP^T_m
+        // (its other readers) completed before the row warps could write P^T_m, dS^T_m
         const uint32_t so = (uint32_t)((m % S) * L::kSlot);
         const uint32_t tP = tmem + 2 * D + 128 + 64 * x;
 #pragma unroll
@@ -1101,7 +1106,7 @@ static cudaError_t launch_dq_slots(const Plan& p, const BwdPlan& bp, const BwdAr
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: it holds all 512 TMEM columns
   cudaError_t e = cudaFuncSetAttribute(flash_dq_kernel<D, MODE, SL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dq_kernel<D, MODE, SL><<<c.B * c.H * prm.npairs, kBwThreads, smem, s>>>(mq, mo, mk, mv, mkc, mvc, prm);
+  flash_dq_kernel<D, MODE, SL><<<c.B * c.H * prm.npairs, kDqThreads, smem, s>>>(mq, mo, mk, mv, mkc, mvc, prm);
   return cudaGetLastError();
 }
 
@@ -1208,7 +1213,7 @@ static cudaError_t launch_dkdv_slots(const Plan& p, const BwdPlan& bp, const Bwd
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (512 TMEM columns)
   cudaError_t e = cudaFuncSetAttribute(flash_dkdv_kernel<D, MODE, SL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  flash_dkdv_kernel<D, MODE, SL><<<grid, kBwThreads, smem, s>>>(mq, mo, mk, mv, prm);
+  flash_dkdv_kernel<D, MODE, SL><<<grid, kDqThreads, smem, s>>>(mq, mo, mk, mv, prm);
   return cudaGetLastError();
 }
 
