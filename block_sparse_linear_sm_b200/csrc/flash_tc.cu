@@ -126,8 +126,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   constexpr int Q_FULL = 0, K_FULL = 1, K_EMPTY = K_FULL + kKSlots, V_FULL = K_EMPTY + kKSlots,
                 V_EMPTY = V_FULL + kVSlots, S_FULL = V_EMPTY + kVSlots, P_FULL = S_FULL + 2,
                 O_DONE = P_FULL + 2, SP_FULL = O_DONE + 1, SP1_FULL = SP_FULL + 1, NUM_DONE = SP1_FULL + 1,
-                NUM_READ = NUM_DONE + 2;
-  static_assert(NUM_READ < 32, "barrier area holds 32 mbarriers");
+                NUM_READ = NUM_DONE + 4, O_LAST = NUM_READ + 1;
+  // O_DONE completes once per P V product; O_LAST once, after the last one
+  static_assert(O_LAST < 32, "barrier area holds 32 mbarriers");
 
   // ---- unit decode ----------------------------------------------------------
   const int Hkv = prm.H / prm.group;
@@ -183,11 +184,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       tc::mbar_init(bar(P_FULL + b), 4);
     }
     tc::mbar_init(bar(O_DONE), 1);
+    tc::mbar_init(bar(O_LAST), 1);
     tc::mbar_init(bar(SP_FULL), 1);
     tc::mbar_init(bar(SP1_FULL), 1);
-    tc::mbar_init(bar(NUM_DONE), 1);
-    tc::mbar_init(bar(NUM_DONE + 1), 1);
-    tc::mbar_init(bar(NUM_READ), 2);
+    for (int x = 0; x < 4; ++x) tc::mbar_init(bar(NUM_DONE + x), 1);  // (column pass, half)
+    tc::mbar_init(bar(NUM_READ), 4);
     tc::fence_mbar_init();
     // Q does not depend on the block lists: its load overlaps the list merge
     tc::prefetch_tensormap(&tmQ);
@@ -455,6 +456,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                             (n > 0 || kk > 0) ? 1u : 0u);
           tc::mma_commit(bar(O_DONE));
           tc::mma_commit(bar(V_EMPTY + slot));
+          if (n == T - 1) tc::mma_commit(bar(O_LAST));
           // buffer b is free once PV_n has read P_n: S_{n+2} goes in behind it
           // (tcgen05 operations of one thread execute in issue order)
           if (n + 2 < T) issue_s(n + 2);
@@ -462,27 +464,30 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         __syncwarp();
       }
       if (FUSE && ok) {
-        // num = phi(Q) S'_i (M = 128 rows, N = D, K = D) into the S columns, one query
-        // block at a time: the second waits until the first block's rows are read
-        constexpr uint32_t kIdN = tc::idesc_bf16(128, D, false, true);
+        // num = phi(Q) S'_i into the 128 free S columns, 64 output columns per pass: half
+        // hf's product (M = 128 rows, N = 64, K = D, B = S'_{i_hf}) goes to columns
+        // 64 hf .. 64 hf + 63, so both halves' rows are ready together; the next pass
+        // waits until all four softmax warps have read this one
+        constexpr uint32_t kIdN = tc::idesc_bf16(128, 64, false, true);
         const uint64_t dS = tc::sw128_desc(sKV, D * 128, 1024);
         ok = __all_sync(kAll, tc::mbar_wait(bar(SP_FULL), 0, abort));
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          if (!valid_h[hf]) break;
-          if (hf == 1 && !(__all_sync(kAll, tc::mbar_wait(bar(NUM_READ), 0, abort)) &&
-                           __all_sync(kAll, tc::mbar_wait(bar(SP1_FULL), 0, abort)))) {
-            ok = false;
-            break;
-          }
-          tc::fence_after_sync();
-          if (tc::elect_one()) {
+        for (int pass = 0; pass < D / 64 && ok; ++pass) {
+          if (pass > 0) ok = __all_sync(kAll, tc::mbar_wait(bar(NUM_READ), (pass - 1) & 1, abort));
+          for (int hf = 0; hf < 2 && ok; ++hf) {
+            if (!valid_h[hf]) continue;
+            if (pass == 0 && hf == 1) ok = __all_sync(kAll, tc::mbar_wait(bar(SP1_FULL), 0, abort));
+            if (!ok) break;
+            tc::fence_after_sync();
+            if (tc::elect_one()) {
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k)
-              tc::mma_bf16_ss(tS0, dQ + (uint32_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4),
-                              dS + (uint32_t)((hf * kKSlots * L::kSlotBytes + k * 2048) >> 4), kIdN, k > 0);
-            tc::mma_commit(bar(NUM_DONE + hf));
+              for (int k = 0; k < D / 16; ++k)
+                tc::mma_bf16_ss(tS0 + 64 * hf, dQ + (uint32_t)(((k >> 2) * 16384 + (k & 3) * 32) >> 4),
+                                dS + (uint32_t)((hf * kKSlots * L::kSlotBytes + pass * D * 128 + k * 2048) >> 4),
+                                kIdN, k > 0);
+              tc::mma_commit(bar(NUM_DONE + 2 * pass + hf));
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
       }
       if (!ok && lane == 0) {
@@ -586,15 +591,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = 0u;  // this half does not use the tile
       }
-      // O rescale needs PV_{n-1} complete (it accumulates into O)
-      if (n > 0) {
+      // Only an O rescale waits for PV_{n-1} (it accumulates into O). P_n's buffer is free
+      // without a wait: S_n went into it after PV_{n-2} had read P_{n-2} (one thread issues
+      // both, in order). When this wait runs, the products PV_0 .. PV_{n-2} have completed
+      // and PV_n has not been issued, so O_DONE has completed n - 1 or n phases and the
+      // parity of phase n - 1 tells the two apart.
+      const bool any_resc = __any_sync(0xffffffffu, resc);
+      if (n > 0 && any_resc) {
         if (!__all_sync(0xffffffffu, tc::mbar_wait(bar(O_DONE), (n - 1) & 1, abort))) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
       }
-      if (__any_sync(0xffffffffu, resc)) {
+      if (any_resc) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
@@ -613,7 +623,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       if (lane == 0) tc::mbar_arrive(bar(P_FULL + b));
     }
     if (ok && T > 0) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(O_DONE), (T - 1) & 1, abort));
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(O_LAST), 0, abort));
       tc::fence_after_sync();
     }
     if (!ok) {
@@ -626,11 +636,12 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           (ok && T > 0 && l_sum > 0.f && t < prm.n_valid) ? m_ref + log2f(l_sum) : INFINITY;
     if (FUSE) {
       // ---- fused epilogue of the layer (three-way mode with a linear branch) ----
-      // den = phi(q) . Z_i from the tiles the producer loaded
+      // den = phi(q) . Z_i from the tiles the producer loaded (four partial sums)
       ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(SP_FULL), 0, abort));
       float den = 0.f;
       if (ok && valid_h[hf]) {
         const float4* z4 = reinterpret_cast<const float4*>(smem + L::kOffKV + D * D * 2 + hf * D * 4);
+        float dp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
           const uint4* frow = reinterpret_cast<const uint4*>(smem + L::kOffQ + p * 16384 + r * 128);
@@ -640,43 +651,51 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             const float4 za = z4[16 * p + 2 * c], zb = z4[16 * p + 2 * c + 1];
             const float2 f0 = unpack_bf16(u.x), f1 = unpack_bf16(u.y), f2 = unpack_bf16(u.z),
                          f3 = unpack_bf16(u.w);
-            den = fmaf(f0.x, za.x, fmaf(f0.y, za.y, fmaf(f1.x, za.z, fmaf(f1.y, za.w, den))));
-            den = fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, fmaf(f3.x, zb.z, fmaf(f3.y, zb.w, den))));
+            dp[0] = fmaf(f0.x, za.x, fmaf(f0.y, za.y, dp[0]));
+            dp[1] = fmaf(f1.x, za.z, fmaf(f1.y, za.w, dp[1]));
+            dp[2] = fmaf(f2.x, zb.x, fmaf(f2.y, zb.y, dp[2]));
+            dp[3] = fmaf(f3.x, zb.z, fmaf(f3.y, zb.w, dp[3]));
           }
         }
+        den = (dp[0] + dp[1]) + (dp[2] + dp[3]);
       }
       const float g = (prm.gate && valid_h[hf] && t < prm.n_valid) ? prm.gate[(size_t)bh_h[hf] * prm.N + t] : 1.f;
       const float cl = den > 0.f ? g / den : 0.f;
-      if (valid_h[hf]) {
-        ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(NUM_DONE + hf), 0, abort));
-        tc::fence_after_sync();
-        const bool live = ok && t < prm.n_valid;
-        const float inv = (live && T > 0 && l_sum > 0.f) ? 1.f / l_sum : 0.f;
-        __nv_bfloat16* og = prm.o + ((size_t)bh_h[hf] * prm.N + t) * D;
+      const bool live = ok && valid_h[hf] && t < prm.n_valid;
+      const float inv = (live && T > 0 && l_sum > 0.f) ? 1.f / l_sum : 0.f;
+      __nv_bfloat16* og = prm.o + ((size_t)bh_h[hf] * prm.N + t) * D;
+      // O = O_s / l + (g / den) num, 64 columns per pass of the num product
 #pragma unroll 1
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t ov[16], nv[16];
-          if (ok) {
-            if (T > 0) tc::tmem_ld16(tO + 16 * c, ov);
-            tc::tmem_ld16(tS0 + 16 * c, nv);
-            tc::tmem_ld_wait();
-          }
-          if (!ok || T == 0) {
+      for (int pass = 0; pass < D / 64; ++pass) {
+        if (valid_h[hf]) {
+          ok = ok && __all_sync(0xffffffffu, tc::mbar_wait(bar(NUM_DONE + 2 * pass + hf), 0, abort));
+          tc::fence_after_sync();
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t ov[32], nv[32];
+            if (ok) {
+              if (T > 0) tc::tmem_ld32(tO + 64 * pass + 32 * c, ov);
+              tc::tmem_ld32(tS0 + 64 * hf + 32 * c, nv);
+              tc::tmem_ld_wait();
+            }
+            if (!ok || T == 0) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) ov[j] = 0u;
-          }
-          uint32_t pw[8];
+              for (int j = 0; j < 32; ++j) ov[j] = 0u;
+            }
+            uint32_t pw[16];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            pw[j] = live ? pack_bf16(__uint_as_float(ov[2 * j]) * inv + cl * __uint_as_float(nv[2 * j]),
-                                     __uint_as_float(ov[2 * j + 1]) * inv + cl * __uint_as_float(nv[2 * j + 1]))
-                         : 0u;
-          uint4* dst = reinterpret_cast<uint4*>(og + 16 * c);
-          dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-          dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+            for (int j = 0; j < 16; ++j)
+              pw[j] = live ? pack_bf16(__uint_as_float(ov[2 * j]) * inv + cl * __uint_as_float(nv[2 * j]),
+                                       __uint_as_float(ov[2 * j + 1]) * inv + cl * __uint_as_float(nv[2 * j + 1]))
+                           : 0u;
+            uint4* dst = reinterpret_cast<uint4*>(og + 64 * pass + 32 * c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pw[4 * j], pw[4 * j + 1], pw[4 * j + 2], pw[4 * j + 3]);
+          }
         }
-        if (hf == 0) {
-          // this block's rows of the num columns are read: the next block may overwrite them
+        if (pass + 1 < D / 64) {
+          // this pass's num columns are read (every softmax warp arrives, with or without
+          // a valid half): the next pass may overwrite them
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(bar(NUM_READ));
