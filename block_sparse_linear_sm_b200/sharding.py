@@ -227,6 +227,31 @@ def pair_costs(cfg: wl.LayerConfig, crit: Optional[np.ndarray] = None) -> np.nda
     return cost
 
 
+def distributed_pair_costs(cfg: wl.LayerConfig, world: int, rank: int, route_local, dist) -> np.ndarray:
+    """pair_costs of the whole layer on every rank, each rank routing only its probe
+    groups (as distributed_costs does for the head level): one all_gather of a padded
+    float64 [ceil(H_kv / world), npairs] block per rank."""
+    import torch
+
+    npairs = (cfg.nqb + 1) // 2
+    mine = probe_units(cfg, world, rank)
+    local = pair_costs(local_config(cfg, mine), route_local(mine)) if mine else np.zeros((0, npairs))
+    width = (cfg.H_kv + world - 1) // world
+    buf = torch.zeros((width, npairs), dtype=torch.float64)
+    if len(mine):
+        buf[:len(mine)] = torch.from_numpy(np.asarray(local, dtype=np.float64))
+    backend = dist.get_backend() if hasattr(dist, "get_backend") else "gloo"
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    buf = buf.to(dev)
+    parts = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(parts, buf)
+    costs = np.zeros((cfg.H_kv, npairs))
+    for r, part in enumerate(parts):
+        units = probe_units(cfg, world, r)
+        costs[units] = part.cpu().numpy()[:len(units)]
+    return costs
+
+
 def fixed_costs(cfg: wl.LayerConfig, costs: np.ndarray, share: float = 0.5) -> np.ndarray:
     """Work of a KV group that every call holding any of its query blocks repeats (routing,
     key pooling, linear states), as ``share`` of the group's mean per-head flash work. With

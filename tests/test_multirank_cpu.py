@@ -281,3 +281,60 @@ def test_pair_costs_sum_to_the_unit_costs():
         pc = sh.pair_costs(c, crit)
         assert pc.shape == (c.H_kv, (c.nqb + 1) // 2)
         np.testing.assert_allclose(pc.sum(axis=1), sh.unit_costs(c, crit), rtol=1e-12)
+
+
+def _block_rank_main(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = wl.small_config(N=1024, N_valid=1000, H=10, H_kv=5, k_h=3, k_l=2)
+        full = _fake_routing(cfg)
+        group = cfg.H // cfg.H_kv
+        routed = []
+
+        def route_local(units):
+            routed.extend(units)
+            heads = [u * group + g for u in units for g in range(group)]
+            return full[:, heads]
+        costs = sh.distributed_pair_costs(cfg, world, rank, route_local, dist)
+        shard = sh.BlockShard(cfg, world, rank, costs)
+        q.put((rank, (costs.tolist(), sorted(routed), shard.plan, shard.pieces)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_block_level_costs_and_plan_agree_two_gloo_ranks():
+    """The block level across two gloo ranks: each routes every second KV group, the
+    all_gather gives both the whole layer's per-pair costs (equal to the single-process
+    estimate), both compute the same plan, and each takes its own pieces of it."""
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_block_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=100) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    cfg = wl.small_config(N=1024, N_valid=1000, H=10, H_kv=5, k_h=3, k_l=2)
+    want = sh.pair_costs(cfg, _fake_routing(cfg))
+    for r in (0, 1):
+        np.testing.assert_allclose(np.array(res[r][0]), want, rtol=1e-12)
+    assert res[0][1] == [0, 2, 4] and res[1][1] == [1, 3]
+    assert res[0][2] == res[1][2]
+    assert res[0][3] == res[0][2][0] and res[1][3] == res[1][2][1]
