@@ -150,9 +150,9 @@ sla_status sla_forward_host(const void* q_host, const void* k_host, const void* 
     if (threeway && cfg->has_proj && cfg->proj_per_head) wpu += (size_t)h0 * wp_head;
     const char* wgu = cfg->has_gate ? (const char*)w_g + (size_t)h0 * wg_head : (const char*)w_g;
     if (!ok(cudaStreamWaitEvent(s, ev_in[u], 0))) break;
-    const sla_status fs = sla_forward(base + hp.off_q + oq, base + hp.off_k + okv, base + hp.off_v + okv, wpu, wgu,
-                                      &hp.unit, base + hp.off_out + oq, nullptr,
-                                      base + hp.off_ws + (size_t)u * hp.ws_unit, hp.ws_unit, s);
+    const sla_status fs = forward_single_stream(base + hp.off_q + oq, base + hp.off_k + okv, base + hp.off_v + okv,
+                                                wpu, wgu, &hp.unit, base + hp.off_out + oq, nullptr,
+                                                base + hp.off_ws + (size_t)u * hp.ws_unit, hp.ws_unit, s);
     if (fs != SLA_OK) {
       result = fs;
       break;

@@ -24,6 +24,8 @@ unsigned long long g_scratch_ctx[kMaxDevices] = {};  // id of the context the ad
 typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
+}  // namespace
+
 // Process-unique id of the current CUDA context (0 if it cannot be read). A device
 // reset ends the primary context; the next one has another id, and the array then
 // has another device address.
@@ -48,6 +50,8 @@ unsigned long long current_context_id() {
   if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
   return 0;
 }
+
+namespace {
 
 // Device address of g_route_scratch on the current device. The host-side name
 // of the array is only a stand-in, so the address is looked up (with that device

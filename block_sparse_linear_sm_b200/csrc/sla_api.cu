@@ -1,5 +1,6 @@
 // C ABI of the sparse+linear attention layer: validation, workspace plan and
 // the launch sequence. See include/sla.h for the contract of each entry point.
+#include <mutex>
 #include <math.h>
 #include <string.h>
 
@@ -182,10 +183,32 @@ cudaError_t route_stages(const Plan& p, const Args& a, cudaStream_t s) {
   return e;
 }
 
+// The library's side stream of the current device and context (created on first use,
+// non-blocking, kept until the process exits), or null when the context cannot be told
+// apart. The linear-state stage runs on it beside the routing.
+static cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  static unsigned long long ctxs[64] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (streams[dev] == nullptr || ctxs[dev] != ctx) {
+    cudaStream_t st = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    streams[dev] = st;
+    ctxs[dev] = ctx;
+  }
+  return streams[dev];
+}
+
 static sla_status forward_impl(const void* q, const void* k, const void* v, const void* w_p,
                                const void* w_g, const sla_config* cfg, void* out, int8_t* mask_out,
                                void* ws, size_t ws_bytes, void* stream, void* const* events,
-                               int32_t n_events, int32_t qb_begin = 0, int32_t qb_end = -1) {
+                               int32_t n_events, int32_t qb_begin = 0, int32_t qb_end = -1,
+                               bool may_fork = true) {
   Plan p;
   sla_status st = check_config(cfg);
   if (st != SLA_OK) return st;
@@ -222,12 +245,55 @@ static sla_status forward_impl(const void* q, const void* k, const void* v, cons
   a.neg = nullptr;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(a.status, 0, 8, s) != cudaSuccess) return SLA_ERR_CUDA;
-  if (events && cudaEventRecord((cudaEvent_t)events[0], s) != cudaSuccess) return SLA_ERR_CUDA;
-  for (int i = 0; i < ns; ++i) {
-    if (run_stage(stages[i], p, a, s) != cudaSuccess) return SLA_ERR_CUDA;
-    if (events && cudaEventRecord((cudaEvent_t)events[i + 1], s) != cudaSuccess) return SLA_ERR_CUDA;
+  // The linear states need only K and V (and, with smooth-K, the pooled keys): after the
+  // pooling pass they run on the side stream while the pooled scores and the
+  // classification run on `stream`, which waits for them before the aggregation. A call
+  // that times its stages runs them in order on `stream`.
+  cudaStream_t side = (may_fork && !events) ? side_stream() : nullptr;
+  bool has_state = false;
+  for (int i = 0; i < ns; ++i) has_state = has_state || stages[i] == kState;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  if (side && has_state) {
+    if (cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess) return SLA_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventDestroy(ev_fork);
+      return SLA_ERR_CUDA;
+    }
+  } else {
+    side = nullptr;
   }
-  return SLA_OK;
+  sla_status result = SLA_OK;
+  if (events && cudaEventRecord((cudaEvent_t)events[0], s) != cudaSuccess) result = SLA_ERR_CUDA;
+  for (int i = 0; i < ns && result == SLA_OK; ++i) {
+    if (side && stages[i] == kState) continue;  // already enqueued on the side stream
+    if (side && stages[i] == kAggregate && cudaStreamWaitEvent(s, ev_join, 0) != cudaSuccess) {
+      result = SLA_ERR_CUDA;
+      break;
+    }
+    if (run_stage(stages[i], p, a, s) != cudaSuccess) {
+      result = SLA_ERR_CUDA;
+      break;
+    }
+    if (side && stages[i] == kPool &&
+        (cudaEventRecord(ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess ||
+         run_stage(kState, p, a, side) != cudaSuccess || cudaEventRecord(ev_join, side) != cudaSuccess)) {
+      result = SLA_ERR_CUDA;
+      break;
+    }
+    if (events && cudaEventRecord((cudaEvent_t)events[i + 1], s) != cudaSuccess) result = SLA_ERR_CUDA;
+  }
+  if (side) {
+    // the events are released once they have completed
+    cudaEventDestroy(ev_fork);
+    cudaEventDestroy(ev_join);
+  }
+  return result;
+}
+
+sla_status forward_single_stream(const void* q, const void* k, const void* v, const void* w_p, const void* w_g,
+                                 const sla_config* cfg, void* out, int8_t* mask_out, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  return forward_impl(q, k, v, w_p, w_g, cfg, out, mask_out, ws, ws_bytes, stream, nullptr, 0, 0, -1, false);
 }
 
 // ---------------------------------------------------------------------------

@@ -46,6 +46,14 @@ struct Plan {
 
 bool make_plan(const sla_config* c, Plan* p);
 
+// process-unique id of the current CUDA context, 0 if it cannot be read (noalloc.cu)
+unsigned long long current_context_id();
+// sla_forward without the internal side stream (callers that run several layers on their
+// own streams at once, where one shared side stream would serialise them)
+sla_status forward_single_stream(const void* q, const void* k, const void* v, const void* w_p, const void* w_g,
+                                 const sla_config* cfg, void* out, int8_t* mask_out, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 // Raw pointers of one launch.
 struct Args {
   const __nv_bfloat16* q;

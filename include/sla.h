@@ -56,7 +56,12 @@
  *   attention and the linear states, and their output rows are written as 0.
  * - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
  *   enqueues work on it and returns; nothing synchronises except
- *   sla_check_device_status.
+ *   sla_check_device_status. sla_forward (and sla_forward_blocks) run the
+ *   linear-state stage on a side stream the library creates once per device and
+ *   context: forked from `stream` after the pooling pass with an event and joined
+ *   back before the aggregation, so the call stays ordered on `stream` as a whole
+ *   (also under CUDA-graph capture). The timed and host-buffer entry points run
+ *   every stage on their own stream.
  * - `ws` is caller-owned device scratch of at least sla_workspace_bytes(cfg)
  *   bytes, 256-byte aligned. Its contents need no initialisation and are
  *   clobbered. Calls that share one `ws` must not overlap on the GPU.
