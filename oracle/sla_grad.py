@@ -239,6 +239,9 @@ def block_grads(cfg, q, k, v, w_p, w_g, d_out, classes, b: int, q_blocks, k_bloc
     Padding rows (index >= N_valid) contribute nothing and get zero rows.
     """
     c = so.OracleCfg.of(cfg)
+    if c.mode != 0 and c.nsa_branches:
+        return _block_grads_nsa(c, q, k, v, w_g if c.has_gate else None, d_out, classes, b, q_blocks, k_blocks,
+                                heads)
     if c.mode != 0:
         return _block_grads_topn(c, q, k, v, d_out, classes, b, q_blocks, k_blocks, heads)
     nb, bl, nv, d, s = c.nb, c.block, c.N_valid, c.d, c.sm_scale
@@ -454,4 +457,143 @@ def _block_grads_topn(c, q, k, v, d_out, sels, b, q_blocks, k_blocks, heads=None
                 r = rows_of(i)
                 dv[:nk] += P[:, selc].T @ dO[r]
                 dk[:nk] += s * dSm[:, selc].T @ Q[r]
+    return out
+
+
+def _softmax_rows(x: np.ndarray, allow: np.ndarray) -> np.ndarray:
+    """Row softmax of x over the allowed entries (rows with none give 0)."""
+    x = np.where(allow, x, -np.inf)
+    m = x.max(axis=1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.where(allow, np.exp(x - m), 0.0)
+    den = e.sum(axis=1, keepdims=True)
+    return np.where(den > 0, e / np.where(den > 0, den, 1.0), 0.0)
+
+
+def _block_grads_nsa(c, q, k, v, w_g, d_out, sels, b, q_blocks, k_blocks, heads=None):
+    """NSA's three branches (top-n mode with nsa_branches) block by block. Per query head h
+    and valid row t: o_b = softmax attention of branch b (compressed keys and values A K,
+    A V with t attending block c when c * stride + length - 1 <= t; the selected blocks of
+    t's block; the window t - window < s <= t), O = sum_b g_b o_b, g_b = sigmoid(q_t .
+    w_g[h][b]) (1 without gates). With dO_b = g_b dO: D_b = dO_b . o_b, dP_b = dO_b V_b^T,
+    dS_b = P_b (dP_b - D_b); dq += s dS_b K_b + sum_b dlogit_b w_g[h][b] with dlogit_b =
+    (dO . o_b) g_b (1 - g_b); dK_b += s dS_b^T q, dV_b += P_b^T dO_b; the compressed keys'
+    and values' gradients go back to each token of their block with weight 1 / length.
+    The compressed branch runs over every valid row of each head (a compressed key's
+    gradient gathers from every later query). dk, dv sum over the KV group's heads in
+    ``heads``; dw_g[h] (all three rows) for every head in ``heads``."""
+    nb, bl, nv, d, s = c.nb, c.block, c.N_valid, c.d, c.sm_scale
+    length, stride = c.cmp_block, c.cmp_stride
+    n_c = (nv - length) // stride + 1 if nv >= length else 0
+    heads = list(range(c.H)) if heads is None else list(heads)
+    q_blocks, k_blocks = list(q_blocks), list(k_blocks)
+    out = dict(dq={}, dk={}, dv={}, dw_g={}, dw_p=None)
+    rows_of = lambda i: slice(i * bl, min((i + 1) * bl, nv))
+    clast = np.arange(n_c) * stride + length - 1  # query t attends block c when clast[c] <= t
+    for hk in sorted({h // c.group for h in heads}):
+        K = np.asarray(k[b, hk], dtype=np.float64)
+        V = np.asarray(v[b, hk], dtype=np.float64)
+        Kc = np.stack([K[j * stride:j * stride + length].mean(axis=0) for j in range(n_c)]) if n_c else np.zeros((0, d))
+        Vc = np.stack([V[j * stride:j * stride + length].mean(axis=0) for j in range(n_c)]) if n_c else np.zeros((0, d))
+        sel_rows = sels[b][hk]
+        dKc, dVc = np.zeros((n_c, d)), np.zeros((n_c, d))
+        dk = {j: np.zeros((bl, d)) for j in k_blocks}
+        dv = {j: np.zeros((bl, d)) for j in k_blocks}
+        for h in [x for x in heads if x // c.group == hk]:
+            Q = np.asarray(q[b, h], dtype=np.float64)
+            dO = np.asarray(d_out[b, h], dtype=np.float64).copy()
+            dO[nv:] = 0.0
+            if w_g is not None:
+                g = so.sigmoid(Q @ np.asarray(w_g[h], dtype=np.float64).T)  # [N, 3]
+            else:
+                g = np.ones((c.N, 3))
+            dlogit = np.zeros((c.N, 3))
+            dq_cmp = {}
+            # ---- compressed branch over every valid row
+            for r0 in range(0, nv, 4096):
+                r1 = min(nv, r0 + 4096)
+                t = np.arange(r0, r1)
+                if n_c == 0:
+                    continue
+                allow = clast[None, :] <= t[:, None]
+                P = _softmax_rows(Q[r0:r1] @ Kc.T * s, allow)
+                oc = P @ Vc
+                dOc = g[r0:r1, 0:1] * dO[r0:r1]
+                dS = P * (dOc @ Vc.T - (dOc * oc).sum(axis=1, keepdims=True))
+                dKc += s * dS.T @ Q[r0:r1]
+                dVc += P.T @ dOc
+                dlogit[r0:r1, 0] = (dO[r0:r1] * oc).sum(axis=1)
+                for i in q_blocks:
+                    r = rows_of(i)
+                    lo, hi = max(r.start, r0), min(r.stop, r1)
+                    if lo < hi:
+                        dq_cmp.setdefault(i, np.zeros((bl, d)))[lo - r.start:hi - r.start] = \
+                            s * dS[lo - r0:hi - r0] @ Kc
+
+            # ---- selected and window branches of query block i
+            def branch(i, kind):
+                r = rows_of(i)
+                t = np.arange(r.start, r.stop)[:, None]
+                if kind == "sel":
+                    blocks = sorted(int(j) for j in sel_rows[i])
+                else:
+                    first = max(0, (i * bl - c.window + 1) // bl) if c.window > 0 else i + 1
+                    blocks = list(range(first, i + 1))
+                toks = np.concatenate([np.arange(j * bl, min((j + 1) * bl, nv)) for j in blocks]) \
+                    if blocks else np.zeros(0, np.int64)
+                if toks.size == 0 or r.start >= r.stop:
+                    return toks, None, None, None
+                sj = toks[None, :]
+                allow = (sj <= t) & ((sj > t - c.window) if kind == "win" else True)
+                P = _softmax_rows(Q[r] @ K[toks].T * s, allow)
+                ob = P @ V[toks]
+                gb = g[r, 1 if kind == "sel" else 2][:, None]
+                dOb = gb * dO[r]
+                dS = P * (dOb @ V[toks].T - (dOb * ob).sum(axis=1, keepdims=True))
+                return toks, P, dS, (ob, dOb)
+
+            for i in range(nb):
+                r = rows_of(i)
+                if r.start >= r.stop:
+                    continue
+                for col, kind in ((1, "sel"), (2, "win")):
+                    toks, P, dS, extra = branch(i, kind)
+                    if P is None:
+                        continue
+                    ob, dOb = extra
+                    dlogit[r, col] = (dO[r] * ob).sum(axis=1)
+                    n = r.stop - r.start
+                    if i in q_blocks:
+                        dq_cmp.setdefault(i, np.zeros((bl, d)))[:n] += s * dS @ K[toks]
+                    for j in k_blocks:
+                        rk = slice(j * bl, min((j + 1) * bl, nv))
+                        nk = rk.stop - rk.start
+                        selc = (toks >= rk.start) & (toks < rk.stop)
+                        if nk <= 0 or not selc.any():
+                            continue
+                        dv[j][:nk] += P[:, selc].T @ dOb
+                        dk[j][:nk] += s * dS[:, selc].T @ Q[r]
+            dlogit = dlogit * g * (1.0 - g) if w_g is not None else np.zeros_like(dlogit)
+            dlogit[nv:] = 0.0
+            for i in q_blocks:
+                r = rows_of(i)
+                rows = dq_cmp.get(i, np.zeros((bl, d))).copy()
+                n = max(0, r.stop - r.start)
+                if w_g is not None and n > 0:
+                    rows[:n] += dlogit[r] @ np.asarray(w_g[h], dtype=np.float64)
+                out["dq"][(h, i)] = rows
+            if w_g is not None:
+                out["dw_g"][h] = dlogit.T @ Q
+        # ---- the compressed keys' and values' gradients back to their tokens
+        for j in k_blocks:
+            for x in range(bl):
+                tok = j * bl + x
+                if tok >= nv:
+                    continue
+                cs = [cc for cc in range(n_c) if cc * stride <= tok <= cc * stride + length - 1]
+                for cc in cs:
+                    dk[j][x] += dKc[cc] / length
+                    dv[j][x] += dVc[cc] / length
+            out["dk"][(hk, j)] = dk[j]
+            out["dv"][(hk, j)] = dv[j]
     return out

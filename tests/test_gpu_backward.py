@@ -301,3 +301,44 @@ def test_full_size_topn_backward_on_sampled_blocks():
         errs[key + "_elem"] = elem_ratio(pr)
     print("nsa_causal", errs)
     assert all(e <= REL for e in errs.values()), errs
+
+
+def test_full_length_nsa_branches_backward_on_sampled_blocks():
+    """NSA's three branches at the preset's full sequence length (N = 65536, d = 128, top 16,
+    window 512, compressed blocks of 32 at stride 16, gates), one KV group of four query heads:
+    dq on four query blocks of every head, dk and dv on three key blocks of the KV head
+    (complete: they sum over the group's heads) and dw_g in full, against the oracle's
+    block-by-block statement of the three branches."""
+    from gpu_util import LazyF64
+
+    c = wl.preset("nsa_branches").replace(name="nsa_branches_group4", H=4, H_kv=1)
+    x = wl.generate(c)
+    run = DeviceRun(c, x, route=False)
+    dob = d_out_bits(c, 23)
+    dout = to_dev(dob)
+    dq, dk, dv = torch.empty_like(run.q), torch.empty_like(run.k), torch.empty_like(run.v)
+    dw_g = torch.full((c.H, 3, c.d), float("nan"), dtype=torch.float32, device="cuda")
+    bws = torch.empty(sla.sla_backward_workspace_bytes(c), dtype=torch.uint8, device="cuda")
+    sla.sla_backward(run.q, run.k, run.v, None, run.w_g, c, run.out, dout, dq, dk, dv, None, dw_g, run.ws, bws)
+    assert sla.sla_check_device_status(bws) == (0, 0)
+    nb, bl = c.nqb, c.block
+    qb, kb = [1, 17, nb // 2, nb - 1], [0, nb // 2 + 1, nb - 1]
+    ref = sla_grad.block_grads(c, LazyF64(x.q), LazyF64(x.k), LazyF64(x.v), None, x.f64("w_g"), LazyF64(dob),
+                               topn_selection(run), 0, qb, kb)
+
+    def rel(pairs):
+        num = sum(float(np.sum((g - r) ** 2)) for g, r in pairs)
+        den = sum(float(np.sum(r ** 2)) for _, r in pairs)
+        return (num / den) ** 0.5
+
+    pairs = {"dq": [(bf16_to_f64(dq[0, h, i * bl:(i + 1) * bl]), r) for (h, i), r in ref["dq"].items()]}
+    for key, t in (("dk", dk), ("dv", dv)):
+        pairs[key] = [(bf16_to_f64(t[0, hk, j * bl:(j + 1) * bl]), r) for (hk, j), r in ref[key].items()]
+    g = dw_g.double().cpu().numpy()
+    pairs["dw_g"] = [(g[h], r) for h, r in ref["dw_g"].items()]
+    errs = {}
+    for key, pr in pairs.items():
+        errs[key] = rel(pr)
+        errs[key + "_elem"] = elem_ratio(pr)
+    print("nsa_branches_group4", errs)
+    assert all(e <= REL for e in errs.values()), errs

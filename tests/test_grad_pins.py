@@ -192,6 +192,10 @@ BLOCK_CASES = {
     "smooth_k_linear_all_gqa": dict(smooth_k=1, linear_all=1, H=4, H_kv=2, N=256, k_h=2, k_l=1),
     "topn_window_gqa": dict(mode=1, causal=1, top_n=2, window=40, k_h=0, k_l=0, has_proj=0, has_gate=0,
                             H=4, H_kv=2, N=256, N_valid=250),
+    "nsa_gates_gqa": dict(mode=1, causal=1, top_n=2, window=40, k_h=0, k_l=0, has_proj=0, has_gate=1,
+                          nsa_branches=1, cmp_block=16, cmp_stride=8, H=4, H_kv=2, N=256, N_valid=256),
+    "nsa_ragged_no_gates": dict(mode=1, causal=1, top_n=1, window=24, k_h=0, k_l=0, has_proj=0, has_gate=0,
+                                nsa_branches=1, cmp_block=32, cmp_stride=16, H=3, H_kv=1, N=320, N_valid=301),
 }
 
 
@@ -215,6 +219,7 @@ def test_block_grads_equal_autograd(name):
                 assert np.abs(rows - want).max() <= 1e-10 * scale(ref[key]), (name, key, hk, j)
         if c.has_proj and c.mode == 0:
             assert np.abs(got["dw_p"] - ref["dw_p"]).max() <= 1e-10 * scale(ref["dw_p"])
-        if c.has_gate and c.mode == 0:
+        if c.has_gate and (c.mode == 0 or c.nsa_branches):
+            assert len(got["dw_g"]) == c.H
             for h, row in got["dw_g"].items():
                 assert np.abs(row - ref["dw_g"][h]).max() <= 1e-10 * scale(ref["dw_g"])
