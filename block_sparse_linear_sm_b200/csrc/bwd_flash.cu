@@ -563,7 +563,11 @@ struct DkvLayout {
   static constexpr int kOffBar = kOffLD + SL * 512;
   static constexpr int kOffMisc = kOffBar + 32 * 8;
   static constexpr int kSmem = kOffMisc + 64;
-  static constexpr int kTmemCols = 512;  // dV, dK: 2 D; S^T / dP^T: 128; P^T / dS^T: 2 x 64 (bf16 pairs)
+  // TMEM: dV, dK: 2 D; S^T / dP^T: 128; P^T / dS^T: 64 (bf16 pairs); K: D / 2 (the A operand
+  // of S^T = K Q_i^T, bf16 pairs)
+  static constexpr int kTmemCols = 512;
+  static constexpr int kKCol = 2 * D + 192;
+  static_assert(kKCol + D / 2 <= kTmemCols, "TMEM columns");
 };
 
 struct DkvParams {
@@ -637,9 +641,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   uint32_t* dlist = prm.dlist + (size_t)blockIdx.x * prm.list_cap;
   auto bar = [&](int k) -> uint32_t { return sbase + L::kOffBar + 8 * k; };
   // one S^T / dP^T buffer: SP_FULL (products done), S_READ (row warps have loaded them);
-  // two P^T / dS^T buffers: DS_FULL (written), PS_FREE (dV / dK products done)
+  // one P^T / dS^T buffer: DS_FULL (written), PS_FREE (dV / dK products done); K_TMEM: the
+  // row warps have copied K into TMEM
   constexpr int KV_FULL = 0, LOADED = 1, SLOT_FREE = LOADED + S, SP_FULL = SLOT_FREE + S, S_READ = SP_FULL + 1,
-                DS_FULL = S_READ + 1, PS_FREE = DS_FULL + 2, ACC_DONE = PS_FREE + 2;
+                DS_FULL = S_READ + 1, PS_FREE = DS_FULL + 1, ACC_DONE = PS_FREE + 1, K_TMEM = ACC_DONE + 1;
   const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sR = sbase + L::kOffRing;
   auto head_of = [&](int g) { return b * prm.H + hk * prm.group + g; };
   // list tag -> (query head of the group, branch of lse / delta)
@@ -655,11 +660,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     }
     tc::mbar_init(bar(SP_FULL), 1);
     tc::mbar_init(bar(S_READ), kRowWarps);
-    for (int x = 0; x < 2; ++x) {
-      tc::mbar_init(bar(DS_FULL + x), kRowWarps);
-      tc::mbar_init(bar(PS_FREE + x), 1);
-    }
+    tc::mbar_init(bar(DS_FULL), kRowWarps);
+    tc::mbar_init(bar(PS_FREE), 1);
     tc::mbar_init(bar(ACC_DONE), 1);
+    tc::mbar_init(bar(K_TMEM), kRowWarps);
     tc::fence_mbar_init();
     tc::mbar_expect_tx(bar(KV_FULL), 4 * NP * 8192);
     for (int hf = 0; hf < 2; ++hf)
@@ -776,21 +780,23 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     constexpr uint32_t kAll = 0xffffffffu;
     constexpr uint32_t kIdS = tc::idesc_bf16(128, 64, false, false);
     // base descriptors; a byte offset off is added as off >> 4 (start-address field)
-    const uint64_t dKd = tc::sw128_desc(sK, 16, 1024), dVd = tc::sw128_desc(sV, 16, 1024);
+    const uint64_t dVd = tc::sw128_desc(sV, 16, 1024);
     const uint64_t dRk = tc::sw128_desc(sR, 16, 1024);    // ring tiles, K-major
-    // S^T = K Q_i^T, dP^T = V dO_i^T (M = 128 keys, N = 64 queries) into the S buffer
+    // S^T = K Q_i^T (A = K in TMEM: only Q_i is read from shared memory, full rate at
+    // N = 64), dP^T = V dO_i^T (M = 128 keys, N = 64 queries) into the S buffer
     auto issue_sp = [&](int m) {
       const uint32_t so = (uint32_t)((m % S) * L::kSlot);
       const uint32_t tS = tmem + 2 * D;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ko = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32), qo = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
-        tc::mma_bf16_ss(tS, dKd + (ko >> 4), dRk + ((so + qo) >> 4), kIdS, k > 0);
+        tc::mma_bf16_ts(tS, tmem + L::kKCol + 8 * k, dRk + ((so + qo) >> 4), kIdS, k > 0);
         tc::mma_bf16_ss(tS + 64, dVd + (ko >> 4), dRk + ((so + L::kTile + qo) >> 4), kIdS, k > 0);
       }
       tc::mma_commit(bar(SP_FULL));
     };
-    bool ok = T == 0 || __all_sync(kAll, tc::mbar_wait(bar(KV_FULL), 0, abort));
+    bool ok = T == 0 || (__all_sync(kAll, tc::mbar_wait(bar(KV_FULL), 0, abort)) &&
+                         __all_sync(kAll, tc::mbar_wait(bar(K_TMEM), 0, abort)));
     for (int m = 0; m < T && ok; ++m) {
       // the S buffer is free once the row warps have loaded S^T_{m-1}, dP^T_{m-1}: the
       // products of tile m run while they compute P^T_{m-1} and dS^T_{m-1}
@@ -811,8 +817,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const uint64_t dRn = tc::sw128_desc(sR, 8192, 1024);  // ring tiles, N-major (64-row panels)
     bool ok = true;
     for (int m = 0; m < T && ok; ++m) {
-      const int x = m & 1;
-      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL + x), (m >> 1) & 1, abort));
+      ok = __all_sync(kAll, tc::mbar_wait(bar(DS_FULL), m & 1, abort));
       if (!ok) break;
       tc::fence_after_sync();
       if (tc::elect_one()) {
@@ -820,7 +825,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         // B = dO_i / Q_i N-major. The slot is released after these products: S^T_m, dP^T_m
         // (its other readers) completed before the row warps could write P^T_m, dS^T_m
         const uint32_t so = (uint32_t)((m % S) * L::kSlot);
-        const uint32_t tP = tmem + 2 * D + 128 + 64 * x;
+        const uint32_t tP = tmem + 2 * D + 128;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
@@ -828,14 +833,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           tc::mma_bf16_ts(tmem + D, tP + 32 + 8 * kk, dRn + ((so + kk * 2048) >> 4), kIdA, acc);
         }
         tc::mma_commit(bar(SLOT_FREE + m % S));
-        tc::mma_commit(bar(PS_FREE + x));
+        tc::mma_commit(bar(PS_FREE));
         if (m == T - 1) tc::mma_commit(bar(ACC_DONE));
       }
       __syncwarp();
     }
-    // the last two P / dS buffers' releases: no commit is in flight at exit
-    for (int m = (T > 2 ? T - 2 : 0); m < T && ok; ++m)
-      ok = __all_sync(kAll, tc::mbar_wait(bar(PS_FREE + (m & 1)), (m >> 1) & 1, abort));
+    // the last release of the P / dS buffer: no commit is in flight at exit
+    if (ok && T > 0) ok = __all_sync(kAll, tc::mbar_wait(bar(PS_FREE), (T - 1) & 1, abort));
     if (!ok && lane == 0) {
       *abort = 1;
       report(prm.status, SLA_ERR_DEVICE_TIMEOUT, kDetailTimeout);
@@ -850,9 +854,33 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = prm.scale_log2;
     bool ok = true;
+    if (T > 0) {
+      // key row r (the TMEM lane) into columns kKCol.. as bf16 pairs, this warpgroup's half of
+      // the features: from the swizzled K tile (16-byte chunk c of a row at c ^ (row & 7))
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(KV_FULL), 0, abort));
+      if (ok) {
+        constexpr int CH = D / 16;  // 16-byte chunks per warpgroup half: 8 (D = 128) or 4
+        uint32_t kv[CH * 4];
+#pragma unroll
+        for (int x2 = 0; x2 < CH; ++x2) {
+          const int chunk = hw * CH + x2;  // of the row's D / 8 chunks
+          const int p = chunk >> 3, c = chunk & 7;
+          const uint4 u = *reinterpret_cast<const uint4*>(smem + L::kOffK + p * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+          kv[4 * x2] = u.x; kv[4 * x2 + 1] = u.y; kv[4 * x2 + 2] = u.z; kv[4 * x2 + 3] = u.w;
+        }
+        if constexpr (CH * 4 == 32)
+          tc::tmem_st32(tmem + lane_off + L::kKCol + 32 * hw, *reinterpret_cast<const uint32_t(*)[32]>(kv));
+        else
+          tc::tmem_st16(tmem + lane_off + L::kKCol + 16 * hw, *reinterpret_cast<const uint32_t(*)[16]>(kv));
+        tc::tmem_st_wait();
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(K_TMEM));
+    }
     uint32_t e_next = T > 0 ? dlist[0] : 0u;  // list entries are read one tile ahead
     for (int m = 0; m < T && ok; ++m) {
-      const int x = m & 1, slot = m % S;
+      const int slot = m % S;
       const uint32_t e = e_next;
       if (m + 1 < T) e_next = dlist[m + 1];
       const bool act = vkey && ((e >> (kActBit + hf)) & 1u);
@@ -914,17 +942,18 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         pw[j] = pack_bf16(p0, p1);
         dw[j] = pack_bf16(tc::f2_lo(d2), tc::f2_hi(d2));
       }
-      // P / dS buffer x was last read by the products of tile m - 2
-      if (m >= 2 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(PS_FREE + x), ((m - 2) >> 1) & 1, abort))))
+      // the P / dS buffer was last read by the products of tile m - 1 (PS_FREE has then
+      // completed m - 1 or m phases: the products of tile m need this tile's P and dS)
+      if (m >= 1 && !(ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(PS_FREE), (m - 1) & 1, abort))))
         break;
       tc::fence_after_sync();
-      const uint32_t tP = tmem + lane_off + 2 * D + 128 + 64 * x;
+      const uint32_t tP = tmem + lane_off + 2 * D + 128;
       tc::tmem_st16(tP + 16 * hw, pw);
       tc::tmem_st16(tP + 32 + 16 * hw, dw);
       tc::tmem_st_wait();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(DS_FULL + x));
+      if (lane == 0) tc::mbar_arrive(bar(DS_FULL));
     }
     if (ok && T > 0) {
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(ACC_DONE), 0, abort));
