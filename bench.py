@@ -694,7 +694,7 @@ def main():
         return None if bits is None else torch.from_numpy(bits).view(torch.bfloat16).to(dev)
 
     q, k, v, w_p, w_g = up(x.q), up(x.k), up(x.v), up(x.w_p), up(x.w_g)
-    full_cfg, shard_info = cfg, None
+    full_cfg, shard_info, bshard, full_inputs = cfg, None, None, None
     if args.shard == "heads":
         # one layer split over the ranks by KV group: estimate each group's work from its
         # routed tiles (every rank routes every world-th group; the costs are all-gathered),
@@ -706,9 +706,16 @@ def main():
             return route_lists(sla, torch, sh.local_config(cfg, units), sh.gather_heads(q, heads),
                                sh.gather_heads(k, units), dev)
         if dist is None:
-            costs = sh.unit_costs(cfg, route_lists(sla, torch, cfg, q, k, dev))
+            full_lists = route_lists(sla, torch, cfg, q, k, dev)
+            costs = sh.unit_costs(cfg, full_lists)
+            pcosts = sh.pair_costs(cfg, full_lists)
         else:
             costs = sh.distributed_costs(cfg, world, rank, route_local, dist)
+            pcosts = sh.distributed_pair_costs(cfg, world, rank, route_local, dist)
+        # db-SP's block level on the same routing: KV groups cut into runs of query-block
+        # pairs (measured after the head-level timing, on the full inputs)
+        bshard = sh.BlockShard(cfg, world, rank, pcosts)
+        full_inputs = (q, k, v, w_p, w_g)
         shard = sh.HeadShard(cfg, world, rank, costs)
         if any(not p for p in shard.plan):  # the same plan on every rank: all of them stop here
             raise RuntimeError(f"{world} ranks but only {cfg.H_kv} KV groups to share")
@@ -854,6 +861,41 @@ def main():
         (sg_ms,) = max_over_ranks(dist, dev, h0.elapsed_time(h1) / args.steps)
         shard_info["with_gather_ms_per_step"] = sg_ms
         shard_info["with_gather"] = "eager sla_forward on the local heads + all_gather_heads (NCCL), max over ranks"
+
+    if bshard is not None:
+        # the block level: this rank's pieces (KV group, range of query-block pairs) through
+        # sla_forward_blocks on the full inputs, max over ranks
+        qf, kf, vf, wpf, wgf = full_inputs
+        outf = torch.empty(full_cfg.B, full_cfg.H, full_cfg.N, full_cfg.d, dtype=torch.bfloat16, device=dev)
+        wss = {}
+
+        def ws_for(lc):
+            if lc.name not in wss:
+                wss[lc.name] = torch.empty(sla.sla_workspace_bytes(lc), dtype=torch.uint8, device=dev)
+            return wss[lc.name]
+        for _ in range(args.warmup):
+            bshard.run(sla, qf, kf, vf, wpf, wgf, outf, ws_for)
+        torch.cuda.synchronize()
+        barrier()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.steps):
+            bshard.run(sla, qf, kf, vf, wpf, wgf, outf, ws_for)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        for wsb in wss.values():
+            stb, detb = sla.sla_check_device_status(wsb)
+            if stb != 0:
+                raise RuntimeError(f"device status {stb} ({detb}) in the block-level steps")
+        (blk_ms,) = max_over_ranks(dist, dev, b0.elapsed_time(b1) / args.steps)
+        bl_loads = sh.block_plan_loads(bshard.costs, bshard.fixed, bshard.plan)
+        shard_info["block_level"] = {
+            "pieces": [[list(pc) for pc in pcs] for pcs in bshard.plan],
+            "estimated_loads": bl_loads, "imbalance": max(bl_loads) / (sum(bl_loads) / len(bl_loads)),
+            "ms_per_step": blk_ms,
+            "what": "db-SP's block level: (KV group, first pair, end pair) pieces per rank, each run through "
+                    "sla_forward_blocks on the full inputs (eager), max over ranks"}
+        del outf, wss
 
     # end to end: pinned host inputs -> device, layer, output -> host
     if shard_info is None:

@@ -313,22 +313,39 @@ class BlockShard:
         self.plan = block_plan(self.costs, self.fixed, world)
         self.pieces = self.plan[rank]
 
+    def calls(self) -> List[tuple]:
+        """The sla_forward_blocks calls that run this rank's pieces: (first group, end group,
+        first query block, end query block). Consecutive pieces that each cover a whole group
+        merge into one call over the range of groups; a partial piece is a call of its own."""
+        c = self.cfg
+        npairs = (c.nqb + 1) // 2
+        out: List[tuple] = []
+        for u, p0, p1 in self.pieces:
+            qb0, qb1 = 2 * p0, min(2 * p1, c.nqb)
+            whole = p0 == 0 and p1 == npairs
+            if whole and out and out[-1][1] == u and out[-1][2] == 0 and out[-1][3] == c.nqb:
+                out[-1] = (out[-1][0], u + 1, 0, c.nqb)
+            else:
+                out.append((u, u + 1, qb0, qb1))
+        return out
+
     def run(self, sla, q, k, v, w_p, w_g, out, ws_for, stream=None):
         """Runs this rank's pieces; ``out`` [B, H, N, d] receives their rows (the others
-        are not written). ``ws_for(local_cfg)`` returns a workspace for that config."""
+        are not written). ``ws_for(local_cfg)`` returns a workspace for that config. The
+        heads of a range of groups are a slice of dimension 1, a view without a copy when
+        B = 1; otherwise they are copied to a contiguous buffer (and the rows back)."""
         c = self.cfg
         group = c.H // c.H_kv
-        for u, p0, p1 in self.pieces:
-            heads = query_heads(c, [u])
-            lc = local_config(c, [u])
-            lq, lk, lv = gather_heads(q, heads), gather_heads(k, [u]), gather_heads(v, [u])
+        for u0, u1, qb0, qb1 in self.calls():
+            h0, h1 = u0 * group, u1 * group
+            lc = local_config(c, list(range(u0, u1)))
+            lq, lk, lv = (x[:, a:b].contiguous() for x, a, b in ((q, h0, h1), (k, u0, u1), (v, u0, u1)))
             lwp = w_p
             if w_p is not None and c.proj_per_head:
-                lwp = w_p[u * group:(u + 1) * group].contiguous()
-            lwg = None if w_g is None else w_g[u * group:(u + 1) * group].contiguous()
-            lout = out[:, u * group:(u + 1) * group]
+                lwp = w_p[h0:h1].contiguous()
+            lwg = None if w_g is None else w_g[h0:h1].contiguous()
+            lout = out[:, h0:h1]
             local = lout if lout.is_contiguous() else lout.contiguous()
-            qb0, qb1 = 2 * p0, min(2 * p1, c.nqb)
             sla.sla_forward_blocks(lq, lk, lv, lwp, lwg, lc, qb0, qb1, local, None, ws_for(lc), stream)
             if local is not lout:
                 lout[:, :, qb0 * 64:qb1 * 64] = local[:, :, qb0 * 64:qb1 * 64]

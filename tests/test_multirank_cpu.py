@@ -283,6 +283,50 @@ def test_pair_costs_sum_to_the_unit_costs():
         np.testing.assert_allclose(pc.sum(axis=1), sh.unit_costs(c, crit), rtol=1e-12)
 
 
+def test_block_shard_calls_merge_whole_groups_and_cover_every_row():
+    """BlockShard's calls: consecutive whole groups run as one sla_forward_blocks call over
+    a range of heads, a partial group as a call over its query blocks; run on two ranks
+    with a stand-in for the library (it copies its q rows of the given query blocks into
+    out) writes every output row exactly once, from the right heads, through views when
+    B = 1."""
+    import torch
+
+    sys.path.insert(0, ROOT)
+    from block_sparse_linear_sm_b200 import sharding as sh
+    from block_sparse_linear_sm_b200 import workloads as wl
+
+    cfg = wl.small_config(N=1024, N_valid=1000, H=10, H_kv=5, k_h=3, k_l=2)
+    npairs = (cfg.nqb + 1) // 2
+    costs, fixed = np.ones((cfg.H_kv, npairs)), np.zeros(cfg.H_kv)
+    shards = [sh.BlockShard(cfg, 2, r, costs, fixed) for r in range(2)]
+    assert shards[0].calls() == [(0, 2, 0, cfg.nqb), (2, 3, 0, 8)]
+    assert shards[1].calls() == [(2, 3, 8, cfg.nqb), (3, 5, 0, cfg.nqb)]
+
+    q = torch.arange(cfg.B * cfg.H * cfg.N * 2, dtype=torch.float32).view(cfg.B, cfg.H, cfg.N, 2)
+    kv = torch.zeros(cfg.B, cfg.H_kv, cfg.N, 2)
+    out = torch.full_like(q, -1.0)
+    writes = torch.zeros(cfg.B, cfg.H, cfg.N, dtype=torch.int32)
+    seen = []
+
+    class FakeLib:
+        @staticmethod
+        def sla_forward_blocks(lq, lk, lv, lwp, lwg, lc, qb0, qb1, lout, mask, ws, stream):
+            assert lq.shape[1] == lc.H and lk.shape[1] == lc.H_kv and lout.shape == lq.shape
+            seen.append((lc.H, qb0, qb1, lq.untyped_storage().data_ptr() == q.untyped_storage().data_ptr()))
+            lout[:, :, qb0 * 64:qb1 * 64] = lq[:, :, qb0 * 64:qb1 * 64]
+
+    base = out.untyped_storage().data_ptr()
+    for r, shard in enumerate(shards):
+        before = out.clone()
+        shard.run(FakeLib, q, kv, kv, None, None, out, lambda lc: None)
+        writes += (out != before).any(-1).int()
+    assert torch.equal(out, q)
+    assert int(writes.max()) == 1 and int(writes.min()) >= 0
+    assert out.untyped_storage().data_ptr() == base
+    assert [s[:3] for s in seen] == [(4, 0, cfg.nqb), (2, 0, 8), (2, 8, cfg.nqb), (4, 0, cfg.nqb)]
+    assert all(s[3] for s in seen)  # B = 1: the heads are views of q, not copies
+
+
 def _block_rank_main(rank, world, port, q):
     import datetime
 
