@@ -316,10 +316,13 @@ bool make_bwd_plan(const Plan& p, BwdPlan* b) {
     return o;
   };
   b->off_status = take(256);
+  b->off_ctr = take(256);
   b->off_delta = take((b->nsa ? 3 : 1) * B * H * N * 4);     // D_t = dO_t . O_s,t (NSA: dO_t . o_b,t)
   b->off_bits = take(B * H * p.nkb * (size_t)b->words * 4);  // query blocks of each key block
   // merged (query head, query block) list of each pair of key blocks
   b->off_dlist = take(B * Hkv * (size_t)((p.nkb + 1) / 2) * dkdv_list_cap(p) * 4);
+  if (c.mode == SLA_MODE_TOPN_WINDOW)
+    b->off_lbits = take(B * Hkv * (size_t)((p.nkb + 1) / 2) * 4 * b->words * 4);
   if (b->nsa) {
     b->off_lse3 = take(3 * B * H * N * 4);
     if (c.has_gate) b->off_dlogit = take(3 * B * H * N * 4);

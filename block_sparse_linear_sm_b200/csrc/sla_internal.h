@@ -102,6 +102,8 @@ struct BwdPlan {
   int cmp_items;  // NSA: work items of the compressed-key dK / dV kernel per KV head
   size_t off_status, off_delta, off_dqacc, off_dkacc, off_dvacc, off_drow, off_maskt, off_dh, off_dz,
       off_dwp, off_kcolp, off_kcol, off_bits, off_dlist, total;
+  size_t off_ctr;  // unit counters of the persistent flash kernels (dQ, dK / dV, compressed-key dK / dV)
+  size_t off_lbits;  // top-n modes: the dK / dV loader's four query-block bitmaps per unit
   // NSA: per-branch log-sum-exp with the gate folded in [3][B*H][N], gate-logit gradients
   // [3][B*H][N], compressed-key gradients dKc, dVc [B*H_kv][ncmp_pad][d] (fp32), the
   // compressed-key kernel's lists and raw partials
