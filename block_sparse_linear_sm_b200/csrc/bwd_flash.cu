@@ -88,6 +88,10 @@ enum NsaBranch { kBrCmp = 0, kBrSel = 1, kBrWin = 2 };
 constexpr int kMmaWarp = 8, kProdWarp = 9, kRowWarps = 8, kDqWarp = 10, kLoadWarp = 11;
 constexpr int kBwThreads = 384;
 constexpr int kListReaders = kRowWarps + 3;  // warps that arrive on a unit's LIST_FREE
+// The loader takes the next unit when the producer has this many tiles of the current one
+// left to load (at once for shorter units): time to build the list and load the stationary
+// tiles, without committing a long unit to a CTA long before it can start.
+constexpr int kClaimLead = 64;
 
 // merged list of two bitmaps (warp 0, ascending). Entry = index (bits 0-12) | a0 << 13 | a1 << 14
 // | s0 << 15 | s1 << 16 | tag << 17: a0 / a1 = the index is in bitmap a0 / a1 ("active" for
@@ -266,8 +270,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   constexpr int LOADED = 0, SLOT_FREE = S, SP_FULL = 2 * S, S_READ = SP_FULL + 2, DS_FULL = S_READ + 2,
                 DS_FREE = DS_FULL + 2, LIST_FULL = DS_FREE + 2, LIST_FREE = LIST_FULL + 2, Q_FULL = LIST_FREE + 2,
                 DO_FULL = Q_FULL + 1, Q_TMEM = DO_FULL + 1, PROD_DONE = Q_TMEM + 1, ACC_DONE = PROD_DONE + 1,
-                ACC_FREE = ACC_DONE + 1;
-  static_assert(ACC_FREE < 32, "mbarriers");
+                ACC_FREE = ACC_DONE + 1, CLAIM = ACC_FREE + 1;
+  static_assert(CLAIM < 32, "mbarriers");
   if (tid == 0) {
     misc[2] = 0;
     for (int x = 0; x < S; ++x) {
@@ -288,6 +292,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     tc::mbar_init(bar(PROD_DONE), 1);
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::mbar_init(bar(ACC_FREE), kRowWarps);
+    tc::mbar_init(bar(CLAIM), 1);
     tc::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -310,6 +315,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     uint32_t* words = lists + 2 * prm.list_cap;
     int prev = -1;
     for (int u = 0;; ++u) {
+      // the next unit is taken once the producer is within kClaimLead tiles of the current
+      // unit's end: a unit is committed to this CTA only shortly before it can start
+      if (u >= 1) ok = __all_sync(kAll, tc::mbar_wait(bar(CLAIM), (u - 1) & 1, abort));
+      if (!ok) break;
       int x = 0;
       if (lane == 0) x = atomicAdd(prm.counter, 1);
       x = __shfl_sync(kAll, x, 0);
@@ -378,7 +387,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         if (x < 0) break;
         const uint32_t* ml = unit_list(u);
         const int bkv = kv_head(x / prm.npairs);
+        const int claim_at = T > kClaimLead ? T - kClaimLead : 0;
+        if (claim_at == 0) tc::mbar_arrive(bar(CLAIM));
         for (int m = 0; m < T && ok; ++m, ++g) {
+          if (m == claim_at && m > 0) tc::mbar_arrive(bar(CLAIM));
           const int slot = g % S;
           if (g >= S && !(ok = tc::mbar_wait(bar(SLOT_FREE + slot), ((g / S) - 1) & 1, abort))) break;
           const uint32_t e = ml[m];
@@ -918,8 +930,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   constexpr int LOADED = 0, SLOT_FREE = S, SP_FULL = 2 * S, S_READ = SP_FULL + 1, DS_FULL = S_READ + 1,
                 PS_FREE = DS_FULL + 1, LIST_FULL = PS_FREE + 1, LIST_FREE = LIST_FULL + 2, K_FULL = LIST_FREE + 2,
                 V_FULL = K_FULL + 1, K_TMEM = V_FULL + 1, PROD_DONE = K_TMEM + 1, ACC_DONE = PROD_DONE + 1,
-                ACC_FREE = ACC_DONE + 1;
-  static_assert(ACC_FREE < 32, "mbarriers");
+                ACC_FREE = ACC_DONE + 1, CLAIM = ACC_FREE + 1;
+  static_assert(CLAIM < 32, "mbarriers");
   const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sR = sbase + L::kOffRing;
 
   if (tid == 0) {
@@ -942,6 +954,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     tc::mbar_init(bar(PROD_DONE), 1);
     tc::mbar_init(bar(ACC_DONE), 1);
     tc::mbar_init(bar(ACC_FREE), kRowWarps);
+    tc::mbar_init(bar(CLAIM), 1);
     tc::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -961,6 +974,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     // TMEM) and V (once the previous unit's products are done)
     int prev = -1;
     for (int u = 0;; ++u) {
+      // the next unit is taken once the producer is within kClaimLead tiles of the current
+      // unit's end: a unit is committed to this CTA only shortly before it can start
+      if (u >= 1) ok = __all_sync(kAll, tc::mbar_wait(bar(CLAIM), (u - 1) & 1, abort));
+      if (!ok) break;
       int x = 0;
       if (lane == 0) x = atomicAdd(prm.counter, 1);
       x = __shfl_sync(kAll, x, 0);
@@ -1036,7 +1053,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         const int bkv = dkdv_unit<TOPN, NSAC>(prm, x).bkv;
         const int bh0 = (bkv / Hkv) * prm.H + (bkv % Hkv) * prm.group;  // the group's first query head
         uint32_t e_next = T > 0 ? dl[0] : 0u;  // list entries are read one tile ahead
+        const int claim_at = T > kClaimLead ? T - kClaimLead : 0;
+        if (claim_at == 0) tc::mbar_arrive(bar(CLAIM));
         for (int m = 0; m < T && ok; ++m, ++g) {
+          if (m == claim_at && m > 0) tc::mbar_arrive(bar(CLAIM));
           const int slot = g % S;
           const uint32_t e = e_next;
           if (m + 1 < T) e_next = dl[m + 1];
