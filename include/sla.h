@@ -356,7 +356,11 @@ SLA_API sla_status sla_permute_tokens(const void* x, void* y, const int32_t* ord
  *   bws                     device scratch of sla_backward_workspace_bytes(cfg)
  *                           bytes, 256-byte aligned; its first 256 bytes hold
  *                           this call's device status word (read it with
- *                           sla_check_device_status(bws, ...))
+ *                           sla_check_device_status(bws, ...)). The flash
+ *                           stages run persistent kernels (one CTA per SM) that
+ *                           take their work units from counters in bws, zeroed
+ *                           on `stream` before each launch: calls that share one
+ *                           bws must not overlap on the GPU
  *   smooth-K        phi and phi' of k - m (m the head's mean valid key); every valid
  *                   row of dk also gets -1/N_valid times the head's summed
  *                   linear-branch gradient with respect to k - m
